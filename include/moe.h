@@ -1,0 +1,233 @@
+/*
+ * moe.h -- C ABI of the chunked MoE forward hot path for one NVIDIA B200 (sm_100a).
+ *
+ * The method is "Chunk MoE" as described in the MindSpeed article
+ * "昇腾MindSpeed分块专家计算Chunk MoE: 让通信藏进计算、显存轻装上阵" (cited below
+ * as [ChunkMoE] with the article's section heading). One MoE layer's forward
+ * pass is split along tokens into N chunks of T_chunk = ceil(T/N) tokens
+ * ([ChunkMoE] "一组关键公式"), adjacent chunks run as a pair with a double-buffered
+ * expert workspace ([ChunkMoE] "一张专业时序图"), and the split/count metadata of
+ * every chunk is computed at once and reaches the host in one device-to-host
+ * copy ([ChunkMoE] "一张专业时序图", the paragraph on batched_pre_dispatch_metadata).
+ * Per chunk the steps are: permute (dispatch), expert computation, unpermute
+ * (combine) ([ChunkMoE] "核心原理").  The article's All-to-All exchanges become a
+ * local layout on one GPU: permuted rows are rank-major (virtual EP group
+ * ascending) and expert-contiguous, so no collective runs.
+ *
+ * The expert FFN is SwiGLU without biases:
+ *     y = W_down[e] · ( silu(W_gate[e] · x) ⊙ (W_up[e] · x) ),  silu(z) = z / (1 + e^-z)
+ * (the article does not state the FFN form; SwiGLU is this library's fixed choice).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - "dev" pointers are CUDA device pointers; "host" pointers are ordinary host memory.
+ *  - bf16 tensors are passed as `void*` / `const void*`; each element is an IEEE
+ *    bfloat16 (16 bits, row-major).  fp32 is `float`, indices are int32.
+ *  - Weights are K-major (the nn.Linear layout):
+ *        W_gate_up [E][2I][H]  rows 0..I-1 of expert e are W_gate[e], rows I..2I-1 are W_up[e];
+ *        W_down    [E][H][I].
+ *  - `stream` is a cudaStream_t passed as `void*` (NULL = legacy default stream).
+ *  - Every call returns a moe_status_t and never aborts, traps or exits.  Argument
+ *    checks run on the host before anything is launched.  A call that returns an
+ *    error other than MOE_ERR_INDEX / MOE_ERR_CUDA has launched nothing.
+ *  - The caller owns every buffer, including the workspace.  The library keeps,
+ *    per device and created on first use, one extra non-blocking stream, a few
+ *    events and one pinned host staging block; nothing else persists between calls.
+ *  - Calls are not thread-safe with respect to each other on the same device.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_ABI_VERSION 1
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_ARG = 1,         /* null pointer, bad dimension, E % ep_groups != 0, k > E, ... */
+  MOE_ERR_INDEX = 2,       /* a top_k_index entry outside [0, E) (detected on the device)  */
+  MOE_ERR_ALIGN = 3,       /* a pointer that is not 16-byte aligned                        */
+  MOE_ERR_WORKSPACE = 4,   /* ws_bytes smaller than the size the query functions return    */
+  MOE_ERR_CUDA = 5,        /* a CUDA runtime or driver call failed                         */
+  MOE_ERR_TIMEOUT = 6,     /* a kernel gave up a bounded wait (never expected)             */
+  MOE_ERR_UNSUPPORTED = 7  /* shape outside the kernels' limits (see MOE_MAX_*)            */
+} moe_status_t;
+
+/* Kernel limits.  Shapes beyond them return MOE_ERR_UNSUPPORTED. */
+#define MOE_MAX_EXPERTS 1024   /* E  */
+#define MOE_MAX_TOPK 32        /* k  */
+
+/* Shape of one MoE layer call.
+ *   T          tokens (rows of hidden / out), T >= 0; T * k < 2^31
+ *   H          hidden size, H > 0, H % 8 == 0
+ *   I          expert intermediate size, I > 0, I % 8 == 0
+ *   E          routed experts, 1 <= E <= MOE_MAX_EXPERTS
+ *   k          experts per token, 1 <= k <= min(E, MOE_MAX_TOPK)
+ *   ep_groups  G virtual expert-parallel ranks; group g owns experts
+ *              [g*E/G, (g+1)*E/G); E % G == 0; 0 is read as 1
+ *   num_chunks N >= 0; 0 means "do not split" and is read as 1
+ *              ([ChunkMoE] "操作指南" step 3: both chunk settings 0 => no split). */
+typedef struct {
+  int64_t T;
+  int32_t H, I, E, k, ep_groups, num_chunks;
+} moe_shape_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* moe_status_string(moe_status_t status);
+
+/* MOE_ABI_VERSION of the loaded library. */
+int32_t moe_abi_version(void);
+
+/* Chunk partition, host arithmetic only ([ChunkMoE] "一组关键公式": T_chunk = ceil(T/N)).
+ * Writes N_eff + 1 bounds, N_eff = max(num_chunks, 1): chunk c holds tokens
+ * [bounds[c], bounds[c+1]) with bounds[c] = min(T, c * T_chunk).  Trailing chunks may
+ * be empty (T=49, N=8 gives seven chunks of 7 and one of 0).
+ * Errors: MOE_ERR_ARG if bounds is NULL, T < 0 or num_chunks < 0. */
+moe_status_t moe_chunk_bounds(int64_t T, int32_t num_chunks, int64_t* bounds /* host [N_eff+1] */);
+
+/* Device workspace, in bytes, that moe_metadata needs for these sizes; 0 if invalid. */
+size_t moe_metadata_workspace_bytes(int64_t T, int32_t k, int32_t E, int32_t ep_groups,
+                                    int32_t num_chunks);
+
+/* Device workspace, in bytes, that moe_forward needs for this shape; 0 if invalid.
+ * It holds the metadata and min(N_eff, 2) expert buffers of T_chunk*k rows, each
+ * (H + I) bf16 values per row: the pair double buffer of [ChunkMoE] "一组关键公式"
+ * (W_pair = O(2 * T_chunk)).  The permuted input rows and the expert output rows share
+ * one buffer, because the down projection runs only after the gate/up projection has
+ * consumed every permuted row of the chunk. */
+size_t moe_workspace_bytes(const moe_shape_t* shape);
+
+/* Batched pre-dispatch metadata for all chunks ([ChunkMoE] "一张专业时序图", the
+ * batched_pre_dispatch_metadata paragraph: one pass for all chunks, one host copy).
+ *
+ * In:  top_k_index  dev int32 [T][k], entries in [0, E)
+ * Out (host, caller-allocated, N_eff = max(num_chunks, 1), G = max(ep_groups, 1)):
+ *   send_splits   [N_eff][G]   rows of chunk c bound for virtual EP group g
+ *   recv_splits   [N_eff][G]   rows group g receives from this rank; on one GPU the
+ *                              only source rank is this one, so recv == send
+ *   expert_counts [N_eff][E]   rows of chunk c routed to expert e
+ *   chunk_bounds  [N_eff + 1]  as moe_chunk_bounds
+ * Out (dev, optional: pass NULL to skip):
+ *   dst_rows   int32 [T*k]  dst_rows[t*k+j] = chunk-local row of copy (t,j) in the
+ *                           permuted layout: experts ascending (hence groups ascending,
+ *                           "rank-major"), and inside one expert the flat index t*k+j
+ *                           ascending (a stable order).
+ *   src_tokens int32 [T*k]  src_tokens[bounds[c]*k + r] = global token t of chunk c's
+ *                           permuted row r (the inverse of dst_rows).
+ * workspace: dev, >= moe_metadata_workspace_bytes(...), 256-byte aligned.
+ * The call blocks the host once (the single metadata copy) and leaves the outputs
+ * complete when it returns.
+ * Errors: MOE_ERR_ARG, MOE_ERR_ALIGN, MOE_ERR_WORKSPACE, MOE_ERR_UNSUPPORTED (host
+ * checks); MOE_ERR_INDEX if any index is outside [0, E) (outputs then unspecified);
+ * MOE_ERR_CUDA. */
+moe_status_t moe_metadata(const int32_t* top_k_index, int64_t T, int32_t k, int32_t E,
+                          int32_t ep_groups, int32_t num_chunks, int32_t* send_splits,
+                          int32_t* recv_splits, int32_t* expert_counts, int64_t* chunk_bounds,
+                          int32_t* dst_rows, int32_t* src_tokens, void* workspace,
+                          size_t ws_bytes, void* stream);
+
+/* One MoE layer forward pass, chunked as Chunk MoE ([ChunkMoE] "核心原理",
+ * "一张专业时序图", "一组关键公式"):
+ *     out[t] = bf16( sum_{j<k} top_k_weights[t][j] * FFN_{top_k_index[t][j]}(hidden[t]) )
+ * with the j-sum in fp32 in ascending j.  Steps: metadata for all chunks + one
+ * device-to-host copy (the only host stall); then per chunk c: permute, gate/up grouped
+ * GEMM with SwiGLU, down grouped GEMM, weighted unpermute.  Chunks run as a two-stream
+ * pair pipeline on two workspace buffers: the permute of chunk c+1 and the unpermute of
+ * chunk c-1 overlap the expert GEMMs of chunk c.  The result is bit-identical for every
+ * num_chunks.
+ *
+ * In (dev):  hidden [T][H] bf16, top_k_index [T][k] int32, top_k_weights [T][k] fp32,
+ *            W_gate_up [E][2I][H] bf16, W_down [E][H][I] bf16
+ * Out (dev): out [T][H] bf16, fully overwritten (unspecified after an error)
+ * workspace: dev, >= moe_workspace_bytes(shape), 256-byte aligned; it must not
+ *            overlap any input or output.
+ * hidden, out, W_gate_up, W_down must be 16-byte aligned; top_k_index and
+ * top_k_weights 4-byte aligned.
+ * Synchrony: the host blocks once, on the metadata copy.  Everything after it is
+ * enqueued on `stream` (and on the library's second stream, which is joined back into
+ * `stream` before the call returns); the caller synchronizes `stream` to read `out`.
+ * T == 0 returns MOE_OK and launches nothing.
+ * Errors: as moe_metadata.  A kernel that gives up a bounded wait records it in the
+ * workspace; moe_check_device_status reports it. */
+moe_status_t moe_forward(const moe_shape_t* shape, const void* hidden, const int32_t* top_k_index,
+                         const float* top_k_weights, const void* W_gate_up, const void* W_down,
+                         void* out, void* workspace, size_t ws_bytes, void* stream);
+
+/* Synchronizes `stream` and returns MOE_ERR_TIMEOUT if a kernel of an earlier call that
+ * used this workspace gave up a bounded wait, MOE_ERR_INDEX if its last metadata pass
+ * saw a bad index, else MOE_OK (or MOE_ERR_CUDA). */
+moe_status_t moe_check_device_status(const void* workspace, size_t ws_bytes, void* stream);
+
+/* ---- Stage entry points ------------------------------------------------------------
+ * The kernels of moe_forward, one call each, on caller buffers.  moe_forward does not
+ * call these; they exist so that each step can be run and checked on its own.  None of
+ * them synchronizes.  `status` is a dev uint32 word that a kernel ORs with 2 when it
+ * gives up a bounded wait (the caller zeroes it beforehand). */
+
+/* Permute / dispatch of one chunk ([ChunkMoE] "核心原理", "一张专业时序图"):
+ *   X[dst_rows[t*k+j]] = hidden[t]  for t < Tc, j < k.
+ * hidden dev bf16 [Tc][H]; dst_rows dev int32 [Tc*k] (chunk-local rows, a bijection onto
+ * [0, Tc*k)); X dev bf16 [Tc*k][H].  hidden and X 16-byte aligned. */
+moe_status_t moe_permute(const void* hidden, const int32_t* dst_rows, int64_t Tc, int32_t H,
+                         int32_t k, void* X, void* stream);
+
+/* Expert gate/up projection with SwiGLU, grouped over experts (the expert computation of
+ * [ChunkMoE] "核心原理"): for every row r of expert e (rows offsets[e] .. offsets[e+1]-1)
+ *   Act[r] = bf16( silu(X[r] · W_gate[e]^T) ⊙ (X[r] · W_up[e]^T) ), fp32 accumulation.
+ * X dev bf16 [rows][H]; expert_offsets dev int32 [E+1] (offsets[0] = 0, nondecreasing,
+ * offsets[E] = rows); expert_counts_host host int32 [E] (offsets[e+1] - offsets[e]);
+ * W_gate_up dev bf16 [E][2I][H]; Act dev bf16 [rows][I].  16-byte aligned. */
+moe_status_t moe_grouped_gateup(const void* X, int64_t rows, int32_t H, int32_t I, int32_t E,
+                                const int32_t* expert_offsets, const int32_t* expert_counts_host,
+                                const void* W_gate_up, void* Act, uint32_t* status, void* stream);
+
+/* Expert down projection, grouped over experts:
+ *   Y[r] = bf16( Act[r] · W_down[e]^T ), fp32 accumulation.
+ * Act dev bf16 [rows][I]; W_down dev bf16 [E][H][I]; Y dev bf16 [rows][H]; other
+ * arguments as moe_grouped_gateup.  Y may alias the X of the gate/up call. */
+moe_status_t moe_grouped_down(const void* Act, int64_t rows, int32_t H, int32_t I, int32_t E,
+                              const int32_t* expert_offsets, const int32_t* expert_counts_host,
+                              const void* W_down, void* Y, uint32_t* status, void* stream);
+
+/* Weighted unpermute / combine of one chunk ([ChunkMoE] "核心原理", "一张专业时序图"):
+ *   out[t] = bf16( sum_{j<k} w[t*k+j] * float(Y[dst_rows[t*k+j]]) ), fp32, j ascending.
+ * Y dev bf16 [Tc*k][H]; dst_rows dev int32 [Tc*k]; w dev fp32 [Tc*k]; out dev bf16
+ * [Tc][H].  Y and out 16-byte aligned. */
+moe_status_t moe_unpermute(const void* Y, const int32_t* dst_rows, const float* top_k_weights,
+                           int64_t Tc, int32_t H, int32_t k, void* out, void* stream);
+
+/* ---- Kernel timing -----------------------------------------------------------------
+ * When enabled, every kernel launch of the calls above is bracketed by two CUDA events
+ * recorded on the stream the kernel is launched on.  moe_profile_read synchronizes the
+ * device, converts the pending event pairs into per-kind totals and returns them. */
+typedef enum {
+  MOE_KERNEL_METADATA = 0,  /* the metadata kernels (all passes of one call count as one) */
+  MOE_KERNEL_PERMUTE = 1,
+  MOE_KERNEL_GATEUP = 2,
+  MOE_KERNEL_DOWN = 3,
+  MOE_KERNEL_UNPERMUTE = 4,
+  MOE_KERNEL_KINDS = 5
+} moe_kernel_kind_t;
+
+typedef struct {
+  int64_t launches[MOE_KERNEL_KINDS];  /* timed launches of each kind                    */
+  double ms[MOE_KERNEL_KINDS];         /* summed event-to-event device time, ms           */
+  int64_t rows[MOE_KERNEL_KINDS];      /* summed rows processed: tokens for metadata,
+                                          permuted rows (T_c*k) for the other kinds        */
+  int64_t active_experts[MOE_KERNEL_KINDS]; /* summed experts with >0 rows (GEMM kinds)  */
+  int64_t kernels;                     /* device kernels launched while enabled          */
+} moe_profile_t;
+
+moe_status_t moe_profile_enable(int32_t on);  /* also clears the totals */
+moe_status_t moe_profile_read(moe_profile_t* out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */
