@@ -1,0 +1,458 @@
+"""Benchmark of the chunked MoE layer forward on B200.
+
+One step = one moe_forward call over one batch of synthetic input: metadata for all
+chunks + the single device-to-host copy, then per chunk permute, gate/up GEMM with
+SwiGLU, down GEMM and weighted unpermute, as the two-stream pair pipeline.
+
+Prints ONE JSON line (rank 0).  `value` is tokens/s of the whole job with inputs resident
+in HBM; `e2e` is the same metric through the public call with the step's inputs copied
+from pinned host memory and its output copied back inside the timed region.
+`--impl reference` times the CPU oracle on the same workload instead (a bounded token
+sample per step).  Multi-GPU runs are independent replicas (the path has no exchange).
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+for p in (ROOT, os.path.join(ROOT, "tests")):
+    if p not in sys.path:
+        sys.path.insert(0, p)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from gen import CONFIGS, expert_weights, hidden as gen_hidden, routing  # noqa: E402
+
+METRIC = "MoE fwd tokens/s; grouped-GEMM TFLOP/s and permute GB/s vs B200 peak"
+DEFAULT_CONFIG = "qwen3"
+DEFAULT_CHUNKS = 4
+GEMM_SRC = os.path.join(ROOT, "expert_router_top_b200", "csrc", "gemm.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gateup_traffic.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def workload_name(cfg):
+    return {"qwen3": "qwen3-30b-a3b-shaped layer, one 16k packed sequence",
+            "mixtral": "mixtral-8x7b-shaped layer", "deepseek": "deepseek-v3-shaped routed layer",
+            "tiny": "tiny layer", "edge": "edge-case layer"}.get(cfg.name, cfg.name)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of one GPU's clocks and throttle reasons, every 200 ms."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------- workload
+
+def make_inputs(cfg, device, seed=0, weights=True):
+    idx, w = routing(cfg, seed)
+    x = gen_hidden(cfg.T, cfg.H, seed)
+    out = dict(hidden=x.to(device), idx=torch.from_numpy(idx).to(device),
+               w=torch.from_numpy(w).to(device), hidden_cpu=x, idx_cpu=idx, w_cpu=w)
+    if weights:
+        out["wgu"], out["wd"] = expert_weights(cfg.E, cfg.H, cfg.I, seed, device=device)
+    return out
+
+
+def algorithmic_units(cfg, counts, n_live):
+    """Per-kernel algorithmic work of one step (bytes or flops), from the chunk counts."""
+    H, I, k, T = cfg.H, cfg.I, cfg.k, cfg.T
+    rows = int(counts.sum())
+    active = int((counts > 0).sum())
+    return {
+        # permute: read T rows once, write T*k rows, plus the k destination indices per token
+        "permute_bytes": (T + rows) * H * 2 + rows * 4,
+        # unpermute: read T*k rows and their weights and indices, write T rows
+        "unpermute_bytes": (rows + T) * H * 2 + rows * 8,
+        "gateup_flops": 4.0 * rows * H * I,
+        "down_flops": 2.0 * rows * H * I,
+        # weights of every active expert, re-read once per chunk (the method's N-fold stream)
+        "gateup_weight_bytes": active * 2 * I * H * 2,
+        "down_weight_bytes": active * H * I * 2,
+    }
+
+
+def gemm_src_hash():
+    with open(GEMM_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def traffic_per_launch():
+    """DRAM bytes per gate/up launch from the committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        d = json.load(f)
+    if d.get("gemm_src_sha256_16") != gemm_src_hash():
+        return None
+    return d.get("dram_bytes_per_launch_full_size")
+
+
+# ------------------------------------------------------------------------- oracle arm
+
+def oracle_tokens_per_s(cfg, inputs, budget_s, sample_seed=0, max_tokens=None, seed=0):
+    """Oracle throughput on a bounded, seeded sample of the workload's tokens.
+
+    Draws the weights of the sampled tokens' experts on the host; returns
+    (tokens/s, tokens, seconds, threads)."""
+    import oracle
+    from gen import bits, expert_down, expert_gate_up
+
+    rng = np.random.default_rng(1000 + sample_seed)
+    idx, w = inputs["idx_cpu"], inputs["w_cpu"]
+    xb = bits(inputs["hidden_cpu"])
+
+    def run(n):
+        toks = np.sort(rng.choice(cfg.T, size=n, replace=False))
+        used = sorted(set(idx[toks].reshape(-1).tolist()))
+        remap = {e: i for i, e in enumerate(used)}
+        sidx = np.vectorize(remap.get)(idx[toks]).astype(np.int32)
+        wgu = np.stack([bits(expert_gate_up(e, cfg.H, cfg.I, seed)) for e in used])
+        wd = np.stack([bits(expert_down(e, cfg.H, cfg.I, seed)) for e in used])
+        t0 = time.perf_counter()
+        oracle.forward(xb[toks], sidx, w[toks], wgu, wd)
+        return time.perf_counter() - t0
+
+    threads = oracle.max_threads()
+    n = max(1, min(threads, cfg.T))
+    dt = run(n)
+    per_tok = dt / n
+    target = int(budget_s / max(per_tok, 1e-9))
+    n2 = max(n, min(cfg.T, target, max_tokens or cfg.T))
+    if n2 > n:
+        n, dt = n2, run(n2)
+    return n / dt, n, dt, threads
+
+
+def run_reference(args, cfg):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    inputs = make_inputs(cfg, device="cpu", weights=False)
+    per_step = max(1.0, 150.0 / (args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_tokens_per_s(cfg, inputs, per_step / 4, max_tokens=64)
+    total_tok, total_s, threads, toks = 0, 0.0, 1, 0
+    for i in range(args.steps):
+        tps, toks, dt, threads = oracle_tokens_per_s(cfg, inputs, per_step, sample_seed=i)
+        total_tok += toks
+        total_s += dt
+    value = total_tok / total_s
+    sample = (f"{args.steps} steps, each a seeded sample of ~{toks} of the {cfg.T} tokens "
+              f"(all k={cfg.k} experts per token, fp64), ~{per_step:.0f} s each")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_block(cfg, args.chunks),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_block(cfg, chunks):
+    wbytes = 6 * cfg.E * cfg.H * cfg.I
+    return {"workload": workload_name(cfg), "T": cfg.T, "H": cfg.H, "E": cfg.E, "k": cfg.k,
+            "I": cfg.I, "ep_groups": cfg.G, "num_chunks": chunks, "routing": cfg.routing,
+            "ffn": "SwiGLU", "parallelism": "replicas",
+            "l2": f"inputs larger than L2 ({wbytes / 1e9:.2f} GB of expert weights read per step)"}
+
+
+# ------------------------------------------------------------------------- our arm
+
+def time_steps(moe, inp, cfg, chunks, ws, steps, stream):
+    """Device time of `steps` back-to-back forward calls, ms (CUDA events on `stream`)."""
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    out = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device="cuda")
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(steps):
+        moe.forward(inp["hidden"], inp["idx"], inp["w"], inp["wgu"], inp["wd"],
+                    num_chunks=chunks, ep_groups=cfg.G, out=out, workspace=ws, stream=stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end), out
+
+
+def run_ours(args, cfg):
+    import expert_router_top_b200 as moe
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    moe.load()
+    dev = torch.device("cuda", local)
+    inp = make_inputs(cfg, dev)
+    chunks = args.chunks
+    ws_bytes = moe.workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.G, chunks)
+    ws = moe.alloc_workspace(ws_bytes, dev)
+    stream = torch.cuda.current_stream()
+
+    meta = moe.metadata(inp["idx"], cfg.E, cfg.G, chunks)
+    counts = meta["counts"]
+    n_live = int((np.diff(meta["bounds"]) > 0).sum())
+    units = algorithmic_units(cfg, counts, n_live)
+    active_per_chunk = (counts > 0).sum(1)
+    weight_stream = float(active_per_chunk.sum()) * 6 * cfg.H * cfg.I  # bytes, all chunks
+
+    for _ in range(args.warmup):
+        moe.forward(inp["hidden"], inp["idx"], inp["w"], inp["wgu"], inp["wd"],
+                    num_chunks=chunks, ep_groups=cfg.G, workspace=ws)
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    moe.profile_enable(True)
+    ms, out = time_steps(moe, inp, cfg, chunks, ws, args.steps, stream)
+    if pg:
+        pg.barrier()
+    prof = moe.profile_read()
+    moe.profile_enable(False)
+    clk = clocks.stop() if clocks else None
+
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if pg:
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    ms_max = float(t.item())
+    ms_per_step = ms_max / args.steps
+    value = world * cfg.T * args.steps / (ms_max / 1e3)
+
+    # N = 1 reference point of the same workload (for the <= 5 % loss target), untimed key
+    ms_n1 = None
+    if chunks != 1:
+        ws1 = moe.alloc_workspace(moe.workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.G, 1),
+                                  dev)
+        for _ in range(2):
+            moe.forward(inp["hidden"], inp["idx"], inp["w"], inp["wgu"], inp["wd"],
+                        num_chunks=1, ep_groups=cfg.G, workspace=ws1)
+        ms1, _ = time_steps(moe, inp, cfg, 1, ws1, args.steps, stream)
+        ms_n1 = ms1 / args.steps
+        del ws1
+
+    # ---- end to end through the public call, host buffers, copies inside the region
+    e2e = run_e2e(moe, inp, cfg, chunks, ws, args, stream, dev, pg, world)
+
+    # ---- roofline of the dominant kernel (gate/up grouped GEMM)
+    peaks, peak_src = load_peaks()
+    kinds = {}
+    for kind in moe.KERNEL_KINDS:
+        p = prof[kind]
+        kinds[kind] = dict(launches=p["launches"], ms=p["ms"],
+                           ms_per_step=p["ms"] / args.steps if args.steps else 0.0)
+    steps = args.steps
+    g = prof["gateup"]
+    gu_flops = units["gateup_flops"] * steps
+    gu_tflops = gu_flops / (g["ms"] / 1e3) / 1e12 if g["ms"] > 0 else 0.0
+    d = prof["down"]
+    dn_tflops = units["down_flops"] * steps / (d["ms"] / 1e3) / 1e12 if d["ms"] > 0 else 0.0
+    pm = prof["permute"]
+    pm_gbs = units["permute_bytes"] * steps / (pm["ms"] / 1e3) / 1e9 if pm["ms"] > 0 else 0.0
+    um = prof["unpermute"]
+    um_gbs = units["unpermute_bytes"] * steps / (um["ms"] / 1e3) / 1e9 if um["ms"] > 0 else 0.0
+    gemm_tflops = (units["gateup_flops"] + units["down_flops"]) * steps / \
+        ((g["ms"] + d["ms"]) / 1e3) / 1e12 if g["ms"] + d["ms"] > 0 else 0.0
+    kinds["gateup"]["tflops"] = gu_tflops
+    kinds["down"]["tflops"] = dn_tflops
+    kinds["permute"]["gbs"] = pm_gbs
+    kinds["unpermute"]["gbs"] = um_gbs
+    peak_tc = peaks["bf16_tflops"]
+    traffic = traffic_per_launch()
+    roofline = {"bound": "tensor", "kernel": "gateup_swiglu grouped GEMM (tcgen05)",
+                "achieved": gu_tflops, "peak": peak_tc, "unit": "TFLOP/s",
+                "frac": gu_tflops / peak_tc if peak_tc else None,
+                "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)",
+                "frac_of_sustained": gu_tflops / peaks["bf16_tflops_sustained"],
+                "traffic": traffic}
+
+    ws_per_n = {str(n): moe.workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.G, n)
+                for n in (1, 2, 4)}
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; random-init expert weights of the layer's shape)",
+        "config": config_block(cfg, chunks),
+        "roofline": roofline,
+        "grouped_gemm_tflops": gemm_tflops,
+        "grouped_gemm_frac_of_peak": gemm_tflops / peak_tc,
+        "permute_gbs": pm_gbs, "permute_frac_of_hbm": pm_gbs / peaks["hbm_gbs"],
+        "unpermute_gbs": um_gbs, "unpermute_frac_of_hbm": um_gbs / peaks["hbm_gbs"],
+        "kernels": kinds,
+        "weight_bytes_streamed_per_step": weight_stream,
+        "workspace_bytes": ws_per_n,
+        "ms_per_step_num_chunks_1": ms_n1,
+        "gpu_launches": int(prof["kernels"]),
+        "e2e": e2e,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tps, ntok, dt, threads = oracle_tokens_per_s(cfg, inp, args.cpu_budget_s)
+        line["cpu_baseline"] = {
+            "value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{ntok} seeded tokens of the {cfg.T}-token workload, all k={cfg.k} "
+                      f"experts each, fp64, {dt:.1f} s"}
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_e2e(moe, inp, cfg, chunks, ws, args, stream, dev, pg, world):
+    steps = max(3, min(args.steps, 20))
+    h_pin = inp["hidden_cpu"].pin_memory()
+    i_pin = torch.from_numpy(inp["idx_cpu"]).pin_memory()
+    w_pin = torch.from_numpy(inp["w_cpu"]).pin_memory()
+    o_pin = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16).pin_memory()
+    hd = torch.empty_like(inp["hidden"])
+    idd = torch.empty_like(inp["idx"])
+    wdv = torch.empty_like(inp["w"])
+    out = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device=dev)
+
+    def step():
+        hd.copy_(h_pin, non_blocking=True)
+        idd.copy_(i_pin, non_blocking=True)
+        wdv.copy_(w_pin, non_blocking=True)
+        moe.forward(hd, idd, wdv, inp["wgu"], inp["wd"], num_chunks=chunks, ep_groups=cfg.G,
+                    out=out, workspace=ws, stream=stream)
+        o_pin.copy_(out, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        step()
+    e.record(stream)
+    torch.cuda.synchronize()
+    t = torch.tensor([s.elapsed_time(e)], dtype=torch.float64, device=dev)
+    if pg:
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    ms = float(t.item())
+    h2d = h_pin.numel() * 2 + i_pin.numel() * 4 + w_pin.numel() * 4
+    return {"value": world * cfg.T * steps / (ms / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": o_pin.numel() * 2,
+            "steps": steps}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", choices=sorted(CONFIGS), default=DEFAULT_CONFIG)
+    ap.add_argument("--chunks", type=int, default=DEFAULT_CHUNKS)
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps, always
+    cfg = CONFIGS[args.config]
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+    return run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,283 @@
+"""Chunked MoE forward on one NVIDIA B200 -- thin Python binding of libmoe.so.
+
+Every function here only marshals arguments (tensor pointers, sizes, the current CUDA
+stream) into the C ABI declared in include/moe.h; all the work runs in the library's
+CUDA kernels.  There is no fallback: if libmoe.so is missing or fails to load, every
+call raises.  PyTorch is used for device memory and streams only.
+
+The method is Chunk MoE from the MindSpeed article "昇腾MindSpeed分块专家计算Chunk MoE":
+the layer's tokens are split into N chunks of ceil(T/N) tokens (section 一组关键公式),
+adjacent chunks run as a pair over a double-buffered workspace (section 一张专业时序图),
+and the split/count metadata of all chunks comes back to the host in one copy.
+"""
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe.so")
+
+MOE_OK = 0
+STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_ARG", 2: "MOE_ERR_INDEX", 3: "MOE_ERR_ALIGN",
+                4: "MOE_ERR_WORKSPACE", 5: "MOE_ERR_CUDA", 6: "MOE_ERR_TIMEOUT",
+                7: "MOE_ERR_UNSUPPORTED"}
+KERNEL_KINDS = ("metadata", "permute", "gateup", "down", "unpermute")
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)}")
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("H", ctypes.c_int32), ("I", ctypes.c_int32),
+                ("E", ctypes.c_int32), ("k", ctypes.c_int32), ("ep_groups", ctypes.c_int32),
+                ("num_chunks", ctypes.c_int32)]
+
+
+class Profile(ctypes.Structure):
+    _fields_ = [("launches", ctypes.c_int64 * 5), ("ms", ctypes.c_double * 5),
+                ("rows", ctypes.c_int64 * 5), ("active_experts", ctypes.c_int64 * 5),
+                ("kernels", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def load():
+    """Load libmoe.so (built in-tree by build.py); raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          f"`python -m expert_router_top_b200.build` (nvcc, sm_100a)")
+    L = ctypes.CDLL(LIB_PATH)
+    p, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    st = ctypes.c_int
+    L.moe_status_string.argtypes = [st]
+    L.moe_status_string.restype = ctypes.c_char_p
+    L.moe_abi_version.argtypes = []
+    L.moe_abi_version.restype = i32
+    L.moe_chunk_bounds.argtypes = [i64, i32, p]
+    L.moe_chunk_bounds.restype = st
+    L.moe_metadata_workspace_bytes.argtypes = [i64, i32, i32, i32, i32]
+    L.moe_metadata_workspace_bytes.restype = sz
+    L.moe_workspace_bytes.argtypes = [ctypes.POINTER(Shape)]
+    L.moe_workspace_bytes.restype = sz
+    L.moe_metadata.argtypes = [p, i64, i32, i32, i32, i32, p, p, p, p, p, p, p, sz, p]
+    L.moe_metadata.restype = st
+    L.moe_forward.argtypes = [ctypes.POINTER(Shape), p, p, p, p, p, p, p, sz, p]
+    L.moe_forward.restype = st
+    L.moe_check_device_status.argtypes = [p, sz, p]
+    L.moe_check_device_status.restype = st
+    L.moe_permute.argtypes = [p, p, i64, i32, i32, p, p]
+    L.moe_permute.restype = st
+    L.moe_grouped_gateup.argtypes = [p, i64, i32, i32, i32, p, p, p, p, p, p]
+    L.moe_grouped_gateup.restype = st
+    L.moe_grouped_down.argtypes = [p, i64, i32, i32, i32, p, p, p, p, p, p]
+    L.moe_grouped_down.restype = st
+    L.moe_unpermute.argtypes = [p, p, p, i64, i32, i32, p, p]
+    L.moe_unpermute.restype = st
+    L.moe_profile_enable.argtypes = [i32]
+    L.moe_profile_enable.restype = st
+    L.moe_profile_read.argtypes = [ctypes.POINTER(Profile)]
+    L.moe_profile_read.restype = st
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return load().moe_status_string(status).decode()
+
+
+def _check(status: int, what: str):
+    if status != MOE_OK:
+        raise MoEError(status, what)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, np.ndarray):
+        return t.ctypes.data_as(ctypes.c_void_p)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, dtype, name, device=True):
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if device and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+
+
+def shape(T, H, I, E, k, ep_groups=1, num_chunks=1) -> Shape:
+    return Shape(T, H, I, E, k, ep_groups, num_chunks)
+
+
+def chunk_bounds(T: int, num_chunks: int) -> np.ndarray:
+    b = np.zeros(max(num_chunks, 1) + 1, np.int64)
+    _check(load().moe_chunk_bounds(T, num_chunks, _ptr(b)), "moe_chunk_bounds")
+    return b
+
+
+def workspace_bytes(T, H, I, E, k, ep_groups=1, num_chunks=1) -> int:
+    s = shape(T, H, I, E, k, ep_groups, num_chunks)
+    return int(load().moe_workspace_bytes(ctypes.byref(s)))
+
+
+def metadata_workspace_bytes(T, k, E, ep_groups=1, num_chunks=1) -> int:
+    return int(load().moe_metadata_workspace_bytes(T, k, E, ep_groups, num_chunks))
+
+
+def alloc_workspace(nbytes: int, device=None) -> torch.Tensor:
+    """A caller-owned device workspace (uint8, 256-byte aligned by the allocator)."""
+    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device or "cuda")
+
+
+def metadata(top_k_index: torch.Tensor, E: int, ep_groups: int = 1, num_chunks: int = 1,
+             with_permutation: bool = False, workspace: torch.Tensor = None, stream=None):
+    """Batched metadata for every chunk (one device pass, one host copy).
+
+    Returns a dict of numpy arrays: send/recv [N,G], counts [N,E], bounds [N+1]; with
+    with_permutation also torch int32 dst [T*k] and src_tok [T*k] on the device."""
+    _need(top_k_index, torch.int32, "top_k_index")
+    T, k = top_k_index.shape
+    n = max(num_chunks, 1)
+    G = max(ep_groups, 1)
+    send = np.zeros((n, G), np.int32)
+    recv = np.zeros((n, G), np.int32)
+    counts = np.zeros((n, E), np.int32)
+    bounds = np.zeros(n + 1, np.int64)
+    dst = src = None
+    if with_permutation:
+        dst = torch.empty(T * k, dtype=torch.int32, device=top_k_index.device)
+        src = torch.empty(T * k, dtype=torch.int32, device=top_k_index.device)
+    if workspace is None:
+        workspace = alloc_workspace(metadata_workspace_bytes(T, k, E, ep_groups, num_chunks),
+                                    top_k_index.device)
+    _check(load().moe_metadata(_ptr(top_k_index), T, k, E, ep_groups, num_chunks, _ptr(send),
+                               _ptr(recv), _ptr(counts), _ptr(bounds), _ptr(dst), _ptr(src),
+                               _ptr(workspace), workspace.numel(), _stream(stream)),
+           "moe_metadata")
+    out = dict(send=send, recv=recv, counts=counts, bounds=bounds)
+    if with_permutation:
+        out["dst"], out["src_tok"] = dst, src
+    return out
+
+
+def forward(hidden, top_k_index, top_k_weights, W_gate_up, W_down, num_chunks: int = 1,
+            ep_groups: int = 1, out=None, workspace=None, stream=None):
+    """One MoE layer forward, chunked as Chunk MoE.  Returns out [T,H] bf16.
+
+    hidden [T,H] bf16, top_k_index [T,k] int32, top_k_weights [T,k] fp32,
+    W_gate_up [E,2I,H] bf16 (gate rows then up rows), W_down [E,H,I] bf16; all on the
+    same CUDA device.  Asynchronous after its single metadata copy."""
+    _need(hidden, torch.bfloat16, "hidden")
+    _need(top_k_index, torch.int32, "top_k_index")
+    _need(top_k_weights, torch.float32, "top_k_weights")
+    _need(W_gate_up, torch.bfloat16, "W_gate_up")
+    _need(W_down, torch.bfloat16, "W_down")
+    T, H = hidden.shape
+    E, twoI, H2 = W_gate_up.shape
+    I = twoI // 2
+    k = top_k_index.shape[1]
+    if H2 != H or tuple(W_down.shape) != (E, H, I) or tuple(top_k_index.shape) != (T, k) \
+            or tuple(top_k_weights.shape) != (T, k):
+        raise ValueError("inconsistent shapes")
+    s = shape(T, H, I, E, k, ep_groups, num_chunks)
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=hidden.device)
+    if workspace is None:
+        workspace = alloc_workspace(load().moe_workspace_bytes(ctypes.byref(s)), hidden.device)
+    _check(load().moe_forward(ctypes.byref(s), _ptr(hidden), _ptr(top_k_index),
+                              _ptr(top_k_weights), _ptr(W_gate_up), _ptr(W_down), _ptr(out),
+                              _ptr(workspace), workspace.numel(), _stream(stream)),
+           "moe_forward")
+    return out
+
+
+def check_device_status(workspace, stream=None):
+    _check(load().moe_check_device_status(_ptr(workspace), workspace.numel(), _stream(stream)),
+           "moe_check_device_status")
+
+
+def permute(hidden, dst_rows, k: int, X=None, stream=None):
+    _need(hidden, torch.bfloat16, "hidden")
+    _need(dst_rows, torch.int32, "dst_rows")
+    Tc, H = hidden.shape
+    if X is None:
+        X = torch.empty((Tc * k, H), dtype=torch.bfloat16, device=hidden.device)
+    _check(load().moe_permute(_ptr(hidden), _ptr(dst_rows), Tc, H, k, _ptr(X), _stream(stream)),
+           "moe_permute")
+    return X
+
+
+def _grouped(fn, A, offsets_dev, counts_host, W, out, status, stream, H, I, what):
+    _need(A, torch.bfloat16, "A")
+    _need(offsets_dev, torch.int32, "expert_offsets")
+    _need(W, torch.bfloat16, "W")
+    counts_host = np.ascontiguousarray(counts_host, dtype=np.int32)
+    rows = A.shape[0]
+    E = counts_host.shape[0]
+    own_status = status is None
+    if own_status:
+        status = torch.zeros(4, dtype=torch.int32, device=A.device)
+    _check(fn(_ptr(A), rows, H, I, E, _ptr(offsets_dev), _ptr(counts_host), _ptr(W), _ptr(out),
+              _ptr(status), _stream(stream)), what)
+    return out, status
+
+
+def grouped_gateup(X, expert_offsets, expert_counts, W_gate_up, Act=None, status=None,
+                   stream=None):
+    """Act[r] = bf16(silu(X[r] W_gate[e]^T) * (X[r] W_up[e]^T)) for the rows of each expert."""
+    E, twoI, H = W_gate_up.shape
+    I = twoI // 2
+    if Act is None:
+        Act = torch.empty((X.shape[0], I), dtype=torch.bfloat16, device=X.device)
+    return _grouped(load().moe_grouped_gateup, X, expert_offsets, expert_counts, W_gate_up, Act,
+                    status, stream, H, I, "moe_grouped_gateup")
+
+
+def grouped_down(Act, expert_offsets, expert_counts, W_down, Y=None, status=None, stream=None):
+    """Y[r] = bf16(Act[r] W_down[e]^T) for the rows of each expert."""
+    E, H, I = W_down.shape
+    if Y is None:
+        Y = torch.empty((Act.shape[0], H), dtype=torch.bfloat16, device=Act.device)
+    return _grouped(load().moe_grouped_down, Act, expert_offsets, expert_counts, W_down, Y, status,
+                    stream, H, I, "moe_grouped_down")
+
+
+def unpermute(Y, dst_rows, top_k_weights, k: int, out=None, stream=None):
+    _need(Y, torch.bfloat16, "Y")
+    _need(dst_rows, torch.int32, "dst_rows")
+    _need(top_k_weights, torch.float32, "top_k_weights")
+    H = Y.shape[1]
+    Tc = dst_rows.numel() // k
+    if out is None:
+        out = torch.empty((Tc, H), dtype=torch.bfloat16, device=Y.device)
+    _check(load().moe_unpermute(_ptr(Y), _ptr(dst_rows), _ptr(top_k_weights), Tc, H, k, _ptr(out),
+                                _stream(stream)), "moe_unpermute")
+    return out
+
+
+def profile_enable(on: bool = True):
+    _check(load().moe_profile_enable(1 if on else 0), "moe_profile_enable")
+
+
+def profile_read() -> dict:
+    p = Profile()
+    _check(load().moe_profile_read(ctypes.byref(p)), "moe_profile_read")
+    return {kind: dict(launches=int(p.launches[i]), ms=float(p.ms[i]), rows=int(p.rows[i]),
+                       active_experts=int(p.active_experts[i]))
+            for i, kind in enumerate(KERNEL_KINDS)} | {"kernels": int(p.kernels)}

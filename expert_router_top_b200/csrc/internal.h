@@ -1,0 +1,73 @@
+// internal.h -- declarations shared by the library's translation units (host side).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// ---- metadata (metadata.cu) -----------------------------------------------------------
+
+constexpr int kMetaThreads = 256;       // 8 warps
+constexpr int kMetaSlotsPerTile = 2048; // token copies (t, j) handled by one CTA
+
+struct MetaArgs {
+  const int32_t* idx;  // [T][k]
+  int64_t T;
+  int32_t k, E, G, n_chunks;
+  int64_t t_chunk;          // ceil(T / n_chunks)
+  int32_t tile_tokens;      // tokens per tile (a tile never straddles two chunks)
+  int32_t tiles_per_chunk;  // ceil(t_chunk / tile_tokens)
+  int32_t* hist;            // [n_chunks * tiles_per_chunk][E] scratch
+  int32_t* dst;             // [T*k] chunk-local row of each copy
+  int32_t* src_tok;         // [T*k] or nullptr
+  int32_t* counts;          // [n_chunks][E]
+  int32_t* offsets;         // [n_chunks][E+1]
+  int32_t* splits;          // [n_chunks][G]
+  uint32_t* status;         // device status word
+};
+
+inline int32_t meta_tile_tokens(int32_t k) {
+  int32_t t = kMetaSlotsPerTile / k;
+  return t < 1 ? 1 : t;
+}
+
+cudaError_t launch_metadata(const MetaArgs& a, cudaStream_t s);
+
+// ---- permute / unpermute (permute.cu) ----------------------------------------------------
+
+cudaError_t launch_permute(const void* hidden, const int32_t* dst, int64_t Tc, int32_t H,
+                           int32_t k, void* X, cudaStream_t s);
+cudaError_t launch_unpermute(const void* Y, const int32_t* dst, const float* w, int64_t Tc,
+                             int32_t H, int32_t k, void* out, cudaStream_t s);
+
+// ---- grouped GEMM (gemm.cu) -------------------------------------------------------------
+
+constexpr int kGemmBM = 128;     // rows per tile (one tcgen05.mma M=128 per CTA)
+constexpr int kGemmBN = 256;     // MMA N: 128 gate + 128 up columns, or 256 down columns
+constexpr int kGemmBK = 64;      // K per pipeline stage (one 128-byte swizzle row)
+constexpr int kGemmStages = 4;
+constexpr int kGemmThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+
+struct GemmArgs {
+  const void* A;          // [rows][K] bf16 (permuted X, or Act)
+  int64_t rows;           // rows in A and in the output
+  const void* B;          // weights [E][b_rows][K]
+  void* out;              // [rows][out_cols] bf16
+  const int32_t* offsets; // dev [E+1]
+  int32_t E;
+  int32_t K;              // H for gate/up, I for down
+  int32_t out_cols;       // I for gate/up, H for down
+  int32_t b_rows;         // 2I for gate/up, H for down
+  int64_t total_tiles;    // sum over experts of ceil(rows_e / 128) * n_tiles
+  uint32_t* status;
+};
+
+// Number of 128-row x N-column output tiles for the given host counts.
+int64_t gemm_total_tiles(const int32_t* counts_host, int32_t E, int32_t out_cols, bool swiglu);
+
+cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cudaStream_t s,
+                                int* err_detail);
+
+}  // namespace moe

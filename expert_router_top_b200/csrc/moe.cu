@@ -1,0 +1,583 @@
+// moe.cu -- C ABI of the chunked MoE forward pass: argument checks, workspace layout,
+// the single metadata copy, and the two-stream pair pipeline over the chunks.
+//
+// Chunk MoE article ("昇腾MindSpeed分块专家计算Chunk MoE"):
+//   一组关键公式  T_chunk = ceil(T/N); the pair double buffer W_pair = O(2 * T_chunk)
+//   一张专业时序图 forward_pair over adjacent chunks c and n = c+1: Expert(c) overlaps the
+//                 dispatch of n, Expert(n) overlaps the combine of c; the first dispatch and
+//                 the last combine stay exposed; batched_pre_dispatch_metadata does one
+//                 pass and one host copy for all chunks
+//   核心原理      permute -> expert computation -> unpermute per chunk
+//   操作指南      a chunk setting of 0 means no split
+// On one GPU the article's All-to-All dispatch/combine become the permute/unpermute
+// layout itself: rows are expert-contiguous and rank-major, so nothing crosses devices.
+//
+// Stream roles inside moe_forward: the caller's stream M runs metadata, permute and
+// unpermute; the library's stream G runs the two expert GEMMs.  Chunk c uses workspace
+// buffer c % 2.  Enqueue order on M is P(0) P(1) U(0) P(2) U(1) ... U(last), so P(c+1)
+// runs beside the GEMMs of c and U(c) beside the GEMMs of c+1; P(c+2) follows U(c) on M,
+// which frees buffer c % 2 for it.
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+#include <vector>
+
+#include "device.cuh"
+#include "internal.h"
+#include "moe.h"
+
+namespace {
+
+using namespace moe;
+
+constexpr size_t kAlign = 256;
+constexpr int kStatusWords = 4;  // packed block: status words, then counts, then splits
+constexpr int kMaxDevices = 64;
+constexpr int32_t kMaxChunks = MOE_MAX_CHUNKS;
+
+size_t al(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+struct Dims {
+  int64_t T;
+  int32_t k, E, G, n;  // n = effective chunk count
+  int64_t t_chunk;
+  int32_t tile_tokens, tiles_per_chunk;
+};
+
+struct Layout {
+  size_t packed, packed_bytes, offsets, hist, dst, src;
+  size_t xy[2], act[2];
+  int nbuf;
+  int64_t rows_cap;
+  size_t total;
+};
+
+Dims make_dims(int64_t T, int32_t k, int32_t E, int32_t ep_groups, int32_t num_chunks) {
+  Dims d;
+  d.T = T;
+  d.k = k;
+  d.E = E;
+  d.G = ep_groups > 0 ? ep_groups : 1;
+  d.n = num_chunks > 0 ? num_chunks : 1;
+  d.t_chunk = (T + d.n - 1) / d.n;
+  d.tile_tokens = meta_tile_tokens(k);
+  d.tiles_per_chunk = (int32_t)((d.t_chunk + d.tile_tokens - 1) / d.tile_tokens);
+  if (d.tiles_per_chunk < 1) d.tiles_per_chunk = 1;
+  return d;
+}
+
+// Workspace layout.  with_buffers: the expert buffers of moe_forward; with_dst/with_src:
+// scratch for the permutation when the caller does not provide it.
+Layout make_layout(const Dims& d, int32_t H, int32_t I, bool with_buffers, bool with_dst,
+                   bool with_src) {
+  Layout L{};
+  size_t o = 0;
+  L.packed = o;
+  L.packed_bytes = sizeof(int32_t) * (kStatusWords + (size_t)d.n * d.E + (size_t)d.n * d.G);
+  o += al(L.packed_bytes);
+  L.offsets = o;
+  o += al(sizeof(int32_t) * (size_t)d.n * (d.E + 1));
+  L.hist = o;
+  o += al(sizeof(int32_t) * (size_t)d.n * d.tiles_per_chunk * d.E);
+  L.dst = o;
+  if (with_dst) o += al(sizeof(int32_t) * (size_t)(d.T * d.k));
+  L.src = o;
+  if (with_src) o += al(sizeof(int32_t) * (size_t)(d.T * d.k));
+  L.nbuf = 0;
+  L.rows_cap = d.t_chunk * d.k;
+  if (with_buffers) {
+    // the pair double buffer: one buffer for N = 1, two otherwise
+    L.nbuf = d.n >= 2 ? 2 : 1;
+    for (int b = 0; b < L.nbuf; ++b) {
+      L.xy[b] = o;
+      o += al(sizeof(uint16_t) * (size_t)L.rows_cap * H);
+      L.act[b] = o;
+      o += al(sizeof(uint16_t) * (size_t)L.rows_cap * I);
+    }
+  }
+  L.total = o;
+  return L;
+}
+
+moe_status_t check_routing_dims(int64_t T, int32_t k, int32_t E, int32_t ep_groups,
+                                int32_t num_chunks) {
+  if (T < 0 || k <= 0 || E <= 0 || ep_groups < 0 || num_chunks < 0) return MOE_ERR_ARG;
+  const int32_t G = ep_groups > 0 ? ep_groups : 1;
+  if (k > E || E % G != 0) return MOE_ERR_ARG;
+  if (E > MOE_MAX_EXPERTS || k > MOE_MAX_TOPK || num_chunks > kMaxChunks) return MOE_ERR_UNSUPPORTED;
+  if (T * (int64_t)k >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status_t check_shape(const moe_shape_t* s) {
+  if (!s) return MOE_ERR_ARG;
+  moe_status_t st = check_routing_dims(s->T, s->k, s->E, s->ep_groups, s->num_chunks);
+  if (st != MOE_OK) return st;
+  if (s->H <= 0 || s->I <= 0 || s->H % 8 != 0 || s->I % 8 != 0) return MOE_ERR_ARG;
+  return MOE_OK;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// ---- per-device context -------------------------------------------------------------------
+
+struct DeviceCtx {
+  bool ready = false;
+  int num_sms = 0;
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_start = nullptr, ev_join = nullptr, ev_perm[2] = {}, ev_gemm[2] = {};
+  int32_t* host_stage = nullptr;
+  size_t host_stage_bytes = 0;
+};
+
+DeviceCtx g_ctx[kMaxDevices];
+std::mutex g_mu;
+
+moe_status_t get_ctx(DeviceCtx** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceCtx& c = g_ctx[dev];
+  if (!c.ready) {
+    if (cudaDeviceGetAttribute(&c.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (cudaStreamCreateWithFlags(&c.side, cudaStreamNonBlocking) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    const unsigned fl = cudaEventDisableTiming;
+    if (cudaEventCreateWithFlags(&c.ev_start, fl) != cudaSuccess ||
+        cudaEventCreateWithFlags(&c.ev_join, fl) != cudaSuccess ||
+        cudaEventCreateWithFlags(&c.ev_perm[0], fl) != cudaSuccess ||
+        cudaEventCreateWithFlags(&c.ev_perm[1], fl) != cudaSuccess ||
+        cudaEventCreateWithFlags(&c.ev_gemm[0], fl) != cudaSuccess ||
+        cudaEventCreateWithFlags(&c.ev_gemm[1], fl) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    c.ready = true;
+  }
+  *out = &c;
+  return MOE_OK;
+}
+
+moe_status_t ensure_host_stage(DeviceCtx* c, size_t bytes) {
+  if (c->host_stage_bytes >= bytes) return MOE_OK;
+  if (c->host_stage) cudaFreeHost(c->host_stage);
+  c->host_stage = nullptr;
+  c->host_stage_bytes = 0;
+  size_t want = bytes < 65536 ? 65536 : bytes;
+  void* p = nullptr;
+  if (cudaMallocHost(&p, want) != cudaSuccess) return MOE_ERR_CUDA;
+  c->host_stage = static_cast<int32_t*>(p);
+  c->host_stage_bytes = want;
+  return MOE_OK;
+}
+
+// ---- kernel timing ------------------------------------------------------------------------
+
+struct ProfRec {
+  int kind;
+  cudaEvent_t a, b;
+  int64_t rows, active;
+  int kernels;
+};
+
+struct Prof {
+  bool on = false;
+  std::vector<ProfRec> pending;
+  std::vector<cudaEvent_t> pool;
+  moe_profile_t tot{};
+} g_prof;
+
+cudaEvent_t prof_event() {
+  if (!g_prof.pool.empty()) {
+    cudaEvent_t e = g_prof.pool.back();
+    g_prof.pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+struct ProfScope {
+  bool on;
+  ProfRec r;
+  cudaStream_t s;
+  ProfScope(int kind, cudaStream_t st, int64_t rows, int64_t active, int kernels)
+      : on(g_prof.on), s(st) {
+    if (!on) return;
+    r.kind = kind;
+    r.rows = rows;
+    r.active = active;
+    r.kernels = kernels;
+    r.a = prof_event();
+    r.b = prof_event();
+    cudaEventRecord(r.a, s);
+  }
+  ~ProfScope() {
+    if (!on) return;
+    cudaEventRecord(r.b, s);
+    g_prof.pending.push_back(r);
+  }
+};
+
+moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+moe_status_t run_metadata(const Dims& d, const int32_t* idx, uint8_t* ws, const Layout& L,
+                          int32_t* dst, int32_t* src, cudaStream_t s) {
+  MetaArgs a;
+  a.idx = idx;
+  a.T = d.T;
+  a.k = d.k;
+  a.E = d.E;
+  a.G = d.G;
+  a.n_chunks = d.n;
+  a.t_chunk = d.t_chunk;
+  a.tile_tokens = d.tile_tokens;
+  a.tiles_per_chunk = d.tiles_per_chunk;
+  a.hist = reinterpret_cast<int32_t*>(ws + L.hist);
+  a.dst = dst;
+  a.src_tok = src;
+  int32_t* packed = reinterpret_cast<int32_t*>(ws + L.packed);
+  a.status = reinterpret_cast<uint32_t*>(packed);
+  a.counts = packed + kStatusWords;
+  a.splits = a.counts + (size_t)d.n * d.E;
+  a.offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+  if (cudaMemsetAsync(packed, 0, sizeof(int32_t) * kStatusWords, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  {
+    ProfScope ps(MOE_KERNEL_METADATA, s, d.T, 0, 3);
+    if (launch_metadata(a, s) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+// The single device-to-host copy of {status, counts, splits} for every chunk.
+moe_status_t fetch_packed(DeviceCtx* c, const uint8_t* ws, const Layout& L, cudaStream_t s) {
+  moe_status_t st = ensure_host_stage(c, L.packed_bytes);
+  if (st != MOE_OK) return st;
+  if (cudaMemcpyAsync(c->host_stage, ws + L.packed, L.packed_bytes, cudaMemcpyDeviceToHost, s) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  const uint32_t status = static_cast<uint32_t>(c->host_stage[0]);
+  if (status & MOE_DEV_BAD_INDEX) return MOE_ERR_INDEX;
+  if (status & MOE_DEV_TIMEOUT) return MOE_ERR_TIMEOUT;
+  return MOE_OK;
+}
+
+int64_t active_experts(const int32_t* counts, int32_t E) {
+  int64_t a = 0;
+  for (int32_t e = 0; e < E; ++e) a += counts[e] > 0;
+  return a;
+}
+
+moe_status_t gemm_call(const void* A, int64_t rows, const void* B, void* out,
+                       const int32_t* offsets_dev, const int32_t* counts_host, int32_t E,
+                       int32_t K, int32_t out_cols, int32_t b_rows, bool swiglu,
+                       uint32_t* status, int num_sms, cudaStream_t s) {
+  GemmArgs g;
+  g.A = A;
+  g.rows = rows;
+  g.B = B;
+  g.out = out;
+  g.offsets = offsets_dev;
+  g.E = E;
+  g.K = K;
+  g.out_cols = out_cols;
+  g.b_rows = b_rows;
+  g.total_tiles = gemm_total_tiles(counts_host, E, out_cols, swiglu);
+  g.status = status;
+  if (g.total_tiles == 0) return MOE_OK;
+  int detail = 0;
+  ProfScope ps(swiglu ? MOE_KERNEL_GATEUP : MOE_KERNEL_DOWN, s, rows,
+               active_experts(counts_host, E), 1);
+  cudaError_t e = launch_grouped_gemm(g, swiglu, num_sms, s, &detail);
+  if (e != cudaSuccess) return detail == 1 ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+}  // namespace
+
+// ========================================================================================
+// C ABI
+// ========================================================================================
+
+extern "C" {
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_ARG: return "MOE_ERR_ARG: invalid argument";
+    case MOE_ERR_INDEX: return "MOE_ERR_INDEX: top_k_index entry outside [0, E)";
+    case MOE_ERR_ALIGN: return "MOE_ERR_ALIGN: pointer not 16-byte aligned";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace too small";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: CUDA call failed";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT: a kernel gave up a bounded wait";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: shape outside kernel limits";
+  }
+  return "unknown moe_status_t";
+}
+
+int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+moe_status_t moe_chunk_bounds(int64_t T, int32_t num_chunks, int64_t* bounds) {
+  if (!bounds || T < 0 || num_chunks < 0) return MOE_ERR_ARG;
+  const int64_t n = num_chunks > 0 ? num_chunks : 1;
+  const int64_t tc = (T + n - 1) / n;
+  for (int64_t c = 0; c <= n; ++c) bounds[c] = c * tc < T ? c * tc : T;
+  return MOE_OK;
+}
+
+size_t moe_metadata_workspace_bytes(int64_t T, int32_t k, int32_t E, int32_t ep_groups,
+                                    int32_t num_chunks) {
+  if (check_routing_dims(T, k, E, ep_groups, num_chunks) != MOE_OK) return 0;
+  return make_layout(make_dims(T, k, E, ep_groups, num_chunks), 8, 8, false, true, true).total;
+}
+
+size_t moe_workspace_bytes(const moe_shape_t* s) {
+  if (check_shape(s) != MOE_OK) return 0;
+  return make_layout(make_dims(s->T, s->k, s->E, s->ep_groups, s->num_chunks), s->H, s->I, true,
+                     true, true)
+      .total;
+}
+
+moe_status_t moe_metadata(const int32_t* top_k_index, int64_t T, int32_t k, int32_t E,
+                          int32_t ep_groups, int32_t num_chunks, int32_t* send_splits,
+                          int32_t* recv_splits, int32_t* expert_counts, int64_t* chunk_bounds,
+                          int32_t* dst_rows, int32_t* src_tokens, void* workspace,
+                          size_t ws_bytes, void* stream) {
+  moe_status_t st = check_routing_dims(T, k, E, ep_groups, num_chunks);
+  if (st != MOE_OK) return st;
+  if (!send_splits || !recv_splits || !expert_counts || !chunk_bounds) return MOE_ERR_ARG;
+  if (T > 0 && (!top_k_index || !workspace)) return MOE_ERR_ARG;
+  if (!aligned(top_k_index, 4) || !aligned(dst_rows, 4) || !aligned(src_tokens, 4) ||
+      !aligned(workspace, kAlign))
+    return MOE_ERR_ALIGN;
+  const Dims d = make_dims(T, k, E, ep_groups, num_chunks);
+  moe_chunk_bounds(T, num_chunks, chunk_bounds);
+  if (T == 0) {
+    memset(send_splits, 0, sizeof(int32_t) * (size_t)d.n * d.G);
+    memset(recv_splits, 0, sizeof(int32_t) * (size_t)d.n * d.G);
+    memset(expert_counts, 0, sizeof(int32_t) * (size_t)d.n * d.E);
+    return MOE_OK;
+  }
+  const Layout L = make_layout(d, 8, 8, false, dst_rows == nullptr, false);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  DeviceCtx* ctx = nullptr;
+  if ((st = get_ctx(&ctx)) != MOE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* dst = dst_rows ? dst_rows : reinterpret_cast<int32_t*>(ws + L.dst);
+  if ((st = run_metadata(d, top_k_index, ws, L, dst, src_tokens, s)) != MOE_OK) return st;
+  if ((st = fetch_packed(ctx, ws, L, s)) != MOE_OK) return st;
+  const int32_t* counts = ctx->host_stage + kStatusWords;
+  const int32_t* splits = counts + (size_t)d.n * d.E;
+  memcpy(expert_counts, counts, sizeof(int32_t) * (size_t)d.n * d.E);
+  memcpy(send_splits, splits, sizeof(int32_t) * (size_t)d.n * d.G);
+  memcpy(recv_splits, splits, sizeof(int32_t) * (size_t)d.n * d.G);  // one source rank
+  return MOE_OK;
+}
+
+moe_status_t moe_forward(const moe_shape_t* shape, const void* hidden, const int32_t* top_k_index,
+                         const float* top_k_weights, const void* W_gate_up, const void* W_down,
+                         void* out, void* workspace, size_t ws_bytes, void* stream) {
+  moe_status_t st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  const int64_t T = shape->T;
+  const int32_t H = shape->H, I = shape->I, E = shape->E, k = shape->k;
+  if (T == 0) return MOE_OK;
+  if (!hidden || !top_k_index || !top_k_weights || !W_gate_up || !W_down || !out || !workspace)
+    return MOE_ERR_ARG;
+  if (!aligned(hidden, 16) || !aligned(out, 16) || !aligned(W_gate_up, 16) ||
+      !aligned(W_down, 16) || !aligned(top_k_index, 4) || !aligned(top_k_weights, 4) ||
+      !aligned(workspace, kAlign))
+    return MOE_ERR_ALIGN;
+  const Dims d = make_dims(T, k, E, shape->ep_groups, shape->num_chunks);
+  const Layout L = make_layout(d, H, I, true, true, true);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  DeviceCtx* ctx = nullptr;
+  if ((st = get_ctx(&ctx)) != MOE_OK) return st;
+  cudaStream_t sm = static_cast<cudaStream_t>(stream);
+  cudaStream_t sg = ctx->side;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* dst = reinterpret_cast<int32_t*>(ws + L.dst);
+  int32_t* src = reinterpret_cast<int32_t*>(ws + L.src);
+  uint32_t* dev_status = reinterpret_cast<uint32_t*>(ws + L.packed);
+
+  // 1) metadata for all chunks, 2) the one device-to-host copy (the only host stall)
+  if ((st = run_metadata(d, top_k_index, ws, L, dst, src, sm)) != MOE_OK) return st;
+  if ((st = fetch_packed(ctx, ws, L, sm)) != MOE_OK) return st;
+  // Copy what the pipeline needs out of the shared staging block.
+  std::vector<int32_t> counts(ctx->host_stage + kStatusWords,
+                              ctx->host_stage + kStatusWords + (size_t)d.n * d.E);
+  std::vector<int64_t> bounds((size_t)d.n + 1);
+  moe_chunk_bounds(T, shape->num_chunks, bounds.data());
+  int n_live = 0;  // chunks with tokens; only trailing chunks can be empty
+  while (n_live < d.n && bounds[n_live + 1] > bounds[n_live]) ++n_live;
+
+  const uint16_t* hid = static_cast<const uint16_t*>(hidden);
+  uint16_t* outp = static_cast<uint16_t*>(out);
+  auto xy = [&](int c) { return ws + L.xy[c % L.nbuf]; };
+  auto act = [&](int c) { return ws + L.act[c % L.nbuf]; };
+  auto len = [&](int c) { return bounds[c + 1] - bounds[c]; };
+
+  auto permute = [&](int c) -> moe_status_t {
+    ProfScope ps(MOE_KERNEL_PERMUTE, sm, len(c) * k, 0, 1);
+    if (launch_permute(hid + bounds[c] * H, dst + bounds[c] * k, len(c), H, k, xy(c), sm) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (cudaEventRecord(ctx->ev_perm[c & 1], sm) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+  };
+  auto experts = [&](int c) -> moe_status_t {
+    if (cudaStreamWaitEvent(sg, ctx->ev_perm[c & 1], 0) != cudaSuccess) return MOE_ERR_CUDA;
+    const int64_t rows = len(c) * k;
+    const int32_t* cnt = counts.data() + (size_t)c * E;
+    const int32_t* offs = reinterpret_cast<const int32_t*>(ws + L.offsets) + (size_t)c * (E + 1);
+    moe_status_t s2 = gemm_call(xy(c), rows, W_gate_up, act(c), offs, cnt, E, H, I, 2 * I, true,
+                                dev_status, ctx->num_sms, sg);
+    if (s2 != MOE_OK) return s2;
+    s2 = gemm_call(act(c), rows, W_down, xy(c), offs, cnt, E, I, H, H, false, dev_status,
+                   ctx->num_sms, sg);
+    if (s2 != MOE_OK) return s2;
+    if (cudaEventRecord(ctx->ev_gemm[c & 1], sg) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+  };
+  auto unpermute = [&](int c) -> moe_status_t {
+    if (cudaStreamWaitEvent(sm, ctx->ev_gemm[c & 1], 0) != cudaSuccess) return MOE_ERR_CUDA;
+    ProfScope ps(MOE_KERNEL_UNPERMUTE, sm, len(c) * k, 0, 1);
+    if (launch_unpermute(xy(c), dst + bounds[c] * k, top_k_weights + bounds[c] * k, len(c), H, k,
+                         outp + bounds[c] * H, sm) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  };
+
+  // 3) the pair pipeline
+  if (cudaEventRecord(ctx->ev_start, sm) != cudaSuccess ||
+      cudaStreamWaitEvent(sg, ctx->ev_start, 0) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (n_live > 0) {
+    if ((st = permute(0)) != MOE_OK || (st = experts(0)) != MOE_OK) return st;
+    for (int c = 0; c < n_live; ++c) {
+      if (c + 1 < n_live) {
+        if ((st = permute(c + 1)) != MOE_OK || (st = experts(c + 1)) != MOE_OK) return st;
+      }
+      if ((st = unpermute(c)) != MOE_OK) return st;
+    }
+  }
+  if (cudaEventRecord(ctx->ev_join, sg) != cudaSuccess ||
+      cudaStreamWaitEvent(sm, ctx->ev_join, 0) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status_t moe_check_device_status(const void* workspace, size_t ws_bytes, void* stream) {
+  if (!workspace || ws_bytes < sizeof(uint32_t)) return MOE_ERR_ARG;
+  uint32_t st = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&st, workspace, sizeof st, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (st & MOE_DEV_TIMEOUT) return MOE_ERR_TIMEOUT;
+  if (st & MOE_DEV_BAD_INDEX) return MOE_ERR_INDEX;
+  return MOE_OK;
+}
+
+moe_status_t moe_permute(const void* hidden, const int32_t* dst_rows, int64_t Tc, int32_t H,
+                         int32_t k, void* X, void* stream) {
+  if (Tc < 0 || H <= 0 || H % 8 || k <= 0 || k > MOE_MAX_TOPK) return MOE_ERR_ARG;
+  if (Tc == 0) return MOE_OK;
+  if (!hidden || !dst_rows || !X) return MOE_ERR_ARG;
+  if (!aligned(hidden, 16) || !aligned(X, 16) || !aligned(dst_rows, 4)) return MOE_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ProfScope ps(MOE_KERNEL_PERMUTE, s, Tc * k, 0, 1);
+  return cuda_status(launch_permute(hidden, dst_rows, Tc, H, k, X, s));
+}
+
+moe_status_t moe_unpermute(const void* Y, const int32_t* dst_rows, const float* top_k_weights,
+                           int64_t Tc, int32_t H, int32_t k, void* out, void* stream) {
+  if (Tc < 0 || H <= 0 || H % 8 || k <= 0 || k > MOE_MAX_TOPK) return MOE_ERR_ARG;
+  if (Tc == 0) return MOE_OK;
+  if (!Y || !dst_rows || !top_k_weights || !out) return MOE_ERR_ARG;
+  if (!aligned(Y, 16) || !aligned(out, 16) || !aligned(dst_rows, 4) || !aligned(top_k_weights, 4))
+    return MOE_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ProfScope ps(MOE_KERNEL_UNPERMUTE, s, Tc * k, 0, 1);
+  return cuda_status(launch_unpermute(Y, dst_rows, top_k_weights, Tc, H, k, out, s));
+}
+
+static moe_status_t grouped_common(const void* A, int64_t rows, int32_t H, int32_t I, int32_t E,
+                                   const int32_t* offsets, const int32_t* counts_host,
+                                   const void* W, void* out, uint32_t* status, void* stream,
+                                   bool swiglu) {
+  if (rows < 0 || H <= 0 || I <= 0 || H % 8 || I % 8 || E <= 0) return MOE_ERR_ARG;
+  if (E > MOE_MAX_EXPERTS || rows >= ((int64_t)1 << 31)) return MOE_ERR_UNSUPPORTED;
+  if (rows == 0) return MOE_OK;
+  if (!A || !offsets || !counts_host || !W || !out || !status) return MOE_ERR_ARG;
+  if (!aligned(A, 16) || !aligned(W, 16) || !aligned(out, 16) || !aligned(offsets, 4) ||
+      !aligned(status, 4))
+    return MOE_ERR_ALIGN;
+  int64_t sum = 0;
+  for (int32_t e = 0; e < E; ++e) {
+    if (counts_host[e] < 0) return MOE_ERR_ARG;
+    sum += counts_host[e];
+  }
+  if (sum != rows) return MOE_ERR_ARG;
+  DeviceCtx* ctx = nullptr;
+  moe_status_t st = get_ctx(&ctx);
+  if (st != MOE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (swiglu)
+    return gemm_call(A, rows, W, out, offsets, counts_host, E, H, I, 2 * I, true, status,
+                     ctx->num_sms, s);
+  return gemm_call(A, rows, W, out, offsets, counts_host, E, I, H, H, false, status,
+                   ctx->num_sms, s);
+}
+
+moe_status_t moe_grouped_gateup(const void* X, int64_t rows, int32_t H, int32_t I, int32_t E,
+                                const int32_t* expert_offsets, const int32_t* expert_counts_host,
+                                const void* W_gate_up, void* Act, uint32_t* status, void* stream) {
+  return grouped_common(X, rows, H, I, E, expert_offsets, expert_counts_host, W_gate_up, Act,
+                        status, stream, true);
+}
+
+moe_status_t moe_grouped_down(const void* Act, int64_t rows, int32_t H, int32_t I, int32_t E,
+                              const int32_t* expert_offsets, const int32_t* expert_counts_host,
+                              const void* W_down, void* Y, uint32_t* status, void* stream) {
+  return grouped_common(Act, rows, H, I, E, expert_offsets, expert_counts_host, W_down, Y, status,
+                        stream, false);
+}
+
+moe_status_t moe_profile_enable(int32_t on) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  for (auto& r : g_prof.pending) {
+    g_prof.pool.push_back(r.a);
+    g_prof.pool.push_back(r.b);
+  }
+  g_prof.pending.clear();
+  g_prof.tot = moe_profile_t{};
+  g_prof.on = on != 0;
+  return MOE_OK;
+}
+
+moe_status_t moe_profile_read(moe_profile_t* out) {
+  if (!out) return MOE_ERR_ARG;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_prof.pending.empty() && cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  for (auto& r : g_prof.pending) {
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) return MOE_ERR_CUDA;
+    g_prof.tot.launches[r.kind] += 1;
+    g_prof.tot.ms[r.kind] += ms;
+    g_prof.tot.rows[r.kind] += r.rows;
+    g_prof.tot.active_experts[r.kind] += r.active;
+    g_prof.tot.kernels += r.kernels;
+    g_prof.pool.push_back(r.a);
+    g_prof.pool.push_back(r.b);
+  }
+  g_prof.pending.clear();
+  *out = g_prof.tot;
+  return MOE_OK;
+}
+
+}  // extern "C"

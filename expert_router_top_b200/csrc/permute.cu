@@ -1,0 +1,133 @@
+// permute.cu -- dispatch (permute) and weighted combine (unpermute) of one chunk.
+//
+// Chunk MoE article ("昇腾MindSpeed分块专家计算Chunk MoE"), section 核心原理: permute
+// groups the token copies by expert before the expert computation, unpermute restores
+// token order and merges the k copies afterwards; section 一张专业时序图 lists
+// top_k_weights among the inputs split per chunk, and the merge is weighted by them.
+//
+// Both kernels are HBM-bound row movers: one warp per token, 16-byte (8 x bf16) vector
+// accesses, every lane a different 16-byte column of the row, so each warp instruction
+// touches 512 contiguous bytes.
+//   permute:   reads token row t once, writes its k copies   ->  (1 + k) * H * 2 bytes
+//   unpermute: reads the k expert rows of token t, writes one ->  (k + 1) * H * 2 bytes
+#include "device.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kRowThreads = 256;          // 8 tokens per CTA
+constexpr int kTokPerCta = kRowThreads / 32;
+
+__device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// X[dst[t*k+j]] = hidden[t] for every j < k.
+template <int U>
+__global__ void __launch_bounds__(kRowThreads) permute_kernel(const uint4* __restrict__ hidden,
+                                                              const int32_t* __restrict__ dst,
+                                                              int64_t Tc, int32_t H8, int32_t k,
+                                                              uint4* __restrict__ X) {
+  const int64_t t = (int64_t)blockIdx.x * kTokPerCta + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= Tc) return;
+  const int32_t d_lane = lane < k ? dst[t * k + lane] : 0;
+  const uint4* src = hidden + t * H8;
+  for (int32_t v0 = 0; v0 < H8; v0 += 32 * U) {
+    uint4 val[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int32_t v = v0 + u * 32 + lane;
+      if (v < H8) val[u] = ldg_stream(src + v);
+    }
+    for (int j = 0; j < k; ++j) {
+      const int32_t d = __shfl_sync(0xffffffffu, d_lane, j);
+      uint4* row = X + (int64_t)d * H8;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int32_t v = v0 + u * 32 + lane;
+        if (v < H8) row[v] = val[u];
+      }
+    }
+  }
+}
+
+// out[t] = bf16( sum_{j<k} w[t*k+j] * Y[dst[t*k+j]] ), fp32 accumulation, j ascending.
+template <int U>
+__global__ void __launch_bounds__(kRowThreads) unpermute_kernel(const uint4* __restrict__ Y,
+                                                                const int32_t* __restrict__ dst,
+                                                                const float* __restrict__ w,
+                                                                int64_t Tc, int32_t H8, int32_t k,
+                                                                uint4* __restrict__ out) {
+  const int64_t t = (int64_t)blockIdx.x * kTokPerCta + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= Tc) return;
+  const int32_t d_lane = lane < k ? dst[t * k + lane] : 0;
+  const float w_lane = lane < k ? w[t * k + lane] : 0.f;
+  for (int32_t v0 = 0; v0 < H8; v0 += 32 * U) {
+    float acc[U][8];
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
+    for (int j = 0; j < k; ++j) {
+      const int32_t d = __shfl_sync(0xffffffffu, d_lane, j);
+      const float wj = __shfl_sync(0xffffffffu, w_lane, j);
+      const uint4* row = Y + (int64_t)d * H8;
+      uint4 y[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int32_t v = v0 + u * 32 + lane;
+        y[u] = v < H8 ? ldg_stream(row + v) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const uint32_t q[4] = {y[u].x, y[u].y, y[u].z, y[u].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[u][2 * i] = fmaf(wj, bf16lo(q[i]), acc[u][2 * i]);
+          acc[u][2 * i + 1] = fmaf(wj, bf16hi(q[i]), acc[u][2 * i + 1]);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int32_t v = v0 + u * 32 + lane;
+      if (v < H8) {
+        uint4 o;
+        o.x = pack_bf16x2(acc[u][0], acc[u][1]);
+        o.y = pack_bf16x2(acc[u][2], acc[u][3]);
+        o.z = pack_bf16x2(acc[u][4], acc[u][5]);
+        o.w = pack_bf16x2(acc[u][6], acc[u][7]);
+        out[t * H8 + v] = o;
+      }
+    }
+  }
+}
+
+inline unsigned grid_for(int64_t Tc) { return (unsigned)((Tc + kTokPerCta - 1) / kTokPerCta); }
+
+}  // namespace
+
+cudaError_t launch_permute(const void* hidden, const int32_t* dst, int64_t Tc, int32_t H,
+                           int32_t k, void* X, cudaStream_t s) {
+  if (Tc <= 0) return cudaSuccess;
+  permute_kernel<4><<<grid_for(Tc), kRowThreads, 0, s>>>(
+      static_cast<const uint4*>(hidden), dst, Tc, H / 8, k, static_cast<uint4*>(X));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpermute(const void* Y, const int32_t* dst, const float* w, int64_t Tc,
+                             int32_t H, int32_t k, void* out, cudaStream_t s) {
+  if (Tc <= 0) return cudaSuccess;
+  unpermute_kernel<2><<<grid_for(Tc), kRowThreads, 0, s>>>(
+      static_cast<const uint4*>(Y), dst, w, Tc, H / 8, k, static_cast<uint4*>(out));
+  return cudaGetLastError();
+}
+
+}  // namespace moe

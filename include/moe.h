@@ -47,6 +47,12 @@ extern "C" {
 
 #define MOE_ABI_VERSION 1
 
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
 typedef enum {
   MOE_OK = 0,
   MOE_ERR_ARG = 1,         /* null pointer, bad dimension, E % ep_groups != 0, k > E, ... */
@@ -61,6 +67,7 @@ typedef enum {
 /* Kernel limits.  Shapes beyond them return MOE_ERR_UNSUPPORTED. */
 #define MOE_MAX_EXPERTS 1024   /* E  */
 #define MOE_MAX_TOPK 32        /* k  */
+#define MOE_MAX_CHUNKS 1048576 /* num_chunks */
 
 /* Shape of one MoE layer call.
  *   T          tokens (rows of hidden / out), T >= 0; T * k < 2^31
@@ -78,20 +85,20 @@ typedef struct {
 } moe_shape_t;
 
 /* Human-readable name of a status code (static string, never NULL). */
-const char* moe_status_string(moe_status_t status);
+MOE_API const char* moe_status_string(moe_status_t status);
 
 /* MOE_ABI_VERSION of the loaded library. */
-int32_t moe_abi_version(void);
+MOE_API int32_t moe_abi_version(void);
 
 /* Chunk partition, host arithmetic only ([ChunkMoE] "一组关键公式": T_chunk = ceil(T/N)).
  * Writes N_eff + 1 bounds, N_eff = max(num_chunks, 1): chunk c holds tokens
  * [bounds[c], bounds[c+1]) with bounds[c] = min(T, c * T_chunk).  Trailing chunks may
  * be empty (T=49, N=8 gives seven chunks of 7 and one of 0).
  * Errors: MOE_ERR_ARG if bounds is NULL, T < 0 or num_chunks < 0. */
-moe_status_t moe_chunk_bounds(int64_t T, int32_t num_chunks, int64_t* bounds /* host [N_eff+1] */);
+MOE_API moe_status_t moe_chunk_bounds(int64_t T, int32_t num_chunks, int64_t* bounds /* host [N_eff+1] */);
 
 /* Device workspace, in bytes, that moe_metadata needs for these sizes; 0 if invalid. */
-size_t moe_metadata_workspace_bytes(int64_t T, int32_t k, int32_t E, int32_t ep_groups,
+MOE_API size_t moe_metadata_workspace_bytes(int64_t T, int32_t k, int32_t E, int32_t ep_groups,
                                     int32_t num_chunks);
 
 /* Device workspace, in bytes, that moe_forward needs for this shape; 0 if invalid.
@@ -100,7 +107,7 @@ size_t moe_metadata_workspace_bytes(int64_t T, int32_t k, int32_t E, int32_t ep_
  * (W_pair = O(2 * T_chunk)).  The permuted input rows and the expert output rows share
  * one buffer, because the down projection runs only after the gate/up projection has
  * consumed every permuted row of the chunk. */
-size_t moe_workspace_bytes(const moe_shape_t* shape);
+MOE_API size_t moe_workspace_bytes(const moe_shape_t* shape);
 
 /* Batched pre-dispatch metadata for all chunks ([ChunkMoE] "一张专业时序图", the
  * batched_pre_dispatch_metadata paragraph: one pass for all chunks, one host copy).
@@ -125,7 +132,7 @@ size_t moe_workspace_bytes(const moe_shape_t* shape);
  * Errors: MOE_ERR_ARG, MOE_ERR_ALIGN, MOE_ERR_WORKSPACE, MOE_ERR_UNSUPPORTED (host
  * checks); MOE_ERR_INDEX if any index is outside [0, E) (outputs then unspecified);
  * MOE_ERR_CUDA. */
-moe_status_t moe_metadata(const int32_t* top_k_index, int64_t T, int32_t k, int32_t E,
+MOE_API moe_status_t moe_metadata(const int32_t* top_k_index, int64_t T, int32_t k, int32_t E,
                           int32_t ep_groups, int32_t num_chunks, int32_t* send_splits,
                           int32_t* recv_splits, int32_t* expert_counts, int64_t* chunk_bounds,
                           int32_t* dst_rows, int32_t* src_tokens, void* workspace,
@@ -154,14 +161,14 @@ moe_status_t moe_metadata(const int32_t* top_k_index, int64_t T, int32_t k, int3
  * T == 0 returns MOE_OK and launches nothing.
  * Errors: as moe_metadata.  A kernel that gives up a bounded wait records it in the
  * workspace; moe_check_device_status reports it. */
-moe_status_t moe_forward(const moe_shape_t* shape, const void* hidden, const int32_t* top_k_index,
+MOE_API moe_status_t moe_forward(const moe_shape_t* shape, const void* hidden, const int32_t* top_k_index,
                          const float* top_k_weights, const void* W_gate_up, const void* W_down,
                          void* out, void* workspace, size_t ws_bytes, void* stream);
 
 /* Synchronizes `stream` and returns MOE_ERR_TIMEOUT if a kernel of an earlier call that
  * used this workspace gave up a bounded wait, MOE_ERR_INDEX if its last metadata pass
  * saw a bad index, else MOE_OK (or MOE_ERR_CUDA). */
-moe_status_t moe_check_device_status(const void* workspace, size_t ws_bytes, void* stream);
+MOE_API moe_status_t moe_check_device_status(const void* workspace, size_t ws_bytes, void* stream);
 
 /* ---- Stage entry points ------------------------------------------------------------
  * The kernels of moe_forward, one call each, on caller buffers.  moe_forward does not
@@ -173,7 +180,7 @@ moe_status_t moe_check_device_status(const void* workspace, size_t ws_bytes, voi
  *   X[dst_rows[t*k+j]] = hidden[t]  for t < Tc, j < k.
  * hidden dev bf16 [Tc][H]; dst_rows dev int32 [Tc*k] (chunk-local rows, a bijection onto
  * [0, Tc*k)); X dev bf16 [Tc*k][H].  hidden and X 16-byte aligned. */
-moe_status_t moe_permute(const void* hidden, const int32_t* dst_rows, int64_t Tc, int32_t H,
+MOE_API moe_status_t moe_permute(const void* hidden, const int32_t* dst_rows, int64_t Tc, int32_t H,
                          int32_t k, void* X, void* stream);
 
 /* Expert gate/up projection with SwiGLU, grouped over experts (the expert computation of
@@ -182,7 +189,7 @@ moe_status_t moe_permute(const void* hidden, const int32_t* dst_rows, int64_t Tc
  * X dev bf16 [rows][H]; expert_offsets dev int32 [E+1] (offsets[0] = 0, nondecreasing,
  * offsets[E] = rows); expert_counts_host host int32 [E] (offsets[e+1] - offsets[e]);
  * W_gate_up dev bf16 [E][2I][H]; Act dev bf16 [rows][I].  16-byte aligned. */
-moe_status_t moe_grouped_gateup(const void* X, int64_t rows, int32_t H, int32_t I, int32_t E,
+MOE_API moe_status_t moe_grouped_gateup(const void* X, int64_t rows, int32_t H, int32_t I, int32_t E,
                                 const int32_t* expert_offsets, const int32_t* expert_counts_host,
                                 const void* W_gate_up, void* Act, uint32_t* status, void* stream);
 
@@ -190,7 +197,7 @@ moe_status_t moe_grouped_gateup(const void* X, int64_t rows, int32_t H, int32_t 
  *   Y[r] = bf16( Act[r] · W_down[e]^T ), fp32 accumulation.
  * Act dev bf16 [rows][I]; W_down dev bf16 [E][H][I]; Y dev bf16 [rows][H]; other
  * arguments as moe_grouped_gateup.  Y may alias the X of the gate/up call. */
-moe_status_t moe_grouped_down(const void* Act, int64_t rows, int32_t H, int32_t I, int32_t E,
+MOE_API moe_status_t moe_grouped_down(const void* Act, int64_t rows, int32_t H, int32_t I, int32_t E,
                               const int32_t* expert_offsets, const int32_t* expert_counts_host,
                               const void* W_down, void* Y, uint32_t* status, void* stream);
 
@@ -198,7 +205,7 @@ moe_status_t moe_grouped_down(const void* Act, int64_t rows, int32_t H, int32_t 
  *   out[t] = bf16( sum_{j<k} w[t*k+j] * float(Y[dst_rows[t*k+j]]) ), fp32, j ascending.
  * Y dev bf16 [Tc*k][H]; dst_rows dev int32 [Tc*k]; w dev fp32 [Tc*k]; out dev bf16
  * [Tc][H].  Y and out 16-byte aligned. */
-moe_status_t moe_unpermute(const void* Y, const int32_t* dst_rows, const float* top_k_weights,
+MOE_API moe_status_t moe_unpermute(const void* Y, const int32_t* dst_rows, const float* top_k_weights,
                            int64_t Tc, int32_t H, int32_t k, void* out, void* stream);
 
 /* ---- Kernel timing -----------------------------------------------------------------
@@ -223,8 +230,8 @@ typedef struct {
   int64_t kernels;                     /* device kernels launched while enabled          */
 } moe_profile_t;
 
-moe_status_t moe_profile_enable(int32_t on);  /* also clears the totals */
-moe_status_t moe_profile_read(moe_profile_t* out);
+MOE_API moe_status_t moe_profile_enable(int32_t on);  /* also clears the totals */
+MOE_API moe_status_t moe_profile_read(moe_profile_t* out);
 
 #ifdef __cplusplus
 }
