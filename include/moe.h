@@ -138,6 +138,42 @@ MOE_API moe_status_t moe_metadata(const int32_t* top_k_index, int64_t T, int32_t
                           int32_t* dst_rows, int32_t* src_tokens, void* workspace,
                           size_t ws_bytes, void* stream);
 
+/* Size of the fixed device scratch array behind moe_metadata_noalloc (1 MiB). */
+#define MOE_NOALLOC_SCRATCH_BYTES (1u << 20)
+
+/* moe_metadata for callers that cannot allocate.  The Chunk MoE pages have no
+ * counterpart of this entry point; it exists for callers that must not allocate device
+ * or pinned host memory where they need the routing metadata: a runtime whose device
+ * memory belongs entirely to its own caching allocator and forbids out-of-band
+ * cudaMalloc/cudaFree (cudaFree also synchronizes the whole device), a latency-critical
+ * serving path that cannot pay for an allocation, or a plugin that is handed only its
+ * inputs and outputs.
+ *
+ * Same results as moe_metadata, with these differences:
+ *  - No workspace argument: the scratch (status word, per-chunk counts, offsets and
+ *    splits, per-tile histograms) lives in one file-scope device array of
+ *    MOE_NOALLOC_SCRATCH_BYTES that every GPU which loads the library holds until the
+ *    process exits.  The call needs
+ *        a(16 + 4*N*(E+G)) + a(4*N*(E+1)) + a(4*N*ceil(ceil(T/N) / floor(2048/k))*E)
+ *    bytes of it (a() rounds up to 256, N = max(num_chunks,1), G = max(ep_groups,1));
+ *    larger sizes return MOE_ERR_WORKSPACE before anything is launched.
+ *  - dst_rows is required (not NULL) when T > 0; src_tokens stays optional.
+ *  - It allocates nothing: no cudaMalloc/cudaFree, no pinned host block, no stream or
+ *    event creation; the packed results come back through a fixed host array.
+ *  - The first call on each device looks up the device address of the scratch array
+ *    (cudaGetSymbolAddress, with that device current); make that first call before any
+ *    stream capture.
+ *  - Every call shares the one array and finds the previous call's contents in it; the
+ *    call clears the status word and overwrites everything else it reads.  Calls whose
+ *    work overlaps on the GPU (several streams or host threads) race on the array and
+ *    on the host array: serialize them.
+ * Errors: as moe_metadata, plus MOE_ERR_WORKSPACE for sizes beyond the array. */
+MOE_API moe_status_t moe_metadata_noalloc(const int32_t* top_k_index, int64_t T, int32_t k,
+                                          int32_t E, int32_t ep_groups, int32_t num_chunks,
+                                          int32_t* send_splits, int32_t* recv_splits,
+                                          int32_t* expert_counts, int64_t* chunk_bounds,
+                                          int32_t* dst_rows, int32_t* src_tokens, void* stream);
+
 /* One MoE layer forward pass, chunked as Chunk MoE ([ChunkMoE] "核心原理",
  * "一张专业时序图", "一组关键公式"):
  *     out[t] = bf16( sum_{j<k} top_k_weights[t][j] * FFN_{top_k_index[t][j]}(hidden[t]) )
