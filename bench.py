@@ -53,6 +53,19 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def max_over_ranks(ms, dist_mod=None, device="cpu"):
+    """The slowest rank's time: every multi-GPU number is the max over ranks."""
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    if dist_mod is not None:
+        dist_mod.all_reduce(t, op=dist_mod.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world, tokens_per_rank, steps, ms_max):
+    """Whole-job throughput: the tokens all replicas processed / the slowest rank's time."""
+    return world * tokens_per_rank * steps / (ms_max / 1e3)
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -308,12 +321,9 @@ def run_ours(args, cfg):
     moe.profile_enable(False)
     clk = clocks.stop() if clocks else None
 
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if pg:
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, pg, dev)
     ms_per_step = ms_max / args.steps
-    value = world * cfg.T * args.steps / (ms_max / 1e3)
+    value = job_tokens_per_s(world, cfg.T, args.steps, ms_max)
 
     # N = 1 reference point of the same workload (for the <= 5 % loss target), untimed key
     ms_n1 = None
@@ -426,12 +436,9 @@ def run_e2e(moe, inp, cfg, chunks, ws, args, stream, dev, pg, world):
         step()
     e.record(stream)
     torch.cuda.synchronize()
-    t = torch.tensor([s.elapsed_time(e)], dtype=torch.float64, device=dev)
-    if pg:
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-    ms = float(t.item())
+    ms = max_over_ranks(s.elapsed_time(e), pg, dev)
     h2d = h_pin.numel() * 2 + i_pin.numel() * 4 + w_pin.numel() * 4
-    return {"value": world * cfg.T * steps / (ms / 1e3), "unit": "tokens/s",
+    return {"value": job_tokens_per_s(world, cfg.T, steps, ms), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": o_pin.numel() * 2,
             "steps": steps}
 
