@@ -29,16 +29,55 @@
 #include "device.cuh"
 #include "internal.h"
 
+// Build-time tuning knobs (the defaults are the shipped configuration).
+#ifndef MOE_GEMM_2SM
+#define MOE_GEMM_2SM 0  // 1: CTA pairs (tcgen05 cta_group::2, 256-row tiles); 0: single CTAs
+#endif
+#ifndef MOE_GEMM_BK
+#define MOE_GEMM_BK 64  // K per stage: 64 (128-byte swizzle rows) or 32 (64-byte swizzle rows)
+#endif
+#ifndef MOE_GEMM_STAGES
+#define MOE_GEMM_STAGES (MOE_GEMM_BK == 64 ? 4 : 8)  // single-CTA ring depth
+#endif
+#ifndef MOE_GEMM_STAGES_2SM
+#define MOE_GEMM_STAGES_2SM (MOE_GEMM_BK == 64 ? 6 : 12)  // CTA-pair ring depth
+#endif
+#ifndef MOE_GEMM_L2_PROMO
+#define MOE_GEMM_L2_PROMO 2  // TMA L2 promotion: 0 none, 1 128 B, 2 256 B
+#endif
+#ifndef MOE_GEMM_ORDER
+#define MOE_GEMM_ORDER 0  // tile order inside an expert: 0 M tile fastest, 1 N tile fastest
+#endif
+#ifndef MOE_GEMM_EPI_STAGE
+#define MOE_GEMM_EPI_STAGE 1  // 1: stage output blocks in shared memory for coalesced stores
+#endif
+#ifndef MOE_GEMM_B_POLICY
+#define MOE_GEMM_B_POLICY 2  // L2 policy of weight loads: 0 normal, 1 evict_first, 2 evict_last
+#endif
+
 namespace moe {
 namespace {
 
-constexpr int BM = kGemmBM, BN = kGemmBN, BK = kGemmBK, STAGES = kGemmStages;
-constexpr uint32_t kABytes = BM * BK * 2;  // 16 KB
-constexpr uint32_t kBBytes = BN * BK * 2;  // 32 KB
-constexpr uint32_t kStageBytes = kABytes + kBBytes;
-constexpr uint32_t kTmemCols = 2 * BN;  // two accumulators
-constexpr uint32_t kIdesc = umma_idesc_bf16_f32(BM, BN);
+constexpr int BN = kGemmBN, BK = MOE_GEMM_BK;
+static_assert(BK == 64 || BK == 32, "K block of 64 (128-byte swizzle) or 32 (64-byte swizzle)");
+constexpr uint32_t kSwizzleBytes = BK * 2;  // one swizzled row = the K block of one matrix row
+constexpr int kRowsPerCta = 128;            // accumulator rows per CTA (TMEM lanes)
+constexpr uint32_t kTmemCols = 2 * BN;      // two accumulators of BN fp32 columns
 constexpr int kMaxE = 1024;
+
+// Geometry of one variant: single CTA (128x256 tiles) or CTA pair (256x256 tiles, each
+// CTA staging its 128 A rows and half of the 256 B rows).
+template <bool kPair>
+struct Geo {
+  static constexpr int kTileM = kPair ? 2 * kRowsPerCta : kRowsPerCta;
+  static constexpr int kStages = kPair ? MOE_GEMM_STAGES_2SM : MOE_GEMM_STAGES;
+  static constexpr uint32_t kABytes = kRowsPerCta * BK * 2;                 // 16 KB
+  static constexpr uint32_t kBRows = kPair ? BN / 2 : BN;                   // B rows per CTA
+  static constexpr uint32_t kBBytes = kBRows * BK * 2;                      // 16 or 32 KB
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes;                // per CTA
+  static constexpr uint32_t kTxBytes = kPair ? 2 * kStageBytes : kStageBytes;  // per stage
+  static constexpr uint32_t kIdesc = umma_idesc_bf16_f32(kTileM, BN);
+};
 
 struct KParams {
   const int32_t* offsets;
@@ -53,9 +92,10 @@ struct KParams {
   int32_t total_tiles;
 };
 
+template <int kStages>
 struct SmemCtl {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
@@ -64,14 +104,27 @@ struct SmemCtl {
 };
 
 constexpr size_t kCtlBytes = 256;
-static_assert(sizeof(SmemCtl) <= kCtlBytes, "control block");
-constexpr size_t kSmemBytes = 1024 /*alignment slack*/ + STAGES * kStageBytes + kCtlBytes +
-                              2 * (kMaxE + 1) * sizeof(int32_t);
+static_assert(sizeof(SmemCtl<MOE_GEMM_STAGES_2SM>) <= kCtlBytes, "control block");
+static_assert(sizeof(SmemCtl<MOE_GEMM_STAGES>) <= kCtlBytes, "control block");
+
+// Epilogue staging: per epilogue warp one block of 32 rows x 32 bf16 columns, rows padded
+// to 80 bytes so that both the row-wise writes and the 8-rows-per-instruction reads are
+// free of bank conflicts within each 8-lane phase.
+constexpr int kEpiRowBytes = 80;
+constexpr int kEpiWarpBytes = 32 * kEpiRowBytes;
+constexpr size_t kTablesBytes = (2 * (kMaxE + 1) * sizeof(int32_t) + 15) & ~size_t(15);
+
+template <bool kPair>
+constexpr size_t smem_bytes() {
+  return 1024 /*alignment slack*/ + Geo<kPair>::kStages * Geo<kPair>::kStageBytes + kCtlBytes +
+         kTablesBytes + (MOE_GEMM_EPI_STAGE ? 4 * kEpiWarpBytes : 0);
+}
 
 struct Tile {
   int32_t e, n, m;
 };
 
+template <int kTileM>
 __device__ __forceinline__ Tile decode_tile(int32_t L, const int32_t* tile_start,
                                             const int32_t* off, int32_t E, int32_t n_tiles) {
   // largest e with tile_start[e] <= L; that expert has at least one tile
@@ -81,31 +134,84 @@ __device__ __forceinline__ Tile decode_tile(int32_t L, const int32_t* tile_start
     if (tile_start[mid] <= L) lo = mid;
     else hi = mid - 1;
   }
-  const int32_t mt = (off[lo + 1] - off[lo] + BM - 1) / BM;
+  const int32_t mt = (off[lo + 1] - off[lo] + kTileM - 1) / kTileM;
   const int32_t local = L - tile_start[lo];
   Tile t;
   t.e = lo;
+#if MOE_GEMM_ORDER == 0
   t.n = local / mt;
   t.m = local - t.n * mt;
   (void)n_tiles;
+#else
+  t.m = local / n_tiles;
+  t.n = local - t.m * n_tiles;
+#endif
   return t;
 }
 
-template <bool kSwiGLU>
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                        const __grid_constant__ CUtensorMap tmB, const KParams p) {
+// Stores the 32 x 32 bf16 block of one epilogue warp: lane i holds row (32 q + i) of the
+// tile as 16 packed bf16 pairs.  Rows at or past rows_valid (past the expert's end) and
+// columns at or past out_cols are never written.
+__device__ __forceinline__ void store_block(const uint32_t (&packed)[16], uint8_t* wbuf, int lane,
+                                            int q, bool row_ok, int32_t rows_valid,
+                                            int64_t row_base, int32_t col0, const KParams& p) {
+#if MOE_GEMM_EPI_STAGE
+  uint4* mine = reinterpret_cast<uint4*>(wbuf + lane * kEpiRowBytes);
+#pragma unroll
+  for (int v = 0; v < 4; ++v)
+    mine[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+  __syncwarp();
+  // 8 rows x 64 contiguous bytes per instruction: lane = 4 * (row % 8) + 16-byte segment
+  const int seg = lane & 3;
+  const int32_t col = col0 + seg * 8;
+#pragma unroll
+  for (int pass = 0; pass < 4; ++pass) {
+    const int rr = pass * 8 + (lane >> 2);
+    const uint4 v = *reinterpret_cast<const uint4*>(wbuf + rr * kEpiRowBytes + seg * 16);
+    const int32_t tr = q * 32 + rr;  // row inside the CTA's 128 rows
+    if (tr < rows_valid && col < p.out_cols)
+      *reinterpret_cast<uint4*>(p.out + (row_base + tr) * p.out_cols + col) = v;
+  }
+  __syncwarp();
+  (void)row_ok;
+#else
+  (void)wbuf;
+  (void)rows_valid;
+  if (row_ok) {
+    uint4* dst = reinterpret_cast<uint4*>(p.out + (row_base + q * 32 + lane) * p.out_cols + col0);
+#pragma unroll
+    for (int v = 0; v < 4; ++v)
+      if (col0 + v * 8 < p.out_cols)
+        dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+  }
+#endif
+}
+
+// One persistent CTA (kPair = false) or CTA pair (kPair = true, cluster of 2) per tile
+// stream.  In a pair, the even CTA ("leader") owns the full-stage barriers and the MMA
+// issue; both CTAs load their own halves, run their own epilogue on their own TMEM rows,
+// and report back to the leader.
+template <bool kSwiGLU, bool kPair>
+__device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensorMap* tmB,
+                                          const KParams& p) {
+  using G = Geo<kPair>;
+  constexpr int STAGES = G::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * kABytes;
-  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(smem + STAGES * kStageBytes);
-  int32_t* off = reinterpret_cast<int32_t*>(smem + STAGES * kStageBytes + kCtlBytes);
+  uint8_t* sB = smem + STAGES * G::kABytes;
+  SmemCtl<STAGES>* ctl = reinterpret_cast<SmemCtl<STAGES>*>(smem + STAGES * G::kStageBytes);
+  int32_t* off = reinterpret_cast<int32_t*>(smem + STAGES * G::kStageBytes + kCtlBytes);
   int32_t* tile_start = off + (kMaxE + 1);
+  uint8_t* epi_stage = smem + STAGES * G::kStageBytes + kCtlBytes + kTablesBytes;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int32_t E = p.E;
+  const uint32_t rank = kPair ? cluster_cta_rank() : 0;
+  const bool leader = rank == 0;
+  const int32_t stream_id = kPair ? (int32_t)(blockIdx.x >> 1) : (int32_t)blockIdx.x;
+  const int32_t n_streams = kPair ? (int32_t)(gridDim.x >> 1) : (int32_t)gridDim.x;
 
   // ---- set-up: expert offsets, tile prefix, barriers, TMEM ----
   for (int32_t i = threadIdx.x; i <= E; i += kGemmThreads) off[i] = p.offsets[i];
@@ -116,19 +222,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&ctl->tfull[b], 1);
-      mbar_init(&ctl->tempty[b], 4 * 32);
+      mbar_init(&ctl->tempty[b], (kPair ? 2 : 1) * 4 * 32);
     }
     mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(tmA);
+    tma_prefetch_desc(tmB);
   }
   if (warp == 1) {
-    tmem_alloc(&ctl->tmem_base, kTmemCols);
-    tmem_relinquish();
+    if (kPair) {
+      tmem_alloc_pair(&ctl->tmem_base, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&ctl->tmem_base, kTmemCols);
+      tmem_relinquish();
+    }
   }
   __syncthreads();
   if (warp == 2) {
@@ -136,7 +247,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int32_t per = (E + 31) / 32;
     const int32_t e0 = lane * per, e1 = min(E, e0 + per);
     int32_t sum = 0;
-    for (int32_t e = e0; e < e1; ++e) sum += ((off[e + 1] - off[e] + BM - 1) / BM) * p.n_tiles;
+    for (int32_t e = e0; e < e1; ++e)
+      sum += ((off[e + 1] - off[e] + G::kTileM - 1) / G::kTileM) * p.n_tiles;
     int32_t incl = sum;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -146,44 +258,62 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int32_t run = incl - sum;
     for (int32_t e = e0; e < e1; ++e) {
       tile_start[e] = run;
-      run += ((off[e + 1] - off[e] + BM - 1) / BM) * p.n_tiles;
+      run += ((off[e + 1] - off[e] + G::kTileM - 1) / G::kTileM) * p.n_tiles;
     }
     if (lane == 31) tile_start[E] = incl;
   }
   tc_fence_before();
-  __syncthreads();
+  if (kPair) cluster_sync();  // the peer's loads target the leader's barriers: init first
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
   volatile int* abort = &ctl->abort;
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
+    // ---------------- TMA producer (both CTAs) ----------------
     if (lane == 0) {
-      const uint64_t pol_w = l2_policy_evict_last();    // weights: reused by many M tiles
+#if MOE_GEMM_B_POLICY == 1
+      const uint64_t pol_w = l2_policy_evict_first();
+#elif MOE_GEMM_B_POLICY == 2
+      const uint64_t pol_w = l2_policy_evict_last();
+#else
+      const uint64_t pol_w = l2_policy_evict_normal();
+#endif
       const uint64_t pol_a = l2_policy_evict_normal();
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;  // per-stage bits, for the abort drain
       bool ok = true;
-      for (int32_t L = blockIdx.x; L < p.total_tiles && ok; L += gridDim.x) {
-        const Tile t = decode_tile(L, tile_start, off, E, p.n_tiles);
-        const int32_t row0 = off[t.e] + t.m * BM;
-        const int32_t brow = t.e * p.b_rows + t.n * (kSwiGLU ? BN / 2 : BN);
+      for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
+        const Tile t = decode_tile<G::kTileM>(L, tile_start, off, E, p.n_tiles);
+        const int32_t row0 = off[t.e] + t.m * G::kTileM + (int32_t)rank * kRowsPerCta;
+        int32_t brow;
+        if (kSwiGLU)  // pair: the even CTA stages the gate rows, the odd one the up rows
+          brow = t.e * p.b_rows + t.n * (BN / 2) + (kPair ? (int32_t)rank * p.up_off : 0);
+        else
+          brow = t.e * p.b_rows + t.n * BN + (kPair ? (int32_t)rank * (BN / 2) : 0);
         for (int32_t kb = 0; kb < p.num_kb; ++kb) {
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort, p.status)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&ctl->full[stage], kStageBytes);
-          uint8_t* a_dst = sA + stage * kABytes;
-          uint8_t* b_dst = sB + stage * kBBytes;
-          tma_load_2d(a_dst, &tmA, &ctl->full[stage], kb * BK, row0, pol_a);
-          if (kSwiGLU) {
-            tma_load_2d(b_dst, &tmB, &ctl->full[stage], kb * BK, brow, pol_w);
-            tma_load_2d(b_dst + kBBytes / 2, &tmB, &ctl->full[stage], kb * BK, brow + p.up_off,
-                        pol_w);
+          uint8_t* a_dst = sA + stage * G::kABytes;
+          uint8_t* b_dst = sB + stage * G::kBBytes;
+          if (kPair) {
+            if (leader) mbar_arrive_expect_tx(&ctl->full[stage], G::kTxBytes);
+            const uint32_t bar = mapa_shared(smem_u32(&ctl->full[stage]), 0);
+            tma_load_2d_pair(a_dst, tmA, bar, kb * BK, row0, pol_a);
+            tma_load_2d_pair(b_dst, tmB, bar, kb * BK, brow, pol_w);
           } else {
-            tma_load_2d(b_dst, &tmB, &ctl->full[stage], kb * BK, brow, pol_w);
+            mbar_arrive_expect_tx(&ctl->full[stage], G::kTxBytes);
+            tma_load_2d(a_dst, tmA, &ctl->full[stage], kb * BK, row0, pol_a);
+            if (kSwiGLU) {
+              tma_load_2d(b_dst, tmB, &ctl->full[stage], kb * BK, brow, pol_w);
+              tma_load_2d(b_dst + G::kBBytes / 2, tmB, &ctl->full[stage], kb * BK,
+                          brow + p.up_off, pol_w);
+            } else {
+              tma_load_2d(b_dst, tmB, &ctl->full[stage], kb * BK, brow, pol_w);
+            }
           }
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
@@ -193,20 +323,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
-      if (!ok) {
+      if (!ok && leader) {
         // wait (bounded) for the copies already issued, so none lands after exit
         for (int s = 0; s < STAGES; ++s)
           if (armed & (1u << s)) mbar_drain(&ctl->full[s], (armed_parity >> s) & 1u, 100000000ull);
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
+    // ---------------- MMA issuer (the leader only) ----------------
+    if (lane == 0 && leader) {
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true, issued = false;
       int32_t it = 0;
-      for (int32_t L = blockIdx.x; L < p.total_tiles && ok; L += gridDim.x, ++it) {
+      for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams, ++it) {
         const int buf = it & 1;
         const uint32_t tphase = (it >> 1) & 1;
         if (!mbar_wait(&ctl->tempty[buf], tphase ^ 1u, abort, p.status)) {
@@ -221,44 +351,53 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(sA + stage * kABytes);
-          const uint32_t b_addr = smem_u32(sB + stage * kBBytes);
+          const uint32_t a_addr = smem_u32(sA + stage * G::kABytes);
+          const uint32_t b_addr = smem_u32(sB + stage * G::kBBytes);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            // advance 16 bf16 = 32 bytes along K inside the 128-byte swizzled row
-            umma_bf16(d_tmem, sw128_kmajor_desc(a_addr + kk * 32),
-                      sw128_kmajor_desc(b_addr + kk * 32), kIdesc, (kb | kk) != 0);
+            // advance 16 bf16 = 32 bytes along K inside the swizzled row
+            const uint64_t ad = kmajor_desc<kSwizzleBytes>(a_addr + kk * 32);
+            const uint64_t bd = kmajor_desc<kSwizzleBytes>(b_addr + kk * 32);
+            if (kPair) umma_bf16_pair(d_tmem, ad, bd, G::kIdesc, (kb | kk) != 0);
+            else umma_bf16(d_tmem, ad, bd, G::kIdesc, (kb | kk) != 0);
           }
           issued = true;
-          umma_commit(&ctl->empty[stage]);
+          if (kPair) umma_commit_pair(&ctl->empty[stage], 0x3);
+          else umma_commit(&ctl->empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        umma_commit(&ctl->tfull[buf]);
+        if (kPair) umma_commit_pair(&ctl->tfull[buf], 0x3);
+        else umma_commit(&ctl->tfull[buf]);
       }
       if (!ok && issued) {
         // every MMA issued so far must finish before TMEM is released
-        umma_commit(&ctl->drain);
+        if (kPair) umma_commit_pair(&ctl->drain, 0x1);
+        else umma_commit(&ctl->drain);
         mbar_drain(&ctl->drain, 0, 100000000ull);
       }
     }
   } else {
-    // ---------------- epilogue (warps 2..5) ----------------
+    // ---------------- epilogue (warps 2..5 of both CTAs) ----------------
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int r = q * 32 + lane;
+    uint8_t* wbuf = epi_stage + (warp - 2) * kEpiWarpBytes;
+    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&ctl->tempty[0]), 0);
+    const uint32_t tempty_leader1 = mapa_shared(smem_u32(&ctl->tempty[1]), 0);
     int32_t it = 0;
-    for (int32_t L = blockIdx.x; L < p.total_tiles; L += gridDim.x, ++it) {
+    for (int32_t L = stream_id; L < p.total_tiles; L += n_streams, ++it) {
       const int buf = it & 1;
       const uint32_t tphase = (it >> 1) & 1;
       if (!mbar_wait(&ctl->tfull[buf], tphase, abort, p.status)) break;
       tc_fence_after();
-      const Tile t = decode_tile(L, tile_start, off, E, p.n_tiles);
-      const int32_t rows_valid = off[t.e + 1] - off[t.e] - t.m * BM;
+      const Tile t = decode_tile<G::kTileM>(L, tile_start, off, E, p.n_tiles);
+      const int32_t first = t.m * G::kTileM + (int32_t)rank * kRowsPerCta;  // in the expert
+      const int32_t rows_valid = off[t.e + 1] - off[t.e] - first;
       const bool row_ok = r < rows_valid;
-      const int64_t row = (int64_t)off[t.e] + t.m * BM + r;
+      const int64_t row_base = (int64_t)off[t.e] + first;  // output row of TMEM lane 0
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * BN;
       if (kSwiGLU) {
 #pragma unroll 1
@@ -268,23 +407,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tmem_ld_32cols(t_row + BN / 2 + c * 32, u);
           tmem_ld_wait2(g, u);
           const int32_t col0 = t.n * (BN / 2) + c * 32;
-          if (row_ok) {
-            uint32_t packed[16];
+          uint32_t packed[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
-              const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
-              const float a0 = g0 / (1.0f + __expf(-g0)) * u0;
-              const float a1 = g1 / (1.0f + __expf(-g1)) * u1;
-              packed[i] = pack_bf16x2(a0, a1);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(p.out + row * p.out_cols + col0);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              if (col0 + v * 8 < p.out_cols)
-                dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2],
-                                    packed[4 * v + 3]);
+          for (int i = 0; i < 16; ++i) {
+            const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+            const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+            const float a0 = g0 / (1.0f + __expf(-g0)) * u0;
+            const float a1 = g1 / (1.0f + __expf(-g1)) * u1;
+            packed[i] = pack_bf16x2(a0, a1);
           }
+          store_block(packed, wbuf, lane, q, row_ok, rows_valid, row_base, col0, p);
         }
       } else {
 #pragma unroll 1
@@ -293,32 +425,43 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tmem_ld_32cols(t_row + c * 32, acc);
           tmem_ld_wait(acc);
           const int32_t col0 = t.n * BN + c * 32;
-          if (row_ok) {
-            uint32_t packed[16];
+          uint32_t packed[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              packed[i] = pack_bf16x2(__uint_as_float(acc[2 * i]), __uint_as_float(acc[2 * i + 1]));
-            uint4* dst = reinterpret_cast<uint4*>(p.out + row * p.out_cols + col0);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              if (col0 + v * 8 < p.out_cols)
-                dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2],
-                                    packed[4 * v + 3]);
-          }
+          for (int i = 0; i < 16; ++i)
+            packed[i] = pack_bf16x2(__uint_as_float(acc[2 * i]), __uint_as_float(acc[2 * i + 1]));
+          store_block(packed, wbuf, lane, q, row_ok, rows_valid, row_base, col0, p);
         }
       }
       tc_fence_before();
-      mbar_arrive(&ctl->tempty[buf]);
+      if (kPair) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
+      else mbar_arrive(&ctl->tempty[buf]);
     }
   }
 
   tc_fence_before();
-  __syncthreads();
+  if (kPair) cluster_sync();  // both CTAs are done with each other's barriers, smem, TMEM
+  else __syncthreads();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if (kPair) tmem_dealloc_pair(tmem_base, kTmemCols);
+    else tmem_dealloc(tmem_base, kTmemCols);
   }
+}
+
+template <bool kSwiGLU>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB, const KParams p) {
+  gemm_body<kSwiGLU, false>(&tmA, &tmB, p);
+}
+
+// Launched with a cluster of 2 CTAs (cudaLaunchAttributeClusterDimension).
+template <bool kSwiGLU>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                             const __grid_constant__ CUtensorMap tmB, const KParams p) {
+  gemm_body<kSwiGLU, true>(&tmA, &tmB, p);
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -340,7 +483,7 @@ EncodeTiledFn get_encode_fn() {
 }
 
 // 2-D bf16 tensor map over a row-major [rows][cols] matrix with a box of
-// box_rows x 64 columns and the 128-byte swizzle; out-of-range elements read as zero.
+// box_rows x BK columns and the matching swizzle; out-of-range elements read as zero.
 bool make_map(CUtensorMap* m, const void* base, int64_t rows, int32_t cols, int32_t box_rows) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
@@ -349,8 +492,11 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int32_t cols, int3
   const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             BK == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+             MOE_GEMM_L2_PROMO == 2   ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+             : MOE_GEMM_L2_PROMO == 1 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
+                                      : CU_TENSOR_MAP_L2_PROMOTION_NONE,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -358,14 +504,16 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int32_t cols, int3
 
 int64_t gemm_total_tiles(const int32_t* counts_host, int32_t E, int32_t out_cols, bool swiglu) {
   const int32_t bn = swiglu ? BN / 2 : BN;
+  const int32_t tm = Geo<MOE_GEMM_2SM != 0>::kTileM;
   const int64_t n_tiles = (out_cols + bn - 1) / bn;
   int64_t m_tiles = 0;
-  for (int32_t e = 0; e < E; ++e) m_tiles += (counts_host[e] + BM - 1) / BM;
+  for (int32_t e = 0; e < E; ++e) m_tiles += (counts_host[e] + tm - 1) / tm;
   return m_tiles * n_tiles;
 }
 
 cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cudaStream_t s,
                                 int* err_detail) {
+  constexpr bool kPair = MOE_GEMM_2SM != 0;
   *err_detail = 0;
   if (a.total_tiles <= 0) return cudaSuccess;
   if (a.total_tiles > 0x7fffffff || a.E > kMaxE) {
@@ -374,8 +522,9 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
   }
   CUtensorMap mA, mB;
   const int32_t bn = swiglu ? BN / 2 : BN;
-  if (!make_map(&mA, a.A, a.rows, a.K, BM) ||
-      !make_map(&mB, a.B, (int64_t)a.E * a.b_rows, a.K, swiglu ? BN / 2 : BN)) {
+  if (!make_map(&mA, a.A, a.rows, a.K, kRowsPerCta) ||
+      !make_map(&mB, a.B, (int64_t)a.E * a.b_rows, a.K,
+                kPair ? BN / 2 : (swiglu ? BN / 2 : BN))) {
     *err_detail = 2;
     return cudaErrorInvalidValue;
   }
@@ -390,18 +539,45 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
   p.b_rows = a.b_rows;
   p.up_off = swiglu ? a.out_cols : 0;
   p.total_tiles = (int32_t)a.total_tiles;
-  const int grid = (int)(a.total_tiles < num_sms ? a.total_tiles : num_sms);
+  constexpr size_t smem = smem_bytes<kPair>();
   cudaError_t e;
-  if (swiglu) {
-    e = cudaFuncSetAttribute(grouped_gemm_kernel<true>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  if (kPair) {
+    auto k = swiglu ? grouped_gemm_pair_kernel<true> : grouped_gemm_pair_kernel<false>;
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    grouped_gemm_kernel<true><<<grid, kGemmThreads, kSmemBytes, s>>>(mA, mB, p);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // persistent: as many CTA pairs as can be resident at once
+    static int max_pairs[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int& mp = max_pairs[dev & 63];
+    if (mp <= 0) {
+      cfg.gridDim = dim3(num_sms, 1, 1);
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, (void*)k, &cfg) != cudaSuccess || n <= 0)
+        n = num_sms / 2;
+      mp = n < num_sms / 2 ? n : num_sms / 2;
+    }
+    const int streams = (int)(a.total_tiles < mp ? a.total_tiles : mp);
+    cfg.gridDim = dim3(2 * streams, 1, 1);
+    e = cudaLaunchKernelEx(&cfg, k, mA, mB, p);
+    if (e != cudaSuccess) return e;
   } else {
-    e = cudaFuncSetAttribute(grouped_gemm_kernel<false>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    auto k = swiglu ? grouped_gemm_kernel<true> : grouped_gemm_kernel<false>;
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    grouped_gemm_kernel<false><<<grid, kGemmThreads, kSmemBytes, s>>>(mA, mB, p);
+    const int streams = (int)(a.total_tiles < num_sms ? a.total_tiles : num_sms);
+    k<<<streams, kGemmThreads, smem, s>>>(mA, mB, p);
   }
   return cudaGetLastError();
 }
