@@ -238,7 +238,7 @@ def run_reference(args, cfg):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_block(cfg, args.chunks),
+        "config": config_block(cfg, args.chunks, args.dispatch),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -248,17 +248,18 @@ def run_reference(args, cfg):
     return 0
 
 
-def config_block(cfg, chunks):
+def config_block(cfg, chunks, dispatch="separate"):
     wbytes = 6 * cfg.E * cfg.H * cfg.I
     return {"workload": workload_name(cfg), "T": cfg.T, "H": cfg.H, "E": cfg.E, "k": cfg.k,
-            "I": cfg.I, "ep_groups": cfg.G, "num_chunks": chunks, "routing": cfg.routing,
+            "I": cfg.I, "ep_groups": cfg.G, "num_chunks": chunks, "dispatch": dispatch,
+            "routing": cfg.routing,
             "ffn": "SwiGLU", "parallelism": "replicas",
             "l2": f"inputs larger than L2 ({wbytes / 1e9:.2f} GB of expert weights read per step)"}
 
 
 # ------------------------------------------------------------------------- our arm
 
-def time_steps(moe, inp, cfg, chunks, ws, steps, stream):
+def time_steps(moe, inp, cfg, chunks, ws, steps, stream, dispatch="separate"):
     """Device time of `steps` back-to-back forward calls, ms (CUDA events on `stream`)."""
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
@@ -267,7 +268,8 @@ def time_steps(moe, inp, cfg, chunks, ws, steps, stream):
     start.record(stream)
     for _ in range(steps):
         moe.forward(inp["hidden"], inp["idx"], inp["w"], inp["wgu"], inp["wd"],
-                    num_chunks=chunks, ep_groups=cfg.G, out=out, workspace=ws, stream=stream)
+                    num_chunks=chunks, ep_groups=cfg.G, out=out, workspace=ws, stream=stream,
+                    dispatch=dispatch)
     end.record(stream)
     torch.cuda.synchronize()
     return start.elapsed_time(end), out
@@ -303,7 +305,7 @@ def run_ours(args, cfg):
 
     for _ in range(args.warmup):
         moe.forward(inp["hidden"], inp["idx"], inp["w"], inp["wgu"], inp["wd"],
-                    num_chunks=chunks, ep_groups=cfg.G, workspace=ws)
+                    num_chunks=chunks, ep_groups=cfg.G, workspace=ws, dispatch=args.dispatch)
     torch.cuda.synchronize()
 
     clocks = ClockSampler(local) if rank == 0 else None
@@ -314,7 +316,7 @@ def run_ours(args, cfg):
         pg.barrier()
     torch.cuda.synchronize()
     moe.profile_enable(True)
-    ms, out = time_steps(moe, inp, cfg, chunks, ws, args.steps, stream)
+    ms, out = time_steps(moe, inp, cfg, chunks, ws, args.steps, stream, args.dispatch)
     if pg:
         pg.barrier()
     prof = moe.profile_read()
@@ -332,8 +334,8 @@ def run_ours(args, cfg):
                                   dev)
         for _ in range(2):
             moe.forward(inp["hidden"], inp["idx"], inp["w"], inp["wgu"], inp["wd"],
-                        num_chunks=1, ep_groups=cfg.G, workspace=ws1)
-        ms1, _ = time_steps(moe, inp, cfg, 1, ws1, args.steps, stream)
+                        num_chunks=1, ep_groups=cfg.G, workspace=ws1, dispatch=args.dispatch)
+        ms1, _ = time_steps(moe, inp, cfg, 1, ws1, args.steps, stream, args.dispatch)
         ms_n1 = ms1 / args.steps
         del ws1
 
@@ -379,7 +381,7 @@ def run_ours(args, cfg):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; random-init expert weights of the layer's shape)",
-        "config": config_block(cfg, chunks),
+        "config": config_block(cfg, chunks, args.dispatch),
         "roofline": roofline,
         "grouped_gemm_tflops": gemm_tflops,
         "grouped_gemm_frac_of_peak": gemm_tflops / peak_tc,
@@ -423,7 +425,7 @@ def run_e2e(moe, inp, cfg, chunks, ws, args, stream, dev, pg, world):
         idd.copy_(i_pin, non_blocking=True)
         wdv.copy_(w_pin, non_blocking=True)
         moe.forward(hd, idd, wdv, inp["wgu"], inp["wd"], num_chunks=chunks, ep_groups=cfg.G,
-                    out=out, workspace=ws, stream=stream)
+                    out=out, workspace=ws, stream=stream, dispatch=args.dispatch)
         o_pin.copy_(out, non_blocking=True)
 
     step()
@@ -451,6 +453,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", choices=sorted(CONFIGS), default=DEFAULT_CONFIG)
     ap.add_argument("--chunks", type=int, default=DEFAULT_CHUNKS)
+    ap.add_argument("--dispatch", choices=["separate", "fused"], default="separate",
+                    help="separate: permute kernel first; fused: the gate/up GEMM gathers its "
+                         "rows from hidden")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

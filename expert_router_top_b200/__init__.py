@@ -72,6 +72,9 @@ def load():
     L.moe_metadata.restype = st
     L.moe_forward.argtypes = [ctypes.POINTER(Shape), p, p, p, p, p, p, p, sz, p]
     L.moe_forward.restype = st
+    L.moe_forward_ex.argtypes = [ctypes.POINTER(Shape), p, p, p, p, p, p, p, sz, ctypes.c_uint32,
+                                 p]
+    L.moe_forward_ex.restype = st
     L.moe_check_device_status.argtypes = [p, sz, p]
     L.moe_check_device_status.restype = st
     L.moe_permute.argtypes = [p, p, i64, i32, i32, p, p]
@@ -176,13 +179,21 @@ def metadata(top_k_index: torch.Tensor, E: int, ep_groups: int = 1, num_chunks: 
     return out
 
 
+FWD_FUSED_DISPATCH = 1
+
+
 def forward(hidden, top_k_index, top_k_weights, W_gate_up, W_down, num_chunks: int = 1,
-            ep_groups: int = 1, out=None, workspace=None, stream=None):
+            ep_groups: int = 1, out=None, workspace=None, stream=None,
+            dispatch: str = "separate"):
     """One MoE layer forward, chunked as Chunk MoE.  Returns out [T,H] bf16.
 
     hidden [T,H] bf16, top_k_index [T,k] int32, top_k_weights [T,k] fp32,
     W_gate_up [E,2I,H] bf16 (gate rows then up rows), W_down [E,H,I] bf16; all on the
-    same CUDA device.  Asynchronous after its single metadata copy."""
+    same CUDA device.  Asynchronous after its single metadata copy.
+    dispatch="separate": a permute kernel writes the permuted rows first; "fused": the
+    gate/up GEMM gathers its rows from `hidden`.  Both give identical bits."""
+    if dispatch not in ("fused", "separate"):
+        raise ValueError(f"dispatch must be 'fused' or 'separate', not {dispatch!r}")
     _need(hidden, torch.bfloat16, "hidden")
     _need(top_k_index, torch.int32, "top_k_index")
     _need(top_k_weights, torch.float32, "top_k_weights")
@@ -200,10 +211,11 @@ def forward(hidden, top_k_index, top_k_weights, W_gate_up, W_down, num_chunks: i
         out = torch.empty((T, H), dtype=torch.bfloat16, device=hidden.device)
     if workspace is None:
         workspace = alloc_workspace(load().moe_workspace_bytes(ctypes.byref(s)), hidden.device)
-    _check(load().moe_forward(ctypes.byref(s), _ptr(hidden), _ptr(top_k_index),
-                              _ptr(top_k_weights), _ptr(W_gate_up), _ptr(W_down), _ptr(out),
-                              _ptr(workspace), workspace.numel(), _stream(stream)),
-           "moe_forward")
+    flags = FWD_FUSED_DISPATCH if dispatch == "fused" else 0
+    _check(load().moe_forward_ex(ctypes.byref(s), _ptr(hidden), _ptr(top_k_index),
+                                 _ptr(top_k_weights), _ptr(W_gate_up), _ptr(W_down), _ptr(out),
+                                 _ptr(workspace), workspace.numel(), flags, _stream(stream)),
+           "moe_forward_ex")
     return out
 
 

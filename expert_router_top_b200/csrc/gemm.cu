@@ -90,6 +90,7 @@ struct KParams {
   int32_t b_rows;    // B rows per expert
   int32_t up_off;    // row offset of W_up inside one expert's W_gate_up (= I)
   int32_t total_tiles;
+  const int32_t* gather;  // gathered A: token row of each permuted row (nullptr: plain A)
 };
 
 template <int kStages>
@@ -191,11 +192,12 @@ __device__ __forceinline__ void store_block(const uint32_t (&packed)[16], uint8_
 // stream.  In a pair, the even CTA ("leader") owns the full-stage barriers and the MMA
 // issue; both CTAs load their own halves, run their own epilogue on their own TMEM rows,
 // and report back to the leader.
-template <bool kSwiGLU, bool kPair>
+template <bool kSwiGLU, bool kPair, bool kGather>
 __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensorMap* tmB,
                                           const KParams& p) {
   using G = Geo<kPair>;
   constexpr int STAGES = G::kStages;
+  static_assert(!(kGather && kPair), "gathered A rows are implemented for single CTAs");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -269,7 +271,57 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   const uint32_t tmem_base = ctl->tmem_base;
   volatile int* abort = &ctl->abort;
 
-  if (warp == 0) {
+  if (warp == 0 && kGather) {
+    // ---------------- TMA producer, gathered A (whole warp) ----------------
+    // Lane l gathers rows 4l..4l+3 of the tile straight from the source rows (tile::gather4,
+    // a box one row high); lane 0 also waits for the stage, arms it and loads the weights.
+    const uint64_t pol_w = l2_policy_evict_last();
+    const uint64_t pol_a = l2_policy_evict_normal();
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t armed = 0, armed_parity = 0;
+    bool ok = true;
+    for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
+      const Tile t = decode_tile<G::kTileM>(L, tile_start, off, E, p.n_tiles);
+      const int32_t row0 = off[t.e] + t.m * G::kTileM;
+      const int32_t last = off[t.e + 1] - 1;  // rows past the expert reuse its last row
+      int32_t src[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) src[i] = p.gather[min(row0 + 4 * lane + i, last)];
+      const int32_t brow = t.e * p.b_rows + t.n * (BN / 2);
+      for (int32_t kb = 0; kb < p.num_kb; ++kb) {
+        int go = 1;
+        if (lane == 0) {
+          if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort, p.status)) go = 0;
+          if (go) {
+            mbar_arrive_expect_tx(&ctl->full[stage], G::kTxBytes);
+            uint8_t* b_dst = sB + stage * G::kBBytes;
+            tma_load_2d(b_dst, tmB, &ctl->full[stage], kb * BK, brow, pol_w);
+            if (kSwiGLU)
+              tma_load_2d(b_dst + G::kBBytes / 2, tmB, &ctl->full[stage], kb * BK,
+                          brow + p.up_off, pol_w);
+          }
+        }
+        go = __shfl_sync(0xffffffffu, go, 0);  // also orders the gathers after the wait
+        if (!go) {
+          ok = false;
+          break;
+        }
+        tma_gather4(sA + stage * G::kABytes + lane * 4 * (BK * 2), tmA, &ctl->full[stage],
+                    kb * BK, src[0], src[1], src[2], src[3], pol_a);
+        armed |= 1u << stage;
+        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      for (int s = 0; s < STAGES; ++s)
+        if (armed & (1u << s)) mbar_drain(&ctl->full[s], (armed_parity >> s) & 1u, 100000000ull);
+    }
+  } else if (warp == 0) {
     // ---------------- TMA producer (both CTAs) ----------------
     if (lane == 0) {
 #if MOE_GEMM_B_POLICY == 1
@@ -449,11 +501,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   }
 }
 
-template <bool kSwiGLU>
+template <bool kSwiGLU, bool kGather>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, const KParams p) {
-  gemm_body<kSwiGLU, false>(&tmA, &tmB, p);
+  gemm_body<kSwiGLU, false, kGather>(&tmA, &tmB, p);
 }
 
 // Launched with a cluster of 2 CTAs (cudaLaunchAttributeClusterDimension).
@@ -461,7 +513,7 @@ template <bool kSwiGLU>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmB, const KParams p) {
-  gemm_body<kSwiGLU, true>(&tmA, &tmB, p);
+  gemm_body<kSwiGLU, true, false>(&tmA, &tmB, p);
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -502,6 +554,8 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int32_t cols, int3
 
 }  // namespace
 
+bool gemm_supports_gather() { return MOE_GEMM_2SM == 0; }
+
 int64_t gemm_total_tiles(const int32_t* counts_host, int32_t E, int32_t out_cols, bool swiglu) {
   const int32_t bn = swiglu ? BN / 2 : BN;
   const int32_t tm = Geo<MOE_GEMM_2SM != 0>::kTileM;
@@ -522,7 +576,14 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
   }
   CUtensorMap mA, mB;
   const int32_t bn = swiglu ? BN / 2 : BN;
-  if (!make_map(&mA, a.A, a.rows, a.K, kRowsPerCta) ||
+  const bool gather = a.gather != nullptr;
+  if (gather && (kPair || !swiglu)) {
+    *err_detail = 1;
+    return cudaErrorInvalidValue;
+  }
+  const bool map_a_ok = gather ? make_map(&mA, a.gather_src, a.gather_src_rows, a.K, 1)
+                               : make_map(&mA, a.A, a.rows, a.K, kRowsPerCta);
+  if (!map_a_ok ||
       !make_map(&mB, a.B, (int64_t)a.E * a.b_rows, a.K,
                 kPair ? BN / 2 : (swiglu ? BN / 2 : BN))) {
     *err_detail = 2;
@@ -539,6 +600,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
   p.b_rows = a.b_rows;
   p.up_off = swiglu ? a.out_cols : 0;
   p.total_tiles = (int32_t)a.total_tiles;
+  p.gather = a.gather;
   constexpr size_t smem = smem_bytes<kPair>();
   cudaError_t e;
   if (kPair) {
@@ -573,7 +635,8 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
     e = cudaLaunchKernelEx(&cfg, k, mA, mB, p);
     if (e != cudaSuccess) return e;
   } else {
-    auto k = swiglu ? grouped_gemm_kernel<true> : grouped_gemm_kernel<false>;
+    auto k = gather ? grouped_gemm_kernel<true, true>
+                    : (swiglu ? grouped_gemm_kernel<true, false> : grouped_gemm_kernel<false, false>);
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int streams = (int)(a.total_tiles < num_sms ? a.total_tiles : num_sms);

@@ -60,7 +60,15 @@ struct GemmArgs {
   int32_t b_rows;         // 2I for gate/up, H for down
   int64_t total_tiles;    // sum over experts of ceil(rows_e / 128) * n_tiles
   uint32_t* status;
+  // Gathered A (gate/up only): A row r is row gather[r] of gather_src [gather_src_rows][K]
+  // instead of row r of A.  nullptr = plain A.
+  const int32_t* gather = nullptr;
+  const void* gather_src = nullptr;
+  int64_t gather_src_rows = 0;
 };
+
+// True when the build's grouped GEMM supports a gathered A operand.
+bool gemm_supports_gather();
 
 // Number of 128-row x N-column output tiles for the given host counts.
 int64_t gemm_total_tiles(const int32_t* counts_host, int32_t E, int32_t out_cols, bool swiglu);

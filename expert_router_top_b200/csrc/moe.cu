@@ -126,7 +126,8 @@ struct DeviceCtx {
   bool ready = false;
   int num_sms = 0;
   cudaStream_t side = nullptr;
-  cudaEvent_t ev_start = nullptr, ev_join = nullptr, ev_perm[2] = {}, ev_gemm[2] = {};
+  cudaEvent_t ev_start = nullptr, ev_join = nullptr, ev_perm[2] = {}, ev_gemm[2] = {},
+              ev_unperm[2] = {};
   int32_t* host_stage = nullptr;
   size_t host_stage_bytes = 0;
 };
@@ -150,7 +151,9 @@ moe_status_t get_ctx(DeviceCtx** out) {
         cudaEventCreateWithFlags(&c.ev_perm[0], fl) != cudaSuccess ||
         cudaEventCreateWithFlags(&c.ev_perm[1], fl) != cudaSuccess ||
         cudaEventCreateWithFlags(&c.ev_gemm[0], fl) != cudaSuccess ||
-        cudaEventCreateWithFlags(&c.ev_gemm[1], fl) != cudaSuccess)
+        cudaEventCreateWithFlags(&c.ev_gemm[1], fl) != cudaSuccess ||
+        cudaEventCreateWithFlags(&c.ev_unperm[0], fl) != cudaSuccess ||
+        cudaEventCreateWithFlags(&c.ev_unperm[1], fl) != cudaSuccess)
       return MOE_ERR_CUDA;
     c.ready = true;
   }
@@ -274,8 +277,13 @@ int64_t active_experts(const int32_t* counts, int32_t E) {
 moe_status_t gemm_call(const void* A, int64_t rows, const void* B, void* out,
                        const int32_t* offsets_dev, const int32_t* counts_host, int32_t E,
                        int32_t K, int32_t out_cols, int32_t b_rows, bool swiglu,
-                       uint32_t* status, int num_sms, cudaStream_t s) {
+                       uint32_t* status, int num_sms, cudaStream_t s,
+                       const int32_t* gather = nullptr, const void* gather_src = nullptr,
+                       int64_t gather_src_rows = 0) {
   GemmArgs g;
+  g.gather = gather;
+  g.gather_src = gather_src;
+  g.gather_src_rows = gather_src_rows;
   g.A = A;
   g.rows = rows;
   g.B = B;
@@ -381,11 +389,21 @@ moe_status_t moe_metadata(const int32_t* top_k_index, int64_t T, int32_t k, int3
 moe_status_t moe_forward(const moe_shape_t* shape, const void* hidden, const int32_t* top_k_index,
                          const float* top_k_weights, const void* W_gate_up, const void* W_down,
                          void* out, void* workspace, size_t ws_bytes, void* stream) {
+  return moe_forward_ex(shape, hidden, top_k_index, top_k_weights, W_gate_up, W_down, out,
+                        workspace, ws_bytes, 0u, stream);
+}
+
+moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
+                            const int32_t* top_k_index, const float* top_k_weights,
+                            const void* W_gate_up, const void* W_down, void* out,
+                            void* workspace, size_t ws_bytes, uint32_t flags, void* stream) {
+  if (flags & ~MOE_FWD_FUSED_DISPATCH) return MOE_ERR_ARG;
   moe_status_t st = check_shape(shape);
   if (st != MOE_OK) return st;
   const int64_t T = shape->T;
   const int32_t H = shape->H, I = shape->I, E = shape->E, k = shape->k;
   if (T == 0) return MOE_OK;
+  const bool fused = (flags & MOE_FWD_FUSED_DISPATCH) && gemm_supports_gather();
   if (!hidden || !top_k_index || !top_k_weights || !W_gate_up || !W_down || !out || !workspace)
     return MOE_ERR_ARG;
   if (!aligned(hidden, 16) || !aligned(out, 16) || !aligned(W_gate_up, 16) ||
@@ -430,12 +448,20 @@ moe_status_t moe_forward(const moe_shape_t* shape, const void* hidden, const int
     return MOE_OK;
   };
   auto experts = [&](int c) -> moe_status_t {
-    if (cudaStreamWaitEvent(sg, ctx->ev_perm[c & 1], 0) != cudaSuccess) return MOE_ERR_CUDA;
+    // separate dispatch: wait for P(c); fused: wait until U(c-2) has read buffer c % 2
+    if (!fused) {
+      if (cudaStreamWaitEvent(sg, ctx->ev_perm[c & 1], 0) != cudaSuccess) return MOE_ERR_CUDA;
+    } else if (c >= 2) {
+      if (cudaStreamWaitEvent(sg, ctx->ev_unperm[c & 1], 0) != cudaSuccess) return MOE_ERR_CUDA;
+    }
     const int64_t rows = len(c) * k;
     const int32_t* cnt = counts.data() + (size_t)c * E;
     const int32_t* offs = reinterpret_cast<const int32_t*>(ws + L.offsets) + (size_t)c * (E + 1);
-    moe_status_t s2 = gemm_call(xy(c), rows, W_gate_up, act(c), offs, cnt, E, H, I, 2 * I, true,
-                                dev_status, ctx->num_sms, sg);
+    moe_status_t s2 =
+        fused ? gemm_call(nullptr, rows, W_gate_up, act(c), offs, cnt, E, H, I, 2 * I, true,
+                          dev_status, ctx->num_sms, sg, src + bounds[c] * k, hidden, T)
+              : gemm_call(xy(c), rows, W_gate_up, act(c), offs, cnt, E, H, I, 2 * I, true,
+                          dev_status, ctx->num_sms, sg);
     if (s2 != MOE_OK) return s2;
     s2 = gemm_call(act(c), rows, W_down, xy(c), offs, cnt, E, I, H, H, false, dev_status,
                    ctx->num_sms, sg);
@@ -449,6 +475,7 @@ moe_status_t moe_forward(const moe_shape_t* shape, const void* hidden, const int
     if (launch_unpermute(xy(c), dst + bounds[c] * k, top_k_weights + bounds[c] * k, len(c), H, k,
                          outp + bounds[c] * H, sm) != cudaSuccess)
       return MOE_ERR_CUDA;
+    if (fused && cudaEventRecord(ctx->ev_unperm[c & 1], sm) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
   };
 
@@ -456,13 +483,22 @@ moe_status_t moe_forward(const moe_shape_t* shape, const void* hidden, const int
   if (cudaEventRecord(ctx->ev_start, sm) != cudaSuccess ||
       cudaStreamWaitEvent(sg, ctx->ev_start, 0) != cudaSuccess)
     return MOE_ERR_CUDA;
-  if (n_live > 0) {
+  if (n_live > 0 && !fused) {
+    // M: P(0) P(1) U(0) P(2) U(1) ...; G: E(0) E(1) E(2) ...
     if ((st = permute(0)) != MOE_OK || (st = experts(0)) != MOE_OK) return st;
     for (int c = 0; c < n_live; ++c) {
       if (c + 1 < n_live) {
         if ((st = permute(c + 1)) != MOE_OK || (st = experts(c + 1)) != MOE_OK) return st;
       }
       if ((st = unpermute(c)) != MOE_OK) return st;
+    }
+  } else if (n_live > 0) {
+    // G: E(0) E(1) E(2) ... (E(c+2) after U(c) freed buffer c % 2); M: U(0) U(1) ...
+    if ((st = experts(0)) != MOE_OK) return st;
+    if (n_live > 1 && (st = experts(1)) != MOE_OK) return st;
+    for (int c = 0; c < n_live; ++c) {
+      if ((st = unpermute(c)) != MOE_OK) return st;
+      if (c + 2 < n_live && (st = experts(c + 2)) != MOE_OK) return st;
     }
   }
   if (cudaEventRecord(ctx->ev_join, sg) != cudaSuccess ||

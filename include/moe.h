@@ -201,6 +201,25 @@ MOE_API moe_status_t moe_forward(const moe_shape_t* shape, const void* hidden, c
                          const float* top_k_weights, const void* W_gate_up, const void* W_down,
                          void* out, void* workspace, size_t ws_bytes, void* stream);
 
+/* Flags of moe_forward_ex. */
+#define MOE_FWD_FUSED_DISPATCH 1u /* gather the gate/up GEMM's rows from hidden; no permute */
+
+/* moe_forward with a choice of dispatch.  flags = 0 (what moe_forward does): the permute
+ * kernel writes the permuted rows (the article's separate permute step) and the pipeline
+ * overlaps the permute of chunk c+1 and the unpermute of chunk c-1 with the expert GEMMs
+ * of chunk c.  flags = MOE_FWD_FUSED_DISPATCH: the gate/up GEMM loads each permuted row
+ * straight from `hidden` (TMA row gathers through the permutation's inverse map), so no
+ * permuted copy of the input is written or read, and the pipeline overlaps the unpermute
+ * of chunk c with the expert GEMMs of chunk c+1; on B200 the row gathers currently make
+ * the gate/up GEMM slower than the permute they replace.  Both give bit-identical
+ * outputs; arguments, workspace and errors are as moe_forward (unknown flag bits:
+ * MOE_ERR_ARG). */
+MOE_API moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
+                                    const int32_t* top_k_index, const float* top_k_weights,
+                                    const void* W_gate_up, const void* W_down, void* out,
+                                    void* workspace, size_t ws_bytes, uint32_t flags,
+                                    void* stream);
+
 /* Synchronizes `stream` and returns MOE_ERR_TIMEOUT if a kernel of an earlier call that
  * used this workspace gave up a bounded wait, MOE_ERR_INDEX if its last metadata pass
  * saw a bad index, else MOE_OK (or MOE_ERR_CUDA). */

@@ -121,6 +121,14 @@ def test_forward_argument_checks_run_on_host():
     assert _fwd(moe.shape(0, 64, 64, 8, 2)) == 0                      # T = 0: no work
 
 
+def test_forward_ex_rejects_unknown_flags():
+    L = moe.load()
+    v = ctypes.c_void_p
+    good = moe.shape(64, 64, 64, 8, 2, 2, 4)
+    assert L.moe_forward_ex(ctypes.byref(good), v(FAKE), v(FAKE), v(FAKE), v(FAKE), v(FAKE),
+                            v(FAKE), v(FAKE), 1 << 40, 2, None) == 1
+
+
 def test_stage_argument_checks_run_on_host():
     L = moe.load()
     v = ctypes.c_void_p

@@ -14,9 +14,9 @@ from parity import assert_layer_close, to_f64
 pytestmark = pytest.mark.gpu
 
 
-def _run(moe, inp, N, G=1):
+def _run(moe, inp, N, G=1, dispatch="separate"):
     out = moe.forward(inp["hidden"], inp["idx"], inp["w"], inp["wgu"], inp["wd"], num_chunks=N,
-                      ep_groups=G)
+                      ep_groups=G, dispatch=dispatch)
     torch.cuda.synchronize()
     return out
 
@@ -26,21 +26,32 @@ def _oracle(inp_cpu, tokens=None):
                           bits(inp_cpu["wgu"]), bits(inp_cpu["wd"]), tokens=tokens)
 
 
+@pytest.mark.parametrize("dispatch", ["fused", "separate"])
 @pytest.mark.parametrize("name", ["tiny", "edge", "edge_pair01", "edge_varlen", "edge_varlen7"])
-def test_forward_small_configs_all_tokens(moe, name):
+def test_forward_small_configs_all_tokens(moe, name, dispatch):
     cfg = CONFIGS[name]
     cpu = layer_inputs(cfg)
     gpu = {k: v.cuda() for k, v in cpu.items()}
     ref = _oracle(cpu)
     outs = []
     for N in cfg.chunks:
-        out = _run(moe, gpu, N, cfg.G)
-        assert_layer_close(out, ref, f"{name} N={N}")
+        out = _run(moe, gpu, N, cfg.G, dispatch)
+        assert_layer_close(out, ref, f"{name} N={N} {dispatch}")
         outs.append(out)
-    base = _run(moe, gpu, 1, cfg.G)
-    assert_layer_close(base, ref, f"{name} N=1")
+    base = _run(moe, gpu, 1, cfg.G, dispatch)
+    assert_layer_close(base, ref, f"{name} N=1 {dispatch}")
     for N, o in zip(cfg.chunks, outs):
-        assert torch.equal(o, base), f"{name}: N={N} output differs from N=1"
+        assert torch.equal(o, base), f"{name}: N={N} output differs from N=1 ({dispatch})"
+
+
+@pytest.mark.parametrize("name", ["tiny", "edge", "edge_pair01", "edge_varlen"])
+def test_fused_and_separate_dispatch_are_bit_identical(moe, name):
+    """Gathering the gate/up GEMM's rows from `hidden` reads the same bf16 values as the
+    permute kernel writes, so the two dispatch modes must agree bit for bit."""
+    cfg = CONFIGS[name]
+    gpu = {k: v.cuda() for k, v in layer_inputs(cfg).items()}
+    for N in (1,) + tuple(cfg.chunks):
+        assert torch.equal(_run(moe, gpu, N, cfg.G, "fused"), _run(moe, gpu, N, cfg.G, "separate"))
 
 
 def test_forward_chunk_invariance_many_N(moe):
@@ -131,5 +142,7 @@ def test_forward_full_size_sampled(moe, name, n_tok):
             base = out
         else:
             assert torch.equal(out, base), f"{name}: N={N} differs from N={cfg.chunks[0]}"
+    # the fused-dispatch path gives the same bits
+    assert torch.equal(_run(moe, gpu, cfg.chunks[-1], cfg.G, "fused"), base)
     # properties at full size: finite everywhere
     assert bool(torch.isfinite(base.float()).all())
