@@ -75,6 +75,10 @@ def load():
     L.moe_forward_ex.argtypes = [ctypes.POINTER(Shape), p, p, p, p, p, p, p, sz, ctypes.c_uint32,
                                  p]
     L.moe_forward_ex.restype = st
+    L.moe_workspace_bytes_host.argtypes = [ctypes.POINTER(Shape)]
+    L.moe_workspace_bytes_host.restype = sz
+    L.moe_forward_host.argtypes = [ctypes.POINTER(Shape), p, p, p, p, p, p, p, sz, p]
+    L.moe_forward_host.restype = st
     L.moe_check_device_status.argtypes = [p, sz, p]
     L.moe_check_device_status.restype = st
     L.moe_permute.argtypes = [p, p, i64, i32, i32, p, p]
@@ -216,6 +220,39 @@ def forward(hidden, top_k_index, top_k_weights, W_gate_up, W_down, num_chunks: i
                                  _ptr(top_k_weights), _ptr(W_gate_up), _ptr(W_down), _ptr(out),
                                  _ptr(workspace), workspace.numel(), flags, _stream(stream)),
            "moe_forward_ex")
+    return out
+
+
+def workspace_bytes_host(T, H, I, E, k, ep_groups=1, num_chunks=1) -> int:
+    s = shape(T, H, I, E, k, ep_groups, num_chunks)
+    return int(load().moe_workspace_bytes_host(ctypes.byref(s)))
+
+
+def forward_host(hidden, top_k_index, top_k_weights, W_gate_up, W_down, num_chunks: int = 1,
+                 ep_groups: int = 1, out=None, workspace=None, stream=None):
+    """moe_forward_host: activations in host memory (CPU tensors; pinned ones let the
+    per-chunk copies overlap the kernels), weights on the device.  Returns out [T,H] bf16
+    on the host, complete when the call returns."""
+    _need(hidden, torch.bfloat16, "hidden", device=False)
+    _need(top_k_index, torch.int32, "top_k_index", device=False)
+    _need(top_k_weights, torch.float32, "top_k_weights", device=False)
+    _need(W_gate_up, torch.bfloat16, "W_gate_up")
+    _need(W_down, torch.bfloat16, "W_down")
+    if hidden.is_cuda or top_k_index.is_cuda or top_k_weights.is_cuda:
+        raise ValueError("forward_host takes host (CPU) activations")
+    T, H = hidden.shape
+    E, twoI, _ = W_gate_up.shape
+    k = top_k_index.shape[1]
+    s = shape(T, H, twoI // 2, E, k, ep_groups, num_chunks)
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, pin_memory=hidden.is_pinned())
+    if workspace is None:
+        workspace = alloc_workspace(load().moe_workspace_bytes_host(ctypes.byref(s)),
+                                    W_gate_up.device)
+    _check(load().moe_forward_host(ctypes.byref(s), _ptr(hidden), _ptr(top_k_index),
+                                   _ptr(top_k_weights), _ptr(W_gate_up), _ptr(W_down), _ptr(out),
+                                   _ptr(workspace), workspace.numel(), _stream(stream)),
+           "moe_forward_host")
     return out
 
 

@@ -100,6 +100,34 @@ Layout make_layout(const Dims& d, int32_t H, int32_t I, bool with_buffers, bool 
   return L;
 }
 
+// Extra device staging of moe_forward_host, placed after the moe_forward layout.
+struct HostStaging {
+  size_t idx, w, in[2], out[2], total;
+};
+
+HostStaging make_host_staging(const Dims& d, int32_t H, size_t base) {
+  HostStaging h{};
+  size_t o = base;
+  h.idx = o;
+  o += al(sizeof(int32_t) * (size_t)(d.T * d.k));
+  h.w = o;
+  o += al(sizeof(float) * (size_t)(d.T * d.k));
+  const int nbuf = d.n >= 2 ? 2 : 1;
+  for (int b = 0; b < 2; ++b) {
+    if (b < nbuf) {
+      h.in[b] = o;
+      o += al(sizeof(uint16_t) * (size_t)d.t_chunk * H);
+      h.out[b] = o;
+      o += al(sizeof(uint16_t) * (size_t)d.t_chunk * H);
+    } else {
+      h.in[b] = h.in[0];
+      h.out[b] = h.out[0];
+    }
+  }
+  h.total = o;
+  return h;
+}
+
 moe_status_t check_routing_dims(int64_t T, int32_t k, int32_t E, int32_t ep_groups,
                                 int32_t num_chunks) {
   if (T < 0 || k <= 0 || E <= 0 || ep_groups < 0 || num_chunks < 0) return MOE_ERR_ARG;
@@ -128,6 +156,10 @@ struct DeviceCtx {
   cudaStream_t side = nullptr;
   cudaEvent_t ev_start = nullptr, ev_join = nullptr, ev_perm[2] = {}, ev_gemm[2] = {},
               ev_unperm[2] = {};
+  // host-buffer forward: copy-in / copy-out streams and their events
+  cudaStream_t copy_in = nullptr, copy_out = nullptr;
+  cudaEvent_t ev_in[2] = {}, ev_in_free[2] = {}, ev_out[2] = {}, ev_out_free[2] = {},
+              ev_copy_join = nullptr;
   int32_t* host_stage = nullptr;
   size_t host_stage_bytes = 0;
 };
@@ -155,6 +187,16 @@ moe_status_t get_ctx(DeviceCtx** out) {
         cudaEventCreateWithFlags(&c.ev_unperm[0], fl) != cudaSuccess ||
         cudaEventCreateWithFlags(&c.ev_unperm[1], fl) != cudaSuccess)
       return MOE_ERR_CUDA;
+    if (cudaStreamCreateWithFlags(&c.copy_in, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&c.copy_out, cudaStreamNonBlocking) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    for (int b = 0; b < 2; ++b)
+      if (cudaEventCreateWithFlags(&c.ev_in[b], fl) != cudaSuccess ||
+          cudaEventCreateWithFlags(&c.ev_in_free[b], fl) != cudaSuccess ||
+          cudaEventCreateWithFlags(&c.ev_out[b], fl) != cudaSuccess ||
+          cudaEventCreateWithFlags(&c.ev_out_free[b], fl) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (cudaEventCreateWithFlags(&c.ev_copy_join, fl) != cudaSuccess) return MOE_ERR_CUDA;
     c.ready = true;
   }
   *out = &c;
@@ -503,6 +545,151 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
   }
   if (cudaEventRecord(ctx->ev_join, sg) != cudaSuccess ||
       cudaStreamWaitEvent(sm, ctx->ev_join, 0) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+size_t moe_workspace_bytes_host(const moe_shape_t* s) {
+  if (check_shape(s) != MOE_OK) return 0;
+  const Dims d = make_dims(s->T, s->k, s->E, s->ep_groups, s->num_chunks);
+  const Layout L = make_layout(d, s->H, s->I, true, true, true);
+  return make_host_staging(d, s->H, L.total).total;
+}
+
+moe_status_t moe_forward_host(const moe_shape_t* shape, const void* hidden_host,
+                              const int32_t* top_k_index_host, const float* top_k_weights_host,
+                              const void* W_gate_up, const void* W_down, void* out_host,
+                              void* workspace, size_t ws_bytes, void* stream) {
+  moe_status_t st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  const int64_t T = shape->T;
+  const int32_t H = shape->H, I = shape->I, E = shape->E, k = shape->k;
+  if (T == 0) return MOE_OK;
+  if (!hidden_host || !top_k_index_host || !top_k_weights_host || !W_gate_up || !W_down ||
+      !out_host || !workspace)
+    return MOE_ERR_ARG;
+  if (!aligned(W_gate_up, 16) || !aligned(W_down, 16) || !aligned(workspace, kAlign) ||
+      !aligned(top_k_index_host, 4) || !aligned(top_k_weights_host, 4) ||
+      !aligned(hidden_host, 2) || !aligned(out_host, 2))
+    return MOE_ERR_ALIGN;
+  const Dims d = make_dims(T, k, E, shape->ep_groups, shape->num_chunks);
+  const Layout L = make_layout(d, H, I, true, true, true);
+  const HostStaging hs = make_host_staging(d, H, L.total);
+  if (ws_bytes < hs.total) return MOE_ERR_WORKSPACE;
+  DeviceCtx* ctx = nullptr;
+  if ((st = get_ctx(&ctx)) != MOE_OK) return st;
+  cudaStream_t sm = static_cast<cudaStream_t>(stream);
+  cudaStream_t sg = ctx->side, ci = ctx->copy_in, co = ctx->copy_out;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* dst = reinterpret_cast<int32_t*>(ws + L.dst);
+  int32_t* src = reinterpret_cast<int32_t*>(ws + L.src);
+  uint32_t* dev_status = reinterpret_cast<uint32_t*>(ws + L.packed);
+  int32_t* idx_dev = reinterpret_cast<int32_t*>(ws + hs.idx);
+  float* w_dev = reinterpret_cast<float*>(ws + hs.w);
+  const size_t row_bytes = sizeof(uint16_t) * (size_t)H;
+  const uint8_t* hid_h = static_cast<const uint8_t*>(hidden_host);
+  uint8_t* out_h = static_cast<uint8_t*>(out_host);
+
+  // routing arrays first: the metadata of every chunk needs all of them
+  if (cudaMemcpyAsync(idx_dev, top_k_index_host, sizeof(int32_t) * (size_t)(T * k),
+                      cudaMemcpyHostToDevice, sm) != cudaSuccess ||
+      cudaMemcpyAsync(w_dev, top_k_weights_host, sizeof(float) * (size_t)(T * k),
+                      cudaMemcpyHostToDevice, sm) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  std::vector<int64_t> bounds((size_t)d.n + 1);
+  moe_chunk_bounds(T, shape->num_chunks, bounds.data());
+  int n_live = 0;
+  while (n_live < d.n && bounds[n_live + 1] > bounds[n_live]) ++n_live;
+  auto len = [&](int c) { return bounds[c + 1] - bounds[c]; };
+  // copy-in of chunk c into input buffer c % 2 (after P(c-2) has read it)
+  auto copy_in = [&](int c) -> moe_status_t {
+    if (c >= 2 && cudaStreamWaitEvent(ci, ctx->ev_in_free[c & 1], 0) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (cudaMemcpyAsync(ws + hs.in[c & 1], hid_h + bounds[c] * row_bytes, len(c) * row_bytes,
+                        cudaMemcpyHostToDevice, ci) != cudaSuccess ||
+        cudaEventRecord(ctx->ev_in[c & 1], ci) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  };
+  // the first two chunks' rows can travel while the metadata runs
+  if (cudaEventRecord(ctx->ev_start, sm) != cudaSuccess ||
+      cudaStreamWaitEvent(ci, ctx->ev_start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(co, ctx->ev_start, 0) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  for (int c = 0; c < n_live && c < 2; ++c)
+    if ((st = copy_in(c)) != MOE_OK) return st;
+
+  if ((st = run_metadata(d, idx_dev, ws, L, dst, src, sm)) != MOE_OK) return st;
+  if ((st = fetch_packed(ctx, ws, L, sm)) != MOE_OK) return st;
+  std::vector<int32_t> counts(ctx->host_stage + kStatusWords,
+                              ctx->host_stage + kStatusWords + (size_t)d.n * d.E);
+
+  auto xy = [&](int c) { return ws + L.xy[c % L.nbuf]; };
+  auto act = [&](int c) { return ws + L.act[c % L.nbuf]; };
+  auto permute = [&](int c) -> moe_status_t {
+    if (cudaStreamWaitEvent(sm, ctx->ev_in[c & 1], 0) != cudaSuccess) return MOE_ERR_CUDA;
+    {
+      ProfScope ps(MOE_KERNEL_PERMUTE, sm, len(c) * k, 0, 1);
+      if (launch_permute(ws + hs.in[c & 1], dst + bounds[c] * k, len(c), H, k, xy(c), sm) !=
+          cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
+    if (cudaEventRecord(ctx->ev_perm[c & 1], sm) != cudaSuccess ||
+        cudaEventRecord(ctx->ev_in_free[c & 1], sm) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return c + 2 < n_live ? copy_in(c + 2) : MOE_OK;
+  };
+  auto experts = [&](int c) -> moe_status_t {
+    if (cudaStreamWaitEvent(sg, ctx->ev_perm[c & 1], 0) != cudaSuccess) return MOE_ERR_CUDA;
+    const int64_t rows = len(c) * k;
+    const int32_t* cnt = counts.data() + (size_t)c * E;
+    const int32_t* offs = reinterpret_cast<const int32_t*>(ws + L.offsets) + (size_t)c * (E + 1);
+    moe_status_t s2 = gemm_call(xy(c), rows, W_gate_up, act(c), offs, cnt, E, H, I, 2 * I, true,
+                                dev_status, ctx->num_sms, sg);
+    if (s2 != MOE_OK) return s2;
+    s2 = gemm_call(act(c), rows, W_down, xy(c), offs, cnt, E, I, H, H, false, dev_status,
+                   ctx->num_sms, sg);
+    if (s2 != MOE_OK) return s2;
+    return cudaEventRecord(ctx->ev_gemm[c & 1], sg) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  };
+  auto unpermute = [&](int c) -> moe_status_t {
+    if (cudaStreamWaitEvent(sm, ctx->ev_gemm[c & 1], 0) != cudaSuccess) return MOE_ERR_CUDA;
+    if (c >= 2 && cudaStreamWaitEvent(sm, ctx->ev_out_free[c & 1], 0) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    {
+      ProfScope ps(MOE_KERNEL_UNPERMUTE, sm, len(c) * k, 0, 1);
+      if (launch_unpermute(xy(c), dst + bounds[c] * k, w_dev + bounds[c] * k, len(c), H, k,
+                           ws + hs.out[c & 1], sm) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
+    // copy-out of chunk c beside the next chunk's GEMMs
+    if (cudaEventRecord(ctx->ev_out[c & 1], sm) != cudaSuccess ||
+        cudaStreamWaitEvent(co, ctx->ev_out[c & 1], 0) != cudaSuccess ||
+        cudaMemcpyAsync(out_h + bounds[c] * row_bytes, ws + hs.out[c & 1], len(c) * row_bytes,
+                        cudaMemcpyDeviceToHost, co) != cudaSuccess ||
+        cudaEventRecord(ctx->ev_out_free[c & 1], co) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  };
+
+  if (cudaEventRecord(ctx->ev_start, sm) != cudaSuccess ||
+      cudaStreamWaitEvent(sg, ctx->ev_start, 0) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (n_live > 0) {
+    if ((st = permute(0)) != MOE_OK || (st = experts(0)) != MOE_OK) return st;
+    for (int c = 0; c < n_live; ++c) {
+      if (c + 1 < n_live) {
+        if ((st = permute(c + 1)) != MOE_OK || (st = experts(c + 1)) != MOE_OK) return st;
+      }
+      if ((st = unpermute(c)) != MOE_OK) return st;
+    }
+  }
+  // join every stream into `stream` and wait for out_host
+  if (cudaEventRecord(ctx->ev_join, sg) != cudaSuccess ||
+      cudaStreamWaitEvent(sm, ctx->ev_join, 0) != cudaSuccess ||
+      cudaEventRecord(ctx->ev_copy_join, co) != cudaSuccess ||
+      cudaStreamWaitEvent(sm, ctx->ev_copy_join, 0) != cudaSuccess ||
+      cudaStreamSynchronize(sm) != cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;
 }

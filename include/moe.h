@@ -220,6 +220,28 @@ MOE_API moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden
                                     void* workspace, size_t ws_bytes, uint32_t flags,
                                     void* stream);
 
+/* Device workspace, in bytes, that moe_forward_host needs: the moe_forward workspace plus
+ * device staging for the routing arrays (T*k int32 + T*k fp32) and min(N_eff, 2) input
+ * and output buffers of T_chunk rows of H bf16.  0 if the shape is invalid. */
+MOE_API size_t moe_workspace_bytes_host(const moe_shape_t* shape);
+
+/* moe_forward with the activations in host memory: hidden_host [T][H] bf16,
+ * top_k_index_host [T][k] int32, top_k_weights_host [T][k] fp32 and out_host [T][H] bf16
+ * are host pointers (pinned memory lets the copies overlap the kernels; pageable memory
+ * works but serializes them); the weights stay on the device.  The routing arrays go to
+ * the device first (the metadata needs all of them); then chunk c's input rows are copied
+ * in while the expert GEMMs of chunk c-1 run, and chunk c's output rows are copied out
+ * while the GEMMs of chunk c+1 run, on two library copy streams beside the pair pipeline
+ * ([ChunkMoE] "一张专业时序图": transfers hidden behind the neighbouring chunk's compute).
+ * The call returns when out_host is complete (it synchronizes `stream`).  Results are
+ * bit-identical to moe_forward.  workspace: dev, >= moe_workspace_bytes_host(shape).
+ * Errors: as moe_forward. */
+MOE_API moe_status_t moe_forward_host(const moe_shape_t* shape, const void* hidden_host,
+                                      const int32_t* top_k_index_host,
+                                      const float* top_k_weights_host, const void* W_gate_up,
+                                      const void* W_down, void* out_host, void* workspace,
+                                      size_t ws_bytes, void* stream);
+
 /* Synchronizes `stream` and returns MOE_ERR_TIMEOUT if a kernel of an earlier call that
  * used this workspace gave up a bounded wait, MOE_ERR_INDEX if its last metadata pass
  * saw a bad index, else MOE_OK (or MOE_ERR_CUDA). */

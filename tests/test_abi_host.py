@@ -121,6 +121,17 @@ def test_forward_argument_checks_run_on_host():
     assert _fwd(moe.shape(0, 64, 64, 8, 2)) == 0                      # T = 0: no work
 
 
+def test_host_workspace_adds_staging():
+    for name in ("qwen3", "tiny"):
+        cfg = CONFIGS[name]
+        for N in (1, 2, 4):
+            dev = moe.workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.G, N)
+            host = moe.workspace_bytes_host(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.G, N)
+            tc = -(-cfg.T // N)
+            staging = 8 * cfg.T * cfg.k + min(N, 2) * 2 * tc * cfg.H * 2
+            assert dev + staging <= host <= dev + staging + 8 * 256
+
+
 def test_forward_ex_rejects_unknown_flags():
     L = moe.load()
     v = ctypes.c_void_p

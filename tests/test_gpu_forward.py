@@ -54,6 +54,24 @@ def test_fused_and_separate_dispatch_are_bit_identical(moe, name):
         assert torch.equal(_run(moe, gpu, N, cfg.G, "fused"), _run(moe, gpu, N, cfg.G, "separate"))
 
 
+@pytest.mark.parametrize("pinned", [True, False])
+@pytest.mark.parametrize("name", ["tiny", "edge", "edge_varlen", "edge_varlen7"])
+def test_forward_host_buffers_match_device_forward(moe, name, pinned):
+    """moe_forward_host (activations in host memory, copies pipelined per chunk) gives the
+    same bits as moe_forward on device-resident inputs, for every chunking."""
+    cfg = CONFIGS[name]
+    cpu = layer_inputs(cfg)
+    gpu = {k: v.cuda() for k, v in cpu.items()}
+    h = cpu["hidden"].pin_memory() if pinned else cpu["hidden"]
+    i = cpu["idx"].pin_memory() if pinned else cpu["idx"]
+    w = cpu["w"].pin_memory() if pinned else cpu["w"]
+    for N in (1, 2, 3) + tuple(cfg.chunks):
+        ref = _run(moe, gpu, N, cfg.G)
+        got = moe.forward_host(h, i, w, gpu["wgu"], gpu["wd"], num_chunks=N, ep_groups=cfg.G)
+        assert not got.is_cuda
+        assert torch.equal(got, ref.cpu()), f"{name} N={N} pinned={pinned}"
+
+
 def test_forward_chunk_invariance_many_N(moe):
     cfg = CONFIGS["edge"]
     gpu = {k: v.cuda() for k, v in layer_inputs(cfg).items()}
