@@ -150,7 +150,7 @@ def algorithmic_units(cfg, counts, n_live):
     """Per-kernel algorithmic work of one step (bytes or flops), from the chunk counts."""
     H, I, k, T = cfg.H, cfg.I, cfg.k, cfg.T
     rows = int(counts.sum())
-    active = int((counts > 0).sum())
+    active = int((counts > 0).sum())  # (chunk, expert) pairs with rows: weights streamed
     return {
         # permute: read T rows once, write T*k rows, plus the k destination indices per token
         "permute_bytes": (T + rows) * H * 2 + rows * 4,
@@ -161,6 +161,9 @@ def algorithmic_units(cfg, counts, n_live):
         # weights of every active expert, re-read once per chunk (the method's N-fold stream)
         "gateup_weight_bytes": active * 2 * I * H * 2,
         "down_weight_bytes": active * H * I * 2,
+        # gate/up kernel, whole step: W_gate_up of each chunk's active experts (re-read per
+        # chunk), permuted rows read, Act written
+        "gateup_alg_bytes": active * 2 * I * H * 2 + rows * H * 2 + rows * I * 2,
     }
 
 
@@ -169,14 +172,15 @@ def gemm_src_hash():
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def traffic_per_launch():
+def traffic_per_launch(cfg_name, chunks):
     """DRAM bytes per gate/up launch from the committed ncu summary, if it was taken on
-    the current kernel source; else None."""
+    the current kernel source, this workload and this chunking; else None."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
     with open(TRAFFIC_FILE) as f:
         d = json.load(f)
-    if d.get("gemm_src_sha256_16") != gemm_src_hash():
+    if (d.get("gemm_src_sha256_16") != gemm_src_hash() or d.get("num_chunks") != chunks
+            or d.get("config") != cfg_name):
         return None
     return d.get("dram_bytes_per_launch_full_size")
 
@@ -350,14 +354,10 @@ def run_ours(args, cfg):
         kinds[kind] = dict(launches=p["launches"], ms=p["ms"],
                            ms_per_step=p["ms"] / args.steps if args.steps else 0.0)
     steps = args.steps
-    g = prof["gateup"]
-    gu_flops = units["gateup_flops"] * steps
-    gu_tflops = gu_flops / (g["ms"] / 1e3) / 1e12 if g["ms"] > 0 else 0.0
-    d = prof["down"]
+    g, d, pm, um = prof["gateup"], prof["down"], prof["permute"], prof["unpermute"]
+    gu_tflops = units["gateup_flops"] * steps / (g["ms"] / 1e3) / 1e12 if g["ms"] > 0 else 0.0
     dn_tflops = units["down_flops"] * steps / (d["ms"] / 1e3) / 1e12 if d["ms"] > 0 else 0.0
-    pm = prof["permute"]
     pm_gbs = units["permute_bytes"] * steps / (pm["ms"] / 1e3) / 1e9 if pm["ms"] > 0 else 0.0
-    um = prof["unpermute"]
     um_gbs = units["unpermute_bytes"] * steps / (um["ms"] / 1e3) / 1e9 if um["ms"] > 0 else 0.0
     gemm_tflops = (units["gateup_flops"] + units["down_flops"]) * steps / \
         ((g["ms"] + d["ms"]) / 1e3) / 1e12 if g["ms"] + d["ms"] > 0 else 0.0
@@ -365,14 +365,33 @@ def run_ours(args, cfg):
     kinds["down"]["tflops"] = dn_tflops
     kinds["permute"]["gbs"] = pm_gbs
     kinds["unpermute"]["gbs"] = um_gbs
+    # per gate/up launch: algorithmic flops and bytes (weights of the chunk's active experts,
+    # the permuted rows read, Act written), averaged over the step's launches
+    n_gu = max(1, g["launches"] // max(1, steps))
+    gu_flops_l = units["gateup_flops"] / n_gu
+    gu_bytes_l = units["gateup_alg_bytes"] / n_gu
+    t_l = g["ms"] / max(1, g["launches"]) / 1e3  # s per launch
+    peak_tc, peak_bw = peaks["bf16_tflops"], peaks["hbm_gbs"]
+    t_tensor = gu_flops_l / (peak_tc * 1e12)
+    t_mem = gu_bytes_l / (peak_bw * 1e9)
+    traffic = traffic_per_launch(cfg.name, chunks)
+    if t_mem > t_tensor:
+        roofline = {"bound": "hbm", "achieved": gu_bytes_l / t_l / 1e9 if t_l else 0.0,
+                    "peak": peak_bw, "unit": "GB/s"}
+    else:
+        roofline = {"bound": "tensor", "achieved": gu_flops_l / t_l / 1e12 if t_l else 0.0,
+                    "peak": peak_tc, "unit": "TFLOP/s"}
+    roofline["frac"] = roofline["achieved"] / roofline["peak"]
+    roofline.update({
+        "traffic": traffic,
+        "kernel": "grouped_gemm_kernel<gate/up + SwiGLU> (tcgen05)",
+        "peak_source": f"{peak_src}: MEASURED_PEAKS.json (bf16 burst, HBM copy)",
+        "per_launch": {"flops": gu_flops_l, "bytes": gu_bytes_l, "ms": t_l * 1e3,
+                       "roofline_ms": max(t_tensor, t_mem) * 1e3},
+        "frac_of_roofline_time": max(t_tensor, t_mem) / t_l if t_l else None,
+        "tensor_frac": gu_flops_l / t_l / 1e12 / peak_tc if t_l else None,
+        "hbm_frac": gu_bytes_l / t_l / 1e9 / peak_bw if t_l else None})
     peak_tc = peaks["bf16_tflops"]
-    traffic = traffic_per_launch()
-    roofline = {"bound": "tensor", "kernel": "gateup_swiglu grouped GEMM (tcgen05)",
-                "achieved": gu_tflops, "peak": peak_tc, "unit": "TFLOP/s",
-                "frac": gu_tflops / peak_tc if peak_tc else None,
-                "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)",
-                "frac_of_sustained": gu_tflops / peaks["bf16_tflops_sustained"],
-                "traffic": traffic}
 
     ws_per_n = {str(n): moe.workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.G, n)
                 for n in (1, 2, 4)}
@@ -391,6 +410,7 @@ def run_ours(args, cfg):
         "weight_bytes_streamed_per_step": weight_stream,
         "workspace_bytes": ws_per_n,
         "ms_per_step_num_chunks_1": ms_n1,
+        "send_splits": meta["send"].tolist() if cfg.G > 1 else None,
         "gpu_launches": int(prof["kernels"]),
         "e2e": e2e,
         "clocks": clk,
