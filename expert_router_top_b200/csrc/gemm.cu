@@ -51,6 +51,12 @@
 #ifndef MOE_GEMM_EPI_STAGE
 #define MOE_GEMM_EPI_STAGE 1  // 1: stage output blocks in shared memory for coalesced stores
 #endif
+#ifndef MOE_GEMM_DOWN_POLICY
+#define MOE_GEMM_DOWN_POLICY 2  // L2 policy of the down GEMM's weights (same codes as below)
+#endif
+#ifndef MOE_GEMM_BAND
+#define MOE_GEMM_BAND 16  // M tiles per raster band: an expert's A rows stay in L2 across N tiles
+#endif
 #ifndef MOE_GEMM_B_POLICY
 #define MOE_GEMM_B_POLICY 2  // L2 policy of weight loads: 0 normal, 1 evict_first, 2 evict_last
 #endif
@@ -91,6 +97,7 @@ struct KParams {
   int32_t up_off;    // row offset of W_up inside one expert's W_gate_up (= I)
   int32_t total_tiles;
   const int32_t* gather;  // gathered A: token row of each permuted row (nullptr: plain A)
+  int32_t reverse;        // 1: walk the tiles (hence the experts) in descending order
 };
 
 template <int kStages>
@@ -140,9 +147,13 @@ __device__ __forceinline__ Tile decode_tile(int32_t L, const int32_t* tile_start
   Tile t;
   t.e = lo;
 #if MOE_GEMM_ORDER == 0
-  t.n = local / mt;
-  t.m = local - t.n * mt;
-  (void)n_tiles;
+  // bands of up to MOE_GEMM_BAND M tiles; inside a band M is fastest, then N
+  const int32_t band_tiles = MOE_GEMM_BAND * n_tiles;
+  const int32_t b = local / band_tiles;
+  const int32_t inner = local - b * band_tiles;
+  const int32_t width = min(MOE_GEMM_BAND, mt - b * MOE_GEMM_BAND);
+  t.n = inner / width;
+  t.m = b * MOE_GEMM_BAND + (inner - t.n * width);
 #else
   t.m = local / n_tiles;
   t.n = local - t.m * n_tiles;
@@ -282,7 +293,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
     uint32_t armed = 0, armed_parity = 0;
     bool ok = true;
     for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
-      const Tile t = decode_tile<G::kTileM>(L, tile_start, off, E, p.n_tiles);
+      const Tile t = decode_tile<G::kTileM>(p.reverse ? p.total_tiles - 1 - L : L, tile_start,
+                                            off, E, p.n_tiles);
       const int32_t row0 = off[t.e] + t.m * G::kTileM;
       const int32_t last = off[t.e + 1] - 1;  // rows past the expert reuse its last row
       int32_t src[4];
@@ -324,20 +336,18 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   } else if (warp == 0) {
     // ---------------- TMA producer (both CTAs) ----------------
     if (lane == 0) {
-#if MOE_GEMM_B_POLICY == 1
-      const uint64_t pol_w = l2_policy_evict_first();
-#elif MOE_GEMM_B_POLICY == 2
-      const uint64_t pol_w = l2_policy_evict_last();
-#else
-      const uint64_t pol_w = l2_policy_evict_normal();
-#endif
+      const int pol_code = kSwiGLU ? MOE_GEMM_B_POLICY : MOE_GEMM_DOWN_POLICY;
+      const uint64_t pol_w = pol_code == 1   ? l2_policy_evict_first()
+                             : pol_code == 2 ? l2_policy_evict_last()
+                                             : l2_policy_evict_normal();
       const uint64_t pol_a = l2_policy_evict_normal();
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;  // per-stage bits, for the abort drain
       bool ok = true;
       for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
-        const Tile t = decode_tile<G::kTileM>(L, tile_start, off, E, p.n_tiles);
+        const Tile t = decode_tile<G::kTileM>(p.reverse ? p.total_tiles - 1 - L : L, tile_start,
+                                              off, E, p.n_tiles);
         const int32_t row0 = off[t.e] + t.m * G::kTileM + (int32_t)rank * kRowsPerCta;
         int32_t brow;
         if (kSwiGLU)  // pair: the even CTA stages the gate rows, the odd one the up rows
@@ -445,7 +455,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       const uint32_t tphase = (it >> 1) & 1;
       if (!mbar_wait(&ctl->tfull[buf], tphase, abort, p.status)) break;
       tc_fence_after();
-      const Tile t = decode_tile<G::kTileM>(L, tile_start, off, E, p.n_tiles);
+      const Tile t = decode_tile<G::kTileM>(p.reverse ? p.total_tiles - 1 - L : L, tile_start,
+                                            off, E, p.n_tiles);
       const int32_t first = t.m * G::kTileM + (int32_t)rank * kRowsPerCta;  // in the expert
       const int32_t rows_valid = off[t.e + 1] - off[t.e] - first;
       const bool row_ok = r < rows_valid;
@@ -601,6 +612,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
   p.up_off = swiglu ? a.out_cols : 0;
   p.total_tiles = (int32_t)a.total_tiles;
   p.gather = a.gather;
+  p.reverse = a.reverse ? 1 : 0;
   constexpr size_t smem = smem_bytes<kPair>();
   cudaError_t e;
   if (kPair) {

@@ -65,6 +65,7 @@ struct GemmArgs {
   const int32_t* gather = nullptr;
   const void* gather_src = nullptr;
   int64_t gather_src_rows = 0;
+  bool reverse = false;  // walk the tiles (and so the experts) in descending order
 };
 
 // True when the build's grouped GEMM supports a gathered A operand.

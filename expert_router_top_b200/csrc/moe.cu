@@ -316,13 +316,18 @@ int64_t active_experts(const int32_t* counts, int32_t E) {
   return a;
 }
 
+#ifndef MOE_ALTERNATE_ORDER
+#define MOE_ALTERNATE_ORDER 0  // 1: odd chunks walk the experts in descending order
+#endif
+
 moe_status_t gemm_call(const void* A, int64_t rows, const void* B, void* out,
                        const int32_t* offsets_dev, const int32_t* counts_host, int32_t E,
                        int32_t K, int32_t out_cols, int32_t b_rows, bool swiglu,
                        uint32_t* status, int num_sms, cudaStream_t s,
                        const int32_t* gather = nullptr, const void* gather_src = nullptr,
-                       int64_t gather_src_rows = 0) {
+                       int64_t gather_src_rows = 0, bool reverse = false) {
   GemmArgs g;
+  g.reverse = reverse;
   g.gather = gather;
   g.gather_src = gather_src;
   g.gather_src_rows = gather_src_rows;
@@ -480,6 +485,7 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
   auto xy = [&](int c) { return ws + L.xy[c % L.nbuf]; };
   auto act = [&](int c) { return ws + L.act[c % L.nbuf]; };
   auto len = [&](int c) { return bounds[c + 1] - bounds[c]; };
+  auto rev = [&](int c) { return MOE_ALTERNATE_ORDER && (c & 1); };
 
   auto permute = [&](int c) -> moe_status_t {
     ProfScope ps(MOE_KERNEL_PERMUTE, sm, len(c) * k, 0, 1);
@@ -501,12 +507,12 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
     const int32_t* offs = reinterpret_cast<const int32_t*>(ws + L.offsets) + (size_t)c * (E + 1);
     moe_status_t s2 =
         fused ? gemm_call(nullptr, rows, W_gate_up, act(c), offs, cnt, E, H, I, 2 * I, true,
-                          dev_status, ctx->num_sms, sg, src + bounds[c] * k, hidden, T)
+                          dev_status, ctx->num_sms, sg, src + bounds[c] * k, hidden, T, rev(c))
               : gemm_call(xy(c), rows, W_gate_up, act(c), offs, cnt, E, H, I, 2 * I, true,
-                          dev_status, ctx->num_sms, sg);
+                          dev_status, ctx->num_sms, sg, nullptr, nullptr, 0, rev(c));
     if (s2 != MOE_OK) return s2;
     s2 = gemm_call(act(c), rows, W_down, xy(c), offs, cnt, E, I, H, H, false, dev_status,
-                   ctx->num_sms, sg);
+                   ctx->num_sms, sg, nullptr, nullptr, 0, rev(c));
     if (s2 != MOE_OK) return s2;
     if (cudaEventRecord(ctx->ev_gemm[c & 1], sg) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
@@ -644,11 +650,12 @@ moe_status_t moe_forward_host(const moe_shape_t* shape, const void* hidden_host,
     const int64_t rows = len(c) * k;
     const int32_t* cnt = counts.data() + (size_t)c * E;
     const int32_t* offs = reinterpret_cast<const int32_t*>(ws + L.offsets) + (size_t)c * (E + 1);
+    const bool r = MOE_ALTERNATE_ORDER && (c & 1);
     moe_status_t s2 = gemm_call(xy(c), rows, W_gate_up, act(c), offs, cnt, E, H, I, 2 * I, true,
-                                dev_status, ctx->num_sms, sg);
+                                dev_status, ctx->num_sms, sg, nullptr, nullptr, 0, r);
     if (s2 != MOE_OK) return s2;
     s2 = gemm_call(act(c), rows, W_down, xy(c), offs, cnt, E, I, H, H, false, dev_status,
-                   ctx->num_sms, sg);
+                   ctx->num_sms, sg, nullptr, nullptr, 0, r);
     if (s2 != MOE_OK) return s2;
     return cudaEventRecord(ctx->ev_gemm[c & 1], sg) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   };

@@ -16,32 +16,42 @@ from . import build as _build
 _lib = None
 
 
+def use_library(path=None):
+    """Point the wrappers at another build of oracle.c (None: the default build).  The
+    tests use it to run the pins against deliberately broken copies of the oracle."""
+    global _lib
+    _lib = None if path is None else _bind(ctypes.CDLL(path))
+
+
 def lib():
     global _lib
     if _lib is None:
-        path = _build.build()
-        L = ctypes.CDLL(path)
-        i32, i64, p, d = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
-        L.oracle_effective_chunks.argtypes = [i32]
-        L.oracle_effective_chunks.restype = ctypes.c_int
-        L.oracle_chunk_bounds.argtypes = [i64, i32, p]
-        L.oracle_chunk_bounds.restype = None
-        L.oracle_metadata.argtypes = [p, i64, i32, i32, i32, i32, p, p, p, p, p, p]
-        L.oracle_metadata.restype = i64
-        L.oracle_forward.argtypes = [p, p, p, p, p, i64, i32, i32, i32, i32, p, i64, p, d]
-        L.oracle_forward.restype = i64
-        L.oracle_permute.argtypes = [p, p, i64, i32, i32, p]
-        L.oracle_permute.restype = None
-        L.oracle_gateup_rows.argtypes = [p, p, i64, p, i32, i32, p, d]
-        L.oracle_gateup_rows.restype = None
-        L.oracle_down_rows.argtypes = [p, p, i64, p, i32, i32, p, d]
-        L.oracle_down_rows.restype = None
-        L.oracle_unpermute.argtypes = [p, p, p, i64, i32, i32, p]
-        L.oracle_unpermute.restype = None
-        L.oracle_max_threads.argtypes = []
-        L.oracle_max_threads.restype = ctypes.c_int
-        _lib = L
+        _lib = _bind(ctypes.CDLL(_build.build()))
     return _lib
+
+
+def _bind(L):
+    """Declare the argument and return types of the oracle's C functions on L."""
+    i32, i64, p, d = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
+    L.oracle_effective_chunks.argtypes = [i32]
+    L.oracle_effective_chunks.restype = ctypes.c_int
+    L.oracle_chunk_bounds.argtypes = [i64, i32, p]
+    L.oracle_chunk_bounds.restype = None
+    L.oracle_metadata.argtypes = [p, i64, i32, i32, i32, i32, p, p, p, p, p, p]
+    L.oracle_metadata.restype = i64
+    L.oracle_forward.argtypes = [p, p, p, p, p, i64, i32, i32, i32, i32, p, i64, p, d]
+    L.oracle_forward.restype = i64
+    L.oracle_permute.argtypes = [p, p, i64, i32, i32, p]
+    L.oracle_permute.restype = None
+    L.oracle_gateup_rows.argtypes = [p, p, i64, p, i32, i32, p, d]
+    L.oracle_gateup_rows.restype = None
+    L.oracle_down_rows.argtypes = [p, p, i64, p, i32, i32, p, d]
+    L.oracle_down_rows.restype = None
+    L.oracle_unpermute.argtypes = [p, p, p, i64, i32, i32, p]
+    L.oracle_unpermute.restype = None
+    L.oracle_max_threads.argtypes = []
+    L.oracle_max_threads.restype = ctypes.c_int
+    return L
 
 
 def _c(a, dtype):

@@ -70,6 +70,8 @@ GEMM_CASES = {
     "one_row_experts": (64, 64, [1] * 7 + [0]),
     "edge": (1024, 1408, None),
     "skewed": (512, 384, [0, 0, 2000, 3, 0, 640, 1, 0]),
+    # an expert of 40 row tiles spans several 16-tile raster bands
+    "big_expert": (256, 264, [5000, 3, 0, 700]),
 }
 
 
