@@ -39,6 +39,12 @@ def _bind(L):
     L.oracle_chunk_bounds.restype = None
     L.oracle_metadata.argtypes = [p, i64, i32, i32, i32, i32, p, p, p, p, p, p]
     L.oracle_metadata.restype = i64
+    L.oracle_metadata_sized.argtypes = [p, i64, i32, i32, i32, i32, i64, p, p, p, p, p, p]
+    L.oracle_metadata_sized.restype = i64
+    L.oracle_resolve_chunks.argtypes = [i64, i32, i32, p, p]
+    L.oracle_resolve_chunks.restype = ctypes.c_int
+    L.oracle_chunk_bounds_sized.argtypes = [i64, i32, i64, p]
+    L.oracle_chunk_bounds_sized.restype = None
     L.oracle_forward.argtypes = [p, p, p, p, p, i64, i32, i32, i32, i32, p, i64, p, d]
     L.oracle_forward.restype = i64
     L.oracle_permute.argtypes = [p, p, i64, i32, i32, p]
@@ -78,7 +84,24 @@ def chunk_bounds(T: int, num_chunks: int) -> np.ndarray:
     return b
 
 
-def metadata(idx, E: int, G: int, num_chunks: int):
+def resolve_chunks(T: int, num_chunks: int, chunk_size: int = 0):
+    """(n_chunks, t_chunk, warned) from the two chunk settings."""
+    n = ctypes.c_int32(0)
+    tc = ctypes.c_int64(0)
+    r = lib().oracle_resolve_chunks(T, num_chunks, chunk_size, ctypes.byref(n), ctypes.byref(tc))
+    if r < 0:
+        raise ValueError("negative chunk setting")
+    return int(n.value), int(tc.value), bool(r)
+
+
+def chunk_bounds_sized(T: int, num_chunks: int, chunk_size: int = 0) -> np.ndarray:
+    n, tc, _ = resolve_chunks(T, num_chunks, chunk_size)
+    b = np.zeros(n + 1, dtype=np.int64)
+    lib().oracle_chunk_bounds_sized(T, n, tc, _ptr(b))
+    return b
+
+
+def metadata(idx, E: int, G: int, num_chunks: int, chunk_size: int = 0):
     """Per-chunk counts/offsets/splits and the permutation of every (t, j) copy.
 
     Returns a dict with counts [N,E], offsets [N,E+1], send [N,G], recv [N,G],
@@ -87,17 +110,17 @@ def metadata(idx, E: int, G: int, num_chunks: int):
     idx = _c(idx, np.int32)
     T, k = idx.shape
     G = max(int(G), 1)
-    n = effective_chunks(num_chunks)
+    n, tc, _ = resolve_chunks(T, num_chunks, chunk_size)
     out = dict(
         counts=np.zeros((n, E), np.int32), offsets=np.zeros((n, E + 1), np.int32),
         send=np.zeros((n, G), np.int32), recv=np.zeros((n, G), np.int32),
         dst=np.full(T * k, -1, np.int32), src_tok=np.full(T * k, -1, np.int32))
-    bad = lib().oracle_metadata(_ptr(idx), T, k, E, G, num_chunks, _ptr(out["counts"]),
-                                _ptr(out["offsets"]), _ptr(out["send"]), _ptr(out["recv"]),
-                                _ptr(out["dst"]), _ptr(out["src_tok"]))
+    bad = lib().oracle_metadata_sized(_ptr(idx), T, k, E, G, n, tc, _ptr(out["counts"]),
+                                      _ptr(out["offsets"]), _ptr(out["send"]), _ptr(out["recv"]),
+                                      _ptr(out["dst"]), _ptr(out["src_tok"]))
     if bad:
         raise ValueError(f"{bad} top_k_index entries outside [0, {E})")
-    out["bounds"] = chunk_bounds(T, num_chunks)
+    out["bounds"] = chunk_bounds_sized(T, num_chunks, chunk_size)
     return out
 
 

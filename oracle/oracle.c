@@ -18,6 +18,8 @@
  *  R3 recv splits on one GPU equal the send splits (one source rank).
  *  R5 An empty chunk or a zero-row expert contributes nothing and is valid.
  *  R6 Duplicate experts in one token's k choices are independent slots; both add.
+ *  R7 A chunk size S (with no chunk count) means chunks of exactly S tokens, the last one
+ *     holding the remainder.
  *
  * Parity pins: none of these functions is "parity unpinned"; the pins are the
  * property, brute-force, closed-form and golden-fixture tests in tests/.
@@ -57,6 +59,41 @@ void oracle_chunk_bounds(int64_t T, int32_t num_chunks, int64_t* bounds) {
   }
 }
 
+/* Chunking from the two settings of [ChunkMoE] "操作指南" step 3: moe_num_chunks and
+ * moe_chunk_size should not both be positive; when both are, moe_num_chunks wins (and a
+ * warning is due); when both are 0 the input is not split.  A chunk size S alone means
+ * chunks of S tokens, the last one holding the rest (reading R7).  With num_chunks = N the
+ * chunk size is T_chunk = ceil(T/N) ("一组关键公式").
+ * Writes the chunk count and chunk size; returns 1 if the warning is due, 0 if not, and
+ * -1 for a negative setting. */
+int oracle_resolve_chunks(int64_t T, int32_t num_chunks, int32_t chunk_size, int32_t* n_out,
+                          int64_t* t_chunk_out) {
+  if (T < 0 || num_chunks < 0 || chunk_size < 0) return -1;
+  if (num_chunks > 0) {
+    *n_out = num_chunks;
+    *t_chunk_out = (T + num_chunks - 1) / num_chunks;
+    return chunk_size > 0;
+  }
+  if (chunk_size > 0) {
+    int64_t n = (T + chunk_size - 1) / chunk_size;
+    *n_out = (int32_t)(n > 0 ? n : 1);
+    *t_chunk_out = chunk_size;
+    return 0;
+  }
+  *n_out = 1;
+  *t_chunk_out = T;
+  return 0;
+}
+
+/* Chunk bounds for a resolved chunk count n and chunk size: chunk c = tokens
+ * [min(T, c*t_chunk), min(T, (c+1)*t_chunk)). */
+void oracle_chunk_bounds_sized(int64_t T, int32_t n, int64_t t_chunk, int64_t* bounds) {
+  for (int64_t c = 0; c <= n; ++c) {
+    int64_t b = c * t_chunk;
+    bounds[c] = b < T ? b : T;
+  }
+}
+
 /* Batched pre-dispatch metadata ([ChunkMoE] "一张专业时序图", batched_pre_dispatch_metadata
  * paragraph: splits to send/receive, per-rank token counts, per-expert token counts for
  * all chunks) and the permutation of [ChunkMoE] "核心原理" (permute groups each token
@@ -72,17 +109,16 @@ void oracle_chunk_bounds(int64_t T, int32_t num_chunks, int64_t* bounds) {
  * token of row r of chunk c).  Any may be NULL.
  * Returns the number of index entries outside [0, E); on a nonzero return the outputs
  * are unspecified.  This enumeration is O(E * T * k): slow on purpose, plainly right. */
-int64_t oracle_metadata(const int32_t* idx, int64_t T, int32_t k, int32_t E, int32_t G,
-                        int32_t num_chunks, int32_t* counts, int32_t* offsets, int32_t* send,
-                        int32_t* recv, int32_t* dst, int32_t* src_tok) {
+int64_t oracle_metadata_sized(const int32_t* idx, int64_t T, int32_t k, int32_t E, int32_t G,
+                              int32_t n, int64_t t_chunk, int32_t* counts, int32_t* offsets,
+                              int32_t* send, int32_t* recv, int32_t* dst, int32_t* src_tok) {
   int64_t bad = 0;
   for (int64_t s = 0; s < T * (int64_t)k; ++s)
     if (idx[s] < 0 || idx[s] >= E) ++bad;
   if (bad) return bad;
   if (G <= 0) G = 1;
-  int32_t n = oracle_effective_chunks(num_chunks);
   int64_t* bounds = (int64_t*)malloc(sizeof(int64_t) * (size_t)(n + 1));
-  oracle_chunk_bounds(T, num_chunks, bounds);
+  oracle_chunk_bounds_sized(T, n, t_chunk, bounds);
   int32_t per_group = E / G;
   for (int32_t c = 0; c < n; ++c) {
     int64_t t0 = bounds[c], t1 = bounds[c + 1];
@@ -113,6 +149,17 @@ int64_t oracle_metadata(const int32_t* idx, int64_t T, int32_t k, int32_t E, int
   }
   free(bounds);
   return 0;
+}
+
+/* The same with chunks from num_chunks alone (T_chunk = ceil(T/N)). */
+int64_t oracle_metadata(const int32_t* idx, int64_t T, int32_t k, int32_t E, int32_t G,
+                        int32_t num_chunks, int32_t* counts, int32_t* offsets, int32_t* send,
+                        int32_t* recv, int32_t* dst, int32_t* src_tok) {
+  int32_t n = 1;
+  int64_t t_chunk = T;
+  if (oracle_resolve_chunks(T, num_chunks, 0, &n, &t_chunk) < 0) return -1;
+  return oracle_metadata_sized(idx, T, k, E, G, n, t_chunk, counts, offsets, send, recv, dst,
+                               src_tok);
 }
 
 /* Gate/up half of the SwiGLU expert ([ChunkMoE] "核心原理" expert computation; FFN form

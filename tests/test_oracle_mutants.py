@@ -30,6 +30,12 @@ MUTANTS = [
     ("only the first choice", "for (int32_t j = 0; j < k; ++j) {\n      int32_t e = idx[t * k + j];",
      "for (int32_t j = 0; j < 1; ++j) {\n      int32_t e = idx[t * k + j];"),
     ("chunk size floor(T/N)", "int64_t t_chunk = (T + n - 1) / n;", "int64_t t_chunk = T / n + (T % n > 1);"),
+    ("resolved chunk size floor(T/N)", "*t_chunk_out = (T + num_chunks - 1) / num_chunks;",
+     "*t_chunk_out = T / num_chunks + (T % num_chunks > 1);"),
+    ("chunk size wins over chunk count", "  if (num_chunks > 0) {\n    *n_out = num_chunks;",
+     "  if (num_chunks > 0 && chunk_size == 0) {\n    *n_out = num_chunks;"),
+    ("chunk size split evenly", "*t_chunk_out = chunk_size;\n    return 0;",
+     "*t_chunk_out = (T + *n_out - 1) / *n_out;\n    return 0;"),
     ("N=0 read as 0 chunks", "return num_chunks <= 0 ? 1 : num_chunks;", "return num_chunks < 0 ? 1 : (num_chunks ? num_chunks : 2);"),
     ("copies of an expert in reverse order", "for (int64_t t = t0; t < t1; ++t) {\n        for (int32_t j = 0; j < k; ++j) {\n          if (idx[t * k + j] != e) continue;",
      "for (int64_t t = t1 - 1; t >= t0; --t) {\n        for (int32_t j = 0; j < k; ++j) {\n          if (idx[t * k + j] != e) continue;"),
@@ -42,6 +48,7 @@ MUTANTS = [
 
 PIN_TESTS = [
     pins.test_chunk_bounds_golden,
+    pins.test_chunk_settings_golden,
     pins.test_metadata_golden,
     lambda: pins.test_metadata_bruteforce(3, 2, 3),
     lambda: pins.test_metadata_bruteforce(2, 2, 4),

@@ -34,6 +34,33 @@ def test_chunk_bounds_golden():
             assert b[1] - b[0] == case["T_chunk"]
 
 
+def test_chunk_settings_golden():
+    """moe_num_chunks / moe_chunk_size precedence (section 操作指南 step 3)."""
+    for case in _load("chunk_settings.json")["cases"]:
+        n, tc, warn = oracle.resolve_chunks(case["T"], case["num_chunks"], case["chunk_size"])
+        assert (n, tc, warn) == (case["n"], case["t_chunk"], case["warn"]), case
+        b = oracle.chunk_bounds_sized(case["T"], case["num_chunks"], case["chunk_size"])
+        assert b.tolist() == case["bounds"], case
+    with pytest.raises(ValueError):
+        oracle.resolve_chunks(10, 0, -1)
+
+
+def test_chunk_size_metadata_properties():
+    """Metadata with a chunk size obeys the same unique-permutation properties per chunk."""
+    rng = np.random.default_rng(4)
+    idx = rng.integers(0, 16, size=(1000, 4)).astype(np.int32)
+    for S in (1, 7, 143, 999, 1000, 5000):
+        m = oracle.metadata(idx, 16, 4, 0, chunk_size=S)
+        b = m["bounds"]
+        assert b[0] == 0 and b[-1] == 1000 and (np.diff(b)[:-1] == min(S, 1000)).all()
+        flat = idx.reshape(-1)
+        for c in range(len(b) - 1):
+            e_c = flat[b[c] * 4:b[c + 1] * 4]
+            assert m["counts"][c].tolist() == np.bincount(e_c, minlength=16).tolist()
+            d = m["dst"][b[c] * 4:b[c + 1] * 4]
+            assert sorted(d.tolist()) == list(range(len(e_c)))
+
+
 @pytest.mark.parametrize("T", [0, 1, 2, 7, 49, 100, 1000, 4097])
 @pytest.mark.parametrize("N", [0, 1, 2, 3, 4, 7, 8, 16])
 def test_chunk_bounds_properties(T, N):
