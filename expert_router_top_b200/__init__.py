@@ -12,6 +12,7 @@ and the split/count metadata of all chunks comes back to the host in one copy.
 """
 import ctypes
 import os
+import warnings
 
 import numpy as np
 import torch
@@ -35,7 +36,7 @@ class MoEError(RuntimeError):
 class Shape(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int64), ("H", ctypes.c_int32), ("I", ctypes.c_int32),
                 ("E", ctypes.c_int32), ("k", ctypes.c_int32), ("ep_groups", ctypes.c_int32),
-                ("num_chunks", ctypes.c_int32)]
+                ("num_chunks", ctypes.c_int32), ("chunk_size", ctypes.c_int32)]
 
 
 class Profile(ctypes.Structure):
@@ -64,6 +65,12 @@ def load():
     L.moe_abi_version.restype = i32
     L.moe_chunk_bounds.argtypes = [i64, i32, p]
     L.moe_chunk_bounds.restype = st
+    L.moe_resolve_chunks.argtypes = [ctypes.POINTER(Shape), p, p]
+    L.moe_resolve_chunks.restype = st
+    L.moe_last_warning.argtypes = []
+    L.moe_last_warning.restype = ctypes.c_char_p
+    L.moe_metadata_shape.argtypes = [ctypes.POINTER(Shape), p, p, p, p, p, p, p, p, sz, p]
+    L.moe_metadata_shape.restype = st
     L.moe_metadata_workspace_bytes.argtypes = [i64, i32, i32, i32, i32]
     L.moe_metadata_workspace_bytes.restype = sz
     L.moe_workspace_bytes.argtypes = [ctypes.POINTER(Shape)]
@@ -104,6 +111,9 @@ def status_string(status: int) -> str:
 def _check(status: int, what: str):
     if status != MOE_OK:
         raise MoEError(status, what)
+    msg = load().moe_last_warning()
+    if msg:
+        warnings.warn(f"{what}: {msg.decode()}", stacklevel=3)
 
 
 def _ptr(t):
@@ -128,8 +138,18 @@ def _need(t, dtype, name, device=True):
         raise ValueError(f"{name} must be a CUDA tensor")
 
 
-def shape(T, H, I, E, k, ep_groups=1, num_chunks=1) -> Shape:
-    return Shape(T, H, I, E, k, ep_groups, num_chunks)
+def shape(T, H, I, E, k, ep_groups=1, num_chunks=1, chunk_size=0) -> Shape:
+    return Shape(T, H, I, E, k, ep_groups, num_chunks, chunk_size)
+
+
+def resolve_chunks(T: int, num_chunks: int = 0, chunk_size: int = 0):
+    """(chunk count, tokens per chunk) under the num_chunks / chunk_size precedence rule."""
+    n = ctypes.c_int32(0)
+    tc = ctypes.c_int64(0)
+    s = shape(T, 8, 8, 1, 1, 1, num_chunks, chunk_size)
+    _check(load().moe_resolve_chunks(ctypes.byref(s), ctypes.byref(n), ctypes.byref(tc)),
+           "moe_resolve_chunks")
+    return int(n.value), int(tc.value)
 
 
 def chunk_bounds(T: int, num_chunks: int) -> np.ndarray:
@@ -138,8 +158,8 @@ def chunk_bounds(T: int, num_chunks: int) -> np.ndarray:
     return b
 
 
-def workspace_bytes(T, H, I, E, k, ep_groups=1, num_chunks=1) -> int:
-    s = shape(T, H, I, E, k, ep_groups, num_chunks)
+def workspace_bytes(T, H, I, E, k, ep_groups=1, num_chunks=1, chunk_size=0) -> int:
+    s = shape(T, H, I, E, k, ep_groups, num_chunks, chunk_size)
     return int(load().moe_workspace_bytes(ctypes.byref(s)))
 
 
@@ -153,14 +173,15 @@ def alloc_workspace(nbytes: int, device=None) -> torch.Tensor:
 
 
 def metadata(top_k_index: torch.Tensor, E: int, ep_groups: int = 1, num_chunks: int = 1,
-             with_permutation: bool = False, workspace: torch.Tensor = None, stream=None):
+             with_permutation: bool = False, workspace: torch.Tensor = None, stream=None,
+             chunk_size: int = 0):
     """Batched metadata for every chunk (one device pass, one host copy).
 
     Returns a dict of numpy arrays: send/recv [N,G], counts [N,E], bounds [N+1]; with
     with_permutation also torch int32 dst [T*k] and src_tok [T*k] on the device."""
     _need(top_k_index, torch.int32, "top_k_index")
     T, k = top_k_index.shape
-    n = max(num_chunks, 1)
+    n = resolve_chunks(T, num_chunks, chunk_size)[0] if chunk_size > 0 else max(num_chunks, 1)
     G = max(ep_groups, 1)
     send = np.zeros((n, G), np.int32)
     recv = np.zeros((n, G), np.int32)
@@ -170,13 +191,23 @@ def metadata(top_k_index: torch.Tensor, E: int, ep_groups: int = 1, num_chunks: 
     if with_permutation:
         dst = torch.empty(T * k, dtype=torch.int32, device=top_k_index.device)
         src = torch.empty(T * k, dtype=torch.int32, device=top_k_index.device)
-    if workspace is None:
-        workspace = alloc_workspace(metadata_workspace_bytes(T, k, E, ep_groups, num_chunks),
-                                    top_k_index.device)
-    _check(load().moe_metadata(_ptr(top_k_index), T, k, E, ep_groups, num_chunks, _ptr(send),
-                               _ptr(recv), _ptr(counts), _ptr(bounds), _ptr(dst), _ptr(src),
-                               _ptr(workspace), workspace.numel(), _stream(stream)),
-           "moe_metadata")
+    if chunk_size > 0:
+        s = shape(T, 8, 8, E, k, ep_groups, num_chunks, chunk_size)
+        if workspace is None:
+            workspace = alloc_workspace(load().moe_workspace_bytes(ctypes.byref(s)),
+                                        top_k_index.device)
+        _check(load().moe_metadata_shape(ctypes.byref(s), _ptr(top_k_index), _ptr(send),
+                                         _ptr(recv), _ptr(counts), _ptr(bounds), _ptr(dst),
+                                         _ptr(src), _ptr(workspace), workspace.numel(),
+                                         _stream(stream)), "moe_metadata_shape")
+    else:
+        if workspace is None:
+            workspace = alloc_workspace(metadata_workspace_bytes(T, k, E, ep_groups, num_chunks),
+                                        top_k_index.device)
+        _check(load().moe_metadata(_ptr(top_k_index), T, k, E, ep_groups, num_chunks, _ptr(send),
+                                   _ptr(recv), _ptr(counts), _ptr(bounds), _ptr(dst), _ptr(src),
+                                   _ptr(workspace), workspace.numel(), _stream(stream)),
+               "moe_metadata")
     out = dict(send=send, recv=recv, counts=counts, bounds=bounds)
     if with_permutation:
         out["dst"], out["src_tok"] = dst, src
@@ -188,7 +219,7 @@ FWD_FUSED_DISPATCH = 1
 
 def forward(hidden, top_k_index, top_k_weights, W_gate_up, W_down, num_chunks: int = 1,
             ep_groups: int = 1, out=None, workspace=None, stream=None,
-            dispatch: str = "separate"):
+            dispatch: str = "separate", chunk_size: int = 0):
     """One MoE layer forward, chunked as Chunk MoE.  Returns out [T,H] bf16.
 
     hidden [T,H] bf16, top_k_index [T,k] int32, top_k_weights [T,k] fp32,
@@ -210,7 +241,7 @@ def forward(hidden, top_k_index, top_k_weights, W_gate_up, W_down, num_chunks: i
     if H2 != H or tuple(W_down.shape) != (E, H, I) or tuple(top_k_index.shape) != (T, k) \
             or tuple(top_k_weights.shape) != (T, k):
         raise ValueError("inconsistent shapes")
-    s = shape(T, H, I, E, k, ep_groups, num_chunks)
+    s = shape(T, H, I, E, k, ep_groups, num_chunks, chunk_size)
     if out is None:
         out = torch.empty((T, H), dtype=torch.bfloat16, device=hidden.device)
     if workspace is None:
@@ -223,13 +254,13 @@ def forward(hidden, top_k_index, top_k_weights, W_gate_up, W_down, num_chunks: i
     return out
 
 
-def workspace_bytes_host(T, H, I, E, k, ep_groups=1, num_chunks=1) -> int:
-    s = shape(T, H, I, E, k, ep_groups, num_chunks)
+def workspace_bytes_host(T, H, I, E, k, ep_groups=1, num_chunks=1, chunk_size=0) -> int:
+    s = shape(T, H, I, E, k, ep_groups, num_chunks, chunk_size)
     return int(load().moe_workspace_bytes_host(ctypes.byref(s)))
 
 
 def forward_host(hidden, top_k_index, top_k_weights, W_gate_up, W_down, num_chunks: int = 1,
-                 ep_groups: int = 1, out=None, workspace=None, stream=None):
+                 ep_groups: int = 1, out=None, workspace=None, stream=None, chunk_size: int = 0):
     """moe_forward_host: activations in host memory (CPU tensors; pinned ones let the
     per-chunk copies overlap the kernels), weights on the device.  Returns out [T,H] bf16
     on the host, complete when the call returns."""
@@ -243,7 +274,7 @@ def forward_host(hidden, top_k_index, top_k_weights, W_gate_up, W_down, num_chun
     T, H = hidden.shape
     E, twoI, _ = W_gate_up.shape
     k = top_k_index.shape[1]
-    s = shape(T, H, twoI // 2, E, k, ep_groups, num_chunks)
+    s = shape(T, H, twoI // 2, E, k, ep_groups, num_chunks, chunk_size)
     if out is None:
         out = torch.empty((T, H), dtype=torch.bfloat16, pin_memory=hidden.is_pinned())
     if workspace is None:

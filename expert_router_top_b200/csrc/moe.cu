@@ -21,6 +21,7 @@
 #include <string.h>
 
 #include <mutex>
+#include <string>
 #include <vector>
 
 #include "device.cuh"
@@ -53,14 +54,40 @@ struct Layout {
   size_t total;
 };
 
-Dims make_dims(int64_t T, int32_t k, int32_t E, int32_t ep_groups, int32_t num_chunks) {
+thread_local std::string g_warning;
+
+// [ChunkMoE] "操作指南" step 3: num_chunks wins over chunk_size (with a warning); a chunk
+// size alone gives chunks of exactly chunk_size tokens; both 0 means one chunk.
+void resolve_chunking(int64_t T, int32_t num_chunks, int32_t chunk_size, int64_t* n,
+                      int64_t* t_chunk) {
+  if (num_chunks > 0) {
+    *n = num_chunks;
+    *t_chunk = (T + num_chunks - 1) / num_chunks;
+    if (chunk_size > 0)
+      g_warning = "moe_num_chunks and moe_chunk_size are both > 0: moe_num_chunks (" +
+                  std::to_string(num_chunks) + ") is used, moe_chunk_size (" +
+                  std::to_string(chunk_size) + ") is ignored";
+  } else if (chunk_size > 0) {
+    const int64_t c = (T + chunk_size - 1) / chunk_size;
+    *n = c > 0 ? c : 1;
+    *t_chunk = chunk_size;
+  } else {
+    *n = 1;
+    *t_chunk = T;
+  }
+}
+
+Dims make_dims(int64_t T, int32_t k, int32_t E, int32_t ep_groups, int32_t num_chunks,
+               int32_t chunk_size = 0) {
   Dims d;
   d.T = T;
   d.k = k;
   d.E = E;
   d.G = ep_groups > 0 ? ep_groups : 1;
-  d.n = num_chunks > 0 ? num_chunks : 1;
-  d.t_chunk = (T + d.n - 1) / d.n;
+  int64_t n = 1, tc = T;
+  resolve_chunking(T, num_chunks, chunk_size, &n, &tc);
+  d.n = (int32_t)n;
+  d.t_chunk = tc < T ? tc : T;  // a chunk size above T still means one chunk of T tokens
   d.tile_tokens = meta_tile_tokens(k);
   d.tiles_per_chunk = (int32_t)((d.t_chunk + d.tile_tokens - 1) / d.tile_tokens);
   if (d.tiles_per_chunk < 1) d.tiles_per_chunk = 1;
@@ -128,6 +155,12 @@ HostStaging make_host_staging(const Dims& d, int32_t H, size_t base) {
   return h;
 }
 
+std::vector<int64_t> dims_bounds(const Dims& d) {
+  std::vector<int64_t> b((size_t)d.n + 1);
+  for (int64_t c = 0; c <= d.n; ++c) b[c] = c * d.t_chunk < d.T ? c * d.t_chunk : d.T;
+  return b;
+}
+
 moe_status_t check_routing_dims(int64_t T, int32_t k, int32_t E, int32_t ep_groups,
                                 int32_t num_chunks) {
   if (T < 0 || k <= 0 || E <= 0 || ep_groups < 0 || num_chunks < 0) return MOE_ERR_ARG;
@@ -139,9 +172,14 @@ moe_status_t check_routing_dims(int64_t T, int32_t k, int32_t E, int32_t ep_grou
 }
 
 moe_status_t check_shape(const moe_shape_t* s) {
+  g_warning.clear();
   if (!s) return MOE_ERR_ARG;
   moe_status_t st = check_routing_dims(s->T, s->k, s->E, s->ep_groups, s->num_chunks);
   if (st != MOE_OK) return st;
+  if (s->chunk_size < 0) return MOE_ERR_ARG;
+  int64_t n = 1, tc = 0;
+  resolve_chunking(s->T, s->num_chunks, s->chunk_size, &n, &tc);
+  if (n > kMaxChunks) return MOE_ERR_UNSUPPORTED;
   if (s->H <= 0 || s->I <= 0 || s->H % 8 != 0 || s->I % 8 != 0) return MOE_ERR_ARG;
   return MOE_OK;
 }
@@ -391,26 +429,38 @@ size_t moe_metadata_workspace_bytes(int64_t T, int32_t k, int32_t E, int32_t ep_
 
 size_t moe_workspace_bytes(const moe_shape_t* s) {
   if (check_shape(s) != MOE_OK) return 0;
-  return make_layout(make_dims(s->T, s->k, s->E, s->ep_groups, s->num_chunks), s->H, s->I, true,
-                     true, true)
+  return make_layout(make_dims(s->T, s->k, s->E, s->ep_groups, s->num_chunks, s->chunk_size),
+                     s->H, s->I, true, true, true)
       .total;
 }
 
-moe_status_t moe_metadata(const int32_t* top_k_index, int64_t T, int32_t k, int32_t E,
-                          int32_t ep_groups, int32_t num_chunks, int32_t* send_splits,
-                          int32_t* recv_splits, int32_t* expert_counts, int64_t* chunk_bounds,
-                          int32_t* dst_rows, int32_t* src_tokens, void* workspace,
-                          size_t ws_bytes, void* stream) {
-  moe_status_t st = check_routing_dims(T, k, E, ep_groups, num_chunks);
-  if (st != MOE_OK) return st;
+moe_status_t moe_resolve_chunks(const moe_shape_t* shape, int32_t* n_chunks,
+                                int64_t* chunk_tokens) {
+  g_warning.clear();
+  if (!shape || !n_chunks || !chunk_tokens) return MOE_ERR_ARG;
+  if (shape->T < 0 || shape->num_chunks < 0 || shape->chunk_size < 0) return MOE_ERR_ARG;
+  int64_t n = 1, tc = 0;
+  resolve_chunking(shape->T, shape->num_chunks, shape->chunk_size, &n, &tc);
+  if (n > kMaxChunks) return MOE_ERR_UNSUPPORTED;
+  *n_chunks = (int32_t)n;
+  *chunk_tokens = tc;
+  return MOE_OK;
+}
+
+const char* moe_last_warning(void) { return g_warning.c_str(); }
+
+static moe_status_t metadata_impl(const Dims& d, const int32_t* top_k_index, int32_t* send_splits,
+                                  int32_t* recv_splits, int32_t* expert_counts,
+                                  int64_t* chunk_bounds, int32_t* dst_rows, int32_t* src_tokens,
+                                  void* workspace, size_t ws_bytes, void* stream) {
   if (!send_splits || !recv_splits || !expert_counts || !chunk_bounds) return MOE_ERR_ARG;
-  if (T > 0 && (!top_k_index || !workspace)) return MOE_ERR_ARG;
+  if (d.T > 0 && (!top_k_index || !workspace)) return MOE_ERR_ARG;
   if (!aligned(top_k_index, 4) || !aligned(dst_rows, 4) || !aligned(src_tokens, 4) ||
       !aligned(workspace, kAlign))
     return MOE_ERR_ALIGN;
-  const Dims d = make_dims(T, k, E, ep_groups, num_chunks);
-  moe_chunk_bounds(T, num_chunks, chunk_bounds);
-  if (T == 0) {
+  const std::vector<int64_t> bounds = dims_bounds(d);
+  memcpy(chunk_bounds, bounds.data(), sizeof(int64_t) * bounds.size());
+  if (d.T == 0) {
     memset(send_splits, 0, sizeof(int32_t) * (size_t)d.n * d.G);
     memset(recv_splits, 0, sizeof(int32_t) * (size_t)d.n * d.G);
     memset(expert_counts, 0, sizeof(int32_t) * (size_t)d.n * d.E);
@@ -419,7 +469,8 @@ moe_status_t moe_metadata(const int32_t* top_k_index, int64_t T, int32_t k, int3
   const Layout L = make_layout(d, 8, 8, false, dst_rows == nullptr, false);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   DeviceCtx* ctx = nullptr;
-  if ((st = get_ctx(&ctx)) != MOE_OK) return st;
+  moe_status_t st = get_ctx(&ctx);
+  if (st != MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int32_t* dst = dst_rows ? dst_rows : reinterpret_cast<int32_t*>(ws + L.dst);
@@ -431,6 +482,31 @@ moe_status_t moe_metadata(const int32_t* top_k_index, int64_t T, int32_t k, int3
   memcpy(send_splits, splits, sizeof(int32_t) * (size_t)d.n * d.G);
   memcpy(recv_splits, splits, sizeof(int32_t) * (size_t)d.n * d.G);  // one source rank
   return MOE_OK;
+}
+
+moe_status_t moe_metadata(const int32_t* top_k_index, int64_t T, int32_t k, int32_t E,
+                          int32_t ep_groups, int32_t num_chunks, int32_t* send_splits,
+                          int32_t* recv_splits, int32_t* expert_counts, int64_t* chunk_bounds,
+                          int32_t* dst_rows, int32_t* src_tokens, void* workspace,
+                          size_t ws_bytes, void* stream) {
+  moe_status_t st = check_routing_dims(T, k, E, ep_groups, num_chunks);
+  if (st != MOE_OK) return st;
+  return metadata_impl(make_dims(T, k, E, ep_groups, num_chunks), top_k_index, send_splits,
+                       recv_splits, expert_counts, chunk_bounds, dst_rows, src_tokens,
+                       workspace, ws_bytes, stream);
+}
+
+moe_status_t moe_metadata_shape(const moe_shape_t* shape, const int32_t* top_k_index,
+                                int32_t* send_splits, int32_t* recv_splits,
+                                int32_t* expert_counts, int64_t* chunk_bounds, int32_t* dst_rows,
+                                int32_t* src_tokens, void* workspace, size_t ws_bytes,
+                                void* stream) {
+  moe_status_t st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  return metadata_impl(make_dims(shape->T, shape->k, shape->E, shape->ep_groups,
+                                 shape->num_chunks, shape->chunk_size),
+                       top_k_index, send_splits, recv_splits, expert_counts, chunk_bounds,
+                       dst_rows, src_tokens, workspace, ws_bytes, stream);
 }
 
 moe_status_t moe_forward(const moe_shape_t* shape, const void* hidden, const int32_t* top_k_index,
@@ -457,7 +533,7 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
       !aligned(W_down, 16) || !aligned(top_k_index, 4) || !aligned(top_k_weights, 4) ||
       !aligned(workspace, kAlign))
     return MOE_ERR_ALIGN;
-  const Dims d = make_dims(T, k, E, shape->ep_groups, shape->num_chunks);
+  const Dims d = make_dims(T, k, E, shape->ep_groups, shape->num_chunks, shape->chunk_size);
   const Layout L = make_layout(d, H, I, true, true, true);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   DeviceCtx* ctx = nullptr;
@@ -475,8 +551,7 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
   // Copy what the pipeline needs out of the shared staging block.
   std::vector<int32_t> counts(ctx->host_stage + kStatusWords,
                               ctx->host_stage + kStatusWords + (size_t)d.n * d.E);
-  std::vector<int64_t> bounds((size_t)d.n + 1);
-  moe_chunk_bounds(T, shape->num_chunks, bounds.data());
+  std::vector<int64_t> bounds = dims_bounds(d);
   int n_live = 0;  // chunks with tokens; only trailing chunks can be empty
   while (n_live < d.n && bounds[n_live + 1] > bounds[n_live]) ++n_live;
 
@@ -557,7 +632,7 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
 
 size_t moe_workspace_bytes_host(const moe_shape_t* s) {
   if (check_shape(s) != MOE_OK) return 0;
-  const Dims d = make_dims(s->T, s->k, s->E, s->ep_groups, s->num_chunks);
+  const Dims d = make_dims(s->T, s->k, s->E, s->ep_groups, s->num_chunks, s->chunk_size);
   const Layout L = make_layout(d, s->H, s->I, true, true, true);
   return make_host_staging(d, s->H, L.total).total;
 }
@@ -578,7 +653,7 @@ moe_status_t moe_forward_host(const moe_shape_t* shape, const void* hidden_host,
       !aligned(top_k_index_host, 4) || !aligned(top_k_weights_host, 4) ||
       !aligned(hidden_host, 2) || !aligned(out_host, 2))
     return MOE_ERR_ALIGN;
-  const Dims d = make_dims(T, k, E, shape->ep_groups, shape->num_chunks);
+  const Dims d = make_dims(T, k, E, shape->ep_groups, shape->num_chunks, shape->chunk_size);
   const Layout L = make_layout(d, H, I, true, true, true);
   const HostStaging hs = make_host_staging(d, H, L.total);
   if (ws_bytes < hs.total) return MOE_ERR_WORKSPACE;
@@ -602,8 +677,7 @@ moe_status_t moe_forward_host(const moe_shape_t* shape, const void* hidden_host,
       cudaMemcpyAsync(w_dev, top_k_weights_host, sizeof(float) * (size_t)(T * k),
                       cudaMemcpyHostToDevice, sm) != cudaSuccess)
     return MOE_ERR_CUDA;
-  std::vector<int64_t> bounds((size_t)d.n + 1);
-  moe_chunk_bounds(T, shape->num_chunks, bounds.data());
+  std::vector<int64_t> bounds = dims_bounds(d);
   int n_live = 0;
   while (n_live < d.n && bounds[n_live + 1] > bounds[n_live]) ++n_live;
   auto len = [&](int c) { return bounds[c + 1] - bounds[c]; };

@@ -45,7 +45,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 1
+#define MOE_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define MOE_API __attribute__((visibility("default")))
@@ -77,11 +77,13 @@ typedef enum {
  *   k          experts per token, 1 <= k <= min(E, MOE_MAX_TOPK)
  *   ep_groups  G virtual expert-parallel ranks; group g owns experts
  *              [g*E/G, (g+1)*E/G); E % G == 0; 0 is read as 1
- *   num_chunks N >= 0; 0 means "do not split" and is read as 1
- *              ([ChunkMoE] "操作指南" step 3: both chunk settings 0 => no split). */
+ *   num_chunks N >= 0: split into N chunks of T_chunk = ceil(T/N) tokens
+ *   chunk_size S >= 0: split into chunks of exactly S tokens (the last holds the rest)
+ *              ([ChunkMoE] "操作指南" step 3: set only one of the two; if both are > 0,
+ *              num_chunks wins and moe_last_warning() says so; both 0 => no split). */
 typedef struct {
   int64_t T;
-  int32_t H, I, E, k, ep_groups, num_chunks;
+  int32_t H, I, E, k, ep_groups, num_chunks, chunk_size;
 } moe_shape_t;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -96,6 +98,19 @@ MOE_API int32_t moe_abi_version(void);
  * be empty (T=49, N=8 gives seven chunks of 7 and one of 0).
  * Errors: MOE_ERR_ARG if bounds is NULL, T < 0 or num_chunks < 0. */
 MOE_API moe_status_t moe_chunk_bounds(int64_t T, int32_t num_chunks, int64_t* bounds /* host [N_eff+1] */);
+
+/* The chunking a shape asks for ([ChunkMoE] "操作指南" step 3): writes the chunk count
+ * (>= 1) and the chunk size in tokens.  When both num_chunks and chunk_size are > 0,
+ * num_chunks wins and moe_last_warning() returns a warning.  Host arithmetic only.
+ * Errors: MOE_ERR_ARG for a NULL argument or a negative setting; MOE_ERR_UNSUPPORTED for
+ * more than MOE_MAX_CHUNKS chunks. */
+MOE_API moe_status_t moe_resolve_chunks(const moe_shape_t* shape, int32_t* n_chunks,
+                                        int64_t* chunk_tokens);
+
+/* The warning of the last call on this host thread that takes a shape (moe_resolve_chunks,
+ * moe_workspace_bytes*, moe_metadata_shape, moe_forward*), or "" if it gave none.  The
+ * string stays valid until the thread's next such call. */
+MOE_API const char* moe_last_warning(void);
 
 /* Device workspace, in bytes, that moe_metadata needs for these sizes; 0 if invalid. */
 MOE_API size_t moe_metadata_workspace_bytes(int64_t T, int32_t k, int32_t E, int32_t ep_groups,
@@ -173,6 +188,16 @@ MOE_API moe_status_t moe_metadata_noalloc(const int32_t* top_k_index, int64_t T,
                                           int32_t* send_splits, int32_t* recv_splits,
                                           int32_t* expert_counts, int64_t* chunk_bounds,
                                           int32_t* dst_rows, int32_t* src_tokens, void* stream);
+
+/* moe_metadata with the chunking of a shape (num_chunks or chunk_size, see moe_shape_t;
+ * H and I are not used).  The host arrays hold N_eff = the chunk count of
+ * moe_resolve_chunks(shape) rows.  workspace: >= moe_workspace_bytes of the same shape (any
+ * valid H, I; H = I = 8 gives the smallest size).  Otherwise as moe_metadata. */
+MOE_API moe_status_t moe_metadata_shape(const moe_shape_t* shape, const int32_t* top_k_index,
+                                        int32_t* send_splits, int32_t* recv_splits,
+                                        int32_t* expert_counts, int64_t* chunk_bounds,
+                                        int32_t* dst_rows, int32_t* src_tokens, void* workspace,
+                                        size_t ws_bytes, void* stream);
 
 /* One MoE layer forward pass, chunked as Chunk MoE ([ChunkMoE] "核心原理",
  * "一张专业时序图", "一组关键公式"):

@@ -40,7 +40,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_abi_version_and_status_strings():
     L = moe.load()
-    assert L.moe_abi_version() == 1
+    assert L.moe_abi_version() == 2
     for code, name in moe.STATUS_NAMES.items():
         assert moe.status_string(code).startswith(name)
     assert "unknown" in moe.status_string(99)
@@ -52,6 +52,38 @@ def test_chunk_bounds_match_oracle():
             assert moe.chunk_bounds(T, N).tolist() == oracle.chunk_bounds(T, N).tolist()
     with pytest.raises(moe.MoEError):
         moe.chunk_bounds(-1, 2)
+
+
+def test_resolve_chunks_matches_oracle():
+    """num_chunks / chunk_size precedence (Chunk MoE, section 操作指南 step 3)."""
+    import warnings
+    for T in (0, 1, 10, 49, 1000, 16384):
+        for N in (0, 1, 3, 8):
+            for S in (0, 1, 4, 143, 5000):
+                ref_n, ref_tc, ref_warn = oracle.resolve_chunks(T, N, S)
+                with warnings.catch_warnings(record=True) as caught:
+                    warnings.simplefilter("always")
+                    n, tc = moe.resolve_chunks(T, N, S)
+                assert n == ref_n and tc == ref_tc, (T, N, S)
+                assert (len(caught) > 0) == ref_warn, (T, N, S)
+                if ref_warn:
+                    assert "moe_num_chunks" in str(caught[0].message)
+
+
+def test_chunk_size_workspace_and_limits():
+    cfg = CONFIGS["qwen3"]
+    # chunks of 4096 tokens: the same buffers as num_chunks=4
+    a = moe.workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.G, 0, 4096)
+    b = moe.workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.G, 4, 0)
+    assert a == b
+    # a chunk size above T is one chunk of T tokens
+    assert moe.workspace_bytes(100, 64, 64, 8, 2, 1, 0, 10**6) == moe.workspace_bytes(
+        100, 64, 64, 8, 2, 1, 1, 0)
+    assert moe.workspace_bytes(100, 64, 64, 8, 2, 1, 0, -5) == 0
+    with pytest.raises(moe.MoEError):
+        moe.resolve_chunks(10, 0, -1)
+    with pytest.raises(moe.MoEError):  # more than MOE_MAX_CHUNKS chunks
+        moe.resolve_chunks(10**9, 0, 1)
 
 
 def _ws(cfg, N):

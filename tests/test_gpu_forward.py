@@ -72,6 +72,31 @@ def test_forward_host_buffers_match_device_forward(moe, name, pinned):
         assert torch.equal(got, ref.cpu()), f"{name} N={N} pinned={pinned}"
 
 
+@pytest.mark.parametrize("S", [1, 143, 333, 1000])
+def test_forward_chunk_size(moe, S):
+    """moe_chunk_size: chunks of exactly S tokens give the unsplit bits; with both
+    settings > 0 the chunk count wins and a warning is raised."""
+    cfg = CONFIGS["edge"]
+    cpu = layer_inputs(cfg)
+    gpu = {k: v.cuda() for k, v in cpu.items()}
+    base = _run(moe, gpu, 1)
+    out = moe.forward(gpu["hidden"], gpu["idx"], gpu["w"], gpu["wgu"], gpu["wd"], num_chunks=0,
+                      chunk_size=S)
+    torch.cuda.synchronize()
+    assert torch.equal(out, base)
+    with pytest.warns(UserWarning, match="moe_num_chunks"):
+        out2 = moe.forward(gpu["hidden"], gpu["idx"], gpu["w"], gpu["wgu"], gpu["wd"],
+                           num_chunks=3, chunk_size=S)
+    torch.cuda.synchronize()
+    assert torch.equal(out2, base)
+    host = moe.forward_host(cpu["hidden"].pin_memory(), cpu["idx"].pin_memory(),
+                            cpu["w"].pin_memory(), gpu["wgu"], gpu["wd"], num_chunks=0,
+                            chunk_size=S)
+    assert torch.equal(host, base.cpu())
+    if S == 333:
+        assert_layer_close(out, _oracle(cpu), "chunk_size=333")
+
+
 def test_forward_chunk_invariance_many_N(moe):
     cfg = CONFIGS["edge"]
     gpu = {k: v.cuda() for k, v in layer_inputs(cfg).items()}

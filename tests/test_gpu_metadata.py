@@ -9,10 +9,10 @@ from gen import CONFIGS, routing
 pytestmark = pytest.mark.gpu
 
 
-def _compare(moe, idx_np, E, G, N):
+def _compare(moe, idx_np, E, G, N, S=0):
     idx = torch.from_numpy(idx_np).cuda()
-    got = moe.metadata(idx, E, G, N, with_permutation=True)
-    ref = oracle.metadata(idx_np, E, G, N)
+    got = moe.metadata(idx, E, G, N, with_permutation=True, chunk_size=S)
+    ref = oracle.metadata(idx_np, E, G, N, chunk_size=S)
     np.testing.assert_array_equal(got["bounds"], ref["bounds"])
     np.testing.assert_array_equal(got["counts"], ref["counts"])
     np.testing.assert_array_equal(got["send"], ref["send"])
@@ -63,6 +63,15 @@ def test_metadata_random_shapes(moe, seed):
             continue
         idx = rng.integers(0, E, size=(T, k)).astype(np.int32)
         _compare(moe, idx, E, G, N)
+
+
+@pytest.mark.parametrize("S", [1, 7, 143, 256, 999, 1000, 5000])
+def test_metadata_chunk_size(moe, S):
+    """Chunks of exactly S tokens (moe_chunk_size, section 操作指南 step 3)."""
+    cfg = CONFIGS["edge"]
+    idx, _ = routing(cfg)
+    got = _compare(moe, idx, cfg.E, 4, 0, S)
+    assert got["bounds"][1] == min(S, cfg.T)
 
 
 def test_metadata_many_tiles_per_chunk(moe):
