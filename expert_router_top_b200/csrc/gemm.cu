@@ -57,6 +57,15 @@
 #ifndef MOE_GEMM_BAND
 #define MOE_GEMM_BAND 16  // M tiles per raster band: an expert's A rows stay in L2 across N tiles
 #endif
+#ifndef MOE_GEMM_B4D
+#define MOE_GEMM_B4D 0  // gate/up: one 4-D box fetches the gate and the up rows of a tile
+#endif
+#ifndef MOE_GEMM_PREFETCH
+#define MOE_GEMM_PREFETCH 0  // K blocks of L2 prefetch ahead of the smem loads (0: none)
+#endif
+#ifndef MOE_GEMM_PREFETCH_A
+#define MOE_GEMM_PREFETCH_A 0  // 1: prefetch the A rows too, not only the weights
+#endif
 #ifndef MOE_GEMM_B_POLICY
 #define MOE_GEMM_B_POLICY 2  // L2 policy of weight loads: 0 normal, 1 evict_first, 2 evict_last
 #endif
@@ -98,6 +107,7 @@ struct KParams {
   int32_t total_tiles;
   const int32_t* gather;  // gathered A: token row of each permuted row (nullptr: plain A)
   int32_t reverse;        // 1: walk the tiles (hence the experts) in descending order
+  int32_t b4d;            // 1: tmB is the 4-D gate/up view (one box per stage)
 };
 
 template <int kStages>
@@ -345,16 +355,40 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;  // per-stage bits, for the abort drain
       bool ok = true;
-      for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
+      // A row and B row of the tile at linear index L (of this CTA's tile stream)
+      int32_t t_e = 0, t_n = 0;
+      auto coords = [&](int32_t L, int32_t& row0, int32_t& brow) {
         const Tile t = decode_tile<G::kTileM>(p.reverse ? p.total_tiles - 1 - L : L, tile_start,
                                               off, E, p.n_tiles);
-        const int32_t row0 = off[t.e] + t.m * G::kTileM + (int32_t)rank * kRowsPerCta;
-        int32_t brow;
+        t_e = t.e;
+        t_n = t.n;
+        row0 = off[t.e] + t.m * G::kTileM + (int32_t)rank * kRowsPerCta;
         if (kSwiGLU)  // pair: the even CTA stages the gate rows, the odd one the up rows
           brow = t.e * p.b_rows + t.n * (BN / 2) + (kPair ? (int32_t)rank * p.up_off : 0);
         else
           brow = t.e * p.b_rows + t.n * BN + (kPair ? (int32_t)rank * (BN / 2) : 0);
+      };
+      // L2 prefetch of K block kb of the tile at (row0, brow): the weight box(es), and the
+      // A box when asked; nothing lands in shared memory and nothing is waited for
+      auto prefetch = [&](int32_t row0, int32_t brow, int32_t kb) {
+        if (!p.b4d) {  // (the 4-D gate/up view is not prefetched)
+          tma_prefetch_2d(tmB, kb * BK, brow);
+          if (kSwiGLU && !kPair) tma_prefetch_2d(tmB, kb * BK, brow + p.up_off);
+        }
+        if (MOE_GEMM_PREFETCH_A) tma_prefetch_2d(tmA, kb * BK, row0);
+      };
+      int32_t nrow0 = 0, nbrow = 0;
+      for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
+        int32_t row0, brow;
+        const bool has_next = L + n_streams < p.total_tiles;
+        if (MOE_GEMM_PREFETCH > 0 && has_next) coords(L + n_streams, nrow0, nbrow);
+        coords(L, row0, brow);  // last, so that t_e / t_n describe this tile
         for (int32_t kb = 0; kb < p.num_kb; ++kb) {
+          if (MOE_GEMM_PREFETCH > 0) {
+            const int32_t pk = kb + MOE_GEMM_PREFETCH;
+            if (pk < p.num_kb) prefetch(row0, brow, pk);
+            else if (has_next && pk - p.num_kb < p.num_kb) prefetch(nrow0, nbrow, pk - p.num_kb);
+          }
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort, p.status)) {
             ok = false;
             break;
@@ -369,7 +403,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
           } else {
             mbar_arrive_expect_tx(&ctl->full[stage], G::kTxBytes);
             tma_load_2d(a_dst, tmA, &ctl->full[stage], kb * BK, row0, pol_a);
-            if (kSwiGLU) {
+            if (kSwiGLU && p.b4d) {
+              // {K, row in block, 128-row block n, 2e + gate/up}: gate block n, then up block n
+              tma_load_4d(b_dst, tmB, &ctl->full[stage], kb * BK, 0, t_n, 2 * t_e, pol_w);
+            } else if (kSwiGLU) {
               tma_load_2d(b_dst, tmB, &ctl->full[stage], kb * BK, brow, pol_w);
               tma_load_2d(b_dst + G::kBBytes / 2, tmB, &ctl->full[stage], kb * BK,
                           brow + p.up_off, pol_w);
@@ -563,6 +600,26 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int32_t cols, int3
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 4-D view of W_gate_up [E][2I][K] for one-box gate/up loads: dims {K, 128, I/128, 2E}
+// with strides {2K, 128*2K, I*2K} bytes; box {BK, 128, 1, 2} = the gate rows and the up rows
+// of one 128-column output block of one expert, in that order.
+bool make_map_gateup4d(CUtensorMap* m, const void* base, int32_t E, int32_t I, int32_t K) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc || I % 128 != 0) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)K, 128, (cuuint64_t)(I / 128), (cuuint64_t)(2 * E)};
+  const cuuint64_t strides[3] = {(cuuint64_t)K * 2, (cuuint64_t)128 * K * 2,
+                                 (cuuint64_t)I * K * 2};
+  const cuuint32_t box[4] = {(cuuint32_t)BK, 128, 1, 2};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             BK == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+             MOE_GEMM_L2_PROMO == 2   ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+             : MOE_GEMM_L2_PROMO == 1 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
+                                      : CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 bool gemm_supports_gather() { return MOE_GEMM_2SM == 0; }
@@ -594,9 +651,12 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
   }
   const bool map_a_ok = gather ? make_map(&mA, a.gather_src, a.gather_src_rows, a.K, 1)
                                : make_map(&mA, a.A, a.rows, a.K, kRowsPerCta);
+  // one-box gate/up weights (single-CTA, plain A, I a multiple of 128)
+  const bool b4d = MOE_GEMM_B4D && swiglu && !kPair && !gather && a.out_cols % 128 == 0 &&
+                   make_map_gateup4d(&mB, a.B, a.E, a.out_cols, a.K);
   if (!map_a_ok ||
-      !make_map(&mB, a.B, (int64_t)a.E * a.b_rows, a.K,
-                kPair ? BN / 2 : (swiglu ? BN / 2 : BN))) {
+      (!b4d && !make_map(&mB, a.B, (int64_t)a.E * a.b_rows, a.K,
+                         kPair ? BN / 2 : (swiglu ? BN / 2 : BN)))) {
     *err_detail = 2;
     return cudaErrorInvalidValue;
   }
@@ -613,6 +673,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
   p.total_tiles = (int32_t)a.total_tiles;
   p.gather = a.gather;
   p.reverse = a.reverse ? 1 : 0;
+  p.b4d = b4d ? 1 : 0;
   constexpr size_t smem = smem_bytes<kPair>();
   cudaError_t e;
   if (kPair) {
