@@ -55,6 +55,8 @@ def _bind(L):
     L.oracle_down_rows.restype = None
     L.oracle_unpermute.argtypes = [p, p, p, i64, i32, i32, p]
     L.oracle_unpermute.restype = None
+    L.oracle_backward.argtypes = [p, p, p, p, p, p, i64, i32, i32, i32, i32, p, p, p, p, d]
+    L.oracle_backward.restype = i64
     L.oracle_max_threads.argtypes = []
     L.oracle_max_threads.restype = ctypes.c_int
     return L
@@ -192,3 +194,28 @@ def unpermute(Y_bits, dst, w, k: int):
     out = np.zeros((Tc, H), np.float64)
     lib().oracle_unpermute(_ptr(Y_bits), _ptr(dst), _ptr(w), Tc, H, k, _ptr(out))
     return out
+
+
+def backward(hidden_bits, idx, w, wgu_bits, wd_bits, dout_bits, nthreads: int = 0):
+    """fp64 gradients of sum(out * dout): returns (d_hidden [T,H], d_weights [T,k],
+    dW_gate_up [E,2I,H], dW_down [E,H,I])."""
+    hidden_bits = _c(hidden_bits, np.uint16)
+    idx = _c(idx, np.int32)
+    w = _c(w, np.float32)
+    wgu_bits = _c(wgu_bits, np.uint16)
+    wd_bits = _c(wd_bits, np.uint16)
+    dout_bits = _c(dout_bits, np.uint16)
+    T, H = hidden_bits.shape
+    E, twoI, _ = wgu_bits.shape
+    I = twoI // 2
+    k = idx.shape[1]
+    dx = np.zeros((T, H), np.float64)
+    dw = np.zeros((T, k), np.float64)
+    dwgu = np.zeros((E, 2 * I, H), np.float64)
+    dwd = np.zeros((E, H, I), np.float64)
+    bad = lib().oracle_backward(_ptr(hidden_bits), _ptr(idx), _ptr(w), _ptr(wgu_bits),
+                                _ptr(wd_bits), _ptr(dout_bits), T, H, I, E, k, _ptr(dx), _ptr(dw),
+                                _ptr(dwgu), _ptr(dwd), nthreads)
+    if bad:
+        raise ValueError("top_k_index entries outside [0, E)")
+    return dx, dw, dwgu, dwd

@@ -295,3 +295,120 @@ void oracle_unpermute(const uint16_t* Y, const int32_t* dst, const float* w, int
     }
   }
 }
+
+/* ---- backward ---------------------------------------------------------------------------
+ * Gradient of the layer output with respect to its inputs and expert weights.  The article
+ * trains through this layer: its backward pass mirrors the forward chunk pipeline through
+ * autograd, with the expert computation optionally recomputed (chunk_moe_recompute)
+ * ([ChunkMoE] "一张专业时序图", last paragraph of the timing discussion; "一组关键公式" on
+ * recompute).  The mathematics is the chain rule through the definition of oracle_forward;
+ * for one copy (t, j) with e = idx[t][j], x = hidden[t]:
+ *   g = Wg x, u = Wu x, sig = 1/(1+e^-g), h = g sig u, y = Wd h
+ *   d_w[t][j] = <dout[t], y>;  dy = w[t][j] dout[t];  dh = Wd^T dy
+ *   du = dh * g sig;  dg = dh * u * (sig + g sig (1 - sig))
+ *   d_x[t] += Wg^T dg + Wu^T du;  dWd[e] += dy h^T;  dWg[e] += dg x^T;  dWu[e] += du x^T
+ * All fp64.  dWgu is [E][2I][H] (gate rows then up rows), dWd is [E][H][I]; both are
+ * overwritten.  Returns the number of out-of-range indices (nonzero: outputs unspecified). */
+int64_t oracle_backward(const uint16_t* hidden, const int32_t* idx, const float* w,
+                        const uint16_t* wgu, const uint16_t* wd, const uint16_t* dout, int64_t T,
+                        int32_t H, int32_t I, int32_t E, int32_t k, double* dx, double* dw,
+                        double* dWgu, double* dWd, int nthreads) {
+  set_threads(nthreads);
+  for (int64_t s = 0; s < T * (int64_t)k; ++s)
+    if (idx[s] < 0 || idx[s] >= E) return 1;
+  memset(dWgu, 0, sizeof(double) * (size_t)E * 2 * I * H);
+  memset(dWd, 0, sizeof(double) * (size_t)E * H * I);
+  /* per expert (parallel): every copy routed to e, in flat order */
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int32_t e = 0; e < E; ++e) {
+    double* x = (double*)malloc(sizeof(double) * (size_t)H);
+    double* g = (double*)malloc(sizeof(double) * (size_t)I);
+    double* u = (double*)malloc(sizeof(double) * (size_t)I);
+    double* h = (double*)malloc(sizeof(double) * (size_t)I);
+    double* dy = (double*)malloc(sizeof(double) * (size_t)H);
+    double* dh = (double*)malloc(sizeof(double) * (size_t)I);
+    const uint16_t* wg = wgu + (int64_t)e * 2 * I * H;
+    const uint16_t* wu = wg + (int64_t)I * H;
+    const uint16_t* wde = wd + (int64_t)e * H * I;
+    double* dwg = dWgu + (int64_t)e * 2 * I * H;
+    double* dwu = dwg + (int64_t)I * H;
+    double* dwd = dWd + (int64_t)e * H * I;
+    for (int64_t t = 0; t < T; ++t) {
+      for (int32_t j = 0; j < k; ++j) {
+        if (idx[t * k + j] != e) continue;
+        for (int32_t c = 0; c < H; ++c) x[c] = bf16_to_f64(hidden[t * H + c]);
+        for (int32_t i = 0; i < I; ++i) {
+          double a = 0.0, b = 0.0;
+          for (int32_t c = 0; c < H; ++c) {
+            a += bf16_to_f64(wg[(int64_t)i * H + c]) * x[c];
+            b += bf16_to_f64(wu[(int64_t)i * H + c]) * x[c];
+          }
+          g[i] = a;
+          u[i] = b;
+          h[i] = silu(a) * b;
+        }
+        double wt = (double)w[t * k + j];
+        for (int32_t o = 0; o < H; ++o) dy[o] = wt * bf16_to_f64(dout[t * H + o]);
+        for (int32_t i = 0; i < I; ++i) {
+          double a = 0.0;
+          for (int32_t o = 0; o < H; ++o) a += bf16_to_f64(wde[(int64_t)o * I + i]) * dy[o];
+          dh[i] = a;
+        }
+        for (int32_t o = 0; o < H; ++o)
+          for (int32_t i = 0; i < I; ++i) dwd[(int64_t)o * I + i] += dy[o] * h[i];
+        for (int32_t i = 0; i < I; ++i) {
+          double sig = 1.0 / (1.0 + exp(-g[i]));
+          double du = dh[i] * g[i] * sig;
+          double dg = dh[i] * u[i] * (sig + g[i] * sig * (1.0 - sig));
+          for (int32_t c = 0; c < H; ++c) {
+            dwg[(int64_t)i * H + c] += dg * x[c];
+            dwu[(int64_t)i * H + c] += du * x[c];
+          }
+        }
+      }
+    }
+    free(x); free(g); free(u); free(h); free(dy); free(dh);
+  }
+  /* per token (parallel): d_x and d_w */
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t t = 0; t < T; ++t) {
+    double* h = (double*)malloc(sizeof(double) * (size_t)I);
+    double* y = (double*)malloc(sizeof(double) * (size_t)H);
+    double* dy = (double*)malloc(sizeof(double) * (size_t)H);
+    double* dh = (double*)malloc(sizeof(double) * (size_t)I);
+    double* out = dx + t * H;
+    for (int32_t c = 0; c < H; ++c) out[c] = 0.0;
+    for (int32_t j = 0; j < k; ++j) {
+      int32_t e = idx[t * k + j];
+      const uint16_t* wg = wgu + (int64_t)e * 2 * I * H;
+      const uint16_t* wu = wg + (int64_t)I * H;
+      const uint16_t* wde = wd + (int64_t)e * H * I;
+      gateup_row(hidden + t * H, wgu + (int64_t)e * 2 * I * H, H, I, h);
+      down_row(h, wde, H, I, y);
+      double dot = 0.0;
+      for (int32_t o = 0; o < H; ++o) dot += bf16_to_f64(dout[t * H + o]) * y[o];
+      dw[t * k + j] = dot;
+      double wt = (double)w[t * k + j];
+      for (int32_t o = 0; o < H; ++o) dy[o] = wt * bf16_to_f64(dout[t * H + o]);
+      for (int32_t i = 0; i < I; ++i) {
+        double a = 0.0;
+        for (int32_t o = 0; o < H; ++o) a += bf16_to_f64(wde[(int64_t)o * I + i]) * dy[o];
+        dh[i] = a;
+      }
+      for (int32_t i = 0; i < I; ++i) {
+        double gi = 0.0, ui = 0.0;
+        for (int32_t c = 0; c < H; ++c) {
+          gi += bf16_to_f64(wg[(int64_t)i * H + c]) * bf16_to_f64(hidden[t * H + c]);
+          ui += bf16_to_f64(wu[(int64_t)i * H + c]) * bf16_to_f64(hidden[t * H + c]);
+        }
+        double sig = 1.0 / (1.0 + exp(-gi));
+        double du = dh[i] * gi * sig;
+        double dg = dh[i] * ui * (sig + gi * sig * (1.0 - sig));
+        for (int32_t c = 0; c < H; ++c)
+          out[c] += bf16_to_f64(wg[(int64_t)i * H + c]) * dg + bf16_to_f64(wu[(int64_t)i * H + c]) * du;
+      }
+    }
+    free(h); free(y); free(dy); free(dh);
+  }
+  return 0;
+}

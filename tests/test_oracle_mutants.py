@@ -46,6 +46,19 @@ MUTANTS = [
      "double wt = 1.0;\n      for (int32_t c = 0; c < H; ++c) o[c] += wt * bf16_to_f64(y[c]);"),
 ]
 
+BACKWARD_MUTANTS = [
+    ("dW_gate: sigmoid derivative sign", "double dg = dh[i] * u[i] * (sig + g[i] * sig * (1.0 - sig));",
+     "double dg = dh[i] * u[i] * (sig - g[i] * sig * (1.0 - sig));"),
+    ("dW_up: silu dropped", "double du = dh[i] * g[i] * sig;", "double du = dh[i] * sig;"),
+    ("dW_down: routing weight dropped",
+     "for (int32_t o = 0; o < H; ++o) dy[o] = wt * bf16_to_f64(dout[t * H + o]);\n        for (int32_t i = 0; i < I; ++i) {\n          double a = 0.0;",
+     "for (int32_t o = 0; o < H; ++o) dy[o] = bf16_to_f64(dout[t * H + o]);\n        for (int32_t i = 0; i < I; ++i) {\n          double a = 0.0;"),
+    ("d_x: up path dropped", "out[c] += bf16_to_f64(wg[(int64_t)i * H + c]) * dg + bf16_to_f64(wu[(int64_t)i * H + c]) * du;",
+     "out[c] += bf16_to_f64(wg[(int64_t)i * H + c]) * dg;"),
+    ("d_w: dot with dy", "for (int32_t o = 0; o < H; ++o) dot += bf16_to_f64(dout[t * H + o]) * y[o];",
+     "for (int32_t o = 0; o < H; ++o) dot += bf16_to_f64(dout[t * H + o]) * y[o] * w[t * k + j];"),
+]
+
 PIN_TESTS = [
     pins.test_chunk_bounds_golden,
     pins.test_chunk_settings_golden,
@@ -101,3 +114,25 @@ def test_pins_catch_planted_mistake(name, old, new):
         finally:
             oracle.use_library(None)
     assert caught, f"no pin caught the planted mistake '{name}'"
+
+
+@pytest.mark.parametrize("name,old,new", BACKWARD_MUTANTS, ids=[m[0] for m in BACKWARD_MUTANTS])
+def test_backward_pins_catch_planted_mistake(name, old, new):
+    import test_oracle_backward_pins as bpins
+    text = open(SRC).read()
+    assert text.count(old) == 1, f"mutation site for '{name}' not found exactly once"
+    with tempfile.TemporaryDirectory() as d:
+        oracle.use_library(_build(text.replace(old, new), d))
+        caught = False
+        try:
+            for t in (lambda: bpins.test_backward_matches_fp64_autodiff(0),
+                      bpins.test_weight_gradient_is_the_exact_derivative,
+                      bpins.test_identity_like_experts_input_gradient_closed_form):
+                try:
+                    t()
+                except AssertionError:
+                    caught = True
+                    break
+        finally:
+            oracle.use_library(None)
+    assert caught, f"no backward pin caught the planted mistake '{name}'"
