@@ -27,8 +27,9 @@ MUTANTS = [
      "double acc = 0.0;\n    for (int32_t i = 0; i < I; ++i) acc += bf16_to_f64(wd_e[(int64_t)i * H + o]) * h[i];"),
     ("routing weight dropped", "for (int32_t c = 0; c < H; ++c) acc[c] += wt * y[c];",
      "for (int32_t c = 0; c < H; ++c) acc[c] += y[c];"),
-    ("only the first choice", "for (int32_t j = 0; j < k; ++j) {\n      int32_t e = idx[t * k + j];",
-     "for (int32_t j = 0; j < 1; ++j) {\n      int32_t e = idx[t * k + j];"),
+    ("only the first choice",
+     "for (int32_t j = 0; j < k; ++j) {\n      int32_t e = idx[t * k + j];\n      if (e < 0 || e >= E) {",
+     "for (int32_t j = 0; j < 1; ++j) {\n      int32_t e = idx[t * k + j];\n      if (e < 0 || e >= E) {"),
     ("chunk size floor(T/N)", "int64_t t_chunk = (T + n - 1) / n;", "int64_t t_chunk = T / n + (T % n > 1);"),
     ("resolved chunk size floor(T/N)", "*t_chunk_out = (T + num_chunks - 1) / num_chunks;",
      "*t_chunk_out = T / num_chunks + (T % num_chunks > 1);"),
