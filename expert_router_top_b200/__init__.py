@@ -86,6 +86,10 @@ def load():
     L.moe_workspace_bytes_host.restype = sz
     L.moe_forward_host.argtypes = [ctypes.POINTER(Shape), p, p, p, p, p, p, p, sz, p]
     L.moe_forward_host.restype = st
+    L.moe_backward_workspace_bytes.argtypes = [ctypes.POINTER(Shape)]
+    L.moe_backward_workspace_bytes.restype = sz
+    L.moe_backward.argtypes = [ctypes.POINTER(Shape), p, p, p, p, p, p, p, p, p, p, p, sz, p]
+    L.moe_backward.restype = st
     L.moe_check_device_status.argtypes = [p, sz, p]
     L.moe_check_device_status.restype = st
     L.moe_permute.argtypes = [p, p, i64, i32, i32, p, p]
@@ -285,6 +289,36 @@ def forward_host(hidden, top_k_index, top_k_weights, W_gate_up, W_down, num_chun
                                    _ptr(workspace), workspace.numel(), _stream(stream)),
            "moe_forward_host")
     return out
+
+
+def backward(hidden, top_k_index, top_k_weights, W_gate_up, W_down, d_out, num_chunks: int = 1,
+             ep_groups: int = 1, chunk_size: int = 0, workspace=None, stream=None):
+    """Backward of forward() for the loss sum(out * d_out), with the expert computation
+    recomputed chunk by chunk.  Returns (d_hidden bf16 [T,H], d_weights fp32 [T,k],
+    dW_gate_up fp32 [E,2I,H], dW_down fp32 [E,H,I])."""
+    for t, dt, name in ((hidden, torch.bfloat16, "hidden"), (top_k_index, torch.int32, "top_k_index"),
+                        (top_k_weights, torch.float32, "top_k_weights"),
+                        (W_gate_up, torch.bfloat16, "W_gate_up"), (W_down, torch.bfloat16, "W_down"),
+                        (d_out, torch.bfloat16, "d_out")):
+        _need(t, dt, name)
+    T, H = hidden.shape
+    E, twoI, _ = W_gate_up.shape
+    I = twoI // 2
+    k = top_k_index.shape[1]
+    s = shape(T, H, I, E, k, ep_groups, num_chunks, chunk_size)
+    dev = hidden.device
+    d_hidden = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    d_weights = torch.empty((T, k), dtype=torch.float32, device=dev)
+    dW_gate_up = torch.empty((E, 2 * I, H), dtype=torch.float32, device=dev)
+    dW_down = torch.empty((E, H, I), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = alloc_workspace(load().moe_backward_workspace_bytes(ctypes.byref(s)), dev)
+    _check(load().moe_backward(ctypes.byref(s), _ptr(hidden), _ptr(top_k_index),
+                               _ptr(top_k_weights), _ptr(W_gate_up), _ptr(W_down), _ptr(d_out),
+                               _ptr(d_hidden), _ptr(d_weights), _ptr(dW_gate_up), _ptr(dW_down),
+                               _ptr(workspace), workspace.numel(), _stream(stream)),
+           "moe_backward")
+    return d_hidden, d_weights, dW_gate_up, dW_down
 
 
 def check_device_status(workspace, stream=None):

@@ -1,0 +1,587 @@
+// backward.cu -- backward pass of the chunked MoE layer, with the expert computation
+// recomputed per chunk.
+//
+// The Chunk MoE article ("昇腾MindSpeed分块专家计算Chunk MoE") trains through this layer:
+// the backward pass mirrors the forward chunk pipeline (section 一张专业时序图, the last
+// paragraph on the timing diagram) and the expert computation may be recomputed to keep the
+// activation peak low (chunk_moe_recompute, sections 一组关键公式 and 操作指南).  For one
+// copy (t, j) routed to expert e, with x = hidden[t]:
+//   g = W_gate x, u = W_up x, h = silu(g) u, y = W_down h        (recomputed)
+//   d_w[t][j] = <dout[t], y>;  dY = w[t][j] dout[t];  dh = W_down^T dY
+//   du = dh silu(g);  dg = dh u silu'(g);  dX = W_gate^T dg + W_up^T du
+//   d_hidden[t] = sum_j dX;  dW_down[e] += dY h^T;  dW_gate|up[e] += dg|du x^T
+//
+// Backward buffers hold each expert's rows padded to a multiple of 64 (zero rows), so that
+// the weight-gradient GEMMs reduce over an expert's rows in whole 64-row K blocks.
+//
+// The GEMMs run on one tcgen05 kernel (one CTA per SM, TMA producer warp, one MMA thread,
+// four epilogue warps, 4-stage ring, double-buffered TMEM, as the forward kernel) in four
+// modes:
+//   kRawGU    [g u] = X W_gate_up^T           A rows K-major, B K-major   epilogue: g, u, h
+//   kDSwiGLU  dh = dY W_down                  B MN-major                  epilogue: dg, du
+//   kDPlain   dX = [dg du] W_gate_up          B MN-major                  epilogue: bf16 store
+//   kWGrad    dW[e] += S_A[e]^T S_B[e]        A and B MN-major, K = rows  epilogue: fp32 +=
+// MN-major operands use the 128-byte-swizzled MN-major canonical layout: 64-element MN
+// blocks of 64 K rows x 128 B (8 KB apart: the leading byte offset), 8-row K groups 1 KB
+// apart (the stride byte offset); one MMA K step of 16 advances 2 KB.
+#include <string.h>
+
+#include <vector>
+
+#include "device.cuh"
+#include "internal.h"
+#include "moe.h"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int kThreads = 192;
+constexpr uint32_t kABytes = BM * BK * 2, kBBytes = BN * BK * 2, kStageBytes = kABytes + kBBytes;
+constexpr uint32_t kTmemCols = 2 * BN;
+constexpr int kMaxE = 1024;
+constexpr int kPadRows = 64;  // backward rows of one expert are padded to this multiple
+
+enum Mode { kRawGU = 0, kDSwiGLU = 1, kDPlain = 2, kWGrad = 3 };
+
+struct BParams {
+  const int32_t* offsets;  // padded expert row offsets [E+1] (multiples of 64)
+  uint32_t* status;
+  int32_t E;
+  int32_t m_tiles;   // kWGrad: M tiles per expert
+  int32_t n_tiles;   // N tiles per expert
+  int32_t num_kb;    // row-grouped modes: K blocks
+  int32_t M;         // kWGrad: rows of the gradient
+  int32_t N;         // output columns
+  int32_t I;         // gate/up split of 2I-wide tensors
+  int32_t b_rows;    // rows of one expert's weight matrix in B
+  int32_t total_tiles;
+  __nv_bfloat16* out0;      // kRawGU: GU [rows][2I]; kDSwiGLU: dGU [rows][2I]; kDPlain: [rows][N]
+  __nv_bfloat16* out1;      // kRawGU: Act [rows][I]
+  const __nv_bfloat16* aux; // kDSwiGLU: GU [rows][2I]
+  float* acc;               // kWGrad: [E][M][N] fp32, accumulated into
+};
+
+struct Ctl {
+  uint64_t full[STAGES], empty[STAGES], tfull[2], tempty[2], drain;
+  uint32_t tmem_base;
+  int abort;
+};
+constexpr size_t kCtlBytes = 256;
+static_assert(sizeof(Ctl) <= kCtlBytes, "control block");
+constexpr size_t kSmem = 1024 + STAGES * kStageBytes + kCtlBytes + 2 * (kMaxE + 1) * 4;
+
+__host__ __device__ constexpr uint32_t idesc(bool a_mn, bool b_mn) {
+  return umma_idesc_bf16_f32(BM, BN) | (a_mn ? 1u << 15 : 0u) | (b_mn ? 1u << 16 : 0u);
+}
+
+// MN-major operand descriptor (128-byte swizzle): LBO = 8 KB between 64-element MN blocks,
+// SBO = 1 KB between 8-row K groups, version 1, swizzle mode 2.
+__device__ __forceinline__ uint64_t mn_desc(uint32_t addr) {
+  return static_cast<uint64_t>((addr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>(8192 >> 4) << 16) |
+         (static_cast<uint64_t>(1024 >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+struct Tile {
+  int32_t e, m, n;
+};
+
+template <int kMode>
+__device__ __forceinline__ Tile decode(int32_t L, const int32_t* ts, const int32_t* off,
+                                       int32_t E, const BParams& p) {
+  int32_t lo = 0, hi = E - 1;
+  while (lo < hi) {
+    const int32_t mid = (lo + hi + 1) >> 1;
+    if (ts[mid] <= L) lo = mid;
+    else hi = mid - 1;
+  }
+  const int32_t local = L - ts[lo];
+  Tile t;
+  t.e = lo;
+  if (kMode == kWGrad) {
+    t.m = local / p.n_tiles;
+    t.n = local - t.m * p.n_tiles;
+  } else {
+    const int32_t mt = (off[lo + 1] - off[lo] + BM - 1) / BM;
+    t.n = local / mt;
+    t.m = local - t.n * mt;
+  }
+  return t;
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+
+template <int kMode>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                    const __grid_constant__ CUtensorMap tmB, const BParams p) {
+  constexpr bool kAmn = kMode == kWGrad;
+  constexpr bool kBmn = kMode != kRawGU;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * kABytes;
+  Ctl* ctl = reinterpret_cast<Ctl*>(smem + STAGES * kStageBytes);
+  int32_t* off = reinterpret_cast<int32_t*>(smem + STAGES * kStageBytes + kCtlBytes);
+  int32_t* ts = off + (kMaxE + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int32_t E = p.E;
+
+  for (int32_t i = threadIdx.x; i <= E; i += kThreads) off[i] = p.offsets[i];
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&ctl->full[s], 1);
+      mbar_init(&ctl->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctl->tfull[b], 1);
+      mbar_init(&ctl->tempty[b], 4 * 32);
+    }
+    mbar_init(&ctl->drain, 1);
+    ctl->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&ctl->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  if (warp == 2) {  // exclusive prefix of tiles per expert
+    const int32_t per = (E + 31) / 32;
+    const int32_t e0 = lane * per, e1 = min(E, e0 + per);
+    auto tiles_of = [&](int32_t e) -> int32_t {
+      const int32_t rows = off[e + 1] - off[e];
+      if (kMode == kWGrad) return rows > 0 ? p.m_tiles * p.n_tiles : 0;
+      return ((rows + BM - 1) / BM) * p.n_tiles;
+    };
+    int32_t sum = 0;
+    for (int32_t e = e0; e < e1; ++e) sum += tiles_of(e);
+    int32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int32_t run = incl - sum;
+    for (int32_t e = e0; e < e1; ++e) {
+      ts[e] = run;
+      run += tiles_of(e);
+    }
+    if (lane == 31) ts[E] = incl;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = ctl->tmem_base;
+  volatile int* abort = &ctl->abort;
+
+  if (warp == 0) {
+    if (lane == 0) {  // ---------------- TMA producer ----------------
+      const uint64_t pol = l2_policy_evict_normal();
+      int stage = 0;
+      uint32_t phase = 0, armed = 0, armed_parity = 0;
+      bool ok = true;
+      for (int32_t L = blockIdx.x; L < p.total_tiles && ok; L += gridDim.x) {
+        const Tile t = decode<kMode>(L, ts, off, E, p);
+        const int32_t nkb = kMode == kWGrad ? (off[t.e + 1] - off[t.e]) / BK : p.num_kb;
+        for (int32_t kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&ctl->full[stage], kStageBytes);
+          uint8_t* a = sA + stage * kABytes;
+          uint8_t* b = sB + stage * kBBytes;
+          uint64_t* bar = &ctl->full[stage];
+          if (kMode == kWGrad) {
+            const int32_t r0 = off[t.e] + kb * BK;  // K rows of this block
+            for (int q = 0; q < 2; ++q)
+              tma_load_2d(a + q * 8192, &tmA, bar, t.m * BM + q * 64, r0, pol);
+            for (int q = 0; q < 4; ++q)
+              tma_load_2d(b + q * 8192, &tmB, bar, t.n * BN + q * 64, r0, pol);
+          } else {
+            const int32_t row0 = off[t.e] + t.m * BM;
+            tma_load_2d(a, &tmA, bar, kb * BK, row0, pol);
+            if (kMode == kRawGU) {
+              const int32_t brow = t.e * p.b_rows + t.n * (BN / 2);
+              tma_load_2d(b, &tmB, bar, kb * BK, brow, pol);
+              tma_load_2d(b + kBBytes / 2, &tmB, bar, kb * BK, brow + p.I, pol);
+            } else {  // MN-major weights: K rows of expert e, 4 blocks of 64 output columns
+              const int32_t krow = t.e * p.b_rows + kb * BK;
+              for (int q = 0; q < 4; ++q)
+                tma_load_2d(b + q * 8192, &tmB, bar, t.n * BN + q * 64, krow, pol);
+            }
+          }
+          armed |= 1u << stage;
+          armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok)
+        for (int s = 0; s < STAGES; ++s)
+          if (armed & (1u << s)) mbar_drain(&ctl->full[s], (armed_parity >> s) & 1u, 100000000ull);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {  // ---------------- MMA issuer ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true, issued = false;
+      int32_t it = 0;
+      for (int32_t L = blockIdx.x; L < p.total_tiles && ok; L += gridDim.x, ++it) {
+        const Tile t = decode<kMode>(L, ts, off, E, p);
+        const int32_t nkb = kMode == kWGrad ? (off[t.e + 1] - off[t.e]) / BK : p.num_kb;
+        const int buf = it & 1;
+        if (!mbar_wait(&ctl->tempty[buf], ((it >> 1) & 1) ^ 1u, abort, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * BN;
+        for (int32_t kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&ctl->full[stage], phase, abort, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * kABytes);
+          const uint32_t b_addr = smem_u32(sB + stage * kBBytes);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = kAmn ? mn_desc(a_addr + kk * 2048) : kmajor_desc<128>(a_addr + kk * 32);
+            const uint64_t bd = kBmn ? mn_desc(b_addr + kk * 2048) : kmajor_desc<128>(b_addr + kk * 32);
+            umma_bf16(d_tmem, ad, bd, idesc(kAmn, kBmn), (kb | kk) != 0);
+          }
+          issued = true;
+          umma_commit(&ctl->empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&ctl->tfull[buf]);
+      }
+      if (!ok && issued) {
+        umma_commit(&ctl->drain);
+        mbar_drain(&ctl->drain, 0, 100000000ull);
+      }
+    }
+  } else {  // ---------------- epilogue (warps 2..5) ----------------
+    const int q = warp & 3;
+    const int r = q * 32 + lane;  // accumulator row (TMEM lane)
+    int32_t it = 0;
+    for (int32_t L = blockIdx.x; L < p.total_tiles; L += gridDim.x, ++it) {
+      const int buf = it & 1;
+      if (!mbar_wait(&ctl->tfull[buf], (it >> 1) & 1, abort, p.status)) break;
+      tc_fence_after();
+      const Tile t = decode<kMode>(L, ts, off, E, p);
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * BN;
+      if (kMode == kWGrad) {
+        const int32_t m = t.m * BM + r;
+        float* dst = p.acc + ((int64_t)t.e * p.M + m) * p.N;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld_32cols(t_row + c * 32, v);
+          tmem_ld_wait(v);
+          const int32_t col0 = t.n * BN + c * 32;
+          if (m < p.M) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              if (col0 + 4 * i < p.N) {
+                float4* d4 = reinterpret_cast<float4*>(dst + col0 + 4 * i);
+                float4 o = *d4;
+                o.x += __uint_as_float(v[4 * i]);
+                o.y += __uint_as_float(v[4 * i + 1]);
+                o.z += __uint_as_float(v[4 * i + 2]);
+                o.w += __uint_as_float(v[4 * i + 3]);
+                *d4 = o;
+              }
+            }
+          }
+        }
+      } else {
+        const int32_t rows_valid = off[t.e + 1] - off[t.e] - t.m * BM;
+        const bool row_ok = r < rows_valid;
+        const int64_t row = (int64_t)off[t.e] + t.m * BM + r;
+        if (kMode == kRawGU) {
+#pragma unroll 1
+          for (int c = 0; c < (BN / 2) / 32; ++c) {
+            uint32_t g[32], u[32];
+            tmem_ld_32cols(t_row + c * 32, g);
+            tmem_ld_32cols(t_row + BN / 2 + c * 32, u);
+            tmem_ld_wait2(g, u);
+            const int32_t col0 = t.n * (BN / 2) + c * 32;
+            if (row_ok) {
+              uint32_t pg[16], pu[16], ph[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+                const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+                pg[i] = pack_bf16x2(g0, g1);
+                pu[i] = pack_bf16x2(u0, u1);
+                ph[i] = pack_bf16x2(silu_f(g0) * u0, silu_f(g1) * u1);
+              }
+              __nv_bfloat16* gu = p.out0 + row * 2 * p.I;
+              __nv_bfloat16* act = p.out1 + row * p.I;
+#pragma unroll
+              for (int v4 = 0; v4 < 4; ++v4) {
+                if (col0 + v4 * 8 < p.I) {
+                  const int32_t cc = col0 + v4 * 8;
+                  *reinterpret_cast<uint4*>(gu + cc) =
+                      make_uint4(pg[4 * v4], pg[4 * v4 + 1], pg[4 * v4 + 2], pg[4 * v4 + 3]);
+                  *reinterpret_cast<uint4*>(gu + p.I + cc) =
+                      make_uint4(pu[4 * v4], pu[4 * v4 + 1], pu[4 * v4 + 2], pu[4 * v4 + 3]);
+                  *reinterpret_cast<uint4*>(act + cc) =
+                      make_uint4(ph[4 * v4], ph[4 * v4 + 1], ph[4 * v4 + 2], ph[4 * v4 + 3]);
+                }
+              }
+            }
+          }
+        } else {
+#pragma unroll 1
+          for (int c = 0; c < BN / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld_32cols(t_row + c * 32, v);
+            tmem_ld_wait(v);
+            const int32_t col0 = t.n * BN + c * 32;
+            if (!row_ok) continue;
+            if (kMode == kDSwiGLU) {
+              const __nv_bfloat16* gu = p.aux + row * 2 * p.I;
+              __nv_bfloat16* dgu = p.out0 + row * 2 * p.I;
+#pragma unroll
+              for (int v4 = 0; v4 < 4; ++v4) {
+                const int32_t cc = col0 + v4 * 8;
+                if (cc >= p.I) continue;
+                const uint4 gq = *reinterpret_cast<const uint4*>(gu + cc);
+                const uint4 uq = *reinterpret_cast<const uint4*>(gu + p.I + cc);
+                const uint32_t ga[4] = {gq.x, gq.y, gq.z, gq.w};
+                const uint32_t ua[4] = {uq.x, uq.y, uq.z, uq.w};
+                uint32_t dg[4], du[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  float dgv[2], duv[2];
+#pragma unroll
+                  for (int h = 0; h < 2; ++h) {
+                    const float gv = h ? bf16hi(ga[i]) : bf16lo(ga[i]);
+                    const float uv = h ? bf16hi(ua[i]) : bf16lo(ua[i]);
+                    const float dh = __uint_as_float(v[v4 * 8 + 2 * i + h]);
+                    const float sig = 1.0f / (1.0f + __expf(-gv));
+                    duv[h] = dh * gv * sig;
+                    dgv[h] = dh * uv * (sig + gv * sig * (1.0f - sig));
+                  }
+                  dg[i] = pack_bf16x2(dgv[0], dgv[1]);
+                  du[i] = pack_bf16x2(duv[0], duv[1]);
+                }
+                *reinterpret_cast<uint4*>(dgu + cc) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
+                *reinterpret_cast<uint4*>(dgu + p.I + cc) = make_uint4(du[0], du[1], du[2], du[3]);
+              }
+            } else {  // kDPlain
+              __nv_bfloat16* o = p.out0 + row * p.N;
+#pragma unroll
+              for (int v4 = 0; v4 < 4; ++v4) {
+                const int32_t cc = col0 + v4 * 8;
+                if (cc >= p.N) continue;
+                uint32_t pk[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                  pk[i] = pack_bf16x2(__uint_as_float(v[v4 * 8 + 2 * i]),
+                                      __uint_as_float(v[v4 * 8 + 2 * i + 1]));
+                *reinterpret_cast<uint4*>(o + cc) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&ctl->tempty[buf]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ---- row kernels ----------------------------------------------------------------------
+
+constexpr int kRowThreads = 256;
+constexpr int kTokPerCta = kRowThreads / 32;
+
+// Padded expert offsets of every chunk: offp[c][e] = sum_{e' < e} roundup(counts[c][e'], 64).
+__global__ void pad_offsets_kernel(const int32_t* counts, int32_t E, int32_t* offp) {
+  if (threadIdx.x != 0) return;
+  const int32_t c = blockIdx.x;
+  int32_t run = 0;
+  for (int32_t e = 0; e < E; ++e) {
+    offp[(int64_t)c * (E + 1) + e] = run;
+    run += (counts[(int64_t)c * E + e] + kPadRows - 1) / kPadRows * kPadRows;
+  }
+  offp[(int64_t)c * (E + 1) + E] = run;
+}
+
+// Padded row of each copy of one chunk: dstp = dst - off[e] + offp[e].
+__global__ void pad_rows_kernel(const int32_t* idx, const int32_t* dst, const int32_t* off,
+                                const int32_t* offp, int64_t n, int32_t* dstp) {
+  const int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (s >= n) return;
+  const int32_t e = idx[s];
+  dstp[s] = dst[s] - off[e] + offp[e];
+}
+
+// dY[dstp(t,j)] = bf16(w[t][j] * dout[t]) and d_w[t][j] = <dout[t], Y[dstp(t,j)]> (fp32,
+// warp tree reduction in a fixed order): one warp per token.
+__global__ void __launch_bounds__(kRowThreads)
+    dy_dw_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ Y,
+                 const int32_t* __restrict__ dstp, const float* __restrict__ w, int64_t Tc,
+                 int32_t H8, int32_t k, uint4* __restrict__ dY, float* __restrict__ dw) {
+  const int64_t t = (int64_t)blockIdx.x * kTokPerCta + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= Tc) return;
+  for (int j = 0; j < k; ++j) {
+    const int32_t d = dstp[t * k + j];
+    const float wj = w[t * k + j];
+    float dot = 0.f;
+    for (int32_t v = lane; v < H8; v += 32) {
+      const uint4 g = dout[t * H8 + v];
+      const uint4 y = Y[(int64_t)d * H8 + v];
+      const uint32_t ga[4] = {g.x, g.y, g.z, g.w};
+      const uint32_t ya[4] = {y.x, y.y, y.z, y.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        dot = fmaf(bf16lo(ga[i]), bf16lo(ya[i]), dot);
+        dot = fmaf(bf16hi(ga[i]), bf16hi(ya[i]), dot);
+        o[i] = pack_bf16x2(wj * bf16lo(ga[i]), wj * bf16hi(ga[i]));
+      }
+      dY[(int64_t)d * H8 + v] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+#pragma unroll
+    for (int sh = 16; sh > 0; sh >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, sh);
+    if (lane == 0) dw[t * k + j] = dot;
+  }
+}
+
+// d_hidden[t] = bf16( sum_{j<k} dX[dstp(t,j)] ), fp32 in ascending j.
+__global__ void __launch_bounds__(kRowThreads)
+    sum_rows_kernel(const uint4* __restrict__ dX, const int32_t* __restrict__ dstp, int64_t Tc,
+                    int32_t H8, int32_t k, uint4* __restrict__ out) {
+  const int64_t t = (int64_t)blockIdx.x * kTokPerCta + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= Tc) return;
+  for (int32_t v = lane; v < H8; v += 32) {
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int j = 0; j < k; ++j) {
+      const uint4 x = dX[(int64_t)dstp[t * k + j] * H8 + v];
+      const uint32_t xa[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[2 * i] += bf16lo(xa[i]);
+        acc[2 * i + 1] += bf16hi(xa[i]);
+      }
+    }
+    out[t * H8 + v] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                                 pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+  }
+}
+
+template <int kMode>
+cudaError_t launch_mode(const CUtensorMap& mA, const CUtensorMap& mB, const BParams& p,
+                        int num_sms, cudaStream_t s) {
+  if (p.total_tiles <= 0) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(bwd_gemm_kernel<kMode>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
+  if (e != cudaSuccess) return e;
+  const int grid = p.total_tiles < num_sms ? p.total_tiles : num_sms;
+  bwd_gemm_kernel<kMode><<<grid, kThreads, kSmem, s>>>(mA, mB, p);
+  return cudaGetLastError();
+}
+
+inline unsigned row_grid(int64_t Tc) { return (unsigned)((Tc + kTokPerCta - 1) / kTokPerCta); }
+
+}  // namespace
+
+int bwd_pad_rows() { return kPadRows; }
+
+cudaError_t launch_bwd_gemm(const BwdGemmArgs& a, int num_sms, cudaStream_t s) {
+  if (a.E > kMaxE) return cudaErrorInvalidValue;
+  // host tile count from the padded per-expert rows
+  int64_t tiles = 0;
+  // N tiles: kRawGU pairs 128 gate with 128 up columns per tile; the others are 256 wide
+  const int32_t n_tiles = a.mode == kRawGU ? (a.I + BN / 2 - 1) / (BN / 2) : (a.N + BN - 1) / BN;
+  for (int32_t e = 0; e < a.E; ++e) {
+    const int64_t rows = a.rows_pad_host[e];
+    if (a.mode == kWGrad) tiles += rows > 0 ? (int64_t)((a.M + BM - 1) / BM) * n_tiles : 0;
+    else tiles += (rows + BM - 1) / BM * n_tiles;
+  }
+  if (tiles <= 0) return cudaSuccess;
+  if (tiles > 0x7fffffff) return cudaErrorInvalidValue;
+  CUtensorMap mA, mB;
+  const bool a_mn = a.mode == kWGrad;
+  const bool b_mn = a.mode != kRawGU;
+  if (!make_tma_2d_bf16(&mA, a.A, a.A_rows, a.A_cols, a_mn ? BK : BM) ||
+      !make_tma_2d_bf16(&mB, a.B, a.B_rows, a.B_cols, b_mn ? BK : BN / 2))
+    return cudaErrorInvalidValue;
+  BParams p;
+  p.offsets = a.offsets;
+  p.status = a.status;
+  p.E = a.E;
+  p.m_tiles = (a.M + BM - 1) / BM;
+  p.n_tiles = n_tiles;
+  p.num_kb = (a.K + BK - 1) / BK;
+  p.M = a.M;
+  p.N = a.N;
+  p.I = a.I;
+  p.b_rows = a.b_rows;
+  p.total_tiles = (int32_t)tiles;
+  p.out0 = static_cast<__nv_bfloat16*>(a.out0);
+  p.out1 = static_cast<__nv_bfloat16*>(a.out1);
+  p.aux = static_cast<const __nv_bfloat16*>(a.aux);
+  p.acc = a.acc;
+  switch (a.mode) {
+    case kRawGU: return launch_mode<kRawGU>(mA, mB, p, num_sms, s);
+    case kDSwiGLU: return launch_mode<kDSwiGLU>(mA, mB, p, num_sms, s);
+    case kDPlain: return launch_mode<kDPlain>(mA, mB, p, num_sms, s);
+    case kWGrad: return launch_mode<kWGrad>(mA, mB, p, num_sms, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_pad_offsets(const int32_t* counts, int32_t E, int32_t n_chunks, int32_t* offp,
+                               cudaStream_t s) {
+  pad_offsets_kernel<<<n_chunks, 32, 0, s>>>(counts, E, offp);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pad_rows(const int32_t* idx, const int32_t* dst, const int32_t* off,
+                            const int32_t* offp, int64_t n, int32_t* dstp, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  pad_rows_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(idx, dst, off, offp, n, dstp);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dy_dw(const void* dout, const void* Y, const int32_t* dstp, const float* w,
+                         int64_t Tc, int32_t H, int32_t k, void* dY, float* dw, cudaStream_t s) {
+  if (Tc <= 0) return cudaSuccess;
+  dy_dw_kernel<<<row_grid(Tc), kRowThreads, 0, s>>>(
+      static_cast<const uint4*>(dout), static_cast<const uint4*>(Y), dstp, w, Tc, H / 8, k,
+      static_cast<uint4*>(dY), dw);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sum_rows(const void* dX, const int32_t* dstp, int64_t Tc, int32_t H, int32_t k,
+                            void* out, cudaStream_t s) {
+  if (Tc <= 0) return cudaSuccess;
+  sum_rows_kernel<<<row_grid(Tc), kRowThreads, 0, s>>>(static_cast<const uint4*>(dX), dstp, Tc,
+                                                       H / 8, k, static_cast<uint4*>(out));
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -622,6 +622,11 @@ bool make_map_gateup4d(CUtensorMap* m, const void* base, int32_t E, int32_t I, i
 
 }  // namespace
 
+bool make_tma_2d_bf16(CUtensorMap* m, const void* base, int64_t rows, int32_t cols,
+                      int32_t box_rows) {
+  return make_map(m, base, rows, cols, box_rows);
+}
+
 bool gemm_supports_gather() { return MOE_GEMM_2SM == 0; }
 
 int64_t gemm_total_tiles(const int32_t* counts_host, int32_t E, int32_t out_cols, bool swiglu) {

@@ -68,6 +68,11 @@ struct GemmArgs {
   bool reverse = false;  // walk the tiles (and so the experts) in descending order
 };
 
+// 2-D bf16 tensor map over a row-major [rows][cols] matrix: boxes of box_rows x 64 columns,
+// 128-byte swizzle, zero fill outside the matrix.
+bool make_tma_2d_bf16(CUtensorMap* m, const void* base, int64_t rows, int32_t cols,
+                      int32_t box_rows);
+
 // True when the build's grouped GEMM supports a gathered A operand.
 bool gemm_supports_gather();
 
@@ -76,5 +81,43 @@ int64_t gemm_total_tiles(const int32_t* counts_host, int32_t E, int32_t out_cols
 
 cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cudaStream_t s,
                                 int* err_detail);
+
+// ---- backward (backward.cu) ------------------------------------------------------------
+
+enum BwdGemmMode { kBwdRawGU = 0, kBwdDSwiGLU = 1, kBwdDPlain = 2, kBwdWGrad = 3 };
+
+struct BwdGemmArgs {
+  int mode;                    // BwdGemmMode
+  const void* A;               // bf16 [A_rows][A_cols]
+  int64_t A_rows;
+  int32_t A_cols;
+  const void* B;               // bf16 [B_rows][B_cols]
+  int64_t B_rows;
+  int32_t B_cols;
+  const int32_t* offsets;      // dev [E+1] padded expert row offsets
+  const int32_t* rows_pad_host;  // host [E] padded rows per expert
+  int32_t E;
+  int32_t M;                   // kBwdWGrad: gradient rows
+  int32_t N;                   // output columns
+  int32_t K;                   // row-grouped modes: reduction length
+  int32_t I;                   // gate/up split of 2I-wide tensors
+  int32_t b_rows;              // rows of one expert's weight matrix in B
+  void* out0;
+  void* out1;
+  const void* aux;
+  float* acc;
+  uint32_t* status;
+};
+
+int bwd_pad_rows();
+cudaError_t launch_bwd_gemm(const BwdGemmArgs& a, int num_sms, cudaStream_t s);
+cudaError_t launch_pad_offsets(const int32_t* counts, int32_t E, int32_t n_chunks, int32_t* offp,
+                               cudaStream_t s);
+cudaError_t launch_pad_rows(const int32_t* idx, const int32_t* dst, const int32_t* off,
+                            const int32_t* offp, int64_t n, int32_t* dstp, cudaStream_t s);
+cudaError_t launch_dy_dw(const void* dout, const void* Y, const int32_t* dstp, const float* w,
+                         int64_t Tc, int32_t H, int32_t k, void* dY, float* dw, cudaStream_t s);
+cudaError_t launch_sum_rows(const void* dX, const int32_t* dstp, int64_t Tc, int32_t H, int32_t k,
+                            void* out, cudaStream_t s);
 
 }  // namespace moe

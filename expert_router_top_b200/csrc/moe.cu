@@ -775,6 +775,177 @@ moe_status_t moe_forward_host(const moe_shape_t* shape, const void* hidden_host,
   return MOE_OK;
 }
 
+// ---- backward -------------------------------------------------------------------------
+
+namespace {
+
+struct BwdLayout {
+  Layout meta;  // metadata regions (status/counts/splits, offsets, histograms, dst, src)
+  size_t offp, dstp, xp, gu, act, ydx, dy, dgu, total;
+  int64_t rows_cap;
+};
+
+BwdLayout make_bwd_layout(const Dims& d, int32_t H, int32_t I) {
+  BwdLayout B{};
+  B.meta = make_layout(d, 8, 8, false, true, true);
+  size_t o = B.meta.total;
+  B.rows_cap = d.t_chunk * d.k + (int64_t)d.E * (bwd_pad_rows() - 1);
+  B.offp = o;
+  o += al(sizeof(int32_t) * (size_t)d.n * (d.E + 1));
+  B.dstp = o;
+  o += al(sizeof(int32_t) * (size_t)(d.T * d.k));
+  const size_t R = (size_t)B.rows_cap;
+  B.xp = o;
+  o += al(2 * R * H);
+  B.gu = o;
+  o += al(2 * R * 2 * I);
+  B.act = o;
+  o += al(2 * R * I);
+  B.ydx = o;  // recomputed Y rows, later dX rows
+  o += al(2 * R * H);
+  B.dy = o;
+  o += al(2 * R * H);
+  B.dgu = o;
+  o += al(2 * R * 2 * I);
+  B.total = o;
+  return B;
+}
+
+moe_status_t check_bwd_shape(const moe_shape_t* s) {
+  moe_status_t st = check_shape(s);
+  if (st != MOE_OK) return st;
+  if (s->H % 64 != 0 || s->I % 32 != 0) return MOE_ERR_ARG;
+  return MOE_OK;
+}
+
+}  // namespace
+
+size_t moe_backward_workspace_bytes(const moe_shape_t* s) {
+  if (check_bwd_shape(s) != MOE_OK) return 0;
+  const Dims d = make_dims(s->T, s->k, s->E, s->ep_groups, s->num_chunks, s->chunk_size);
+  return make_bwd_layout(d, s->H, s->I).total;
+}
+
+moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
+                          const int32_t* top_k_index, const float* top_k_weights,
+                          const void* W_gate_up, const void* W_down, const void* d_out,
+                          void* d_hidden, float* d_weights, float* dW_gate_up, float* dW_down,
+                          void* workspace, size_t ws_bytes, void* stream) {
+  moe_status_t st = check_bwd_shape(shape);
+  if (st != MOE_OK) return st;
+  const int64_t T = shape->T;
+  const int32_t H = shape->H, I = shape->I, E = shape->E, k = shape->k;
+  if (!W_gate_up || !W_down || !dW_gate_up || !dW_down) return MOE_ERR_ARG;
+  if (T > 0 && (!hidden || !top_k_index || !top_k_weights || !d_out || !d_hidden ||
+                !d_weights || !workspace))
+    return MOE_ERR_ARG;
+  if (!aligned(hidden, 16) || !aligned(d_out, 16) || !aligned(d_hidden, 16) ||
+      !aligned(W_gate_up, 16) || !aligned(W_down, 16) || !aligned(dW_gate_up, 16) ||
+      !aligned(dW_down, 16) || !aligned(top_k_index, 4) || !aligned(top_k_weights, 4) ||
+      !aligned(d_weights, 4) || !aligned(workspace, kAlign))
+    return MOE_ERR_ALIGN;
+  const Dims d = make_dims(T, k, E, shape->ep_groups, shape->num_chunks, shape->chunk_size);
+  const BwdLayout B = make_bwd_layout(d, H, I);
+  if (T > 0 && ws_bytes < B.total) return MOE_ERR_WORKSPACE;
+  DeviceCtx* ctx = nullptr;
+  if ((st = get_ctx(&ctx)) != MOE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the weight gradients are sums over all chunks: start from zero
+  if (cudaMemsetAsync(dW_gate_up, 0, sizeof(float) * (size_t)E * 2 * I * H, s) != cudaSuccess ||
+      cudaMemsetAsync(dW_down, 0, sizeof(float) * (size_t)E * H * I, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (T == 0) return MOE_OK;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* dst = reinterpret_cast<int32_t*>(ws + B.meta.dst);
+  int32_t* src = reinterpret_cast<int32_t*>(ws + B.meta.src);
+  uint32_t* dev_status = reinterpret_cast<uint32_t*>(ws + B.meta.packed);
+  if ((st = run_metadata(d, top_k_index, ws, B.meta, dst, src, s)) != MOE_OK) return st;
+  if ((st = fetch_packed(ctx, ws, B.meta, s)) != MOE_OK) return st;
+  std::vector<int32_t> counts(ctx->host_stage + kStatusWords,
+                              ctx->host_stage + kStatusWords + (size_t)d.n * d.E);
+  const int32_t* counts_dev = reinterpret_cast<const int32_t*>(ws + B.meta.packed) + kStatusWords;
+  int32_t* offp = reinterpret_cast<int32_t*>(ws + B.offp);
+  int32_t* dstp = reinterpret_cast<int32_t*>(ws + B.dstp);
+  if (launch_pad_offsets(counts_dev, E, d.n, offp, s) != cudaSuccess) return MOE_ERR_CUDA;
+  const std::vector<int64_t> bounds = dims_bounds(d);
+  const int pad = bwd_pad_rows();
+  const uint16_t* hid = static_cast<const uint16_t*>(hidden);
+  const uint16_t* dout = static_cast<const uint16_t*>(d_out);
+  uint16_t* dx_out = static_cast<uint16_t*>(d_hidden);
+  std::vector<int32_t> rows_pad((size_t)E);
+  for (int c = 0; c < d.n; ++c) {
+    const int64_t t0 = bounds[c], len = bounds[c + 1] - bounds[c];
+    if (len == 0) continue;
+    const int32_t* cnt = counts.data() + (size_t)c * E;
+    int64_t R = 0;
+    for (int32_t e = 0; e < E; ++e) {
+      rows_pad[e] = (cnt[e] + pad - 1) / pad * pad;
+      R += rows_pad[e];
+    }
+    const int32_t* off_c = reinterpret_cast<const int32_t*>(ws + B.meta.offsets) + (size_t)c * (E + 1);
+    const int32_t* offp_c = offp + (size_t)c * (E + 1);
+    int32_t* dstp_c = dstp + t0 * k;
+    void* xp = ws + B.xp;
+    void* gu = ws + B.gu;
+    void* act = ws + B.act;
+    void* ydx = ws + B.ydx;
+    void* dy = ws + B.dy;
+    void* dgu = ws + B.dgu;
+    // zero the padded row buffers that seed every pad row (X and dY)
+    if (cudaMemsetAsync(xp, 0, 2 * (size_t)R * H, s) != cudaSuccess ||
+        cudaMemsetAsync(dy, 0, 2 * (size_t)R * H, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (launch_pad_rows(top_k_index + t0 * k, dst + t0 * k, off_c, offp_c, len * k, dstp_c, s) !=
+            cudaSuccess ||
+        launch_permute(hid + t0 * H, dstp_c, len, H, k, xp, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    BwdGemmArgs g{};
+    g.offsets = offp_c;
+    g.rows_pad_host = rows_pad.data();
+    g.E = E;
+    g.I = I;
+    g.status = dev_status;
+    // recompute g, u, h
+    g.mode = kBwdRawGU;
+    g.A = xp, g.A_rows = R, g.A_cols = H;
+    g.B = W_gate_up, g.B_rows = (int64_t)E * 2 * I, g.B_cols = H;
+    g.N = 2 * I, g.K = H, g.b_rows = 2 * I, g.out0 = gu, g.out1 = act;
+    if (launch_bwd_gemm(g, ctx->num_sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    // recompute Y = h W_down^T (the forward down GEMM on the padded rows)
+    if ((st = gemm_call(act, R, W_down, ydx, offp_c, rows_pad.data(), E, I, H, H, false,
+                        dev_status, ctx->num_sms, s)) != MOE_OK)
+      return st;
+    if (launch_dy_dw(dout + t0 * H, ydx, dstp_c, top_k_weights + t0 * k, len, H, k, dy,
+                     d_weights + t0 * k, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    // dh = dY W_down, SwiGLU backward in the epilogue -> [dg du]
+    g.mode = kBwdDSwiGLU;
+    g.A = dy, g.A_rows = R, g.A_cols = H;
+    g.B = W_down, g.B_rows = (int64_t)E * H, g.B_cols = I;
+    g.N = I, g.K = H, g.b_rows = H, g.out0 = dgu, g.out1 = nullptr, g.aux = gu;
+    if (launch_bwd_gemm(g, ctx->num_sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    // dX = [dg du] W_gate_up
+    g.mode = kBwdDPlain;
+    g.A = dgu, g.A_rows = R, g.A_cols = 2 * I;
+    g.B = W_gate_up, g.B_rows = (int64_t)E * 2 * I, g.B_cols = H;
+    g.N = H, g.K = 2 * I, g.b_rows = 2 * I, g.out0 = ydx, g.aux = nullptr;
+    if (launch_bwd_gemm(g, ctx->num_sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_sum_rows(ydx, dstp_c, len, H, k, dx_out + t0 * H, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    // dW_down[e] += dY^T h ;  dW_gate_up[e] += [dg du]^T X
+    g.mode = kBwdWGrad;
+    g.A = dy, g.A_rows = R, g.A_cols = H;
+    g.B = act, g.B_rows = R, g.B_cols = I;
+    g.M = H, g.N = I, g.acc = dW_down, g.out0 = nullptr;
+    if (launch_bwd_gemm(g, ctx->num_sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    g.A = dgu, g.A_rows = R, g.A_cols = 2 * I;
+    g.B = xp, g.B_rows = R, g.B_cols = H;
+    g.M = 2 * I, g.N = H, g.acc = dW_gate_up;
+    if (launch_bwd_gemm(g, ctx->num_sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
 moe_status_t moe_check_device_status(const void* workspace, size_t ws_bytes, void* stream) {
   if (!workspace || ws_bytes < sizeof(uint32_t)) return MOE_ERR_ARG;
   uint32_t st = 0;

@@ -267,6 +267,32 @@ MOE_API moe_status_t moe_forward_host(const moe_shape_t* shape, const void* hidd
                                       const void* W_down, void* out_host, void* workspace,
                                       size_t ws_bytes, void* stream);
 
+/* Device workspace, in bytes, that moe_backward needs for this shape; 0 if the shape is
+ * invalid for it (moe_backward also needs H % 64 == 0 and I % 32 == 0). */
+MOE_API size_t moe_backward_workspace_bytes(const moe_shape_t* shape);
+
+/* Backward pass of moe_forward, chunk by chunk, with the expert computation recomputed
+ * from `hidden` (the recompute setting of [ChunkMoE] "操作指南"; the backward mirrors the
+ * forward chunking, "一张专业时序图").  For the loss sum(out * d_out):
+ *   d_hidden [T][H] bf16          gradient of hidden (sum of the k copies' gradients, fp32
+ *                                 in ascending j, one rounding)
+ *   d_weights [T][k] fp32         d_weights[t][j] = <d_out[t], W_down[e] h(t,j)>
+ *   dW_gate_up [E][2I][H] fp32    gradient of W_gate_up (gate rows, then up rows)
+ *   dW_down [E][H][I] fp32        gradient of W_down
+ * All four outputs are overwritten.  Inputs as moe_forward plus d_out [T][H] bf16.  The
+ * intermediate g, u, h, Y, dY, dg, du and dX rows are bf16 (fp32 accumulation in every GEMM
+ * and reduction); each expert's rows are padded to a multiple of 64 inside the workspace.
+ * d_hidden and d_weights are bit-identical for every chunking; dW_* are sums over chunks
+ * in chunk order (fp32), equal up to rounding.  workspace: dev, >=
+ * moe_backward_workspace_bytes(shape).  The host blocks once, on the metadata copy.
+ * Errors: as moe_forward; MOE_ERR_ARG also for H % 64 or I % 32 != 0. */
+MOE_API moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
+                                  const int32_t* top_k_index, const float* top_k_weights,
+                                  const void* W_gate_up, const void* W_down, const void* d_out,
+                                  void* d_hidden, float* d_weights, float* dW_gate_up,
+                                  float* dW_down, void* workspace, size_t ws_bytes,
+                                  void* stream);
+
 /* Synchronizes `stream` and returns MOE_ERR_TIMEOUT if a kernel of an earlier call that
  * used this workspace gave up a bounded wait, MOE_ERR_INDEX if its last metadata pass
  * saw a bad index, else MOE_OK (or MOE_ERR_CUDA). */

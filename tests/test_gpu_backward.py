@@ -1,0 +1,75 @@
+"""Backward pass (expert computation recomputed per chunk) against the fp64 oracle.
+
+Tolerances: d_hidden is a bf16 output built from bf16 intermediates (the layer's bar:
+relative Frobenius <= 1e-2, |err| <= 3e-2 + 2e-2 |ref|).  d_weights, dW_gate_up and dW_down
+are fp32 sums of products of bf16-rounded intermediates: each term carries a relative error
+of ~2^-8, and the terms of the weight gradients are heavy-tailed (dg = dh u silu'(g) is a
+product of three roughly Gaussian factors), so an entry whose few terms cancel keeps an
+absolute error of a few per cent of the gradient's RMS.  Bar: relative Frobenius <= 1e-2
+and |err| <= 2e-2 |ref| + 1e-1 rms(ref)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gen import CONFIGS, LayerConfig, bf16_normal, bits, layer_inputs
+from parity import assert_layer_close, rel_frobenius, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def assert_grad_close(got, ref, what):
+    got = got if isinstance(got, np.ndarray) else to_f64(got)
+    fro = rel_frobenius(got, ref)
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    worst = float((np.abs(got - ref) / (2e-2 * np.abs(ref) + 1e-1 * rms + 1e-30)).max())
+    assert fro <= 1e-2, f"{what}: relative Frobenius {fro:.3e}"
+    assert worst <= 1.0, f"{what}: elementwise bound exceeded ({worst:.3f})"
+    return fro
+
+
+MID = LayerConfig("mid", 300, 512, 16, 4, 384, "normal", chunks=(1, 3))
+
+
+def _run(moe, cfg, N=1, S=0):
+    cpu = layer_inputs(cfg)
+    dout = bf16_normal((cfg.T, cfg.H), 1.0, 99)
+    gpu = {k: v.cuda() for k, v in cpu.items()}
+    res = moe.backward(gpu["hidden"], gpu["idx"], gpu["w"], gpu["wgu"], gpu["wd"], dout.cuda(),
+                       num_chunks=N, ep_groups=cfg.G, chunk_size=S)
+    torch.cuda.synchronize()
+    return cpu, dout, res
+
+
+@pytest.mark.parametrize("cfg", [CONFIGS["tiny"], MID, CONFIGS["edge_varlen"]],
+                         ids=["tiny", "mid", "edge_varlen"])
+def test_backward_matches_oracle(moe, cfg):
+    cpu, dout, (dx, dw, dwgu, dwd) = _run(moe, cfg, N=cfg.chunks[-1])
+    rx, rw, rgu, rd = oracle.backward(bits(cpu["hidden"]), cpu["idx"].numpy(), cpu["w"].numpy(),
+                                      bits(cpu["wgu"]), bits(cpu["wd"]), bits(dout))
+    stats = dict(d_hidden=assert_layer_close(dx, rx, f"{cfg.name} d_hidden")["rel_fro"],
+                 d_weights=assert_grad_close(dw, rw, f"{cfg.name} d_weights"),
+                 dW_gate_up=assert_grad_close(dwgu, rgu, f"{cfg.name} dW_gate_up"),
+                 dW_down=assert_grad_close(dwd, rd, f"{cfg.name} dW_down"))
+    print(cfg.name, {k: f"{v:.2e}" for k, v in stats.items()})
+
+
+def test_backward_chunk_invariance(moe):
+    cfg = MID
+    _, _, base = _run(moe, cfg, N=1)
+    for N, S in ((2, 0), (3, 0), (7, 0), (0, 64)):
+        _, _, got = _run(moe, cfg, N=N, S=S)
+        assert torch.equal(got[0], base[0]), f"d_hidden differs at N={N} S={S}"
+        assert torch.equal(got[1], base[1]), f"d_weights differs at N={N} S={S}"
+        for a, b, name in ((got[2], base[2], "dW_gate_up"), (got[3], base[3], "dW_down")):
+            assert rel_frobenius(to_f64(a), to_f64(b)) < 1e-5, f"{name} at N={N} S={S}"
+
+
+def test_backward_zero_tokens(moe):
+    cfg = CONFIGS["tiny"]
+    gpu = {k: v.cuda() for k, v in layer_inputs(cfg).items()}
+    d = torch.zeros((0, cfg.H), dtype=torch.bfloat16, device="cuda")
+    dx, dw, dwgu, dwd = moe.backward(gpu["hidden"][:0], gpu["idx"][:0], gpu["w"][:0], gpu["wgu"],
+                                     gpu["wd"], d)
+    torch.cuda.synchronize()
+    assert dx.shape == (0, cfg.H) and not dwgu.any() and not dwd.any()
