@@ -24,7 +24,9 @@ MOE_OK = 0
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_ARG", 2: "MOE_ERR_INDEX", 3: "MOE_ERR_ALIGN",
                 4: "MOE_ERR_WORKSPACE", 5: "MOE_ERR_CUDA", 6: "MOE_ERR_TIMEOUT",
                 7: "MOE_ERR_UNSUPPORTED"}
-KERNEL_KINDS = ("metadata", "permute", "gateup", "down", "unpermute")
+KERNEL_KINDS = ("metadata", "permute", "gateup", "down", "unpermute", "bwd_gateup", "bwd_dswiglu",
+                "bwd_dx", "bwd_wgrad", "bwd_rows")
+_NK = len(KERNEL_KINDS)  # MOE_KERNEL_KINDS
 
 
 class MoEError(RuntimeError):
@@ -40,8 +42,8 @@ class Shape(ctypes.Structure):
 
 
 class Profile(ctypes.Structure):
-    _fields_ = [("launches", ctypes.c_int64 * 5), ("ms", ctypes.c_double * 5),
-                ("rows", ctypes.c_int64 * 5), ("active_experts", ctypes.c_int64 * 5),
+    _fields_ = [("launches", ctypes.c_int64 * _NK), ("ms", ctypes.c_double * _NK),
+                ("rows", ctypes.c_int64 * _NK), ("active_experts", ctypes.c_int64 * _NK),
                 ("kernels", ctypes.c_int64)]
 
 

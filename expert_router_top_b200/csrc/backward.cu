@@ -20,7 +20,8 @@
 //   kRawGU    [g u] = X W_gate_up^T           A rows K-major, B K-major   epilogue: g, u, h
 //   kDSwiGLU  dh = dY W_down                  B MN-major                  epilogue: dg, du
 //   kDPlain   dX = [dg du] W_gate_up          B MN-major                  epilogue: bf16 store
-//   kWGrad    dW[e] += S_A[e]^T S_B[e]        A and B MN-major, K = rows  epilogue: fp32 +=
+//   kWGrad    dW[e] += S_A[e]^T S_B[e]        A and B MN-major, K = rows  epilogue: TMA fp32
+//                                                                        store / add-reduce
 // MN-major operands use the 128-byte-swizzled MN-major canonical layout: 64-element MN
 // blocks of 64 K rows x 128 B (8 KB apart: the leading byte offset), 8-row K groups 1 KB
 // apart (the stride byte offset); one MMA K step of 16 advances 2 KB.
@@ -59,7 +60,9 @@ struct BParams {
   __nv_bfloat16* out0;      // kRawGU: GU [rows][2I]; kDSwiGLU: dGU [rows][2I]; kDPlain: [rows][N]
   __nv_bfloat16* out1;      // kRawGU: Act [rows][I]
   const __nv_bfloat16* aux; // kDSwiGLU: GU [rows][2I]
-  float* acc;               // kWGrad: [E][M][N] fp32, accumulated into
+  float* acc;               // kWGrad: [E][M][N] fp32 (written through tmC)
+  const int32_t* first;     // kWGrad: [E] first chunk with rows of each expert
+  int32_t chunk;            // kWGrad: this chunk
 };
 
 struct Ctl {
@@ -69,7 +72,12 @@ struct Ctl {
 };
 constexpr size_t kCtlBytes = 256;
 static_assert(sizeof(Ctl) <= kCtlBytes, "control block");
-constexpr size_t kSmem = 1024 + STAGES * kStageBytes + kCtlBytes + 2 * (kMaxE + 1) * 4;
+// kWGrad output staging: one 32 x 32 fp32 box (4 KB, 128-byte swizzled) per epilogue warp
+constexpr uint32_t kOutBoxBytes = 32 * 32 * 4;
+constexpr uint32_t kOutBytes = 4 * kOutBoxBytes;
+constexpr size_t kSmem =
+    1024 + STAGES * kStageBytes + kOutBytes + kCtlBytes + 2 * (kMaxE + 1) * 4;
+static_assert(kSmem <= 232448, "shared memory per CTA");
 
 __host__ __device__ constexpr uint32_t idesc(bool a_mn, bool b_mn) {
   return umma_idesc_bf16_f32(BM, BN) | (a_mn ? 1u << 15 : 0u) | (b_mn ? 1u << 16 : 0u);
@@ -114,7 +122,8 @@ __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)
 template <int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                    const __grid_constant__ CUtensorMap tmB, const BParams p) {
+                    const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmC, const BParams p) {
   constexpr bool kAmn = kMode == kWGrad;
   constexpr bool kBmn = kMode != kRawGU;
   extern __shared__ uint8_t smem_raw[];
@@ -122,8 +131,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * kABytes;
-  Ctl* ctl = reinterpret_cast<Ctl*>(smem + STAGES * kStageBytes);
-  int32_t* off = reinterpret_cast<int32_t*>(smem + STAGES * kStageBytes + kCtlBytes);
+  uint8_t* sOut = smem + STAGES * kStageBytes;  // 1024-byte aligned
+  Ctl* ctl = reinterpret_cast<Ctl*>(sOut + kOutBytes);
+  int32_t* off = reinterpret_cast<int32_t*>(sOut + kOutBytes + kCtlBytes);
   int32_t* ts = off + (kMaxE + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int32_t E = p.E;
@@ -276,32 +286,59 @@ __global__ void __launch_bounds__(kThreads, 1)
     int32_t it = 0;
     for (int32_t L = blockIdx.x; L < p.total_tiles; L += gridDim.x, ++it) {
       const int buf = it & 1;
+      const Tile t = decode<kMode>(L, ts, off, E, p);
+      // kDSwiGLU: the saved g and u of this thread's row, one 32-column block ahead of the
+      // accumulator; the first block is requested before the accumulator is ready
+      uint4 gq[4], uq[4];
+      const int32_t rows_here = off[t.e + 1] - off[t.e] - t.m * BM;
+      const int64_t row_g = (int64_t)off[t.e] + t.m * BM + r;
+      auto load_aux = [&](int c, uint4 (&g)[4], uint4 (&u)[4]) {
+        const uint4* gu4 = reinterpret_cast<const uint4*>(p.aux + row_g * 2 * p.I);
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4) {
+          const int32_t cc = t.n * BN + c * 32 + v4 * 8;
+          if (r < rows_here && cc < p.I) {
+            g[v4] = __ldg(gu4 + cc / 8);
+            u[v4] = __ldg(gu4 + (p.I + cc) / 8);
+          } else {
+            g[v4] = make_uint4(0, 0, 0, 0);
+            u[v4] = g[v4];
+          }
+        }
+      };
+      if (kMode == kDSwiGLU) load_aux(0, gq, uq);
       if (!mbar_wait(&ctl->tfull[buf], (it >> 1) & 1, abort, p.status)) break;
       tc_fence_after();
-      const Tile t = decode<kMode>(L, ts, off, E, p);
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * BN;
       if (kMode == kWGrad) {
-        const int32_t m = t.m * BM + r;
-        float* dst = p.acc + ((int64_t)t.e * p.M + m) * p.N;
+        // Each warp owns accumulator rows q*32..q*32+31: per 32-column block it stages the
+        // 32 x 32 fp32 block in shared memory (16-byte chunk i of row `lane` at i ^ (lane % 8),
+        // the 128-byte swizzle of the tensor map) and one lane stores it -- the expert's first
+        // chunk with rows -- or adds it into dW with one TMA reduction.  Each element of dW
+        // gets one store or add per chunk, in chunk order.
+        uint8_t* box = sOut + q * kOutBoxBytes;
+        const int32_t m0 = t.m * BM + q * 32;
+        const bool store = p.first[t.e] == p.chunk;
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t v[32];
           tmem_ld_32cols(t_row + c * 32, v);
+          if (lane == 0) bulk_wait_read_all();  // the previous box has left shared memory
+          __syncwarp();
           tmem_ld_wait(v);
-          const int32_t col0 = t.n * BN + c * 32;
-          if (m < p.M) {
+          float4* row4 = reinterpret_cast<float4*>(box + lane * 128);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              if (col0 + 4 * i < p.N) {
-                float4* d4 = reinterpret_cast<float4*>(dst + col0 + 4 * i);
-                float4 o = *d4;
-                o.x += __uint_as_float(v[4 * i]);
-                o.y += __uint_as_float(v[4 * i + 1]);
-                o.z += __uint_as_float(v[4 * i + 2]);
-                o.w += __uint_as_float(v[4 * i + 3]);
-                *d4 = o;
-              }
-            }
+          for (int i = 0; i < 8; ++i)
+            row4[i ^ (lane & 7)] =
+                make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                            __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+          fence_async_smem();
+          __syncwarp();
+          const int32_t col0 = t.n * BN + c * 32;
+          if (lane == 0 && m0 < p.M && col0 < p.N) {
+            if (store) tma_store_3d(&tmC, box, col0, m0, t.e);
+            else tma_reduce_add_3d(&tmC, box, col0, m0, t.e);
+            bulk_commit();
           }
         }
       } else {
@@ -347,20 +384,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < BN / 32; ++c) {
             uint32_t v[32];
             tmem_ld_32cols(t_row + c * 32, v);
+            uint4 gn[4], un[4];
+            if (kMode == kDSwiGLU && c + 1 < BN / 32) load_aux(c + 1, gn, un);
             tmem_ld_wait(v);
             const int32_t col0 = t.n * BN + c * 32;
             if (!row_ok) continue;
             if (kMode == kDSwiGLU) {
-              const __nv_bfloat16* gu = p.aux + row * 2 * p.I;
               __nv_bfloat16* dgu = p.out0 + row * 2 * p.I;
 #pragma unroll
               for (int v4 = 0; v4 < 4; ++v4) {
                 const int32_t cc = col0 + v4 * 8;
                 if (cc >= p.I) continue;
-                const uint4 gq = *reinterpret_cast<const uint4*>(gu + cc);
-                const uint4 uq = *reinterpret_cast<const uint4*>(gu + p.I + cc);
-                const uint32_t ga[4] = {gq.x, gq.y, gq.z, gq.w};
-                const uint32_t ua[4] = {uq.x, uq.y, uq.z, uq.w};
+                const uint32_t ga[4] = {gq[v4].x, gq[v4].y, gq[v4].z, gq[v4].w};
+                const uint32_t ua[4] = {uq[v4].x, uq[v4].y, uq[v4].z, uq[v4].w};
                 uint32_t dg[4], du[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
@@ -379,6 +415,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 *reinterpret_cast<uint4*>(dgu + cc) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
                 *reinterpret_cast<uint4*>(dgu + p.I + cc) = make_uint4(du[0], du[1], du[2], du[3]);
+              }
+#pragma unroll
+              for (int v4 = 0; v4 < 4; ++v4) {
+                gq[v4] = gn[v4];
+                uq[v4] = un[v4];
               }
             } else {  // kDPlain
               __nv_bfloat16* o = p.out0 + row * p.N;
@@ -400,6 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&ctl->tempty[buf]);
     }
+    if (kMode == kWGrad && lane == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -425,6 +467,16 @@ __global__ void pad_offsets_kernel(const int32_t* counts, int32_t E, int32_t* of
     run += (counts[(int64_t)c * E + e] + kPadRows - 1) / kPadRows * kPadRows;
   }
   offp[(int64_t)c * (E + 1) + E] = run;
+}
+
+// first[e] = the first chunk in which expert e has rows (n_chunks if none).
+__global__ void first_chunk_kernel(const int32_t* counts, int32_t E, int32_t n_chunks,
+                                   int32_t* first) {
+  const int32_t e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= E) return;
+  int32_t c = 0;
+  while (c < n_chunks && counts[(int64_t)c * E + e] == 0) ++c;
+  first[e] = c;
 }
 
 // Padded row of each copy of one chunk: dstp = dst - off[e] + offp[e].
@@ -493,14 +545,14 @@ __global__ void __launch_bounds__(kRowThreads)
 }
 
 template <int kMode>
-cudaError_t launch_mode(const CUtensorMap& mA, const CUtensorMap& mB, const BParams& p,
-                        int num_sms, cudaStream_t s) {
+cudaError_t launch_mode(const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mC,
+                        const BParams& p, int num_sms, cudaStream_t s) {
   if (p.total_tiles <= 0) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(bwd_gemm_kernel<kMode>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
   if (e != cudaSuccess) return e;
   const int grid = p.total_tiles < num_sms ? p.total_tiles : num_sms;
-  bwd_gemm_kernel<kMode><<<grid, kThreads, kSmem, s>>>(mA, mB, p);
+  bwd_gemm_kernel<kMode><<<grid, kThreads, kSmem, s>>>(mA, mB, mC, p);
   return cudaGetLastError();
 }
 
@@ -523,12 +575,18 @@ cudaError_t launch_bwd_gemm(const BwdGemmArgs& a, int num_sms, cudaStream_t s) {
   }
   if (tiles <= 0) return cudaSuccess;
   if (tiles > 0x7fffffff) return cudaErrorInvalidValue;
-  CUtensorMap mA, mB;
+  CUtensorMap mA, mB, mC;
   const bool a_mn = a.mode == kWGrad;
   const bool b_mn = a.mode != kRawGU;
   if (!make_tma_2d_bf16(&mA, a.A, a.A_rows, a.A_cols, a_mn ? BK : BM) ||
       !make_tma_2d_bf16(&mB, a.B, a.B_rows, a.B_cols, b_mn ? BK : BN / 2))
     return cudaErrorInvalidValue;
+  if (a.mode == kWGrad) {
+    if (!a.acc || !a.first || !make_tma_3d_f32(&mC, a.acc, a.E, a.M, a.N))
+      return cudaErrorInvalidValue;
+  } else {
+    mC = mA;  // unused
+  }
   BParams p;
   p.offsets = a.offsets;
   p.status = a.status;
@@ -545,18 +603,21 @@ cudaError_t launch_bwd_gemm(const BwdGemmArgs& a, int num_sms, cudaStream_t s) {
   p.out1 = static_cast<__nv_bfloat16*>(a.out1);
   p.aux = static_cast<const __nv_bfloat16*>(a.aux);
   p.acc = a.acc;
+  p.first = a.first;
+  p.chunk = a.chunk;
   switch (a.mode) {
-    case kRawGU: return launch_mode<kRawGU>(mA, mB, p, num_sms, s);
-    case kDSwiGLU: return launch_mode<kDSwiGLU>(mA, mB, p, num_sms, s);
-    case kDPlain: return launch_mode<kDPlain>(mA, mB, p, num_sms, s);
-    case kWGrad: return launch_mode<kWGrad>(mA, mB, p, num_sms, s);
+    case kRawGU: return launch_mode<kRawGU>(mA, mB, mC, p, num_sms, s);
+    case kDSwiGLU: return launch_mode<kDSwiGLU>(mA, mB, mC, p, num_sms, s);
+    case kDPlain: return launch_mode<kDPlain>(mA, mB, mC, p, num_sms, s);
+    case kWGrad: return launch_mode<kWGrad>(mA, mB, mC, p, num_sms, s);
   }
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_pad_offsets(const int32_t* counts, int32_t E, int32_t n_chunks, int32_t* offp,
-                               cudaStream_t s) {
+                               int32_t* first, cudaStream_t s) {
   pad_offsets_kernel<<<n_chunks, 32, 0, s>>>(counts, E, offp);
+  first_chunk_kernel<<<(E + 127) / 128, 128, 0, s>>>(counts, E, n_chunks, first);
   return cudaGetLastError();
 }
 

@@ -627,6 +627,18 @@ bool make_tma_2d_bf16(CUtensorMap* m, const void* base, int64_t rows, int32_t co
   return make_map(m, base, rows, cols, box_rows);
 }
 
+bool make_tma_3d_f32(CUtensorMap* m, void* base, int32_t E, int32_t M, int32_t N) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc || N % 4 != 0) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)M, (cuuint64_t)E};
+  const cuuint64_t strides[2] = {(cuuint64_t)N * 4, (cuuint64_t)M * N * 4};
+  const cuuint32_t box[3] = {32, 32, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool gemm_supports_gather() { return MOE_GEMM_2SM == 0; }
 
 int64_t gemm_total_tiles(const int32_t* counts_host, int32_t E, int32_t out_cols, bool swiglu) {

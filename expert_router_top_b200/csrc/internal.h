@@ -77,6 +77,9 @@ bool make_tma_2d_bf16(CUtensorMap* m, const void* base, int64_t rows, int32_t co
 bool gemm_supports_gather();
 
 // Number of 128-row x N-column output tiles for the given host counts.
+// 3-D fp32 tensor map over [E][M][N] (row-major per expert) with a 32 x 32 box and the
+// 128-byte swizzle: the target of the weight-gradient stores and add-reductions.
+bool make_tma_3d_f32(CUtensorMap* m, void* base, int32_t E, int32_t M, int32_t N);
 int64_t gemm_total_tiles(const int32_t* counts_host, int32_t E, int32_t out_cols, bool swiglu);
 
 cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cudaStream_t s,
@@ -105,14 +108,16 @@ struct BwdGemmArgs {
   void* out0;
   void* out1;
   const void* aux;
-  float* acc;
+  float* acc;                  // kBwdWGrad: [E][M][N] fp32 gradient
+  const int32_t* first;        // kBwdWGrad: dev [E] first chunk with rows of each expert
+  int32_t chunk;               // kBwdWGrad: this chunk (store where first == chunk, else add)
   uint32_t* status;
 };
 
 int bwd_pad_rows();
 cudaError_t launch_bwd_gemm(const BwdGemmArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_pad_offsets(const int32_t* counts, int32_t E, int32_t n_chunks, int32_t* offp,
-                               cudaStream_t s);
+                               int32_t* first, cudaStream_t s);
 cudaError_t launch_pad_rows(const int32_t* idx, const int32_t* dst, const int32_t* off,
                             const int32_t* offp, int64_t n, int32_t* dstp, cudaStream_t s);
 cudaError_t launch_dy_dw(const void* dout, const void* Y, const int32_t* dstp, const float* w,

@@ -781,7 +781,7 @@ namespace {
 
 struct BwdLayout {
   Layout meta;  // metadata regions (status/counts/splits, offsets, histograms, dst, src)
-  size_t offp, dstp, xp, gu, act, ydx, dy, dgu, total;
+  size_t offp, first, dstp, xp, gu, act, ydx, dy, dgu, total;
   int64_t rows_cap;
 };
 
@@ -792,6 +792,8 @@ BwdLayout make_bwd_layout(const Dims& d, int32_t H, int32_t I) {
   B.rows_cap = d.t_chunk * d.k + (int64_t)d.E * (bwd_pad_rows() - 1);
   B.offp = o;
   o += al(sizeof(int32_t) * (size_t)d.n * (d.E + 1));
+  B.first = o;
+  o += al(sizeof(int32_t) * (size_t)d.E);
   B.dstp = o;
   o += al(sizeof(int32_t) * (size_t)(d.T * d.k));
   const size_t R = (size_t)B.rows_cap;
@@ -850,11 +852,14 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
   DeviceCtx* ctx = nullptr;
   if ((st = get_ctx(&ctx)) != MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the weight gradients are sums over all chunks: start from zero
-  if (cudaMemsetAsync(dW_gate_up, 0, sizeof(float) * (size_t)E * 2 * I * H, s) != cudaSuccess ||
-      cudaMemsetAsync(dW_down, 0, sizeof(float) * (size_t)E * H * I, s) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  if (T == 0) return MOE_OK;
+  const size_t gu_per_e = (size_t)2 * I * H, dn_per_e = (size_t)H * I;  // fp32 elements
+  auto zero_experts = [&](int32_t e0, int32_t e1) {
+    return cudaMemsetAsync(dW_gate_up + e0 * gu_per_e, 0, sizeof(float) * (e1 - e0) * gu_per_e,
+                           s) == cudaSuccess &&
+           cudaMemsetAsync(dW_down + e0 * dn_per_e, 0, sizeof(float) * (e1 - e0) * dn_per_e, s) ==
+               cudaSuccess;
+  };
+  if (T == 0) return zero_experts(0, E) ? MOE_OK : MOE_ERR_CUDA;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int32_t* dst = reinterpret_cast<int32_t*>(ws + B.meta.dst);
   int32_t* src = reinterpret_cast<int32_t*>(ws + B.meta.src);
@@ -865,8 +870,25 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
                               ctx->host_stage + kStatusWords + (size_t)d.n * d.E);
   const int32_t* counts_dev = reinterpret_cast<const int32_t*>(ws + B.meta.packed) + kStatusWords;
   int32_t* offp = reinterpret_cast<int32_t*>(ws + B.offp);
+  int32_t* first = reinterpret_cast<int32_t*>(ws + B.first);
   int32_t* dstp = reinterpret_cast<int32_t*>(ws + B.dstp);
-  if (launch_pad_offsets(counts_dev, E, d.n, offp, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_pad_offsets(counts_dev, E, d.n, offp, first, s) != cudaSuccess) return MOE_ERR_CUDA;
+  // The weight-gradient GEMM of an expert's first chunk with rows stores its tiles and later
+  // chunks add to them, so only experts that no chunk routes to are zeroed here (runs of
+  // consecutive such experts take one memset per gradient).
+  std::vector<char> routed((size_t)E, 0);
+  for (int c = 0; c < d.n; ++c)
+    for (int32_t e = 0; e < E; ++e) routed[e] |= counts[(size_t)c * E + e] > 0;
+  for (int32_t e0 = 0; e0 < E;) {
+    if (routed[e0]) {
+      ++e0;
+      continue;
+    }
+    int32_t e1 = e0 + 1;
+    while (e1 < E && !routed[e1]) ++e1;
+    if (!zero_experts(e0, e1)) return MOE_ERR_CUDA;
+    e0 = e1;
+  }
   const std::vector<int64_t> bounds = dims_bounds(d);
   const int pad = bwd_pad_rows();
   const uint16_t* hid = static_cast<const uint16_t*>(hidden);
@@ -895,53 +917,69 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
     if (cudaMemsetAsync(xp, 0, 2 * (size_t)R * H, s) != cudaSuccess ||
         cudaMemsetAsync(dy, 0, 2 * (size_t)R * H, s) != cudaSuccess)
       return MOE_ERR_CUDA;
-    if (launch_pad_rows(top_k_index + t0 * k, dst + t0 * k, off_c, offp_c, len * k, dstp_c, s) !=
-            cudaSuccess ||
-        launch_permute(hid + t0 * H, dstp_c, len, H, k, xp, s) != cudaSuccess)
-      return MOE_ERR_CUDA;
+    {
+      ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len * k, 0, 2);
+      if (launch_pad_rows(top_k_index + t0 * k, dst + t0 * k, off_c, offp_c, len * k, dstp_c,
+                          s) != cudaSuccess ||
+          launch_permute(hid + t0 * H, dstp_c, len, H, k, xp, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
+    const int64_t active = active_experts(cnt, E);
+    auto bwd_gemm = [&](int kind, const BwdGemmArgs& a) {
+      ProfScope ps(kind, s, R, active, 1);
+      return launch_bwd_gemm(a, ctx->num_sms, s);
+    };
     BwdGemmArgs g{};
     g.offsets = offp_c;
     g.rows_pad_host = rows_pad.data();
     g.E = E;
     g.I = I;
     g.status = dev_status;
+    g.first = first;
+    g.chunk = c;
     // recompute g, u, h
     g.mode = kBwdRawGU;
     g.A = xp, g.A_rows = R, g.A_cols = H;
     g.B = W_gate_up, g.B_rows = (int64_t)E * 2 * I, g.B_cols = H;
     g.N = 2 * I, g.K = H, g.b_rows = 2 * I, g.out0 = gu, g.out1 = act;
-    if (launch_bwd_gemm(g, ctx->num_sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (bwd_gemm(MOE_KERNEL_BWD_GATEUP, g) != cudaSuccess) return MOE_ERR_CUDA;
     // recompute Y = h W_down^T (the forward down GEMM on the padded rows)
     if ((st = gemm_call(act, R, W_down, ydx, offp_c, rows_pad.data(), E, I, H, H, false,
                         dev_status, ctx->num_sms, s)) != MOE_OK)
       return st;
-    if (launch_dy_dw(dout + t0 * H, ydx, dstp_c, top_k_weights + t0 * k, len, H, k, dy,
-                     d_weights + t0 * k, s) != cudaSuccess)
-      return MOE_ERR_CUDA;
+    {
+      ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len * k, 0, 1);
+      if (launch_dy_dw(dout + t0 * H, ydx, dstp_c, top_k_weights + t0 * k, len, H, k, dy,
+                       d_weights + t0 * k, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
     // dh = dY W_down, SwiGLU backward in the epilogue -> [dg du]
     g.mode = kBwdDSwiGLU;
     g.A = dy, g.A_rows = R, g.A_cols = H;
     g.B = W_down, g.B_rows = (int64_t)E * H, g.B_cols = I;
     g.N = I, g.K = H, g.b_rows = H, g.out0 = dgu, g.out1 = nullptr, g.aux = gu;
-    if (launch_bwd_gemm(g, ctx->num_sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (bwd_gemm(MOE_KERNEL_BWD_DSWIGLU, g) != cudaSuccess) return MOE_ERR_CUDA;
     // dX = [dg du] W_gate_up
     g.mode = kBwdDPlain;
     g.A = dgu, g.A_rows = R, g.A_cols = 2 * I;
     g.B = W_gate_up, g.B_rows = (int64_t)E * 2 * I, g.B_cols = H;
     g.N = H, g.K = 2 * I, g.b_rows = 2 * I, g.out0 = ydx, g.aux = nullptr;
-    if (launch_bwd_gemm(g, ctx->num_sms, s) != cudaSuccess) return MOE_ERR_CUDA;
-    if (launch_sum_rows(ydx, dstp_c, len, H, k, dx_out + t0 * H, s) != cudaSuccess)
-      return MOE_ERR_CUDA;
+    if (bwd_gemm(MOE_KERNEL_BWD_DX, g) != cudaSuccess) return MOE_ERR_CUDA;
+    {
+      ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len * k, 0, 1);
+      if (launch_sum_rows(ydx, dstp_c, len, H, k, dx_out + t0 * H, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
     // dW_down[e] += dY^T h ;  dW_gate_up[e] += [dg du]^T X
     g.mode = kBwdWGrad;
     g.A = dy, g.A_rows = R, g.A_cols = H;
     g.B = act, g.B_rows = R, g.B_cols = I;
     g.M = H, g.N = I, g.acc = dW_down, g.out0 = nullptr;
-    if (launch_bwd_gemm(g, ctx->num_sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (bwd_gemm(MOE_KERNEL_BWD_WGRAD, g) != cudaSuccess) return MOE_ERR_CUDA;
     g.A = dgu, g.A_rows = R, g.A_cols = 2 * I;
     g.B = xp, g.B_rows = R, g.B_cols = H;
     g.M = 2 * I, g.N = H, g.acc = dW_gate_up;
-    if (launch_bwd_gemm(g, ctx->num_sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (bwd_gemm(MOE_KERNEL_BWD_WGRAD, g) != cudaSuccess) return MOE_ERR_CUDA;
   }
   return MOE_OK;
 }

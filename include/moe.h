@@ -45,7 +45,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 2
+#define MOE_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define MOE_API __attribute__((visibility("default")))
@@ -346,7 +346,13 @@ typedef enum {
   MOE_KERNEL_GATEUP = 2,
   MOE_KERNEL_DOWN = 3,
   MOE_KERNEL_UNPERMUTE = 4,
-  MOE_KERNEL_KINDS = 5
+  /* moe_backward (its recomputed down GEMM counts as MOE_KERNEL_DOWN) */
+  MOE_KERNEL_BWD_GATEUP = 5,   /* recomputed [g u] = X W_gate_up^T with h = silu(g) u      */
+  MOE_KERNEL_BWD_DSWIGLU = 6,  /* dh = dY W_down with the SwiGLU backward -> [dg du]        */
+  MOE_KERNEL_BWD_DX = 7,       /* dX = [dg du] W_gate_up                                    */
+  MOE_KERNEL_BWD_WGRAD = 8,    /* dW_down += dY^T h and dW_gate_up += [dg du]^T X           */
+  MOE_KERNEL_BWD_ROWS = 9,     /* row kernels: padded permute, dY and d_weights, d_hidden   */
+  MOE_KERNEL_KINDS = 10
 } moe_kernel_kind_t;
 
 typedef struct {

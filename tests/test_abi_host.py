@@ -40,7 +40,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_abi_version_and_status_strings():
     L = moe.load()
-    assert L.moe_abi_version() == 2
+    assert L.moe_abi_version() == 3
     for code, name in moe.STATUS_NAMES.items():
         assert moe.status_string(code).startswith(name)
     assert "unknown" in moe.status_string(99)
