@@ -11,6 +11,7 @@ from pinned host memory and its output copied back inside the timed region.
 sample per step).  Multi-GPU runs are independent replicas (the path has no exchange).
 """
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -31,6 +32,8 @@ import torch  # noqa: E402
 from gen import CONFIGS, expert_weights, hidden as gen_hidden, routing  # noqa: E402
 
 METRIC = "MoE fwd tokens/s; grouped-GEMM TFLOP/s and permute GB/s vs B200 peak"
+METRIC_BWD = "MoE bwd tokens/s (expert computation recomputed per chunk)"
+METRIC_TRAIN = "MoE fwd+bwd tokens/s (expert computation recomputed per chunk)"
 DEFAULT_CONFIG = "qwen3"
 DEFAULT_CHUNKS = 4
 GEMM_SRC = os.path.join(ROOT, "expert_router_top_b200", "csrc", "gemm.cu")
@@ -39,9 +42,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 def workload_name(cfg):
-    return {"qwen3": "qwen3-30b-a3b-shaped layer, one 16k packed sequence",
+    name = {"qwen3": "qwen3-30b-a3b-shaped layer, one 16k packed sequence",
             "mixtral": "mixtral-8x7b-shaped layer", "deepseek": "deepseek-v3-shaped routed layer",
             "tiny": "tiny layer", "edge": "edge-case layer"}.get(cfg.name, cfg.name)
+    if cfg.name in CONFIGS and cfg.T != CONFIGS[cfg.name].T:
+        name += f" (token count overridden: {cfg.T})"
+    return name
 
 
 def load_peaks():
@@ -187,9 +193,11 @@ def traffic_per_launch(cfg_name, chunks):
 
 # ------------------------------------------------------------------------- oracle arm
 
-def oracle_tokens_per_s(cfg, inputs, budget_s, sample_seed=0, max_tokens=None, seed=0):
+def oracle_tokens_per_s(cfg, inputs, budget_s, sample_seed=0, max_tokens=None, seed=0,
+                        kind="forward"):
     """Oracle throughput on a bounded, seeded sample of the workload's tokens.
 
+    kind: "forward", "backward" (gradients of sum(out * d_out)) or "train" (both).
     Draws the weights of the sampled tokens' experts on the host; returns
     (tokens/s, tokens, seconds, threads)."""
     import oracle
@@ -206,8 +214,12 @@ def oracle_tokens_per_s(cfg, inputs, budget_s, sample_seed=0, max_tokens=None, s
         sidx = np.vectorize(remap.get)(idx[toks]).astype(np.int32)
         wgu = np.stack([bits(expert_gate_up(e, cfg.H, cfg.I, seed)) for e in used])
         wd = np.stack([bits(expert_down(e, cfg.H, cfg.I, seed)) for e in used])
+        dout = bits(gen_hidden(n, cfg.H, 50 + sample_seed)) if kind != "forward" else None
         t0 = time.perf_counter()
-        oracle.forward(xb[toks], sidx, w[toks], wgu, wd)
+        if kind != "backward":
+            oracle.forward(xb[toks], sidx, w[toks], wgu, wd)
+        if kind != "forward":
+            oracle.backward(xb[toks], sidx, w[toks], wgu, wd, dout)
         return time.perf_counter() - t0
 
     threads = oracle.max_threads()
@@ -429,6 +441,153 @@ def run_ours(args, cfg):
     return 0
 
 
+def backward_units(cfg, counts):
+    """Algorithmic work of one moe_backward call from the chunk counts: flops per GEMM
+    kind and the weight-gradient GEMMs' bytes (operands read once; dW written by each
+    expert's first chunk with rows, read and written by its later chunks)."""
+    H, I = cfg.H, cfg.I
+    rows_c = counts.sum(1).astype(np.float64)
+    rows = float(rows_c.sum())
+    active = counts > 0
+    seen_before = np.cumsum(active, axis=0) - active  # chunks with rows before chunk c
+    dw_bytes = 12.0 * H * I * (active.sum() + (active & (seen_before > 0)).sum())
+    return {
+        "flops": {"bwd_gateup": 4 * rows * H * I, "down": 2 * rows * H * I,
+                  "bwd_dswiglu": 2 * rows * H * I, "bwd_dx": 4 * rows * H * I,
+                  "bwd_wgrad": 6 * rows * H * I},
+        "wgrad_bytes": float((rows_c * (2 * H + 3 * I) * 2).sum()) + dw_bytes,
+    }
+
+
+def run_backward(args, cfg):
+    """--pass backward|train: time moe_backward (train: moe_forward then moe_backward) per
+    step; the roofline object is for the weight-gradient GEMMs, the largest backward kind."""
+    import expert_router_top_b200 as moe
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    moe.load()
+    dev = torch.device("cuda", local)
+    inp = make_inputs(cfg, dev)
+    chunks = args.chunks
+    train = args.pass_ == "train"
+    dout = gen_hidden(cfg.T, cfg.H, 77).to(dev)
+    bws = moe.alloc_workspace(moe.backward_workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k,
+                                                           cfg.G, chunks), dev)
+    fws = moe.alloc_workspace(moe.workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.G,
+                                                  chunks), dev) if train else None
+    stream = torch.cuda.current_stream()
+    meta = moe.metadata(inp["idx"], cfg.E, cfg.G, chunks)
+    units = backward_units(cfg, meta["counts"])
+    out = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device=dev)
+    grads = moe.backward_buffers(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, dev)
+
+    def step():
+        if train:
+            moe.forward(inp["hidden"], inp["idx"], inp["w"], inp["wgu"], inp["wd"],
+                        num_chunks=chunks, ep_groups=cfg.G, out=out, workspace=fws,
+                        stream=stream)
+        moe.backward(inp["hidden"], inp["idx"], inp["w"], inp["wgu"], inp["wd"], dout,
+                     num_chunks=chunks, ep_groups=cfg.G, workspace=bws, stream=stream,
+                     out=grads)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    moe.profile_enable(True)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    prof = moe.profile_read()
+    moe.profile_enable(False)
+    clk = clocks.stop() if clocks else None
+    ms_max = max_over_ranks(start.elapsed_time(end), pg, dev)
+    steps = args.steps
+    peaks, peak_src = load_peaks()
+    kinds = {}
+    for kind in moe.KERNEL_KINDS:
+        p = prof[kind]
+        if not p["launches"]:
+            continue
+        kinds[kind] = dict(launches=p["launches"], ms_per_step=p["ms"] / steps)
+        fl = units["flops"].get(kind)
+        if fl and p["ms"] > 0:
+            kinds[kind]["tflops"] = fl * steps / (p["ms"] / 1e3) / 1e12
+    # roofline of the weight-gradient GEMMs (both launches of every chunk, whole step)
+    wg = prof["bwd_wgrad"]
+    t = wg["ms"] / steps / 1e3
+    f, b = units["flops"]["bwd_wgrad"], units["wgrad_bytes"]
+    t_tensor, t_mem = f / (peaks["bf16_tflops"] * 1e12), b / (peaks["hbm_gbs"] * 1e9)
+    if t_mem > t_tensor:
+        roofline = {"bound": "hbm", "achieved": b / t / 1e9, "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s"}
+    else:
+        roofline = {"bound": "tensor", "achieved": f / t / 1e12, "peak": peaks["bf16_tflops"],
+                    "unit": "TFLOP/s"}
+    roofline["frac"] = roofline["achieved"] / roofline["peak"]
+    n_wg = max(1, wg["launches"] // max(1, steps))
+    roofline.update({
+        "traffic": None,
+        "kernel": "bwd_gemm_kernel<weight gradient> (tcgen05, TMA store / add-reduce epilogue)",
+        "peak_source": f"{peak_src}: MEASURED_PEAKS.json (bf16 burst, HBM copy)",
+        "per_launch": {"flops": f / n_wg, "bytes": b / n_wg, "ms": t * 1e3 / n_wg,
+                       "roofline_ms": max(t_tensor, t_mem) * 1e3 / n_wg},
+        "tensor_frac": f / t / 1e12 / peaks["bf16_tflops"],
+        "hbm_frac": b / t / 1e9 / peaks["hbm_gbs"]})
+    gemm_fl = sum(v for k2, v in units["flops"].items())
+    gemm_ms = sum(prof[k2]["ms"] for k2 in units["flops"]) / steps
+    ws_per_n = {str(n): moe.backward_workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.G, n)
+                for n in (1, 2, 4)}
+    line = {
+        "metric": METRIC_TRAIN if train else METRIC_BWD,
+        "value": job_tokens_per_s(world, cfg.T, steps, ms_max), "unit": "tokens/s",
+        "n_gpus": world, "steps": steps, "warmup": args.warmup, "ms_per_step": ms_max / steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; random-init expert weights of the layer's shape)",
+        "config": dict(config_block(cfg, chunks), **{"pass": args.pass_}),
+        "roofline": roofline,
+        "grouped_gemm_tflops": gemm_fl / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None,
+        "kernels": kinds,
+        "backward_workspace_bytes": ws_per_n,
+        "gpu_launches": int(prof["kernels"]),
+        "e2e": None,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tps, ntok, dt, threads = oracle_tokens_per_s(cfg, inp, args.cpu_budget_s,
+                                                     kind=args.pass_)
+        line["cpu_baseline"] = {
+            "value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{ntok} seeded tokens of the {cfg.T}-token workload, all k={cfg.k} "
+                      f"experts each, fp64 {args.pass_}, {dt:.1f} s"}
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_e2e(moe, inp, cfg, chunks, ws, args, stream, dev, pg, world):
     """The same metric through moe_forward_host: each step copies its hidden rows, routing
     indices and weights from pinned host memory and its output back to pinned host memory
@@ -474,13 +633,23 @@ def main():
     ap.add_argument("--dispatch", choices=["separate", "fused"], default="separate",
                     help="separate: permute kernel first; fused: the gate/up GEMM gathers its "
                          "rows from hidden")
+    ap.add_argument("--pass", dest="pass_", choices=["forward", "backward", "train"],
+                    default="forward",
+                    help="forward (the layer's headline), backward (moe_backward alone) or "
+                         "train (forward then backward per step)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override the workload's token count (small cases for profiling)")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps, always
     cfg = CONFIGS[args.config]
+    if args.tokens > 0:
+        cfg = dataclasses.replace(cfg, T=args.tokens)
     if args.impl == "reference":
         return run_reference(args, cfg)
+    if args.pass_ != "forward":
+        return run_backward(args, cfg)
     return run_ours(args, cfg)
 
 

@@ -293,11 +293,24 @@ def forward_host(hidden, top_k_index, top_k_weights, W_gate_up, W_down, num_chun
     return out
 
 
+def backward_workspace_bytes(T, H, I, E, k, ep_groups=1, num_chunks=1, chunk_size=0) -> int:
+    s = shape(T, H, I, E, k, ep_groups, num_chunks, chunk_size)
+    return int(load().moe_backward_workspace_bytes(ctypes.byref(s)))
+
+
+def backward_buffers(T, H, I, E, k, device):
+    """Output tensors of backward(): (d_hidden, d_weights, dW_gate_up, dW_down)."""
+    return (torch.empty((T, H), dtype=torch.bfloat16, device=device),
+            torch.empty((T, k), dtype=torch.float32, device=device),
+            torch.empty((E, 2 * I, H), dtype=torch.float32, device=device),
+            torch.empty((E, H, I), dtype=torch.float32, device=device))
+
+
 def backward(hidden, top_k_index, top_k_weights, W_gate_up, W_down, d_out, num_chunks: int = 1,
-             ep_groups: int = 1, chunk_size: int = 0, workspace=None, stream=None):
+             ep_groups: int = 1, chunk_size: int = 0, workspace=None, stream=None, out=None):
     """Backward of forward() for the loss sum(out * d_out), with the expert computation
     recomputed chunk by chunk.  Returns (d_hidden bf16 [T,H], d_weights fp32 [T,k],
-    dW_gate_up fp32 [E,2I,H], dW_down fp32 [E,H,I])."""
+    dW_gate_up fp32 [E,2I,H], dW_down fp32 [E,H,I]), written into `out` when given."""
     for t, dt, name in ((hidden, torch.bfloat16, "hidden"), (top_k_index, torch.int32, "top_k_index"),
                         (top_k_weights, torch.float32, "top_k_weights"),
                         (W_gate_up, torch.bfloat16, "W_gate_up"), (W_down, torch.bfloat16, "W_down"),
@@ -309,10 +322,16 @@ def backward(hidden, top_k_index, top_k_weights, W_gate_up, W_down, d_out, num_c
     k = top_k_index.shape[1]
     s = shape(T, H, I, E, k, ep_groups, num_chunks, chunk_size)
     dev = hidden.device
-    d_hidden = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
-    d_weights = torch.empty((T, k), dtype=torch.float32, device=dev)
-    dW_gate_up = torch.empty((E, 2 * I, H), dtype=torch.float32, device=dev)
-    dW_down = torch.empty((E, H, I), dtype=torch.float32, device=dev)
+    if out is None:
+        out = backward_buffers(T, H, I, E, k, dev)
+    d_hidden, d_weights, dW_gate_up, dW_down = out
+    for t, dt, shp, name in ((d_hidden, torch.bfloat16, (T, H), "d_hidden"),
+                             (d_weights, torch.float32, (T, k), "d_weights"),
+                             (dW_gate_up, torch.float32, (E, 2 * I, H), "dW_gate_up"),
+                             (dW_down, torch.float32, (E, H, I), "dW_down")):
+        _need(t, dt, name)
+        if tuple(t.shape) != shp:
+            raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {shp}")
     if workspace is None:
         workspace = alloc_workspace(load().moe_backward_workspace_bytes(ctypes.byref(s)), dev)
     _check(load().moe_backward(ctypes.byref(s), _ptr(hidden), _ptr(top_k_index),

@@ -57,6 +57,12 @@
 #ifndef MOE_GEMM_BAND
 #define MOE_GEMM_BAND 16  // M tiles per raster band: an expert's A rows stay in L2 across N tiles
 #endif
+#ifndef MOE_GEMM_PACKED_B
+// 1: B is read from a tile-packed weight layout in which the 256 B rows of one tile and one
+// K block (gate rows then up rows for gate/up) are one contiguous 32 KB block, fetched with
+// one box per stage
+#define MOE_GEMM_PACKED_B 0
+#endif
 #ifndef MOE_GEMM_B4D
 #define MOE_GEMM_B4D 0  // gate/up: one 4-D box fetches the gate and the up rows of a tile
 #endif
@@ -403,7 +409,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
           } else {
             mbar_arrive_expect_tx(&ctl->full[stage], G::kTxBytes);
             tma_load_2d(a_dst, tmA, &ctl->full[stage], kb * BK, row0, pol_a);
-            if (kSwiGLU && p.b4d) {
+            if (MOE_GEMM_PACKED_B) {
+              const int32_t prow = ((t_e * p.n_tiles + t_n) * p.num_kb + kb) * BN;
+              tma_load_2d(b_dst, tmB, &ctl->full[stage], 0, prow, pol_w);
+            } else if (kSwiGLU && p.b4d) {
               // {K, row in block, 128-row block n, 2e + gate/up}: gate block n, then up block n
               tma_load_4d(b_dst, tmB, &ctl->full[stage], kb * BK, 0, t_n, 2 * t_e, pol_w);
             } else if (kSwiGLU) {
@@ -671,9 +680,14 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
   // one-box gate/up weights (single-CTA, plain A, I a multiple of 128)
   const bool b4d = MOE_GEMM_B4D && swiglu && !kPair && !gather && a.out_cols % 128 == 0 &&
                    make_map_gateup4d(&mB, a.B, a.E, a.out_cols, a.K);
-  if (!map_a_ok ||
-      (!b4d && !make_map(&mB, a.B, (int64_t)a.E * a.b_rows, a.K,
-                         kPair ? BN / 2 : (swiglu ? BN / 2 : BN)))) {
+  const int64_t packed_rows =
+      (int64_t)a.E * ((a.out_cols + bn - 1) / bn) * ((a.K + BK - 1) / BK) * BN;
+  const bool map_b_ok =
+      b4d || (MOE_GEMM_PACKED_B && !kPair && !gather
+                  ? make_map(&mB, a.B, packed_rows, BK, BN)
+                  : make_map(&mB, a.B, (int64_t)a.E * a.b_rows, a.K,
+                             kPair ? BN / 2 : (swiglu ? BN / 2 : BN)));
+  if (!map_a_ok || !map_b_ok) {
     *err_detail = 2;
     return cudaErrorInvalidValue;
   }

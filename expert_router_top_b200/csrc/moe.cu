@@ -198,6 +198,10 @@ struct DeviceCtx {
   cudaStream_t copy_in = nullptr, copy_out = nullptr;
   cudaEvent_t ev_in[2] = {}, ev_in_free[2] = {}, ev_out[2] = {}, ev_out_free[2] = {},
               ev_copy_join = nullptr;
+  // backward pipeline: permuted rows ready (per X slot), recomputed Y ready, dY ready, dX
+  // ready, d_hidden rows summed (per buffer), all of a chunk's GEMMs done (per X slot)
+  cudaEvent_t ev_bp[3] = {}, ev_bf[2] = {}, ev_bdy[2] = {}, ev_bdx[2] = {}, ev_bsum[2] = {},
+              ev_bw[3] = {};
   int32_t* host_stage = nullptr;
   size_t host_stage_bytes = 0;
 };
@@ -235,6 +239,16 @@ moe_status_t get_ctx(DeviceCtx** out) {
           cudaEventCreateWithFlags(&c.ev_out_free[b], fl) != cudaSuccess)
         return MOE_ERR_CUDA;
     if (cudaEventCreateWithFlags(&c.ev_copy_join, fl) != cudaSuccess) return MOE_ERR_CUDA;
+    for (int b = 0; b < 3; ++b)
+      if (cudaEventCreateWithFlags(&c.ev_bp[b], fl) != cudaSuccess ||
+          cudaEventCreateWithFlags(&c.ev_bw[b], fl) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    for (int b = 0; b < 2; ++b)
+      if (cudaEventCreateWithFlags(&c.ev_bf[b], fl) != cudaSuccess ||
+          cudaEventCreateWithFlags(&c.ev_bdy[b], fl) != cudaSuccess ||
+          cudaEventCreateWithFlags(&c.ev_bdx[b], fl) != cudaSuccess ||
+          cudaEventCreateWithFlags(&c.ev_bsum[b], fl) != cudaSuccess)
+        return MOE_ERR_CUDA;
     c.ready = true;
   }
   *out = &c;
@@ -781,10 +795,15 @@ namespace {
 
 struct BwdLayout {
   Layout meta;  // metadata regions (status/counts/splits, offsets, histograms, dst, src)
-  size_t offp, first, dstp, xp, gu, act, ydx, dy, dgu, total;
+  size_t offp, first, dstp, total;
+  int nx, nb;  // X slots (3 when three or more chunks) and buffer sets of the other rows
+  size_t xp[3], gu[2], act[2], ydx[2], dy[2], dgu[2];
   int64_t rows_cap;
 };
 
+// Every chunk's rows, padded per expert to a multiple of 64, fit in rows_cap rows.  The
+// pipeline keeps chunk c's permuted rows in X slot c % 3 (they are read until the chunk's
+// last weight-gradient GEMM) and its other row buffers in set c % 2.
 BwdLayout make_bwd_layout(const Dims& d, int32_t H, int32_t I) {
   BwdLayout B{};
   B.meta = make_layout(d, 8, 8, false, true, true);
@@ -797,18 +816,24 @@ BwdLayout make_bwd_layout(const Dims& d, int32_t H, int32_t I) {
   B.dstp = o;
   o += al(sizeof(int32_t) * (size_t)(d.T * d.k));
   const size_t R = (size_t)B.rows_cap;
-  B.xp = o;
-  o += al(2 * R * H);
-  B.gu = o;
-  o += al(2 * R * 2 * I);
-  B.act = o;
-  o += al(2 * R * I);
-  B.ydx = o;  // recomputed Y rows, later dX rows
-  o += al(2 * R * H);
-  B.dy = o;
-  o += al(2 * R * H);
-  B.dgu = o;
-  o += al(2 * R * 2 * I);
+  B.nx = d.n >= 3 ? 3 : d.n;
+  B.nb = d.n >= 2 ? 2 : 1;
+  for (int b = 0; b < B.nx; ++b) {
+    B.xp[b] = o;
+    o += al(2 * R * H);
+  }
+  for (int b = 0; b < B.nb; ++b) {
+    B.gu[b] = o;
+    o += al(2 * R * 2 * I);
+    B.act[b] = o;
+    o += al(2 * R * I);
+    B.ydx[b] = o;  // recomputed Y rows, later dX rows
+    o += al(2 * R * H);
+    B.dy[b] = o;
+    o += al(2 * R * H);
+    B.dgu[b] = o;
+    o += al(2 * R * 2 * I);
+  }
   B.total = o;
   return B;
 }
@@ -890,97 +915,143 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
     e0 = e1;
   }
   const std::vector<int64_t> bounds = dims_bounds(d);
+  int n_live = 0;  // chunks with tokens; only trailing chunks can be empty
+  while (n_live < d.n && bounds[n_live + 1] > bounds[n_live]) ++n_live;
   const int pad = bwd_pad_rows();
   const uint16_t* hid = static_cast<const uint16_t*>(hidden);
   const uint16_t* dout = static_cast<const uint16_t*>(d_out);
   uint16_t* dx_out = static_cast<uint16_t*>(d_hidden);
-  std::vector<int32_t> rows_pad((size_t)E);
-  for (int c = 0; c < d.n; ++c) {
-    const int64_t t0 = bounds[c], len = bounds[c + 1] - bounds[c];
-    if (len == 0) continue;
-    const int32_t* cnt = counts.data() + (size_t)c * E;
-    int64_t R = 0;
+  cudaStream_t sg = ctx->side;
+  // padded rows per expert and their total, per chunk
+  std::vector<int32_t> rows_pad((size_t)d.n * E);
+  std::vector<int64_t> R((size_t)d.n, 0);
+  for (int c = 0; c < d.n; ++c)
     for (int32_t e = 0; e < E; ++e) {
-      rows_pad[e] = (cnt[e] + pad - 1) / pad * pad;
-      R += rows_pad[e];
+      const int32_t v = (counts[(size_t)c * E + e] + pad - 1) / pad * pad;
+      rows_pad[(size_t)c * E + e] = v;
+      R[c] += v;
     }
-    const int32_t* off_c = reinterpret_cast<const int32_t*>(ws + B.meta.offsets) + (size_t)c * (E + 1);
-    const int32_t* offp_c = offp + (size_t)c * (E + 1);
-    int32_t* dstp_c = dstp + t0 * k;
-    void* xp = ws + B.xp;
-    void* gu = ws + B.gu;
-    void* act = ws + B.act;
-    void* ydx = ws + B.ydx;
-    void* dy = ws + B.dy;
-    void* dgu = ws + B.dgu;
-    // zero the padded row buffers that seed every pad row (X and dY)
-    if (cudaMemsetAsync(xp, 0, 2 * (size_t)R * H, s) != cudaSuccess ||
-        cudaMemsetAsync(dy, 0, 2 * (size_t)R * H, s) != cudaSuccess)
+  auto x_of = [&](int c) { return ws + B.xp[c % B.nx]; };
+  auto buf = [&](const size_t(&a)[2], int c) { return ws + a[c % B.nb]; };
+  auto off_c = [&](int c) {
+    return reinterpret_cast<const int32_t*>(ws + B.meta.offsets) + (size_t)c * (E + 1);
+  };
+  auto offp_c = [&](int c) -> const int32_t* { return offp + (size_t)c * (E + 1); };
+  auto dstp_c = [&](int c) { return dstp + bounds[c] * k; };
+  auto len = [&](int c) { return bounds[c + 1] - bounds[c]; };
+  auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+
+  // P(c), stream M: padded permute of the chunk's rows into X slot c % 3 (zero pad rows)
+  auto P = [&](int c) -> moe_status_t {
+    if (c >= 3 && !ok(cudaStreamWaitEvent(s, ctx->ev_bw[c % 3], 0))) return MOE_ERR_CUDA;
+    ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(c) * k, 0, 2);
+    if (!ok(cudaMemsetAsync(x_of(c), 0, 2 * (size_t)R[c] * H, s)) ||
+        !ok(launch_pad_rows(top_k_index + bounds[c] * k, dst + bounds[c] * k, off_c(c), offp_c(c),
+                            len(c) * k, dstp_c(c), s)) ||
+        !ok(launch_permute(hid + bounds[c] * H, dstp_c(c), len(c), H, k, x_of(c), s)) ||
+        !ok(cudaEventRecord(ctx->ev_bp[c % 3], s)))
       return MOE_ERR_CUDA;
-    {
-      ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len * k, 0, 2);
-      if (launch_pad_rows(top_k_index + t0 * k, dst + t0 * k, off_c, offp_c, len * k, dstp_c,
-                          s) != cudaSuccess ||
-          launch_permute(hid + t0 * H, dstp_c, len, H, k, xp, s) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    }
-    const int64_t active = active_experts(cnt, E);
-    auto bwd_gemm = [&](int kind, const BwdGemmArgs& a) {
-      ProfScope ps(kind, s, R, active, 1);
-      return launch_bwd_gemm(a, ctx->num_sms, s);
-    };
-    BwdGemmArgs g{};
-    g.offsets = offp_c;
-    g.rows_pad_host = rows_pad.data();
-    g.E = E;
-    g.I = I;
-    g.status = dev_status;
-    g.first = first;
+    return MOE_OK;
+  };
+  BwdGemmArgs g0{};
+  g0.E = E;
+  g0.I = I;
+  g0.status = dev_status;
+  g0.first = first;
+  auto bwd_gemm = [&](int kind, const BwdGemmArgs& a, int c) {
+    ProfScope ps(kind, sg, R[c], active_experts(counts.data() + (size_t)c * E, E), 1);
+    return launch_bwd_gemm(a, ctx->num_sms, sg);
+  };
+  // F(c), stream G: recompute [g u], h and Y = h W_down^T on the padded rows
+  auto F = [&](int c) -> moe_status_t {
+    if (!ok(cudaStreamWaitEvent(sg, ctx->ev_bp[c % 3], 0))) return MOE_ERR_CUDA;
+    if (c >= 2 && !ok(cudaStreamWaitEvent(sg, ctx->ev_bsum[c % 2], 0))) return MOE_ERR_CUDA;
+    BwdGemmArgs g = g0;
+    g.offsets = offp_c(c);
+    g.rows_pad_host = rows_pad.data() + (size_t)c * E;
     g.chunk = c;
-    // recompute g, u, h
     g.mode = kBwdRawGU;
-    g.A = xp, g.A_rows = R, g.A_cols = H;
+    g.A = x_of(c), g.A_rows = R[c], g.A_cols = H;
     g.B = W_gate_up, g.B_rows = (int64_t)E * 2 * I, g.B_cols = H;
-    g.N = 2 * I, g.K = H, g.b_rows = 2 * I, g.out0 = gu, g.out1 = act;
-    if (bwd_gemm(MOE_KERNEL_BWD_GATEUP, g) != cudaSuccess) return MOE_ERR_CUDA;
-    // recompute Y = h W_down^T (the forward down GEMM on the padded rows)
-    if ((st = gemm_call(act, R, W_down, ydx, offp_c, rows_pad.data(), E, I, H, H, false,
-                        dev_status, ctx->num_sms, s)) != MOE_OK)
-      return st;
-    {
-      ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len * k, 0, 1);
-      if (launch_dy_dw(dout + t0 * H, ydx, dstp_c, top_k_weights + t0 * k, len, H, k, dy,
-                       d_weights + t0 * k, s) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    }
-    // dh = dY W_down, SwiGLU backward in the epilogue -> [dg du]
+    g.N = 2 * I, g.K = H, g.b_rows = 2 * I, g.out0 = buf(B.gu, c), g.out1 = buf(B.act, c);
+    if (!ok(bwd_gemm(MOE_KERNEL_BWD_GATEUP, g, c))) return MOE_ERR_CUDA;
+    moe_status_t s2 = gemm_call(buf(B.act, c), R[c], W_down, buf(B.ydx, c), offp_c(c),
+                                rows_pad.data() + (size_t)c * E, E, I, H, H, false, dev_status,
+                                ctx->num_sms, sg);
+    if (s2 != MOE_OK) return s2;
+    return ok(cudaEventRecord(ctx->ev_bf[c % 2], sg)) ? MOE_OK : MOE_ERR_CUDA;
+  };
+  // DY(c), stream M: dY = w dout (zero pad rows) and d_weights
+  auto DY = [&](int c) -> moe_status_t {
+    if (!ok(cudaStreamWaitEvent(s, ctx->ev_bf[c % 2], 0))) return MOE_ERR_CUDA;
+    ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(c) * k, 0, 1);
+    if (!ok(cudaMemsetAsync(buf(B.dy, c), 0, 2 * (size_t)R[c] * H, s)) ||
+        !ok(launch_dy_dw(dout + bounds[c] * H, buf(B.ydx, c), dstp_c(c),
+                         top_k_weights + bounds[c] * k, len(c), H, k, buf(B.dy, c),
+                         d_weights + bounds[c] * k, s)) ||
+        !ok(cudaEventRecord(ctx->ev_bdy[c % 2], s)))
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  };
+  // Bk(c), stream G: dh with the SwiGLU backward, dX, then both weight gradients
+  auto Bk = [&](int c) -> moe_status_t {
+    if (!ok(cudaStreamWaitEvent(sg, ctx->ev_bdy[c % 2], 0))) return MOE_ERR_CUDA;
+    BwdGemmArgs g = g0;
+    g.offsets = offp_c(c);
+    g.rows_pad_host = rows_pad.data() + (size_t)c * E;
+    g.chunk = c;
     g.mode = kBwdDSwiGLU;
-    g.A = dy, g.A_rows = R, g.A_cols = H;
+    g.A = buf(B.dy, c), g.A_rows = R[c], g.A_cols = H;
     g.B = W_down, g.B_rows = (int64_t)E * H, g.B_cols = I;
-    g.N = I, g.K = H, g.b_rows = H, g.out0 = dgu, g.out1 = nullptr, g.aux = gu;
-    if (bwd_gemm(MOE_KERNEL_BWD_DSWIGLU, g) != cudaSuccess) return MOE_ERR_CUDA;
-    // dX = [dg du] W_gate_up
+    g.N = I, g.K = H, g.b_rows = H, g.out0 = buf(B.dgu, c), g.aux = buf(B.gu, c);
+    if (!ok(bwd_gemm(MOE_KERNEL_BWD_DSWIGLU, g, c))) return MOE_ERR_CUDA;
     g.mode = kBwdDPlain;
-    g.A = dgu, g.A_rows = R, g.A_cols = 2 * I;
+    g.A = buf(B.dgu, c), g.A_rows = R[c], g.A_cols = 2 * I;
     g.B = W_gate_up, g.B_rows = (int64_t)E * 2 * I, g.B_cols = H;
-    g.N = H, g.K = 2 * I, g.b_rows = 2 * I, g.out0 = ydx, g.aux = nullptr;
-    if (bwd_gemm(MOE_KERNEL_BWD_DX, g) != cudaSuccess) return MOE_ERR_CUDA;
-    {
-      ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len * k, 0, 1);
-      if (launch_sum_rows(ydx, dstp_c, len, H, k, dx_out + t0 * H, s) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    }
-    // dW_down[e] += dY^T h ;  dW_gate_up[e] += [dg du]^T X
+    g.N = H, g.K = 2 * I, g.b_rows = 2 * I, g.out0 = buf(B.ydx, c), g.aux = nullptr;
+    if (!ok(bwd_gemm(MOE_KERNEL_BWD_DX, g, c)) || !ok(cudaEventRecord(ctx->ev_bdx[c % 2], sg)))
+      return MOE_ERR_CUDA;
+    // dW_down[e] (+)= dY^T h ;  dW_gate_up[e] (+)= [dg du]^T X
     g.mode = kBwdWGrad;
-    g.A = dy, g.A_rows = R, g.A_cols = H;
-    g.B = act, g.B_rows = R, g.B_cols = I;
+    g.A = buf(B.dy, c), g.A_rows = R[c], g.A_cols = H;
+    g.B = buf(B.act, c), g.B_rows = R[c], g.B_cols = I;
     g.M = H, g.N = I, g.acc = dW_down, g.out0 = nullptr;
-    if (bwd_gemm(MOE_KERNEL_BWD_WGRAD, g) != cudaSuccess) return MOE_ERR_CUDA;
-    g.A = dgu, g.A_rows = R, g.A_cols = 2 * I;
-    g.B = xp, g.B_rows = R, g.B_cols = H;
+    if (!ok(bwd_gemm(MOE_KERNEL_BWD_WGRAD, g, c))) return MOE_ERR_CUDA;
+    g.A = buf(B.dgu, c), g.A_rows = R[c], g.A_cols = 2 * I;
+    g.B = x_of(c), g.B_rows = R[c], g.B_cols = H;
     g.M = 2 * I, g.N = H, g.acc = dW_gate_up;
-    if (bwd_gemm(MOE_KERNEL_BWD_WGRAD, g) != cudaSuccess) return MOE_ERR_CUDA;
+    if (!ok(bwd_gemm(MOE_KERNEL_BWD_WGRAD, g, c)) || !ok(cudaEventRecord(ctx->ev_bw[c % 3], sg)))
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  };
+  // S(c), stream M: d_hidden rows = sum over the k copies of dX
+  auto S = [&](int c) -> moe_status_t {
+    if (!ok(cudaStreamWaitEvent(s, ctx->ev_bdx[c % 2], 0))) return MOE_ERR_CUDA;
+    ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(c) * k, 0, 1);
+    if (!ok(launch_sum_rows(buf(B.ydx, c), dstp_c(c), len(c), H, k, dx_out + bounds[c] * H, s)) ||
+        !ok(cudaEventRecord(ctx->ev_bsum[c % 2], s)))
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  };
+
+  // The mirrored pair pipeline.  G: F(0) F(1) B(0) F(2) B(1) F(3) ... B(n-1);
+  // M: P(0) P(1) DY(0) P(2) S(0) DY(1) P(3) S(1) ...  Chunk c+2's permute overlaps chunk c's
+  // GEMMs and every row kernel after the first permute overlaps a neighbouring chunk's GEMMs.
+  // Host enqueue order keeps each event wait on the record it is meant for.
+  if (!ok(cudaEventRecord(ctx->ev_start, s)) || !ok(cudaStreamWaitEvent(sg, ctx->ev_start, 0)))
+    return MOE_ERR_CUDA;
+  if (n_live > 0) {
+    if ((st = P(0)) != MOE_OK || (st = F(0)) != MOE_OK) return st;
+    if (n_live > 1 && ((st = P(1)) != MOE_OK || (st = F(1)) != MOE_OK)) return st;
+    for (int c = 0; c < n_live; ++c) {
+      if ((st = DY(c)) != MOE_OK) return st;
+      if (c + 2 < n_live && (st = P(c + 2)) != MOE_OK) return st;
+      if ((st = Bk(c)) != MOE_OK || (st = S(c)) != MOE_OK) return st;
+      if (c + 2 < n_live && (st = F(c + 2)) != MOE_OK) return st;
+    }
   }
+  if (!ok(cudaEventRecord(ctx->ev_join, sg)) || !ok(cudaStreamWaitEvent(s, ctx->ev_join, 0)))
+    return MOE_ERR_CUDA;
   return MOE_OK;
 }
 
