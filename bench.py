@@ -443,13 +443,15 @@ def run_ours(args, cfg):
 
 def backward_units(cfg, counts):
     """Algorithmic work of one moe_backward call from the chunk counts: flops per GEMM
-    kind and the weight-gradient GEMMs' bytes (operands read once; dW written by each
-    expert's first chunk with rows, read and written by its later chunks)."""
+    kind and the weight-gradient GEMMs' bytes.  The weight gradients run once per pair of
+    adjacent chunks (0,1), (2,3), ...: operands are read once; dW is written by the pair in
+    which an expert first has rows and read and written by every later pair with its rows."""
     H, I = cfg.H, cfg.I
     rows_c = counts.sum(1).astype(np.float64)
     rows = float(rows_c.sum())
-    active = counts > 0
-    seen_before = np.cumsum(active, axis=0) - active  # chunks with rows before chunk c
+    pairs = np.stack([counts[i:i + 2].sum(0) for i in range(0, counts.shape[0], 2)])
+    active = pairs > 0
+    seen_before = np.cumsum(active, axis=0) - active  # earlier pairs with rows
     dw_bytes = 12.0 * H * I * (active.sum() + (active & (seen_before > 0)).sum())
     return {
         "flops": {"bwd_gateup": 4 * rows * H * I, "down": 2 * rows * H * I,

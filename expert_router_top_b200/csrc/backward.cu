@@ -21,7 +21,7 @@
 //   kDSwiGLU  dh = dY W_down                  B MN-major                  epilogue: dg, du
 //   kDPlain   dX = [dg du] W_gate_up          B MN-major                  epilogue: bf16 store
 //   kWGrad    dW[e] += S_A[e]^T S_B[e]        A and B MN-major, K = rows  epilogue: TMA fp32
-//                                                                        store / add-reduce
+//             (K = the rows of one chunk, or of a pair of chunks)       store / add-reduce
 // MN-major operands use the 128-byte-swizzled MN-major canonical layout: 64-element MN
 // blocks of 64 K rows x 128 B (8 KB apart: the leading byte offset), 8-row K groups 1 KB
 // apart (the stride byte offset); one MMA K step of 16 advances 2 KB.
@@ -37,7 +37,14 @@ namespace moe {
 namespace {
 
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr int kThreads = 192;
+// Epilogue warps per mode: eight (two per TMEM lane quarter, each taking half of the tile's
+// columns) where the epilogue does per-element math; four for the weight gradients, whose
+// epilogue is a TMA store per block and whose staging buffer is sized for four warps.
+template <int kMode>
+struct Cfg {
+  static constexpr int kEpi = kMode == 3 ? 4 : 8;
+  static constexpr int kThreads = 64 + 32 * kEpi;
+};
 constexpr uint32_t kABytes = BM * BK * 2, kBBytes = BN * BK * 2, kStageBytes = kABytes + kBBytes;
 constexpr uint32_t kTmemCols = 2 * BN;
 constexpr int kMaxE = 1024;
@@ -62,7 +69,9 @@ struct BParams {
   const __nv_bfloat16* aux; // kDSwiGLU: GU [rows][2I]
   float* acc;               // kWGrad: [E][M][N] fp32 (written through tmC)
   const int32_t* first;     // kWGrad: [E] first chunk with rows of each expert
-  int32_t chunk;            // kWGrad: this chunk
+  int32_t chunk;            // kWGrad: first chunk of this launch
+  int32_t chunk_last;       // kWGrad: last chunk of this launch (chunk + 1 for a pair)
+  const int32_t* offsets1;  // kWGrad: padded offsets [E+1] of the pair's second chunk, or null
 };
 
 struct Ctl {
@@ -76,7 +85,7 @@ static_assert(sizeof(Ctl) <= kCtlBytes, "control block");
 constexpr uint32_t kOutBoxBytes = 32 * 32 * 4;
 constexpr uint32_t kOutBytes = 4 * kOutBoxBytes;
 constexpr size_t kSmem =
-    1024 + STAGES * kStageBytes + kOutBytes + kCtlBytes + 2 * (kMaxE + 1) * 4;
+    1024 + STAGES * kStageBytes + kOutBytes + kCtlBytes + 3 * (kMaxE + 1) * 4;
 static_assert(kSmem <= 232448, "shared memory per CTA");
 
 __host__ __device__ constexpr uint32_t idesc(bool a_mn, bool b_mn) {
@@ -117,13 +126,15 @@ __device__ __forceinline__ Tile decode(int32_t L, const int32_t* ts, const int32
   return t;
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 template <int kMode>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ CUtensorMap tmC, const BParams p) {
+                    const __grid_constant__ CUtensorMap tmC,
+                    const __grid_constant__ CUtensorMap tmA1,
+                    const __grid_constant__ CUtensorMap tmB1, const BParams p) {
   constexpr bool kAmn = kMode == kWGrad;
   constexpr bool kBmn = kMode != kRawGU;
   extern __shared__ uint8_t smem_raw[];
@@ -135,10 +146,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   Ctl* ctl = reinterpret_cast<Ctl*>(sOut + kOutBytes);
   int32_t* off = reinterpret_cast<int32_t*>(sOut + kOutBytes + kCtlBytes);
   int32_t* ts = off + (kMaxE + 1);
+  // kWGrad over a pair of chunks: K runs over the expert's padded rows of the first chunk
+  // (offsets off, operands tmA/tmB), then of the second (off1, tmA1/tmB1)
+  int32_t* off1 = ts + (kMaxE + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int32_t E = p.E;
 
-  for (int32_t i = threadIdx.x; i <= E; i += kThreads) off[i] = p.offsets[i];
+  constexpr int kEpi = Cfg<kMode>::kEpi;
+  for (int32_t i = threadIdx.x; i <= E; i += Cfg<kMode>::kThreads) {
+    off[i] = p.offsets[i];
+    if (kMode == kWGrad) off1[i] = p.offsets1 ? p.offsets1[i] : 0;
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&ctl->full[s], 1);
@@ -146,7 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&ctl->tfull[b], 1);
-      mbar_init(&ctl->tempty[b], 4 * 32);
+      mbar_init(&ctl->tempty[b], kEpi * 32);
     }
     mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
@@ -162,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int32_t e0 = lane * per, e1 = min(E, e0 + per);
     auto tiles_of = [&](int32_t e) -> int32_t {
       const int32_t rows = off[e + 1] - off[e];
-      if (kMode == kWGrad) return rows > 0 ? p.m_tiles * p.n_tiles : 0;
+      if (kMode == kWGrad) return rows + off1[e + 1] - off1[e] > 0 ? p.m_tiles * p.n_tiles : 0;
       return ((rows + BM - 1) / BM) * p.n_tiles;
     };
     int32_t sum = 0;
@@ -194,7 +212,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int32_t L = blockIdx.x; L < p.total_tiles && ok; L += gridDim.x) {
         const Tile t = decode<kMode>(L, ts, off, E, p);
-        const int32_t nkb = kMode == kWGrad ? (off[t.e + 1] - off[t.e]) / BK : p.num_kb;
+        const int32_t nkb0 = (off[t.e + 1] - off[t.e]) / BK;
+        const int32_t nkb = kMode == kWGrad ? nkb0 + (off1[t.e + 1] - off1[t.e]) / BK : p.num_kb;
         for (int32_t kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort, p.status)) {
             ok = false;
@@ -205,11 +224,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* b = sB + stage * kBBytes;
           uint64_t* bar = &ctl->full[stage];
           if (kMode == kWGrad) {
-            const int32_t r0 = off[t.e] + kb * BK;  // K rows of this block
-            for (int q = 0; q < 2; ++q)
-              tma_load_2d(a + q * 8192, &tmA, bar, t.m * BM + q * 64, r0, pol);
-            for (int q = 0; q < 4; ++q)
-              tma_load_2d(b + q * 8192, &tmB, bar, t.n * BN + q * 64, r0, pol);
+            const bool seg0 = kb < nkb0;
+            const int32_t r0 = seg0 ? off[t.e] + kb * BK : off1[t.e] + (kb - nkb0) * BK;
+            const CUtensorMap* ma = seg0 ? &tmA : &tmA1;
+            const CUtensorMap* mb = seg0 ? &tmB : &tmB1;
+            for (int q = 0; q < 2; ++q) tma_load_2d(a + q * 8192, ma, bar, t.m * BM + q * 64, r0, pol);
+            for (int q = 0; q < 4; ++q) tma_load_2d(b + q * 8192, mb, bar, t.n * BN + q * 64, r0, pol);
           } else {
             const int32_t row0 = off[t.e] + t.m * BM;
             tma_load_2d(a, &tmA, bar, kb * BK, row0, pol);
@@ -243,7 +263,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int32_t it = 0;
       for (int32_t L = blockIdx.x; L < p.total_tiles && ok; L += gridDim.x, ++it) {
         const Tile t = decode<kMode>(L, ts, off, E, p);
-        const int32_t nkb = kMode == kWGrad ? (off[t.e + 1] - off[t.e]) / BK : p.num_kb;
+        const int32_t nkb = kMode == kWGrad
+                                ? (off[t.e + 1] - off[t.e] + off1[t.e + 1] - off1[t.e]) / BK
+                                : p.num_kb;
         const int buf = it & 1;
         if (!mbar_wait(&ctl->tempty[buf], ((it >> 1) & 1) ^ 1u, abort, p.status)) {
           ok = false;
@@ -281,7 +303,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {  // ---------------- epilogue (warps 2..5) ----------------
-    const int q = warp & 3;
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    // column half of this warp when two warps share a lane quarter
+    const int part = (warp - 2) >> 2;
+    constexpr int kParts = kEpi / 4;
+    constexpr int kC = BN / 32 / kParts;        // 32-column blocks per warp
+    constexpr int kCgu = BN / 2 / 32 / kParts;  // gate/up column-block pairs per warp
     const int r = q * 32 + lane;  // accumulator row (TMEM lane)
     int32_t it = 0;
     for (int32_t L = blockIdx.x; L < p.total_tiles; L += gridDim.x, ++it) {
@@ -306,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       };
-      if (kMode == kDSwiGLU) load_aux(0, gq, uq);
+      if (kMode == kDSwiGLU) load_aux(part * kC, gq, uq);
       if (!mbar_wait(&ctl->tfull[buf], (it >> 1) & 1, abort, p.status)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * BN;
@@ -318,9 +345,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // gets one store or add per chunk, in chunk order.
         uint8_t* box = sOut + q * kOutBoxBytes;
         const int32_t m0 = t.m * BM + q * 32;
-        const bool store = p.first[t.e] == p.chunk;
+        const bool store = p.first[t.e] >= p.chunk && p.first[t.e] <= p.chunk_last;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = part * kC; c < (part + 1) * kC; ++c) {
           uint32_t v[32];
           tmem_ld_32cols(t_row + c * 32, v);
           if (lane == 0) bulk_wait_read_all();  // the previous box has left shared memory
@@ -347,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t row = (int64_t)off[t.e] + t.m * BM + r;
         if (kMode == kRawGU) {
 #pragma unroll 1
-          for (int c = 0; c < (BN / 2) / 32; ++c) {
+          for (int c = part * kCgu; c < (part + 1) * kCgu; ++c) {
             uint32_t g[32], u[32];
             tmem_ld_32cols(t_row + c * 32, g);
             tmem_ld_32cols(t_row + BN / 2 + c * 32, u);
@@ -381,11 +408,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         } else {
 #pragma unroll 1
-          for (int c = 0; c < BN / 32; ++c) {
+          for (int c = part * kC; c < (part + 1) * kC; ++c) {
             uint32_t v[32];
             tmem_ld_32cols(t_row + c * 32, v);
             uint4 gn[4], un[4];
-            if (kMode == kDSwiGLU && c + 1 < BN / 32) load_aux(c + 1, gn, un);
+            if (kMode == kDSwiGLU && c + 1 < (part + 1) * kC) load_aux(c + 1, gn, un);
             tmem_ld_wait(v);
             const int32_t col0 = t.n * BN + c * 32;
             if (!row_ok) continue;
@@ -406,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float gv = h ? bf16hi(ga[i]) : bf16lo(ga[i]);
                     const float uv = h ? bf16hi(ua[i]) : bf16lo(ua[i]);
                     const float dh = __uint_as_float(v[v4 * 8 + 2 * i + h]);
-                    const float sig = 1.0f / (1.0f + __expf(-gv));
+                    const float sig = __fdividef(1.0f, 1.0f + __expf(-gv));
                     duv[h] = dh * gv * sig;
                     dgv[h] = dh * uv * (sig + gv * sig * (1.0f - sig));
                   }
@@ -546,13 +573,14 @@ __global__ void __launch_bounds__(kRowThreads)
 
 template <int kMode>
 cudaError_t launch_mode(const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mC,
-                        const BParams& p, int num_sms, cudaStream_t s) {
+                        const CUtensorMap& mA1, const CUtensorMap& mB1, const BParams& p,
+                        int num_sms, cudaStream_t s) {
   if (p.total_tiles <= 0) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(bwd_gemm_kernel<kMode>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
   if (e != cudaSuccess) return e;
   const int grid = p.total_tiles < num_sms ? p.total_tiles : num_sms;
-  bwd_gemm_kernel<kMode><<<grid, kThreads, kSmem, s>>>(mA, mB, mC, p);
+  bwd_gemm_kernel<kMode><<<grid, Cfg<kMode>::kThreads, kSmem, s>>>(mA, mB, mC, mA1, mB1, p);
   return cudaGetLastError();
 }
 
@@ -569,13 +597,14 @@ cudaError_t launch_bwd_gemm(const BwdGemmArgs& a, int num_sms, cudaStream_t s) {
   // N tiles: kRawGU pairs 128 gate with 128 up columns per tile; the others are 256 wide
   const int32_t n_tiles = a.mode == kRawGU ? (a.I + BN / 2 - 1) / (BN / 2) : (a.N + BN - 1) / BN;
   for (int32_t e = 0; e < a.E; ++e) {
-    const int64_t rows = a.rows_pad_host[e];
+    const int64_t rows =
+        a.rows_pad_host[e] + (a.mode == kWGrad && a.rows_pad_host1 ? a.rows_pad_host1[e] : 0);
     if (a.mode == kWGrad) tiles += rows > 0 ? (int64_t)((a.M + BM - 1) / BM) * n_tiles : 0;
     else tiles += (rows + BM - 1) / BM * n_tiles;
   }
   if (tiles <= 0) return cudaSuccess;
   if (tiles > 0x7fffffff) return cudaErrorInvalidValue;
-  CUtensorMap mA, mB, mC;
+  CUtensorMap mA, mB, mC, mA1, mB1;
   const bool a_mn = a.mode == kWGrad;
   const bool b_mn = a.mode != kRawGU;
   if (!make_tma_2d_bf16(&mA, a.A, a.A_rows, a.A_cols, a_mn ? BK : BM) ||
@@ -586,6 +615,16 @@ cudaError_t launch_bwd_gemm(const BwdGemmArgs& a, int num_sms, cudaStream_t s) {
       return cudaErrorInvalidValue;
   } else {
     mC = mA;  // unused
+  }
+  const bool pair = a.mode == kWGrad && a.offsets1 != nullptr;
+  if (pair) {
+    if (!a.A1 || !a.B1 || !a.rows_pad_host1 ||
+        !make_tma_2d_bf16(&mA1, a.A1, a.A1_rows, a.A_cols, BK) ||
+        !make_tma_2d_bf16(&mB1, a.B1, a.B1_rows, a.B_cols, BK))
+      return cudaErrorInvalidValue;
+  } else {
+    mA1 = mA;  // unused
+    mB1 = mB;
   }
   BParams p;
   p.offsets = a.offsets;
@@ -605,11 +644,13 @@ cudaError_t launch_bwd_gemm(const BwdGemmArgs& a, int num_sms, cudaStream_t s) {
   p.acc = a.acc;
   p.first = a.first;
   p.chunk = a.chunk;
+  p.chunk_last = pair ? a.chunk + 1 : a.chunk;
+  p.offsets1 = pair ? a.offsets1 : nullptr;
   switch (a.mode) {
-    case kRawGU: return launch_mode<kRawGU>(mA, mB, mC, p, num_sms, s);
-    case kDSwiGLU: return launch_mode<kDSwiGLU>(mA, mB, mC, p, num_sms, s);
-    case kDPlain: return launch_mode<kDPlain>(mA, mB, mC, p, num_sms, s);
-    case kWGrad: return launch_mode<kWGrad>(mA, mB, mC, p, num_sms, s);
+    case kRawGU: return launch_mode<kRawGU>(mA, mB, mC, mA1, mB1, p, num_sms, s);
+    case kDSwiGLU: return launch_mode<kDSwiGLU>(mA, mB, mC, mA1, mB1, p, num_sms, s);
+    case kDPlain: return launch_mode<kDPlain>(mA, mB, mC, mA1, mB1, p, num_sms, s);
+    case kWGrad: return launch_mode<kWGrad>(mA, mB, mC, mA1, mB1, p, num_sms, s);
   }
   return cudaErrorInvalidValue;
 }

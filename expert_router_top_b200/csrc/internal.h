@@ -110,7 +110,16 @@ struct BwdGemmArgs {
   const void* aux;
   float* acc;                  // kBwdWGrad: [E][M][N] fp32 gradient
   const int32_t* first;        // kBwdWGrad: dev [E] first chunk with rows of each expert
-  int32_t chunk;               // kBwdWGrad: this chunk (store where first == chunk, else add)
+  int32_t chunk;               // kBwdWGrad: this chunk (store where first is this launch's
+                               // chunk or its pair's second chunk, else add)
+  // kBwdWGrad over a pair of chunks (null offsets1: one chunk): the second chunk's operands,
+  // rows, padded offsets (dev [E+1]) and padded rows per expert (host [E])
+  const void* A1;
+  int64_t A1_rows;
+  const void* B1;
+  int64_t B1_rows;
+  const int32_t* offsets1;
+  const int32_t* rows_pad_host1;
   uint32_t* status;
 };
 

@@ -993,8 +993,8 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
       return MOE_ERR_CUDA;
     return MOE_OK;
   };
-  // Bk(c), stream G: dh with the SwiGLU backward, dX, then both weight gradients
-  auto Bk = [&](int c) -> moe_status_t {
+  // Bd(c), stream G: dh with the SwiGLU backward, then dX
+  auto Bd = [&](int c) -> moe_status_t {
     if (!ok(cudaStreamWaitEvent(sg, ctx->ev_bdy[c % 2], 0))) return MOE_ERR_CUDA;
     BwdGemmArgs g = g0;
     g.offsets = offp_c(c);
@@ -1011,16 +1011,43 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
     g.N = H, g.K = 2 * I, g.b_rows = 2 * I, g.out0 = buf(B.ydx, c), g.aux = nullptr;
     if (!ok(bwd_gemm(MOE_KERNEL_BWD_DX, g, c)) || !ok(cudaEventRecord(ctx->ev_bdx[c % 2], sg)))
       return MOE_ERR_CUDA;
-    // dW_down[e] (+)= dY^T h ;  dW_gate_up[e] (+)= [dg du]^T X
+    return MOE_OK;
+  };
+  // W(c, c1), stream G: both weight gradients over the rows of chunk c and, when c1 > c,
+  // of chunk c1 = c + 1 in the same GEMM (K runs over both chunks' rows of each expert):
+  //   dW_down[e] (+)= dY^T h ;  dW_gate_up[e] (+)= [dg du]^T X
+  // An expert's first chunk with rows stores; later launches add.
+  auto W = [&](int c, int c1) -> moe_status_t {
+    BwdGemmArgs g = g0;
+    g.offsets = offp_c(c);
+    g.rows_pad_host = rows_pad.data() + (size_t)c * E;
+    g.chunk = c;
+    if (c1 > c) {
+      g.offsets1 = offp_c(c1);
+      g.rows_pad_host1 = rows_pad.data() + (size_t)c1 * E;
+      g.A1_rows = g.B1_rows = R[c1];
+    }
+    const int64_t rows_both = R[c] + (c1 > c ? R[c1] : 0);
+    std::vector<int32_t> both(counts.begin() + (size_t)c * E, counts.begin() + (size_t)c * E + E);
+    if (c1 > c)
+      for (int32_t e = 0; e < E; ++e) both[e] += counts[(size_t)c1 * E + e];
+    const int64_t active = active_experts(both.data(), E);
+    auto launch = [&](const BwdGemmArgs& a) {
+      ProfScope ps(MOE_KERNEL_BWD_WGRAD, sg, rows_both, active, 1);
+      return launch_bwd_gemm(a, ctx->num_sms, sg);
+    };
     g.mode = kBwdWGrad;
     g.A = buf(B.dy, c), g.A_rows = R[c], g.A_cols = H;
     g.B = buf(B.act, c), g.B_rows = R[c], g.B_cols = I;
+    if (c1 > c) g.A1 = buf(B.dy, c1), g.B1 = buf(B.act, c1);
     g.M = H, g.N = I, g.acc = dW_down, g.out0 = nullptr;
-    if (!ok(bwd_gemm(MOE_KERNEL_BWD_WGRAD, g, c))) return MOE_ERR_CUDA;
+    if (!ok(launch(g))) return MOE_ERR_CUDA;
     g.A = buf(B.dgu, c), g.A_rows = R[c], g.A_cols = 2 * I;
     g.B = x_of(c), g.B_rows = R[c], g.B_cols = H;
+    if (c1 > c) g.A1 = buf(B.dgu, c1), g.B1 = x_of(c1);
     g.M = 2 * I, g.N = H, g.acc = dW_gate_up;
-    if (!ok(bwd_gemm(MOE_KERNEL_BWD_WGRAD, g, c)) || !ok(cudaEventRecord(ctx->ev_bw[c % 3], sg)))
+    if (!ok(launch(g)) || !ok(cudaEventRecord(ctx->ev_bw[c % 3], sg)) ||
+        (c1 > c && !ok(cudaEventRecord(ctx->ev_bw[c1 % 3], sg))))
       return MOE_ERR_CUDA;
     return MOE_OK;
   };
@@ -1034,20 +1061,28 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
     return MOE_OK;
   };
 
-  // The mirrored pair pipeline.  G: F(0) F(1) B(0) F(2) B(1) F(3) ... B(n-1);
-  // M: P(0) P(1) DY(0) P(2) S(0) DY(1) P(3) S(1) ...  Chunk c+2's permute overlaps chunk c's
-  // GEMMs and every row kernel after the first permute overlaps a neighbouring chunk's GEMMs.
-  // Host enqueue order keeps each event wait on the record it is meant for.
+  // The mirrored pair pipeline, over pairs of adjacent chunks (c0, c1) = (2m, 2m+1):
+  //   G: F(c0) F(c1) Bd(c0) Bd(c1) W(c0,c1) F(c0+2) F(c1+2) ...
+  //   M: P(c0) P(c1) DY(c0) DY(c1) S(c0) S(c1) P(c0+2) P(c1+2) ...
+  // The row kernels of one chunk overlap the GEMMs of the other chunk of the pair or of the
+  // next pair, and the weight gradients of a pair are one GEMM per weight (half the dW
+  // read-modify-write passes of per-chunk launches).  Host enqueue order keeps each event
+  // wait on the record it is meant for.
   if (!ok(cudaEventRecord(ctx->ev_start, s)) || !ok(cudaStreamWaitEvent(sg, ctx->ev_start, 0)))
     return MOE_ERR_CUDA;
   if (n_live > 0) {
     if ((st = P(0)) != MOE_OK || (st = F(0)) != MOE_OK) return st;
     if (n_live > 1 && ((st = P(1)) != MOE_OK || (st = F(1)) != MOE_OK)) return st;
-    for (int c = 0; c < n_live; ++c) {
-      if ((st = DY(c)) != MOE_OK) return st;
-      if (c + 2 < n_live && (st = P(c + 2)) != MOE_OK) return st;
-      if ((st = Bk(c)) != MOE_OK || (st = S(c)) != MOE_OK) return st;
-      if (c + 2 < n_live && (st = F(c + 2)) != MOE_OK) return st;
+    for (int c0 = 0; c0 < n_live; c0 += 2) {
+      const int c1 = c0 + 1 < n_live ? c0 + 1 : c0;
+      if ((st = DY(c0)) != MOE_OK || (c1 > c0 && (st = DY(c1)) != MOE_OK)) return st;
+      if ((st = Bd(c0)) != MOE_OK || (c1 > c0 && (st = Bd(c1)) != MOE_OK)) return st;
+      if ((st = S(c0)) != MOE_OK || (c1 > c0 && (st = S(c1)) != MOE_OK)) return st;
+      if (c0 + 2 < n_live && (st = P(c0 + 2)) != MOE_OK) return st;
+      if ((st = W(c0, c1)) != MOE_OK) return st;
+      if (c0 + 3 < n_live && (st = P(c0 + 3)) != MOE_OK) return st;
+      if (c0 + 2 < n_live && (st = F(c0 + 2)) != MOE_OK) return st;
+      if (c0 + 3 < n_live && (st = F(c0 + 3)) != MOE_OK) return st;
     }
   }
   if (!ok(cudaEventRecord(ctx->ev_join, sg)) || !ok(cudaStreamWaitEvent(s, ctx->ev_join, 0)))

@@ -7,16 +7,17 @@ from gen import LayerConfig
 
 
 def test_backward_units_hand_worked():
-    """Two chunks, two experts: counts [[1, 0], [2, 3]].  Expert 0 has rows in both chunks
-    (stored by chunk 0, read and written by chunk 1), expert 1 only in chunk 1 (stored)."""
+    """Three chunks, two experts: counts [[1, 0], [2, 3], [0, 4]].  The weight gradients run
+    per pair of chunks, (0, 1) then (2): the first pair stores dW of both experts, the
+    second reads and writes expert 1's."""
     cfg = LayerConfig("u", T=3, H=64, E=2, k=2, I=32, routing="normal")
-    u = bench.backward_units(cfg, np.array([[1, 0], [2, 3]], np.int32))
+    u = bench.backward_units(cfg, np.array([[1, 0], [2, 3], [0, 4]], np.int32))
     H, I = 64, 32
-    rows = 6
+    rows = 10
     assert u["flops"]["bwd_wgrad"] == 6 * rows * H * I
     assert sum(u["flops"].values()) == 18 * rows * H * I
     operands = rows * (2 * H + 3 * I) * 2
-    dw = 12 * H * I * (3 + 1)  # 3 (chunk, expert) stores or adds written, 1 of them also read
+    dw = 12 * H * I * (3 + 1)  # 3 (pair, expert) stores or adds written, 1 of them also read
     assert u["wgrad_bytes"] == pytest.approx(operands + dw)
 
 
