@@ -152,8 +152,10 @@ def make_inputs(cfg, device, seed=0, weights=True):
     return out
 
 
-def algorithmic_units(cfg, counts, n_live):
-    """Per-kernel algorithmic work of one step (bytes or flops), from the chunk counts."""
+def algorithmic_units(cfg, counts, n_live, dispatch="separate"):
+    """Per-kernel algorithmic work of one step (bytes or flops), from the chunk counts.
+    With the fused dispatch the gate/up GEMM reads each token row of `hidden` (T rows)
+    instead of the T*k permuted rows."""
     H, I, k, T = cfg.H, cfg.I, cfg.k, cfg.T
     rows = int(counts.sum())
     active = int((counts > 0).sum())  # (chunk, expert) pairs with rows: weights streamed
@@ -169,7 +171,8 @@ def algorithmic_units(cfg, counts, n_live):
         "down_weight_bytes": active * H * I * 2,
         # gate/up kernel, whole step: W_gate_up of each chunk's active experts (re-read per
         # chunk), permuted rows read, Act written
-        "gateup_alg_bytes": active * 2 * I * H * 2 + rows * H * 2 + rows * I * 2,
+        "gateup_alg_bytes": active * 2 * I * H * 2 + (T if dispatch == "fused" else rows) * H * 2
+        + rows * I * 2,
     }
 
 
@@ -178,15 +181,15 @@ def gemm_src_hash():
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def traffic_per_launch(cfg_name, chunks):
+def traffic_per_launch(cfg_name, chunks, dispatch):
     """DRAM bytes per gate/up launch from the committed ncu summary, if it was taken on
-    the current kernel source, this workload and this chunking; else None."""
+    the current kernel source, this workload, this chunking and this dispatch; else None."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
     with open(TRAFFIC_FILE) as f:
         d = json.load(f)
     if (d.get("gemm_src_sha256_16") != gemm_src_hash() or d.get("num_chunks") != chunks
-            or d.get("config") != cfg_name):
+            or d.get("config") != cfg_name or d.get("dispatch") != dispatch):
         return None
     return d.get("dram_bytes_per_launch_full_size")
 
@@ -264,7 +267,7 @@ def run_reference(args, cfg):
     return 0
 
 
-def config_block(cfg, chunks, dispatch="separate"):
+def config_block(cfg, chunks, dispatch="auto"):
     wbytes = 6 * cfg.E * cfg.H * cfg.I
     return {"workload": workload_name(cfg), "T": cfg.T, "H": cfg.H, "E": cfg.E, "k": cfg.k,
             "I": cfg.I, "ep_groups": cfg.G, "num_chunks": chunks, "dispatch": dispatch,
@@ -275,7 +278,7 @@ def config_block(cfg, chunks, dispatch="separate"):
 
 # ------------------------------------------------------------------------- our arm
 
-def time_steps(moe, inp, cfg, chunks, ws, steps, stream, dispatch="separate"):
+def time_steps(moe, inp, cfg, chunks, ws, steps, stream, dispatch="auto"):
     """Device time of `steps` back-to-back forward calls, ms (CUDA events on `stream`)."""
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
@@ -315,7 +318,9 @@ def run_ours(args, cfg):
     meta = moe.metadata(inp["idx"], cfg.E, cfg.G, chunks)
     counts = meta["counts"]
     n_live = int((np.diff(meta["bounds"]) > 0).sum())
-    units = algorithmic_units(cfg, counts, n_live)
+    dispatch = moe.forward_dispatch(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, args.dispatch, cfg.G,
+                                    chunks)
+    units = algorithmic_units(cfg, counts, n_live, dispatch)
     active_per_chunk = (counts > 0).sum(1)
     weight_stream = float(active_per_chunk.sum()) * 6 * cfg.H * cfg.I  # bytes, all chunks
 
@@ -386,7 +391,7 @@ def run_ours(args, cfg):
     peak_tc, peak_bw = peaks["bf16_tflops"], peaks["hbm_gbs"]
     t_tensor = gu_flops_l / (peak_tc * 1e12)
     t_mem = gu_bytes_l / (peak_bw * 1e9)
-    traffic = traffic_per_launch(cfg.name, chunks)
+    traffic = traffic_per_launch(cfg.name, chunks, dispatch)
     if t_mem > t_tensor:
         roofline = {"bound": "hbm", "achieved": gu_bytes_l / t_l / 1e9 if t_l else 0.0,
                     "peak": peak_bw, "unit": "GB/s"}
@@ -396,7 +401,8 @@ def run_ours(args, cfg):
     roofline["frac"] = roofline["achieved"] / roofline["peak"]
     roofline.update({
         "traffic": traffic,
-        "kernel": "grouped_gemm_kernel<gate/up + SwiGLU> (tcgen05)",
+        "kernel": "grouped_gemm_kernel<gate/up + SwiGLU" + (", gathered A rows" if dispatch == "fused"
+                                                             else "") + "> (tcgen05)",
         "peak_source": f"{peak_src}: MEASURED_PEAKS.json (bf16 burst, HBM copy)",
         "per_launch": {"flops": gu_flops_l, "bytes": gu_bytes_l, "ms": t_l * 1e3,
                        "roofline_ms": max(t_tensor, t_mem) * 1e3},
@@ -412,7 +418,7 @@ def run_ours(args, cfg):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; random-init expert weights of the layer's shape)",
-        "config": config_block(cfg, chunks, args.dispatch),
+        "config": config_block(cfg, chunks, dispatch),
         "roofline": roofline,
         "grouped_gemm_tflops": gemm_tflops,
         "grouped_gemm_frac_of_peak": gemm_tflops / peak_tc,
@@ -632,9 +638,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", choices=sorted(CONFIGS), default=DEFAULT_CONFIG)
     ap.add_argument("--chunks", type=int, default=DEFAULT_CHUNKS)
-    ap.add_argument("--dispatch", choices=["separate", "fused"], default="separate",
+    ap.add_argument("--dispatch", choices=["auto", "separate", "fused"], default="auto",
                     help="separate: permute kernel first; fused: the gate/up GEMM gathers its "
-                         "rows from hidden")
+                         "rows from hidden; auto: the library's choice for the shape")
     ap.add_argument("--pass", dest="pass_", choices=["forward", "backward", "train"],
                     default="forward",
                     help="forward (the layer's headline), backward (moe_backward alone) or "

@@ -84,6 +84,8 @@ def load():
     L.moe_forward_ex.argtypes = [ctypes.POINTER(Shape), p, p, p, p, p, p, p, sz, ctypes.c_uint32,
                                  p]
     L.moe_forward_ex.restype = st
+    L.moe_forward_dispatch.argtypes = [ctypes.POINTER(Shape), ctypes.c_uint32]
+    L.moe_forward_dispatch.restype = i32
     L.moe_workspace_bytes_host.argtypes = [ctypes.POINTER(Shape)]
     L.moe_workspace_bytes_host.restype = sz
     L.moe_forward_host.argtypes = [ctypes.POINTER(Shape), p, p, p, p, p, p, p, sz, p]
@@ -221,20 +223,37 @@ def metadata(top_k_index: torch.Tensor, E: int, ep_groups: int = 1, num_chunks: 
 
 
 FWD_FUSED_DISPATCH = 1
+FWD_SEPARATE_DISPATCH = 2
+_DISPATCH = {"auto": 0, "fused": FWD_FUSED_DISPATCH, "separate": FWD_SEPARATE_DISPATCH}
+
+
+def _dispatch_flags(dispatch):
+    if dispatch not in _DISPATCH:
+        raise ValueError(f"dispatch must be one of {sorted(_DISPATCH)}, not {dispatch!r}")
+    return _DISPATCH[dispatch]
+
+
+def forward_dispatch(T, H, I, E, k, dispatch="auto", ep_groups=1, num_chunks=1) -> str:
+    """The dispatch ("fused" or "separate") that forward() takes for this shape."""
+    s = shape(T, H, I, E, k, ep_groups, num_chunks, 0)
+    r = int(load().moe_forward_dispatch(ctypes.byref(s), _dispatch_flags(dispatch)))
+    if r < 0:
+        raise ValueError("invalid dispatch flags")
+    return "fused" if r == 1 else "separate"
 
 
 def forward(hidden, top_k_index, top_k_weights, W_gate_up, W_down, num_chunks: int = 1,
             ep_groups: int = 1, out=None, workspace=None, stream=None,
-            dispatch: str = "separate", chunk_size: int = 0):
+            dispatch: str = "auto", chunk_size: int = 0):
     """One MoE layer forward, chunked as Chunk MoE.  Returns out [T,H] bf16.
 
     hidden [T,H] bf16, top_k_index [T,k] int32, top_k_weights [T,k] fp32,
     W_gate_up [E,2I,H] bf16 (gate rows then up rows), W_down [E,H,I] bf16; all on the
     same CUDA device.  Asynchronous after its single metadata copy.
     dispatch="separate": a permute kernel writes the permuted rows first; "fused": the
-    gate/up GEMM gathers its rows from `hidden`.  Both give identical bits."""
-    if dispatch not in ("fused", "separate"):
-        raise ValueError(f"dispatch must be 'fused' or 'separate', not {dispatch!r}")
+    gate/up GEMM gathers its rows from `hidden`; "auto": the library's choice for the
+    shape (forward_dispatch).  All give identical bits."""
+    _dispatch_flags(dispatch)
     _need(hidden, torch.bfloat16, "hidden")
     _need(top_k_index, torch.int32, "top_k_index")
     _need(top_k_weights, torch.float32, "top_k_weights")
@@ -252,7 +271,7 @@ def forward(hidden, top_k_index, top_k_weights, W_gate_up, W_down, num_chunks: i
         out = torch.empty((T, H), dtype=torch.bfloat16, device=hidden.device)
     if workspace is None:
         workspace = alloc_workspace(load().moe_workspace_bytes(ctypes.byref(s)), hidden.device)
-    flags = FWD_FUSED_DISPATCH if dispatch == "fused" else 0
+    flags = _dispatch_flags(dispatch)
     _check(load().moe_forward_ex(ctypes.byref(s), _ptr(hidden), _ptr(top_k_index),
                                  _ptr(top_k_weights), _ptr(W_gate_up), _ptr(W_down), _ptr(out),
                                  _ptr(workspace), workspace.numel(), flags, _stream(stream)),

@@ -112,6 +112,9 @@ struct KParams {
   int32_t up_off;    // row offset of W_up inside one expert's W_gate_up (= I)
   int32_t total_tiles;
   const int32_t* gather;  // gathered A: token row of each permuted row (nullptr: plain A)
+  const uint8_t* gsrc;    // gathered A: the token rows (hidden), and their stride in bytes
+  int64_t gsrc_stride;
+  int32_t K;              // gathered A: valid K columns (the rest of the last block reads 0)
   int32_t reverse;        // 1: walk the tiles (hence the experts) in descending order
   int32_t b4d;            // 1: tmB is the 4-D gate/up view (one box per stage)
 };
@@ -243,10 +246,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   const int32_t n_streams = kPair ? (int32_t)(gridDim.x >> 1) : (int32_t)gridDim.x;
 
   // ---- set-up: expert offsets, tile prefix, barriers, TMEM ----
-  for (int32_t i = threadIdx.x; i <= E; i += kGemmThreads) off[i] = p.offsets[i];
+  for (int32_t i = threadIdx.x; i <= E; i += blockDim.x) off[i] = p.offsets[i];
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&ctl->full[s], 1);
+      // gathered A: the weight producer's arrival plus one per A-gathering thread
+      mbar_init(&ctl->full[s], kGather ? 1 + kGatherThreads : 1);
       mbar_init(&ctl->empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -299,56 +303,97 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   volatile int* abort = &ctl->abort;
 
   if (warp == 0 && kGather) {
-    // ---------------- TMA producer, gathered A (whole warp) ----------------
-    // Lane l gathers rows 4l..4l+3 of the tile straight from the source rows (tile::gather4,
-    // a box one row high); lane 0 also waits for the stage, arms it and loads the weights.
-    const uint64_t pol_w = l2_policy_evict_last();
-    const uint64_t pol_a = l2_policy_evict_normal();
+    // ---------------- weight producer, gathered A (lane 0) ----------------
+    // The A rows of a stage come from the gathering warps (below); this lane arms the stage
+    // with the weight bytes and loads the weight box(es) with TMA.
+    if (lane == 0) {
+      const uint64_t pol_w = l2_policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_parity = 0;
+      bool ok = true;
+      for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
+        const Tile t = decode_tile<G::kTileM>(p.reverse ? p.total_tiles - 1 - L : L, tile_start,
+                                              off, E, p.n_tiles);
+        const int32_t brow = t.e * p.b_rows + t.n * (kSwiGLU ? BN / 2 : BN);
+        for (int32_t kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&ctl->full[stage], G::kBBytes);
+          uint8_t* b_dst = sB + stage * G::kBBytes;
+          tma_load_2d(b_dst, tmB, &ctl->full[stage], kb * BK, brow, pol_w);
+          if (kSwiGLU)
+            tma_load_2d(b_dst + G::kBBytes / 2, tmB, &ctl->full[stage], kb * BK, brow + p.up_off,
+                        pol_w);
+          armed |= 1u << stage;
+          armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok)
+        for (int s = 0; s < STAGES; ++s)
+          if (armed & (1u << s)) mbar_drain(&ctl->full[s], (armed_parity >> s) & 1u, 100000000ull);
+    }
+  } else if (kGather && warp >= kGemmThreads / 32) {
+    // ---------------- A producers, gathered rows (4 warps, LSU) ----------------
+    // The tile's 128 A rows are the token rows src_tok[row] of `hidden`.  Per K block, lane
+    // (8 s + j) of gathering warp w copies 16-byte chunk j of rows 32 w + 4 i + s (i < 8) with
+    // cp.async, into the 128-byte-swizzled K-major layout the MMA reads (chunk j of row r at
+    // position j ^ (r % 8)); a warp instruction covers 4 whole 128-byte row segments.  A
+    // thread keeps kDepth + 1 stages of copies in flight; when its oldest stage has landed it
+    // makes the writes visible to the async proxy and arrives on that stage's full barrier.
+    constexpr int kDepth = STAGES - 2;
+    const int gw = warp - kGemmThreads / 32, j = lane & 7, sub = lane >> 3;
     int stage = 0;
     uint32_t phase = 0;
-    uint32_t armed = 0, armed_parity = 0;
+    int32_t issued = 0, arrived = 0;
     bool ok = true;
     for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
       const Tile t = decode_tile<G::kTileM>(p.reverse ? p.total_tiles - 1 - L : L, tile_start,
                                             off, E, p.n_tiles);
       const int32_t row0 = off[t.e] + t.m * G::kTileM;
-      const int32_t last = off[t.e + 1] - 1;  // rows past the expert reuse its last row
-      int32_t src[4];
+      const int32_t last = off[t.e + 1] - 1;  // rows past the expert re-read its last row
+      const uint8_t* src[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) src[i] = p.gather[min(row0 + 4 * lane + i, last)];
-      const int32_t brow = t.e * p.b_rows + t.n * (BN / 2);
+      for (int i = 0; i < 8; ++i) {
+        const int32_t r = gw * 32 + 4 * i + sub;
+        src[i] = p.gsrc + (int64_t)p.gather[min(row0 + r, last)] * p.gsrc_stride + j * 16;
+      }
       for (int32_t kb = 0; kb < p.num_kb; ++kb) {
-        int go = 1;
-        if (lane == 0) {
-          if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort, p.status)) go = 0;
-          if (go) {
-            mbar_arrive_expect_tx(&ctl->full[stage], G::kTxBytes);
-            uint8_t* b_dst = sB + stage * G::kBBytes;
-            tma_load_2d(b_dst, tmB, &ctl->full[stage], kb * BK, brow, pol_w);
-            if (kSwiGLU)
-              tma_load_2d(b_dst + G::kBBytes / 2, tmB, &ctl->full[stage], kb * BK,
-                          brow + p.up_off, pol_w);
-          }
-        }
-        go = __shfl_sync(0xffffffffu, go, 0);  // also orders the gathers after the wait
-        if (!go) {
+        if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort, p.status)) {
           ok = false;
           break;
         }
-        tma_gather4(sA + stage * G::kABytes + lane * 4 * (BK * 2), tmA, &ctl->full[stage],
-                    kb * BK, src[0], src[1], src[2], src[3], pol_a);
-        armed |= 1u << stage;
-        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+        const uint32_t a = smem_u32(sA + stage * G::kABytes);
+        const uint32_t nbytes = (kb * BK + j * 8 < p.K) ? 16u : 0u;  // zero past K
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int32_t r = gw * 32 + 4 * i + sub;
+          cp_async_16(a + r * (BK * 2) + ((j ^ (r & 7)) << 4), src[i] + kb * (BK * 2), nbytes);
+        }
+        cp_async_commit();
+        ++issued;
+        if (issued - arrived > kDepth) {
+          cp_async_wait<kDepth>();
+          fence_async_smem();
+          mbar_arrive(&ctl->full[arrived % STAGES]);
+          ++arrived;
+        }
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1u;
         }
       }
     }
-    if (!ok && lane == 0) {
-      for (int s = 0; s < STAGES; ++s)
-        if (armed & (1u << s)) mbar_drain(&ctl->full[s], (armed_parity >> s) & 1u, 100000000ull);
-    }
+    cp_async_wait<0>();
+    fence_async_smem();
+    for (; arrived < issued; ++arrived) mbar_arrive(&ctl->full[arrived % STAGES]);
+    (void)ok;
   } else if (warp == 0) {
     // ---------------- TMA producer (both CTAs) ----------------
     if (lane == 0) {
@@ -488,7 +533,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
         mbar_drain(&ctl->drain, 0, 100000000ull);
       }
     }
-  } else {
+  } else if (warp < kGemmThreads / 32) {
     // ---------------- epilogue (warps 2..5 of both CTAs) ----------------
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int r = q * 32 + lane;
@@ -559,7 +604,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
 }
 
 template <bool kSwiGLU, bool kGather>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kGather ? kGemmThreads + kGatherThreads : kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, const KParams p) {
   gemm_body<kSwiGLU, false, kGather>(&tmA, &tmB, p);
@@ -675,7 +720,8 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
     *err_detail = 1;
     return cudaErrorInvalidValue;
   }
-  const bool map_a_ok = gather ? make_map(&mA, a.gather_src, a.gather_src_rows, a.K, 1)
+  // (gathered A is copied by the gathering warps; its map is built but unused)
+  const bool map_a_ok = gather ? make_map(&mA, a.gather_src, a.gather_src_rows, a.K, kRowsPerCta)
                                : make_map(&mA, a.A, a.rows, a.K, kRowsPerCta);
   // one-box gate/up weights (single-CTA, plain A, I a multiple of 128)
   const bool b4d = MOE_GEMM_B4D && swiglu && !kPair && !gather && a.out_cols % 128 == 0 &&
@@ -703,6 +749,9 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
   p.up_off = swiglu ? a.out_cols : 0;
   p.total_tiles = (int32_t)a.total_tiles;
   p.gather = a.gather;
+  p.gsrc = static_cast<const uint8_t*>(a.gather_src);
+  p.gsrc_stride = (int64_t)a.K * 2;
+  p.K = a.K;
   p.reverse = a.reverse ? 1 : 0;
   p.b4d = b4d ? 1 : 0;
   constexpr size_t smem = smem_bytes<kPair>();
@@ -744,7 +793,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int streams = (int)(a.total_tiles < num_sms ? a.total_tiles : num_sms);
-    k<<<streams, kGemmThreads, smem, s>>>(mA, mB, p);
+    k<<<streams, gather ? kGemmThreads + kGatherThreads : kGemmThreads, smem, s>>>(mA, mB, p);
   }
   return cudaGetLastError();
 }

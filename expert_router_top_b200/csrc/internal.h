@@ -47,6 +47,7 @@ cudaError_t launch_unpermute(const void* Y, const int32_t* dst, const float* w, 
 constexpr int kGemmBM = 128;     // rows per tile (one tcgen05.mma M=128 per CTA)
 constexpr int kGemmBN = 256;     // MMA N: 128 gate + 128 up columns, or 256 down columns
 constexpr int kGemmThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int kGatherThreads = 128;  // gathered A: warps 6-9 copy the token rows
 
 struct GemmArgs {
   const void* A;          // [rows][K] bf16 (permuted X, or Act)

@@ -523,6 +523,17 @@ moe_status_t moe_metadata_shape(const moe_shape_t* shape, const int32_t* top_k_i
                        dst_rows, src_tokens, workspace, ws_bytes, stream);
 }
 
+int32_t moe_forward_dispatch(const moe_shape_t* shape, uint32_t flags) {
+  const uint32_t both = MOE_FWD_FUSED_DISPATCH | MOE_FWD_SEPARATE_DISPATCH;
+  if ((flags & ~both) || (flags & both) == both || !shape) return -1;
+  if (!gemm_supports_gather() || (flags & MOE_FWD_SEPARATE_DISPATCH)) return 0;
+  if (flags & MOE_FWD_FUSED_DISPATCH) return 1;
+  if (check_shape(shape) != MOE_OK) return 0;
+  const Dims d = make_dims(shape->T, shape->k, shape->E, shape->ep_groups, shape->num_chunks,
+                           shape->chunk_size);
+  return 4 * d.t_chunk * d.k >= (int64_t)d.E * shape->I ? 1 : 0;
+}
+
 moe_status_t moe_forward(const moe_shape_t* shape, const void* hidden, const int32_t* top_k_index,
                          const float* top_k_weights, const void* W_gate_up, const void* W_down,
                          void* out, void* workspace, size_t ws_bytes, void* stream) {
@@ -534,13 +545,14 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
                             const int32_t* top_k_index, const float* top_k_weights,
                             const void* W_gate_up, const void* W_down, void* out,
                             void* workspace, size_t ws_bytes, uint32_t flags, void* stream) {
-  if (flags & ~MOE_FWD_FUSED_DISPATCH) return MOE_ERR_ARG;
   moe_status_t st = check_shape(shape);
   if (st != MOE_OK) return st;
+  const int32_t choice = moe_forward_dispatch(shape, flags);
+  if (choice < 0) return MOE_ERR_ARG;
   const int64_t T = shape->T;
   const int32_t H = shape->H, I = shape->I, E = shape->E, k = shape->k;
   if (T == 0) return MOE_OK;
-  const bool fused = (flags & MOE_FWD_FUSED_DISPATCH) && gemm_supports_gather();
+  const bool fused = choice == 1;
   if (!hidden || !top_k_index || !top_k_weights || !W_gate_up || !W_down || !out || !workspace)
     return MOE_ERR_ARG;
   if (!aligned(hidden, 16) || !aligned(out, 16) || !aligned(W_gate_up, 16) ||

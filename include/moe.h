@@ -45,7 +45,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 3
+#define MOE_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define MOE_API __attribute__((visibility("default")))
@@ -227,23 +227,30 @@ MOE_API moe_status_t moe_forward(const moe_shape_t* shape, const void* hidden, c
                          void* out, void* workspace, size_t ws_bytes, void* stream);
 
 /* Flags of moe_forward_ex. */
-#define MOE_FWD_FUSED_DISPATCH 1u /* gather the gate/up GEMM's rows from hidden; no permute */
+#define MOE_FWD_FUSED_DISPATCH 1u    /* gather the gate/up GEMM's rows from hidden; no permute */
+#define MOE_FWD_SEPARATE_DISPATCH 2u /* permute kernel first, as the article's permute step */
 
-/* moe_forward with a choice of dispatch.  flags = 0 (what moe_forward does): the permute
- * kernel writes the permuted rows (the article's separate permute step) and the pipeline
- * overlaps the permute of chunk c+1 and the unpermute of chunk c-1 with the expert GEMMs
- * of chunk c.  flags = MOE_FWD_FUSED_DISPATCH: the gate/up GEMM loads each permuted row
- * straight from `hidden` (TMA row gathers through the permutation's inverse map), so no
- * permuted copy of the input is written or read, and the pipeline overlaps the unpermute
- * of chunk c with the expert GEMMs of chunk c+1; on B200 the row gathers currently make
- * the gate/up GEMM slower than the permute they replace.  Both give bit-identical
- * outputs; arguments, workspace and errors are as moe_forward (unknown flag bits:
- * MOE_ERR_ARG). */
+/* moe_forward with a choice of dispatch.  MOE_FWD_SEPARATE_DISPATCH: the permute kernel
+ * writes the permuted rows (the article's separate permute step) and the pipeline overlaps
+ * the permute of chunk c+1 and the unpermute of chunk c-1 with the expert GEMMs of chunk c.
+ * MOE_FWD_FUSED_DISPATCH: the gate/up GEMM copies each permuted row's K blocks straight from
+ * `hidden` through the permutation's inverse map (four gathering warps per CTA), so no
+ * permuted copy of the input is written or read, and the pipeline overlaps the unpermute of
+ * chunk c with the expert GEMMs of chunk c+1.  flags = 0 (what moe_forward does) chooses
+ * fused when a chunk holds at least I/4 rows per expert on average (4 * T_chunk * k >= E * I):
+ * the permuted copy it saves is then a sizeable share of the GEMMs' memory traffic, which
+ * the expert weights dominate otherwise (there the gathers cost more than they save).
+ * Every choice gives bit-identical outputs; arguments, workspace and errors are as
+ * moe_forward (unknown flag bits, or both flags: MOE_ERR_ARG). */
 MOE_API moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
                                     const int32_t* top_k_index, const float* top_k_weights,
                                     const void* W_gate_up, const void* W_down, void* out,
                                     void* workspace, size_t ws_bytes, uint32_t flags,
                                     void* stream);
+
+/* The dispatch moe_forward_ex takes for this shape and these flags: 1 fused, 0 separate,
+ * -1 invalid flags. */
+MOE_API int32_t moe_forward_dispatch(const moe_shape_t* shape, uint32_t flags);
 
 /* Device workspace, in bytes, that moe_forward_host needs: the moe_forward workspace plus
  * device staging for the routing arrays (T*k int32 + T*k fp32) and min(N_eff, 2) input
