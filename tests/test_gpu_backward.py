@@ -12,7 +12,8 @@ import pytest
 import torch
 
 import oracle
-from gen import CONFIGS, LayerConfig, bf16_normal, bits, layer_inputs
+from gen import (CONFIGS, LayerConfig, bf16_normal, bits, expert_down, expert_gate_up,
+                 expert_weights, hidden, layer_inputs, routing)
 from parity import assert_layer_close, rel_frobenius, to_f64
 
 pytestmark = pytest.mark.gpu
@@ -73,3 +74,39 @@ def test_backward_zero_tokens(moe):
                                      gpu["wd"], d)
     torch.cuda.synchronize()
     assert dx.shape == (0, cfg.H) and not dwgu.any() and not dwd.any()
+
+
+def test_backward_full_size_sampled(moe):
+    """The Qwen3-shaped 16k layer at num_chunks=4, as the benchmark runs it: the weight
+    gradients of two experts (the least-routed one with rows and one of median load), and
+    d_hidden and d_weights of every token routed to them, against the oracle run on exactly
+    those tokens (all k experts of each token included, so every compared value is whole)."""
+    cfg = CONFIGS["qwen3"]
+    idx, w = routing(cfg)
+    x = hidden(cfg.T, cfg.H)
+    dout = bf16_normal((cfg.T, cfg.H), 1.0, 99)
+    wgu, wd = expert_weights(cfg.E, cfg.H, cfg.I, device="cuda")
+    dx, dw, dwgu, dwd = moe.backward(x.cuda(), torch.from_numpy(idx).cuda(),
+                                     torch.from_numpy(w).cuda(), wgu, wd, dout.cuda(),
+                                     num_chunks=4)
+    torch.cuda.synchronize()
+    counts = np.bincount(idx.reshape(-1), minlength=cfg.E)
+    live = np.flatnonzero(counts)
+    e_small = int(live[np.argmin(counts[live])])
+    e_mid = int(live[np.argsort(counts[live])[len(live) // 2]])
+    toks = np.flatnonzero(((idx == e_small) | (idx == e_mid)).any(1))
+    used = sorted(set(idx[toks].reshape(-1).tolist()))
+    remap = {e: i for i, e in enumerate(used)}
+    sub_idx = np.vectorize(remap.get)(idx[toks]).astype(np.int32)
+    sub_wgu = np.stack([bits(expert_gate_up(e, cfg.H, cfg.I)) for e in used])
+    sub_wd = np.stack([bits(expert_down(e, cfg.H, cfg.I)) for e in used])
+    rx, rw, rgu, rd = oracle.backward(bits(x[torch.from_numpy(toks)]), sub_idx, w[toks], sub_wgu,
+                                      sub_wd, bits(dout[torch.from_numpy(toks)]))
+    t_d = torch.from_numpy(toks).cuda()
+    assert_layer_close(dx[t_d], rx, "qwen3 N=4 d_hidden (sampled tokens)")
+    assert_grad_close(dw[t_d], rw, "qwen3 N=4 d_weights (sampled tokens)")
+    for e in (e_small, e_mid):
+        assert_grad_close(dwgu[e], rgu[remap[e]], f"qwen3 N=4 dW_gate_up[{e}]")
+        assert_grad_close(dwd[e], rd[remap[e]], f"qwen3 N=4 dW_down[{e}]")
+    assert bool(torch.isfinite(dwgu).all()) and bool(torch.isfinite(dwd).all())
+    assert bool(torch.isfinite(dx.float()).all())

@@ -185,7 +185,8 @@ def test_forward_full_size_sampled(moe, name, n_tok):
             base = out
         else:
             assert torch.equal(out, base), f"{name}: N={N} differs from N={cfg.chunks[0]}"
-    # the fused-dispatch path gives the same bits
-    assert torch.equal(_run(moe, gpu, cfg.chunks[-1], cfg.G, "fused"), base)
+    # both dispatch paths give the same bits as the default choice
+    for dispatch in ("separate", "fused"):
+        assert torch.equal(_run(moe, gpu, cfg.chunks[-1], cfg.G, dispatch), base), dispatch
     # properties at full size: finite everywhere
     assert bool(torch.isfinite(base.float()).all())
