@@ -152,13 +152,16 @@ def make_inputs(cfg, device, seed=0, weights=True):
     return out
 
 
-def algorithmic_units(cfg, counts, n_live, dispatch="separate"):
+def algorithmic_units(cfg, counts, n_live, dispatch="separate", pair_gemms=False):
     """Per-kernel algorithmic work of one step (bytes or flops), from the chunk counts.
     With the fused dispatch the gate/up GEMM reads each token row of `hidden` (T rows)
-    instead of the T*k permuted rows."""
+    instead of the T*k permuted rows, and with pair GEMMs each GEMM launch serves the two
+    chunks of a pair, so an expert's weights are streamed once per pair."""
     H, I, k, T = cfg.H, cfg.I, cfg.k, cfg.T
     rows = int(counts.sum())
-    active = int((counts > 0).sum())  # (chunk, expert) pairs with rows: weights streamed
+    if pair_gemms:
+        counts = np.stack([counts[i:i + 2].sum(0) for i in range(0, counts.shape[0], 2)])
+    active = int((counts > 0).sum())  # (launch, expert) pairs with rows: weights streamed
     return {
         # permute: read T rows once, write T*k rows, plus the k destination indices per token
         "permute_bytes": (T + rows) * H * 2 + rows * 4,
@@ -181,7 +184,7 @@ def gemm_src_hash():
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def traffic_per_launch(cfg_name, chunks, dispatch):
+def traffic_per_launch(cfg_name, chunks, dispatch, pair_gemms=False):
     """DRAM bytes per gate/up launch from the committed ncu summary, if it was taken on
     the current kernel source, this workload, this chunking and this dispatch; else None."""
     if not os.path.exists(TRAFFIC_FILE):
@@ -189,7 +192,8 @@ def traffic_per_launch(cfg_name, chunks, dispatch):
     with open(TRAFFIC_FILE) as f:
         d = json.load(f)
     if (d.get("gemm_src_sha256_16") != gemm_src_hash() or d.get("num_chunks") != chunks
-            or d.get("config") != cfg_name or d.get("dispatch") != dispatch):
+            or d.get("config") != cfg_name or d.get("dispatch") != dispatch
+            or bool(d.get("pair_gemms", False)) != pair_gemms):
         return None
     return d.get("dram_bytes_per_launch_full_size")
 
@@ -278,7 +282,7 @@ def config_block(cfg, chunks, dispatch="auto"):
 
 # ------------------------------------------------------------------------- our arm
 
-def time_steps(moe, inp, cfg, chunks, ws, steps, stream, dispatch="auto"):
+def time_steps(moe, inp, cfg, chunks, ws, steps, stream, dispatch="auto", pair_gemms=True):
     """Device time of `steps` back-to-back forward calls, ms (CUDA events on `stream`)."""
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
@@ -288,7 +292,7 @@ def time_steps(moe, inp, cfg, chunks, ws, steps, stream, dispatch="auto"):
     for _ in range(steps):
         moe.forward(inp["hidden"], inp["idx"], inp["w"], inp["wgu"], inp["wd"],
                     num_chunks=chunks, ep_groups=cfg.G, out=out, workspace=ws, stream=stream,
-                    dispatch=dispatch)
+                    dispatch=dispatch, pair_gemms=pair_gemms)
     end.record(stream)
     torch.cuda.synchronize()
     return start.elapsed_time(end), out
@@ -320,13 +324,15 @@ def run_ours(args, cfg):
     n_live = int((np.diff(meta["bounds"]) > 0).sum())
     dispatch = moe.forward_dispatch(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, args.dispatch, cfg.G,
                                     chunks)
-    units = algorithmic_units(cfg, counts, n_live, dispatch)
-    active_per_chunk = (counts > 0).sum(1)
-    weight_stream = float(active_per_chunk.sum()) * 6 * cfg.H * cfg.I  # bytes, all chunks
+    pair_gemms = dispatch == "fused" and not args.per_chunk_gemms
+    units = algorithmic_units(cfg, counts, n_live, dispatch, pair_gemms)
+    weight_stream = float(units["gateup_weight_bytes"] + units["down_weight_bytes"])
 
+    pair = not args.per_chunk_gemms
     for _ in range(args.warmup):
         moe.forward(inp["hidden"], inp["idx"], inp["w"], inp["wgu"], inp["wd"],
-                    num_chunks=chunks, ep_groups=cfg.G, workspace=ws, dispatch=args.dispatch)
+                    num_chunks=chunks, ep_groups=cfg.G, workspace=ws, dispatch=args.dispatch,
+                    pair_gemms=pair)
     torch.cuda.synchronize()
 
     clocks = ClockSampler(local) if rank == 0 else None
@@ -337,7 +343,7 @@ def run_ours(args, cfg):
         pg.barrier()
     torch.cuda.synchronize()
     moe.profile_enable(True)
-    ms, out = time_steps(moe, inp, cfg, chunks, ws, args.steps, stream, args.dispatch)
+    ms, out = time_steps(moe, inp, cfg, chunks, ws, args.steps, stream, args.dispatch, pair)
     if pg:
         pg.barrier()
     prof = moe.profile_read()
@@ -391,7 +397,7 @@ def run_ours(args, cfg):
     peak_tc, peak_bw = peaks["bf16_tflops"], peaks["hbm_gbs"]
     t_tensor = gu_flops_l / (peak_tc * 1e12)
     t_mem = gu_bytes_l / (peak_bw * 1e9)
-    traffic = traffic_per_launch(cfg.name, chunks, dispatch)
+    traffic = traffic_per_launch(cfg.name, chunks, dispatch, pair_gemms)
     if t_mem > t_tensor:
         roofline = {"bound": "hbm", "achieved": gu_bytes_l / t_l / 1e9 if t_l else 0.0,
                     "peak": peak_bw, "unit": "GB/s"}
@@ -418,7 +424,8 @@ def run_ours(args, cfg):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; random-init expert weights of the layer's shape)",
-        "config": config_block(cfg, chunks, dispatch),
+        "config": dict(config_block(cfg, chunks, dispatch),
+                       gemm_sweep="per pair of chunks" if pair_gemms else "per chunk"),
         "roofline": roofline,
         "grouped_gemm_tflops": gemm_tflops,
         "grouped_gemm_frac_of_peak": gemm_tflops / peak_tc,
@@ -645,6 +652,8 @@ def main():
                     default="forward",
                     help="forward (the layer's headline), backward (moe_backward alone) or "
                          "train (forward then backward per step)")
+    ap.add_argument("--per-chunk-gemms", action="store_true",
+                    help="fused dispatch: one GEMM sweep per chunk instead of per pair")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the workload's token count (small cases for profiling)")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)

@@ -242,9 +242,12 @@ def forward_dispatch(T, H, I, E, k, dispatch="auto", ep_groups=1, num_chunks=1) 
     return "fused" if r == 1 else "separate"
 
 
+FWD_PER_CHUNK_GEMMS = 4
+
+
 def forward(hidden, top_k_index, top_k_weights, W_gate_up, W_down, num_chunks: int = 1,
             ep_groups: int = 1, out=None, workspace=None, stream=None,
-            dispatch: str = "auto", chunk_size: int = 0):
+            dispatch: str = "auto", chunk_size: int = 0, pair_gemms: bool = True):
     """One MoE layer forward, chunked as Chunk MoE.  Returns out [T,H] bf16.
 
     hidden [T,H] bf16, top_k_index [T,k] int32, top_k_weights [T,k] fp32,
@@ -252,7 +255,8 @@ def forward(hidden, top_k_index, top_k_weights, W_gate_up, W_down, num_chunks: i
     same CUDA device.  Asynchronous after its single metadata copy.
     dispatch="separate": a permute kernel writes the permuted rows first; "fused": the
     gate/up GEMM gathers its rows from `hidden`; "auto": the library's choice for the
-    shape (forward_dispatch).  All give identical bits."""
+    shape (forward_dispatch).  pair_gemms=False: with the fused dispatch, one GEMM sweep per
+    chunk instead of one per pair of chunks.  All give identical bits."""
     _dispatch_flags(dispatch)
     _need(hidden, torch.bfloat16, "hidden")
     _need(top_k_index, torch.int32, "top_k_index")
@@ -271,7 +275,7 @@ def forward(hidden, top_k_index, top_k_weights, W_gate_up, W_down, num_chunks: i
         out = torch.empty((T, H), dtype=torch.bfloat16, device=hidden.device)
     if workspace is None:
         workspace = alloc_workspace(load().moe_workspace_bytes(ctypes.byref(s)), hidden.device)
-    flags = _dispatch_flags(dispatch)
+    flags = _dispatch_flags(dispatch) | (0 if pair_gemms else FWD_PER_CHUNK_GEMMS)
     _check(load().moe_forward_ex(ctypes.byref(s), _ptr(hidden), _ptr(top_k_index),
                                  _ptr(top_k_weights), _ptr(W_gate_up), _ptr(W_down), _ptr(out),
                                  _ptr(workspace), workspace.numel(), flags, _stream(stream)),

@@ -57,6 +57,12 @@
 #ifndef MOE_GEMM_BAND
 #define MOE_GEMM_BAND 16  // M tiles per raster band: an expert's A rows stay in L2 across N tiles
 #endif
+#ifndef MOE_GEMM_WPREFETCH
+// > 0: one more warp walks the weight (B) rows of the tile stream up to this many K blocks
+// ahead of the TMA producer, prefetching each 128-byte block row into L2 (LSU prefetches,
+// so the TMA unit and shared memory are not involved)
+#define MOE_GEMM_WPREFETCH 0
+#endif
 #ifndef MOE_GEMM_PACKED_B
 // 1: B is read from a tile-packed weight layout in which the 256 B rows of one tile and one
 // K block (gate rows then up rows for gate/up) are one contiguous 32 KB block, fetched with
@@ -114,7 +120,13 @@ struct KParams {
   const int32_t* gather;  // gathered A: token row of each permuted row (nullptr: plain A)
   const uint8_t* gsrc;    // gathered A: the token rows (hidden), and their stride in bytes
   int64_t gsrc_stride;
-  int32_t K;              // gathered A: valid K columns (the rest of the last block reads 0)
+  int32_t K;              // valid K columns (gathered A: the rest of the last block reads 0)
+  const uint8_t* bsrc;    // B (weights) base, for the weight prefetch warp
+  // A second row segment sharing the tile sweep (the other chunk of a pair): its expert
+  // offsets [E+1] (nullptr: one segment), output rows, and gathered-A source rows.
+  const int32_t* offsets1;
+  __nv_bfloat16* out1;
+  const int32_t* gather1;
   int32_t reverse;        // 1: walk the tiles (hence the experts) in descending order
   int32_t b4d;            // 1: tmB is the 4-D gate/up view (one box per stage)
 };
@@ -128,7 +140,15 @@ struct SmemCtl {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
+  uint32_t prod_iter;  // K blocks the TMA producer has issued (read by the prefetch warp)
 };
+
+// Threads of one CTA: producer, MMA, 4 epilogue warps; + 4 gathering warps (gathered A);
+// + 1 weight prefetch warp (MOE_GEMM_WPREFETCH).
+template <bool kGather>
+__host__ __device__ constexpr int gemm_threads() {
+  return kGemmThreads + (kGather ? kGatherThreads : 0) + (MOE_GEMM_WPREFETCH ? 32 : 0);
+}
 
 constexpr size_t kCtlBytes = 256;
 static_assert(sizeof(SmemCtl<MOE_GEMM_STAGES_2SM>) <= kCtlBytes, "control block");
@@ -139,7 +159,7 @@ static_assert(sizeof(SmemCtl<MOE_GEMM_STAGES>) <= kCtlBytes, "control block");
 // free of bank conflicts within each 8-lane phase.
 constexpr int kEpiRowBytes = 80;
 constexpr int kEpiWarpBytes = 32 * kEpiRowBytes;
-constexpr size_t kTablesBytes = (2 * (kMaxE + 1) * sizeof(int32_t) + 15) & ~size_t(15);
+constexpr size_t kTablesBytes = (3 * (kMaxE + 1) * sizeof(int32_t) + 15) & ~size_t(15);
 
 template <bool kPair>
 constexpr size_t smem_bytes() {
@@ -147,13 +167,16 @@ constexpr size_t smem_bytes() {
          kTablesBytes + (MOE_GEMM_EPI_STAGE ? 4 * kEpiWarpBytes : 0);
 }
 
+// A tile: expert e, column tile n, row tile m over the expert's rows of both segments
+// (segment 0's row tiles first), i.e. row tile ml of segment seg.
 struct Tile {
-  int32_t e, n, m;
+  int32_t e, n, m, seg, ml;
 };
 
 template <int kTileM>
 __device__ __forceinline__ Tile decode_tile(int32_t L, const int32_t* tile_start,
-                                            const int32_t* off, int32_t E, int32_t n_tiles) {
+                                            const int32_t* off, const int32_t* off1, int32_t E,
+                                            int32_t n_tiles) {
   // largest e with tile_start[e] <= L; that expert has at least one tile
   int32_t lo = 0, hi = E - 1;
   while (lo < hi) {
@@ -161,7 +184,8 @@ __device__ __forceinline__ Tile decode_tile(int32_t L, const int32_t* tile_start
     if (tile_start[mid] <= L) lo = mid;
     else hi = mid - 1;
   }
-  const int32_t mt = (off[lo + 1] - off[lo] + kTileM - 1) / kTileM;
+  const int32_t mt0 = (off[lo + 1] - off[lo] + kTileM - 1) / kTileM;
+  const int32_t mt = mt0 + (off1 ? (off1[lo + 1] - off1[lo] + kTileM - 1) / kTileM : 0);
   const int32_t local = L - tile_start[lo];
   Tile t;
   t.e = lo;
@@ -177,6 +201,8 @@ __device__ __forceinline__ Tile decode_tile(int32_t L, const int32_t* tile_start
   t.m = local / n_tiles;
   t.n = local - t.m * n_tiles;
 #endif
+  t.seg = t.m >= mt0 ? 1 : 0;
+  t.ml = t.m - (t.seg ? mt0 : 0);
   return t;
 }
 
@@ -185,7 +211,8 @@ __device__ __forceinline__ Tile decode_tile(int32_t L, const int32_t* tile_start
 // columns at or past out_cols are never written.
 __device__ __forceinline__ void store_block(const uint32_t (&packed)[16], uint8_t* wbuf, int lane,
                                             int q, bool row_ok, int32_t rows_valid,
-                                            int64_t row_base, int32_t col0, const KParams& p) {
+                                            int64_t row_base, int32_t col0, const KParams& p,
+                                            __nv_bfloat16* out) {
 #if MOE_GEMM_EPI_STAGE
   uint4* mine = reinterpret_cast<uint4*>(wbuf + lane * kEpiRowBytes);
 #pragma unroll
@@ -201,7 +228,7 @@ __device__ __forceinline__ void store_block(const uint32_t (&packed)[16], uint8_
     const uint4 v = *reinterpret_cast<const uint4*>(wbuf + rr * kEpiRowBytes + seg * 16);
     const int32_t tr = q * 32 + rr;  // row inside the CTA's 128 rows
     if (tr < rows_valid && col < p.out_cols)
-      *reinterpret_cast<uint4*>(p.out + (row_base + tr) * p.out_cols + col) = v;
+      *reinterpret_cast<uint4*>(out + (row_base + tr) * p.out_cols + col) = v;
   }
   __syncwarp();
   (void)row_ok;
@@ -209,7 +236,7 @@ __device__ __forceinline__ void store_block(const uint32_t (&packed)[16], uint8_
   (void)wbuf;
   (void)rows_valid;
   if (row_ok) {
-    uint4* dst = reinterpret_cast<uint4*>(p.out + (row_base + q * 32 + lane) * p.out_cols + col0);
+    uint4* dst = reinterpret_cast<uint4*>(out + (row_base + q * 32 + lane) * p.out_cols + col0);
 #pragma unroll
     for (int v = 0; v < 4; ++v)
       if (col0 + v * 8 < p.out_cols)
@@ -224,7 +251,7 @@ __device__ __forceinline__ void store_block(const uint32_t (&packed)[16], uint8_
 // and report back to the leader.
 template <bool kSwiGLU, bool kPair, bool kGather>
 __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensorMap* tmB,
-                                          const KParams& p) {
+                                          const CUtensorMap* tmA1, const KParams& p) {
   using G = Geo<kPair>;
   constexpr int STAGES = G::kStages;
   static_assert(!(kGather && kPair), "gathered A rows are implemented for single CTAs");
@@ -236,6 +263,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   SmemCtl<STAGES>* ctl = reinterpret_cast<SmemCtl<STAGES>*>(smem + STAGES * G::kStageBytes);
   int32_t* off = reinterpret_cast<int32_t*>(smem + STAGES * G::kStageBytes + kCtlBytes);
   int32_t* tile_start = off + (kMaxE + 1);
+  int32_t* off1 = tile_start + (kMaxE + 1);
+  const int32_t* off1p = p.offsets1 ? off1 : nullptr;  // second row segment, if any
   uint8_t* epi_stage = smem + STAGES * G::kStageBytes + kCtlBytes + kTablesBytes;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -246,7 +275,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   const int32_t n_streams = kPair ? (int32_t)(gridDim.x >> 1) : (int32_t)gridDim.x;
 
   // ---- set-up: expert offsets, tile prefix, barriers, TMEM ----
-  for (int32_t i = threadIdx.x; i <= E; i += blockDim.x) off[i] = p.offsets[i];
+  for (int32_t i = threadIdx.x; i <= E; i += blockDim.x) {
+    off[i] = p.offsets[i];
+    if (p.offsets1) off1[i] = p.offsets1[i];
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       // gathered A: the weight producer's arrival plus one per A-gathering thread
@@ -259,6 +291,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
     }
     mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
+    ctl->prod_iter = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -280,8 +313,12 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
     const int32_t per = (E + 31) / 32;
     const int32_t e0 = lane * per, e1 = min(E, e0 + per);
     int32_t sum = 0;
-    for (int32_t e = e0; e < e1; ++e)
-      sum += ((off[e + 1] - off[e] + G::kTileM - 1) / G::kTileM) * p.n_tiles;
+    auto tiles_of = [&](int32_t e) {
+      int32_t mt = (off[e + 1] - off[e] + G::kTileM - 1) / G::kTileM;
+      if (off1p) mt += (off1p[e + 1] - off1p[e] + G::kTileM - 1) / G::kTileM;
+      return mt * p.n_tiles;
+    };
+    for (int32_t e = e0; e < e1; ++e) sum += tiles_of(e);
     int32_t incl = sum;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -291,7 +328,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
     int32_t run = incl - sum;
     for (int32_t e = e0; e < e1; ++e) {
       tile_start[e] = run;
-      run += ((off[e + 1] - off[e] + G::kTileM - 1) / G::kTileM) * p.n_tiles;
+      run += tiles_of(e);
     }
     if (lane == 31) tile_start[E] = incl;
   }
@@ -314,7 +351,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       bool ok = true;
       for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
         const Tile t = decode_tile<G::kTileM>(p.reverse ? p.total_tiles - 1 - L : L, tile_start,
-                                              off, E, p.n_tiles);
+                                              off, off1p, E, p.n_tiles);
         const int32_t brow = t.e * p.b_rows + t.n * (kSwiGLU ? BN / 2 : BN);
         for (int32_t kb = 0; kb < p.num_kb; ++kb) {
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort, p.status)) {
@@ -327,6 +364,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
           if (kSwiGLU)
             tma_load_2d(b_dst + G::kBBytes / 2, tmB, &ctl->full[stage], kb * BK, brow + p.up_off,
                         pol_w);
+          if (MOE_GEMM_WPREFETCH) *reinterpret_cast<volatile uint32_t*>(&ctl->prod_iter) += 1;
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -338,6 +376,46 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       if (!ok)
         for (int s = 0; s < STAGES; ++s)
           if (armed & (1u << s)) mbar_drain(&ctl->full[s], (armed_parity >> s) & 1u, 100000000ull);
+    }
+  } else if (MOE_GEMM_WPREFETCH && !kPair && warp == gemm_threads<kGather>() / 32 - 1) {
+    // ---------------- weight prefetch warp ----------------
+    // Walks the same tile stream as the producer; K block i of the stream (all B rows of the
+    // tile, one 128-byte segment each) is prefetched into L2 once the producer has issued
+    // block i - MOE_GEMM_WPREFETCH.  The wait on the producer's counter is bounded.
+    const volatile uint32_t* prog = &ctl->prod_iter;
+    const int64_t row_bytes = (int64_t)p.K * 2;
+    uint32_t i = 0;
+    bool ok = true;
+    for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
+      const Tile t = decode_tile<G::kTileM>(p.reverse ? p.total_tiles - 1 - L : L, tile_start,
+                                            off, off1p, E, p.n_tiles);
+      const int32_t half = kSwiGLU ? BN / 2 : BN;  // rows per B half (gate, up) or all rows
+      const int32_t nrows = min(half, p.out_cols - t.n * half);
+      const int64_t r0 = (int64_t)t.e * p.b_rows + t.n * half;
+      for (int32_t kb = 0; kb < p.num_kb; ++kb, ++i) {
+        if (*prog + MOE_GEMM_WPREFETCH <= i) {
+          const uint64_t t0 = global_timer_ns();
+          while (*prog + MOE_GEMM_WPREFETCH <= i) {
+            if (*abort) {
+              ok = false;
+              break;
+            }
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+              *abort = 1;
+              atomicOr(p.status, MOE_DEV_TIMEOUT);
+              ok = false;
+              break;
+            }
+            __nanosleep(128);
+          }
+          if (!ok) break;
+        }
+        const uint8_t* base = p.bsrc + r0 * row_bytes + kb * (BK * 2);
+        for (int32_t r = lane; r < nrows; r += 32) {
+          prefetch_l2_last(base + r * row_bytes);
+          if (kSwiGLU) prefetch_l2_last(base + ((int64_t)p.up_off + r) * row_bytes);
+        }
+      }
     }
   } else if (kGather && warp >= kGemmThreads / 32) {
     // ---------------- A producers, gathered rows (4 warps, LSU) ----------------
@@ -355,14 +433,16 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
     bool ok = true;
     for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
       const Tile t = decode_tile<G::kTileM>(p.reverse ? p.total_tiles - 1 - L : L, tile_start,
-                                            off, E, p.n_tiles);
-      const int32_t row0 = off[t.e] + t.m * G::kTileM;
-      const int32_t last = off[t.e + 1] - 1;  // rows past the expert re-read its last row
+                                            off, off1p, E, p.n_tiles);
+      const int32_t* offs = t.seg ? off1 : off;
+      const int32_t* gat = t.seg ? p.gather1 : p.gather;
+      const int32_t row0 = offs[t.e] + t.ml * G::kTileM;
+      const int32_t last = offs[t.e + 1] - 1;  // rows past the expert re-read its last row
       const uint8_t* src[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int32_t r = gw * 32 + 4 * i + sub;
-        src[i] = p.gsrc + (int64_t)p.gather[min(row0 + r, last)] * p.gsrc_stride + j * 16;
+        src[i] = p.gsrc + (int64_t)gat[min(row0 + r, last)] * p.gsrc_stride + j * 16;
       }
       for (int32_t kb = 0; kb < p.num_kb; ++kb) {
         if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort, p.status)) {
@@ -407,13 +487,14 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       uint32_t armed = 0, armed_parity = 0;  // per-stage bits, for the abort drain
       bool ok = true;
       // A row and B row of the tile at linear index L (of this CTA's tile stream)
-      int32_t t_e = 0, t_n = 0;
+      int32_t t_e = 0, t_n = 0, t_seg = 0;
       auto coords = [&](int32_t L, int32_t& row0, int32_t& brow) {
         const Tile t = decode_tile<G::kTileM>(p.reverse ? p.total_tiles - 1 - L : L, tile_start,
-                                              off, E, p.n_tiles);
+                                              off, off1p, E, p.n_tiles);
         t_e = t.e;
         t_n = t.n;
-        row0 = off[t.e] + t.m * G::kTileM + (int32_t)rank * kRowsPerCta;
+        t_seg = t.seg;
+        row0 = (t.seg ? off1 : off)[t.e] + t.ml * G::kTileM + (int32_t)rank * kRowsPerCta;
         if (kSwiGLU)  // pair: the even CTA stages the gate rows, the odd one the up rows
           brow = t.e * p.b_rows + t.n * (BN / 2) + (kPair ? (int32_t)rank * p.up_off : 0);
         else
@@ -433,7 +514,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
         int32_t row0, brow;
         const bool has_next = L + n_streams < p.total_tiles;
         if (MOE_GEMM_PREFETCH > 0 && has_next) coords(L + n_streams, nrow0, nbrow);
-        coords(L, row0, brow);  // last, so that t_e / t_n describe this tile
+        coords(L, row0, brow);  // last, so that t_e / t_n / t_seg describe this tile
+        const CUtensorMap* mapA = t_seg ? tmA1 : tmA;
         for (int32_t kb = 0; kb < p.num_kb; ++kb) {
           if (MOE_GEMM_PREFETCH > 0) {
             const int32_t pk = kb + MOE_GEMM_PREFETCH;
@@ -449,11 +531,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
           if (kPair) {
             if (leader) mbar_arrive_expect_tx(&ctl->full[stage], G::kTxBytes);
             const uint32_t bar = mapa_shared(smem_u32(&ctl->full[stage]), 0);
-            tma_load_2d_pair(a_dst, tmA, bar, kb * BK, row0, pol_a);
+            tma_load_2d_pair(a_dst, mapA, bar, kb * BK, row0, pol_a);
             tma_load_2d_pair(b_dst, tmB, bar, kb * BK, brow, pol_w);
           } else {
             mbar_arrive_expect_tx(&ctl->full[stage], G::kTxBytes);
-            tma_load_2d(a_dst, tmA, &ctl->full[stage], kb * BK, row0, pol_a);
+            tma_load_2d(a_dst, mapA, &ctl->full[stage], kb * BK, row0, pol_a);
             if (MOE_GEMM_PACKED_B) {
               const int32_t prow = ((t_e * p.n_tiles + t_n) * p.num_kb + kb) * BN;
               tma_load_2d(b_dst, tmB, &ctl->full[stage], 0, prow, pol_w);
@@ -468,6 +550,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
               tma_load_2d(b_dst, tmB, &ctl->full[stage], kb * BK, brow, pol_w);
             }
           }
+          if (MOE_GEMM_WPREFETCH) *reinterpret_cast<volatile uint32_t*>(&ctl->prod_iter) += 1;
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -547,11 +630,13 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       if (!mbar_wait(&ctl->tfull[buf], tphase, abort, p.status)) break;
       tc_fence_after();
       const Tile t = decode_tile<G::kTileM>(p.reverse ? p.total_tiles - 1 - L : L, tile_start,
-                                            off, E, p.n_tiles);
-      const int32_t first = t.m * G::kTileM + (int32_t)rank * kRowsPerCta;  // in the expert
-      const int32_t rows_valid = off[t.e + 1] - off[t.e] - first;
+                                            off, off1p, E, p.n_tiles);
+      const int32_t* offs = t.seg ? off1 : off;
+      __nv_bfloat16* out = t.seg ? p.out1 : p.out;
+      const int32_t first = t.ml * G::kTileM + (int32_t)rank * kRowsPerCta;  // in the expert
+      const int32_t rows_valid = offs[t.e + 1] - offs[t.e] - first;
       const bool row_ok = r < rows_valid;
-      const int64_t row_base = (int64_t)off[t.e] + first;  // output row of TMEM lane 0
+      const int64_t row_base = (int64_t)offs[t.e] + first;  // output row of TMEM lane 0
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * BN;
       if (kSwiGLU) {
 #pragma unroll 1
@@ -570,7 +655,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
             const float a1 = g1 / (1.0f + __expf(-g1)) * u1;
             packed[i] = pack_bf16x2(a0, a1);
           }
-          store_block(packed, wbuf, lane, q, row_ok, rows_valid, row_base, col0, p);
+          store_block(packed, wbuf, lane, q, row_ok, rows_valid, row_base, col0, p, out);
         }
       } else {
 #pragma unroll 1
@@ -583,7 +668,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             packed[i] = pack_bf16x2(__uint_as_float(acc[2 * i]), __uint_as_float(acc[2 * i + 1]));
-          store_block(packed, wbuf, lane, q, row_ok, rows_valid, row_base, col0, p);
+          store_block(packed, wbuf, lane, q, row_ok, rows_valid, row_base, col0, p, out);
         }
       }
       tc_fence_before();
@@ -604,18 +689,20 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
 }
 
 template <bool kSwiGLU, bool kGather>
-__global__ void __launch_bounds__(kGather ? kGemmThreads + kGatherThreads : kGemmThreads, 1)
+__global__ void __launch_bounds__(gemm_threads<kGather>(), 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                        const __grid_constant__ CUtensorMap tmB, const KParams p) {
-  gemm_body<kSwiGLU, false, kGather>(&tmA, &tmB, p);
+                        const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmA1, const KParams p) {
+  gemm_body<kSwiGLU, false, kGather>(&tmA, &tmB, &tmA1, p);
 }
 
 // Launched with a cluster of 2 CTAs (cudaLaunchAttributeClusterDimension).
 template <bool kSwiGLU>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
-                             const __grid_constant__ CUtensorMap tmB, const KParams p) {
-  gemm_body<kSwiGLU, true, false>(&tmA, &tmB, p);
+                             const __grid_constant__ CUtensorMap tmB,
+                             const __grid_constant__ CUtensorMap tmA1, const KParams p) {
+  gemm_body<kSwiGLU, true, false>(&tmA, &tmB, &tmA1, p);
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -713,10 +800,12 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
     *err_detail = 1;
     return cudaErrorInvalidValue;
   }
-  CUtensorMap mA, mB;
+  CUtensorMap mA, mB, mA1;
   const int32_t bn = swiglu ? BN / 2 : BN;
   const bool gather = a.gather != nullptr;
-  if (gather && (kPair || !swiglu)) {
+  const bool two = a.offsets1 != nullptr;  // a second row segment (the pair's other chunk)
+  if ((gather && (kPair || !swiglu)) || (two && kPair) ||
+      (two && (!a.out1 || (gather ? !a.gather1 : !a.A1)))) {
     *err_detail = 1;
     return cudaErrorInvalidValue;
   }
@@ -733,7 +822,9 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
                   ? make_map(&mB, a.B, packed_rows, BK, BN)
                   : make_map(&mB, a.B, (int64_t)a.E * a.b_rows, a.K,
                              kPair ? BN / 2 : (swiglu ? BN / 2 : BN)));
-  if (!map_a_ok || !map_b_ok) {
+  const bool map_a1_ok =
+      two && !gather ? make_map(&mA1, a.A1, a.rows1, a.K, kRowsPerCta) : (mA1 = mA, true);
+  if (!map_a_ok || !map_b_ok || !map_a1_ok) {
     *err_detail = 2;
     return cudaErrorInvalidValue;
   }
@@ -752,8 +843,12 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
   p.gsrc = static_cast<const uint8_t*>(a.gather_src);
   p.gsrc_stride = (int64_t)a.K * 2;
   p.K = a.K;
+  p.bsrc = static_cast<const uint8_t*>(a.B);
   p.reverse = a.reverse ? 1 : 0;
   p.b4d = b4d ? 1 : 0;
+  p.offsets1 = two ? a.offsets1 : nullptr;
+  p.out1 = two ? static_cast<__nv_bfloat16*>(a.out1) : nullptr;
+  p.gather1 = two ? a.gather1 : nullptr;
   constexpr size_t smem = smem_bytes<kPair>();
   cudaError_t e;
   if (kPair) {
@@ -785,7 +880,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
     }
     const int streams = (int)(a.total_tiles < mp ? a.total_tiles : mp);
     cfg.gridDim = dim3(2 * streams, 1, 1);
-    e = cudaLaunchKernelEx(&cfg, k, mA, mB, p);
+    e = cudaLaunchKernelEx(&cfg, k, mA, mB, mA1, p);
     if (e != cudaSuccess) return e;
   } else {
     auto k = gather ? grouped_gemm_kernel<true, true>
@@ -793,7 +888,8 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int streams = (int)(a.total_tiles < num_sms ? a.total_tiles : num_sms);
-    k<<<streams, gather ? kGemmThreads + kGatherThreads : kGemmThreads, smem, s>>>(mA, mB, p);
+    k<<<streams, gather ? gemm_threads<true>() : gemm_threads<false>(), smem, s>>>(mA, mB, mA1,
+                                                                                     p);
   }
   return cudaGetLastError();
 }

@@ -67,6 +67,15 @@ struct GemmArgs {
   const void* gather_src = nullptr;
   int64_t gather_src_rows = 0;
   bool reverse = false;  // walk the tiles (and so the experts) in descending order
+  // A second row segment in the same tile sweep (the other chunk of a pair: the weights of
+  // each expert tile are then fetched once for both): its expert offsets (dev [E+1]; nullptr
+  // = one segment), A rows (A1 [rows1][K], or gathered through gather1), and output rows.
+  // total_tiles then counts the tiles of both segments.
+  const int32_t* offsets1 = nullptr;
+  const void* A1 = nullptr;
+  int64_t rows1 = 0;
+  const int32_t* gather1 = nullptr;
+  void* out1 = nullptr;
 };
 
 // 2-D bf16 tensor map over a row-major [rows][cols] matrix: boxes of box_rows x 64 columns,

@@ -372,13 +372,35 @@ int64_t active_experts(const int32_t* counts, int32_t E) {
 #define MOE_ALTERNATE_ORDER 0  // 1: odd chunks walk the experts in descending order
 #endif
 
+// The second row segment of a grouped GEMM that serves both chunks of a pair.
+struct Seg1 {
+  const void* A = nullptr;           // [rows][K], or nullptr with gathered A
+  int64_t rows = 0;
+  const int32_t* offsets = nullptr;  // dev [E+1]
+  const int32_t* counts = nullptr;   // host [E]
+  const int32_t* gather = nullptr;   // gathered A: token row of each of its rows
+  void* out = nullptr;
+};
+
 moe_status_t gemm_call(const void* A, int64_t rows, const void* B, void* out,
                        const int32_t* offsets_dev, const int32_t* counts_host, int32_t E,
                        int32_t K, int32_t out_cols, int32_t b_rows, bool swiglu,
                        uint32_t* status, int num_sms, cudaStream_t s,
                        const int32_t* gather = nullptr, const void* gather_src = nullptr,
-                       int64_t gather_src_rows = 0, bool reverse = false) {
+                       int64_t gather_src_rows = 0, bool reverse = false,
+                       const Seg1* seg1 = nullptr) {
   GemmArgs g;
+  int64_t rows_all = rows, active = active_experts(counts_host, E);
+  if (seg1) {
+    g.offsets1 = seg1->offsets;
+    g.A1 = seg1->A;
+    g.rows1 = seg1->rows;
+    g.gather1 = seg1->gather;
+    g.out1 = seg1->out;
+    rows_all += seg1->rows;
+    active = 0;  // experts with rows in either segment
+    for (int32_t e = 0; e < E; ++e) active += (counts_host[e] + seg1->counts[e]) > 0;
+  }
   g.reverse = reverse;
   g.gather = gather;
   g.gather_src = gather_src;
@@ -392,12 +414,12 @@ moe_status_t gemm_call(const void* A, int64_t rows, const void* B, void* out,
   g.K = K;
   g.out_cols = out_cols;
   g.b_rows = b_rows;
-  g.total_tiles = gemm_total_tiles(counts_host, E, out_cols, swiglu);
+  g.total_tiles = gemm_total_tiles(counts_host, E, out_cols, swiglu) +
+                  (seg1 ? gemm_total_tiles(seg1->counts, E, out_cols, swiglu) : 0);
   g.status = status;
   if (g.total_tiles == 0) return MOE_OK;
   int detail = 0;
-  ProfScope ps(swiglu ? MOE_KERNEL_GATEUP : MOE_KERNEL_DOWN, s, rows,
-               active_experts(counts_host, E), 1);
+  ProfScope ps(swiglu ? MOE_KERNEL_GATEUP : MOE_KERNEL_DOWN, s, rows_all, active, 1);
   cudaError_t e = launch_grouped_gemm(g, swiglu, num_sms, s, &detail);
   if (e != cudaSuccess) return detail == 1 ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
   return MOE_OK;
@@ -525,12 +547,15 @@ moe_status_t moe_metadata_shape(const moe_shape_t* shape, const int32_t* top_k_i
 
 int32_t moe_forward_dispatch(const moe_shape_t* shape, uint32_t flags) {
   const uint32_t both = MOE_FWD_FUSED_DISPATCH | MOE_FWD_SEPARATE_DISPATCH;
-  if ((flags & ~both) || (flags & both) == both || !shape) return -1;
+  if ((flags & ~(both | MOE_FWD_PER_CHUNK_GEMMS)) || (flags & both) == both || !shape) return -1;
   if (!gemm_supports_gather() || (flags & MOE_FWD_SEPARATE_DISPATCH)) return 0;
   if (flags & MOE_FWD_FUSED_DISPATCH) return 1;
   if (check_shape(shape) != MOE_OK) return 0;
   const Dims d = make_dims(shape->T, shape->k, shape->E, shape->ep_groups, shape->num_chunks,
                            shape->chunk_size);
+  // two or more chunks: the pair sweeps halve the weight stream, which outweighs the cost
+  // of the row gathers; one chunk: gather only when the permuted copy is a sizeable share
+  if (d.n >= 2) return 1;
   return 4 * d.t_chunk * d.k >= (int64_t)d.E * shape->I ? 1 : 0;
 }
 
@@ -553,6 +578,8 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
   const int32_t H = shape->H, I = shape->I, E = shape->E, k = shape->k;
   if (T == 0) return MOE_OK;
   const bool fused = choice == 1;
+  // fused dispatch: one GEMM sweep per pair of chunks unless asked for per-chunk GEMMs
+  const bool pair_gemms = fused && !(flags & MOE_FWD_PER_CHUNK_GEMMS);
   if (!hidden || !top_k_index || !top_k_weights || !W_gate_up || !W_down || !out || !workspace)
     return MOE_ERR_ARG;
   if (!aligned(hidden, 16) || !aligned(out, 16) || !aligned(W_gate_up, 16) ||
@@ -640,6 +667,48 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
         if ((st = permute(c + 1)) != MOE_OK || (st = experts(c + 1)) != MOE_OK) return st;
       }
       if ((st = unpermute(c)) != MOE_OK) return st;
+    }
+  } else if (n_live > 0 && pair_gemms) {
+    // Pairs (c0, c1) = (2m, 2m+1), chunk c in buffer c % 2.  G: GU(m) D(m) GU(m+1) D(m+1) ...
+    // where GU / D are the gate/up and down GEMMs of both chunks of the pair in one tile
+    // sweep (each expert's weight tiles are fetched once for the pair); D(m+1) waits until
+    // U(c0), U(c1) have read the pair's Y rows.  M: U(c0) U(c1) after D(m), beside GU(m+1).
+    auto seg = [&](int c, const void* A, void* out) {
+      Seg1 g1;
+      g1.A = A;
+      g1.rows = len(c) * k;
+      g1.offsets = reinterpret_cast<const int32_t*>(ws + L.offsets) + (size_t)c * (E + 1);
+      g1.counts = counts.data() + (size_t)c * E;
+      g1.gather = A ? nullptr : src + bounds[c] * k;
+      g1.out = out;
+      return g1;
+    };
+    for (int c0 = 0; c0 < n_live; c0 += 2) {
+      const bool two = c0 + 1 < n_live;
+      const int c1 = c0 + 1;
+      const Seg1 s0 = seg(c0, nullptr, act(c0));
+      Seg1 s1 = two ? seg(c1, nullptr, act(c1)) : Seg1{};
+      moe_status_t s2 = gemm_call(nullptr, s0.rows, W_gate_up, act(c0), s0.offsets, s0.counts,
+                                  E, H, I, 2 * I, true, dev_status, ctx->num_sms, sg, s0.gather,
+                                  hidden, T, false, two ? &s1 : nullptr);
+      if (s2 != MOE_OK) return s2;
+      if (c0 >= 2 && cudaStreamWaitEvent(sg, ctx->ev_unperm[0], 0) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      if (two) s1 = seg(c1, act(c1), xy(c1));
+      s2 = gemm_call(act(c0), s0.rows, W_down, xy(c0), s0.offsets, s0.counts, E, I, H, H, false,
+                     dev_status, ctx->num_sms, sg, nullptr, nullptr, 0, false,
+                     two ? &s1 : nullptr);
+      if (s2 != MOE_OK) return s2;
+      if (cudaEventRecord(ctx->ev_gemm[0], sg) != cudaSuccess ||
+          cudaStreamWaitEvent(sm, ctx->ev_gemm[0], 0) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      for (int c = c0; c <= (two ? c1 : c0); ++c) {
+        ProfScope ps(MOE_KERNEL_UNPERMUTE, sm, len(c) * k, 0, 1);
+        if (launch_unpermute(xy(c), dst + bounds[c] * k, top_k_weights + bounds[c] * k, len(c),
+                             H, k, outp + bounds[c] * H, sm) != cudaSuccess)
+          return MOE_ERR_CUDA;
+      }
+      if (cudaEventRecord(ctx->ev_unperm[0], sm) != cudaSuccess) return MOE_ERR_CUDA;
     }
   } else if (n_live > 0) {
     // G: E(0) E(1) E(2) ... (E(c+2) after U(c) freed buffer c % 2); M: U(0) U(1) ...

@@ -229,17 +229,22 @@ MOE_API moe_status_t moe_forward(const moe_shape_t* shape, const void* hidden, c
 /* Flags of moe_forward_ex. */
 #define MOE_FWD_FUSED_DISPATCH 1u    /* gather the gate/up GEMM's rows from hidden; no permute */
 #define MOE_FWD_SEPARATE_DISPATCH 2u /* permute kernel first, as the article's permute step */
+#define MOE_FWD_PER_CHUNK_GEMMS 4u   /* fused dispatch: one GEMM sweep per chunk, not per pair */
 
 /* moe_forward with a choice of dispatch.  MOE_FWD_SEPARATE_DISPATCH: the permute kernel
  * writes the permuted rows (the article's separate permute step) and the pipeline overlaps
  * the permute of chunk c+1 and the unpermute of chunk c-1 with the expert GEMMs of chunk c.
  * MOE_FWD_FUSED_DISPATCH: the gate/up GEMM copies each permuted row's K blocks straight from
  * `hidden` through the permutation's inverse map (four gathering warps per CTA), so no
- * permuted copy of the input is written or read, and the pipeline overlaps the unpermute of
- * chunk c with the expert GEMMs of chunk c+1.  flags = 0 (what moe_forward does) chooses
- * fused when a chunk holds at least I/4 rows per expert on average (4 * T_chunk * k >= E * I):
- * the permuted copy it saves is then a sizeable share of the GEMMs' memory traffic, which
- * the expert weights dominate otherwise (there the gathers cost more than they save).
+ * permuted copy of the input is written or read.  With the fused dispatch the two chunks of
+ * each pair (2m, 2m+1) share one tile sweep per GEMM, so each expert's weight tiles are
+ * fetched once per pair rather than once per chunk (MOE_FWD_PER_CHUNK_GEMMS: one sweep per
+ * chunk), and the unpermutes of pair m overlap the gate/up GEMM of pair m+1; the workspace
+ * is unchanged (the pair's two chunk buffers are resident anyway).  flags = 0 (what
+ * moe_forward does) chooses fused whenever there are two or more chunks (the pair sweeps
+ * halve the weight stream), and with one chunk when it holds at least I/4 rows per expert
+ * on average (4 * T * k >= E * I: the permuted copy it saves is then a sizeable share of
+ * the GEMMs' memory traffic, which the expert weights dominate otherwise).
  * Every choice gives bit-identical outputs; arguments, workspace and errors are as
  * moe_forward (unknown flag bits, or both flags: MOE_ERR_ARG). */
 MOE_API moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,

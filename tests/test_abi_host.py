@@ -168,7 +168,7 @@ def test_forward_ex_rejects_unknown_flags():
     L = moe.load()
     v = ctypes.c_void_p
     good = moe.shape(64, 64, 64, 8, 2, 2, 4)
-    for flags in (4, 3):  # an unknown bit; both dispatch flags at once
+    for flags in (8, 3):  # an unknown bit; both dispatch flags at once
         assert L.moe_forward_ex(ctypes.byref(good), v(FAKE), v(FAKE), v(FAKE), v(FAKE), v(FAKE),
                                 v(FAKE), v(FAKE), 1 << 40, flags, None) == 1
 
@@ -224,15 +224,17 @@ def test_profile_api_without_launches():
 
 def test_forward_dispatch_choice():
     """moe_forward_dispatch (host logic): flags force a dispatch; flags = 0 gathers in the
-    gate/up GEMM when a chunk holds at least I/4 rows per expert (4 T_chunk k >= E I)."""
+    gate/up GEMM whenever there are two or more chunks (pair sweeps), and with one chunk
+    when it holds at least I/4 rows per expert (4 T k >= E I)."""
     import expert_router_top_b200 as moe
     q, m, d = CONFIGS["qwen3"], CONFIGS["mixtral"], CONFIGS["deepseek"]
-    for N, want in ((1, "fused"), (4, "fused"), (8, "separate")):  # 4*2048*8 < 128*768
-        assert moe.forward_dispatch(q.T, q.H, q.I, q.E, q.k, num_chunks=N) == want
-    for N in (1, 4):
-        assert moe.forward_dispatch(m.T, m.H, m.I, m.E, m.k, num_chunks=N) == "separate"
-        assert moe.forward_dispatch(d.T, d.H, d.I, d.E, d.k, ep_groups=d.G, num_chunks=N) == "separate"
-    # the boundary: 4 * 96 * 2 = 768 = 8 * 96
+    for N in (1, 2, 4, 8):
+        assert moe.forward_dispatch(q.T, q.H, q.I, q.E, q.k, num_chunks=N) == "fused"
+    assert moe.forward_dispatch(m.T, m.H, m.I, m.E, m.k, num_chunks=1) == "separate"
+    assert moe.forward_dispatch(m.T, m.H, m.I, m.E, m.k, num_chunks=2) == "fused"
+    assert moe.forward_dispatch(d.T, d.H, d.I, d.E, d.k, ep_groups=d.G) == "separate"
+    assert moe.forward_dispatch(d.T, d.H, d.I, d.E, d.k, ep_groups=d.G, num_chunks=4) == "fused"
+    # the one-chunk boundary: 4 * 96 * 2 = 768 = 8 * 96
     assert moe.forward_dispatch(96, 64, 96, 8, 2) == "fused"
     assert moe.forward_dispatch(95, 64, 96, 8, 2) == "separate"
     assert moe.forward_dispatch(q.T, q.H, q.I, q.E, q.k, "separate", num_chunks=4) == "separate"
@@ -240,4 +242,5 @@ def test_forward_dispatch_choice():
     L = moe.load()
     s = moe.shape(16, 64, 64, 4, 2, 1, 1, 0)
     assert L.moe_forward_dispatch(ctypes.byref(s), 3) == -1
-    assert L.moe_forward_dispatch(ctypes.byref(s), 4) == -1
+    assert L.moe_forward_dispatch(ctypes.byref(s), 8) == -1
+    assert L.moe_forward_dispatch(ctypes.byref(s), 4) == 0  # a valid flag; auto: separate here

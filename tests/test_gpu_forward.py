@@ -14,9 +14,9 @@ from parity import assert_layer_close, to_f64
 pytestmark = pytest.mark.gpu
 
 
-def _run(moe, inp, N, G=1, dispatch="separate"):
+def _run(moe, inp, N, G=1, dispatch="separate", pair_gemms=True):
     out = moe.forward(inp["hidden"], inp["idx"], inp["w"], inp["wgu"], inp["wd"], num_chunks=N,
-                      ep_groups=G, dispatch=dispatch)
+                      ep_groups=G, dispatch=dispatch, pair_gemms=pair_gemms)
     torch.cuda.synchronize()
     return out
 
@@ -52,6 +52,21 @@ def test_fused_and_separate_dispatch_are_bit_identical(moe, name):
     gpu = {k: v.cuda() for k, v in layer_inputs(cfg).items()}
     for N in (1,) + tuple(cfg.chunks):
         assert torch.equal(_run(moe, gpu, N, cfg.G, "fused"), _run(moe, gpu, N, cfg.G, "separate"))
+
+
+@pytest.mark.parametrize("name", ["tiny", "edge", "edge_pair01", "edge_varlen", "edge_varlen7"])
+def test_pair_gemms_match_per_chunk_gemms(moe, name):
+    """With the fused dispatch, both chunks of a pair share one tile sweep per GEMM; each
+    row's arithmetic is unchanged, so the output equals the per-chunk sweeps bit for bit,
+    for even and odd chunk counts (the last chunk of an odd count is alone)."""
+    cfg = CONFIGS[name]
+    gpu = {k: v.cuda() for k, v in layer_inputs(cfg).items()}
+    base = _run(moe, gpu, 1, cfg.G, "separate")
+    for N in (2, 3, 4, 5, 8) + tuple(cfg.chunks):
+        a = _run(moe, gpu, N, cfg.G, "fused", pair_gemms=True)
+        b = _run(moe, gpu, N, cfg.G, "fused", pair_gemms=False)
+        assert torch.equal(a, b), f"{name} N={N}: pair sweep differs from per-chunk sweeps"
+        assert torch.equal(a, base), f"{name} N={N}: differs from N=1"
 
 
 @pytest.mark.parametrize("pinned", [True, False])
