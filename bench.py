@@ -82,7 +82,8 @@ def dist_env():
 # ------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi samples of one GPU's clocks and throttle reasons, every 200 ms."""
+    """nvidia-smi samples of one GPU's clocks and throttle reasons, every 50 ms, each with
+    its host arrival time so that only the samples taken during the timed region count."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -98,7 +99,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -108,9 +109,11 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.perf_counter(), line.strip()))
 
-    def stop(self):
+    def stop(self, t0=None, t1=None):
+        """Summary of the samples that arrived in [t0, t1 + 0.1 s] (host perf_counter
+        times of the timed region; all samples when not given)."""
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -122,7 +125,10 @@ class ClockSampler:
             self.thread.join(timeout=2)
         sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        lines = self.lines
+        if t0 is not None:
+            lines = [x for x in self.lines if t0 <= x[0] <= t1 + 0.1]
+        for _, ln in lines:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
@@ -138,6 +144,19 @@ class ClockSampler:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+def spin_up(step, seconds=0.5):
+    """Run `step` untimed for `seconds` of device time so that the SM clocks have left their
+    idle state before the warm-up and timed steps; returns the number of calls."""
+    n, t_end = 0, time.perf_counter() + seconds
+    while time.perf_counter() < t_end:
+        step()
+        n += 1
+        if n % 8 == 0:
+            torch.cuda.synchronize()
+    torch.cuda.synchronize()
+    return n
 
 
 # ---------------------------------------------------------------------- workload
@@ -329,26 +348,31 @@ def run_ours(args, cfg):
     weight_stream = float(units["gateup_weight_bytes"] + units["down_weight_bytes"])
 
     pair = not args.per_chunk_gemms
-    for _ in range(args.warmup):
+
+    def fwd_step():
         moe.forward(inp["hidden"], inp["idx"], inp["w"], inp["wgu"], inp["wd"],
                     num_chunks=chunks, ep_groups=cfg.G, workspace=ws, dispatch=args.dispatch,
                     pair_gemms=pair)
-    torch.cuda.synchronize()
 
     clocks = ClockSampler(local) if rank == 0 else None
     if clocks:
         clocks.start()
-        time.sleep(0.3)
+    spinup = spin_up(fwd_step)
+    for _ in range(args.warmup):
+        fwd_step()
+    torch.cuda.synchronize()
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
     moe.profile_enable(True)
+    t0 = time.perf_counter()
     ms, out = time_steps(moe, inp, cfg, chunks, ws, args.steps, stream, args.dispatch, pair)
+    t1 = time.perf_counter()
     if pg:
         pg.barrier()
     prof = moe.profile_read()
     moe.profile_enable(False)
-    clk = clocks.stop() if clocks else None
+    clk = clocks.stop(t0, t1) if clocks else None
 
     ms_max = max_over_ranks(ms, pg, dev)
     ms_per_step = ms_max / args.steps
@@ -437,6 +461,7 @@ def run_ours(args, cfg):
         "ms_per_step_num_chunks_1": ms_n1,
         "send_splits": meta["send"].tolist() if cfg.G > 1 else None,
         "gpu_launches": int(prof["kernels"]),
+        "spinup_steps": spinup,
         "e2e": e2e,
         "clocks": clk,
     }
@@ -514,28 +539,30 @@ def run_backward(args, cfg):
                      num_chunks=chunks, ep_groups=cfg.G, workspace=bws, stream=stream,
                      out=grads)
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
     clocks = ClockSampler(local) if rank == 0 else None
     if clocks:
         clocks.start()
-        time.sleep(0.3)
+    spinup = spin_up(step)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
     moe.profile_enable(True)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
     start.record(stream)
     for _ in range(args.steps):
         step()
     end.record(stream)
     torch.cuda.synchronize()
+    t1 = time.perf_counter()
     if pg:
         pg.barrier()
     prof = moe.profile_read()
     moe.profile_enable(False)
-    clk = clocks.stop() if clocks else None
+    clk = clocks.stop(t0, t1) if clocks else None
     ms_max = max_over_ranks(start.elapsed_time(end), pg, dev)
     steps = args.steps
     peaks, peak_src = load_peaks()
@@ -585,6 +612,7 @@ def run_backward(args, cfg):
         "kernels": kinds,
         "backward_workspace_bytes": ws_per_n,
         "gpu_launches": int(prof["kernels"]),
+        "spinup_steps": spinup,
         "e2e": None,
         "clocks": clk,
     }
@@ -640,7 +668,7 @@ def run_e2e(moe, inp, cfg, chunks, ws, args, stream, dev, pg, world):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", choices=sorted(CONFIGS), default=DEFAULT_CONFIG)
