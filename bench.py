@@ -438,6 +438,8 @@ def run_ours(args, cfg):
                        "roofline_ms": max(t_tensor, t_mem) * 1e3},
         "frac_of_roofline_time": max(t_tensor, t_mem) / t_l if t_l else None,
         "tensor_frac": gu_flops_l / t_l / 1e12 / peak_tc if t_l else None,
+        "tensor_frac_of_sustained": gu_flops_l / t_l / 1e12 / peaks["bf16_tflops_sustained"]
+        if t_l else None,
         "hbm_frac": gu_bytes_l / t_l / 1e9 / peak_bw if t_l else None})
     peak_tc = peaks["bf16_tflops"]
 
@@ -595,6 +597,7 @@ def run_backward(args, cfg):
         "per_launch": {"flops": f / n_wg, "bytes": b / n_wg, "ms": t * 1e3 / n_wg,
                        "roofline_ms": max(t_tensor, t_mem) * 1e3 / n_wg},
         "tensor_frac": f / t / 1e12 / peaks["bf16_tflops"],
+        "tensor_frac_of_sustained": f / t / 1e12 / peaks["bf16_tflops_sustained"],
         "hbm_frac": b / t / 1e9 / peaks["hbm_gbs"]})
     gemm_fl = sum(v for k2, v in units["flops"].items())
     gemm_ms = sum(prof[k2]["ms"] for k2 in units["flops"]) / steps

@@ -71,7 +71,12 @@ struct BParams {
   const int32_t* first;     // kWGrad: [E] first chunk with rows of each expert
   int32_t chunk;            // kWGrad: first chunk of this launch
   int32_t chunk_last;       // kWGrad: last chunk of this launch (chunk + 1 for a pair)
-  const int32_t* offsets1;  // kWGrad: padded offsets [E+1] of the pair's second chunk, or null
+  const int32_t* offsets1;  // padded offsets [E+1] of the pair's second chunk, or null: for
+                            // kWGrad its rows extend K; for the row-grouped modes they are a
+                            // second row segment of the same tile sweep (A rows from tmA1)
+  __nv_bfloat16* out0b;     // row-grouped modes: out0 / out1 / aux of the second segment
+  __nv_bfloat16* out1b;
+  const __nv_bfloat16* auxb;
 };
 
 struct Ctl {
@@ -99,13 +104,15 @@ __device__ __forceinline__ uint64_t mn_desc(uint32_t addr) {
          (static_cast<uint64_t>(1024 >> 4) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// A tile: expert e, column tile n, row tile m (row-grouped modes: over the expert's rows of
+// both segments, segment 0 first, i.e. row tile ml of segment seg).
 struct Tile {
-  int32_t e, m, n;
+  int32_t e, m, n, seg, ml;
 };
 
 template <int kMode>
 __device__ __forceinline__ Tile decode(int32_t L, const int32_t* ts, const int32_t* off,
-                                       int32_t E, const BParams& p) {
+                                       const int32_t* off1, int32_t E, const BParams& p) {
   int32_t lo = 0, hi = E - 1;
   while (lo < hi) {
     const int32_t mid = (lo + hi + 1) >> 1;
@@ -115,13 +122,18 @@ __device__ __forceinline__ Tile decode(int32_t L, const int32_t* ts, const int32
   const int32_t local = L - ts[lo];
   Tile t;
   t.e = lo;
+  t.seg = 0;
   if (kMode == kWGrad) {
     t.m = local / p.n_tiles;
     t.n = local - t.m * p.n_tiles;
+    t.ml = t.m;
   } else {
-    const int32_t mt = (off[lo + 1] - off[lo] + BM - 1) / BM;
+    const int32_t mt0 = (off[lo + 1] - off[lo] + BM - 1) / BM;
+    const int32_t mt = mt0 + (p.offsets1 ? (off1[lo + 1] - off1[lo] + BM - 1) / BM : 0);
     t.n = local / mt;
     t.m = local - t.n * mt;
+    t.seg = t.m >= mt0 ? 1 : 0;
+    t.ml = t.m - (t.seg ? mt0 : 0);
   }
   return t;
 }
@@ -155,7 +167,7 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
   constexpr int kEpi = Cfg<kMode>::kEpi;
   for (int32_t i = threadIdx.x; i <= E; i += Cfg<kMode>::kThreads) {
     off[i] = p.offsets[i];
-    if (kMode == kWGrad) off1[i] = p.offsets1 ? p.offsets1[i] : 0;
+    off1[i] = p.offsets1 ? p.offsets1[i] : 0;
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -181,7 +193,7 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
     auto tiles_of = [&](int32_t e) -> int32_t {
       const int32_t rows = off[e + 1] - off[e];
       if (kMode == kWGrad) return rows + off1[e + 1] - off1[e] > 0 ? p.m_tiles * p.n_tiles : 0;
-      return ((rows + BM - 1) / BM) * p.n_tiles;
+      return ((rows + BM - 1) / BM + (off1[e + 1] - off1[e] + BM - 1) / BM) * p.n_tiles;
     };
     int32_t sum = 0;
     for (int32_t e = e0; e < e1; ++e) sum += tiles_of(e);
@@ -211,7 +223,7 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
       uint32_t phase = 0, armed = 0, armed_parity = 0;
       bool ok = true;
       for (int32_t L = blockIdx.x; L < p.total_tiles && ok; L += gridDim.x) {
-        const Tile t = decode<kMode>(L, ts, off, E, p);
+        const Tile t = decode<kMode>(L, ts, off, off1, E, p);
         const int32_t nkb0 = (off[t.e + 1] - off[t.e]) / BK;
         const int32_t nkb = kMode == kWGrad ? nkb0 + (off1[t.e + 1] - off1[t.e]) / BK : p.num_kb;
         for (int32_t kb = 0; kb < nkb; ++kb) {
@@ -231,8 +243,8 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
             for (int q = 0; q < 2; ++q) tma_load_2d(a + q * 8192, ma, bar, t.m * BM + q * 64, r0, pol);
             for (int q = 0; q < 4; ++q) tma_load_2d(b + q * 8192, mb, bar, t.n * BN + q * 64, r0, pol);
           } else {
-            const int32_t row0 = off[t.e] + t.m * BM;
-            tma_load_2d(a, &tmA, bar, kb * BK, row0, pol);
+            const int32_t row0 = (t.seg ? off1 : off)[t.e] + t.ml * BM;
+            tma_load_2d(a, t.seg ? &tmA1 : &tmA, bar, kb * BK, row0, pol);
             if (kMode == kRawGU) {
               const int32_t brow = t.e * p.b_rows + t.n * (BN / 2);
               tma_load_2d(b, &tmB, bar, kb * BK, brow, pol);
@@ -262,7 +274,7 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
       bool ok = true, issued = false;
       int32_t it = 0;
       for (int32_t L = blockIdx.x; L < p.total_tiles && ok; L += gridDim.x, ++it) {
-        const Tile t = decode<kMode>(L, ts, off, E, p);
+        const Tile t = decode<kMode>(L, ts, off, off1, E, p);
         const int32_t nkb = kMode == kWGrad
                                 ? (off[t.e + 1] - off[t.e] + off1[t.e + 1] - off1[t.e]) / BK
                                 : p.num_kb;
@@ -313,14 +325,16 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
     int32_t it = 0;
     for (int32_t L = blockIdx.x; L < p.total_tiles; L += gridDim.x, ++it) {
       const int buf = it & 1;
-      const Tile t = decode<kMode>(L, ts, off, E, p);
+      const Tile t = decode<kMode>(L, ts, off, off1, E, p);
       // kDSwiGLU: the saved g and u of this thread's row, one 32-column block ahead of the
       // accumulator; the first block is requested before the accumulator is ready
       uint4 gq[4], uq[4];
-      const int32_t rows_here = off[t.e + 1] - off[t.e] - t.m * BM;
-      const int64_t row_g = (int64_t)off[t.e] + t.m * BM + r;
+      const int32_t* offs = t.seg ? off1 : off;
+      const int32_t rows_here = offs[t.e + 1] - offs[t.e] - t.ml * BM;
+      const int64_t row_g = (int64_t)offs[t.e] + t.ml * BM + r;
+      const __nv_bfloat16* aux = t.seg ? p.auxb : p.aux;
       auto load_aux = [&](int c, uint4 (&g)[4], uint4 (&u)[4]) {
-        const uint4* gu4 = reinterpret_cast<const uint4*>(p.aux + row_g * 2 * p.I);
+        const uint4* gu4 = reinterpret_cast<const uint4*>(aux + row_g * 2 * p.I);
 #pragma unroll
         for (int v4 = 0; v4 < 4; ++v4) {
           const int32_t cc = t.n * BN + c * 32 + v4 * 8;
@@ -369,9 +383,11 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
           }
         }
       } else {
-        const int32_t rows_valid = off[t.e + 1] - off[t.e] - t.m * BM;
+        const int32_t rows_valid = offs[t.e + 1] - offs[t.e] - t.ml * BM;
         const bool row_ok = r < rows_valid;
-        const int64_t row = (int64_t)off[t.e] + t.m * BM + r;
+        const int64_t row = (int64_t)offs[t.e] + t.ml * BM + r;
+        __nv_bfloat16* o0 = t.seg ? p.out0b : p.out0;
+        __nv_bfloat16* o1 = t.seg ? p.out1b : p.out1;
         if (kMode == kRawGU) {
 #pragma unroll 1
           for (int c = part * kCgu; c < (part + 1) * kCgu; ++c) {
@@ -390,8 +406,8 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
                 pu[i] = pack_bf16x2(u0, u1);
                 ph[i] = pack_bf16x2(silu_f(g0) * u0, silu_f(g1) * u1);
               }
-              __nv_bfloat16* gu = p.out0 + row * 2 * p.I;
-              __nv_bfloat16* act = p.out1 + row * p.I;
+              __nv_bfloat16* gu = o0 + row * 2 * p.I;
+              __nv_bfloat16* act = o1 + row * p.I;
 #pragma unroll
               for (int v4 = 0; v4 < 4; ++v4) {
                 if (col0 + v4 * 8 < p.I) {
@@ -417,7 +433,7 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
             const int32_t col0 = t.n * BN + c * 32;
             if (!row_ok) continue;
             if (kMode == kDSwiGLU) {
-              __nv_bfloat16* dgu = p.out0 + row * 2 * p.I;
+              __nv_bfloat16* dgu = o0 + row * 2 * p.I;
 #pragma unroll
               for (int v4 = 0; v4 < 4; ++v4) {
                 const int32_t cc = col0 + v4 * 8;
@@ -449,7 +465,7 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
                 uq[v4] = un[v4];
               }
             } else {  // kDPlain
-              __nv_bfloat16* o = p.out0 + row * p.N;
+              __nv_bfloat16* o = o0 + row * p.N;
 #pragma unroll
               for (int v4 = 0; v4 < 4; ++v4) {
                 const int32_t cc = col0 + v4 * 8;
@@ -597,10 +613,9 @@ cudaError_t launch_bwd_gemm(const BwdGemmArgs& a, int num_sms, cudaStream_t s) {
   // N tiles: kRawGU pairs 128 gate with 128 up columns per tile; the others are 256 wide
   const int32_t n_tiles = a.mode == kRawGU ? (a.I + BN / 2 - 1) / (BN / 2) : (a.N + BN - 1) / BN;
   for (int32_t e = 0; e < a.E; ++e) {
-    const int64_t rows =
-        a.rows_pad_host[e] + (a.mode == kWGrad && a.rows_pad_host1 ? a.rows_pad_host1[e] : 0);
-    if (a.mode == kWGrad) tiles += rows > 0 ? (int64_t)((a.M + BM - 1) / BM) * n_tiles : 0;
-    else tiles += (rows + BM - 1) / BM * n_tiles;
+    const int64_t r0 = a.rows_pad_host[e], r1 = a.rows_pad_host1 ? a.rows_pad_host1[e] : 0;
+    if (a.mode == kWGrad) tiles += r0 + r1 > 0 ? (int64_t)((a.M + BM - 1) / BM) * n_tiles : 0;
+    else tiles += ((r0 + BM - 1) / BM + (r1 + BM - 1) / BM) * n_tiles;
   }
   if (tiles <= 0) return cudaSuccess;
   if (tiles > 0x7fffffff) return cudaErrorInvalidValue;
@@ -616,12 +631,18 @@ cudaError_t launch_bwd_gemm(const BwdGemmArgs& a, int num_sms, cudaStream_t s) {
   } else {
     mC = mA;  // unused
   }
-  const bool pair = a.mode == kWGrad && a.offsets1 != nullptr;
-  if (pair) {
+  const bool pair = a.offsets1 != nullptr;
+  if (pair && a.mode == kWGrad) {
     if (!a.A1 || !a.B1 || !a.rows_pad_host1 ||
         !make_tma_2d_bf16(&mA1, a.A1, a.A1_rows, a.A_cols, BK) ||
         !make_tma_2d_bf16(&mB1, a.B1, a.B1_rows, a.B_cols, BK))
       return cudaErrorInvalidValue;
+  } else if (pair) {  // a second row segment: its own A rows, the same weights
+    if (!a.A1 || !a.rows_pad_host1 || !a.out0b || (a.mode == kRawGU && !a.out1b) ||
+        (a.mode == kDSwiGLU && !a.auxb) ||
+        !make_tma_2d_bf16(&mA1, a.A1, a.A1_rows, a.A_cols, BM))
+      return cudaErrorInvalidValue;
+    mB1 = mB;  // unused
   } else {
     mA1 = mA;  // unused
     mB1 = mB;
@@ -646,6 +667,9 @@ cudaError_t launch_bwd_gemm(const BwdGemmArgs& a, int num_sms, cudaStream_t s) {
   p.chunk = a.chunk;
   p.chunk_last = pair ? a.chunk + 1 : a.chunk;
   p.offsets1 = pair ? a.offsets1 : nullptr;
+  p.out0b = static_cast<__nv_bfloat16*>(a.out0b);
+  p.out1b = static_cast<__nv_bfloat16*>(a.out1b);
+  p.auxb = static_cast<const __nv_bfloat16*>(a.auxb);
   switch (a.mode) {
     case kRawGU: return launch_mode<kRawGU>(mA, mB, mC, mA1, mB1, p, num_sms, s);
     case kDSwiGLU: return launch_mode<kDSwiGLU>(mA, mB, mC, mA1, mB1, p, num_sms, s);

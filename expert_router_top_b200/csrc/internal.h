@@ -130,6 +130,12 @@ struct BwdGemmArgs {
   int64_t B1_rows;
   const int32_t* offsets1;
   const int32_t* rows_pad_host1;
+  // row-grouped modes over a pair of chunks: the second chunk's rows are a second row
+  // segment of the same tile sweep (A1 its A rows; out0b / out1b / auxb its outputs and
+  // saved g|u rows), so each weight tile is fetched once for both chunks
+  void* out0b;
+  void* out1b;
+  const void* auxb;
   uint32_t* status;
 };
 

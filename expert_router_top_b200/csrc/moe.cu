@@ -200,8 +200,8 @@ struct DeviceCtx {
               ev_copy_join = nullptr;
   // backward pipeline: permuted rows ready (per X slot), recomputed Y ready, dY ready, dX
   // ready, d_hidden rows summed (per buffer), all of a chunk's GEMMs done (per X slot)
-  cudaEvent_t ev_bp[3] = {}, ev_bf[2] = {}, ev_bdy[2] = {}, ev_bdx[2] = {}, ev_bsum[2] = {},
-              ev_bw[3] = {};
+  cudaEvent_t ev_bp[4] = {}, ev_bf[2] = {}, ev_bdy[2] = {}, ev_bdx[2] = {}, ev_bsum[2] = {},
+              ev_bw[4] = {};
   int32_t* host_stage = nullptr;
   size_t host_stage_bytes = 0;
 };
@@ -239,7 +239,7 @@ moe_status_t get_ctx(DeviceCtx** out) {
           cudaEventCreateWithFlags(&c.ev_out_free[b], fl) != cudaSuccess)
         return MOE_ERR_CUDA;
     if (cudaEventCreateWithFlags(&c.ev_copy_join, fl) != cudaSuccess) return MOE_ERR_CUDA;
-    for (int b = 0; b < 3; ++b)
+    for (int b = 0; b < 4; ++b)
       if (cudaEventCreateWithFlags(&c.ev_bp[b], fl) != cudaSuccess ||
           cudaEventCreateWithFlags(&c.ev_bw[b], fl) != cudaSuccess)
         return MOE_ERR_CUDA;
@@ -877,14 +877,15 @@ namespace {
 struct BwdLayout {
   Layout meta;  // metadata regions (status/counts/splits, offsets, histograms, dst, src)
   size_t offp, first, dstp, total;
-  int nx, nb;  // X slots (3 when three or more chunks) and buffer sets of the other rows
-  size_t xp[3], gu[2], act[2], ydx[2], dy[2], dgu[2];
+  int nx, nb;  // X slots (up to 4: two pairs) and buffer sets of the other rows
+  size_t xp[4], gu[2], act[2], ydx[2], dy[2], dgu[2];
   int64_t rows_cap;
 };
 
 // Every chunk's rows, padded per expert to a multiple of 64, fit in rows_cap rows.  The
-// pipeline keeps chunk c's permuted rows in X slot c % 3 (they are read until the chunk's
-// last weight-gradient GEMM) and its other row buffers in set c % 2.
+// pipeline keeps chunk c's permuted rows in X slot c % 4 (they are read until its pair's
+// weight-gradient GEMM, while the next pair is permuted) and its other row buffers in set
+// c % 2.
 BwdLayout make_bwd_layout(const Dims& d, int32_t H, int32_t I) {
   BwdLayout B{};
   B.meta = make_layout(d, 8, 8, false, true, true);
@@ -897,7 +898,7 @@ BwdLayout make_bwd_layout(const Dims& d, int32_t H, int32_t I) {
   B.dstp = o;
   o += al(sizeof(int32_t) * (size_t)(d.T * d.k));
   const size_t R = (size_t)B.rows_cap;
-  B.nx = d.n >= 3 ? 3 : d.n;
+  B.nx = d.n >= 4 ? 4 : d.n;
   B.nb = d.n >= 2 ? 2 : 1;
   for (int b = 0; b < B.nx; ++b) {
     B.xp[b] = o;
@@ -1022,15 +1023,15 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
   auto len = [&](int c) { return bounds[c + 1] - bounds[c]; };
   auto ok = [](cudaError_t e) { return e == cudaSuccess; };
 
-  // P(c), stream M: padded permute of the chunk's rows into X slot c % 3 (zero pad rows)
+  // P(c), stream M: padded permute of the chunk's rows into X slot c % 4 (zero pad rows)
   auto P = [&](int c) -> moe_status_t {
-    if (c >= 3 && !ok(cudaStreamWaitEvent(s, ctx->ev_bw[c % 3], 0))) return MOE_ERR_CUDA;
+    if (c >= 4 && !ok(cudaStreamWaitEvent(s, ctx->ev_bw[c % 4], 0))) return MOE_ERR_CUDA;
     ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(c) * k, 0, 2);
     if (!ok(cudaMemsetAsync(x_of(c), 0, 2 * (size_t)R[c] * H, s)) ||
         !ok(launch_pad_rows(top_k_index + bounds[c] * k, dst + bounds[c] * k, off_c(c), offp_c(c),
                             len(c) * k, dstp_c(c), s)) ||
         !ok(launch_permute(hid + bounds[c] * H, dstp_c(c), len(c), H, k, x_of(c), s)) ||
-        !ok(cudaEventRecord(ctx->ev_bp[c % 3], s)))
+        !ok(cudaEventRecord(ctx->ev_bp[c % 4], s)))
       return MOE_ERR_CUDA;
     return MOE_OK;
   };
@@ -1039,14 +1040,37 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
   g0.I = I;
   g0.status = dev_status;
   g0.first = first;
-  auto bwd_gemm = [&](int kind, const BwdGemmArgs& a, int c) {
-    ProfScope ps(kind, sg, R[c], active_experts(counts.data() + (size_t)c * E, E), 1);
+  // The pair (c, c1): c1 = c + 1, or c1 = c for the last chunk of an odd count.  Every GEMM
+  // of a pair is one tile sweep over both chunks' rows (the second chunk a second row
+  // segment, or for the weight gradients more K), so each weight tile is fetched once per
+  // pair.
+  auto rows_both = [&](int c, int c1) { return R[c] + (c1 > c ? R[c1] : 0); };
+  auto active_both = [&](int c, int c1) {
+    int64_t a = 0;
+    for (int32_t e = 0; e < E; ++e)
+      a += (counts[(size_t)c * E + e] + (c1 > c ? counts[(size_t)c1 * E + e] : 0)) > 0;
+    return a;
+  };
+  auto launch_pair = [&](int kind, const BwdGemmArgs& a, int c, int c1) {
+    ProfScope ps(kind, sg, rows_both(c, c1), active_both(c, c1), 1);
     return launch_bwd_gemm(a, ctx->num_sms, sg);
   };
-  // F(c), stream G: recompute [g u], h and Y = h W_down^T on the padded rows
-  auto F = [&](int c) -> moe_status_t {
-    if (!ok(cudaStreamWaitEvent(sg, ctx->ev_bp[c % 3], 0))) return MOE_ERR_CUDA;
-    if (c >= 2 && !ok(cudaStreamWaitEvent(sg, ctx->ev_bsum[c % 2], 0))) return MOE_ERR_CUDA;
+  // the second chunk of a pair as a row segment of a row-grouped mode
+  auto seg1 = [&](BwdGemmArgs& g, int c1, const void* A1, void* o0, void* o1, const void* aux) {
+    g.offsets1 = offp_c(c1);
+    g.rows_pad_host1 = rows_pad.data() + (size_t)c1 * E;
+    g.A1 = A1;
+    g.A1_rows = R[c1];
+    g.out0b = o0;
+    g.out1b = o1;
+    g.auxb = aux;
+  };
+  // F(c, c1), stream G: recompute [g u], h and Y = h W_down^T on the padded rows
+  auto F = [&](int c, int c1) -> moe_status_t {
+    for (int x = c; x <= c1; ++x) {
+      if (!ok(cudaStreamWaitEvent(sg, ctx->ev_bp[x % 4], 0))) return MOE_ERR_CUDA;
+      if (x >= 2 && !ok(cudaStreamWaitEvent(sg, ctx->ev_bsum[x % 2], 0))) return MOE_ERR_CUDA;
+    }
     BwdGemmArgs g = g0;
     g.offsets = offp_c(c);
     g.rows_pad_host = rows_pad.data() + (size_t)c * E;
@@ -1055,28 +1079,38 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
     g.A = x_of(c), g.A_rows = R[c], g.A_cols = H;
     g.B = W_gate_up, g.B_rows = (int64_t)E * 2 * I, g.B_cols = H;
     g.N = 2 * I, g.K = H, g.b_rows = 2 * I, g.out0 = buf(B.gu, c), g.out1 = buf(B.act, c);
-    if (!ok(bwd_gemm(MOE_KERNEL_BWD_GATEUP, g, c))) return MOE_ERR_CUDA;
+    if (c1 > c) seg1(g, c1, x_of(c1), buf(B.gu, c1), buf(B.act, c1), nullptr);
+    if (!ok(launch_pair(MOE_KERNEL_BWD_GATEUP, g, c, c1))) return MOE_ERR_CUDA;
+    Seg1 d1;
+    if (c1 > c) {
+      d1.A = buf(B.act, c1);
+      d1.rows = R[c1];
+      d1.offsets = offp_c(c1);
+      d1.counts = rows_pad.data() + (size_t)c1 * E;
+      d1.out = buf(B.ydx, c1);
+    }
     moe_status_t s2 = gemm_call(buf(B.act, c), R[c], W_down, buf(B.ydx, c), offp_c(c),
                                 rows_pad.data() + (size_t)c * E, E, I, H, H, false, dev_status,
-                                ctx->num_sms, sg);
+                                ctx->num_sms, sg, nullptr, nullptr, 0, false,
+                                c1 > c ? &d1 : nullptr);
     if (s2 != MOE_OK) return s2;
-    return ok(cudaEventRecord(ctx->ev_bf[c % 2], sg)) ? MOE_OK : MOE_ERR_CUDA;
+    return ok(cudaEventRecord(ctx->ev_bf[0], sg)) ? MOE_OK : MOE_ERR_CUDA;
   };
   // DY(c), stream M: dY = w dout (zero pad rows) and d_weights
   auto DY = [&](int c) -> moe_status_t {
-    if (!ok(cudaStreamWaitEvent(s, ctx->ev_bf[c % 2], 0))) return MOE_ERR_CUDA;
+    if (!ok(cudaStreamWaitEvent(s, ctx->ev_bf[0], 0))) return MOE_ERR_CUDA;
     ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(c) * k, 0, 1);
     if (!ok(cudaMemsetAsync(buf(B.dy, c), 0, 2 * (size_t)R[c] * H, s)) ||
         !ok(launch_dy_dw(dout + bounds[c] * H, buf(B.ydx, c), dstp_c(c),
                          top_k_weights + bounds[c] * k, len(c), H, k, buf(B.dy, c),
                          d_weights + bounds[c] * k, s)) ||
-        !ok(cudaEventRecord(ctx->ev_bdy[c % 2], s)))
+        !ok(cudaEventRecord(ctx->ev_bdy[0], s)))
       return MOE_ERR_CUDA;
     return MOE_OK;
   };
-  // Bd(c), stream G: dh with the SwiGLU backward, then dX
-  auto Bd = [&](int c) -> moe_status_t {
-    if (!ok(cudaStreamWaitEvent(sg, ctx->ev_bdy[c % 2], 0))) return MOE_ERR_CUDA;
+  // Bd(c, c1), stream G: dh with the SwiGLU backward, then dX
+  auto Bd = [&](int c, int c1) -> moe_status_t {
+    if (!ok(cudaStreamWaitEvent(sg, ctx->ev_bdy[0], 0))) return MOE_ERR_CUDA;
     BwdGemmArgs g = g0;
     g.offsets = offp_c(c);
     g.rows_pad_host = rows_pad.data() + (size_t)c * E;
@@ -1085,19 +1119,25 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
     g.A = buf(B.dy, c), g.A_rows = R[c], g.A_cols = H;
     g.B = W_down, g.B_rows = (int64_t)E * H, g.B_cols = I;
     g.N = I, g.K = H, g.b_rows = H, g.out0 = buf(B.dgu, c), g.aux = buf(B.gu, c);
-    if (!ok(bwd_gemm(MOE_KERNEL_BWD_DSWIGLU, g, c))) return MOE_ERR_CUDA;
+    if (c1 > c) seg1(g, c1, buf(B.dy, c1), buf(B.dgu, c1), nullptr, buf(B.gu, c1));
+    if (!ok(launch_pair(MOE_KERNEL_BWD_DSWIGLU, g, c, c1))) return MOE_ERR_CUDA;
+    g = g0;
+    g.offsets = offp_c(c);
+    g.rows_pad_host = rows_pad.data() + (size_t)c * E;
+    g.chunk = c;
     g.mode = kBwdDPlain;
     g.A = buf(B.dgu, c), g.A_rows = R[c], g.A_cols = 2 * I;
     g.B = W_gate_up, g.B_rows = (int64_t)E * 2 * I, g.B_cols = H;
-    g.N = H, g.K = 2 * I, g.b_rows = 2 * I, g.out0 = buf(B.ydx, c), g.aux = nullptr;
-    if (!ok(bwd_gemm(MOE_KERNEL_BWD_DX, g, c)) || !ok(cudaEventRecord(ctx->ev_bdx[c % 2], sg)))
+    g.N = H, g.K = 2 * I, g.b_rows = 2 * I, g.out0 = buf(B.ydx, c);
+    if (c1 > c) seg1(g, c1, buf(B.dgu, c1), buf(B.ydx, c1), nullptr, nullptr);
+    if (!ok(launch_pair(MOE_KERNEL_BWD_DX, g, c, c1)) ||
+        !ok(cudaEventRecord(ctx->ev_bdx[0], sg)))
       return MOE_ERR_CUDA;
     return MOE_OK;
   };
-  // W(c, c1), stream G: both weight gradients over the rows of chunk c and, when c1 > c,
-  // of chunk c1 = c + 1 in the same GEMM (K runs over both chunks' rows of each expert):
+  // W(c, c1), stream G: both weight gradients, K over the rows of both chunks:
   //   dW_down[e] (+)= dY^T h ;  dW_gate_up[e] (+)= [dg du]^T X
-  // An expert's first chunk with rows stores; later launches add.
+  // An expert's first pair with rows stores; later pairs add.
   auto W = [&](int c, int c1) -> moe_status_t {
     BwdGemmArgs g = g0;
     g.offsets = offp_c(c);
@@ -1108,33 +1148,25 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
       g.rows_pad_host1 = rows_pad.data() + (size_t)c1 * E;
       g.A1_rows = g.B1_rows = R[c1];
     }
-    const int64_t rows_both = R[c] + (c1 > c ? R[c1] : 0);
-    std::vector<int32_t> both(counts.begin() + (size_t)c * E, counts.begin() + (size_t)c * E + E);
-    if (c1 > c)
-      for (int32_t e = 0; e < E; ++e) both[e] += counts[(size_t)c1 * E + e];
-    const int64_t active = active_experts(both.data(), E);
-    auto launch = [&](const BwdGemmArgs& a) {
-      ProfScope ps(MOE_KERNEL_BWD_WGRAD, sg, rows_both, active, 1);
-      return launch_bwd_gemm(a, ctx->num_sms, sg);
-    };
     g.mode = kBwdWGrad;
     g.A = buf(B.dy, c), g.A_rows = R[c], g.A_cols = H;
     g.B = buf(B.act, c), g.B_rows = R[c], g.B_cols = I;
     if (c1 > c) g.A1 = buf(B.dy, c1), g.B1 = buf(B.act, c1);
     g.M = H, g.N = I, g.acc = dW_down, g.out0 = nullptr;
-    if (!ok(launch(g))) return MOE_ERR_CUDA;
+    if (!ok(launch_pair(MOE_KERNEL_BWD_WGRAD, g, c, c1))) return MOE_ERR_CUDA;
     g.A = buf(B.dgu, c), g.A_rows = R[c], g.A_cols = 2 * I;
     g.B = x_of(c), g.B_rows = R[c], g.B_cols = H;
     if (c1 > c) g.A1 = buf(B.dgu, c1), g.B1 = x_of(c1);
     g.M = 2 * I, g.N = H, g.acc = dW_gate_up;
-    if (!ok(launch(g)) || !ok(cudaEventRecord(ctx->ev_bw[c % 3], sg)) ||
-        (c1 > c && !ok(cudaEventRecord(ctx->ev_bw[c1 % 3], sg))))
+    if (!ok(launch_pair(MOE_KERNEL_BWD_WGRAD, g, c, c1)) ||
+        !ok(cudaEventRecord(ctx->ev_bw[c % 4], sg)) ||
+        (c1 > c && !ok(cudaEventRecord(ctx->ev_bw[c1 % 4], sg))))
       return MOE_ERR_CUDA;
     return MOE_OK;
   };
   // S(c), stream M: d_hidden rows = sum over the k copies of dX
   auto S = [&](int c) -> moe_status_t {
-    if (!ok(cudaStreamWaitEvent(s, ctx->ev_bdx[c % 2], 0))) return MOE_ERR_CUDA;
+    if (!ok(cudaStreamWaitEvent(s, ctx->ev_bdx[0], 0))) return MOE_ERR_CUDA;
     ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(c) * k, 0, 1);
     if (!ok(launch_sum_rows(buf(B.ydx, c), dstp_c(c), len(c), H, k, dx_out + bounds[c] * H, s)) ||
         !ok(cudaEventRecord(ctx->ev_bsum[c % 2], s)))
@@ -1142,28 +1174,29 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
     return MOE_OK;
   };
 
-  // The mirrored pair pipeline, over pairs of adjacent chunks (c0, c1) = (2m, 2m+1):
-  //   G: F(c0) F(c1) Bd(c0) Bd(c1) W(c0,c1) F(c0+2) F(c1+2) ...
-  //   M: P(c0) P(c1) DY(c0) DY(c1) S(c0) S(c1) P(c0+2) P(c1+2) ...
-  // The row kernels of one chunk overlap the GEMMs of the other chunk of the pair or of the
-  // next pair, and the weight gradients of a pair are one GEMM per weight (half the dW
-  // read-modify-write passes of per-chunk launches).  Host enqueue order keeps each event
-  // wait on the record it is meant for.
+  // The mirrored pair pipeline over pairs (c, c1) = (2m, 2m+1), every GEMM one sweep over
+  // both chunks of the pair:
+  //   G: F(pair m) Bd(pair m) W(pair m) F(pair m+1) ...
+  //   M: P(c) P(c1) | DY(c) DY(c1) P(c+2) P(c+3) S(c) S(c1) | DY(c+2) ...
+  // The next pair's permutes run beside Bd, the d_hidden sums beside W; G waits for the
+  // pair's two DY row kernels between F and Bd.  Host enqueue order keeps each event wait
+  // on the record it is meant for.
   if (!ok(cudaEventRecord(ctx->ev_start, s)) || !ok(cudaStreamWaitEvent(sg, ctx->ev_start, 0)))
     return MOE_ERR_CUDA;
   if (n_live > 0) {
-    if ((st = P(0)) != MOE_OK || (st = F(0)) != MOE_OK) return st;
-    if (n_live > 1 && ((st = P(1)) != MOE_OK || (st = F(1)) != MOE_OK)) return st;
-    for (int c0 = 0; c0 < n_live; c0 += 2) {
-      const int c1 = c0 + 1 < n_live ? c0 + 1 : c0;
-      if ((st = DY(c0)) != MOE_OK || (c1 > c0 && (st = DY(c1)) != MOE_OK)) return st;
-      if ((st = Bd(c0)) != MOE_OK || (c1 > c0 && (st = Bd(c1)) != MOE_OK)) return st;
-      if ((st = S(c0)) != MOE_OK || (c1 > c0 && (st = S(c1)) != MOE_OK)) return st;
-      if (c0 + 2 < n_live && (st = P(c0 + 2)) != MOE_OK) return st;
-      if ((st = W(c0, c1)) != MOE_OK) return st;
-      if (c0 + 3 < n_live && (st = P(c0 + 3)) != MOE_OK) return st;
-      if (c0 + 2 < n_live && (st = F(c0 + 2)) != MOE_OK) return st;
-      if (c0 + 3 < n_live && (st = F(c0 + 3)) != MOE_OK) return st;
+    auto pair_end = [&](int c) { return c + 1 < n_live ? c + 1 : c; };
+    if ((st = P(0)) != MOE_OK) return st;
+    if (n_live > 1 && (st = P(1)) != MOE_OK) return st;
+    if ((st = F(0, pair_end(0))) != MOE_OK) return st;
+    for (int c = 0; c < n_live; c += 2) {
+      const int c1 = pair_end(c);
+      if ((st = DY(c)) != MOE_OK || (c1 > c && (st = DY(c1)) != MOE_OK)) return st;
+      for (int x = c + 2; x <= c + 3 && x < n_live; ++x)
+        if ((st = P(x)) != MOE_OK) return st;
+      if ((st = Bd(c, c1)) != MOE_OK) return st;
+      if ((st = S(c)) != MOE_OK || (c1 > c && (st = S(c1)) != MOE_OK)) return st;
+      if ((st = W(c, c1)) != MOE_OK) return st;
+      if (c + 2 < n_live && (st = F(c + 2, pair_end(c + 2))) != MOE_OK) return st;
     }
   }
   if (!ok(cudaEventRecord(ctx->ev_join, sg)) || !ok(cudaStreamWaitEvent(s, ctx->ev_join, 0)))

@@ -8,7 +8,7 @@ import pytest
 import torch
 
 import oracle
-from gen import CONFIGS, bits, expert_weights, hidden, layer_inputs, routing
+from gen import CONFIGS, LayerConfig, bits, expert_weights, hidden, layer_inputs, routing
 from parity import assert_layer_close, to_f64
 
 pytestmark = pytest.mark.gpu
@@ -205,3 +205,26 @@ def test_forward_full_size_sampled(moe, name, n_tok):
         assert torch.equal(_run(moe, gpu, cfg.chunks[-1], cfg.G, dispatch), base), dispatch
     # properties at full size: finite everywhere
     assert bool(torch.isfinite(base.float()).all())
+
+
+@pytest.mark.parametrize("E,k,T,H,I", [(1024, 8, 1536, 128, 128),   # MOE_MAX_EXPERTS
+                                       (64, 32, 600, 256, 192),     # MOE_MAX_TOPK
+                                       (1, 1, 300, 64, 64),         # one expert, top-1
+                                       (16, 4, 257, 136, 200)])     # H, I not multiples of 64
+def test_forward_limits_and_odd_shapes(moe, E, k, T, H, I):
+    """The kernels' table and tile limits: the most experts and the largest top-k the ABI
+    takes, a single expert, and widths that are multiples of 8 but not of the 64-wide K
+    block or the 128-wide column tiles (the K tail reads zeros, the column tail is never
+    written), every dispatch, several chunk counts; every element against the oracle."""
+    cfg = LayerConfig("limits", T, H, E, k, I, "normal")
+    cpu = layer_inputs(cfg)
+    gpu = {kk: v.cuda() for kk, v in cpu.items()}
+    ref = _oracle(cpu)
+    base = None
+    for N in (1, 3, 4):
+        for dispatch in ("separate", "fused"):
+            out = _run(moe, gpu, N, 1, dispatch)
+            assert_layer_close(out, ref, f"E={E} k={k} H={H} I={I} N={N} {dispatch}")
+            if base is None:
+                base = out
+            assert torch.equal(out, base), f"N={N} {dispatch} differs"
