@@ -418,7 +418,9 @@ def run_ours(args, cfg):
     gu_flops_l = units["gateup_flops"] / n_gu
     gu_bytes_l = units["gateup_alg_bytes"] / n_gu
     t_l = g["ms"] / max(1, g["launches"]) / 1e3  # s per launch
-    peak_tc, peak_bw = peaks["bf16_tflops"], peaks["hbm_gbs"]
+    # the dominant kernel runs inside a long sequence of steps (after the clock spin-up, at
+    # the power-capped clock): the sustained bf16 figure is its tensor roof
+    peak_tc, peak_bw = peaks["bf16_tflops_sustained"], peaks["hbm_gbs"]
     t_tensor = gu_flops_l / (peak_tc * 1e12)
     t_mem = gu_bytes_l / (peak_bw * 1e9)
     traffic = traffic_per_launch(cfg.name, chunks, dispatch, pair_gemms)
@@ -433,15 +435,13 @@ def run_ours(args, cfg):
         "traffic": traffic,
         "kernel": "grouped_gemm_kernel<gate/up + SwiGLU" + (", gathered A rows" if dispatch == "fused"
                                                              else "") + "> (tcgen05)",
-        "peak_source": f"{peak_src}: MEASURED_PEAKS.json (bf16 burst, HBM copy)",
+        "peak_source": f"{peak_src}: MEASURED_PEAKS.json (bf16 sustained, HBM copy)",
         "per_launch": {"flops": gu_flops_l, "bytes": gu_bytes_l, "ms": t_l * 1e3,
                        "roofline_ms": max(t_tensor, t_mem) * 1e3},
         "frac_of_roofline_time": max(t_tensor, t_mem) / t_l if t_l else None,
         "tensor_frac": gu_flops_l / t_l / 1e12 / peak_tc if t_l else None,
-        "tensor_frac_of_sustained": gu_flops_l / t_l / 1e12 / peaks["bf16_tflops_sustained"]
-        if t_l else None,
+        "tensor_frac_of_burst": gu_flops_l / t_l / 1e12 / peaks["bf16_tflops"] if t_l else None,
         "hbm_frac": gu_bytes_l / t_l / 1e9 / peak_bw if t_l else None})
-    peak_tc = peaks["bf16_tflops"]
 
     ws_per_n = {str(n): moe.workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.G, n)
                 for n in (1, 2, 4)}
@@ -451,7 +451,8 @@ def run_ours(args, cfg):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; random-init expert weights of the layer's shape)",
         "config": dict(config_block(cfg, chunks, dispatch),
-                       gemm_sweep="per pair of chunks" if pair_gemms else "per chunk"),
+                       gemm_sweep="per pair of chunks" if pair_gemms and n_live > 1
+                       else "per chunk"),
         "roofline": roofline,
         "grouped_gemm_tflops": gemm_tflops,
         "grouped_gemm_frac_of_peak": gemm_tflops / peak_tc,
@@ -581,23 +582,24 @@ def run_backward(args, cfg):
     wg = prof["bwd_wgrad"]
     t = wg["ms"] / steps / 1e3
     f, b = units["flops"]["bwd_wgrad"], units["wgrad_bytes"]
-    t_tensor, t_mem = f / (peaks["bf16_tflops"] * 1e12), b / (peaks["hbm_gbs"] * 1e9)
+    peak_tc = peaks["bf16_tflops_sustained"]  # long step sequence, power-capped clock
+    t_tensor, t_mem = f / (peak_tc * 1e12), b / (peaks["hbm_gbs"] * 1e9)
     if t_mem > t_tensor:
         roofline = {"bound": "hbm", "achieved": b / t / 1e9, "peak": peaks["hbm_gbs"],
                     "unit": "GB/s"}
     else:
-        roofline = {"bound": "tensor", "achieved": f / t / 1e12, "peak": peaks["bf16_tflops"],
+        roofline = {"bound": "tensor", "achieved": f / t / 1e12, "peak": peak_tc,
                     "unit": "TFLOP/s"}
     roofline["frac"] = roofline["achieved"] / roofline["peak"]
     n_wg = max(1, wg["launches"] // max(1, steps))
     roofline.update({
         "traffic": None,
         "kernel": "bwd_gemm_kernel<weight gradient> (tcgen05, TMA store / add-reduce epilogue)",
-        "peak_source": f"{peak_src}: MEASURED_PEAKS.json (bf16 burst, HBM copy)",
+        "peak_source": f"{peak_src}: MEASURED_PEAKS.json (bf16 sustained, HBM copy)",
         "per_launch": {"flops": f / n_wg, "bytes": b / n_wg, "ms": t * 1e3 / n_wg,
                        "roofline_ms": max(t_tensor, t_mem) * 1e3 / n_wg},
-        "tensor_frac": f / t / 1e12 / peaks["bf16_tflops"],
-        "tensor_frac_of_sustained": f / t / 1e12 / peaks["bf16_tflops_sustained"],
+        "tensor_frac": f / t / 1e12 / peak_tc,
+        "tensor_frac_of_burst": f / t / 1e12 / peaks["bf16_tflops"],
         "hbm_frac": b / t / 1e9 / peaks["hbm_gbs"]})
     gemm_fl = sum(v for k2, v in units["flops"].items())
     gemm_ms = sum(prof[k2]["ms"] for k2 in units["flops"]) / steps

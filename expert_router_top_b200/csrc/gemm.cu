@@ -651,8 +651,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
           for (int i = 0; i < 16; ++i) {
             const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
             const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
-            const float a0 = g0 / (1.0f + __expf(-g0)) * u0;
-            const float a1 = g1 / (1.0f + __expf(-g1)) * u1;
+            // silu(g) = g / (1 + e^-g); the fast division (no IEEE slow path) is exact to a
+            // few ulp, far below the bf16 rounding of the result
+            const float a0 = __fdividef(g0, 1.0f + __expf(-g0)) * u0;
+            const float a1 = __fdividef(g1, 1.0f + __expf(-g1)) * u1;
             packed[i] = pack_bf16x2(a0, a1);
           }
           store_block(packed, wbuf, lane, q, row_ok, rows_valid, row_base, col0, p, out);
