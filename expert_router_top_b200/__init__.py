@@ -84,6 +84,8 @@ def load():
     L.moe_forward_ex.argtypes = [ctypes.POINTER(Shape), p, p, p, p, p, p, p, sz, ctypes.c_uint32,
                                  p]
     L.moe_forward_ex.restype = st
+    L.moe_selftest_wait_timeout.argtypes = [p, ctypes.c_uint32, p]
+    L.moe_selftest_wait_timeout.restype = st
     L.moe_forward_dispatch.argtypes = [ctypes.POINTER(Shape), ctypes.c_uint32]
     L.moe_forward_dispatch.restype = i32
     L.moe_workspace_bytes_host.argtypes = [ctypes.POINTER(Shape)]
@@ -427,6 +429,14 @@ def unpermute(Y, dst_rows, top_k_weights, k: int, out=None, stream=None):
     _check(load().moe_unpermute(_ptr(Y), _ptr(dst_rows), _ptr(top_k_weights), Tc, H, k, _ptr(out),
                                 _stream(stream)), "moe_unpermute")
     return out
+
+
+def selftest_wait_timeout(limit_us: int = 20000, stream=None):
+    """Run the failure-detection self-test: a device wait that nothing completes must give
+    up after limit_us and report a timeout.  Returns the status code (MOE_ERR_TIMEOUT = 6
+    is the expected outcome); never raises for it."""
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    return int(load().moe_selftest_wait_timeout(_ptr(status), limit_us, _stream(stream)))
 
 
 def profile_enable(on: bool = True):

@@ -11,7 +11,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmoe.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
-SOURCES = ["metadata.cu", "permute.cu", "gemm.cu", "moe.cu", "noalloc.cu", "backward.cu"]
+SOURCES = ["metadata.cu", "permute.cu", "gemm.cu", "moe.cu", "noalloc.cu", "backward.cu", "selftest.cu"]
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",

@@ -68,17 +68,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 }
 
 // Bounded wait for the phase with the given parity.  Returns false when it gave up: on
-// its own timeout (then it sets *abort and ORs MOE_DEV_TIMEOUT into *status) or because
-// another role of the CTA already raised *abort.
+// its own timeout after limit_ns (then it sets *abort and ORs MOE_DEV_TIMEOUT into *status)
+// or because another role of the CTA already raised *abort.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          uint32_t* status) {
+                                          uint32_t* status, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t n = 1;; ++n) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((n & 31u) == 0) {
       if (*abort) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         *abort = 1;
         atomicOr(status, MOE_DEV_TIMEOUT);
         return false;

@@ -24,6 +24,8 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "device.cuh"
 #include "internal.h"
 #include "moe.h"
@@ -319,6 +321,18 @@ struct ProfScope {
 
 moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
+// NVTX range on the host timeline around the enqueue of one call, pair or chunk (a profiler
+// such as Nsight Systems shows it beside the kernels it launched; without one attached the
+// push and pop are no-ops).
+struct NvtxRange {
+  explicit NvtxRange(const char* fmt, int a = 0, int b = 0) {
+    char buf[96];
+    snprintf(buf, sizeof buf, fmt, a, b);
+    nvtxRangePushA(buf);
+  }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+
 moe_status_t run_metadata(const Dims& d, const int32_t* idx, uint8_t* ws, const Layout& L,
                           int32_t* dst, int32_t* src, cudaStream_t s) {
   MetaArgs a;
@@ -570,6 +584,7 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
                             const int32_t* top_k_index, const float* top_k_weights,
                             const void* W_gate_up, const void* W_down, void* out,
                             void* workspace, size_t ws_bytes, uint32_t flags, void* stream) {
+  NvtxRange range("moe_forward");
   moe_status_t st = check_shape(shape);
   if (st != MOE_OK) return st;
   const int32_t choice = moe_forward_dispatch(shape, flags);
@@ -684,6 +699,7 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
       return g1;
     };
     for (int c0 = 0; c0 < n_live; c0 += 2) {
+      NvtxRange pr("moe_forward pair: chunks %d-%d", c0, c0 + 1 < n_live ? c0 + 1 : c0);
       const bool two = c0 + 1 < n_live;
       const int c1 = c0 + 1;
       const Seg1 s0 = seg(c0, nullptr, act(c0));
@@ -732,7 +748,22 @@ size_t moe_workspace_bytes_host(const moe_shape_t* s) {
   return make_host_staging(d, s->H, L.total).total;
 }
 
+moe_status_t moe_forward_host_impl(const moe_shape_t* shape, const void* hidden_host,
+                                   const int32_t* top_k_index_host,
+                                   const float* top_k_weights_host, const void* W_gate_up,
+                                   const void* W_down, void* out_host, void* workspace,
+                                   size_t ws_bytes, void* stream);
+
 moe_status_t moe_forward_host(const moe_shape_t* shape, const void* hidden_host,
+                              const int32_t* top_k_index_host, const float* top_k_weights_host,
+                              const void* W_gate_up, const void* W_down, void* out_host,
+                              void* workspace, size_t ws_bytes, void* stream) {
+  NvtxRange range("moe_forward_host");
+  return moe_forward_host_impl(shape, hidden_host, top_k_index_host, top_k_weights_host,
+                               W_gate_up, W_down, out_host, workspace, ws_bytes, stream);
+}
+
+moe_status_t moe_forward_host_impl(const moe_shape_t* shape, const void* hidden_host,
                               const int32_t* top_k_index_host, const float* top_k_weights_host,
                               const void* W_gate_up, const void* W_down, void* out_host,
                               void* workspace, size_t ws_bytes, void* stream) {
@@ -940,6 +971,7 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
                           const void* W_gate_up, const void* W_down, const void* d_out,
                           void* d_hidden, float* d_weights, float* dW_gate_up, float* dW_down,
                           void* workspace, size_t ws_bytes, void* stream) {
+  NvtxRange range("moe_backward");
   moe_status_t st = check_bwd_shape(shape);
   if (st != MOE_OK) return st;
   const int64_t T = shape->T;
@@ -1190,6 +1222,7 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
     if ((st = F(0, pair_end(0))) != MOE_OK) return st;
     for (int c = 0; c < n_live; c += 2) {
       const int c1 = pair_end(c);
+      NvtxRange pr("moe_backward pair: chunks %d-%d", c, c1);
       if ((st = DY(c)) != MOE_OK || (c1 > c && (st = DY(c1)) != MOE_OK)) return st;
       for (int x = c + 2; x <= c + 3 && x < n_live; ++x)
         if ((st = P(x)) != MOE_OK) return st;

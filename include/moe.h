@@ -348,6 +348,16 @@ MOE_API moe_status_t moe_grouped_down(const void* Act, int64_t rows, int32_t H, 
 MOE_API moe_status_t moe_unpermute(const void* Y, const int32_t* dst_rows, const float* top_k_weights,
                            int64_t Tc, int32_t H, int32_t k, void* out, void* stream);
 
+/* ---- Failure-detection self-test -------------------------------------------------------
+ * Not part of the Chunk MoE method (the article has no counterpart): it exercises the
+ * library's own failure detection.  Launches one kernel whose bounded mbarrier wait has
+ * no arrival to wait for; after limit_us microseconds (1 .. 1000000) the wait gives up,
+ * sets MOE_DEV_TIMEOUT in *status (dev uint32, overwritten) and the kernel returns, the
+ * CUDA context stays usable.  Blocks the host until the kernel ends.  Returns
+ * MOE_ERR_TIMEOUT when the timeout was reported (the expected outcome), MOE_OK if the
+ * wait completed, MOE_ERR_ARG / MOE_ERR_ALIGN / MOE_ERR_CUDA otherwise. */
+MOE_API moe_status_t moe_selftest_wait_timeout(uint32_t* status, uint32_t limit_us, void* stream);
+
 /* ---- Kernel timing -----------------------------------------------------------------
  * When enabled, every kernel launch of the calls above is bracketed by two CUDA events
  * recorded on the stream the kernel is launched on.  moe_profile_read synchronizes the

@@ -244,3 +244,12 @@ def test_forward_dispatch_choice():
     assert L.moe_forward_dispatch(ctypes.byref(s), 3) == -1
     assert L.moe_forward_dispatch(ctypes.byref(s), 8) == -1
     assert L.moe_forward_dispatch(ctypes.byref(s), 4) == 0  # a valid flag; auto: separate here
+
+
+def test_selftest_argument_checks_run_on_host():
+    L = moe.load()
+    v = ctypes.c_void_p
+    assert L.moe_selftest_wait_timeout(None, 1000, None) == 1          # null status
+    assert L.moe_selftest_wait_timeout(v(FAKE), 0, None) == 1          # limit 0
+    assert L.moe_selftest_wait_timeout(v(FAKE), 2000000, None) == 1    # limit above 1 s
+    assert L.moe_selftest_wait_timeout(v(FAKE + 2), 1000, None) == 3   # misaligned

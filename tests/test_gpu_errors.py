@@ -58,3 +58,20 @@ def test_all_tokens_to_one_expert(moe):
     torch.cuda.synchronize()
     assert torch.equal(a, b)
     assert bool(torch.isfinite(a.float()).all())
+
+
+def test_bounded_wait_gives_up_and_reports_timeout(moe):
+    """Failure detection on the device: a bounded mbarrier wait that nothing completes gives
+    up after its limit (20 ms here), reports MOE_ERR_TIMEOUT through the status word and
+    returns; the context stays usable (a forward right after it matches one before it)."""
+    import time
+    cfg = CONFIGS["tiny"]
+    gpu = {k: v.cuda() for k, v in layer_inputs(cfg).items()}
+    before = moe.forward(gpu["hidden"], gpu["idx"], gpu["w"], gpu["wgu"], gpu["wd"], num_chunks=2)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    assert moe.selftest_wait_timeout(20000) == 6  # MOE_ERR_TIMEOUT
+    assert time.perf_counter() - t0 < 5.0
+    after = moe.forward(gpu["hidden"], gpu["idx"], gpu["w"], gpu["wgu"], gpu["wd"], num_chunks=2)
+    torch.cuda.synchronize()
+    assert torch.equal(before, after)
