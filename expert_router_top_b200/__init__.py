@@ -18,7 +18,9 @@ import numpy as np
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libmoe.so")
+# MOE_LIBRARY=checks selects the range-checked build (libmoe_checks.so), used by its tests.
+LIB_PATH = os.path.join(_PKG, "libmoe_checks.so" if os.environ.get("MOE_LIBRARY") == "checks"
+                        else "libmoe.so")
 
 MOE_OK = 0
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_ARG", 2: "MOE_ERR_INDEX", 3: "MOE_ERR_ALIGN",
@@ -84,6 +86,10 @@ def load():
     L.moe_forward_ex.argtypes = [ctypes.POINTER(Shape), p, p, p, p, p, p, p, sz, ctypes.c_uint32,
                                  p]
     L.moe_forward_ex.restype = st
+    L.moe_checks_enabled.argtypes = []
+    L.moe_checks_enabled.restype = i32
+    L.moe_checks_read.argtypes = [p]
+    L.moe_checks_read.restype = st
     L.moe_selftest_wait_timeout.argtypes = [p, ctypes.c_uint32, p]
     L.moe_selftest_wait_timeout.restype = st
     L.moe_forward_dispatch.argtypes = [ctypes.POINTER(Shape), ctypes.c_uint32]
@@ -429,6 +435,19 @@ def unpermute(Y, dst_rows, top_k_weights, k: int, out=None, stream=None):
     _check(load().moe_unpermute(_ptr(Y), _ptr(dst_rows), _ptr(top_k_weights), Tc, H, k, _ptr(out),
                                 _stream(stream)), "moe_unpermute")
     return out
+
+
+def checks_enabled() -> bool:
+    """True when the loaded library is the range-checked build."""
+    return bool(load().moe_checks_enabled())
+
+
+def checks_read() -> int:
+    """Range-violation flags raised since the last read (0: every row index was in range);
+    clears them.  Always 0 with the regular build."""
+    flags = ctypes.c_uint32(0)
+    _check(load().moe_checks_read(ctypes.byref(flags)), "moe_checks_read")
+    return int(flags.value)
 
 
 def selftest_wait_timeout(limit_us: int = 20000, stream=None):

@@ -52,6 +52,8 @@ constexpr int kPadRows = 64;  // backward rows of one expert are padded to this 
 
 enum Mode { kRawGU = 0, kDSwiGLU = 1, kDPlain = 2, kWGrad = 3 };
 
+__device__ uint32_t g_range_flags;  // checks build: a row index outside its buffer was seen
+
 struct BParams {
   const int32_t* offsets;  // padded expert row offsets [E+1] (multiples of 64)
   uint32_t* status;
@@ -74,6 +76,7 @@ struct BParams {
   const int32_t* offsets1;  // padded offsets [E+1] of the pair's second chunk, or null: for
                             // kWGrad its rows extend K; for the row-grouped modes they are a
                             // second row segment of the same tile sweep (A rows from tmA1)
+  int64_t rows0, rows1;     // checks build: rows of the A / output buffers of each segment
   __nv_bfloat16* out0b;     // row-grouped modes: out0 / out1 / aux of the second segment
   __nv_bfloat16* out1b;
   const __nv_bfloat16* auxb;
@@ -384,8 +387,9 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
         }
       } else {
         const int32_t rows_valid = offs[t.e + 1] - offs[t.e] - t.ml * BM;
-        const bool row_ok = r < rows_valid;
         const int64_t row = (int64_t)offs[t.e] + t.ml * BM + r;
+        const bool row_ok =
+            r < rows_valid && check_row(row, t.seg ? p.rows1 : p.rows0, &g_range_flags);
         __nv_bfloat16* o0 = t.seg ? p.out0b : p.out0;
         __nv_bfloat16* o1 = t.seg ? p.out1b : p.out1;
         if (kMode == kRawGU) {
@@ -524,11 +528,12 @@ __global__ void first_chunk_kernel(const int32_t* counts, int32_t E, int32_t n_c
 
 // Padded row of each copy of one chunk: dstp = dst - off[e] + offp[e].
 __global__ void pad_rows_kernel(const int32_t* idx, const int32_t* dst, const int32_t* off,
-                                const int32_t* offp, int64_t n, int32_t* dstp) {
+                                const int32_t* offp, int64_t n, int32_t* dstp, int64_t rows_cap) {
   const int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (s >= n) return;
   const int32_t e = idx[s];
-  dstp[s] = dst[s] - off[e] + offp[e];
+  const int32_t d = dst[s] - off[e] + offp[e];
+  dstp[s] = check_row(d, rows_cap, &g_range_flags) ? d : 0;
 }
 
 // dY[dstp(t,j)] = bf16(w[t][j] * dout[t]) and d_w[t][j] = <dout[t], Y[dstp(t,j)]> (fp32,
@@ -536,12 +541,14 @@ __global__ void pad_rows_kernel(const int32_t* idx, const int32_t* dst, const in
 __global__ void __launch_bounds__(kRowThreads)
     dy_dw_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ Y,
                  const int32_t* __restrict__ dstp, const float* __restrict__ w, int64_t Tc,
-                 int32_t H8, int32_t k, uint4* __restrict__ dY, float* __restrict__ dw) {
+                 int32_t H8, int32_t k, uint4* __restrict__ dY, float* __restrict__ dw,
+                 int64_t rows_cap) {
   const int64_t t = (int64_t)blockIdx.x * kTokPerCta + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= Tc) return;
   for (int j = 0; j < k; ++j) {
     const int32_t d = dstp[t * k + j];
+    if (!check_row(d, rows_cap, &g_range_flags)) continue;  // d is the same in every lane
     const float wj = w[t * k + j];
     float dot = 0.f;
     for (int32_t v = lane; v < H8; v += 32) {
@@ -567,14 +574,16 @@ __global__ void __launch_bounds__(kRowThreads)
 // d_hidden[t] = bf16( sum_{j<k} dX[dstp(t,j)] ), fp32 in ascending j.
 __global__ void __launch_bounds__(kRowThreads)
     sum_rows_kernel(const uint4* __restrict__ dX, const int32_t* __restrict__ dstp, int64_t Tc,
-                    int32_t H8, int32_t k, uint4* __restrict__ out) {
+                    int32_t H8, int32_t k, uint4* __restrict__ out, int64_t rows_cap) {
   const int64_t t = (int64_t)blockIdx.x * kTokPerCta + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= Tc) return;
   for (int32_t v = lane; v < H8; v += 32) {
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     for (int j = 0; j < k; ++j) {
-      const uint4 x = dX[(int64_t)dstp[t * k + j] * H8 + v];
+      const int32_t d = dstp[t * k + j];
+      if (!check_row(d, rows_cap, &g_range_flags)) continue;
+      const uint4 x = dX[(int64_t)d * H8 + v];
       const uint32_t xa[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -667,6 +676,8 @@ cudaError_t launch_bwd_gemm(const BwdGemmArgs& a, int num_sms, cudaStream_t s) {
   p.chunk = a.chunk;
   p.chunk_last = pair ? a.chunk + 1 : a.chunk;
   p.offsets1 = pair ? a.offsets1 : nullptr;
+  p.rows0 = a.A_rows;
+  p.rows1 = a.A1_rows;
   p.out0b = static_cast<__nv_bfloat16*>(a.out0b);
   p.out1b = static_cast<__nv_bfloat16*>(a.out1b);
   p.auxb = static_cast<const __nv_bfloat16*>(a.auxb);
@@ -687,27 +698,39 @@ cudaError_t launch_pad_offsets(const int32_t* counts, int32_t E, int32_t n_chunk
 }
 
 cudaError_t launch_pad_rows(const int32_t* idx, const int32_t* dst, const int32_t* off,
-                            const int32_t* offp, int64_t n, int32_t* dstp, cudaStream_t s) {
+                            const int32_t* offp, int64_t n, int32_t* dstp, int64_t rows_cap,
+                            cudaStream_t s) {
   if (n <= 0) return cudaSuccess;
-  pad_rows_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(idx, dst, off, offp, n, dstp);
+  pad_rows_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(idx, dst, off, offp, n, dstp,
+                                                               rows_cap);
   return cudaGetLastError();
 }
 
 cudaError_t launch_dy_dw(const void* dout, const void* Y, const int32_t* dstp, const float* w,
-                         int64_t Tc, int32_t H, int32_t k, void* dY, float* dw, cudaStream_t s) {
+                         int64_t Tc, int32_t H, int32_t k, void* dY, float* dw, int64_t rows_cap,
+                         cudaStream_t s) {
   if (Tc <= 0) return cudaSuccess;
   dy_dw_kernel<<<row_grid(Tc), kRowThreads, 0, s>>>(
       static_cast<const uint4*>(dout), static_cast<const uint4*>(Y), dstp, w, Tc, H / 8, k,
-      static_cast<uint4*>(dY), dw);
+      static_cast<uint4*>(dY), dw, rows_cap);
   return cudaGetLastError();
 }
 
 cudaError_t launch_sum_rows(const void* dX, const int32_t* dstp, int64_t Tc, int32_t H, int32_t k,
-                            void* out, cudaStream_t s) {
+                            void* out, int64_t rows_cap, cudaStream_t s) {
   if (Tc <= 0) return cudaSuccess;
   sum_rows_kernel<<<row_grid(Tc), kRowThreads, 0, s>>>(static_cast<const uint4*>(dX), dstp, Tc,
-                                                       H / 8, k, static_cast<uint4*>(out));
+                                                       H / 8, k, static_cast<uint4*>(out),
+                                                       rows_cap);
   return cudaGetLastError();
+}
+
+uint32_t checks_take_backward() {
+  uint32_t v = 0, zero = 0;
+  if (!MOE_CHECKS) return 0;
+  cudaMemcpyFromSymbol(&v, g_range_flags, sizeof v);
+  cudaMemcpyToSymbol(g_range_flags, &zero, sizeof zero);
+  return v;
 }
 
 }  // namespace moe

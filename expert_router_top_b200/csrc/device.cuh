@@ -18,6 +18,23 @@ constexpr uint32_t MOE_DEV_TIMEOUT = 2u;
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any wait of a correct run
 
+// Range-checked build (-DMOE_CHECKS=1, libmoe_checks.so): every data-dependent row index is
+// compared with the rows of the buffer it addresses before the access; a violation skips
+// the access and sets a flag that moe_checks_read reports.  No assert, no trap.
+#ifndef MOE_CHECKS
+#define MOE_CHECKS 0
+#endif
+
+// Checks build: true when row d lies inside a buffer of `rows` rows, else records the
+// violation in *flag (one word per translation unit) and returns false.  Always true, and
+// free, in the regular build.
+__device__ __forceinline__ bool check_row(int64_t d, int64_t rows, uint32_t* flag) {
+  if (!MOE_CHECKS) return true;
+  if (d >= 0 && d < rows) return true;
+  atomicOr(flag, 1u);
+  return false;
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

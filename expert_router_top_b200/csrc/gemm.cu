@@ -127,6 +127,8 @@ struct KParams {
   const int32_t* offsets1;
   __nv_bfloat16* out1;
   const int32_t* gather1;
+  int64_t gsrc_rows;             // checks build: rows of the gathered source
+  int64_t out_rows0, out_rows1;  // checks build: rows of out and out1
   int32_t reverse;        // 1: walk the tiles (hence the experts) in descending order
   int32_t b4d;            // 1: tmB is the 4-D gate/up view (one box per stage)
 };
@@ -173,6 +175,8 @@ struct Tile {
   int32_t e, n, m, seg, ml;
 };
 
+__device__ uint32_t g_range_flags;  // checks build: a row index outside its buffer was seen
+
 template <int kTileM>
 __device__ __forceinline__ Tile decode_tile(int32_t L, const int32_t* tile_start,
                                             const int32_t* off, const int32_t* off1, int32_t E,
@@ -212,7 +216,7 @@ __device__ __forceinline__ Tile decode_tile(int32_t L, const int32_t* tile_start
 __device__ __forceinline__ void store_block(const uint32_t (&packed)[16], uint8_t* wbuf, int lane,
                                             int q, bool row_ok, int32_t rows_valid,
                                             int64_t row_base, int32_t col0, const KParams& p,
-                                            __nv_bfloat16* out) {
+                                            __nv_bfloat16* out, int64_t out_rows) {
 #if MOE_GEMM_EPI_STAGE
   uint4* mine = reinterpret_cast<uint4*>(wbuf + lane * kEpiRowBytes);
 #pragma unroll
@@ -227,7 +231,8 @@ __device__ __forceinline__ void store_block(const uint32_t (&packed)[16], uint8_
     const int rr = pass * 8 + (lane >> 2);
     const uint4 v = *reinterpret_cast<const uint4*>(wbuf + rr * kEpiRowBytes + seg * 16);
     const int32_t tr = q * 32 + rr;  // row inside the CTA's 128 rows
-    if (tr < rows_valid && col < p.out_cols)
+    if (tr < rows_valid && col < p.out_cols &&
+        check_row(row_base + tr, out_rows, &g_range_flags))
       *reinterpret_cast<uint4*>(out + (row_base + tr) * p.out_cols + col) = v;
   }
   __syncwarp();
@@ -235,7 +240,7 @@ __device__ __forceinline__ void store_block(const uint32_t (&packed)[16], uint8_
 #else
   (void)wbuf;
   (void)rows_valid;
-  if (row_ok) {
+  if (row_ok && check_row(row_base + q * 32 + lane, out_rows, &g_range_flags)) {
     uint4* dst = reinterpret_cast<uint4*>(out + (row_base + q * 32 + lane) * p.out_cols + col0);
 #pragma unroll
     for (int v = 0; v < 4; ++v)
@@ -442,7 +447,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int32_t r = gw * 32 + 4 * i + sub;
-        src[i] = p.gsrc + (int64_t)gat[min(row0 + r, last)] * p.gsrc_stride + j * 16;
+        int64_t tok = gat[min(row0 + r, last)];
+        if (!check_row(tok, p.gsrc_rows, &g_range_flags)) tok = 0;
+        src[i] = p.gsrc + tok * p.gsrc_stride + j * 16;
       }
       for (int32_t kb = 0; kb < p.num_kb; ++kb) {
         if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort, p.status)) {
@@ -633,6 +640,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
                                             off, off1p, E, p.n_tiles);
       const int32_t* offs = t.seg ? off1 : off;
       __nv_bfloat16* out = t.seg ? p.out1 : p.out;
+      const int64_t out_rows = t.seg ? p.out_rows1 : p.out_rows0;
       const int32_t first = t.ml * G::kTileM + (int32_t)rank * kRowsPerCta;  // in the expert
       const int32_t rows_valid = offs[t.e + 1] - offs[t.e] - first;
       const bool row_ok = r < rows_valid;
@@ -657,7 +665,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
             const float a1 = __fdividef(g1, 1.0f + __expf(-g1)) * u1;
             packed[i] = pack_bf16x2(a0, a1);
           }
-          store_block(packed, wbuf, lane, q, row_ok, rows_valid, row_base, col0, p, out);
+          store_block(packed, wbuf, lane, q, row_ok, rows_valid, row_base, col0, p, out, out_rows);
         }
       } else {
 #pragma unroll 1
@@ -670,7 +678,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             packed[i] = pack_bf16x2(__uint_as_float(acc[2 * i]), __uint_as_float(acc[2 * i + 1]));
-          store_block(packed, wbuf, lane, q, row_ok, rows_valid, row_base, col0, p, out);
+          store_block(packed, wbuf, lane, q, row_ok, rows_valid, row_base, col0, p, out, out_rows);
         }
       }
       tc_fence_before();
@@ -844,6 +852,9 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
   p.gather = a.gather;
   p.gsrc = static_cast<const uint8_t*>(a.gather_src);
   p.gsrc_stride = (int64_t)a.K * 2;
+  p.gsrc_rows = a.gather_src_rows;
+  p.out_rows0 = a.rows;
+  p.out_rows1 = a.rows1;
   p.K = a.K;
   p.bsrc = static_cast<const uint8_t*>(a.B);
   p.reverse = a.reverse ? 1 : 0;
@@ -894,6 +905,14 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
                                                                                      p);
   }
   return cudaGetLastError();
+}
+
+uint32_t checks_take_gemm() {
+  uint32_t v = 0, zero = 0;
+  if (!MOE_CHECKS) return 0;
+  cudaMemcpyFromSymbol(&v, g_range_flags, sizeof v);
+  cudaMemcpyToSymbol(g_range_flags, &zero, sizeof zero);
+  return v;
 }
 
 }  // namespace moe

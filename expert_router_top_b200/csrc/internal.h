@@ -37,10 +37,16 @@ cudaError_t launch_metadata(const MetaArgs& a, cudaStream_t s);
 
 // ---- permute / unpermute (permute.cu) ----------------------------------------------------
 
+// rows_cap: rows of X (permute) or Y (unpermute); the checks build verifies every dst row
+// against it.
 cudaError_t launch_permute(const void* hidden, const int32_t* dst, int64_t Tc, int32_t H,
-                           int32_t k, void* X, cudaStream_t s);
+                           int32_t k, void* X, int64_t rows_cap, cudaStream_t s);
 cudaError_t launch_unpermute(const void* Y, const int32_t* dst, const float* w, int64_t Tc,
-                             int32_t H, int32_t k, void* out, cudaStream_t s);
+                             int32_t H, int32_t k, void* out, int64_t rows_cap, cudaStream_t s);
+// Range-violation flags of the checks build, one word per translation unit: read and clear.
+uint32_t checks_take_permute();
+uint32_t checks_take_gemm();
+uint32_t checks_take_backward();
 
 // ---- grouped GEMM (gemm.cu) -------------------------------------------------------------
 
@@ -144,10 +150,12 @@ cudaError_t launch_bwd_gemm(const BwdGemmArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_pad_offsets(const int32_t* counts, int32_t E, int32_t n_chunks, int32_t* offp,
                                int32_t* first, cudaStream_t s);
 cudaError_t launch_pad_rows(const int32_t* idx, const int32_t* dst, const int32_t* off,
-                            const int32_t* offp, int64_t n, int32_t* dstp, cudaStream_t s);
+                            const int32_t* offp, int64_t n, int32_t* dstp, int64_t rows_cap,
+                            cudaStream_t s);
 cudaError_t launch_dy_dw(const void* dout, const void* Y, const int32_t* dstp, const float* w,
-                         int64_t Tc, int32_t H, int32_t k, void* dY, float* dw, cudaStream_t s);
+                         int64_t Tc, int32_t H, int32_t k, void* dY, float* dw, int64_t rows_cap,
+                         cudaStream_t s);
 cudaError_t launch_sum_rows(const void* dX, const int32_t* dstp, int64_t Tc, int32_t H, int32_t k,
-                            void* out, cudaStream_t s);
+                            void* out, int64_t rows_cap, cudaStream_t s);
 
 }  // namespace moe

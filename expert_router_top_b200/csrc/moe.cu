@@ -632,8 +632,8 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
 
   auto permute = [&](int c) -> moe_status_t {
     ProfScope ps(MOE_KERNEL_PERMUTE, sm, len(c) * k, 0, 1);
-    if (launch_permute(hid + bounds[c] * H, dst + bounds[c] * k, len(c), H, k, xy(c), sm) !=
-        cudaSuccess)
+    if (launch_permute(hid + bounds[c] * H, dst + bounds[c] * k, len(c), H, k, xy(c), L.rows_cap,
+                       sm) != cudaSuccess)
       return MOE_ERR_CUDA;
     if (cudaEventRecord(ctx->ev_perm[c & 1], sm) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
@@ -664,7 +664,7 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
     if (cudaStreamWaitEvent(sm, ctx->ev_gemm[c & 1], 0) != cudaSuccess) return MOE_ERR_CUDA;
     ProfScope ps(MOE_KERNEL_UNPERMUTE, sm, len(c) * k, 0, 1);
     if (launch_unpermute(xy(c), dst + bounds[c] * k, top_k_weights + bounds[c] * k, len(c), H, k,
-                         outp + bounds[c] * H, sm) != cudaSuccess)
+                         outp + bounds[c] * H, L.rows_cap, sm) != cudaSuccess)
       return MOE_ERR_CUDA;
     if (fused && cudaEventRecord(ctx->ev_unperm[c & 1], sm) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
@@ -721,7 +721,7 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
       for (int c = c0; c <= (two ? c1 : c0); ++c) {
         ProfScope ps(MOE_KERNEL_UNPERMUTE, sm, len(c) * k, 0, 1);
         if (launch_unpermute(xy(c), dst + bounds[c] * k, top_k_weights + bounds[c] * k, len(c),
-                             H, k, outp + bounds[c] * H, sm) != cudaSuccess)
+                             H, k, outp + bounds[c] * H, L.rows_cap, sm) != cudaSuccess)
           return MOE_ERR_CUDA;
       }
       if (cudaEventRecord(ctx->ev_unperm[0], sm) != cudaSuccess) return MOE_ERR_CUDA;
@@ -836,8 +836,8 @@ moe_status_t moe_forward_host_impl(const moe_shape_t* shape, const void* hidden_
     if (cudaStreamWaitEvent(sm, ctx->ev_in[c & 1], 0) != cudaSuccess) return MOE_ERR_CUDA;
     {
       ProfScope ps(MOE_KERNEL_PERMUTE, sm, len(c) * k, 0, 1);
-      if (launch_permute(ws + hs.in[c & 1], dst + bounds[c] * k, len(c), H, k, xy(c), sm) !=
-          cudaSuccess)
+      if (launch_permute(ws + hs.in[c & 1], dst + bounds[c] * k, len(c), H, k, xy(c), L.rows_cap,
+                         sm) != cudaSuccess)
         return MOE_ERR_CUDA;
     }
     if (cudaEventRecord(ctx->ev_perm[c & 1], sm) != cudaSuccess ||
@@ -866,7 +866,7 @@ moe_status_t moe_forward_host_impl(const moe_shape_t* shape, const void* hidden_
     {
       ProfScope ps(MOE_KERNEL_UNPERMUTE, sm, len(c) * k, 0, 1);
       if (launch_unpermute(xy(c), dst + bounds[c] * k, w_dev + bounds[c] * k, len(c), H, k,
-                           ws + hs.out[c & 1], sm) != cudaSuccess)
+                           ws + hs.out[c & 1], L.rows_cap, sm) != cudaSuccess)
         return MOE_ERR_CUDA;
     }
     // copy-out of chunk c beside the next chunk's GEMMs
@@ -1061,8 +1061,9 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
     ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(c) * k, 0, 2);
     if (!ok(cudaMemsetAsync(x_of(c), 0, 2 * (size_t)R[c] * H, s)) ||
         !ok(launch_pad_rows(top_k_index + bounds[c] * k, dst + bounds[c] * k, off_c(c), offp_c(c),
-                            len(c) * k, dstp_c(c), s)) ||
-        !ok(launch_permute(hid + bounds[c] * H, dstp_c(c), len(c), H, k, x_of(c), s)) ||
+                            len(c) * k, dstp_c(c), B.rows_cap, s)) ||
+        !ok(launch_permute(hid + bounds[c] * H, dstp_c(c), len(c), H, k, x_of(c), B.rows_cap,
+                           s)) ||
         !ok(cudaEventRecord(ctx->ev_bp[c % 4], s)))
       return MOE_ERR_CUDA;
     return MOE_OK;
@@ -1135,7 +1136,7 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
     if (!ok(cudaMemsetAsync(buf(B.dy, c), 0, 2 * (size_t)R[c] * H, s)) ||
         !ok(launch_dy_dw(dout + bounds[c] * H, buf(B.ydx, c), dstp_c(c),
                          top_k_weights + bounds[c] * k, len(c), H, k, buf(B.dy, c),
-                         d_weights + bounds[c] * k, s)) ||
+                         d_weights + bounds[c] * k, B.rows_cap, s)) ||
         !ok(cudaEventRecord(ctx->ev_bdy[0], s)))
       return MOE_ERR_CUDA;
     return MOE_OK;
@@ -1200,7 +1201,8 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
   auto S = [&](int c) -> moe_status_t {
     if (!ok(cudaStreamWaitEvent(s, ctx->ev_bdx[0], 0))) return MOE_ERR_CUDA;
     ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(c) * k, 0, 1);
-    if (!ok(launch_sum_rows(buf(B.ydx, c), dstp_c(c), len(c), H, k, dx_out + bounds[c] * H, s)) ||
+    if (!ok(launch_sum_rows(buf(B.ydx, c), dstp_c(c), len(c), H, k, dx_out + bounds[c] * H,
+                            B.rows_cap, s)) ||
         !ok(cudaEventRecord(ctx->ev_bsum[c % 2], s)))
       return MOE_ERR_CUDA;
     return MOE_OK;
@@ -1237,6 +1239,15 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
   return MOE_OK;
 }
 
+int32_t moe_checks_enabled(void) { return MOE_CHECKS ? 1 : 0; }
+
+moe_status_t moe_checks_read(uint32_t* flags) {
+  if (!flags) return MOE_ERR_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  *flags = checks_take_permute() | checks_take_gemm() | checks_take_backward();
+  return MOE_OK;
+}
+
 moe_status_t moe_check_device_status(const void* workspace, size_t ws_bytes, void* stream) {
   if (!workspace || ws_bytes < sizeof(uint32_t)) return MOE_ERR_ARG;
   uint32_t st = 0;
@@ -1257,7 +1268,7 @@ moe_status_t moe_permute(const void* hidden, const int32_t* dst_rows, int64_t Tc
   if (!aligned(hidden, 16) || !aligned(X, 16) || !aligned(dst_rows, 4)) return MOE_ERR_ALIGN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   ProfScope ps(MOE_KERNEL_PERMUTE, s, Tc * k, 0, 1);
-  return cuda_status(launch_permute(hidden, dst_rows, Tc, H, k, X, s));
+  return cuda_status(launch_permute(hidden, dst_rows, Tc, H, k, X, Tc * k, s));
 }
 
 moe_status_t moe_unpermute(const void* Y, const int32_t* dst_rows, const float* top_k_weights,
@@ -1269,7 +1280,7 @@ moe_status_t moe_unpermute(const void* Y, const int32_t* dst_rows, const float* 
     return MOE_ERR_ALIGN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   ProfScope ps(MOE_KERNEL_UNPERMUTE, s, Tc * k, 0, 1);
-  return cuda_status(launch_unpermute(Y, dst_rows, top_k_weights, Tc, H, k, out, s));
+  return cuda_status(launch_unpermute(Y, dst_rows, top_k_weights, Tc, H, k, out, Tc * k, s));
 }
 
 static moe_status_t grouped_common(const void* A, int64_t rows, int32_t H, int32_t I, int32_t E,

@@ -27,12 +27,15 @@ __device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
   return v;
 }
 
+__device__ uint32_t g_range_flags;  // checks build: a row index outside its buffer was seen
+
 // X[dst[t*k+j]] = hidden[t] for every j < k.
 template <int U>
 __global__ void __launch_bounds__(kRowThreads) permute_kernel(const uint4* __restrict__ hidden,
                                                               const int32_t* __restrict__ dst,
                                                               int64_t Tc, int32_t H8, int32_t k,
-                                                              uint4* __restrict__ X) {
+                                                              uint4* __restrict__ X,
+                                                              int64_t rows_cap) {
   const int64_t t = (int64_t)blockIdx.x * kTokPerCta + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= Tc) return;
@@ -47,6 +50,7 @@ __global__ void __launch_bounds__(kRowThreads) permute_kernel(const uint4* __res
     }
     for (int j = 0; j < k; ++j) {
       const int32_t d = __shfl_sync(0xffffffffu, d_lane, j);
+      if (!check_row(d, rows_cap, &g_range_flags)) continue;
       uint4* row = X + (int64_t)d * H8;
 #pragma unroll
       for (int u = 0; u < U; ++u) {
@@ -63,7 +67,8 @@ __global__ void __launch_bounds__(kRowThreads) unpermute_kernel(const uint4* __r
                                                                 const int32_t* __restrict__ dst,
                                                                 const float* __restrict__ w,
                                                                 int64_t Tc, int32_t H8, int32_t k,
-                                                                uint4* __restrict__ out) {
+                                                                uint4* __restrict__ out,
+                                                                int64_t rows_cap) {
   const int64_t t = (int64_t)blockIdx.x * kTokPerCta + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= Tc) return;
@@ -78,6 +83,7 @@ __global__ void __launch_bounds__(kRowThreads) unpermute_kernel(const uint4* __r
     for (int j = 0; j < k; ++j) {
       const int32_t d = __shfl_sync(0xffffffffu, d_lane, j);
       const float wj = __shfl_sync(0xffffffffu, w_lane, j);
+      if (!check_row(d, rows_cap, &g_range_flags)) continue;
       const uint4* row = Y + (int64_t)d * H8;
       uint4 y[U];
 #pragma unroll
@@ -115,19 +121,27 @@ inline unsigned grid_for(int64_t Tc) { return (unsigned)((Tc + kTokPerCta - 1) /
 }  // namespace
 
 cudaError_t launch_permute(const void* hidden, const int32_t* dst, int64_t Tc, int32_t H,
-                           int32_t k, void* X, cudaStream_t s) {
+                           int32_t k, void* X, int64_t rows_cap, cudaStream_t s) {
   if (Tc <= 0) return cudaSuccess;
   permute_kernel<4><<<grid_for(Tc), kRowThreads, 0, s>>>(
-      static_cast<const uint4*>(hidden), dst, Tc, H / 8, k, static_cast<uint4*>(X));
+      static_cast<const uint4*>(hidden), dst, Tc, H / 8, k, static_cast<uint4*>(X), rows_cap);
   return cudaGetLastError();
 }
 
 cudaError_t launch_unpermute(const void* Y, const int32_t* dst, const float* w, int64_t Tc,
-                             int32_t H, int32_t k, void* out, cudaStream_t s) {
+                             int32_t H, int32_t k, void* out, int64_t rows_cap, cudaStream_t s) {
   if (Tc <= 0) return cudaSuccess;
   unpermute_kernel<2><<<grid_for(Tc), kRowThreads, 0, s>>>(
-      static_cast<const uint4*>(Y), dst, w, Tc, H / 8, k, static_cast<uint4*>(out));
+      static_cast<const uint4*>(Y), dst, w, Tc, H / 8, k, static_cast<uint4*>(out), rows_cap);
   return cudaGetLastError();
+}
+
+uint32_t checks_take_permute() {
+  uint32_t v = 0, zero = 0;
+  if (!MOE_CHECKS) return 0;
+  cudaMemcpyFromSymbol(&v, g_range_flags, sizeof v);
+  cudaMemcpyToSymbol(g_range_flags, &zero, sizeof zero);
+  return v;
 }
 
 }  // namespace moe

@@ -348,6 +348,17 @@ MOE_API moe_status_t moe_grouped_down(const void* Act, int64_t rows, int32_t H, 
 MOE_API moe_status_t moe_unpermute(const void* Y, const int32_t* dst_rows, const float* top_k_weights,
                            int64_t Tc, int32_t H, int32_t k, void* out, void* stream);
 
+/* ---- Range-checked build ----------------------------------------------------------------
+ * libmoe_checks.so is this library compiled with every data-dependent row index (permuted
+ * and padded rows, gathered token rows, output rows) compared with the rows of the buffer
+ * it addresses before the access; a violation skips the access and raises a flag instead
+ * of faulting (it stands in for a memory sanitizer).  moe_checks_enabled: 1 in that build,
+ * 0 in libmoe.so.  moe_checks_read synchronizes the device, stores the OR of all flags
+ * raised since the last read into *flags (0: every index was in range; always 0 in
+ * libmoe.so) and clears them. */
+MOE_API int32_t moe_checks_enabled(void);
+MOE_API moe_status_t moe_checks_read(uint32_t* flags);
+
 /* ---- Failure-detection self-test -------------------------------------------------------
  * Not part of the Chunk MoE method (the article has no counterpart): it exercises the
  * library's own failure detection.  Launches one kernel whose bounded mbarrier wait has

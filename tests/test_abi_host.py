@@ -253,3 +253,9 @@ def test_selftest_argument_checks_run_on_host():
     assert L.moe_selftest_wait_timeout(v(FAKE), 0, None) == 1          # limit 0
     assert L.moe_selftest_wait_timeout(v(FAKE), 2000000, None) == 1    # limit above 1 s
     assert L.moe_selftest_wait_timeout(v(FAKE + 2), 1000, None) == 3   # misaligned
+
+
+def test_checks_api_in_the_regular_build():
+    L = moe.load()
+    assert L.moe_checks_enabled() == 0
+    assert L.moe_checks_read(None) == 1  # null flags
