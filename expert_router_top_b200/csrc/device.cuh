@@ -130,39 +130,6 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* t
       : "memory");
 }
 
-// Gather of 4 rows (r0..r3, any order) of a 2-D tensor whose map has a box one row high:
-// 4 x box-width elements land in consecutive smem rows, swizzled by smem address.
-__device__ __forceinline__ void tma_gather4(void* smem_dst, const CUtensorMap* tm, uint64_t* bar,
-                                            int32_t c0, int32_t r0, int32_t r1, int32_t r2,
-                                            int32_t r3, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes."
-      "L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(tm)), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1), "r"(r2),
-      "r"(r3), "l"(policy)
-      : "memory");
-}
-
-// 4-D tiled load of one box into shared memory (c0 innermost; c0 * 2 bytes a multiple of 16).
-__device__ __forceinline__ void tma_load_4d(void* smem_dst, const CUtensorMap* tm, uint64_t* bar,
-                                            int32_t c0, int32_t c1, int32_t c2, int32_t c3,
-                                            uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::"
-      "cache_hint [%0], [%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(tm)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
-      "l"(policy)
-      : "memory");
-}
-
-// Prefetch one box of a 2-D tiled tensor into L2 (no shared memory, no completion).
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* tm, int32_t c0, int32_t c1) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
-                   reinterpret_cast<uint64_t>(tm)),
-               "r"(c0), "r"(c1)
-               : "memory");
-}
-
 // 3-D tiled store, or fp32 add-reduction, of one shared-memory box into global memory,
 // completed through the issuing thread's bulk group.  c0 * element size is a multiple of
 // 16 bytes and no coordinate is negative; parts of the box outside the tensor are skipped.
@@ -219,12 +186,6 @@ __device__ __forceinline__ void cp_async_wait() {
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy (TMA).
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// Prefetch the 128-byte line holding `p` into L2 (LSU path, no completion), kept with the
-// evict_last priority.
-__device__ __forceinline__ void prefetch_l2_last(const void* p) {
-  asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p));
 }
 
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {

@@ -57,27 +57,6 @@
 #ifndef MOE_GEMM_BAND
 #define MOE_GEMM_BAND 16  // M tiles per raster band: an expert's A rows stay in L2 across N tiles
 #endif
-#ifndef MOE_GEMM_WPREFETCH
-// > 0: one more warp walks the weight (B) rows of the tile stream up to this many K blocks
-// ahead of the TMA producer, prefetching each 128-byte block row into L2 (LSU prefetches,
-// so the TMA unit and shared memory are not involved)
-#define MOE_GEMM_WPREFETCH 0
-#endif
-#ifndef MOE_GEMM_PACKED_B
-// 1: B is read from a tile-packed weight layout in which the 256 B rows of one tile and one
-// K block (gate rows then up rows for gate/up) are one contiguous 32 KB block, fetched with
-// one box per stage
-#define MOE_GEMM_PACKED_B 0
-#endif
-#ifndef MOE_GEMM_B4D
-#define MOE_GEMM_B4D 0  // gate/up: one 4-D box fetches the gate and the up rows of a tile
-#endif
-#ifndef MOE_GEMM_PREFETCH
-#define MOE_GEMM_PREFETCH 0  // K blocks of L2 prefetch ahead of the smem loads (0: none)
-#endif
-#ifndef MOE_GEMM_PREFETCH_A
-#define MOE_GEMM_PREFETCH_A 0  // 1: prefetch the A rows too, not only the weights
-#endif
 #ifndef MOE_GEMM_B_POLICY
 #define MOE_GEMM_B_POLICY 2  // L2 policy of weight loads: 0 normal, 1 evict_first, 2 evict_last
 #endif
@@ -121,7 +100,6 @@ struct KParams {
   const uint8_t* gsrc;    // gathered A: the token rows (hidden), and their stride in bytes
   int64_t gsrc_stride;
   int32_t K;              // valid K columns (gathered A: the rest of the last block reads 0)
-  const uint8_t* bsrc;    // B (weights) base, for the weight prefetch warp
   // A second row segment sharing the tile sweep (the other chunk of a pair): its expert
   // offsets [E+1] (nullptr: one segment), output rows, and gathered-A source rows.
   const int32_t* offsets1;
@@ -129,8 +107,6 @@ struct KParams {
   const int32_t* gather1;
   int64_t gsrc_rows;             // checks build: rows of the gathered source
   int64_t out_rows0, out_rows1;  // checks build: rows of out and out1
-  int32_t reverse;        // 1: walk the tiles (hence the experts) in descending order
-  int32_t b4d;            // 1: tmB is the 4-D gate/up view (one box per stage)
 };
 
 template <int kStages>
@@ -142,14 +118,12 @@ struct SmemCtl {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
-  uint32_t prod_iter;  // K blocks the TMA producer has issued (read by the prefetch warp)
 };
 
-// Threads of one CTA: producer, MMA, 4 epilogue warps; + 4 gathering warps (gathered A);
-// + 1 weight prefetch warp (MOE_GEMM_WPREFETCH).
+// Threads of one CTA: producer, MMA, 4 epilogue warps; + 4 gathering warps (gathered A).
 template <bool kGather>
 __host__ __device__ constexpr int gemm_threads() {
-  return kGemmThreads + (kGather ? kGatherThreads : 0) + (MOE_GEMM_WPREFETCH ? 32 : 0);
+  return kGemmThreads + (kGather ? kGatherThreads : 0);
 }
 
 constexpr size_t kCtlBytes = 256;
@@ -296,7 +270,6 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
     }
     mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
-    ctl->prod_iter = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -355,7 +328,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       uint32_t armed = 0, armed_parity = 0;
       bool ok = true;
       for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
-        const Tile t = decode_tile<G::kTileM>(p.reverse ? p.total_tiles - 1 - L : L, tile_start,
+        const Tile t = decode_tile<G::kTileM>(L, tile_start,
                                               off, off1p, E, p.n_tiles);
         const int32_t brow = t.e * p.b_rows + t.n * (kSwiGLU ? BN / 2 : BN);
         for (int32_t kb = 0; kb < p.num_kb; ++kb) {
@@ -369,7 +342,6 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
           if (kSwiGLU)
             tma_load_2d(b_dst + G::kBBytes / 2, tmB, &ctl->full[stage], kb * BK, brow + p.up_off,
                         pol_w);
-          if (MOE_GEMM_WPREFETCH) *reinterpret_cast<volatile uint32_t*>(&ctl->prod_iter) += 1;
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -381,46 +353,6 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       if (!ok)
         for (int s = 0; s < STAGES; ++s)
           if (armed & (1u << s)) mbar_drain(&ctl->full[s], (armed_parity >> s) & 1u, 100000000ull);
-    }
-  } else if (MOE_GEMM_WPREFETCH && !kPair && warp == gemm_threads<kGather>() / 32 - 1) {
-    // ---------------- weight prefetch warp ----------------
-    // Walks the same tile stream as the producer; K block i of the stream (all B rows of the
-    // tile, one 128-byte segment each) is prefetched into L2 once the producer has issued
-    // block i - MOE_GEMM_WPREFETCH.  The wait on the producer's counter is bounded.
-    const volatile uint32_t* prog = &ctl->prod_iter;
-    const int64_t row_bytes = (int64_t)p.K * 2;
-    uint32_t i = 0;
-    bool ok = true;
-    for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
-      const Tile t = decode_tile<G::kTileM>(p.reverse ? p.total_tiles - 1 - L : L, tile_start,
-                                            off, off1p, E, p.n_tiles);
-      const int32_t half = kSwiGLU ? BN / 2 : BN;  // rows per B half (gate, up) or all rows
-      const int32_t nrows = min(half, p.out_cols - t.n * half);
-      const int64_t r0 = (int64_t)t.e * p.b_rows + t.n * half;
-      for (int32_t kb = 0; kb < p.num_kb; ++kb, ++i) {
-        if (*prog + MOE_GEMM_WPREFETCH <= i) {
-          const uint64_t t0 = global_timer_ns();
-          while (*prog + MOE_GEMM_WPREFETCH <= i) {
-            if (*abort) {
-              ok = false;
-              break;
-            }
-            if (global_timer_ns() - t0 > kWaitLimitNs) {
-              *abort = 1;
-              atomicOr(p.status, MOE_DEV_TIMEOUT);
-              ok = false;
-              break;
-            }
-            __nanosleep(128);
-          }
-          if (!ok) break;
-        }
-        const uint8_t* base = p.bsrc + r0 * row_bytes + kb * (BK * 2);
-        for (int32_t r = lane; r < nrows; r += 32) {
-          prefetch_l2_last(base + r * row_bytes);
-          if (kSwiGLU) prefetch_l2_last(base + ((int64_t)p.up_off + r) * row_bytes);
-        }
-      }
     }
   } else if (kGather && warp >= kGemmThreads / 32) {
     // ---------------- A producers, gathered rows (4 warps, LSU) ----------------
@@ -437,7 +369,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
     int32_t issued = 0, arrived = 0;
     bool ok = true;
     for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
-      const Tile t = decode_tile<G::kTileM>(p.reverse ? p.total_tiles - 1 - L : L, tile_start,
+      const Tile t = decode_tile<G::kTileM>(L, tile_start,
                                             off, off1p, E, p.n_tiles);
       const int32_t* offs = t.seg ? off1 : off;
       const int32_t* gat = t.seg ? p.gather1 : p.gather;
@@ -493,42 +425,17 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;  // per-stage bits, for the abort drain
       bool ok = true;
-      // A row and B row of the tile at linear index L (of this CTA's tile stream)
-      int32_t t_e = 0, t_n = 0, t_seg = 0;
-      auto coords = [&](int32_t L, int32_t& row0, int32_t& brow) {
-        const Tile t = decode_tile<G::kTileM>(p.reverse ? p.total_tiles - 1 - L : L, tile_start,
-                                              off, off1p, E, p.n_tiles);
-        t_e = t.e;
-        t_n = t.n;
-        t_seg = t.seg;
-        row0 = (t.seg ? off1 : off)[t.e] + t.ml * G::kTileM + (int32_t)rank * kRowsPerCta;
-        if (kSwiGLU)  // pair: the even CTA stages the gate rows, the odd one the up rows
-          brow = t.e * p.b_rows + t.n * (BN / 2) + (kPair ? (int32_t)rank * p.up_off : 0);
-        else
-          brow = t.e * p.b_rows + t.n * BN + (kPair ? (int32_t)rank * (BN / 2) : 0);
-      };
-      // L2 prefetch of K block kb of the tile at (row0, brow): the weight box(es), and the
-      // A box when asked; nothing lands in shared memory and nothing is waited for
-      auto prefetch = [&](int32_t row0, int32_t brow, int32_t kb) {
-        if (!p.b4d) {  // (the 4-D gate/up view is not prefetched)
-          tma_prefetch_2d(tmB, kb * BK, brow);
-          if (kSwiGLU && !kPair) tma_prefetch_2d(tmB, kb * BK, brow + p.up_off);
-        }
-        if (MOE_GEMM_PREFETCH_A) tma_prefetch_2d(tmA, kb * BK, row0);
-      };
-      int32_t nrow0 = 0, nbrow = 0;
       for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
-        int32_t row0, brow;
-        const bool has_next = L + n_streams < p.total_tiles;
-        if (MOE_GEMM_PREFETCH > 0 && has_next) coords(L + n_streams, nrow0, nbrow);
-        coords(L, row0, brow);  // last, so that t_e / t_n / t_seg describe this tile
-        const CUtensorMap* mapA = t_seg ? tmA1 : tmA;
+        // A row and B row of tile L (of this CTA's tile stream)
+        const Tile t = decode_tile<G::kTileM>(L, tile_start, off, off1p, E, p.n_tiles);
+        const int32_t row0 =
+            (t.seg ? off1 : off)[t.e] + t.ml * G::kTileM + (int32_t)rank * kRowsPerCta;
+        const int32_t brow =
+            kSwiGLU  // pair: the even CTA stages the gate rows, the odd one the up rows
+                ? t.e * p.b_rows + t.n * (BN / 2) + (kPair ? (int32_t)rank * p.up_off : 0)
+                : t.e * p.b_rows + t.n * BN + (kPair ? (int32_t)rank * (BN / 2) : 0);
+        const CUtensorMap* mapA = t.seg ? tmA1 : tmA;
         for (int32_t kb = 0; kb < p.num_kb; ++kb) {
-          if (MOE_GEMM_PREFETCH > 0) {
-            const int32_t pk = kb + MOE_GEMM_PREFETCH;
-            if (pk < p.num_kb) prefetch(row0, brow, pk);
-            else if (has_next && pk - p.num_kb < p.num_kb) prefetch(nrow0, nbrow, pk - p.num_kb);
-          }
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort, p.status)) {
             ok = false;
             break;
@@ -543,13 +450,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
           } else {
             mbar_arrive_expect_tx(&ctl->full[stage], G::kTxBytes);
             tma_load_2d(a_dst, mapA, &ctl->full[stage], kb * BK, row0, pol_a);
-            if (MOE_GEMM_PACKED_B) {
-              const int32_t prow = ((t_e * p.n_tiles + t_n) * p.num_kb + kb) * BN;
-              tma_load_2d(b_dst, tmB, &ctl->full[stage], 0, prow, pol_w);
-            } else if (kSwiGLU && p.b4d) {
-              // {K, row in block, 128-row block n, 2e + gate/up}: gate block n, then up block n
-              tma_load_4d(b_dst, tmB, &ctl->full[stage], kb * BK, 0, t_n, 2 * t_e, pol_w);
-            } else if (kSwiGLU) {
+            if (kSwiGLU) {
               tma_load_2d(b_dst, tmB, &ctl->full[stage], kb * BK, brow, pol_w);
               tma_load_2d(b_dst + G::kBBytes / 2, tmB, &ctl->full[stage], kb * BK,
                           brow + p.up_off, pol_w);
@@ -557,7 +458,6 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
               tma_load_2d(b_dst, tmB, &ctl->full[stage], kb * BK, brow, pol_w);
             }
           }
-          if (MOE_GEMM_WPREFETCH) *reinterpret_cast<volatile uint32_t*>(&ctl->prod_iter) += 1;
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -636,7 +536,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       const uint32_t tphase = (it >> 1) & 1;
       if (!mbar_wait(&ctl->tfull[buf], tphase, abort, p.status)) break;
       tc_fence_after();
-      const Tile t = decode_tile<G::kTileM>(p.reverse ? p.total_tiles - 1 - L : L, tile_start,
+      const Tile t = decode_tile<G::kTileM>(L, tile_start,
                                             off, off1p, E, p.n_tiles);
       const int32_t* offs = t.seg ? off1 : off;
       __nv_bfloat16* out = t.seg ? p.out1 : p.out;
@@ -751,26 +651,6 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int32_t cols, int3
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 4-D view of W_gate_up [E][2I][K] for one-box gate/up loads: dims {K, 128, I/128, 2E}
-// with strides {2K, 128*2K, I*2K} bytes; box {BK, 128, 1, 2} = the gate rows and the up rows
-// of one 128-column output block of one expert, in that order.
-bool make_map_gateup4d(CUtensorMap* m, const void* base, int32_t E, int32_t I, int32_t K) {
-  EncodeTiledFn enc = get_encode_fn();
-  if (!enc || I % 128 != 0) return false;
-  const cuuint64_t dims[4] = {(cuuint64_t)K, 128, (cuuint64_t)(I / 128), (cuuint64_t)(2 * E)};
-  const cuuint64_t strides[3] = {(cuuint64_t)K * 2, (cuuint64_t)128 * K * 2,
-                                 (cuuint64_t)I * K * 2};
-  const cuuint32_t box[4] = {(cuuint32_t)BK, 128, 1, 2};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             BK == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
-             MOE_GEMM_L2_PROMO == 2   ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B
-             : MOE_GEMM_L2_PROMO == 1 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
-                                      : CU_TENSOR_MAP_L2_PROMOTION_NONE,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 bool make_tma_2d_bf16(CUtensorMap* m, const void* base, int64_t rows, int32_t cols,
@@ -822,16 +702,8 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
   // (gathered A is copied by the gathering warps; its map is built but unused)
   const bool map_a_ok = gather ? make_map(&mA, a.gather_src, a.gather_src_rows, a.K, kRowsPerCta)
                                : make_map(&mA, a.A, a.rows, a.K, kRowsPerCta);
-  // one-box gate/up weights (single-CTA, plain A, I a multiple of 128)
-  const bool b4d = MOE_GEMM_B4D && swiglu && !kPair && !gather && a.out_cols % 128 == 0 &&
-                   make_map_gateup4d(&mB, a.B, a.E, a.out_cols, a.K);
-  const int64_t packed_rows =
-      (int64_t)a.E * ((a.out_cols + bn - 1) / bn) * ((a.K + BK - 1) / BK) * BN;
-  const bool map_b_ok =
-      b4d || (MOE_GEMM_PACKED_B && !kPair && !gather
-                  ? make_map(&mB, a.B, packed_rows, BK, BN)
-                  : make_map(&mB, a.B, (int64_t)a.E * a.b_rows, a.K,
-                             kPair ? BN / 2 : (swiglu ? BN / 2 : BN)));
+  const bool map_b_ok = make_map(&mB, a.B, (int64_t)a.E * a.b_rows, a.K,
+                                 kPair ? BN / 2 : (swiglu ? BN / 2 : BN));
   const bool map_a1_ok =
       two && !gather ? make_map(&mA1, a.A1, a.rows1, a.K, kRowsPerCta) : (mA1 = mA, true);
   if (!map_a_ok || !map_b_ok || !map_a1_ok) {
@@ -856,9 +728,6 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
   p.out_rows0 = a.rows;
   p.out_rows1 = a.rows1;
   p.K = a.K;
-  p.bsrc = static_cast<const uint8_t*>(a.B);
-  p.reverse = a.reverse ? 1 : 0;
-  p.b4d = b4d ? 1 : 0;
   p.offsets1 = two ? a.offsets1 : nullptr;
   p.out1 = two ? static_cast<__nv_bfloat16*>(a.out1) : nullptr;
   p.gather1 = two ? a.gather1 : nullptr;

@@ -72,7 +72,6 @@ struct GemmArgs {
   const int32_t* gather = nullptr;
   const void* gather_src = nullptr;
   int64_t gather_src_rows = 0;
-  bool reverse = false;  // walk the tiles (and so the experts) in descending order
   // A second row segment in the same tile sweep (the other chunk of a pair: the weights of
   // each expert tile are then fetched once for both): its expert offsets (dev [E+1]; nullptr
   // = one segment), A rows (A1 [rows1][K], or gathered through gather1), and output rows.

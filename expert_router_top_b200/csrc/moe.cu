@@ -382,9 +382,6 @@ int64_t active_experts(const int32_t* counts, int32_t E) {
   return a;
 }
 
-#ifndef MOE_ALTERNATE_ORDER
-#define MOE_ALTERNATE_ORDER 0  // 1: odd chunks walk the experts in descending order
-#endif
 
 // The second row segment of a grouped GEMM that serves both chunks of a pair.
 struct Seg1 {
@@ -401,8 +398,7 @@ moe_status_t gemm_call(const void* A, int64_t rows, const void* B, void* out,
                        int32_t K, int32_t out_cols, int32_t b_rows, bool swiglu,
                        uint32_t* status, int num_sms, cudaStream_t s,
                        const int32_t* gather = nullptr, const void* gather_src = nullptr,
-                       int64_t gather_src_rows = 0, bool reverse = false,
-                       const Seg1* seg1 = nullptr) {
+                       int64_t gather_src_rows = 0, const Seg1* seg1 = nullptr) {
   GemmArgs g;
   int64_t rows_all = rows, active = active_experts(counts_host, E);
   if (seg1) {
@@ -415,7 +411,6 @@ moe_status_t gemm_call(const void* A, int64_t rows, const void* B, void* out,
     active = 0;  // experts with rows in either segment
     for (int32_t e = 0; e < E; ++e) active += (counts_host[e] + seg1->counts[e]) > 0;
   }
-  g.reverse = reverse;
   g.gather = gather;
   g.gather_src = gather_src;
   g.gather_src_rows = gather_src_rows;
@@ -628,7 +623,6 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
   auto xy = [&](int c) { return ws + L.xy[c % L.nbuf]; };
   auto act = [&](int c) { return ws + L.act[c % L.nbuf]; };
   auto len = [&](int c) { return bounds[c + 1] - bounds[c]; };
-  auto rev = [&](int c) { return MOE_ALTERNATE_ORDER && (c & 1); };
 
   auto permute = [&](int c) -> moe_status_t {
     ProfScope ps(MOE_KERNEL_PERMUTE, sm, len(c) * k, 0, 1);
@@ -650,12 +644,12 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
     const int32_t* offs = reinterpret_cast<const int32_t*>(ws + L.offsets) + (size_t)c * (E + 1);
     moe_status_t s2 =
         fused ? gemm_call(nullptr, rows, W_gate_up, act(c), offs, cnt, E, H, I, 2 * I, true,
-                          dev_status, ctx->num_sms, sg, src + bounds[c] * k, hidden, T, rev(c))
+                          dev_status, ctx->num_sms, sg, src + bounds[c] * k, hidden, T)
               : gemm_call(xy(c), rows, W_gate_up, act(c), offs, cnt, E, H, I, 2 * I, true,
-                          dev_status, ctx->num_sms, sg, nullptr, nullptr, 0, rev(c));
+                          dev_status, ctx->num_sms, sg);
     if (s2 != MOE_OK) return s2;
     s2 = gemm_call(act(c), rows, W_down, xy(c), offs, cnt, E, I, H, H, false, dev_status,
-                   ctx->num_sms, sg, nullptr, nullptr, 0, rev(c));
+                   ctx->num_sms, sg);
     if (s2 != MOE_OK) return s2;
     if (cudaEventRecord(ctx->ev_gemm[c & 1], sg) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
@@ -706,14 +700,13 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
       Seg1 s1 = two ? seg(c1, nullptr, act(c1)) : Seg1{};
       moe_status_t s2 = gemm_call(nullptr, s0.rows, W_gate_up, act(c0), s0.offsets, s0.counts,
                                   E, H, I, 2 * I, true, dev_status, ctx->num_sms, sg, s0.gather,
-                                  hidden, T, false, two ? &s1 : nullptr);
+                                  hidden, T, two ? &s1 : nullptr);
       if (s2 != MOE_OK) return s2;
       if (c0 >= 2 && cudaStreamWaitEvent(sg, ctx->ev_unperm[0], 0) != cudaSuccess)
         return MOE_ERR_CUDA;
       if (two) s1 = seg(c1, act(c1), xy(c1));
       s2 = gemm_call(act(c0), s0.rows, W_down, xy(c0), s0.offsets, s0.counts, E, I, H, H, false,
-                     dev_status, ctx->num_sms, sg, nullptr, nullptr, 0, false,
-                     two ? &s1 : nullptr);
+                     dev_status, ctx->num_sms, sg, nullptr, nullptr, 0, two ? &s1 : nullptr);
       if (s2 != MOE_OK) return s2;
       if (cudaEventRecord(ctx->ev_gemm[0], sg) != cudaSuccess ||
           cudaStreamWaitEvent(sm, ctx->ev_gemm[0], 0) != cudaSuccess)
@@ -850,12 +843,11 @@ moe_status_t moe_forward_host_impl(const moe_shape_t* shape, const void* hidden_
     const int64_t rows = len(c) * k;
     const int32_t* cnt = counts.data() + (size_t)c * E;
     const int32_t* offs = reinterpret_cast<const int32_t*>(ws + L.offsets) + (size_t)c * (E + 1);
-    const bool r = MOE_ALTERNATE_ORDER && (c & 1);
     moe_status_t s2 = gemm_call(xy(c), rows, W_gate_up, act(c), offs, cnt, E, H, I, 2 * I, true,
-                                dev_status, ctx->num_sms, sg, nullptr, nullptr, 0, r);
+                                dev_status, ctx->num_sms, sg);
     if (s2 != MOE_OK) return s2;
     s2 = gemm_call(act(c), rows, W_down, xy(c), offs, cnt, E, I, H, H, false, dev_status,
-                   ctx->num_sms, sg, nullptr, nullptr, 0, r);
+                   ctx->num_sms, sg);
     if (s2 != MOE_OK) return s2;
     return cudaEventRecord(ctx->ev_gemm[c & 1], sg) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   };
@@ -1124,8 +1116,7 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
     }
     moe_status_t s2 = gemm_call(buf(B.act, c), R[c], W_down, buf(B.ydx, c), offp_c(c),
                                 rows_pad.data() + (size_t)c * E, E, I, H, H, false, dev_status,
-                                ctx->num_sms, sg, nullptr, nullptr, 0, false,
-                                c1 > c ? &d1 : nullptr);
+                                ctx->num_sms, sg, nullptr, nullptr, 0, c1 > c ? &d1 : nullptr);
     if (s2 != MOE_OK) return s2;
     return ok(cudaEventRecord(ctx->ev_bf[0], sg)) ? MOE_OK : MOE_ERR_CUDA;
   };
