@@ -536,13 +536,12 @@ __global__ void pad_rows_kernel(const int32_t* idx, const int32_t* dst, const in
   dstp[s] = check_row(d, rows_cap, &g_range_flags) ? d : 0;
 }
 
-// dY[dstp(t,j)] = bf16(w[t][j] * dout[t]) and d_w[t][j] = <dout[t], Y[dstp(t,j)]> (fp32,
-// warp tree reduction in a fixed order): one warp per token.
+// dY[dstp(t,j)] = bf16(w[t][j] * dout[t]) for every j < k: a weighted permute of dout that
+// needs nothing from the recomputed forward.  One warp per token.
 __global__ void __launch_bounds__(kRowThreads)
-    dy_dw_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ Y,
-                 const int32_t* __restrict__ dstp, const float* __restrict__ w, int64_t Tc,
-                 int32_t H8, int32_t k, uint4* __restrict__ dY, float* __restrict__ dw,
-                 int64_t rows_cap) {
+    dy_scatter_kernel(const uint4* __restrict__ dout, const int32_t* __restrict__ dstp,
+                      const float* __restrict__ w, int64_t Tc, int32_t H8, int32_t k,
+                      uint4* __restrict__ dY, int64_t rows_cap) {
   const int64_t t = (int64_t)blockIdx.x * kTokPerCta + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= Tc) return;
@@ -550,20 +549,40 @@ __global__ void __launch_bounds__(kRowThreads)
     const int32_t d = dstp[t * k + j];
     if (!check_row(d, rows_cap, &g_range_flags)) continue;  // d is the same in every lane
     const float wj = w[t * k + j];
+    for (int32_t v = lane; v < H8; v += 32) {
+      const uint4 g = dout[t * H8 + v];
+      const uint32_t ga[4] = {g.x, g.y, g.z, g.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o[i] = pack_bf16x2(wj * bf16lo(ga[i]), wj * bf16hi(ga[i]));
+      dY[(int64_t)d * H8 + v] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
+// d_w[t][j] = <dout[t], Y[dstp(t,j)]> in fp32 (lane-strided partial sums, then a warp tree
+// reduction in a fixed order): one warp per token.
+__global__ void __launch_bounds__(kRowThreads)
+    dw_dot_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ Y,
+                  const int32_t* __restrict__ dstp, int64_t Tc, int32_t H8, int32_t k,
+                  float* __restrict__ dw, int64_t rows_cap) {
+  const int64_t t = (int64_t)blockIdx.x * kTokPerCta + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= Tc) return;
+  for (int j = 0; j < k; ++j) {
+    const int32_t d = dstp[t * k + j];
+    if (!check_row(d, rows_cap, &g_range_flags)) continue;
     float dot = 0.f;
     for (int32_t v = lane; v < H8; v += 32) {
       const uint4 g = dout[t * H8 + v];
       const uint4 y = Y[(int64_t)d * H8 + v];
       const uint32_t ga[4] = {g.x, g.y, g.z, g.w};
       const uint32_t ya[4] = {y.x, y.y, y.z, y.w};
-      uint32_t o[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         dot = fmaf(bf16lo(ga[i]), bf16lo(ya[i]), dot);
         dot = fmaf(bf16hi(ga[i]), bf16hi(ya[i]), dot);
-        o[i] = pack_bf16x2(wj * bf16lo(ga[i]), wj * bf16hi(ga[i]));
       }
-      dY[(int64_t)d * H8 + v] = make_uint4(o[0], o[1], o[2], o[3]);
     }
 #pragma unroll
     for (int sh = 16; sh > 0; sh >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, sh);
@@ -706,13 +725,21 @@ cudaError_t launch_pad_rows(const int32_t* idx, const int32_t* dst, const int32_
   return cudaGetLastError();
 }
 
-cudaError_t launch_dy_dw(const void* dout, const void* Y, const int32_t* dstp, const float* w,
-                         int64_t Tc, int32_t H, int32_t k, void* dY, float* dw, int64_t rows_cap,
-                         cudaStream_t s) {
+cudaError_t launch_dy_scatter(const void* dout, const int32_t* dstp, const float* w, int64_t Tc,
+                              int32_t H, int32_t k, void* dY, int64_t rows_cap, cudaStream_t s) {
   if (Tc <= 0) return cudaSuccess;
-  dy_dw_kernel<<<row_grid(Tc), kRowThreads, 0, s>>>(
-      static_cast<const uint4*>(dout), static_cast<const uint4*>(Y), dstp, w, Tc, H / 8, k,
-      static_cast<uint4*>(dY), dw, rows_cap);
+  dy_scatter_kernel<<<row_grid(Tc), kRowThreads, 0, s>>>(static_cast<const uint4*>(dout), dstp, w,
+                                                         Tc, H / 8, k, static_cast<uint4*>(dY),
+                                                         rows_cap);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dw_dot(const void* dout, const void* Y, const int32_t* dstp, int64_t Tc,
+                          int32_t H, int32_t k, float* dw, int64_t rows_cap, cudaStream_t s) {
+  if (Tc <= 0) return cudaSuccess;
+  dw_dot_kernel<<<row_grid(Tc), kRowThreads, 0, s>>>(static_cast<const uint4*>(dout),
+                                                     static_cast<const uint4*>(Y), dstp, Tc,
+                                                     H / 8, k, dw, rows_cap);
   return cudaGetLastError();
 }
 

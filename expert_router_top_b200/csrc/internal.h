@@ -151,9 +151,12 @@ cudaError_t launch_pad_offsets(const int32_t* counts, int32_t E, int32_t n_chunk
 cudaError_t launch_pad_rows(const int32_t* idx, const int32_t* dst, const int32_t* off,
                             const int32_t* offp, int64_t n, int32_t* dstp, int64_t rows_cap,
                             cudaStream_t s);
-cudaError_t launch_dy_dw(const void* dout, const void* Y, const int32_t* dstp, const float* w,
-                         int64_t Tc, int32_t H, int32_t k, void* dY, float* dw, int64_t rows_cap,
-                         cudaStream_t s);
+// dY[dstp(t,j)] = bf16(w[t][j] dout[t]) (needs nothing from the forward), and
+// d_w[t][j] = <dout[t], Y[dstp(t,j)]> (needs the recomputed Y).
+cudaError_t launch_dy_scatter(const void* dout, const int32_t* dstp, const float* w, int64_t Tc,
+                              int32_t H, int32_t k, void* dY, int64_t rows_cap, cudaStream_t s);
+cudaError_t launch_dw_dot(const void* dout, const void* Y, const int32_t* dstp, int64_t Tc,
+                          int32_t H, int32_t k, float* dw, int64_t rows_cap, cudaStream_t s);
 cudaError_t launch_sum_rows(const void* dX, const int32_t* dstp, int64_t Tc, int32_t H, int32_t k,
                             void* out, int64_t rows_cap, cudaStream_t s);
 

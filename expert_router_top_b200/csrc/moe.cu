@@ -1120,21 +1120,31 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
     if (s2 != MOE_OK) return s2;
     return ok(cudaEventRecord(ctx->ev_bf[0], sg)) ? MOE_OK : MOE_ERR_CUDA;
   };
-  // DY(c), stream M: dY = w dout (zero pad rows) and d_weights
-  auto DY = [&](int c) -> moe_status_t {
-    if (!ok(cudaStreamWaitEvent(s, ctx->ev_bf[0], 0))) return MOE_ERR_CUDA;
+  // DYS(c), stream M: dY = w dout into the chunk's padded rows (zero pad rows); it needs
+  // nothing from the recompute, only the previous pair's weight gradients to be done with
+  // this buffer set
+  auto DYS = [&](int c) -> moe_status_t {
     ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(c) * k, 0, 1);
     if (!ok(cudaMemsetAsync(buf(B.dy, c), 0, 2 * (size_t)R[c] * H, s)) ||
-        !ok(launch_dy_dw(dout + bounds[c] * H, buf(B.ydx, c), dstp_c(c),
-                         top_k_weights + bounds[c] * k, len(c), H, k, buf(B.dy, c),
-                         d_weights + bounds[c] * k, B.rows_cap, s)) ||
+        !ok(launch_dy_scatter(dout + bounds[c] * H, dstp_c(c), top_k_weights + bounds[c] * k,
+                              len(c), H, k, buf(B.dy, c), B.rows_cap, s)) ||
         !ok(cudaEventRecord(ctx->ev_bdy[0], s)))
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  };
+  // DW(c), stream M: d_weights = <dout, Y> with the recomputed Y rows
+  auto DW = [&](int c) -> moe_status_t {
+    if (!ok(cudaStreamWaitEvent(s, ctx->ev_bf[0], 0))) return MOE_ERR_CUDA;
+    ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(c) * k, 0, 1);
+    if (!ok(launch_dw_dot(dout + bounds[c] * H, buf(B.ydx, c), dstp_c(c), len(c), H, k,
+                          d_weights + bounds[c] * k, B.rows_cap, s)) ||
+        !ok(cudaEventRecord(ctx->ev_bdy[1], s)))
       return MOE_ERR_CUDA;
     return MOE_OK;
   };
   // Bd(c, c1), stream G: dh with the SwiGLU backward, then dX
   auto Bd = [&](int c, int c1) -> moe_status_t {
-    if (!ok(cudaStreamWaitEvent(sg, ctx->ev_bdy[0], 0))) return MOE_ERR_CUDA;
+    if (!ok(cudaStreamWaitEvent(sg, ctx->ev_bdy[0], 0))) return MOE_ERR_CUDA;  // dY rows
     BwdGemmArgs g = g0;
     g.offsets = offp_c(c);
     g.rows_pad_host = rows_pad.data() + (size_t)c * E;
@@ -1145,6 +1155,8 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
     g.N = I, g.K = H, g.b_rows = H, g.out0 = buf(B.dgu, c), g.aux = buf(B.gu, c);
     if (c1 > c) seg1(g, c1, buf(B.dy, c1), buf(B.dgu, c1), nullptr, buf(B.gu, c1));
     if (!ok(launch_pair(MOE_KERNEL_BWD_DSWIGLU, g, c, c1))) return MOE_ERR_CUDA;
+    // dX overwrites the Y rows: d_weights must have read them
+    if (!ok(cudaStreamWaitEvent(sg, ctx->ev_bdy[1], 0))) return MOE_ERR_CUDA;
     g = g0;
     g.offsets = offp_c(c);
     g.rows_pad_host = rows_pad.data() + (size_t)c * E;
@@ -1184,7 +1196,8 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
     g.M = 2 * I, g.N = H, g.acc = dW_gate_up;
     if (!ok(launch_pair(MOE_KERNEL_BWD_WGRAD, g, c, c1)) ||
         !ok(cudaEventRecord(ctx->ev_bw[c % 4], sg)) ||
-        (c1 > c && !ok(cudaEventRecord(ctx->ev_bw[c1 % 4], sg))))
+        (c1 > c && !ok(cudaEventRecord(ctx->ev_bw[c1 % 4], sg))) ||
+        !ok(cudaEventRecord(ctx->ev_bf[1], sg)))
       return MOE_ERR_CUDA;
     return MOE_OK;
   };
@@ -1201,11 +1214,13 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
 
   // The mirrored pair pipeline over pairs (c, c1) = (2m, 2m+1), every GEMM one sweep over
   // both chunks of the pair:
-  //   G: F(pair m) Bd(pair m) W(pair m) F(pair m+1) ...
-  //   M: P(c) P(c1) | DY(c) DY(c1) P(c+2) P(c+3) S(c) S(c1) | DY(c+2) ...
-  // The next pair's permutes run beside Bd, the d_hidden sums beside W; G waits for the
-  // pair's two DY row kernels between F and Bd.  Host enqueue order keeps each event wait
-  // on the record it is meant for.
+  //   G: F(pair m) DSwiGLU(m) DX(m) W(m) F(pair m+1) ...
+  //   M: P(c) P(c1) DYS(c) DYS(c1) | DW(c) DW(c1) P(c+2) P(c+3) S(c) S(c1) DYS(c+2) ...
+  // dY needs nothing from the recompute, so it is scattered while F runs; d_weights reads
+  // the recomputed Y beside the SwiGLU-backward GEMM, before dX overwrites those rows; the
+  // next pair's permutes run beside the dX and weight-gradient GEMMs, its dY scatter (after
+  // W(m) is done with the buffer set) beside F(m+1).  Host enqueue order keeps each event
+  // wait on the record it is meant for.
   if (!ok(cudaEventRecord(ctx->ev_start, s)) || !ok(cudaStreamWaitEvent(sg, ctx->ev_start, 0)))
     return MOE_ERR_CUDA;
   if (n_live > 0) {
@@ -1213,16 +1228,22 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
     if ((st = P(0)) != MOE_OK) return st;
     if (n_live > 1 && (st = P(1)) != MOE_OK) return st;
     if ((st = F(0, pair_end(0))) != MOE_OK) return st;
+    if ((st = DYS(0)) != MOE_OK || (n_live > 1 && (st = DYS(1)) != MOE_OK)) return st;
     for (int c = 0; c < n_live; c += 2) {
       const int c1 = pair_end(c);
       NvtxRange pr("moe_backward pair: chunks %d-%d", c, c1);
-      if ((st = DY(c)) != MOE_OK || (c1 > c && (st = DY(c1)) != MOE_OK)) return st;
+      if ((st = DW(c)) != MOE_OK || (c1 > c && (st = DW(c1)) != MOE_OK)) return st;
       for (int x = c + 2; x <= c + 3 && x < n_live; ++x)
         if ((st = P(x)) != MOE_OK) return st;
       if ((st = Bd(c, c1)) != MOE_OK) return st;
       if ((st = S(c)) != MOE_OK || (c1 > c && (st = S(c1)) != MOE_OK)) return st;
       if ((st = W(c, c1)) != MOE_OK) return st;
-      if (c + 2 < n_live && (st = F(c + 2, pair_end(c + 2))) != MOE_OK) return st;
+      if (c + 2 < n_live) {
+        if ((st = F(c + 2, pair_end(c + 2))) != MOE_OK) return st;
+        if (!ok(cudaStreamWaitEvent(s, ctx->ev_bf[1], 0))) return MOE_ERR_CUDA;  // W(m) done
+        for (int x = c + 2; x <= c + 3 && x < n_live; ++x)
+          if ((st = DYS(x)) != MOE_OK) return st;
+      }
     }
   }
   if (!ok(cudaEventRecord(ctx->ev_join, sg)) || !ok(cudaStreamWaitEvent(s, ctx->ev_join, 0)))
