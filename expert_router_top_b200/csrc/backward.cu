@@ -141,6 +141,33 @@ __device__ __forceinline__ Tile decode(int32_t L, const int32_t* ts, const int32
   return t;
 }
 
+// One epilogue warp's 32 rows x 32 bf16 columns (lane i holds row i as 16 packed pairs)
+// through 2 KB of shared memory: 16-byte chunk c of row r sits at c ^ ((r >> 1) & 3), which
+// keeps both the row-wise writes and the 8-rows-per-instruction reads free of bank
+// conflicts.  Row rr of the block goes to out + (row0 + rr) * ld + col0; rows at or past
+// nrows and columns at or past ncols are not written.
+__device__ __forceinline__ void store_block_staged(const uint32_t (&pk)[16], uint8_t* wbuf,
+                                                   int lane, __nv_bfloat16* out, int64_t row0,
+                                                   int32_t ld, int32_t col0, int32_t ncols,
+                                                   int32_t nrows, int64_t rows_cap) {
+  uint8_t* mine = wbuf + lane * 64;
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    *reinterpret_cast<uint4*>(mine + ((c ^ ((lane >> 1) & 3)) << 4)) =
+        make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+  __syncwarp();
+  const int seg = lane & 3;
+  const int32_t col = col0 + seg * 8;
+#pragma unroll
+  for (int pass = 0; pass < 4; ++pass) {
+    const int rr = pass * 8 + (lane >> 2);
+    const uint4 v = *reinterpret_cast<const uint4*>(wbuf + rr * 64 + ((seg ^ ((rr >> 1) & 3)) << 4));
+    if (rr < nrows && col < ncols && check_row(row0 + rr, rows_cap, &g_range_flags))
+      *reinterpret_cast<uint4*>(out + (row0 + rr) * ld + col) = v;
+  }
+  __syncwarp();
+}
+
 __device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 template <int kMode>
@@ -386,12 +413,15 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
           }
         }
       } else {
+        // rows of this warp's 32-row block that belong to the expert (the others are the
+        // next expert's), the block's first output row, and the buffers of its segment
         const int32_t rows_valid = offs[t.e + 1] - offs[t.e] - t.ml * BM;
-        const int64_t row = (int64_t)offs[t.e] + t.ml * BM + r;
-        const bool row_ok =
-            r < rows_valid && check_row(row, t.seg ? p.rows1 : p.rows0, &g_range_flags);
+        const int32_t nrows = rows_valid - q * 32;
+        const int64_t row0w = (int64_t)offs[t.e] + t.ml * BM + q * 32;
+        const int64_t cap = t.seg ? p.rows1 : p.rows0;
         __nv_bfloat16* o0 = t.seg ? p.out0b : p.out0;
         __nv_bfloat16* o1 = t.seg ? p.out1b : p.out1;
+        uint8_t* wbuf = sOut + (warp - 2) * 2048;  // 2 KB per epilogue warp
         if (kMode == kRawGU) {
 #pragma unroll 1
           for (int c = part * kCgu; c < (part + 1) * kCgu; ++c) {
@@ -400,31 +430,19 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
             tmem_ld_32cols(t_row + BN / 2 + c * 32, u);
             tmem_ld_wait2(g, u);
             const int32_t col0 = t.n * (BN / 2) + c * 32;
-            if (row_ok) {
-              uint32_t pg[16], pu[16], ph[16];
+            if (nrows <= 0 || col0 >= p.I) continue;  // warp-uniform
+            uint32_t pg[16], pu[16], ph[16];
 #pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
-                const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
-                pg[i] = pack_bf16x2(g0, g1);
-                pu[i] = pack_bf16x2(u0, u1);
-                ph[i] = pack_bf16x2(silu_f(g0) * u0, silu_f(g1) * u1);
-              }
-              __nv_bfloat16* gu = o0 + row * 2 * p.I;
-              __nv_bfloat16* act = o1 + row * p.I;
-#pragma unroll
-              for (int v4 = 0; v4 < 4; ++v4) {
-                if (col0 + v4 * 8 < p.I) {
-                  const int32_t cc = col0 + v4 * 8;
-                  *reinterpret_cast<uint4*>(gu + cc) =
-                      make_uint4(pg[4 * v4], pg[4 * v4 + 1], pg[4 * v4 + 2], pg[4 * v4 + 3]);
-                  *reinterpret_cast<uint4*>(gu + p.I + cc) =
-                      make_uint4(pu[4 * v4], pu[4 * v4 + 1], pu[4 * v4 + 2], pu[4 * v4 + 3]);
-                  *reinterpret_cast<uint4*>(act + cc) =
-                      make_uint4(ph[4 * v4], ph[4 * v4 + 1], ph[4 * v4 + 2], ph[4 * v4 + 3]);
-                }
-              }
+            for (int i = 0; i < 16; ++i) {
+              const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+              const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+              pg[i] = pack_bf16x2(g0, g1);
+              pu[i] = pack_bf16x2(u0, u1);
+              ph[i] = pack_bf16x2(silu_f(g0) * u0, silu_f(g1) * u1);
             }
+            store_block_staged(pg, wbuf, lane, o0, row0w, 2 * p.I, col0, p.I, nrows, cap);
+            store_block_staged(pu, wbuf, lane, o0 + p.I, row0w, 2 * p.I, col0, p.I, nrows, cap);
+            store_block_staged(ph, wbuf, lane, o1, row0w, p.I, col0, p.I, nrows, cap);
           }
         } else {
 #pragma unroll 1
@@ -435,16 +453,14 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
             if (kMode == kDSwiGLU && c + 1 < (part + 1) * kC) load_aux(c + 1, gn, un);
             tmem_ld_wait(v);
             const int32_t col0 = t.n * BN + c * 32;
-            if (!row_ok) continue;
+            const int32_t ncols = kMode == kDSwiGLU ? p.I : p.N;
+            if (nrows <= 0 || col0 >= ncols) continue;  // warp-uniform
             if (kMode == kDSwiGLU) {
-              __nv_bfloat16* dgu = o0 + row * 2 * p.I;
+              uint32_t dg[16], du[16];
 #pragma unroll
               for (int v4 = 0; v4 < 4; ++v4) {
-                const int32_t cc = col0 + v4 * 8;
-                if (cc >= p.I) continue;
                 const uint32_t ga[4] = {gq[v4].x, gq[v4].y, gq[v4].z, gq[v4].w};
                 const uint32_t ua[4] = {uq[v4].x, uq[v4].y, uq[v4].z, uq[v4].w};
-                uint32_t dg[4], du[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                   float dgv[2], duv[2];
@@ -457,30 +473,24 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
                     duv[h] = dh * gv * sig;
                     dgv[h] = dh * uv * (sig + gv * sig * (1.0f - sig));
                   }
-                  dg[i] = pack_bf16x2(dgv[0], dgv[1]);
-                  du[i] = pack_bf16x2(duv[0], duv[1]);
+                  dg[v4 * 4 + i] = pack_bf16x2(dgv[0], dgv[1]);
+                  du[v4 * 4 + i] = pack_bf16x2(duv[0], duv[1]);
                 }
-                *reinterpret_cast<uint4*>(dgu + cc) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
-                *reinterpret_cast<uint4*>(dgu + p.I + cc) = make_uint4(du[0], du[1], du[2], du[3]);
               }
+              store_block_staged(dg, wbuf, lane, o0, row0w, 2 * p.I, col0, p.I, nrows, cap);
+              store_block_staged(du, wbuf, lane, o0 + p.I, row0w, 2 * p.I, col0, p.I, nrows,
+                                 cap);
 #pragma unroll
               for (int v4 = 0; v4 < 4; ++v4) {
                 gq[v4] = gn[v4];
                 uq[v4] = un[v4];
               }
             } else {  // kDPlain
-              __nv_bfloat16* o = o0 + row * p.N;
+              uint32_t pk[16];
 #pragma unroll
-              for (int v4 = 0; v4 < 4; ++v4) {
-                const int32_t cc = col0 + v4 * 8;
-                if (cc >= p.N) continue;
-                uint32_t pk[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                  pk[i] = pack_bf16x2(__uint_as_float(v[v4 * 8 + 2 * i]),
-                                      __uint_as_float(v[v4 * 8 + 2 * i + 1]));
-                *reinterpret_cast<uint4*>(o + cc) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-              }
+              for (int i = 0; i < 16; ++i)
+                pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+              store_block_staged(pk, wbuf, lane, o0, row0w, p.N, col0, p.N, nrows, cap);
             }
           }
         }
