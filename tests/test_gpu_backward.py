@@ -110,3 +110,34 @@ def test_backward_full_size_sampled(moe):
         assert_grad_close(dwd[e], rd[remap[e]], f"qwen3 N=4 dW_down[{e}]")
     assert bool(torch.isfinite(dwgu).all()) and bool(torch.isfinite(dwd).all())
     assert bool(torch.isfinite(dx.float()).all())
+
+
+@pytest.mark.parametrize("E,k,T,H,I", [(1024, 8, 1536, 128, 128),   # MOE_MAX_EXPERTS
+                                       (64, 32, 600, 256, 192),     # MOE_MAX_TOPK
+                                       (1, 1, 300, 64, 64),         # one expert, top-1
+                                       (16, 4, 257, 192, 96)])      # I not a multiple of 64
+def test_backward_limits_and_odd_shapes(moe, E, k, T, H, I):
+    """The backward at the ABI's limits (the most experts, the largest top-k), with a single
+    expert, and with widths that are not multiples of the 128/256 tile widths: every
+    gradient against the oracle at three chunk counts (odd counts leave a pair with one
+    chunk), d_hidden and d_weights bit-identical across them."""
+    cfg = LayerConfig("bwd_limits", T, H, E, k, I, "normal")
+    cpu = layer_inputs(cfg)
+    dout = bf16_normal((T, H), 1.0, 99)
+    gpu = {kk: v.cuda() for kk, v in cpu.items()}
+    rx, rw, rgu, rd = oracle.backward(bits(cpu["hidden"]), cpu["idx"].numpy(), cpu["w"].numpy(),
+                                      bits(cpu["wgu"]), bits(cpu["wd"]), bits(dout))
+    base = None
+    for N in (1, 3, 4):
+        dx, dw, dwgu, dwd = moe.backward(gpu["hidden"], gpu["idx"], gpu["w"], gpu["wgu"],
+                                         gpu["wd"], dout.cuda(), num_chunks=N)
+        torch.cuda.synchronize()
+        tag = f"E={E} k={k} H={H} I={I} N={N}"
+        assert_layer_close(dx, rx, f"{tag} d_hidden")
+        assert_grad_close(dw, rw, f"{tag} d_weights")
+        assert_grad_close(dwgu, rgu, f"{tag} dW_gate_up")
+        assert_grad_close(dwd, rd, f"{tag} dW_down")
+        if base is None:
+            base = (dx, dw)
+        else:
+            assert torch.equal(dx, base[0]) and torch.equal(dw, base[1]), tag
