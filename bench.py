@@ -1,8 +1,11 @@
-"""Benchmark of the chunked MoE layer forward on B200.
+"""Benchmark of the chunked MoE layer on B200.
 
 One step = one moe_forward call over one batch of synthetic input: metadata for all
-chunks + the single device-to-host copy, then per chunk permute, gate/up GEMM with
-SwiGLU, down GEMM and weighted unpermute, as the two-stream pair pipeline.
+chunks + the single device-to-host copy, then the chunks' dispatch (a permute kernel, or
+row gathers inside the gate/up GEMM), gate/up GEMM with SwiGLU, down GEMM and weighted
+unpermute, as the two-stream pair pipeline (with the fused dispatch one GEMM sweep per
+pair of chunks).  `--pass backward` times moe_backward instead, `--pass train` a forward
+and a backward per step.
 
 Prints ONE JSON line (rank 0).  `value` is tokens/s of the whole job with inputs resident
 in HBM; `e2e` is the same metric through the public call with the step's inputs copied
