@@ -66,7 +66,8 @@ struct BParams {
   int32_t I;         // gate/up split of 2I-wide tensors
   int32_t b_rows;    // rows of one expert's weight matrix in B
   int32_t total_tiles;
-  __nv_bfloat16* out0;      // kRawGU: GU [rows][2I]; kDSwiGLU: dGU [rows][2I]; kDPlain: [rows][N]
+  __nv_bfloat16* out0;      // kRawGU: GU [rows][2I]; kDSwiGLU: [dg du] [rows][2I]
+                            // (may be aux: each block is read before it is stored); kDPlain: [rows][N]
   __nv_bfloat16* out1;      // kRawGU: Act [rows][I]
   const __nv_bfloat16* aux; // kDSwiGLU: GU [rows][2I]
   float* acc;               // kWGrad: [E][M][N] fp32 (written through tmC)

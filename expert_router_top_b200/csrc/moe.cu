@@ -202,8 +202,8 @@ struct DeviceCtx {
               ev_copy_join = nullptr;
   // backward pipeline: permuted rows ready (per X slot), recomputed Y ready, dY ready, dX
   // ready, d_hidden rows summed (per buffer), all of a chunk's GEMMs done (per X slot)
-  cudaEvent_t ev_bp[4] = {}, ev_bf[2] = {}, ev_bdy[2] = {}, ev_bdx[2] = {}, ev_bsum[2] = {},
-              ev_bw[4] = {};
+  cudaEvent_t ev_bp[3] = {}, ev_bf[2] = {}, ev_bdy[2] = {}, ev_bdx[2] = {}, ev_bsum[2] = {},
+              ev_bw[3] = {};
   int32_t* host_stage = nullptr;
   size_t host_stage_bytes = 0;
 };
@@ -241,7 +241,7 @@ moe_status_t get_ctx(DeviceCtx** out) {
           cudaEventCreateWithFlags(&c.ev_out_free[b], fl) != cudaSuccess)
         return MOE_ERR_CUDA;
     if (cudaEventCreateWithFlags(&c.ev_copy_join, fl) != cudaSuccess) return MOE_ERR_CUDA;
-    for (int b = 0; b < 4; ++b)
+    for (int b = 0; b < 3; ++b)
       if (cudaEventCreateWithFlags(&c.ev_bp[b], fl) != cudaSuccess ||
           cudaEventCreateWithFlags(&c.ev_bw[b], fl) != cudaSuccess)
         return MOE_ERR_CUDA;
@@ -901,14 +901,16 @@ struct BwdLayout {
   Layout meta;  // metadata regions (status/counts/splits, offsets, histograms, dst, src)
   size_t offp, first, dstp, total;
   int nx, nb;  // X slots (up to 4: two pairs) and buffer sets of the other rows
-  size_t xp[4], gu[2], act[2], ydx[2], dy[2], dgu[2];
+  size_t xp[3], gu[2], act[2], ydx[2], dy[2];  // gu later holds [dg du] in place
   int64_t rows_cap;
 };
 
 // Every chunk's rows, padded per expert to a multiple of 64, fit in rows_cap rows.  The
-// pipeline keeps chunk c's permuted rows in X slot c % 4 (they are read until its pair's
-// weight-gradient GEMM, while the next pair is permuted) and its other row buffers in set
-// c % 2.
+// pipeline keeps chunk c's permuted rows in X slot c % 3 (they are read until its pair's
+// weight-gradient GEMM; the next pair's first chunk is permuted meanwhile) and its other row
+// buffers in set c % 2.  The SwiGLU backward overwrites the saved [g u] rows with [dg du]
+// (each epilogue thread has read a block before any lane stores it), so one buffer holds
+// both.
 BwdLayout make_bwd_layout(const Dims& d, int32_t H, int32_t I) {
   BwdLayout B{};
   B.meta = make_layout(d, 8, 8, false, true, true);
@@ -921,7 +923,7 @@ BwdLayout make_bwd_layout(const Dims& d, int32_t H, int32_t I) {
   B.dstp = o;
   o += al(sizeof(int32_t) * (size_t)(d.T * d.k));
   const size_t R = (size_t)B.rows_cap;
-  B.nx = d.n >= 4 ? 4 : d.n;
+  B.nx = d.n >= 3 ? 3 : d.n;
   B.nb = d.n >= 2 ? 2 : 1;
   for (int b = 0; b < B.nx; ++b) {
     B.xp[b] = o;
@@ -936,8 +938,6 @@ BwdLayout make_bwd_layout(const Dims& d, int32_t H, int32_t I) {
     o += al(2 * R * H);
     B.dy[b] = o;
     o += al(2 * R * H);
-    B.dgu[b] = o;
-    o += al(2 * R * 2 * I);
   }
   B.total = o;
   return B;
@@ -1047,16 +1047,16 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
   auto len = [&](int c) { return bounds[c + 1] - bounds[c]; };
   auto ok = [](cudaError_t e) { return e == cudaSuccess; };
 
-  // P(c), stream M: padded permute of the chunk's rows into X slot c % 4 (zero pad rows)
+  // P(c), stream M: padded permute of the chunk's rows into X slot c % 3 (zero pad rows)
   auto P = [&](int c) -> moe_status_t {
-    if (c >= 4 && !ok(cudaStreamWaitEvent(s, ctx->ev_bw[c % 4], 0))) return MOE_ERR_CUDA;
+    if (c >= 3 && !ok(cudaStreamWaitEvent(s, ctx->ev_bw[c % 3], 0))) return MOE_ERR_CUDA;
     ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(c) * k, 0, 2);
     if (!ok(cudaMemsetAsync(x_of(c), 0, 2 * (size_t)R[c] * H, s)) ||
         !ok(launch_pad_rows(top_k_index + bounds[c] * k, dst + bounds[c] * k, off_c(c), offp_c(c),
                             len(c) * k, dstp_c(c), B.rows_cap, s)) ||
         !ok(launch_permute(hid + bounds[c] * H, dstp_c(c), len(c), H, k, x_of(c), B.rows_cap,
                            s)) ||
-        !ok(cudaEventRecord(ctx->ev_bp[c % 4], s)))
+        !ok(cudaEventRecord(ctx->ev_bp[c % 3], s)))
       return MOE_ERR_CUDA;
     return MOE_OK;
   };
@@ -1093,7 +1093,7 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
   // F(c, c1), stream G: recompute [g u], h and Y = h W_down^T on the padded rows
   auto F = [&](int c, int c1) -> moe_status_t {
     for (int x = c; x <= c1; ++x) {
-      if (!ok(cudaStreamWaitEvent(sg, ctx->ev_bp[x % 4], 0))) return MOE_ERR_CUDA;
+      if (!ok(cudaStreamWaitEvent(sg, ctx->ev_bp[x % 3], 0))) return MOE_ERR_CUDA;
       if (x >= 2 && !ok(cudaStreamWaitEvent(sg, ctx->ev_bsum[x % 2], 0))) return MOE_ERR_CUDA;
     }
     BwdGemmArgs g = g0;
@@ -1152,8 +1152,8 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
     g.mode = kBwdDSwiGLU;
     g.A = buf(B.dy, c), g.A_rows = R[c], g.A_cols = H;
     g.B = W_down, g.B_rows = (int64_t)E * H, g.B_cols = I;
-    g.N = I, g.K = H, g.b_rows = H, g.out0 = buf(B.dgu, c), g.aux = buf(B.gu, c);
-    if (c1 > c) seg1(g, c1, buf(B.dy, c1), buf(B.dgu, c1), nullptr, buf(B.gu, c1));
+    g.N = I, g.K = H, g.b_rows = H, g.out0 = buf(B.gu, c), g.aux = buf(B.gu, c);  // in place
+    if (c1 > c) seg1(g, c1, buf(B.dy, c1), buf(B.gu, c1), nullptr, buf(B.gu, c1));
     if (!ok(launch_pair(MOE_KERNEL_BWD_DSWIGLU, g, c, c1))) return MOE_ERR_CUDA;
     // dX overwrites the Y rows: d_weights must have read them
     if (!ok(cudaStreamWaitEvent(sg, ctx->ev_bdy[1], 0))) return MOE_ERR_CUDA;
@@ -1162,10 +1162,10 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
     g.rows_pad_host = rows_pad.data() + (size_t)c * E;
     g.chunk = c;
     g.mode = kBwdDPlain;
-    g.A = buf(B.dgu, c), g.A_rows = R[c], g.A_cols = 2 * I;
+    g.A = buf(B.gu, c), g.A_rows = R[c], g.A_cols = 2 * I;
     g.B = W_gate_up, g.B_rows = (int64_t)E * 2 * I, g.B_cols = H;
     g.N = H, g.K = 2 * I, g.b_rows = 2 * I, g.out0 = buf(B.ydx, c);
-    if (c1 > c) seg1(g, c1, buf(B.dgu, c1), buf(B.ydx, c1), nullptr, nullptr);
+    if (c1 > c) seg1(g, c1, buf(B.gu, c1), buf(B.ydx, c1), nullptr, nullptr);
     if (!ok(launch_pair(MOE_KERNEL_BWD_DX, g, c, c1)) ||
         !ok(cudaEventRecord(ctx->ev_bdx[0], sg)))
       return MOE_ERR_CUDA;
@@ -1190,13 +1190,13 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
     if (c1 > c) g.A1 = buf(B.dy, c1), g.B1 = buf(B.act, c1);
     g.M = H, g.N = I, g.acc = dW_down, g.out0 = nullptr;
     if (!ok(launch_pair(MOE_KERNEL_BWD_WGRAD, g, c, c1))) return MOE_ERR_CUDA;
-    g.A = buf(B.dgu, c), g.A_rows = R[c], g.A_cols = 2 * I;
+    g.A = buf(B.gu, c), g.A_rows = R[c], g.A_cols = 2 * I;  // [dg du]
     g.B = x_of(c), g.B_rows = R[c], g.B_cols = H;
-    if (c1 > c) g.A1 = buf(B.dgu, c1), g.B1 = x_of(c1);
+    if (c1 > c) g.A1 = buf(B.gu, c1), g.B1 = x_of(c1);
     g.M = 2 * I, g.N = H, g.acc = dW_gate_up;
     if (!ok(launch_pair(MOE_KERNEL_BWD_WGRAD, g, c, c1)) ||
-        !ok(cudaEventRecord(ctx->ev_bw[c % 4], sg)) ||
-        (c1 > c && !ok(cudaEventRecord(ctx->ev_bw[c1 % 4], sg))) ||
+        !ok(cudaEventRecord(ctx->ev_bw[c % 3], sg)) ||
+        (c1 > c && !ok(cudaEventRecord(ctx->ev_bw[c1 % 3], sg))) ||
         !ok(cudaEventRecord(ctx->ev_bf[1], sg)))
       return MOE_ERR_CUDA;
     return MOE_OK;
@@ -1215,12 +1215,12 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
   // The mirrored pair pipeline over pairs (c, c1) = (2m, 2m+1), every GEMM one sweep over
   // both chunks of the pair:
   //   G: F(pair m) DSwiGLU(m) DX(m) W(m) F(pair m+1) ...
-  //   M: P(c) P(c1) DYS(c) DYS(c1) | DW(c) DW(c1) P(c+2) P(c+3) S(c) S(c1) DYS(c+2) ...
+  //   M: P(c) P(c1) DYS(c) DYS(c1) | DW(c) DW(c1) P(c+2) S(c) S(c1) P(c+3) DYS(c+2) ...
   // dY needs nothing from the recompute, so it is scattered while F runs; d_weights reads
   // the recomputed Y beside the SwiGLU-backward GEMM, before dX overwrites those rows; the
-  // next pair's permutes run beside the dX and weight-gradient GEMMs, its dY scatter (after
-  // W(m) is done with the buffer set) beside F(m+1).  Host enqueue order keeps each event
-  // wait on the record it is meant for.
+  // next pair's first permute runs beside the dX and weight-gradient GEMMs, its second (in
+  // chunk c's X slot) and its dY scatter once W(m) is done with those buffers.  Host
+  // enqueue order keeps each event wait on the record it is meant for.
   if (!ok(cudaEventRecord(ctx->ev_start, s)) || !ok(cudaStreamWaitEvent(sg, ctx->ev_start, 0)))
     return MOE_ERR_CUDA;
   if (n_live > 0) {
@@ -1233,11 +1233,13 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
       const int c1 = pair_end(c);
       NvtxRange pr("moe_backward pair: chunks %d-%d", c, c1);
       if ((st = DW(c)) != MOE_OK || (c1 > c && (st = DW(c1)) != MOE_OK)) return st;
-      for (int x = c + 2; x <= c + 3 && x < n_live; ++x)
-        if ((st = P(x)) != MOE_OK) return st;
+      // the next pair's first chunk goes to the slot freed by the previous pair
+      if (c + 2 < n_live && (st = P(c + 2)) != MOE_OK) return st;
       if ((st = Bd(c, c1)) != MOE_OK) return st;
       if ((st = S(c)) != MOE_OK || (c1 > c && (st = S(c1)) != MOE_OK)) return st;
       if ((st = W(c, c1)) != MOE_OK) return st;
+      // its second chunk takes chunk c's slot, free once W(c, c1) has read it
+      if (c + 3 < n_live && (st = P(c + 3)) != MOE_OK) return st;
       if (c + 2 < n_live) {
         if ((st = F(c + 2, pair_end(c + 2))) != MOE_OK) return st;
         if (!ok(cudaStreamWaitEvent(s, ctx->ev_bf[1], 0))) return MOE_ERR_CUDA;  // W(m) done

@@ -299,8 +299,9 @@ MOE_API size_t moe_backward_workspace_bytes(const moe_shape_t* shape);
  * gradients accumulate per pair in fp32 (the first pair with an expert's rows stores, later
  * pairs add through TMA reductions).  d_hidden and d_weights are bit-identical for every
  * chunking; dW_* are equal up to the fp32 summation order.  workspace: dev, >=
- * moe_backward_workspace_bytes(shape): the metadata plus four chunk slots of permuted rows
- * and two chunk sets of the other row buffers.  The host blocks once, on the metadata copy.
+ * moe_backward_workspace_bytes(shape): the metadata plus three chunk slots of permuted rows
+ * and two chunk sets of the other row buffers (dg | du overwrite the recomputed g | u rows in
+ * place).  The host blocks once, on the metadata copy.
  * Errors: as moe_forward; MOE_ERR_ARG also for H % 64 or I % 32 != 0. */
 MOE_API moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
                                   const int32_t* top_k_index, const float* top_k_weights,
