@@ -100,11 +100,10 @@ struct KParams {
   const uint8_t* gsrc;    // gathered A: the token rows (hidden), and their stride in bytes
   int64_t gsrc_stride;
   int32_t K;              // valid K columns (gathered A: the rest of the last block reads 0)
-  // A second row segment sharing the tile sweep (the other chunk of a pair): its expert
-  // offsets [E+1] (nullptr: one segment), output rows, and gathered-A source rows.
+  // A second row segment sharing the tile sweep (plain A only): its expert offsets [E+1]
+  // (nullptr: one segment) and output rows.
   const int32_t* offsets1;
   __nv_bfloat16* out1;
-  const int32_t* gather1;
   int64_t gsrc_rows;             // checks build: rows of the gathered source
   int64_t out_rows0, out_rows1;  // checks build: rows of out and out1
 };
@@ -371,10 +370,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
     for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
       const Tile t = decode_tile<G::kTileM>(L, tile_start,
                                             off, off1p, E, p.n_tiles);
-      const int32_t* offs = t.seg ? off1 : off;
-      const int32_t* gat = t.seg ? p.gather1 : p.gather;
-      const int32_t row0 = offs[t.e] + t.ml * G::kTileM;
-      const int32_t last = offs[t.e + 1] - 1;  // rows past the expert re-read its last row
+      const int32_t* gat = p.gather;  // gathered A has one row segment
+      const int32_t row0 = off[t.e] + t.ml * G::kTileM;
+      const int32_t last = off[t.e + 1] - 1;  // rows past the expert re-read its last row
       const uint8_t* src[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -694,8 +692,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
   const int32_t bn = swiglu ? BN / 2 : BN;
   const bool gather = a.gather != nullptr;
   const bool two = a.offsets1 != nullptr;  // a second row segment (the pair's other chunk)
-  if ((gather && (kPair || !swiglu)) || (two && kPair) ||
-      (two && (!a.out1 || (gather ? !a.gather1 : !a.A1)))) {
+  if ((gather && (kPair || !swiglu || two)) || (two && kPair) || (two && (!a.out1 || !a.A1))) {
     *err_detail = 1;
     return cudaErrorInvalidValue;
   }
@@ -730,7 +727,6 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
   p.K = a.K;
   p.offsets1 = two ? a.offsets1 : nullptr;
   p.out1 = two ? static_cast<__nv_bfloat16*>(a.out1) : nullptr;
-  p.gather1 = two ? a.gather1 : nullptr;
   constexpr size_t smem = smem_bytes<kPair>();
   cudaError_t e;
   if (kPair) {

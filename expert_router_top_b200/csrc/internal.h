@@ -73,13 +73,12 @@ struct GemmArgs {
   const void* gather_src = nullptr;
   int64_t gather_src_rows = 0;
   // A second row segment in the same tile sweep (the other chunk of a pair: the weights of
-  // each expert tile are then fetched once for both): its expert offsets (dev [E+1]; nullptr
-  // = one segment), A rows (A1 [rows1][K], or gathered through gather1), and output rows.
-  // total_tiles then counts the tiles of both segments.
+  // each expert tile are then fetched once for both; plain A only): its expert offsets (dev
+  // [E+1]; nullptr = one segment), A rows (A1 [rows1][K]) and output rows.  total_tiles
+  // then counts the tiles of both segments.
   const int32_t* offsets1 = nullptr;
   const void* A1 = nullptr;
   int64_t rows1 = 0;
-  const int32_t* gather1 = nullptr;
   void* out1 = nullptr;
 };
 

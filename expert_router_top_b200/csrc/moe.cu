@@ -96,8 +96,22 @@ Dims make_dims(int64_t T, int32_t k, int32_t E, int32_t ep_groups, int32_t num_c
   return d;
 }
 
-// Workspace layout.  with_buffers: the expert buffers of moe_forward; with_dst/with_src:
-// scratch for the permutation when the caller does not provide it.
+// The pairs of chunks (2m, 2m+1) as chunks of their own: ceil(n/2) chunks of 2 t_chunk
+// tokens, pair m covering exactly the tokens of its two chunks.  Routing metadata at this
+// granularity lays the rows of each expert out contiguously over both chunks of a pair, so
+// one GEMM sweep serves the pair with row tiles that may span its two chunks.
+Dims pair_dims(const Dims& d) {
+  Dims p = d;
+  p.n = (d.n + 1) / 2;
+  p.t_chunk = 2 * d.t_chunk < d.T ? 2 * d.t_chunk : d.T;
+  p.tiles_per_chunk = (int32_t)((p.t_chunk + p.tile_tokens - 1) / p.tile_tokens);
+  if (p.tiles_per_chunk < 1) p.tiles_per_chunk = 1;
+  return p;
+}
+
+// Workspace layout.  with_buffers: the expert buffers of moe_forward (whose metadata may run
+// per chunk or per pair of chunks); with_dst/with_src: scratch for the permutation when the
+// caller does not provide it.
 Layout make_layout(const Dims& d, int32_t H, int32_t I, bool with_buffers, bool with_dst,
                    bool with_src) {
   Layout L{};
@@ -108,7 +122,12 @@ Layout make_layout(const Dims& d, int32_t H, int32_t I, bool with_buffers, bool 
   L.offsets = o;
   o += al(sizeof(int32_t) * (size_t)d.n * (d.E + 1));
   L.hist = o;
-  o += al(sizeof(int32_t) * (size_t)d.n * d.tiles_per_chunk * d.E);
+  size_t hist_tiles = (size_t)d.n * d.tiles_per_chunk;
+  if (with_buffers) {
+    const Dims p = pair_dims(d);
+    if ((size_t)p.n * p.tiles_per_chunk > hist_tiles) hist_tiles = (size_t)p.n * p.tiles_per_chunk;
+  }
+  o += al(sizeof(int32_t) * hist_tiles * d.E);
   L.dst = o;
   if (with_dst) o += al(sizeof(int32_t) * (size_t)(d.T * d.k));
   L.src = o;
@@ -116,11 +135,14 @@ Layout make_layout(const Dims& d, int32_t H, int32_t I, bool with_buffers, bool 
   L.nbuf = 0;
   L.rows_cap = d.t_chunk * d.k;
   if (with_buffers) {
-    // the pair double buffer: one buffer for N = 1, two otherwise
+    // the pair double buffer: one buffer for N = 1, two otherwise.  The two X|Y buffers are
+    // adjacent, and so are the two Act buffers: a pair's rows fill both as one buffer.
     L.nbuf = d.n >= 2 ? 2 : 1;
     for (int b = 0; b < L.nbuf; ++b) {
       L.xy[b] = o;
       o += al(sizeof(uint16_t) * (size_t)L.rows_cap * H);
+    }
+    for (int b = 0; b < L.nbuf; ++b) {
       L.act[b] = o;
       o += al(sizeof(uint16_t) * (size_t)L.rows_cap * I);
     }
@@ -383,13 +405,12 @@ int64_t active_experts(const int32_t* counts, int32_t E) {
 }
 
 
-// The second row segment of a grouped GEMM that serves both chunks of a pair.
+// The second row segment of a grouped GEMM that serves both chunks of a pair (plain A).
 struct Seg1 {
-  const void* A = nullptr;           // [rows][K], or nullptr with gathered A
+  const void* A = nullptr;           // [rows][K]
   int64_t rows = 0;
   const int32_t* offsets = nullptr;  // dev [E+1]
   const int32_t* counts = nullptr;   // host [E]
-  const int32_t* gather = nullptr;   // gathered A: token row of each of its rows
   void* out = nullptr;
 };
 
@@ -405,7 +426,6 @@ moe_status_t gemm_call(const void* A, int64_t rows, const void* B, void* out,
     g.offsets1 = seg1->offsets;
     g.A1 = seg1->A;
     g.rows1 = seg1->rows;
-    g.gather1 = seg1->gather;
     g.out1 = seg1->out;
     rows_all += seg1->rows;
     active = 0;  // experts with rows in either segment
@@ -608,12 +628,15 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
   int32_t* src = reinterpret_cast<int32_t*>(ws + L.src);
   uint32_t* dev_status = reinterpret_cast<uint32_t*>(ws + L.packed);
 
-  // 1) metadata for all chunks, 2) the one device-to-host copy (the only host stall)
-  if ((st = run_metadata(d, top_k_index, ws, L, dst, src, sm)) != MOE_OK) return st;
+  // 1) metadata for all chunks (with pair sweeps: for all pairs, so that each expert's rows
+  // are contiguous over both chunks of a pair), 2) the one device-to-host copy (the only
+  // host stall)
+  const Dims dm = pair_gemms ? pair_dims(d) : d;
+  if ((st = run_metadata(dm, top_k_index, ws, L, dst, src, sm)) != MOE_OK) return st;
   if ((st = fetch_packed(ctx, ws, L, sm)) != MOE_OK) return st;
   // Copy what the pipeline needs out of the shared staging block.
   std::vector<int32_t> counts(ctx->host_stage + kStatusWords,
-                              ctx->host_stage + kStatusWords + (size_t)d.n * d.E);
+                              ctx->host_stage + kStatusWords + (size_t)dm.n * d.E);
   std::vector<int64_t> bounds = dims_bounds(d);
   int n_live = 0;  // chunks with tokens; only trailing chunks can be empty
   while (n_live < d.n && bounds[n_live + 1] > bounds[n_live]) ++n_live;
@@ -678,43 +701,37 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
       if ((st = unpermute(c)) != MOE_OK) return st;
     }
   } else if (n_live > 0 && pair_gemms) {
-    // Pairs (c0, c1) = (2m, 2m+1), chunk c in buffer c % 2.  G: GU(m) D(m) GU(m+1) D(m+1) ...
-    // where GU / D are the gate/up and down GEMMs of both chunks of the pair in one tile
-    // sweep (each expert's weight tiles are fetched once for the pair); D(m+1) waits until
-    // U(c0), U(c1) have read the pair's Y rows.  M: U(c0) U(c1) after D(m), beside GU(m+1).
-    auto seg = [&](int c, const void* A, void* out) {
-      Seg1 g1;
-      g1.A = A;
-      g1.rows = len(c) * k;
-      g1.offsets = reinterpret_cast<const int32_t*>(ws + L.offsets) + (size_t)c * (E + 1);
-      g1.counts = counts.data() + (size_t)c * E;
-      g1.gather = A ? nullptr : src + bounds[c] * k;
-      g1.out = out;
-      return g1;
-    };
-    for (int c0 = 0; c0 < n_live; c0 += 2) {
-      NvtxRange pr("moe_forward pair: chunks %d-%d", c0, c0 + 1 < n_live ? c0 + 1 : c0);
-      const bool two = c0 + 1 < n_live;
-      const int c1 = c0 + 1;
-      const Seg1 s0 = seg(c0, nullptr, act(c0));
-      Seg1 s1 = two ? seg(c1, nullptr, act(c1)) : Seg1{};
-      moe_status_t s2 = gemm_call(nullptr, s0.rows, W_gate_up, act(c0), s0.offsets, s0.counts,
-                                  E, H, I, 2 * I, true, dev_status, ctx->num_sms, sg, s0.gather,
-                                  hidden, T, two ? &s1 : nullptr);
+    // Pairs (c0, c1) = (2m, 2m+1).  G: GU(m) D(m) GU(m+1) D(m+1) ..., where GU / D are the
+    // gate/up and down GEMMs of the pair in one tile sweep over its rows, laid out per expert
+    // across both chunks (each expert's weight tiles are fetched once for the pair, and a row
+    // tile may hold rows of both chunks); D(m+1) waits until U(c0), U(c1) have read the
+    // pair's Y rows.  M: U(c0) U(c1) after D(m), beside GU(m+1).  The pair's rows fill both
+    // halves of the X|Y and Act double buffers; dst holds pair-local rows.
+    const std::vector<int64_t> pb = dims_bounds(dm);
+    void* y_pair = ws + L.xy[0];
+    void* act_pair = ws + L.act[0];
+    const int64_t pair_cap = L.rows_cap * L.nbuf;
+    for (int m = 0; 2 * m < n_live; ++m) {
+      const int c0 = 2 * m, c1 = 2 * m + 1 < n_live ? 2 * m + 1 : 2 * m;
+      NvtxRange pr("moe_forward pair: chunks %d-%d", c0, c1);
+      const int64_t rows = (pb[m + 1] - pb[m]) * k;
+      const int32_t* cnt = counts.data() + (size_t)m * E;
+      const int32_t* offs = reinterpret_cast<const int32_t*>(ws + L.offsets) + (size_t)m * (E + 1);
+      moe_status_t s2 = gemm_call(nullptr, rows, W_gate_up, act_pair, offs, cnt, E, H, I, 2 * I,
+                                  true, dev_status, ctx->num_sms, sg, src + pb[m] * k, hidden, T);
       if (s2 != MOE_OK) return s2;
-      if (c0 >= 2 && cudaStreamWaitEvent(sg, ctx->ev_unperm[0], 0) != cudaSuccess)
+      if (m > 0 && cudaStreamWaitEvent(sg, ctx->ev_unperm[0], 0) != cudaSuccess)
         return MOE_ERR_CUDA;
-      if (two) s1 = seg(c1, act(c1), xy(c1));
-      s2 = gemm_call(act(c0), s0.rows, W_down, xy(c0), s0.offsets, s0.counts, E, I, H, H, false,
-                     dev_status, ctx->num_sms, sg, nullptr, nullptr, 0, two ? &s1 : nullptr);
+      s2 = gemm_call(act_pair, rows, W_down, y_pair, offs, cnt, E, I, H, H, false, dev_status,
+                     ctx->num_sms, sg);
       if (s2 != MOE_OK) return s2;
       if (cudaEventRecord(ctx->ev_gemm[0], sg) != cudaSuccess ||
           cudaStreamWaitEvent(sm, ctx->ev_gemm[0], 0) != cudaSuccess)
         return MOE_ERR_CUDA;
-      for (int c = c0; c <= (two ? c1 : c0); ++c) {
+      for (int c = c0; c <= c1; ++c) {
         ProfScope ps(MOE_KERNEL_UNPERMUTE, sm, len(c) * k, 0, 1);
-        if (launch_unpermute(xy(c), dst + bounds[c] * k, top_k_weights + bounds[c] * k, len(c),
-                             H, k, outp + bounds[c] * H, L.rows_cap, sm) != cudaSuccess)
+        if (launch_unpermute(y_pair, dst + bounds[c] * k, top_k_weights + bounds[c] * k, len(c),
+                             H, k, outp + bounds[c] * H, pair_cap, sm) != cudaSuccess)
           return MOE_ERR_CUDA;
       }
       if (cudaEventRecord(ctx->ev_unperm[0], sm) != cudaSuccess) return MOE_ERR_CUDA;
@@ -900,7 +917,7 @@ namespace {
 struct BwdLayout {
   Layout meta;  // metadata regions (status/counts/splits, offsets, histograms, dst, src)
   size_t offp, first, dstp, total;
-  int nx, nb;  // X slots (up to 4: two pairs) and buffer sets of the other rows
+  int nx, nb;  // X slots (up to 3) and buffer sets of the other rows
   size_t xp[3], gu[2], act[2], ydx[2], dy[2];  // gu later holds [dg du] in place
   int64_t rows_cap;
 };

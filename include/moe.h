@@ -239,8 +239,10 @@ MOE_API moe_status_t moe_forward(const moe_shape_t* shape, const void* hidden, c
  * permuted copy of the input is written or read.  With the fused dispatch the two chunks of
  * each pair (2m, 2m+1) share one tile sweep per GEMM, so each expert's weight tiles are
  * fetched once per pair rather than once per chunk (MOE_FWD_PER_CHUNK_GEMMS: one sweep per
- * chunk), and the unpermutes of pair m overlap the gate/up GEMM of pair m+1; the workspace
- * is unchanged (the pair's two chunk buffers are resident anyway).  flags = 0 (what
+ * chunk), and the unpermutes of pair m overlap the gate/up GEMM of pair m+1.  The routing
+ * metadata then runs per pair, so each expert's rows are contiguous over both chunks and a
+ * row tile may span them; the workspace is unchanged (the pair's two chunk buffers are
+ * resident anyway and hold its rows as one buffer).  flags = 0 (what
  * moe_forward does) chooses fused whenever there are two or more chunks (the pair sweeps
  * halve the weight stream), and with one chunk when it holds at least I/4 rows per expert
  * on average (4 * T * k >= E * I: the permuted copy it saves is then a sizeable share of
