@@ -21,7 +21,7 @@
 //   kDSwiGLU  dh = dY W_down                  B MN-major                  epilogue: dg, du
 //   kDPlain   dX = [dg du] W_gate_up          B MN-major                  epilogue: bf16 store
 //   kWGrad    dW[e] += S_A[e]^T S_B[e]        A and B MN-major, K = rows  epilogue: TMA fp32
-//             (K = the rows of one chunk, or of a pair of chunks)       store / add-reduce
+//             (K = the expert's padded rows of one pair of chunks)      store / add-reduce
 // MN-major operands use the 128-byte-swizzled MN-major canonical layout: 64-element MN
 // blocks of 64 K rows x 128 B (8 KB apart: the leading byte offset), 8-row K groups 1 KB
 // apart (the stride byte offset); one MMA K step of 16 advances 2 KB.
@@ -71,16 +71,9 @@ struct BParams {
   __nv_bfloat16* out1;      // kRawGU: Act [rows][I]
   const __nv_bfloat16* aux; // kDSwiGLU: GU [rows][2I]
   float* acc;               // kWGrad: [E][M][N] fp32 (written through tmC)
-  const int32_t* first;     // kWGrad: [E] first chunk with rows of each expert
-  int32_t chunk;            // kWGrad: first chunk of this launch
-  int32_t chunk_last;       // kWGrad: last chunk of this launch (chunk + 1 for a pair)
-  const int32_t* offsets1;  // padded offsets [E+1] of the pair's second chunk, or null: for
-                            // kWGrad its rows extend K; for the row-grouped modes they are a
-                            // second row segment of the same tile sweep (A rows from tmA1)
-  int64_t rows0, rows1;     // checks build: rows of the A / output buffers of each segment
-  __nv_bfloat16* out0b;     // row-grouped modes: out0 / out1 / aux of the second segment
-  __nv_bfloat16* out1b;
-  const __nv_bfloat16* auxb;
+  const int32_t* first;     // kWGrad: [E] first unit (pair of chunks) with rows of each expert
+  int32_t chunk;            // kWGrad: the unit of this launch (store where first == chunk)
+  int64_t rows;             // checks build: rows of the A / output buffers
 };
 
 struct Ctl {
@@ -94,7 +87,7 @@ static_assert(sizeof(Ctl) <= kCtlBytes, "control block");
 constexpr uint32_t kOutBoxBytes = 32 * 32 * 4;
 constexpr uint32_t kOutBytes = 4 * kOutBoxBytes;
 constexpr size_t kSmem =
-    1024 + STAGES * kStageBytes + kOutBytes + kCtlBytes + 3 * (kMaxE + 1) * 4;
+    1024 + STAGES * kStageBytes + kOutBytes + kCtlBytes + 2 * (kMaxE + 1) * 4;
 static_assert(kSmem <= 232448, "shared memory per CTA");
 
 __host__ __device__ constexpr uint32_t idesc(bool a_mn, bool b_mn) {
@@ -108,15 +101,14 @@ __device__ __forceinline__ uint64_t mn_desc(uint32_t addr) {
          (static_cast<uint64_t>(1024 >> 4) << 32) | (1ull << 46) | (2ull << 61);
 }
 
-// A tile: expert e, column tile n, row tile m (row-grouped modes: over the expert's rows of
-// both segments, segment 0 first, i.e. row tile ml of segment seg).
+// A tile: expert e, column tile n, row tile m.
 struct Tile {
-  int32_t e, m, n, seg, ml;
+  int32_t e, m, n;
 };
 
 template <int kMode>
 __device__ __forceinline__ Tile decode(int32_t L, const int32_t* ts, const int32_t* off,
-                                       const int32_t* off1, int32_t E, const BParams& p) {
+                                       int32_t E, const BParams& p) {
   int32_t lo = 0, hi = E - 1;
   while (lo < hi) {
     const int32_t mid = (lo + hi + 1) >> 1;
@@ -126,18 +118,13 @@ __device__ __forceinline__ Tile decode(int32_t L, const int32_t* ts, const int32
   const int32_t local = L - ts[lo];
   Tile t;
   t.e = lo;
-  t.seg = 0;
   if (kMode == kWGrad) {
     t.m = local / p.n_tiles;
     t.n = local - t.m * p.n_tiles;
-    t.ml = t.m;
   } else {
-    const int32_t mt0 = (off[lo + 1] - off[lo] + BM - 1) / BM;
-    const int32_t mt = mt0 + (p.offsets1 ? (off1[lo + 1] - off1[lo] + BM - 1) / BM : 0);
+    const int32_t mt = (off[lo + 1] - off[lo] + BM - 1) / BM;
     t.n = local / mt;
     t.m = local - t.n * mt;
-    t.seg = t.m >= mt0 ? 1 : 0;
-    t.ml = t.m - (t.seg ? mt0 : 0);
   }
   return t;
 }
@@ -175,9 +162,7 @@ template <int kMode>
 __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ CUtensorMap tmC,
-                    const __grid_constant__ CUtensorMap tmA1,
-                    const __grid_constant__ CUtensorMap tmB1, const BParams p) {
+                    const __grid_constant__ CUtensorMap tmC, const BParams p) {
   constexpr bool kAmn = kMode == kWGrad;
   constexpr bool kBmn = kMode != kRawGU;
   extern __shared__ uint8_t smem_raw[];
@@ -189,17 +174,11 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
   Ctl* ctl = reinterpret_cast<Ctl*>(sOut + kOutBytes);
   int32_t* off = reinterpret_cast<int32_t*>(sOut + kOutBytes + kCtlBytes);
   int32_t* ts = off + (kMaxE + 1);
-  // kWGrad over a pair of chunks: K runs over the expert's padded rows of the first chunk
-  // (offsets off, operands tmA/tmB), then of the second (off1, tmA1/tmB1)
-  int32_t* off1 = ts + (kMaxE + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int32_t E = p.E;
 
   constexpr int kEpi = Cfg<kMode>::kEpi;
-  for (int32_t i = threadIdx.x; i <= E; i += Cfg<kMode>::kThreads) {
-    off[i] = p.offsets[i];
-    off1[i] = p.offsets1 ? p.offsets1[i] : 0;
-  }
+  for (int32_t i = threadIdx.x; i <= E; i += Cfg<kMode>::kThreads) off[i] = p.offsets[i];
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&ctl->full[s], 1);
@@ -223,8 +202,8 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
     const int32_t e0 = lane * per, e1 = min(E, e0 + per);
     auto tiles_of = [&](int32_t e) -> int32_t {
       const int32_t rows = off[e + 1] - off[e];
-      if (kMode == kWGrad) return rows + off1[e + 1] - off1[e] > 0 ? p.m_tiles * p.n_tiles : 0;
-      return ((rows + BM - 1) / BM + (off1[e + 1] - off1[e] + BM - 1) / BM) * p.n_tiles;
+      if (kMode == kWGrad) return rows > 0 ? p.m_tiles * p.n_tiles : 0;
+      return (rows + BM - 1) / BM * p.n_tiles;
     };
     int32_t sum = 0;
     for (int32_t e = e0; e < e1; ++e) sum += tiles_of(e);
@@ -254,9 +233,8 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
       uint32_t phase = 0, armed = 0, armed_parity = 0;
       bool ok = true;
       for (int32_t L = blockIdx.x; L < p.total_tiles && ok; L += gridDim.x) {
-        const Tile t = decode<kMode>(L, ts, off, off1, E, p);
-        const int32_t nkb0 = (off[t.e + 1] - off[t.e]) / BK;
-        const int32_t nkb = kMode == kWGrad ? nkb0 + (off1[t.e + 1] - off1[t.e]) / BK : p.num_kb;
+        const Tile t = decode<kMode>(L, ts, off, E, p);
+        const int32_t nkb = kMode == kWGrad ? (off[t.e + 1] - off[t.e]) / BK : p.num_kb;
         for (int32_t kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort, p.status)) {
             ok = false;
@@ -267,15 +245,12 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
           uint8_t* b = sB + stage * kBBytes;
           uint64_t* bar = &ctl->full[stage];
           if (kMode == kWGrad) {
-            const bool seg0 = kb < nkb0;
-            const int32_t r0 = seg0 ? off[t.e] + kb * BK : off1[t.e] + (kb - nkb0) * BK;
-            const CUtensorMap* ma = seg0 ? &tmA : &tmA1;
-            const CUtensorMap* mb = seg0 ? &tmB : &tmB1;
-            for (int q = 0; q < 2; ++q) tma_load_2d(a + q * 8192, ma, bar, t.m * BM + q * 64, r0, pol);
-            for (int q = 0; q < 4; ++q) tma_load_2d(b + q * 8192, mb, bar, t.n * BN + q * 64, r0, pol);
+            const int32_t r0 = off[t.e] + kb * BK;
+            for (int q = 0; q < 2; ++q) tma_load_2d(a + q * 8192, &tmA, bar, t.m * BM + q * 64, r0, pol);
+            for (int q = 0; q < 4; ++q) tma_load_2d(b + q * 8192, &tmB, bar, t.n * BN + q * 64, r0, pol);
           } else {
-            const int32_t row0 = (t.seg ? off1 : off)[t.e] + t.ml * BM;
-            tma_load_2d(a, t.seg ? &tmA1 : &tmA, bar, kb * BK, row0, pol);
+            const int32_t row0 = off[t.e] + t.m * BM;
+            tma_load_2d(a, &tmA, bar, kb * BK, row0, pol);
             if (kMode == kRawGU) {
               const int32_t brow = t.e * p.b_rows + t.n * (BN / 2);
               tma_load_2d(b, &tmB, bar, kb * BK, brow, pol);
@@ -305,10 +280,8 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
       bool ok = true, issued = false;
       int32_t it = 0;
       for (int32_t L = blockIdx.x; L < p.total_tiles && ok; L += gridDim.x, ++it) {
-        const Tile t = decode<kMode>(L, ts, off, off1, E, p);
-        const int32_t nkb = kMode == kWGrad
-                                ? (off[t.e + 1] - off[t.e] + off1[t.e + 1] - off1[t.e]) / BK
-                                : p.num_kb;
+        const Tile t = decode<kMode>(L, ts, off, E, p);
+        const int32_t nkb = kMode == kWGrad ? (off[t.e + 1] - off[t.e]) / BK : p.num_kb;
         const int buf = it & 1;
         if (!mbar_wait(&ctl->tempty[buf], ((it >> 1) & 1) ^ 1u, abort, p.status)) {
           ok = false;
@@ -356,14 +329,13 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
     int32_t it = 0;
     for (int32_t L = blockIdx.x; L < p.total_tiles; L += gridDim.x, ++it) {
       const int buf = it & 1;
-      const Tile t = decode<kMode>(L, ts, off, off1, E, p);
+      const Tile t = decode<kMode>(L, ts, off, E, p);
       // kDSwiGLU: the saved g and u of this thread's row, one 32-column block ahead of the
       // accumulator; the first block is requested before the accumulator is ready
       uint4 gq[4], uq[4];
-      const int32_t* offs = t.seg ? off1 : off;
-      const int32_t rows_here = offs[t.e + 1] - offs[t.e] - t.ml * BM;
-      const int64_t row_g = (int64_t)offs[t.e] + t.ml * BM + r;
-      const __nv_bfloat16* aux = t.seg ? p.auxb : p.aux;
+      const int32_t rows_here = off[t.e + 1] - off[t.e] - t.m * BM;
+      const int64_t row_g = (int64_t)off[t.e] + t.m * BM + r;
+      const __nv_bfloat16* aux = p.aux;
       auto load_aux = [&](int c, uint4 (&g)[4], uint4 (&u)[4]) {
         const uint4* gu4 = reinterpret_cast<const uint4*>(aux + row_g * 2 * p.I);
 #pragma unroll
@@ -386,11 +358,11 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
         // Each warp owns accumulator rows q*32..q*32+31: per 32-column block it stages the
         // 32 x 32 fp32 block in shared memory (16-byte chunk i of row `lane` at i ^ (lane % 8),
         // the 128-byte swizzle of the tensor map) and one lane stores it -- the expert's first
-        // chunk with rows -- or adds it into dW with one TMA reduction.  Each element of dW
-        // gets one store or add per chunk, in chunk order.
+        // pair of chunks with rows -- or adds it into dW with one TMA reduction.  Each element
+        // of dW gets one store or add per pair, in pair order.
         uint8_t* box = sOut + q * kOutBoxBytes;
         const int32_t m0 = t.m * BM + q * 32;
-        const bool store = p.first[t.e] >= p.chunk && p.first[t.e] <= p.chunk_last;
+        const bool store = p.first[t.e] == p.chunk;
 #pragma unroll 1
         for (int c = part * kC; c < (part + 1) * kC; ++c) {
           uint32_t v[32];
@@ -415,13 +387,13 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
         }
       } else {
         // rows of this warp's 32-row block that belong to the expert (the others are the
-        // next expert's), the block's first output row, and the buffers of its segment
-        const int32_t rows_valid = offs[t.e + 1] - offs[t.e] - t.ml * BM;
+        // next expert's) and the block's first output row
+        const int32_t rows_valid = off[t.e + 1] - off[t.e] - t.m * BM;
         const int32_t nrows = rows_valid - q * 32;
-        const int64_t row0w = (int64_t)offs[t.e] + t.ml * BM + q * 32;
-        const int64_t cap = t.seg ? p.rows1 : p.rows0;
-        __nv_bfloat16* o0 = t.seg ? p.out0b : p.out0;
-        __nv_bfloat16* o1 = t.seg ? p.out1b : p.out1;
+        const int64_t row0w = (int64_t)off[t.e] + t.m * BM + q * 32;
+        const int64_t cap = p.rows;
+        __nv_bfloat16* o0 = p.out0;
+        __nv_bfloat16* o1 = p.out1;
         uint8_t* wbuf = sOut + (warp - 2) * 2048;  // 2 KB per epilogue warp
         if (kMode == kRawGU) {
 #pragma unroll 1
@@ -628,14 +600,13 @@ __global__ void __launch_bounds__(kRowThreads)
 
 template <int kMode>
 cudaError_t launch_mode(const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mC,
-                        const CUtensorMap& mA1, const CUtensorMap& mB1, const BParams& p,
-                        int num_sms, cudaStream_t s) {
+                        const BParams& p, int num_sms, cudaStream_t s) {
   if (p.total_tiles <= 0) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(bwd_gemm_kernel<kMode>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
   if (e != cudaSuccess) return e;
   const int grid = p.total_tiles < num_sms ? p.total_tiles : num_sms;
-  bwd_gemm_kernel<kMode><<<grid, Cfg<kMode>::kThreads, kSmem, s>>>(mA, mB, mC, mA1, mB1, p);
+  bwd_gemm_kernel<kMode><<<grid, Cfg<kMode>::kThreads, kSmem, s>>>(mA, mB, mC, p);
   return cudaGetLastError();
 }
 
@@ -652,13 +623,13 @@ cudaError_t launch_bwd_gemm(const BwdGemmArgs& a, int num_sms, cudaStream_t s) {
   // N tiles: kRawGU pairs 128 gate with 128 up columns per tile; the others are 256 wide
   const int32_t n_tiles = a.mode == kRawGU ? (a.I + BN / 2 - 1) / (BN / 2) : (a.N + BN - 1) / BN;
   for (int32_t e = 0; e < a.E; ++e) {
-    const int64_t r0 = a.rows_pad_host[e], r1 = a.rows_pad_host1 ? a.rows_pad_host1[e] : 0;
-    if (a.mode == kWGrad) tiles += r0 + r1 > 0 ? (int64_t)((a.M + BM - 1) / BM) * n_tiles : 0;
-    else tiles += ((r0 + BM - 1) / BM + (r1 + BM - 1) / BM) * n_tiles;
+    const int64_t r = a.rows_pad_host[e];
+    if (a.mode == kWGrad) tiles += r > 0 ? (int64_t)((a.M + BM - 1) / BM) * n_tiles : 0;
+    else tiles += (r + BM - 1) / BM * n_tiles;
   }
   if (tiles <= 0) return cudaSuccess;
   if (tiles > 0x7fffffff) return cudaErrorInvalidValue;
-  CUtensorMap mA, mB, mC, mA1, mB1;
+  CUtensorMap mA, mB, mC;
   const bool a_mn = a.mode == kWGrad;
   const bool b_mn = a.mode != kRawGU;
   if (!make_tma_2d_bf16(&mA, a.A, a.A_rows, a.A_cols, a_mn ? BK : BM) ||
@@ -669,22 +640,6 @@ cudaError_t launch_bwd_gemm(const BwdGemmArgs& a, int num_sms, cudaStream_t s) {
       return cudaErrorInvalidValue;
   } else {
     mC = mA;  // unused
-  }
-  const bool pair = a.offsets1 != nullptr;
-  if (pair && a.mode == kWGrad) {
-    if (!a.A1 || !a.B1 || !a.rows_pad_host1 ||
-        !make_tma_2d_bf16(&mA1, a.A1, a.A1_rows, a.A_cols, BK) ||
-        !make_tma_2d_bf16(&mB1, a.B1, a.B1_rows, a.B_cols, BK))
-      return cudaErrorInvalidValue;
-  } else if (pair) {  // a second row segment: its own A rows, the same weights
-    if (!a.A1 || !a.rows_pad_host1 || !a.out0b || (a.mode == kRawGU && !a.out1b) ||
-        (a.mode == kDSwiGLU && !a.auxb) ||
-        !make_tma_2d_bf16(&mA1, a.A1, a.A1_rows, a.A_cols, BM))
-      return cudaErrorInvalidValue;
-    mB1 = mB;  // unused
-  } else {
-    mA1 = mA;  // unused
-    mB1 = mB;
   }
   BParams p;
   p.offsets = a.offsets;
@@ -704,18 +659,12 @@ cudaError_t launch_bwd_gemm(const BwdGemmArgs& a, int num_sms, cudaStream_t s) {
   p.acc = a.acc;
   p.first = a.first;
   p.chunk = a.chunk;
-  p.chunk_last = pair ? a.chunk + 1 : a.chunk;
-  p.offsets1 = pair ? a.offsets1 : nullptr;
-  p.rows0 = a.A_rows;
-  p.rows1 = a.A1_rows;
-  p.out0b = static_cast<__nv_bfloat16*>(a.out0b);
-  p.out1b = static_cast<__nv_bfloat16*>(a.out1b);
-  p.auxb = static_cast<const __nv_bfloat16*>(a.auxb);
+  p.rows = a.A_rows;
   switch (a.mode) {
-    case kRawGU: return launch_mode<kRawGU>(mA, mB, mC, mA1, mB1, p, num_sms, s);
-    case kDSwiGLU: return launch_mode<kDSwiGLU>(mA, mB, mC, mA1, mB1, p, num_sms, s);
-    case kDPlain: return launch_mode<kDPlain>(mA, mB, mC, mA1, mB1, p, num_sms, s);
-    case kWGrad: return launch_mode<kWGrad>(mA, mB, mC, mA1, mB1, p, num_sms, s);
+    case kRawGU: return launch_mode<kRawGU>(mA, mB, mC, p, num_sms, s);
+    case kDSwiGLU: return launch_mode<kDSwiGLU>(mA, mB, mC, p, num_sms, s);
+    case kDPlain: return launch_mode<kDPlain>(mA, mB, mC, p, num_sms, s);
+    case kWGrad: return launch_mode<kWGrad>(mA, mB, mC, p, num_sms, s);
   }
   return cudaErrorInvalidValue;
 }

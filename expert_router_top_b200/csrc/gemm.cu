@@ -100,12 +100,8 @@ struct KParams {
   const uint8_t* gsrc;    // gathered A: the token rows (hidden), and their stride in bytes
   int64_t gsrc_stride;
   int32_t K;              // valid K columns (gathered A: the rest of the last block reads 0)
-  // A second row segment sharing the tile sweep (plain A only): its expert offsets [E+1]
-  // (nullptr: one segment) and output rows.
-  const int32_t* offsets1;
-  __nv_bfloat16* out1;
-  int64_t gsrc_rows;             // checks build: rows of the gathered source
-  int64_t out_rows0, out_rows1;  // checks build: rows of out and out1
+  int64_t gsrc_rows;  // checks build: rows of the gathered source
+  int64_t out_rows;   // checks build: rows of out
 };
 
 template <int kStages>
@@ -134,7 +130,7 @@ static_assert(sizeof(SmemCtl<MOE_GEMM_STAGES>) <= kCtlBytes, "control block");
 // free of bank conflicts within each 8-lane phase.
 constexpr int kEpiRowBytes = 80;
 constexpr int kEpiWarpBytes = 32 * kEpiRowBytes;
-constexpr size_t kTablesBytes = (3 * (kMaxE + 1) * sizeof(int32_t) + 15) & ~size_t(15);
+constexpr size_t kTablesBytes = (2 * (kMaxE + 1) * sizeof(int32_t) + 15) & ~size_t(15);
 
 template <bool kPair>
 constexpr size_t smem_bytes() {
@@ -142,18 +138,16 @@ constexpr size_t smem_bytes() {
          kTablesBytes + (MOE_GEMM_EPI_STAGE ? 4 * kEpiWarpBytes : 0);
 }
 
-// A tile: expert e, column tile n, row tile m over the expert's rows of both segments
-// (segment 0's row tiles first), i.e. row tile ml of segment seg.
+// A tile: expert e, column tile n, row tile m of the expert's rows.
 struct Tile {
-  int32_t e, n, m, seg, ml;
+  int32_t e, n, m;
 };
 
 __device__ uint32_t g_range_flags;  // checks build: a row index outside its buffer was seen
 
 template <int kTileM>
 __device__ __forceinline__ Tile decode_tile(int32_t L, const int32_t* tile_start,
-                                            const int32_t* off, const int32_t* off1, int32_t E,
-                                            int32_t n_tiles) {
+                                            const int32_t* off, int32_t E, int32_t n_tiles) {
   // largest e with tile_start[e] <= L; that expert has at least one tile
   int32_t lo = 0, hi = E - 1;
   while (lo < hi) {
@@ -161,8 +155,7 @@ __device__ __forceinline__ Tile decode_tile(int32_t L, const int32_t* tile_start
     if (tile_start[mid] <= L) lo = mid;
     else hi = mid - 1;
   }
-  const int32_t mt0 = (off[lo + 1] - off[lo] + kTileM - 1) / kTileM;
-  const int32_t mt = mt0 + (off1 ? (off1[lo + 1] - off1[lo] + kTileM - 1) / kTileM : 0);
+  const int32_t mt = (off[lo + 1] - off[lo] + kTileM - 1) / kTileM;
   const int32_t local = L - tile_start[lo];
   Tile t;
   t.e = lo;
@@ -178,8 +171,6 @@ __device__ __forceinline__ Tile decode_tile(int32_t L, const int32_t* tile_start
   t.m = local / n_tiles;
   t.n = local - t.m * n_tiles;
 #endif
-  t.seg = t.m >= mt0 ? 1 : 0;
-  t.ml = t.m - (t.seg ? mt0 : 0);
   return t;
 }
 
@@ -229,7 +220,7 @@ __device__ __forceinline__ void store_block(const uint32_t (&packed)[16], uint8_
 // and report back to the leader.
 template <bool kSwiGLU, bool kPair, bool kGather>
 __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensorMap* tmB,
-                                          const CUtensorMap* tmA1, const KParams& p) {
+                                          const KParams& p) {
   using G = Geo<kPair>;
   constexpr int STAGES = G::kStages;
   static_assert(!(kGather && kPair), "gathered A rows are implemented for single CTAs");
@@ -241,8 +232,6 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   SmemCtl<STAGES>* ctl = reinterpret_cast<SmemCtl<STAGES>*>(smem + STAGES * G::kStageBytes);
   int32_t* off = reinterpret_cast<int32_t*>(smem + STAGES * G::kStageBytes + kCtlBytes);
   int32_t* tile_start = off + (kMaxE + 1);
-  int32_t* off1 = tile_start + (kMaxE + 1);
-  const int32_t* off1p = p.offsets1 ? off1 : nullptr;  // second row segment, if any
   uint8_t* epi_stage = smem + STAGES * G::kStageBytes + kCtlBytes + kTablesBytes;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -253,10 +242,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   const int32_t n_streams = kPair ? (int32_t)(gridDim.x >> 1) : (int32_t)gridDim.x;
 
   // ---- set-up: expert offsets, tile prefix, barriers, TMEM ----
-  for (int32_t i = threadIdx.x; i <= E; i += blockDim.x) {
-    off[i] = p.offsets[i];
-    if (p.offsets1) off1[i] = p.offsets1[i];
-  }
+  for (int32_t i = threadIdx.x; i <= E; i += blockDim.x) off[i] = p.offsets[i];
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       // gathered A: the weight producer's arrival plus one per A-gathering thread
@@ -291,9 +277,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
     const int32_t e0 = lane * per, e1 = min(E, e0 + per);
     int32_t sum = 0;
     auto tiles_of = [&](int32_t e) {
-      int32_t mt = (off[e + 1] - off[e] + G::kTileM - 1) / G::kTileM;
-      if (off1p) mt += (off1p[e + 1] - off1p[e] + G::kTileM - 1) / G::kTileM;
-      return mt * p.n_tiles;
+      return (off[e + 1] - off[e] + G::kTileM - 1) / G::kTileM * p.n_tiles;
     };
     for (int32_t e = e0; e < e1; ++e) sum += tiles_of(e);
     int32_t incl = sum;
@@ -327,8 +311,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       uint32_t armed = 0, armed_parity = 0;
       bool ok = true;
       for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
-        const Tile t = decode_tile<G::kTileM>(L, tile_start,
-                                              off, off1p, E, p.n_tiles);
+        const Tile t = decode_tile<G::kTileM>(L, tile_start, off, E, p.n_tiles);
         const int32_t brow = t.e * p.b_rows + t.n * (kSwiGLU ? BN / 2 : BN);
         for (int32_t kb = 0; kb < p.num_kb; ++kb) {
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort, p.status)) {
@@ -368,10 +351,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
     int32_t issued = 0, arrived = 0;
     bool ok = true;
     for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
-      const Tile t = decode_tile<G::kTileM>(L, tile_start,
-                                            off, off1p, E, p.n_tiles);
+      const Tile t = decode_tile<G::kTileM>(L, tile_start, off, E, p.n_tiles);
       const int32_t* gat = p.gather;  // gathered A has one row segment
-      const int32_t row0 = off[t.e] + t.ml * G::kTileM;
+      const int32_t row0 = off[t.e] + t.m * G::kTileM;
       const int32_t last = off[t.e + 1] - 1;  // rows past the expert re-read its last row
       const uint8_t* src[8];
 #pragma unroll
@@ -425,14 +407,13 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       bool ok = true;
       for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
         // A row and B row of tile L (of this CTA's tile stream)
-        const Tile t = decode_tile<G::kTileM>(L, tile_start, off, off1p, E, p.n_tiles);
-        const int32_t row0 =
-            (t.seg ? off1 : off)[t.e] + t.ml * G::kTileM + (int32_t)rank * kRowsPerCta;
+        const Tile t = decode_tile<G::kTileM>(L, tile_start, off, E, p.n_tiles);
+        const int32_t row0 = off[t.e] + t.m * G::kTileM + (int32_t)rank * kRowsPerCta;
         const int32_t brow =
             kSwiGLU  // pair: the even CTA stages the gate rows, the odd one the up rows
                 ? t.e * p.b_rows + t.n * (BN / 2) + (kPair ? (int32_t)rank * p.up_off : 0)
                 : t.e * p.b_rows + t.n * BN + (kPair ? (int32_t)rank * (BN / 2) : 0);
-        const CUtensorMap* mapA = t.seg ? tmA1 : tmA;
+        const CUtensorMap* mapA = tmA;
         for (int32_t kb = 0; kb < p.num_kb; ++kb) {
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort, p.status)) {
             ok = false;
@@ -534,12 +515,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       const uint32_t tphase = (it >> 1) & 1;
       if (!mbar_wait(&ctl->tfull[buf], tphase, abort, p.status)) break;
       tc_fence_after();
-      const Tile t = decode_tile<G::kTileM>(L, tile_start,
-                                            off, off1p, E, p.n_tiles);
-      const int32_t* offs = t.seg ? off1 : off;
-      __nv_bfloat16* out = t.seg ? p.out1 : p.out;
-      const int64_t out_rows = t.seg ? p.out_rows1 : p.out_rows0;
-      const int32_t first = t.ml * G::kTileM + (int32_t)rank * kRowsPerCta;  // in the expert
+      const Tile t = decode_tile<G::kTileM>(L, tile_start, off, E, p.n_tiles);
+      const int32_t* offs = off;
+      __nv_bfloat16* out = p.out;
+      const int64_t out_rows = p.out_rows;
+      const int32_t first = t.m * G::kTileM + (int32_t)rank * kRowsPerCta;  // in the expert
       const int32_t rows_valid = offs[t.e + 1] - offs[t.e] - first;
       const bool row_ok = r < rows_valid;
       const int64_t row_base = (int64_t)offs[t.e] + first;  // output row of TMEM lane 0
@@ -600,8 +580,8 @@ template <bool kSwiGLU, bool kGather>
 __global__ void __launch_bounds__(gemm_threads<kGather>(), 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
-                        const __grid_constant__ CUtensorMap tmA1, const KParams p) {
-  gemm_body<kSwiGLU, false, kGather>(&tmA, &tmB, &tmA1, p);
+                        const KParams p) {
+  gemm_body<kSwiGLU, false, kGather>(&tmA, &tmB, p);
 }
 
 // Launched with a cluster of 2 CTAs (cudaLaunchAttributeClusterDimension).
@@ -609,8 +589,8 @@ template <bool kSwiGLU>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmB,
-                             const __grid_constant__ CUtensorMap tmA1, const KParams p) {
-  gemm_body<kSwiGLU, true, false>(&tmA, &tmB, &tmA1, p);
+                             const KParams p) {
+  gemm_body<kSwiGLU, true, false>(&tmA, &tmB, p);
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -688,11 +668,10 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
     *err_detail = 1;
     return cudaErrorInvalidValue;
   }
-  CUtensorMap mA, mB, mA1;
+  CUtensorMap mA, mB;
   const int32_t bn = swiglu ? BN / 2 : BN;
   const bool gather = a.gather != nullptr;
-  const bool two = a.offsets1 != nullptr;  // a second row segment (the pair's other chunk)
-  if ((gather && (kPair || !swiglu || two)) || (two && kPair) || (two && (!a.out1 || !a.A1))) {
+  if (gather && (kPair || !swiglu)) {
     *err_detail = 1;
     return cudaErrorInvalidValue;
   }
@@ -701,9 +680,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
                                : make_map(&mA, a.A, a.rows, a.K, kRowsPerCta);
   const bool map_b_ok = make_map(&mB, a.B, (int64_t)a.E * a.b_rows, a.K,
                                  kPair ? BN / 2 : (swiglu ? BN / 2 : BN));
-  const bool map_a1_ok =
-      two && !gather ? make_map(&mA1, a.A1, a.rows1, a.K, kRowsPerCta) : (mA1 = mA, true);
-  if (!map_a_ok || !map_b_ok || !map_a1_ok) {
+  if (!map_a_ok || !map_b_ok) {
     *err_detail = 2;
     return cudaErrorInvalidValue;
   }
@@ -722,11 +699,8 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
   p.gsrc = static_cast<const uint8_t*>(a.gather_src);
   p.gsrc_stride = (int64_t)a.K * 2;
   p.gsrc_rows = a.gather_src_rows;
-  p.out_rows0 = a.rows;
-  p.out_rows1 = a.rows1;
+  p.out_rows = a.rows;
   p.K = a.K;
-  p.offsets1 = two ? a.offsets1 : nullptr;
-  p.out1 = two ? static_cast<__nv_bfloat16*>(a.out1) : nullptr;
   constexpr size_t smem = smem_bytes<kPair>();
   cudaError_t e;
   if (kPair) {
@@ -758,7 +732,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
     }
     const int streams = (int)(a.total_tiles < mp ? a.total_tiles : mp);
     cfg.gridDim = dim3(2 * streams, 1, 1);
-    e = cudaLaunchKernelEx(&cfg, k, mA, mB, mA1, p);
+    e = cudaLaunchKernelEx(&cfg, k, mA, mB, p);
     if (e != cudaSuccess) return e;
   } else {
     auto k = gather ? grouped_gemm_kernel<true, true>
@@ -766,8 +740,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int streams = (int)(a.total_tiles < num_sms ? a.total_tiles : num_sms);
-    k<<<streams, gather ? gemm_threads<true>() : gemm_threads<false>(), smem, s>>>(mA, mB, mA1,
-                                                                                     p);
+    k<<<streams, gather ? gemm_threads<true>() : gemm_threads<false>(), smem, s>>>(mA, mB, p);
   }
   return cudaGetLastError();
 }

@@ -72,14 +72,6 @@ struct GemmArgs {
   const int32_t* gather = nullptr;
   const void* gather_src = nullptr;
   int64_t gather_src_rows = 0;
-  // A second row segment in the same tile sweep (the other chunk of a pair: the weights of
-  // each expert tile are then fetched once for both; plain A only): its expert offsets (dev
-  // [E+1]; nullptr = one segment), A rows (A1 [rows1][K]) and output rows.  total_tiles
-  // then counts the tiles of both segments.
-  const int32_t* offsets1 = nullptr;
-  const void* A1 = nullptr;
-  int64_t rows1 = 0;
-  void* out1 = nullptr;
 };
 
 // 2-D bf16 tensor map over a row-major [rows][cols] matrix: boxes of box_rows x 64 columns,
@@ -123,23 +115,9 @@ struct BwdGemmArgs {
   void* out1;
   const void* aux;
   float* acc;                  // kBwdWGrad: [E][M][N] fp32 gradient
-  const int32_t* first;        // kBwdWGrad: dev [E] first chunk with rows of each expert
-  int32_t chunk;               // kBwdWGrad: this chunk (store where first is this launch's
-                               // chunk or its pair's second chunk, else add)
-  // kBwdWGrad over a pair of chunks (null offsets1: one chunk): the second chunk's operands,
-  // rows, padded offsets (dev [E+1]) and padded rows per expert (host [E])
-  const void* A1;
-  int64_t A1_rows;
-  const void* B1;
-  int64_t B1_rows;
-  const int32_t* offsets1;
-  const int32_t* rows_pad_host1;
-  // row-grouped modes over a pair of chunks: the second chunk's rows are a second row
-  // segment of the same tile sweep (A1 its A rows; out0b / out1b / auxb its outputs and
-  // saved g|u rows), so each weight tile is fetched once for both chunks
-  void* out0b;
-  void* out1b;
-  const void* auxb;
+  const int32_t* first;        // kBwdWGrad: dev [E] first unit (pair of chunks) with rows of
+                               // each expert
+  int32_t chunk;               // kBwdWGrad: this unit (store where first is this unit, else add)
   uint32_t* status;
 };
 

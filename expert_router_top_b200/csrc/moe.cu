@@ -224,8 +224,8 @@ struct DeviceCtx {
               ev_copy_join = nullptr;
   // backward pipeline: permuted rows ready (per X slot), recomputed Y ready, dY ready, dX
   // ready, d_hidden rows summed (per buffer), all of a chunk's GEMMs done (per X slot)
-  cudaEvent_t ev_bp[3] = {}, ev_bf[2] = {}, ev_bdy[2] = {}, ev_bdx[2] = {}, ev_bsum[2] = {},
-              ev_bw[3] = {};
+  cudaEvent_t ev_bp[2] = {}, ev_bf[2] = {}, ev_bdy[2] = {}, ev_bdx[1] = {}, ev_bsum[1] = {},
+              ev_bw[2] = {};
   int32_t* host_stage = nullptr;
   size_t host_stage_bytes = 0;
 };
@@ -263,16 +263,15 @@ moe_status_t get_ctx(DeviceCtx** out) {
           cudaEventCreateWithFlags(&c.ev_out_free[b], fl) != cudaSuccess)
         return MOE_ERR_CUDA;
     if (cudaEventCreateWithFlags(&c.ev_copy_join, fl) != cudaSuccess) return MOE_ERR_CUDA;
-    for (int b = 0; b < 3; ++b)
-      if (cudaEventCreateWithFlags(&c.ev_bp[b], fl) != cudaSuccess ||
-          cudaEventCreateWithFlags(&c.ev_bw[b], fl) != cudaSuccess)
-        return MOE_ERR_CUDA;
     for (int b = 0; b < 2; ++b)
-      if (cudaEventCreateWithFlags(&c.ev_bf[b], fl) != cudaSuccess ||
-          cudaEventCreateWithFlags(&c.ev_bdy[b], fl) != cudaSuccess ||
-          cudaEventCreateWithFlags(&c.ev_bdx[b], fl) != cudaSuccess ||
-          cudaEventCreateWithFlags(&c.ev_bsum[b], fl) != cudaSuccess)
+      if (cudaEventCreateWithFlags(&c.ev_bp[b], fl) != cudaSuccess ||
+          cudaEventCreateWithFlags(&c.ev_bw[b], fl) != cudaSuccess ||
+          cudaEventCreateWithFlags(&c.ev_bf[b], fl) != cudaSuccess ||
+          cudaEventCreateWithFlags(&c.ev_bdy[b], fl) != cudaSuccess)
         return MOE_ERR_CUDA;
+    if (cudaEventCreateWithFlags(&c.ev_bdx[0], fl) != cudaSuccess ||
+        cudaEventCreateWithFlags(&c.ev_bsum[0], fl) != cudaSuccess)
+      return MOE_ERR_CUDA;
     c.ready = true;
   }
   *out = &c;
@@ -405,32 +404,14 @@ int64_t active_experts(const int32_t* counts, int32_t E) {
 }
 
 
-// The second row segment of a grouped GEMM that serves both chunks of a pair (plain A).
-struct Seg1 {
-  const void* A = nullptr;           // [rows][K]
-  int64_t rows = 0;
-  const int32_t* offsets = nullptr;  // dev [E+1]
-  const int32_t* counts = nullptr;   // host [E]
-  void* out = nullptr;
-};
-
 moe_status_t gemm_call(const void* A, int64_t rows, const void* B, void* out,
                        const int32_t* offsets_dev, const int32_t* counts_host, int32_t E,
                        int32_t K, int32_t out_cols, int32_t b_rows, bool swiglu,
                        uint32_t* status, int num_sms, cudaStream_t s,
                        const int32_t* gather = nullptr, const void* gather_src = nullptr,
-                       int64_t gather_src_rows = 0, const Seg1* seg1 = nullptr) {
+                       int64_t gather_src_rows = 0) {
   GemmArgs g;
-  int64_t rows_all = rows, active = active_experts(counts_host, E);
-  if (seg1) {
-    g.offsets1 = seg1->offsets;
-    g.A1 = seg1->A;
-    g.rows1 = seg1->rows;
-    g.out1 = seg1->out;
-    rows_all += seg1->rows;
-    active = 0;  // experts with rows in either segment
-    for (int32_t e = 0; e < E; ++e) active += (counts_host[e] + seg1->counts[e]) > 0;
-  }
+  const int64_t active = active_experts(counts_host, E);
   g.gather = gather;
   g.gather_src = gather_src;
   g.gather_src_rows = gather_src_rows;
@@ -443,12 +424,11 @@ moe_status_t gemm_call(const void* A, int64_t rows, const void* B, void* out,
   g.K = K;
   g.out_cols = out_cols;
   g.b_rows = b_rows;
-  g.total_tiles = gemm_total_tiles(counts_host, E, out_cols, swiglu) +
-                  (seg1 ? gemm_total_tiles(seg1->counts, E, out_cols, swiglu) : 0);
+  g.total_tiles = gemm_total_tiles(counts_host, E, out_cols, swiglu);
   g.status = status;
   if (g.total_tiles == 0) return MOE_OK;
   int detail = 0;
-  ProfScope ps(swiglu ? MOE_KERNEL_GATEUP : MOE_KERNEL_DOWN, s, rows_all, active, 1);
+  ProfScope ps(swiglu ? MOE_KERNEL_GATEUP : MOE_KERNEL_DOWN, s, rows, active, 1);
   cudaError_t e = launch_grouped_gemm(g, swiglu, num_sms, s, &detail);
   if (e != cudaSuccess) return detail == 1 ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
   return MOE_OK;
@@ -915,47 +895,48 @@ moe_status_t moe_forward_host_impl(const moe_shape_t* shape, const void* hidden_
 namespace {
 
 struct BwdLayout {
+  Dims unit;    // the pairs of chunks (2m, 2m+1), each a unit of the pipeline
   Layout meta;  // metadata regions (status/counts/splits, offsets, histograms, dst, src)
   size_t offp, first, dstp, total;
-  int nx, nb;  // X slots (up to 3) and buffer sets of the other rows
-  size_t xp[3], gu[2], act[2], ydx[2], dy[2];  // gu later holds [dg du] in place
+  int nx;  // X buffers: one per pair in flight (up to 2)
+  size_t xp[2], gu, act, ydx, dy;  // gu later holds [dg du] in place; ydx holds Y, then dX
   int64_t rows_cap;
 };
 
-// Every chunk's rows, padded per expert to a multiple of 64, fit in rows_cap rows.  The
-// pipeline keeps chunk c's permuted rows in X slot c % 3 (they are read until its pair's
-// weight-gradient GEMM; the next pair's first chunk is permuted meanwhile) and its other row
-// buffers in set c % 2.  The SwiGLU backward overwrites the saved [g u] rows with [dg du]
-// (each epilogue thread has read a block before any lane stores it), so one buffer holds
-// both.
+// The backward runs per pair of chunks: the metadata is taken per pair, so each expert's
+// rows are contiguous over both chunks and padded once per pair to a multiple of 64; every
+// pair's rows fit in rows_cap rows.  The pipeline keeps pair m's permuted rows in X buffer
+// m % 2 (the next pair is permuted while pair m computes; X is read until the pair's
+// weight-gradient GEMM) and its other rows in one buffer set.  The SwiGLU backward
+// overwrites the saved [g u] rows with [dg du] (each epilogue thread has read a block before
+// any lane stores it), so one buffer holds both.
 BwdLayout make_bwd_layout(const Dims& d, int32_t H, int32_t I) {
   BwdLayout B{};
-  B.meta = make_layout(d, 8, 8, false, true, true);
+  B.unit = pair_dims(d);
+  const Dims& u = B.unit;
+  B.meta = make_layout(u, 8, 8, false, true, true);
   size_t o = B.meta.total;
-  B.rows_cap = d.t_chunk * d.k + (int64_t)d.E * (bwd_pad_rows() - 1);
+  B.rows_cap = u.t_chunk * u.k + (int64_t)u.E * (bwd_pad_rows() - 1);
   B.offp = o;
-  o += al(sizeof(int32_t) * (size_t)d.n * (d.E + 1));
+  o += al(sizeof(int32_t) * (size_t)u.n * (u.E + 1));
   B.first = o;
-  o += al(sizeof(int32_t) * (size_t)d.E);
+  o += al(sizeof(int32_t) * (size_t)u.E);
   B.dstp = o;
-  o += al(sizeof(int32_t) * (size_t)(d.T * d.k));
+  o += al(sizeof(int32_t) * (size_t)(u.T * u.k));
   const size_t R = (size_t)B.rows_cap;
-  B.nx = d.n >= 3 ? 3 : d.n;
-  B.nb = d.n >= 2 ? 2 : 1;
+  B.nx = u.n >= 2 ? 2 : 1;
   for (int b = 0; b < B.nx; ++b) {
     B.xp[b] = o;
     o += al(2 * R * H);
   }
-  for (int b = 0; b < B.nb; ++b) {
-    B.gu[b] = o;
-    o += al(2 * R * 2 * I);
-    B.act[b] = o;
-    o += al(2 * R * I);
-    B.ydx[b] = o;  // recomputed Y rows, later dX rows
-    o += al(2 * R * H);
-    B.dy[b] = o;
-    o += al(2 * R * H);
-  }
+  B.gu = o;
+  o += al(2 * R * 2 * I);
+  B.act = o;
+  o += al(2 * R * I);
+  B.ydx = o;
+  o += al(2 * R * H);
+  B.dy = o;
+  o += al(2 * R * H);
   B.total = o;
   return B;
 }
@@ -1012,21 +993,22 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
   int32_t* dst = reinterpret_cast<int32_t*>(ws + B.meta.dst);
   int32_t* src = reinterpret_cast<int32_t*>(ws + B.meta.src);
   uint32_t* dev_status = reinterpret_cast<uint32_t*>(ws + B.meta.packed);
-  if ((st = run_metadata(d, top_k_index, ws, B.meta, dst, src, s)) != MOE_OK) return st;
+  const Dims& u = B.unit;  // unit m = the pair of chunks (2m, 2m+1)
+  if ((st = run_metadata(u, top_k_index, ws, B.meta, dst, src, s)) != MOE_OK) return st;
   if ((st = fetch_packed(ctx, ws, B.meta, s)) != MOE_OK) return st;
   std::vector<int32_t> counts(ctx->host_stage + kStatusWords,
-                              ctx->host_stage + kStatusWords + (size_t)d.n * d.E);
+                              ctx->host_stage + kStatusWords + (size_t)u.n * E);
   const int32_t* counts_dev = reinterpret_cast<const int32_t*>(ws + B.meta.packed) + kStatusWords;
   int32_t* offp = reinterpret_cast<int32_t*>(ws + B.offp);
   int32_t* first = reinterpret_cast<int32_t*>(ws + B.first);
   int32_t* dstp = reinterpret_cast<int32_t*>(ws + B.dstp);
-  if (launch_pad_offsets(counts_dev, E, d.n, offp, first, s) != cudaSuccess) return MOE_ERR_CUDA;
-  // The weight-gradient GEMM of an expert's first chunk with rows stores its tiles and later
-  // chunks add to them, so only experts that no chunk routes to are zeroed here (runs of
+  if (launch_pad_offsets(counts_dev, E, u.n, offp, first, s) != cudaSuccess) return MOE_ERR_CUDA;
+  // The weight-gradient GEMM of an expert's first pair with rows stores its tiles and later
+  // pairs add to them, so only experts that no chunk routes to are zeroed here (runs of
   // consecutive such experts take one memset per gradient).
   std::vector<char> routed((size_t)E, 0);
-  for (int c = 0; c < d.n; ++c)
-    for (int32_t e = 0; e < E; ++e) routed[e] |= counts[(size_t)c * E + e] > 0;
+  for (int m = 0; m < u.n; ++m)
+    for (int32_t e = 0; e < E; ++e) routed[e] |= counts[(size_t)m * E + e] > 0;
   for (int32_t e0 = 0; e0 < E;) {
     if (routed[e0]) {
       ++e0;
@@ -1037,43 +1019,48 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
     if (!zero_experts(e0, e1)) return MOE_ERR_CUDA;
     e0 = e1;
   }
-  const std::vector<int64_t> bounds = dims_bounds(d);
-  int n_live = 0;  // chunks with tokens; only trailing chunks can be empty
-  while (n_live < d.n && bounds[n_live + 1] > bounds[n_live]) ++n_live;
+  const std::vector<int64_t> bounds = dims_bounds(u);
+  int n_live = 0;  // pairs with tokens; only trailing ones can be empty
+  while (n_live < u.n && bounds[n_live + 1] > bounds[n_live]) ++n_live;
   const int pad = bwd_pad_rows();
   const uint16_t* hid = static_cast<const uint16_t*>(hidden);
   const uint16_t* dout = static_cast<const uint16_t*>(d_out);
   uint16_t* dx_out = static_cast<uint16_t*>(d_hidden);
   cudaStream_t sg = ctx->side;
-  // padded rows per expert and their total, per chunk
-  std::vector<int32_t> rows_pad((size_t)d.n * E);
-  std::vector<int64_t> R((size_t)d.n, 0);
-  for (int c = 0; c < d.n; ++c)
+  // padded rows per expert and their total, per pair
+  std::vector<int32_t> rows_pad((size_t)u.n * E);
+  std::vector<int64_t> R((size_t)u.n, 0);
+  for (int m = 0; m < u.n; ++m)
     for (int32_t e = 0; e < E; ++e) {
-      const int32_t v = (counts[(size_t)c * E + e] + pad - 1) / pad * pad;
-      rows_pad[(size_t)c * E + e] = v;
-      R[c] += v;
+      const int32_t v = (counts[(size_t)m * E + e] + pad - 1) / pad * pad;
+      rows_pad[(size_t)m * E + e] = v;
+      R[m] += v;
     }
-  auto x_of = [&](int c) { return ws + B.xp[c % B.nx]; };
-  auto buf = [&](const size_t(&a)[2], int c) { return ws + a[c % B.nb]; };
-  auto off_c = [&](int c) {
-    return reinterpret_cast<const int32_t*>(ws + B.meta.offsets) + (size_t)c * (E + 1);
+  auto x_of = [&](int m) { return ws + B.xp[m % B.nx]; };
+  uint8_t* const gu = ws + B.gu;    // [g u], later [dg du]
+  uint8_t* const act = ws + B.act;  // h
+  uint8_t* const ydx = ws + B.ydx;  // Y, later dX
+  uint8_t* const dy = ws + B.dy;    // dY
+  auto off_m = [&](int m) {
+    return reinterpret_cast<const int32_t*>(ws + B.meta.offsets) + (size_t)m * (E + 1);
   };
-  auto offp_c = [&](int c) -> const int32_t* { return offp + (size_t)c * (E + 1); };
-  auto dstp_c = [&](int c) { return dstp + bounds[c] * k; };
-  auto len = [&](int c) { return bounds[c + 1] - bounds[c]; };
+  auto offp_m = [&](int m) -> const int32_t* { return offp + (size_t)m * (E + 1); };
+  auto rows_pad_m = [&](int m) { return rows_pad.data() + (size_t)m * E; };
+  auto dstp_m = [&](int m) { return dstp + bounds[m] * k; };
+  auto len = [&](int m) { return bounds[m + 1] - bounds[m]; };
   auto ok = [](cudaError_t e) { return e == cudaSuccess; };
 
-  // P(c), stream M: padded permute of the chunk's rows into X slot c % 3 (zero pad rows)
-  auto P = [&](int c) -> moe_status_t {
-    if (c >= 3 && !ok(cudaStreamWaitEvent(s, ctx->ev_bw[c % 3], 0))) return MOE_ERR_CUDA;
-    ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(c) * k, 0, 2);
-    if (!ok(cudaMemsetAsync(x_of(c), 0, 2 * (size_t)R[c] * H, s)) ||
-        !ok(launch_pad_rows(top_k_index + bounds[c] * k, dst + bounds[c] * k, off_c(c), offp_c(c),
-                            len(c) * k, dstp_c(c), B.rows_cap, s)) ||
-        !ok(launch_permute(hid + bounds[c] * H, dstp_c(c), len(c), H, k, x_of(c), B.rows_cap,
+  // P(m), stream M: padded permute of the pair's rows into X buffer m % 2 (zero pad rows),
+  // once W(m-2) is done with that buffer
+  auto P = [&](int m) -> moe_status_t {
+    if (m >= 2 && !ok(cudaStreamWaitEvent(s, ctx->ev_bw[m % 2], 0))) return MOE_ERR_CUDA;
+    ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(m) * k, 0, 2);
+    if (!ok(cudaMemsetAsync(x_of(m), 0, 2 * (size_t)R[m] * H, s)) ||
+        !ok(launch_pad_rows(top_k_index + bounds[m] * k, dst + bounds[m] * k, off_m(m),
+                            offp_m(m), len(m) * k, dstp_m(m), B.rows_cap, s)) ||
+        !ok(launch_permute(hid + bounds[m] * H, dstp_m(m), len(m), H, k, x_of(m), B.rows_cap,
                            s)) ||
-        !ok(cudaEventRecord(ctx->ev_bp[c % 3], s)))
+        !ok(cudaEventRecord(ctx->ev_bp[m % 2], s)))
       return MOE_ERR_CUDA;
     return MOE_OK;
   };
@@ -1082,186 +1069,124 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
   g0.I = I;
   g0.status = dev_status;
   g0.first = first;
-  // The pair (c, c1): c1 = c + 1, or c1 = c for the last chunk of an odd count.  Every GEMM
-  // of a pair is one tile sweep over both chunks' rows (the second chunk a second row
-  // segment, or for the weight gradients more K), so each weight tile is fetched once per
-  // pair.
-  auto rows_both = [&](int c, int c1) { return R[c] + (c1 > c ? R[c1] : 0); };
-  auto active_both = [&](int c, int c1) {
-    int64_t a = 0;
-    for (int32_t e = 0; e < E; ++e)
-      a += (counts[(size_t)c * E + e] + (c1 > c ? counts[(size_t)c1 * E + e] : 0)) > 0;
-    return a;
+  // A GEMM over the pair's padded rows: one tile sweep per pair, so each weight tile is
+  // fetched once for both chunks, and a row tile may hold rows of both.
+  auto rowwise = [&](int m, int mode) {
+    BwdGemmArgs g = g0;
+    g.mode = mode;
+    g.offsets = offp_m(m);
+    g.rows_pad_host = rows_pad_m(m);
+    g.chunk = m;
+    return g;
   };
-  auto launch_pair = [&](int kind, const BwdGemmArgs& a, int c, int c1) {
-    ProfScope ps(kind, sg, rows_both(c, c1), active_both(c, c1), 1);
+  auto launch_unit = [&](int kind, const BwdGemmArgs& a, int m) {
+    ProfScope ps(kind, sg, R[m], active_experts(rows_pad_m(m), E), 1);
     return launch_bwd_gemm(a, ctx->num_sms, sg);
   };
-  // the second chunk of a pair as a row segment of a row-grouped mode
-  auto seg1 = [&](BwdGemmArgs& g, int c1, const void* A1, void* o0, void* o1, const void* aux) {
-    g.offsets1 = offp_c(c1);
-    g.rows_pad_host1 = rows_pad.data() + (size_t)c1 * E;
-    g.A1 = A1;
-    g.A1_rows = R[c1];
-    g.out0b = o0;
-    g.out1b = o1;
-    g.auxb = aux;
-  };
-  // F(c, c1), stream G: recompute [g u], h and Y = h W_down^T on the padded rows
-  auto F = [&](int c, int c1) -> moe_status_t {
-    for (int x = c; x <= c1; ++x) {
-      if (!ok(cudaStreamWaitEvent(sg, ctx->ev_bp[x % 3], 0))) return MOE_ERR_CUDA;
-      if (x >= 2 && !ok(cudaStreamWaitEvent(sg, ctx->ev_bsum[x % 2], 0))) return MOE_ERR_CUDA;
-    }
-    BwdGemmArgs g = g0;
-    g.offsets = offp_c(c);
-    g.rows_pad_host = rows_pad.data() + (size_t)c * E;
-    g.chunk = c;
-    g.mode = kBwdRawGU;
-    g.A = x_of(c), g.A_rows = R[c], g.A_cols = H;
+  // F(m), stream G: recompute [g u], h and Y = h W_down^T on the padded rows, once P(m) is
+  // done and S(m-1) has read the previous pair's dX rows
+  auto F = [&](int m) -> moe_status_t {
+    if (!ok(cudaStreamWaitEvent(sg, ctx->ev_bp[m % 2], 0))) return MOE_ERR_CUDA;
+    if (m >= 1 && !ok(cudaStreamWaitEvent(sg, ctx->ev_bsum[0], 0))) return MOE_ERR_CUDA;
+    BwdGemmArgs g = rowwise(m, kBwdRawGU);
+    g.A = x_of(m), g.A_rows = R[m], g.A_cols = H;
     g.B = W_gate_up, g.B_rows = (int64_t)E * 2 * I, g.B_cols = H;
-    g.N = 2 * I, g.K = H, g.b_rows = 2 * I, g.out0 = buf(B.gu, c), g.out1 = buf(B.act, c);
-    if (c1 > c) seg1(g, c1, x_of(c1), buf(B.gu, c1), buf(B.act, c1), nullptr);
-    if (!ok(launch_pair(MOE_KERNEL_BWD_GATEUP, g, c, c1))) return MOE_ERR_CUDA;
-    Seg1 d1;
-    if (c1 > c) {
-      d1.A = buf(B.act, c1);
-      d1.rows = R[c1];
-      d1.offsets = offp_c(c1);
-      d1.counts = rows_pad.data() + (size_t)c1 * E;
-      d1.out = buf(B.ydx, c1);
-    }
-    moe_status_t s2 = gemm_call(buf(B.act, c), R[c], W_down, buf(B.ydx, c), offp_c(c),
-                                rows_pad.data() + (size_t)c * E, E, I, H, H, false, dev_status,
-                                ctx->num_sms, sg, nullptr, nullptr, 0, c1 > c ? &d1 : nullptr);
+    g.N = 2 * I, g.K = H, g.b_rows = 2 * I, g.out0 = gu, g.out1 = act;
+    if (!ok(launch_unit(MOE_KERNEL_BWD_GATEUP, g, m))) return MOE_ERR_CUDA;
+    moe_status_t s2 = gemm_call(act, R[m], W_down, ydx, offp_m(m), rows_pad_m(m), E, I, H, H,
+                                false, dev_status, ctx->num_sms, sg);
     if (s2 != MOE_OK) return s2;
     return ok(cudaEventRecord(ctx->ev_bf[0], sg)) ? MOE_OK : MOE_ERR_CUDA;
   };
-  // DYS(c), stream M: dY = w dout into the chunk's padded rows (zero pad rows); it needs
+  // DYS(m), stream M: dY = w dout into the pair's padded rows (zero pad rows); it needs
   // nothing from the recompute, only the previous pair's weight gradients to be done with
-  // this buffer set
-  auto DYS = [&](int c) -> moe_status_t {
-    ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(c) * k, 0, 1);
-    if (!ok(cudaMemsetAsync(buf(B.dy, c), 0, 2 * (size_t)R[c] * H, s)) ||
-        !ok(launch_dy_scatter(dout + bounds[c] * H, dstp_c(c), top_k_weights + bounds[c] * k,
-                              len(c), H, k, buf(B.dy, c), B.rows_cap, s)) ||
+  // the dY rows
+  auto DYS = [&](int m) -> moe_status_t {
+    ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(m) * k, 0, 1);
+    if (!ok(cudaMemsetAsync(dy, 0, 2 * (size_t)R[m] * H, s)) ||
+        !ok(launch_dy_scatter(dout + bounds[m] * H, dstp_m(m), top_k_weights + bounds[m] * k,
+                              len(m), H, k, dy, B.rows_cap, s)) ||
         !ok(cudaEventRecord(ctx->ev_bdy[0], s)))
       return MOE_ERR_CUDA;
     return MOE_OK;
   };
-  // DW(c), stream M: d_weights = <dout, Y> with the recomputed Y rows
-  auto DW = [&](int c) -> moe_status_t {
+  // DW(m), stream M: d_weights = <dout, Y> with the recomputed Y rows
+  auto DW = [&](int m) -> moe_status_t {
     if (!ok(cudaStreamWaitEvent(s, ctx->ev_bf[0], 0))) return MOE_ERR_CUDA;
-    ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(c) * k, 0, 1);
-    if (!ok(launch_dw_dot(dout + bounds[c] * H, buf(B.ydx, c), dstp_c(c), len(c), H, k,
-                          d_weights + bounds[c] * k, B.rows_cap, s)) ||
+    ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(m) * k, 0, 1);
+    if (!ok(launch_dw_dot(dout + bounds[m] * H, ydx, dstp_m(m), len(m), H, k,
+                          d_weights + bounds[m] * k, B.rows_cap, s)) ||
         !ok(cudaEventRecord(ctx->ev_bdy[1], s)))
       return MOE_ERR_CUDA;
     return MOE_OK;
   };
-  // Bd(c, c1), stream G: dh with the SwiGLU backward, then dX
-  auto Bd = [&](int c, int c1) -> moe_status_t {
+  // Bd(m), stream G: dh with the SwiGLU backward, then dX
+  auto Bd = [&](int m) -> moe_status_t {
     if (!ok(cudaStreamWaitEvent(sg, ctx->ev_bdy[0], 0))) return MOE_ERR_CUDA;  // dY rows
-    BwdGemmArgs g = g0;
-    g.offsets = offp_c(c);
-    g.rows_pad_host = rows_pad.data() + (size_t)c * E;
-    g.chunk = c;
-    g.mode = kBwdDSwiGLU;
-    g.A = buf(B.dy, c), g.A_rows = R[c], g.A_cols = H;
+    BwdGemmArgs g = rowwise(m, kBwdDSwiGLU);
+    g.A = dy, g.A_rows = R[m], g.A_cols = H;
     g.B = W_down, g.B_rows = (int64_t)E * H, g.B_cols = I;
-    g.N = I, g.K = H, g.b_rows = H, g.out0 = buf(B.gu, c), g.aux = buf(B.gu, c);  // in place
-    if (c1 > c) seg1(g, c1, buf(B.dy, c1), buf(B.gu, c1), nullptr, buf(B.gu, c1));
-    if (!ok(launch_pair(MOE_KERNEL_BWD_DSWIGLU, g, c, c1))) return MOE_ERR_CUDA;
+    g.N = I, g.K = H, g.b_rows = H, g.out0 = gu, g.aux = gu;  // in place
+    if (!ok(launch_unit(MOE_KERNEL_BWD_DSWIGLU, g, m))) return MOE_ERR_CUDA;
     // dX overwrites the Y rows: d_weights must have read them
     if (!ok(cudaStreamWaitEvent(sg, ctx->ev_bdy[1], 0))) return MOE_ERR_CUDA;
-    g = g0;
-    g.offsets = offp_c(c);
-    g.rows_pad_host = rows_pad.data() + (size_t)c * E;
-    g.chunk = c;
-    g.mode = kBwdDPlain;
-    g.A = buf(B.gu, c), g.A_rows = R[c], g.A_cols = 2 * I;
+    g = rowwise(m, kBwdDPlain);
+    g.A = gu, g.A_rows = R[m], g.A_cols = 2 * I;
     g.B = W_gate_up, g.B_rows = (int64_t)E * 2 * I, g.B_cols = H;
-    g.N = H, g.K = 2 * I, g.b_rows = 2 * I, g.out0 = buf(B.ydx, c);
-    if (c1 > c) seg1(g, c1, buf(B.gu, c1), buf(B.ydx, c1), nullptr, nullptr);
-    if (!ok(launch_pair(MOE_KERNEL_BWD_DX, g, c, c1)) ||
-        !ok(cudaEventRecord(ctx->ev_bdx[0], sg)))
+    g.N = H, g.K = 2 * I, g.b_rows = 2 * I, g.out0 = ydx;
+    if (!ok(launch_unit(MOE_KERNEL_BWD_DX, g, m)) || !ok(cudaEventRecord(ctx->ev_bdx[0], sg)))
       return MOE_ERR_CUDA;
     return MOE_OK;
   };
-  // W(c, c1), stream G: both weight gradients, K over the rows of both chunks:
+  // W(m), stream G: both weight gradients, K over the pair's padded rows:
   //   dW_down[e] (+)= dY^T h ;  dW_gate_up[e] (+)= [dg du]^T X
   // An expert's first pair with rows stores; later pairs add.
-  auto W = [&](int c, int c1) -> moe_status_t {
-    BwdGemmArgs g = g0;
-    g.offsets = offp_c(c);
-    g.rows_pad_host = rows_pad.data() + (size_t)c * E;
-    g.chunk = c;
-    if (c1 > c) {
-      g.offsets1 = offp_c(c1);
-      g.rows_pad_host1 = rows_pad.data() + (size_t)c1 * E;
-      g.A1_rows = g.B1_rows = R[c1];
-    }
-    g.mode = kBwdWGrad;
-    g.A = buf(B.dy, c), g.A_rows = R[c], g.A_cols = H;
-    g.B = buf(B.act, c), g.B_rows = R[c], g.B_cols = I;
-    if (c1 > c) g.A1 = buf(B.dy, c1), g.B1 = buf(B.act, c1);
+  auto W = [&](int m) -> moe_status_t {
+    BwdGemmArgs g = rowwise(m, kBwdWGrad);
+    g.A = dy, g.A_rows = R[m], g.A_cols = H;
+    g.B = act, g.B_rows = R[m], g.B_cols = I;
     g.M = H, g.N = I, g.acc = dW_down, g.out0 = nullptr;
-    if (!ok(launch_pair(MOE_KERNEL_BWD_WGRAD, g, c, c1))) return MOE_ERR_CUDA;
-    g.A = buf(B.gu, c), g.A_rows = R[c], g.A_cols = 2 * I;  // [dg du]
-    g.B = x_of(c), g.B_rows = R[c], g.B_cols = H;
-    if (c1 > c) g.A1 = buf(B.gu, c1), g.B1 = x_of(c1);
+    if (!ok(launch_unit(MOE_KERNEL_BWD_WGRAD, g, m))) return MOE_ERR_CUDA;
+    g.A = gu, g.A_rows = R[m], g.A_cols = 2 * I;  // [dg du]
+    g.B = x_of(m), g.B_rows = R[m], g.B_cols = H;
     g.M = 2 * I, g.N = H, g.acc = dW_gate_up;
-    if (!ok(launch_pair(MOE_KERNEL_BWD_WGRAD, g, c, c1)) ||
-        !ok(cudaEventRecord(ctx->ev_bw[c % 3], sg)) ||
-        (c1 > c && !ok(cudaEventRecord(ctx->ev_bw[c1 % 3], sg))) ||
-        !ok(cudaEventRecord(ctx->ev_bf[1], sg)))
+    if (!ok(launch_unit(MOE_KERNEL_BWD_WGRAD, g, m)) ||
+        !ok(cudaEventRecord(ctx->ev_bw[m % 2], sg)) || !ok(cudaEventRecord(ctx->ev_bf[1], sg)))
       return MOE_ERR_CUDA;
     return MOE_OK;
   };
-  // S(c), stream M: d_hidden rows = sum over the k copies of dX
-  auto S = [&](int c) -> moe_status_t {
+  // S(m), stream M: d_hidden rows = sum over the k copies of dX
+  auto S = [&](int m) -> moe_status_t {
     if (!ok(cudaStreamWaitEvent(s, ctx->ev_bdx[0], 0))) return MOE_ERR_CUDA;
-    ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(c) * k, 0, 1);
-    if (!ok(launch_sum_rows(buf(B.ydx, c), dstp_c(c), len(c), H, k, dx_out + bounds[c] * H,
-                            B.rows_cap, s)) ||
-        !ok(cudaEventRecord(ctx->ev_bsum[c % 2], s)))
+    ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(m) * k, 0, 1);
+    if (!ok(launch_sum_rows(ydx, dstp_m(m), len(m), H, k, dx_out + bounds[m] * H, B.rows_cap,
+                            s)) ||
+        !ok(cudaEventRecord(ctx->ev_bsum[0], s)))
       return MOE_ERR_CUDA;
     return MOE_OK;
   };
 
-  // The mirrored pair pipeline over pairs (c, c1) = (2m, 2m+1), every GEMM one sweep over
-  // both chunks of the pair:
-  //   G: F(pair m) DSwiGLU(m) DX(m) W(m) F(pair m+1) ...
-  //   M: P(c) P(c1) DYS(c) DYS(c1) | DW(c) DW(c1) P(c+2) S(c) S(c1) P(c+3) DYS(c+2) ...
+  // The mirrored pair pipeline, one unit per pair of chunks:
+  //   G: F(0) DSwiGLU(0) DX(0) W(0) F(1) DSwiGLU(1) ...
+  //   M: P(0) DYS(0) | DW(0) P(1) S(0) DYS(1) | DW(1) P(2) S(1) ...
   // dY needs nothing from the recompute, so it is scattered while F runs; d_weights reads
   // the recomputed Y beside the SwiGLU-backward GEMM, before dX overwrites those rows; the
-  // next pair's first permute runs beside the dX and weight-gradient GEMMs, its second (in
-  // chunk c's X slot) and its dY scatter once W(m) is done with those buffers.  Host
-  // enqueue order keeps each event wait on the record it is meant for.
+  // next pair is permuted beside the dX and weight-gradient GEMMs, and its dY is scattered
+  // once W(m) is done with the dY rows.  Host enqueue order keeps each event wait on the
+  // record it is meant for.
   if (!ok(cudaEventRecord(ctx->ev_start, s)) || !ok(cudaStreamWaitEvent(sg, ctx->ev_start, 0)))
     return MOE_ERR_CUDA;
   if (n_live > 0) {
-    auto pair_end = [&](int c) { return c + 1 < n_live ? c + 1 : c; };
-    if ((st = P(0)) != MOE_OK) return st;
-    if (n_live > 1 && (st = P(1)) != MOE_OK) return st;
-    if ((st = F(0, pair_end(0))) != MOE_OK) return st;
-    if ((st = DYS(0)) != MOE_OK || (n_live > 1 && (st = DYS(1)) != MOE_OK)) return st;
-    for (int c = 0; c < n_live; c += 2) {
-      const int c1 = pair_end(c);
-      NvtxRange pr("moe_backward pair: chunks %d-%d", c, c1);
-      if ((st = DW(c)) != MOE_OK || (c1 > c && (st = DW(c1)) != MOE_OK)) return st;
-      // the next pair's first chunk goes to the slot freed by the previous pair
-      if (c + 2 < n_live && (st = P(c + 2)) != MOE_OK) return st;
-      if ((st = Bd(c, c1)) != MOE_OK) return st;
-      if ((st = S(c)) != MOE_OK || (c1 > c && (st = S(c1)) != MOE_OK)) return st;
-      if ((st = W(c, c1)) != MOE_OK) return st;
-      // its second chunk takes chunk c's slot, free once W(c, c1) has read it
-      if (c + 3 < n_live && (st = P(c + 3)) != MOE_OK) return st;
-      if (c + 2 < n_live) {
-        if ((st = F(c + 2, pair_end(c + 2))) != MOE_OK) return st;
+    if ((st = P(0)) != MOE_OK || (st = F(0)) != MOE_OK || (st = DYS(0)) != MOE_OK) return st;
+    for (int m = 0; m < n_live; ++m) {
+      NvtxRange pr("moe_backward pair %d", m, 0);
+      if ((st = DW(m)) != MOE_OK) return st;
+      if (m + 1 < n_live && (st = P(m + 1)) != MOE_OK) return st;
+      if ((st = Bd(m)) != MOE_OK || (st = S(m)) != MOE_OK || (st = W(m)) != MOE_OK) return st;
+      if (m + 1 < n_live) {
+        if ((st = F(m + 1)) != MOE_OK) return st;
         if (!ok(cudaStreamWaitEvent(s, ctx->ev_bf[1], 0))) return MOE_ERR_CUDA;  // W(m) done
-        for (int x = c + 2; x <= c + 3 && x < n_live; ++x)
-          if ((st = DYS(x)) != MOE_OK) return st;
+        if ((st = DYS(m + 1)) != MOE_OK) return st;
       }
     }
   }

@@ -295,15 +295,17 @@ MOE_API size_t moe_backward_workspace_bytes(const moe_shape_t* shape);
  *   dW_down [E][H][I] fp32        gradient of W_down
  * All four outputs are overwritten.  Inputs as moe_forward plus d_out [T][H] bf16.  The
  * intermediate g, u, h, Y, dY, dg, du and dX rows are bf16 (fp32 accumulation in every GEMM
- * and reduction); each expert's rows are padded to a multiple of 64 inside the workspace.
- * Chunks run as the mirrored pair pipeline on the caller's stream and the library's second
- * stream: every GEMM is one tile sweep over both chunks of a pair (2m, 2m+1), the weight
- * gradients accumulate per pair in fp32 (the first pair with an expert's rows stores, later
- * pairs add through TMA reductions).  d_hidden and d_weights are bit-identical for every
- * chunking; dW_* are equal up to the fp32 summation order.  workspace: dev, >=
- * moe_backward_workspace_bytes(shape): the metadata plus three chunk slots of permuted rows
- * and two chunk sets of the other row buffers (dg | du overwrite the recomputed g | u rows in
- * place).  The host blocks once, on the metadata copy.
+ * and reduction).  Chunks run as the mirrored pair pipeline on the caller's stream and the
+ * library's second stream, one unit per pair of chunks (2m, 2m+1): the routing metadata is
+ * taken per pair, so each expert's rows are contiguous over both chunks (padded to a
+ * multiple of 64 inside the workspace), every GEMM is one tile sweep over the pair's rows,
+ * and the weight gradients accumulate per pair in fp32 (the first pair with an expert's
+ * rows stores, later pairs add through TMA reductions).  d_hidden and d_weights are
+ * bit-identical for every chunking; dW_* are equal up to the fp32 summation order.
+ * workspace: dev, >= moe_backward_workspace_bytes(shape): the metadata plus two pair
+ * buffers of permuted rows (the next pair is permuted while one computes) and one pair set
+ * of the other row buffers (dg | du overwrite the recomputed g | u rows in place).  The
+ * host blocks once, on the metadata copy.
  * Errors: as moe_forward; MOE_ERR_ARG also for H % 64 or I % 32 != 0. */
 MOE_API moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
                                   const int32_t* top_k_index, const float* top_k_weights,
