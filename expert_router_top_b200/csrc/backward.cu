@@ -1,5 +1,5 @@
 // backward.cu -- backward pass of the chunked MoE layer, with the expert computation
-// recomputed per chunk.
+// recomputed per pair of chunks (the pipeline's unit).
 //
 // The Chunk MoE article ("昇腾MindSpeed分块专家计算Chunk MoE") trains through this layer:
 // the backward pass mirrors the forward chunk pipeline (section 一张专业时序图, the last
@@ -11,8 +11,10 @@
 //   du = dh silu(g);  dg = dh u silu'(g);  dX = W_gate^T dg + W_up^T du
 //   d_hidden[t] = sum_j dX;  dW_down[e] += dY h^T;  dW_gate|up[e] += dg|du x^T
 //
-// Backward buffers hold each expert's rows padded to a multiple of 64 (zero rows), so that
-// the weight-gradient GEMMs reduce over an expert's rows in whole 64-row K blocks.
+// Backward buffers hold each expert's rows of one unit padded to a multiple of 64 (zero
+// rows), so that the weight-gradient GEMMs reduce over an expert's rows in whole 64-row K
+// blocks.  The helpers below speak of "chunks": the metadata's chunks, which the pipeline
+// makes the pairs of the layer's chunks.
 //
 // The GEMMs run on one tcgen05 kernel (one CTA per SM, TMA producer warp, one MMA thread,
 // four epilogue warps, 4-stage ring, double-buffered TMEM, as the forward kernel) in four

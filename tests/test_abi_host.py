@@ -112,6 +112,38 @@ def test_workspace_follows_pair_double_buffer(name):
         assert _ws(cfg, 4) <= 0.6 * _ws(cfg, 1)  # at least the 40 % cut the method targets
 
 
+def _bwd_row_buffer_bytes(cfg, N):
+    """Backward rows by construction: the units are the pairs of chunks, ceil(N/2) of them,
+    each of at most 2*ceil(T/N) tokens, whose rows padded per expert to 64 fit in
+    tokens*k + 63*E rows; the permuted rows X (H wide) in min(units, 2) unit buffers, and
+    one unit set of [g u] (2I), h (I), Y/dX (H) and dY (H), all bf16."""
+    n = max(N, 1)
+    tu = min(2 * -(-cfg.T // n), cfg.T)
+    units = -(-n // 2)
+    rows = tu * cfg.k + 63 * cfg.E
+    return (min(units, 2) * cfg.H + 3 * cfg.I + 2 * cfg.H) * rows * 2, units, tu
+
+
+@pytest.mark.parametrize("name", ["mixtral", "qwen3", "deepseek", "tiny", "edge", "edge_varlen"])
+def test_backward_workspace_follows_pair_units(name):
+    """The backward's workspace is its row buffers plus metadata arrays (three int32 per
+    routed copy, per-unit offsets and histograms): N=2 is one pair, the size of N=1, and
+    N=4 holds a pair in flight and the next one's permuted rows."""
+    cfg = CONFIGS[name]
+    ws = {}
+    for N in (1, 2, 3, 4, 8):
+        ws[N] = moe.backward_workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.G, N)
+        buf, units, tu = _bwd_row_buffer_bytes(cfg, N)
+        meta = (12 * cfg.T * cfg.k + 4 * cfg.E * units * (tu * cfg.k // 2048 + 2)
+                + 8 * (units + 2) * (cfg.E + 8) + 20 * 256)
+        assert buf <= ws[N] <= buf + meta, (N, ws[N] - buf, meta)
+    assert ws[2] == ws[1]
+    if cfg.T >= 4096:
+        assert ws[8] < ws[4] < ws[1]
+    if name == "qwen3":
+        assert ws[4] < 0.7 * ws[1]  # 1.55 vs 2.35 GB
+
+
 def test_workspace_rejects_bad_shapes():
     assert moe.workspace_bytes(16, 12, 16, 4, 2) == 0       # H % 8
     assert moe.workspace_bytes(16, 16, 16, 4, 5) == 0       # k > E
