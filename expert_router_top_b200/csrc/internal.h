@@ -22,6 +22,7 @@ struct MetaArgs {
   int32_t* hist;            // [n_chunks * tiles_per_chunk][E] scratch
   int32_t* dst;             // [T*k] chunk-local row of each copy
   int32_t* src_tok;         // [T*k] or nullptr
+  int32_t src_relative = 0; // src_tok holds the token's index in its chunk (else in [0, T))
   int32_t* counts;          // [n_chunks][E]
   int32_t* offsets;         // [n_chunks][E+1]
   int32_t* splits;          // [n_chunks][G]

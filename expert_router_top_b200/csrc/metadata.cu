@@ -186,7 +186,7 @@ __global__ void __launch_bounds__(kMetaThreads) meta_finalize_kernel(MetaArgs a)
     if (e < 0 || e >= a.E) continue;
     const int32_t r = off[e] + base[e] + dst[s];
     dst[s] = r;
-    if (src) src[r] = (int32_t)(ts.chunk_tok0 + tok_in_chunk0 + s / a.k);
+    if (src) src[r] = (int32_t)((a.src_relative ? 0 : ts.chunk_tok0) + tok_in_chunk0 + s / a.k);
   }
 }
 

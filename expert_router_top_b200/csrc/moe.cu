@@ -355,8 +355,9 @@ struct NvtxRange {
 };
 
 moe_status_t run_metadata(const Dims& d, const int32_t* idx, uint8_t* ws, const Layout& L,
-                          int32_t* dst, int32_t* src, cudaStream_t s) {
+                          int32_t* dst, int32_t* src, cudaStream_t s, bool src_relative = false) {
   MetaArgs a;
+  a.src_relative = src_relative ? 1 : 0;
   a.idx = idx;
   a.T = d.T;
   a.k = d.k;
@@ -815,7 +816,12 @@ moe_status_t moe_forward_host_impl(const moe_shape_t* shape, const void* hidden_
   for (int c = 0; c < n_live && c < 2; ++c)
     if ((st = copy_in(c)) != MOE_OK) return st;
 
-  if ((st = run_metadata(d, idx_dev, ws, L, dst, src, sm)) != MOE_OK) return st;
+  // Fused dispatch (gate/up GEMM gathering its rows from the chunk's staged input) where one
+  // chunk's permuted copy would be a sizeable share of the GEMM traffic, as moe_forward
+  // decides for one chunk; the gather map then indexes the chunk's own rows.
+  const bool fused =
+      gemm_supports_gather() && 4 * d.t_chunk * d.k >= (int64_t)d.E * shape->I;
+  if ((st = run_metadata(d, idx_dev, ws, L, dst, src, sm, fused)) != MOE_OK) return st;
   if ((st = fetch_packed(ctx, ws, L, sm)) != MOE_OK) return st;
   std::vector<int32_t> counts(ctx->host_stage + kStatusWords,
                               ctx->host_stage + kStatusWords + (size_t)d.n * d.E);
@@ -848,6 +854,27 @@ moe_status_t moe_forward_host_impl(const moe_shape_t* shape, const void* hidden_
     if (s2 != MOE_OK) return s2;
     return cudaEventRecord(ctx->ev_gemm[c & 1], sg) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   };
+  // fused: chunk c's GEMMs gather from input buffer c % 2, which they free after the
+  // gate/up GEMM (the copy-in of chunk c+2 waits for that); buffer c % 2 of the expert rows
+  // is free once U(c-2) has read it
+  auto experts_fused = [&](int c) -> moe_status_t {
+    if (cudaStreamWaitEvent(sg, ctx->ev_in[c & 1], 0) != cudaSuccess ||
+        (c >= 2 && cudaStreamWaitEvent(sg, ctx->ev_unperm[c & 1], 0) != cudaSuccess))
+      return MOE_ERR_CUDA;
+    const int64_t rows = len(c) * k;
+    const int32_t* cnt = counts.data() + (size_t)c * E;
+    const int32_t* offs = reinterpret_cast<const int32_t*>(ws + L.offsets) + (size_t)c * (E + 1);
+    moe_status_t s2 = gemm_call(nullptr, rows, W_gate_up, act(c), offs, cnt, E, H, I, 2 * I, true,
+                                dev_status, ctx->num_sms, sg, src + bounds[c] * k,
+                                ws + hs.in[c & 1], len(c));
+    if (s2 != MOE_OK) return s2;
+    if (cudaEventRecord(ctx->ev_in_free[c & 1], sg) != cudaSuccess) return MOE_ERR_CUDA;
+    s2 = gemm_call(act(c), rows, W_down, xy(c), offs, cnt, E, I, H, H, false, dev_status,
+                   ctx->num_sms, sg);
+    if (s2 != MOE_OK) return s2;
+    if (cudaEventRecord(ctx->ev_gemm[c & 1], sg) != cudaSuccess) return MOE_ERR_CUDA;
+    return c + 2 < n_live ? copy_in(c + 2) : MOE_OK;
+  };
   auto unpermute = [&](int c) -> moe_status_t {
     if (cudaStreamWaitEvent(sm, ctx->ev_gemm[c & 1], 0) != cudaSuccess) return MOE_ERR_CUDA;
     if (c >= 2 && cudaStreamWaitEvent(sm, ctx->ev_out_free[c & 1], 0) != cudaSuccess)
@@ -858,6 +885,7 @@ moe_status_t moe_forward_host_impl(const moe_shape_t* shape, const void* hidden_
                            ws + hs.out[c & 1], L.rows_cap, sm) != cudaSuccess)
         return MOE_ERR_CUDA;
     }
+    if (fused && cudaEventRecord(ctx->ev_unperm[c & 1], sm) != cudaSuccess) return MOE_ERR_CUDA;
     // copy-out of chunk c beside the next chunk's GEMMs
     if (cudaEventRecord(ctx->ev_out[c & 1], sm) != cudaSuccess ||
         cudaStreamWaitEvent(co, ctx->ev_out[c & 1], 0) != cudaSuccess ||
@@ -871,7 +899,15 @@ moe_status_t moe_forward_host_impl(const moe_shape_t* shape, const void* hidden_
   if (cudaEventRecord(ctx->ev_start, sm) != cudaSuccess ||
       cudaStreamWaitEvent(sg, ctx->ev_start, 0) != cudaSuccess)
     return MOE_ERR_CUDA;
-  if (n_live > 0) {
+  if (n_live > 0 && fused) {
+    // G: E(0) E(1) E(2) ... (E(c+2) after U(c) freed buffer c % 2); M: U(0) U(1) ...
+    if ((st = experts_fused(0)) != MOE_OK) return st;
+    if (n_live > 1 && (st = experts_fused(1)) != MOE_OK) return st;
+    for (int c = 0; c < n_live; ++c) {
+      if ((st = unpermute(c)) != MOE_OK) return st;
+      if (c + 2 < n_live && (st = experts_fused(c + 2)) != MOE_OK) return st;
+    }
+  } else if (n_live > 0) {
     if ((st = permute(0)) != MOE_OK || (st = experts(0)) != MOE_OK) return st;
     for (int c = 0; c < n_live; ++c) {
       if (c + 1 < n_live) {

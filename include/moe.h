@@ -272,6 +272,9 @@ MOE_API size_t moe_workspace_bytes_host(const moe_shape_t* shape);
  * in while the expert GEMMs of chunk c-1 run, and chunk c's output rows are copied out
  * while the GEMMs of chunk c+1 run, on two library copy streams beside the pair pipeline
  * ([ChunkMoE] "一张专业时序图": transfers hidden behind the neighbouring chunk's compute).
+ * Each chunk has its own GEMM sweeps; where one chunk's permuted copy would be a sizeable
+ * share of their traffic (4 * T_chunk * k >= E * I), the gate/up GEMM gathers its rows
+ * straight from the chunk's staged input rows instead of a permuted copy.
  * The call returns when out_host is complete (it synchronizes `stream`).  Results are
  * bit-identical to moe_forward.  workspace: dev, >= moe_workspace_bytes_host(shape).
  * Errors: as moe_forward. */

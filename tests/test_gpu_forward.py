@@ -87,6 +87,41 @@ def test_forward_host_buffers_match_device_forward(moe, name, pinned):
         assert torch.equal(got, ref.cpu()), f"{name} N={N} pinned={pinned}"
 
 
+@pytest.mark.parametrize("pinned", [True, False])
+def test_forward_host_fused_gather_from_staged_chunks(moe, pinned):
+    """With few expert columns (E*I small against 4*T_chunk*k) moe_forward_host gathers the
+    gate/up rows straight from each chunk's staged input, through chunk-relative token
+    indices: the same bits as moe_forward for even and odd chunk counts, a ragged last
+    chunk and an empty trailing one, and within the layer's bar of the oracle."""
+    cfg = LayerConfig("host_fused", 601, 256, 3, 2, 32, "normal")  # fused iff T_chunk >= 12
+    cpu = layer_inputs(cfg)
+    gpu = {k: v.cuda() for k, v in cpu.items()}
+    h, i, w = ((t.pin_memory() if pinned else t) for t in (cpu["hidden"], cpu["idx"], cpu["w"]))
+    ref1 = _run(moe, gpu, 1)
+    assert_layer_close(ref1, _oracle(cpu), "host_fused N=1 (device)")
+    # N=35: chunks of 18 tokens, the 34th holds 7 and the 35th none; N=51: 12 tokens, 1 last
+    for N in (1, 2, 3, 5, 35, 51):
+        got = moe.forward_host(h, i, w, gpu["wgu"], gpu["wd"], num_chunks=N)
+        assert torch.equal(got, ref1.cpu()), f"host_fused N={N} pinned={pinned}"
+
+
+def test_forward_host_full_size(moe):
+    """The Qwen3-shaped 16k layer through moe_forward_host at num_chunks=4 (the fused
+    per-chunk path the benchmark's end-to-end number takes) and 8 (the separate one): the
+    same bits as moe_forward on device-resident inputs."""
+    cfg = CONFIGS["qwen3"]
+    idx, w = routing(cfg)
+    x = hidden(cfg.T, cfg.H)
+    wgu, wd = expert_weights(cfg.E, cfg.H, cfg.I, device="cuda")
+    gpu = dict(hidden=x.cuda(), idx=torch.from_numpy(idx).cuda(), w=torch.from_numpy(w).cuda(),
+               wgu=wgu, wd=wd)
+    for N in (4, 8):
+        ref = _run(moe, gpu, N, cfg.G, "auto")
+        got = moe.forward_host(x.pin_memory(), torch.from_numpy(idx).pin_memory(),
+                               torch.from_numpy(w).pin_memory(), wgu, wd, num_chunks=N)
+        assert torch.equal(got, ref.cpu()), f"qwen3 host N={N}"
+
+
 @pytest.mark.parametrize("S", [1, 143, 333, 1000])
 def test_forward_chunk_size(moe, S):
     """moe_chunk_size: chunks of exactly S tokens give the unsplit bits; with both
