@@ -222,8 +222,9 @@ struct DeviceCtx {
   cudaStream_t copy_in = nullptr, copy_out = nullptr;
   cudaEvent_t ev_in[2] = {}, ev_in_free[2] = {}, ev_out[2] = {}, ev_out_free[2] = {},
               ev_copy_join = nullptr;
-  // backward pipeline: permuted rows ready (per X slot), recomputed Y ready, dY ready, dX
-  // ready, d_hidden rows summed (per buffer), all of a chunk's GEMMs done (per X slot)
+  // backward pipeline, one unit per pair of chunks: permuted rows ready (per X buffer),
+  // recomputed Y ready / weight gradients done, dY scattered / d_weights read Y, dX ready,
+  // d_hidden rows summed, a unit's weight gradients done with its X buffer (per X buffer)
   cudaEvent_t ev_bp[2] = {}, ev_bf[2] = {}, ev_bdy[2] = {}, ev_bdx[1] = {}, ev_bsum[1] = {},
               ev_bw[2] = {};
   int32_t* host_stage = nullptr;
