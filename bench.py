@@ -85,20 +85,48 @@ def dist_env():
 # ------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi samples of one GPU's clocks and throttle reasons, every 50 ms, each with
-    its host arrival time so that only the samples taken during the timed region count."""
+    """SM clock, power and clock-event reasons of one GPU, read through NVML every 5 ms by a
+    background thread (nvidia-smi every 50 ms if NVML is unavailable), each sample stamped
+    with its host time so that a summary covers exactly one timed region.  Read-only: it
+    changes no setting of the GPU."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                   "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, gpu_index):
+    def __init__(self, gpu_index, period_s=0.005):
         self.gpu = gpu_index
+        self.period = period_s
+        self.samples = []  # (host time, sm MHz, max sm MHz, reasons set)
         self.proc = None
-        self.lines = []
         self.thread = None
+        self.nvml = None
+        self.source = None
+        self._stop = threading.Event()
+
+    def _nvml_handle(self):
+        import pynvml
+
+        pynvml.nvmlInit()
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.gpu).uuid)
+            h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:  # noqa: BLE001 - fall back to the NVML index
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+        return pynvml, h
 
     def start(self):
+        try:
+            self.nvml = self._nvml_handle()
+            self.source = "nvml"
+            self.thread = threading.Thread(target=self._poll_nvml, daemon=True)
+            self.thread.start()
+            return
+        except Exception:  # noqa: BLE001 - no NVML: sample through nvidia-smi
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
@@ -107,46 +135,77 @@ class ClockSampler:
         except OSError:
             self.proc = None
             return
-        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.source = "nvidia-smi"
+        self.thread = threading.Thread(target=self._read_smi, daemon=True)
         self.thread.start()
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append((time.perf_counter(), line.strip()))
+    def _poll_nvml(self):
+        nv, h = self.nvml
+        smax = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons",
+                              getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
+        while not self._stop.is_set():
+            try:
+                sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                bits = int(get_reasons(h)) if get_reasons else 0
+            except Exception:  # noqa: BLE001 - a failed read is skipped
+                time.sleep(self.period)
+                continue
+            reasons = {n for n, b in self.REASON_BITS.items() if bits & b}
+            self.samples.append((time.perf_counter(), sm, smax, reasons))
+            time.sleep(self.period)
 
-    def stop(self, t0=None, t1=None):
-        """Summary of the samples that arrived in [t0, t1 + 0.1 s] (host perf_counter
-        times of the timed region; all samples when not given)."""
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        if self.thread:
-            self.thread.join(timeout=2)
-        sm, smax, reasons = [], None, set()
+    def _read_smi(self):
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        lines = self.lines
-        if t0 is not None:
-            lines = [x for x in self.lines if t0 <= x[0] <= t1 + 0.1]
-        for _, ln in lines:
-            f = [x.strip() for x in ln.split(",")]
+        for line in self.proc.stdout:
+            f = [x.strip() for x in line.strip().split(",")]
             if len(f) < 9:
                 continue
             try:
-                sm.append(float(f[1]))
-                smax = float(f[2])
+                sm, smax = float(f[1]), float(f[2])
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
+            reasons = {n for n, v in zip(names, f[5:9]) if v.lower() == "active"}
+            self.samples.append((time.perf_counter(), sm, smax, reasons))
+
+    def summary(self, t0=None, t1=None, min_samples=3, widen_to=None):
+        """Median SM clock, max clock and the reasons seen in the samples taken in [t0, t1]
+        (host perf_counter times of a timed region).  With fewer than min_samples there,
+        the window is widened back to widen_to (the start of the untimed steps that ran
+        just before at the same load) and the summary says so."""
+        pts = list(self.samples)
+        window = "all"
+        if t0 is not None:
+            sel = [x for x in pts if t0 <= x[0] <= t1 + self.period]
+            window = "timed region"
+            if len(sel) < min_samples and widen_to is not None:
+                sel = [x for x in pts if widen_to <= x[0] <= t1 + self.period]
+                window = "timed region and the untimed steps just before it"
+            pts = sel
+        if not pts:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        reasons = set()
+        for x in pts:
+            reasons |= x[3]
+        return {"sm_mhz": statistics.median(x[1] for x in pts), "sm_max_mhz": pts[-1][2],
+                "sm_mhz_min": min(x[1] for x in pts), "reasons": sorted(reasons),
+                "samples": len(pts), "window": window, "source": self.source}
+
+    def stop(self):
+        self._stop.set()
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        if self.nvml is not None:
+            try:
+                self.nvml[0].nvmlShutdown()
+            except Exception:  # noqa: BLE001
+                pass
 
 
 def spin_up(step, seconds=0.5):
@@ -294,12 +353,46 @@ def run_reference(args, cfg):
 
 
 def config_block(cfg, chunks, dispatch="auto"):
+    """The workload as both arms print it: the requested dispatch ("auto" = the library's
+    own choice for the shape; the line's top-level `dispatch_resolved` says which ran)."""
     wbytes = 6 * cfg.E * cfg.H * cfg.I
     return {"workload": workload_name(cfg), "T": cfg.T, "H": cfg.H, "E": cfg.E, "k": cfg.k,
             "I": cfg.I, "ep_groups": cfg.G, "num_chunks": chunks, "dispatch": dispatch,
             "routing": cfg.routing,
             "ffn": "SwiGLU", "parallelism": "replicas",
             "l2": f"inputs larger than L2 ({wbytes / 1e9:.2f} GB of expert weights read per step)"}
+
+
+def tensor_peak(peaks, clk):
+    """bf16 tensor roof of a launch timed at the sampled clock: the measured burst figure
+    scaled by (median SM MHz / max SM MHz) of the samples taken while it ran; the burst
+    figure itself when no sample was taken.  Returns (peak TFLOP/s, scale)."""
+    burst = peaks["bf16_tflops"]
+    if clk and clk.get("sm_mhz") and clk.get("sm_max_mhz"):
+        scale = min(1.0, clk["sm_mhz"] / clk["sm_max_mhz"])
+        return burst * scale, scale
+    return burst, 1.0
+
+
+def kernel_rates(prof, units, steps):
+    """Per-kind launches and times of `steps` steps, with each GEMM kind's TFLOP/s and each
+    row kernel's GB/s from the algorithmic work of one step."""
+    kinds = {}
+    for kind in ("metadata", "permute", "gateup", "down", "unpermute"):
+        p = prof[kind]
+        kinds[kind] = dict(launches=p["launches"], ms=p["ms"],
+                           ms_per_step=p["ms"] / steps if steps else 0.0)
+
+    def rate(work, ms, scale):
+        return work * steps / (ms / 1e3) / scale if ms > 0 else 0.0
+
+    kinds["gateup"]["tflops"] = rate(units["gateup_flops"], prof["gateup"]["ms"], 1e12)
+    kinds["down"]["tflops"] = rate(units["down_flops"], prof["down"]["ms"], 1e12)
+    kinds["permute"]["gbs"] = rate(units["permute_bytes"], prof["permute"]["ms"], 1e9)
+    kinds["unpermute"]["gbs"] = rate(units["unpermute_bytes"], prof["unpermute"]["ms"], 1e9)
+    gm = prof["gateup"]["ms"] + prof["down"]["ms"]
+    kinds["grouped_gemm_tflops"] = rate(units["gateup_flops"] + units["down_flops"], gm, 1e12)
+    return kinds
 
 
 # ------------------------------------------------------------------------- our arm
@@ -320,6 +413,144 @@ def time_steps(moe, inp, cfg, chunks, ws, steps, stream, dispatch="auto", pair_g
     return start.elapsed_time(end), out
 
 
+class Runner:
+    """One workload on one GPU: times moe_forward at a given chunk count and dispatch with
+    the library's per-launch events on, with the clock samples of exactly that region."""
+
+    def __init__(self, moe, cfg, inp, dev, stream, clocks, pg=None):
+        self.moe, self.cfg, self.inp, self.dev, self.stream = moe, cfg, inp, dev, stream
+        self.clocks, self.pg = clocks, pg
+
+    def workspace(self, chunks):
+        c = self.cfg
+        return self.moe.alloc_workspace(
+            self.moe.workspace_bytes(c.T, c.H, c.I, c.E, c.k, c.G, chunks), self.dev)
+
+    def resolve(self, chunks, dispatch, per_chunk_gemms=False):
+        c = self.cfg
+        d = self.moe.forward_dispatch(c.T, c.H, c.I, c.E, c.k, dispatch, c.G, chunks)
+        return d, d == "fused" and not per_chunk_gemms
+
+    def measure(self, chunks, dispatch, steps, warmup, per_chunk_gemms=False, spin_s=0.3):
+        moe, c, inp = self.moe, self.cfg, self.inp
+        ws = self.workspace(chunks)
+        resolved, pair = self.resolve(chunks, dispatch, per_chunk_gemms)
+        meta = moe.metadata(inp["idx"], c.E, c.G, chunks)
+        n_live = int((np.diff(meta["bounds"]) > 0).sum())
+        units = algorithmic_units(c, meta["counts"], n_live, resolved, pair)
+
+        def step():
+            moe.forward(inp["hidden"], inp["idx"], inp["w"], inp["wgu"], inp["wd"],
+                        num_chunks=chunks, ep_groups=c.G, workspace=ws, dispatch=dispatch,
+                        pair_gemms=not per_chunk_gemms)
+
+        t_load = time.perf_counter()
+        spin = spin_up(step, spin_s)
+        for _ in range(warmup):
+            step()
+        torch.cuda.synchronize()
+        if self.pg:
+            self.pg.barrier()
+        torch.cuda.synchronize()
+        moe.profile_enable(True)
+        t0 = time.perf_counter()
+        ms, _ = time_steps(moe, inp, c, chunks, ws, steps, self.stream, dispatch,
+                           not per_chunk_gemms)
+        t1 = time.perf_counter()
+        if self.pg:
+            self.pg.barrier()
+        prof = moe.profile_read()
+        moe.profile_enable(False)
+        clk = self.clocks.summary(t0, t1, widen_to=t_load) if self.clocks else None
+        del ws
+        return dict(ms=ms, ms_per_step=ms / steps, steps=steps, prof=prof, clk=clk,
+                    units=units, meta=meta, n_live=n_live, dispatch=resolved, pair_gemms=pair,
+                    spinup_steps=spin,
+                    kinds=kernel_rates(prof, units, steps))
+
+    def timeline(self, chunks, dispatch, calls=3):
+        """Launch records of the last of `calls` back-to-back forward calls, times relative
+        to that call's first launch."""
+        moe, c, inp = self.moe, self.cfg, self.inp
+        ws = self.workspace(chunks)
+        resolved, pair = self.resolve(chunks, dispatch)
+        for _ in range(3):
+            moe.forward(inp["hidden"], inp["idx"], inp["w"], inp["wgu"], inp["wd"],
+                        num_chunks=chunks, ep_groups=c.G, workspace=ws, dispatch=dispatch)
+        torch.cuda.synchronize()
+        moe.profile_enable(True)
+        for _ in range(calls):
+            moe.forward(inp["hidden"], inp["idx"], inp["w"], inp["wgu"], inp["wd"],
+                        num_chunks=chunks, ep_groups=c.G, workspace=ws, dispatch=dispatch)
+        recs = [r for r in moe.profile_timeline() if r["call"] == calls]
+        moe.profile_enable(False)
+        del ws
+        t0 = min(r["start_ms"] for r in recs) if recs else 0.0
+        for r in recs:
+            r["start_ms"] = round(r["start_ms"] - t0, 4)
+            r["end_ms"] = round(r["end_ms"] - t0, 4)
+        return {"num_chunks": chunks, "dispatch": resolved,
+                "gemm_sweep": "per pair of chunks" if pair and chunks > 1 else "per chunk",
+                "step_ms": max((r["end_ms"] for r in recs), default=0.0), "launches": recs}
+
+
+def gemm_roofline(m, peaks, peak_src):
+    """Roofline object of the gate/up GEMM (the dominant kernel) for one measurement: per
+    launch algorithmic flops and bytes over its event time; the tensor roof is the measured
+    burst bf16 figure scaled to the clock sampled during the timed region."""
+    units, g, steps = m["units"], m["prof"]["gateup"], m["steps"]
+    n_gu = max(1, g["launches"] // max(1, steps))
+    flops_l = units["gateup_flops"] / n_gu
+    bytes_l = units["gateup_alg_bytes"] / n_gu
+    t_l = g["ms"] / max(1, g["launches"]) / 1e3  # s per launch
+    peak_tc, scale = tensor_peak(peaks, m["clk"])
+    peak_bw = peaks["hbm_gbs"]
+    t_tensor = flops_l / (peak_tc * 1e12)
+    t_mem = bytes_l / (peak_bw * 1e9)
+    if t_mem > t_tensor:
+        r = {"bound": "hbm", "achieved": bytes_l / t_l / 1e9 if t_l else 0.0, "peak": peak_bw,
+             "unit": "GB/s"}
+    else:
+        r = {"bound": "tensor", "achieved": flops_l / t_l / 1e12 if t_l else 0.0,
+             "peak": peak_tc, "unit": "TFLOP/s"}
+    r["frac"] = r["achieved"] / r["peak"]
+    tf = flops_l / t_l / 1e12 if t_l else 0.0
+    r.update({
+        "kernel": "grouped_gemm_kernel<gate/up + SwiGLU" +
+                  (", gathered A rows" if m["dispatch"] == "fused" else "") + "> (tcgen05)",
+        "peak_source": f"{peak_src}: MEASURED_PEAKS.json bf16_tflops (burst) x sampled clock "
+                       f"ratio {scale:.3f}; HBM copy hbm_gbs",
+        "clock_scale": scale,
+        "per_launch": {"flops": flops_l, "bytes": bytes_l, "ms": t_l * 1e3,
+                       "roofline_ms": max(t_tensor, t_mem) * 1e3},
+        "frac_of_roofline_time": max(t_tensor, t_mem) / t_l if t_l else None,
+        "tensor_frac_of_burst": tf / peaks["bf16_tflops"],
+        "tensor_frac_of_sustained": tf / peaks["bf16_tflops_sustained"],
+        "hbm_frac": bytes_l / t_l / 1e9 / peak_bw if t_l else None})
+    return r
+
+
+def per_n_entry(moe, cfg, m, peaks):
+    k = m["kinds"]
+    peak_tc, _ = tensor_peak(peaks, m["clk"])
+    e = {"ms_per_step": m["ms_per_step"], "tokens_per_s": cfg.T / (m["ms_per_step"] / 1e3),
+         "dispatch": m["dispatch"],
+         "gemm_sweep": "per pair of chunks" if m["pair_gemms"] and m["n_live"] > 1
+         else "per chunk",
+         "gateup_tflops": k["gateup"]["tflops"], "down_tflops": k["down"]["tflops"],
+         "grouped_gemm_tflops": k["grouped_gemm_tflops"],
+         "gateup_frac_of_clock_scaled_burst": k["gateup"]["tflops"] / peak_tc,
+         "gateup_frac_of_burst": k["gateup"]["tflops"] / peaks["bf16_tflops"],
+         "unpermute_ms_per_step": k["unpermute"]["ms_per_step"],
+         "gemm_ms_per_step": k["gateup"]["ms_per_step"] + k["down"]["ms_per_step"],
+         "workspace_bytes": moe.workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.G,
+                                                m["meta"]["counts"].shape[0]),
+         "clocks": m["clk"]}
+    if cfg.G > 1:
+        e["send_splits"] = m["meta"]["send"].tolist()
+    return e
+
+
 def run_ours(args, cfg):
     import expert_router_top_b200 as moe
 
@@ -337,140 +568,97 @@ def run_ours(args, cfg):
     dev = torch.device("cuda", local)
     inp = make_inputs(cfg, dev)
     chunks = args.chunks
-    ws_bytes = moe.workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.G, chunks)
-    ws = moe.alloc_workspace(ws_bytes, dev)
     stream = torch.cuda.current_stream()
-
-    meta = moe.metadata(inp["idx"], cfg.E, cfg.G, chunks)
-    counts = meta["counts"]
-    n_live = int((np.diff(meta["bounds"]) > 0).sum())
-    dispatch = moe.forward_dispatch(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, args.dispatch, cfg.G,
-                                    chunks)
-    pair_gemms = dispatch == "fused" and not args.per_chunk_gemms
-    units = algorithmic_units(cfg, counts, n_live, dispatch, pair_gemms)
-    weight_stream = float(units["gateup_weight_bytes"] + units["down_weight_bytes"])
-
-    pair = not args.per_chunk_gemms
-
-    def fwd_step():
-        moe.forward(inp["hidden"], inp["idx"], inp["w"], inp["wgu"], inp["wd"],
-                    num_chunks=chunks, ep_groups=cfg.G, workspace=ws, dispatch=args.dispatch,
-                    pair_gemms=pair)
-
     clocks = ClockSampler(local) if rank == 0 else None
     if clocks:
         clocks.start()
-    spinup = spin_up(fwd_step)
-    for _ in range(args.warmup):
-        fwd_step()
-    torch.cuda.synchronize()
-    if pg:
-        pg.barrier()
-    torch.cuda.synchronize()
-    moe.profile_enable(True)
-    t0 = time.perf_counter()
-    ms, out = time_steps(moe, inp, cfg, chunks, ws, args.steps, stream, args.dispatch, pair)
-    t1 = time.perf_counter()
-    if pg:
-        pg.barrier()
-    prof = moe.profile_read()
-    moe.profile_enable(False)
-    clk = clocks.stop(t0, t1) if clocks else None
+    run = Runner(moe, cfg, inp, dev, stream, clocks, pg)
+    peaks, peak_src = load_peaks()
 
-    ms_max = max_over_ranks(ms, pg, dev)
+    # ---- the headline: K timed steps at the requested chunk count and dispatch
+    head = run.measure(chunks, args.dispatch, args.steps, args.warmup, args.per_chunk_gemms,
+                       spin_s=0.5)
+    ms_max = max_over_ranks(head["ms"], pg, dev)
     ms_per_step = ms_max / args.steps
     value = job_tokens_per_s(world, cfg.T, args.steps, ms_max)
-
-    # N = 1 reference point of the same workload (for the <= 5 % loss target), untimed key
-    ms_n1 = None
-    if chunks != 1:
-        ws1 = moe.alloc_workspace(moe.workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.G, 1),
-                                  dev)
-        for _ in range(2):
-            moe.forward(inp["hidden"], inp["idx"], inp["w"], inp["wgu"], inp["wd"],
-                        num_chunks=1, ep_groups=cfg.G, workspace=ws1, dispatch=args.dispatch)
-        ms1, _ = time_steps(moe, inp, cfg, 1, ws1, args.steps, stream, args.dispatch)
-        ms_n1 = ms1 / args.steps
-        del ws1
+    units, kinds = head["units"], head["kinds"]
+    weight_stream = float(units["gateup_weight_bytes"] + units["down_weight_bytes"])
 
     # ---- end to end through the public call, host buffers, copies inside the region
+    ws = run.workspace(chunks)
     e2e = run_e2e(moe, inp, cfg, chunks, ws, args, stream, dev, pg, world)
+    del ws
 
-    # ---- roofline of the dominant kernel (gate/up grouped GEMM)
-    peaks, peak_src = load_peaks()
-    kinds = {}
-    for kind in moe.KERNEL_KINDS:
-        p = prof[kind]
-        kinds[kind] = dict(launches=p["launches"], ms=p["ms"],
-                           ms_per_step=p["ms"] / args.steps if args.steps else 0.0)
-    steps = args.steps
-    g, d, pm, um = prof["gateup"], prof["down"], prof["permute"], prof["unpermute"]
-    gu_tflops = units["gateup_flops"] * steps / (g["ms"] / 1e3) / 1e12 if g["ms"] > 0 else 0.0
-    dn_tflops = units["down_flops"] * steps / (d["ms"] / 1e3) / 1e12 if d["ms"] > 0 else 0.0
-    pm_gbs = units["permute_bytes"] * steps / (pm["ms"] / 1e3) / 1e9 if pm["ms"] > 0 else 0.0
-    um_gbs = units["unpermute_bytes"] * steps / (um["ms"] / 1e3) / 1e9 if um["ms"] > 0 else 0.0
-    gemm_tflops = (units["gateup_flops"] + units["down_flops"]) * steps / \
-        ((g["ms"] + d["ms"]) / 1e3) / 1e12 if g["ms"] + d["ms"] > 0 else 0.0
-    kinds["gateup"]["tflops"] = gu_tflops
-    kinds["down"]["tflops"] = dn_tflops
-    kinds["permute"]["gbs"] = pm_gbs
-    kinds["unpermute"]["gbs"] = um_gbs
-    # per gate/up launch: algorithmic flops and bytes (weights of the chunk's active experts,
-    # the permuted rows read, Act written), averaged over the step's launches
-    n_gu = max(1, g["launches"] // max(1, steps))
-    gu_flops_l = units["gateup_flops"] / n_gu
-    gu_bytes_l = units["gateup_alg_bytes"] / n_gu
-    t_l = g["ms"] / max(1, g["launches"]) / 1e3  # s per launch
-    # the dominant kernel runs inside a long sequence of steps (after the clock spin-up, at
-    # the power-capped clock): the sustained bf16 figure is its tensor roof
-    peak_tc, peak_bw = peaks["bf16_tflops_sustained"], peaks["hbm_gbs"]
-    t_tensor = gu_flops_l / (peak_tc * 1e12)
-    t_mem = gu_bytes_l / (peak_bw * 1e9)
-    traffic = traffic_per_launch(cfg.name, chunks, dispatch, pair_gemms)
-    if t_mem > t_tensor:
-        roofline = {"bound": "hbm", "achieved": gu_bytes_l / t_l / 1e9 if t_l else 0.0,
-                    "peak": peak_bw, "unit": "GB/s"}
-    else:
-        roofline = {"bound": "tensor", "achieved": gu_flops_l / t_l / 1e12 if t_l else 0.0,
-                    "peak": peak_tc, "unit": "TFLOP/s"}
-    roofline["frac"] = roofline["achieved"] / roofline["peak"]
-    roofline.update({
-        "traffic": traffic,
-        "kernel": "grouped_gemm_kernel<gate/up + SwiGLU" + (", gathered A rows" if dispatch == "fused"
-                                                             else "") + "> (tcgen05)",
-        "peak_source": f"{peak_src}: MEASURED_PEAKS.json (bf16 sustained, HBM copy)",
-        "per_launch": {"flops": gu_flops_l, "bytes": gu_bytes_l, "ms": t_l * 1e3,
-                       "roofline_ms": max(t_tensor, t_mem) * 1e3},
-        "frac_of_roofline_time": max(t_tensor, t_mem) / t_l if t_l else None,
-        "tensor_frac": gu_flops_l / t_l / 1e12 / peak_tc if t_l else None,
-        "tensor_frac_of_burst": gu_flops_l / t_l / 1e12 / peaks["bf16_tflops"] if t_l else None,
-        "hbm_frac": gu_bytes_l / t_l / 1e9 / peak_bw if t_l else None})
+    roofline = gemm_roofline(head, peaks, peak_src)
+    roofline["traffic"] = traffic_per_launch(cfg.name, chunks, head["dispatch"],
+                                             head["pair_gemms"])
 
-    ws_per_n = {str(n): moe.workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.G, n)
-                for n in (1, 2, 4)}
+    per_n, isolated, timelines = {}, None, None
+    if not args.headline_only:
+        # ---- the same workload at N = 1, 2, 4 (the library's own dispatch choice each)
+        for n in args.per_n:
+            m = head if (n == chunks and args.dispatch == "auto" and not args.per_chunk_gemms) \
+                else run.measure(n, "auto", args.steps, args.warmup)
+            per_n[str(n)] = per_n_entry(moe, cfg, m, peaks)
+        # ---- permute and unpermute exposed: separate dispatch, one chunk, event-timed
+        iso = run.measure(1, "separate", args.steps, args.warmup)
+        ik = iso["kinds"]
+        isolated = {
+            "permute_gbs": ik["permute"]["gbs"],
+            "permute_frac_of_hbm": ik["permute"]["gbs"] / peaks["hbm_gbs"],
+            "unpermute_gbs": ik["unpermute"]["gbs"],
+            "unpermute_frac_of_hbm": ik["unpermute"]["gbs"] / peaks["hbm_gbs"],
+            "permute_bytes_per_step": iso["units"]["permute_bytes"],
+            "unpermute_bytes_per_step": iso["units"]["unpermute_bytes"],
+            "how": "num_chunks=1, separate dispatch: the permute runs before and the unpermute "
+                   "after the expert GEMMs, each alone on the GPU; CUDA events around each "
+                   "launch on its stream; bytes = (T + T*k)*H*2 + 4 (permute) or 8 "
+                   "(unpermute) bytes per (t, j)",
+            "ms_per_step": iso["ms_per_step"], "clocks": iso["clk"]}
+        if args.timeline:
+            timelines = [run.timeline(chunks, "auto"), run.timeline(1, "auto"),
+                         run.timeline(chunks, "separate")]
+            with open(args.timeline, "w") as f:
+                json.dump({"workload": workload_name(cfg), "config": config_block(cfg, chunks),
+                           "timelines": timelines}, f, indent=1)
+    if clocks:
+        clocks.stop()
+
+    ms_n1 = per_n.get("1", {}).get("ms_per_step")
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; random-init expert weights of the layer's shape)",
-        "config": dict(config_block(cfg, chunks, dispatch),
-                       gemm_sweep="per pair of chunks" if pair_gemms and n_live > 1
-                       else "per chunk"),
+        "config": config_block(cfg, chunks, args.dispatch),
+        "dispatch_resolved": head["dispatch"],
+        "gemm_sweep": "per pair of chunks" if head["pair_gemms"] and head["n_live"] > 1
+        else "per chunk",
         "roofline": roofline,
-        "grouped_gemm_tflops": gemm_tflops,
-        "grouped_gemm_frac_of_peak": gemm_tflops / peak_tc,
-        "permute_gbs": pm_gbs, "permute_frac_of_hbm": pm_gbs / peaks["hbm_gbs"],
-        "unpermute_gbs": um_gbs, "unpermute_frac_of_hbm": um_gbs / peaks["hbm_gbs"],
-        "kernels": kinds,
+        "grouped_gemm_tflops": kinds["grouped_gemm_tflops"],
+        "grouped_gemm_frac_of_clock_scaled_burst":
+            kinds["grouped_gemm_tflops"] / tensor_peak(peaks, head["clk"])[0],
+        "grouped_gemm_frac_of_burst": kinds["grouped_gemm_tflops"] / peaks["bf16_tflops"],
+        "permute_gbs": kinds["permute"]["gbs"],
+        "permute_frac_of_hbm": kinds["permute"]["gbs"] / peaks["hbm_gbs"],
+        "unpermute_gbs": kinds["unpermute"]["gbs"],
+        "unpermute_frac_of_hbm": kinds["unpermute"]["gbs"] / peaks["hbm_gbs"],
+        "row_kernels_isolated": isolated,
+        "kernels": {k2: v for k2, v in kinds.items() if isinstance(v, dict)},
         "weight_bytes_streamed_per_step": weight_stream,
-        "workspace_bytes": ws_per_n,
+        "workspace_bytes": {str(n): moe.workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.G,
+                                                        n) for n in (1, 2, 4)},
+        "per_n": per_n or None,
         "ms_per_step_num_chunks_1": ms_n1,
-        "send_splits": meta["send"].tolist() if cfg.G > 1 else None,
-        "gpu_launches": int(prof["kernels"]),
-        "spinup_steps": spinup,
+        "send_splits": head["meta"]["send"].tolist() if cfg.G > 1 else None,
+        "gpu_launches": int(head["prof"]["kernels"]),
+        "spinup_steps": head["spinup_steps"],
         "e2e": e2e,
-        "clocks": clk,
+        "clocks": head["clk"],
+        "peaks": dict(peaks, source=peak_src),
     }
+    if timelines:
+        line["timeline_file"] = args.timeline
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tps, ntok, dt, threads = oracle_tokens_per_s(cfg, inp, args.cpu_budget_s)
         line["cpu_baseline"] = {
@@ -548,6 +736,7 @@ def run_backward(args, cfg):
     clocks = ClockSampler(local) if rank == 0 else None
     if clocks:
         clocks.start()
+    t_load = time.perf_counter()
     spinup = spin_up(step)
     for _ in range(args.warmup):
         step()
@@ -568,7 +757,9 @@ def run_backward(args, cfg):
         pg.barrier()
     prof = moe.profile_read()
     moe.profile_enable(False)
-    clk = clocks.stop(t0, t1) if clocks else None
+    clk = clocks.summary(t0, t1, widen_to=t_load) if clocks else None
+    if clocks:
+        clocks.stop()
     ms_max = max_over_ranks(start.elapsed_time(end), pg, dev)
     steps = args.steps
     peaks, peak_src = load_peaks()
@@ -585,7 +776,7 @@ def run_backward(args, cfg):
     wg = prof["bwd_wgrad"]
     t = wg["ms"] / steps / 1e3
     f, b = units["flops"]["bwd_wgrad"], units["wgrad_bytes"]
-    peak_tc = peaks["bf16_tflops_sustained"]  # long step sequence, power-capped clock
+    peak_tc, scale = tensor_peak(peaks, clk)  # burst figure at the sampled clock
     t_tensor, t_mem = f / (peak_tc * 1e12), b / (peaks["hbm_gbs"] * 1e9)
     if t_mem > t_tensor:
         roofline = {"bound": "hbm", "achieved": b / t / 1e9, "peak": peaks["hbm_gbs"],
@@ -598,11 +789,13 @@ def run_backward(args, cfg):
     roofline.update({
         "traffic": None,
         "kernel": "bwd_gemm_kernel<weight gradient> (tcgen05, TMA store / add-reduce epilogue)",
-        "peak_source": f"{peak_src}: MEASURED_PEAKS.json (bf16 sustained, HBM copy)",
+        "peak_source": f"{peak_src}: MEASURED_PEAKS.json bf16_tflops (burst) x sampled clock "
+                       f"ratio {scale:.3f}; HBM copy hbm_gbs",
+        "clock_scale": scale,
         "per_launch": {"flops": f / n_wg, "bytes": b / n_wg, "ms": t * 1e3 / n_wg,
                        "roofline_ms": max(t_tensor, t_mem) * 1e3 / n_wg},
-        "tensor_frac": f / t / 1e12 / peak_tc,
         "tensor_frac_of_burst": f / t / 1e12 / peaks["bf16_tflops"],
+        "tensor_frac_of_sustained": f / t / 1e12 / peaks["bf16_tflops_sustained"],
         "hbm_frac": b / t / 1e9 / peaks["hbm_gbs"]})
     gemm_fl = sum(v for k2, v in units["flops"].items())
     gemm_ms = sum(prof[k2]["ms"] for k2 in units["flops"]) / steps
@@ -692,6 +885,15 @@ def main():
                     help="fused dispatch: one GEMM sweep per chunk instead of per pair")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the workload's token count (small cases for profiling)")
+    ap.add_argument("--per-n", type=int, nargs="*", default=[1, 2, 4],
+                    help="chunk counts timed for the per_n object (each with the library's "
+                         "own dispatch choice)")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="time the headline case only (no per_n, isolated row kernels, "
+                         "timeline)")
+    ap.add_argument("--timeline", default="",
+                    help="write the launch timeline of one step (headline N and dispatch, "
+                         "N=1, and the separate dispatch at the headline N) to this JSON file")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

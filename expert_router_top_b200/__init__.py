@@ -43,6 +43,15 @@ class Shape(ctypes.Structure):
                 ("num_chunks", ctypes.c_int32), ("chunk_size", ctypes.c_int32)]
 
 
+class LaunchRecord(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("stream", ctypes.c_int32), ("call", ctypes.c_int64),
+                ("rows", ctypes.c_int64), ("start_ms", ctypes.c_double),
+                ("end_ms", ctypes.c_double)]
+
+
+STREAM_NAMES = ("caller", "side", "copy_in", "copy_out")
+
+
 class Profile(ctypes.Structure):
     _fields_ = [("launches", ctypes.c_int64 * _NK), ("ms", ctypes.c_double * _NK),
                 ("rows", ctypes.c_int64 * _NK), ("active_experts", ctypes.c_int64 * _NK),
@@ -116,6 +125,8 @@ def load():
     L.moe_profile_enable.restype = st
     L.moe_profile_read.argtypes = [ctypes.POINTER(Profile)]
     L.moe_profile_read.restype = st
+    L.moe_profile_timeline.argtypes = [ctypes.POINTER(LaunchRecord), i32, ctypes.POINTER(i32)]
+    L.moe_profile_timeline.restype = st
     _lib = L
     return L
 
@@ -468,3 +479,14 @@ def profile_read() -> dict:
     return {kind: dict(launches=int(p.launches[i]), ms=float(p.ms[i]), rows=int(p.rows[i]),
                        active_experts=int(p.active_experts[i]))
             for i, kind in enumerate(KERNEL_KINDS)} | {"kernels": int(p.kernels)}
+
+
+def profile_timeline(capacity: int = 65536) -> list:
+    """The timed launches since profile_enable, in enqueue order: kind, stream, call index,
+    rows and start/end times in ms (CUDA events on the launching stream)."""
+    recs = (LaunchRecord * capacity)()
+    n = ctypes.c_int32(0)
+    _check(load().moe_profile_timeline(recs, capacity, ctypes.byref(n)), "moe_profile_timeline")
+    return [dict(kind=KERNEL_KINDS[r.kind], stream=STREAM_NAMES[r.stream], call=int(r.call),
+                 rows=int(r.rows), start_ms=float(r.start_ms), end_ms=float(r.end_ms))
+            for r in recs[:min(n.value, capacity)]]

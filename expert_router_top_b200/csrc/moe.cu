@@ -299,13 +299,21 @@ struct ProfRec {
   cudaEvent_t a, b;
   int64_t rows, active;
   int kernels;
+  int stream_id;  // 0 the caller's stream, 1 the library's side stream, 2 copy-in, 3 copy-out
+  int64_t call;   // library call (since moe_profile_enable) that launched the kernel
 };
+
+constexpr size_t kTimelineCap = 65536;  // launch records kept for moe_profile_timeline
 
 struct Prof {
   bool on = false;
   std::vector<ProfRec> pending;
   std::vector<cudaEvent_t> pool;
   moe_profile_t tot{};
+  cudaEvent_t origin = nullptr;  // recorded before the first timed launch since enable
+  bool origin_set = false;
+  int64_t calls = 0;
+  std::vector<moe_launch_record_t> timeline;
 } g_prof;
 
 cudaEvent_t prof_event() {
@@ -319,6 +327,23 @@ cudaEvent_t prof_event() {
   return e;
 }
 
+int prof_stream_id(cudaStream_t s) {
+  for (const DeviceCtx& c : g_ctx) {
+    if (!c.ready) continue;
+    if (s == c.side) return 1;
+    if (s == c.copy_in) return 2;
+    if (s == c.copy_out) return 3;
+  }
+  return 0;
+}
+
+// One library call: numbers the launch records of the call (for the timeline).
+struct ProfCall {
+  ProfCall() {
+    if (g_prof.on) ++g_prof.calls;
+  }
+};
+
 struct ProfScope {
   bool on;
   ProfRec r;
@@ -330,6 +355,13 @@ struct ProfScope {
     r.rows = rows;
     r.active = active;
     r.kernels = kernels;
+    r.stream_id = prof_stream_id(st);
+    r.call = g_prof.calls;
+    if (!g_prof.origin_set) {
+      if (!g_prof.origin) g_prof.origin = prof_event();
+      cudaEventRecord(g_prof.origin, s);
+      g_prof.origin_set = true;
+    }
     r.a = prof_event();
     r.b = prof_event();
     cudaEventRecord(r.a, s);
@@ -582,6 +614,7 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
                             const void* W_gate_up, const void* W_down, void* out,
                             void* workspace, size_t ws_bytes, uint32_t flags, void* stream) {
   NvtxRange range("moe_forward");
+  ProfCall prof_call;
   moe_status_t st = check_shape(shape);
   if (st != MOE_OK) return st;
   const int32_t choice = moe_forward_dispatch(shape, flags);
@@ -751,6 +784,7 @@ moe_status_t moe_forward_host(const moe_shape_t* shape, const void* hidden_host,
                               const void* W_gate_up, const void* W_down, void* out_host,
                               void* workspace, size_t ws_bytes, void* stream) {
   NvtxRange range("moe_forward_host");
+  ProfCall prof_call;
   return moe_forward_host_impl(shape, hidden_host, top_k_index_host, top_k_weights_host,
                                W_gate_up, W_down, out_host, workspace, ws_bytes, stream);
 }
@@ -999,6 +1033,7 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
                           void* d_hidden, float* d_weights, float* dW_gate_up, float* dW_down,
                           void* workspace, size_t ws_bytes, void* stream) {
   NvtxRange range("moe_backward");
+  ProfCall prof_call;
   moe_status_t st = check_bwd_shape(shape);
   if (st != MOE_OK) return st;
   const int64_t T = shape->T;
@@ -1326,27 +1361,64 @@ moe_status_t moe_profile_enable(int32_t on) {
   }
   g_prof.pending.clear();
   g_prof.tot = moe_profile_t{};
+  g_prof.timeline.clear();
+  g_prof.origin_set = false;
+  g_prof.calls = 0;
   g_prof.on = on != 0;
+  return MOE_OK;
+}
+
+// Folds the pending event pairs into the totals and the kept launch records.
+static moe_status_t prof_collect() {
+  if (g_prof.pending.empty()) return MOE_OK;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  for (auto& r : g_prof.pending) {
+    float ms = 0.f, t0 = 0.f, t1 = 0.f;
+    if (cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess ||
+        cudaEventElapsedTime(&t0, g_prof.origin, r.a) != cudaSuccess ||
+        cudaEventElapsedTime(&t1, g_prof.origin, r.b) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    g_prof.tot.launches[r.kind] += 1;
+    g_prof.tot.ms[r.kind] += ms;
+    g_prof.tot.rows[r.kind] += r.rows;
+    g_prof.tot.active_experts[r.kind] += r.active;
+    g_prof.tot.kernels += r.kernels;
+    if (g_prof.timeline.size() < kTimelineCap) {
+      moe_launch_record_t t;
+      t.kind = r.kind;
+      t.stream = r.stream_id;
+      t.call = r.call;
+      t.rows = r.rows;
+      t.start_ms = t0;
+      t.end_ms = t1;
+      g_prof.timeline.push_back(t);
+    }
+    g_prof.pool.push_back(r.a);
+    g_prof.pool.push_back(r.b);
+  }
+  g_prof.pending.clear();
   return MOE_OK;
 }
 
 moe_status_t moe_profile_read(moe_profile_t* out) {
   if (!out) return MOE_ERR_ARG;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_prof.pending.empty() && cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
-  for (auto& r : g_prof.pending) {
-    float ms = 0.f;
-    if (cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) return MOE_ERR_CUDA;
-    g_prof.tot.launches[r.kind] += 1;
-    g_prof.tot.ms[r.kind] += ms;
-    g_prof.tot.rows[r.kind] += r.rows;
-    g_prof.tot.active_experts[r.kind] += r.active;
-    g_prof.tot.kernels += r.kernels;
-    g_prof.pool.push_back(r.a);
-    g_prof.pool.push_back(r.b);
-  }
-  g_prof.pending.clear();
+  moe_status_t st = prof_collect();
+  if (st != MOE_OK) return st;
   *out = g_prof.tot;
+  return MOE_OK;
+}
+
+moe_status_t moe_profile_timeline(moe_launch_record_t* records, int32_t capacity,
+                                  int32_t* count) {
+  if (!count || capacity < 0 || (capacity > 0 && !records)) return MOE_ERR_ARG;
+  std::lock_guard<std::mutex> lock(g_mu);
+  moe_status_t st = prof_collect();
+  if (st != MOE_OK) return st;
+  const size_t n = g_prof.timeline.size();
+  const size_t m = n < (size_t)capacity ? n : (size_t)capacity;
+  if (m) memcpy(records, g_prof.timeline.data(), sizeof(moe_launch_record_t) * m);
+  *count = (int32_t)n;
   return MOE_OK;
 }
 

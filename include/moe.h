@@ -412,6 +412,30 @@ typedef struct {
 MOE_API moe_status_t moe_profile_enable(int32_t on);  /* also clears the totals */
 MOE_API moe_status_t moe_profile_read(moe_profile_t* out);
 
+/* One timed launch, for a timeline of the two-stream pipeline (the article's section
+ * 一张专业时序图 draws Expert(c) beside the dispatch/combine of the neighbouring chunk; these
+ * records show which kernels of a call actually ran side by side). */
+typedef struct {
+  int32_t kind;     /* moe_kernel_kind_t                                                    */
+  int32_t stream;   /* 0 the caller's stream, 1 the library's second stream,
+                       2 / 3 the copy-in / copy-out streams of moe_forward_host             */
+  int64_t call;     /* 1-based index of the library call, since moe_profile_enable, that
+                       launched it (moe_forward, moe_forward_host, moe_backward; 0 others)   */
+  int64_t rows;     /* as moe_profile_t.rows                                                */
+  double start_ms;  /* event times in ms, relative to an event recorded on the first timed
+                       launch's stream just before it; events of the other streams may
+                       precede it (negative)                                                */
+  double end_ms;
+} moe_launch_record_t;
+
+/* Synchronizes the device like moe_profile_read, folds the pending launches into the totals
+ * and the kept records (the first 65536 since moe_profile_enable), copies up to `capacity`
+ * records (host array, caller-owned) in enqueue order and sets *count to the number kept.
+ * MOE_ERR_ARG for a null count, a negative capacity or a null array with capacity > 0;
+ * MOE_ERR_CUDA if the device or an event query fails. */
+MOE_API moe_status_t moe_profile_timeline(moe_launch_record_t* records, int32_t capacity,
+                                          int32_t* count);
+
 #ifdef __cplusplus
 }
 #endif

@@ -291,3 +291,20 @@ def test_checks_api_in_the_regular_build():
     L = moe.load()
     assert L.moe_checks_enabled() == 0
     assert L.moe_checks_read(None) == 1  # null flags
+
+
+def test_profile_timeline_argument_checks_and_empty_list():
+    """With nothing timed the timeline call touches no device: it returns zero records;
+    a null count, a negative capacity or a null array with room are MOE_ERR_ARG."""
+    L = moe.load()
+    moe.profile_enable(True)
+    n = ctypes.c_int32(-1)
+    recs = (moe.LaunchRecord * 4)()
+    assert L.moe_profile_timeline(recs, 4, ctypes.byref(n)) == 0 and n.value == 0
+    assert L.moe_profile_timeline(None, 0, ctypes.byref(n)) == 0 and n.value == 0
+    assert L.moe_profile_timeline(recs, 4, None) == 1
+    assert L.moe_profile_timeline(recs, -1, ctypes.byref(n)) == 1
+    assert L.moe_profile_timeline(None, 4, ctypes.byref(n)) == 1
+    assert moe.profile_timeline() == []
+    moe.profile_enable(False)
+    assert ctypes.sizeof(moe.LaunchRecord) == 40

@@ -50,31 +50,54 @@ def test_traffic_reported_only_for_the_captured_launch(monkeypatch):
     assert bench.traffic_per_launch("qwen3", 4, "fused", True) is None
 
 
-class _DoneProc:
-    def terminate(self):
-        pass
-
-    def wait(self, timeout=None):
-        return 0
-
-
 def test_clock_summary_keeps_only_the_timed_window():
-    """nvidia-smi lines (index, sm, max sm, power, active mask, hw, hw thermal, sw thermal,
-    sw power cap): only samples inside the timed region (plus 0.1 s) count; the median SM
-    clock and every active reason among them are reported."""
-    s = bench.ClockSampler(0)
-    s.proc = _DoneProc()
-    ok = "0, {}, 1965, 900, 0x4, Not Active, Not Active, Not Active, {}"
-    s.lines = [(0.5, ok.format(700, "Not Active")),      # before the region
-               (1.0, ok.format(1400, "Active")),
-               (1.2, ok.format(1500, "Not Active")),
-               (1.4, ok.format(1450, "Active")),
-               (1.55, ok.format(1300, "Not Active")),    # within the 0.1 s grace
-               (3.0, "0, 600, 1965, 90, 0x1, Active, Not Active, Not Active, Not Active"),
-               (3.1, "garbage")]
-    out = s.stop(1.0, 1.5)
-    assert out == {"sm_mhz": 1425.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
-                   "samples": 4}
-    s.proc = _DoneProc()
-    every = s.stop()
+    """Samples (host time, SM MHz, max SM MHz, reasons): only those inside the timed region
+    (plus one sampling period) count; the median SM clock and every reason among them are
+    reported; with too few samples inside, the window widens back to the untimed steps
+    just before the region, and says so."""
+    s = bench.ClockSampler(0, period_s=0.05)
+    s.source = "test"
+    s.samples = [(0.5, 700.0, 1965.0, set()),                 # before the region
+                 (1.0, 1400.0, 1965.0, {"sw_power_cap"}),
+                 (1.2, 1500.0, 1965.0, set()),
+                 (1.4, 1450.0, 1965.0, {"sw_power_cap"}),
+                 (1.54, 1300.0, 1965.0, set()),               # within one period after it
+                 (3.0, 600.0, 1965.0, {"hw_slowdown"})]
+    out = s.summary(1.0, 1.5)
+    assert out["sm_mhz"] == 1425.0 and out["sm_max_mhz"] == 1965.0
+    assert out["reasons"] == ["sw_power_cap"] and out["samples"] == 4
+    assert out["sm_mhz_min"] == 1300.0 and out["window"] == "timed region"
+    narrow = s.summary(1.19, 1.21, min_samples=3, widen_to=0.4)
+    assert narrow["samples"] == 3 and narrow["window"].startswith("timed region and")
+    assert s.summary(1.19, 1.21, min_samples=1)["samples"] == 1
+    every = s.summary()
     assert every["samples"] == 6 and "hw_slowdown" in every["reasons"]
+    assert s.summary(5.0, 6.0) is None
+
+
+def test_tensor_peak_scales_the_burst_figure_by_the_sampled_clock():
+    peaks = {"bf16_tflops": 1679.8, "bf16_tflops_sustained": 1394.0, "hbm_gbs": 6549.4}
+    assert bench.tensor_peak(peaks, None) == (1679.8, 1.0)
+    p, sc = bench.tensor_peak(peaks, {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0})
+    assert (p, sc) == (1679.8, 1.0)
+    p, sc = bench.tensor_peak(peaks, {"sm_mhz": 1310.0, "sm_max_mhz": 1965.0})
+    assert sc == pytest.approx(2 / 3) and p == pytest.approx(1679.8 * 2 / 3)
+
+
+def test_gemm_roofline_reproduces_from_its_per_launch_figures():
+    """frac = per_launch.flops / per_launch.ms / (burst x clock ratio), for a tensor-bound
+    gate/up launch (two launches per step, 4 steps)."""
+    cfg = LayerConfig("u", T=16384, H=2048, E=128, k=8, I=768, routing="normal")
+    counts = np.full((2, 128), 512, np.int32)
+    units = bench.algorithmic_units(cfg, counts, 4, "fused", True)
+    peaks = {"bf16_tflops": 1679.8, "bf16_tflops_sustained": 1394.0, "hbm_gbs": 6549.4}
+    m = {"units": units, "steps": 4, "dispatch": "fused",
+         "prof": {"gateup": {"launches": 8, "ms": 8 * 0.4}},
+         "clk": {"sm_mhz": 1800.0, "sm_max_mhz": 1965.0}}
+    r = bench.gemm_roofline(m, peaks, "measured")
+    pl = r["per_launch"]
+    assert r["bound"] == "tensor"
+    assert pl["flops"] == pytest.approx(4.0 * 65536 * 2048 * 768)
+    want = pl["flops"] / (pl["ms"] / 1e3) / 1e12 / (1679.8 * 1800 / 1965)
+    assert r["frac"] == pytest.approx(want)
+    assert r["tensor_frac_of_burst"] == pytest.approx(want * 1800 / 1965)

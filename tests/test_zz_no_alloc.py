@@ -103,3 +103,16 @@ def test_noalloc_rejects_sizes_beyond_the_array(moe, lib):
     st = lib.moe_metadata_noalloc(_p(idx), 600, 2, 8, 1, 1, _p(n), _p(n), _p(n), _p(n), None,
                                   None, None)
     assert st == MOE_ERR_ARG
+
+
+def test_noalloc_defaults_and_empty_input(moe, lib):
+    """num_chunks=0 (no split) and ep_groups=0 (one group) resolve as moe_metadata resolves
+    them, and T=0 returns zero splits, counts and chunk bounds."""
+    cfg = CONFIGS["edge"]
+    idx = torch.from_numpy(routing(cfg)[0]).cuda()
+    _same_as_workspace_version(moe, idx, cfg.E, 0, 0)
+    _same_as_workspace_version(moe, idx, cfg.E, 0, 3)
+    _same_as_workspace_version(moe, idx, cfg.E, 4, 0)
+    empty = torch.zeros((0, cfg.k), dtype=torch.int32, device="cuda")
+    for G, N in ((0, 0), (4, 3)):
+        _same_as_workspace_version(moe, empty, cfg.E, G, N)
