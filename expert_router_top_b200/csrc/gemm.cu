@@ -57,6 +57,9 @@
 #ifndef MOE_GEMM_BAND
 #define MOE_GEMM_BAND 16  // M tiles per raster band: an expert's A rows stay in L2 across N tiles
 #endif
+#ifndef MOE_GEMM_TWO_M
+#define MOE_GEMM_TWO_M 0  // 256-row tiles of two 128-row sub-tiles: bit 0 gate/up, bit 1 down
+#endif
 #ifndef MOE_GEMM_B_POLICY
 #define MOE_GEMM_B_POLICY 2  // L2 policy of weight loads: 0 normal, 1 evict_first, 2 evict_last
 #endif
@@ -71,18 +74,33 @@ constexpr int kRowsPerCta = 128;            // accumulator rows per CTA (TMEM la
 constexpr uint32_t kTmemCols = 2 * BN;      // two accumulators of BN fp32 columns
 constexpr int kMaxE = 1024;
 
-// Geometry of one variant: single CTA (128x256 tiles) or CTA pair (256x256 tiles, each
-// CTA staging its 128 A rows and half of the 256 B rows).
-template <bool kPair>
+#ifndef MOE_GEMM_EPI_WARPS_2M
+#define MOE_GEMM_EPI_WARPS_2M 8  // epilogue warps of the two-sub-tile kernel: 4 or 8
+#endif
+#ifndef MOE_GEMM_STAGES_2M
+#define MOE_GEMM_STAGES_2M 3  // ring depth of the two-sub-tile kernel (64 KB stages)
+#endif
+
+// Geometry of one variant: single CTA with one 128-row A tile (128x256 tiles), single CTA
+// with two 128-row A sub-tiles sharing each B tile (kTwoM, 256x256 tiles: two TMEM
+// accumulators, one per sub-tile), or CTA pair (256x256 tiles, each CTA staging its 128 A
+// rows and half of the 256 B rows).
+template <bool kPair, bool kTwoM = false>
 struct Geo {
-  static constexpr int kTileM = kPair ? 2 * kRowsPerCta : kRowsPerCta;
-  static constexpr int kStages = kPair ? MOE_GEMM_STAGES_2SM : MOE_GEMM_STAGES;
+  static_assert(!(kPair && kTwoM), "two sub-tiles per CTA are a single-CTA variant");
+  static constexpr int kSubM = kTwoM ? 2 : 1;  // 128-row A sub-tiles staged per CTA
+  static constexpr int kTileM = kPair ? 2 * kRowsPerCta : kSubM * kRowsPerCta;
+  static constexpr int kStages =
+      kPair ? MOE_GEMM_STAGES_2SM : (kTwoM ? MOE_GEMM_STAGES_2M : MOE_GEMM_STAGES);
   static constexpr uint32_t kABytes = kRowsPerCta * BK * 2;                 // 16 KB
+  static constexpr uint32_t kAStageBytes = kSubM * kABytes;                 // 16 or 32 KB
   static constexpr uint32_t kBRows = kPair ? BN / 2 : BN;                   // B rows per CTA
   static constexpr uint32_t kBBytes = kBRows * BK * 2;                      // 16 or 32 KB
-  static constexpr uint32_t kStageBytes = kABytes + kBBytes;                // per CTA
+  static constexpr uint32_t kStageBytes = kAStageBytes + kBBytes;           // per CTA
   static constexpr uint32_t kTxBytes = kPair ? 2 * kStageBytes : kStageBytes;  // per stage
-  static constexpr uint32_t kIdesc = umma_idesc_bf16_f32(kTileM, BN);
+  static constexpr uint32_t kIdesc = umma_idesc_bf16_f32(kPair ? 2 * kRowsPerCta : kRowsPerCta, BN);
+  // epilogue warps: kTwoM may use two per TMEM lane quarter (each takes half the columns)
+  static constexpr int kEpiWarps = kTwoM ? MOE_GEMM_EPI_WARPS_2M : 4;
 };
 
 struct KParams {
@@ -115,11 +133,12 @@ struct SmemCtl {
   int abort;
 };
 
-// Threads of one CTA: producer, MMA, 4 epilogue warps; + 4 gathering warps (gathered A).
-template <bool kGather>
+// Threads of one CTA: producer, MMA, the epilogue warps; + 4 gathering warps (gathered A).
+template <bool kGather, bool kTwoM = false>
 __host__ __device__ constexpr int gemm_threads() {
-  return kGemmThreads + (kGather ? kGatherThreads : 0);
+  return 64 + 32 * Geo<false, kTwoM>::kEpiWarps + (kGather ? kGatherThreads : 0);
 }
+static_assert(gemm_threads<false>() == kGemmThreads, "thread layout");
 
 constexpr size_t kCtlBytes = 256;
 static_assert(sizeof(SmemCtl<MOE_GEMM_STAGES_2SM>) <= kCtlBytes, "control block");
@@ -132,11 +151,14 @@ constexpr int kEpiRowBytes = 80;
 constexpr int kEpiWarpBytes = 32 * kEpiRowBytes;
 constexpr size_t kTablesBytes = (2 * (kMaxE + 1) * sizeof(int32_t) + 15) & ~size_t(15);
 
-template <bool kPair>
+template <bool kPair, bool kTwoM = false>
 constexpr size_t smem_bytes() {
-  return 1024 /*alignment slack*/ + Geo<kPair>::kStages * Geo<kPair>::kStageBytes + kCtlBytes +
-         kTablesBytes + (MOE_GEMM_EPI_STAGE ? 4 * kEpiWarpBytes : 0);
+  using G = Geo<kPair, kTwoM>;
+  return 1024 /*alignment slack*/ + G::kStages * G::kStageBytes + kCtlBytes + kTablesBytes +
+         (MOE_GEMM_EPI_STAGE ? G::kEpiWarps * kEpiWarpBytes : 0);
 }
+static_assert(smem_bytes<false, true>() <= 232448, "two-sub-tile kernel exceeds 227 KB");
+static_assert(sizeof(SmemCtl<MOE_GEMM_STAGES_2M>) <= kCtlBytes, "control block");
 
 // A tile: expert e, column tile n, row tile m of the expert's rows.
 struct Tile {
@@ -218,17 +240,29 @@ __device__ __forceinline__ void store_block(const uint32_t (&packed)[16], uint8_
 // stream.  In a pair, the even CTA ("leader") owns the full-stage barriers and the MMA
 // issue; both CTAs load their own halves, run their own epilogue on their own TMEM rows,
 // and report back to the leader.
-template <bool kSwiGLU, bool kPair, bool kGather>
+//
+// kTwoM (single CTA): a tile is 256 rows of one expert by one N tile, staged as two 128-row
+// A sub-tiles that share every B stage, each with its own 128 x 256 TMEM accumulator (the
+// two fill all 512 columns).  Per 64-wide K block the CTA loads 64 KB for twice the MMAs of
+// a 48 KB one-sub-tile stage, so the same shared memory holds 1.5x the MMA time in flight
+// and each SM pulls 2/3 of the bytes per flop.  A tile whose expert ends within its first
+// 128 rows has no second sub-tile (no load, no MMA, no epilogue).  With no second
+// accumulator to alternate with, the MMA warp starts a tile's first-sub-tile MMAs as soon
+// as the epilogue has read that accumulator, and holds back (up to kStages - 1 stages) the
+// second sub-tile's MMAs until the epilogue has read the other one.
+template <bool kSwiGLU, bool kPair, bool kGather, bool kTwoM>
 __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensorMap* tmB,
                                           const KParams& p) {
-  using G = Geo<kPair>;
+  using G = Geo<kPair, kTwoM>;
   constexpr int STAGES = G::kStages;
+  constexpr int kEpiWarps = G::kEpiWarps;
+  constexpr int kFirstGatherWarp = 2 + kEpiWarps;
   static_assert(!(kGather && kPair), "gathered A rows are implemented for single CTAs");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * G::kABytes;
+  uint8_t* sB = smem + STAGES * G::kAStageBytes;
   SmemCtl<STAGES>* ctl = reinterpret_cast<SmemCtl<STAGES>*>(smem + STAGES * G::kStageBytes);
   int32_t* off = reinterpret_cast<int32_t*>(smem + STAGES * G::kStageBytes + kCtlBytes);
   int32_t* tile_start = off + (kMaxE + 1);
@@ -251,7 +285,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&ctl->tfull[b], 1);
-      mbar_init(&ctl->tempty[b], (kPair ? 2 : 1) * 4 * 32);
+      mbar_init(&ctl->tempty[b], (kPair ? 2 : 1) * kEpiWarps * 32);
     }
     mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
@@ -300,6 +334,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   const uint32_t tmem_base = ctl->tmem_base;
   volatile int* abort = &ctl->abort;
 
+  // kTwoM: whether tile t has a second 128-row sub-tile (its expert has rows past the first)
+  auto has_m1 = [&](const Tile& t) {
+    return kTwoM && off[t.e + 1] - off[t.e] > t.m * G::kTileM + kRowsPerCta;
+  };
+
   if (warp == 0 && kGather) {
     // ---------------- weight producer, gathered A (lane 0) ----------------
     // The A rows of a stage come from the gathering warps (below); this lane arms the stage
@@ -336,16 +375,18 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
         for (int s = 0; s < STAGES; ++s)
           if (armed & (1u << s)) mbar_drain(&ctl->full[s], (armed_parity >> s) & 1u, 100000000ull);
     }
-  } else if (kGather && warp >= kGemmThreads / 32) {
+  } else if (kGather && warp >= kFirstGatherWarp) {
     // ---------------- A producers, gathered rows (4 warps, LSU) ----------------
-    // The tile's 128 A rows are the token rows src_tok[row] of `hidden`.  Per K block, lane
-    // (8 s + j) of gathering warp w copies 16-byte chunk j of rows 32 w + 4 i + s (i < 8) with
-    // cp.async, into the 128-byte-swizzled K-major layout the MMA reads (chunk j of row r at
-    // position j ^ (r % 8)); a warp instruction covers 4 whole 128-byte row segments.  A
-    // thread keeps kDepth + 1 stages of copies in flight; when its oldest stage has landed it
-    // makes the writes visible to the async proxy and arrives on that stage's full barrier.
-    constexpr int kDepth = STAGES - 2;
-    const int gw = warp - kGemmThreads / 32, j = lane & 7, sub = lane >> 3;
+    // The tile's A rows are the token rows src_tok[row] of `hidden`.  Per K block, lane
+    // (8 s + j) of gathering warp w copies 16-byte chunk j of rows 32 w + 4 i + s (i < 8) of
+    // each 128-row sub-tile with cp.async, into the 128-byte-swizzled K-major layout the MMA
+    // reads (chunk j of row r at position j ^ (r % 8)); a warp instruction covers 4 whole
+    // 128-byte row segments.  A thread keeps kDepth + 1 stages of copies in flight; when
+    // its oldest stage has landed it makes the writes visible to the async proxy and
+    // arrives on that stage's full barrier.
+    constexpr int kDepth = STAGES - 2 > 0 ? STAGES - 2 : 1;
+    constexpr int kSub = G::kSubM;
+    const int gw = warp - kFirstGatherWarp, j = lane & 7, sub = lane >> 3;
     int stage = 0;
     uint32_t phase = 0;
     int32_t issued = 0, arrived = 0;
@@ -355,25 +396,34 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       const int32_t* gat = p.gather;  // gathered A has one row segment
       const int32_t row0 = off[t.e] + t.m * G::kTileM;
       const int32_t last = off[t.e + 1] - 1;  // rows past the expert re-read its last row
-      const uint8_t* src[8];
+      const int n_sub = has_m1(t) ? 2 : 1;
+      const uint8_t* src[kSub * 8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int32_t r = gw * 32 + 4 * i + sub;
-        int64_t tok = gat[min(row0 + r, last)];
-        if (!check_row(tok, p.gsrc_rows, &g_range_flags)) tok = 0;
-        src[i] = p.gsrc + tok * p.gsrc_stride + j * 16;
-      }
+      for (int h = 0; h < kSub; ++h)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int32_t r = h * kRowsPerCta + gw * 32 + 4 * i + sub;
+          int64_t tok = gat[min(row0 + r, last)];
+          if (!check_row(tok, p.gsrc_rows, &g_range_flags)) tok = 0;
+          src[h * 8 + i] = p.gsrc + tok * p.gsrc_stride + j * 16;
+        }
       for (int32_t kb = 0; kb < p.num_kb; ++kb) {
         if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort, p.status)) {
           ok = false;
           break;
         }
-        const uint32_t a = smem_u32(sA + stage * G::kABytes);
+        const uint32_t a = smem_u32(sA + stage * G::kAStageBytes);
         const uint32_t nbytes = (kb * BK + j * 8 < p.K) ? 16u : 0u;  // zero past K
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int32_t r = gw * 32 + 4 * i + sub;
-          cp_async_16(a + r * (BK * 2) + ((j ^ (r & 7)) << 4), src[i] + kb * (BK * 2), nbytes);
+        for (int h = 0; h < kSub; ++h) {
+          if (h < n_sub) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int32_t r = gw * 32 + 4 * i + sub;
+              cp_async_16(a + h * G::kABytes + r * (BK * 2) + ((j ^ (r & 7)) << 4),
+                          src[h * 8 + i] + kb * (BK * 2), nbytes);
+            }
+          }
         }
         cp_async_commit();
         ++issued;
@@ -413,13 +463,15 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
             kSwiGLU  // pair: the even CTA stages the gate rows, the odd one the up rows
                 ? t.e * p.b_rows + t.n * (BN / 2) + (kPair ? (int32_t)rank * p.up_off : 0)
                 : t.e * p.b_rows + t.n * BN + (kPair ? (int32_t)rank * (BN / 2) : 0);
+        const bool m1 = has_m1(t);
+        const uint32_t tx = kTwoM ? (m1 ? G::kStageBytes : G::kABytes + G::kBBytes) : G::kTxBytes;
         const CUtensorMap* mapA = tmA;
         for (int32_t kb = 0; kb < p.num_kb; ++kb) {
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort, p.status)) {
             ok = false;
             break;
           }
-          uint8_t* a_dst = sA + stage * G::kABytes;
+          uint8_t* a_dst = sA + stage * G::kAStageBytes;
           uint8_t* b_dst = sB + stage * G::kBBytes;
           if (kPair) {
             if (leader) mbar_arrive_expect_tx(&ctl->full[stage], G::kTxBytes);
@@ -427,8 +479,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
             tma_load_2d_pair(a_dst, mapA, bar, kb * BK, row0, pol_a);
             tma_load_2d_pair(b_dst, tmB, bar, kb * BK, brow, pol_w);
           } else {
-            mbar_arrive_expect_tx(&ctl->full[stage], G::kTxBytes);
+            mbar_arrive_expect_tx(&ctl->full[stage], tx);
             tma_load_2d(a_dst, mapA, &ctl->full[stage], kb * BK, row0, pol_a);
+            if (kTwoM && m1)
+              tma_load_2d(a_dst + G::kABytes, mapA, &ctl->full[stage], kb * BK,
+                          row0 + kRowsPerCta, pol_a);
             if (kSwiGLU) {
               tma_load_2d(b_dst, tmB, &ctl->full[stage], kb * BK, brow, pol_w);
               tma_load_2d(b_dst + G::kBBytes / 2, tmB, &ctl->full[stage], kb * BK,
@@ -449,6 +504,90 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
         // wait (bounded) for the copies already issued, so none lands after exit
         for (int s = 0; s < STAGES; ++s)
           if (armed & (1u << s)) mbar_drain(&ctl->full[s], (armed_parity >> s) & 1u, 100000000ull);
+      }
+    }
+  } else if (warp == 1 && kTwoM) {
+    // ---------------- MMA issuer, two sub-tiles per tile ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t use[2] = {0, 0};  // tiles that used accumulator 0 / 1 so far
+      bool ok = true, issued = false;
+      auto mma_sub = [&](int h, int st, int32_t kb) {
+        const uint32_t a_addr = smem_u32(sA + st * G::kAStageBytes + h * G::kABytes);
+        const uint32_t b_addr = smem_u32(sB + st * G::kBBytes);
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          const uint64_t ad = kmajor_desc<kSwizzleBytes>(a_addr + kk * 32);
+          const uint64_t bd = kmajor_desc<kSwizzleBytes>(b_addr + kk * 32);
+          umma_bf16(tmem_base + h * BN, ad, bd, G::kIdesc, (kb | kk) != 0);
+        }
+      };
+      for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
+        const Tile t = decode_tile<G::kTileM>(L, tile_start, off, E, p.n_tiles);
+        const bool m1 = has_m1(t);
+        if (!mbar_wait(&ctl->tempty[0], (use[0] & 1u) ^ 1u, abort, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        bool acc1 = false;        // accumulator 1 read out by the epilogue, this tile
+        int pend_stage[STAGES];   // stages whose second-sub-tile MMAs wait for accumulator 1
+        int32_t pend_kb[STAGES];
+        int npend = 0;
+        for (int32_t kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(&ctl->full[stage], phase, abort, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          mma_sub(0, stage, kb);
+          issued = true;
+          if (kb == p.num_kb - 1) umma_commit(&ctl->tfull[0]);
+          if (m1) {
+            if (!acc1) {
+              acc1 = mbar_test_wait(&ctl->tempty[1], (use[1] & 1u) ^ 1u);
+              if (!acc1 && (npend == STAGES - 1 || kb == p.num_kb - 1)) {
+                if (!mbar_wait(&ctl->tempty[1], (use[1] & 1u) ^ 1u, abort, p.status)) {
+                  ok = false;
+                  break;
+                }
+                acc1 = true;
+              }
+              if (acc1) tc_fence_after();
+            }
+            if (acc1) {
+              for (int i = 0; i < npend; ++i) {
+                mma_sub(1, pend_stage[i], pend_kb[i]);
+                umma_commit(&ctl->empty[pend_stage[i]]);
+              }
+              npend = 0;
+              mma_sub(1, stage, kb);
+              umma_commit(&ctl->empty[stage]);
+            } else {
+              pend_stage[npend] = stage;
+              pend_kb[npend] = kb;
+              ++npend;
+            }
+          } else {
+            umma_commit(&ctl->empty[stage]);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        ++use[0];
+        if (m1) {
+          umma_commit(&ctl->tfull[1]);
+          ++use[1];
+        }
+      }
+      if (!ok && issued) {
+        // every MMA issued so far must finish before TMEM is released
+        umma_commit(&ctl->drain);
+        mbar_drain(&ctl->drain, 0, 100000000ull);
       }
     }
   } else if (warp == 1) {
@@ -473,7 +612,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(sA + stage * G::kABytes);
+          const uint32_t a_addr = smem_u32(sA + stage * G::kAStageBytes);
           const uint32_t b_addr = smem_u32(sB + stage * G::kBBytes);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
@@ -502,66 +641,86 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
         mbar_drain(&ctl->drain, 0, 100000000ull);
       }
     }
-  } else if (warp < kGemmThreads / 32) {
-    // ---------------- epilogue (warps 2..5 of both CTAs) ----------------
+  } else if (warp < 2 + kEpiWarps) {
+    // ---------------- epilogue (warps 2 .. 2 + kEpiWarps - 1 of both CTAs) ----------------
+    // Warp w reads TMEM lanes 32 (w % 4) .. +31 (the lane quarter its SM sub-partition may
+    // access).  kTwoM: two warps per quarter, each taking half of the column chunks; the
+    // tile's accumulators are read one after the other (sub-tile 0, then 1).
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int r = q * 32 + lane;
+    constexpr int kParts = kEpiWarps / 4;  // warps sharing one lane quarter
+    const int half = kParts > 1 ? (warp - 2) / 4 : 0;
     uint8_t* wbuf = epi_stage + (warp - 2) * kEpiWarpBytes;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&ctl->tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&ctl->tempty[1]), 0);
+    uint32_t use[2] = {0, 0};
     int32_t it = 0;
-    for (int32_t L = stream_id; L < p.total_tiles; L += n_streams, ++it) {
-      const int buf = it & 1;
-      const uint32_t tphase = (it >> 1) & 1;
-      if (!mbar_wait(&ctl->tfull[buf], tphase, abort, p.status)) break;
-      tc_fence_after();
+    bool ok = true;
+    for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams, ++it) {
       const Tile t = decode_tile<G::kTileM>(L, tile_start, off, E, p.n_tiles);
-      const int32_t* offs = off;
-      __nv_bfloat16* out = p.out;
-      const int64_t out_rows = p.out_rows;
-      const int32_t first = t.m * G::kTileM + (int32_t)rank * kRowsPerCta;  // in the expert
-      const int32_t rows_valid = offs[t.e + 1] - offs[t.e] - first;
-      const bool row_ok = r < rows_valid;
-      const int64_t row_base = (int64_t)offs[t.e] + first;  // output row of TMEM lane 0
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * BN;
-      if (kSwiGLU) {
+      const int n_acc = has_m1(t) ? 2 : 1;
+      for (int h = 0; h < n_acc; ++h) {
+        // accumulator of this sub-tile: kTwoM h; otherwise alternating per tile
+        const int buf = kTwoM ? h : (it & 1);
+        const uint32_t tphase = kTwoM ? (use[h] & 1u) : ((it >> 1) & 1);
+        if (!mbar_wait(&ctl->tfull[buf], tphase, abort, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int32_t* offs = off;
+        __nv_bfloat16* out = p.out;
+        const int64_t out_rows = p.out_rows;
+        const int32_t first = t.m * G::kTileM + (int32_t)rank * kRowsPerCta + h * kRowsPerCta;
+        const int32_t rows_valid = offs[t.e + 1] - offs[t.e] - first;
+        const bool row_ok = r < rows_valid;
+        const int64_t row_base = (int64_t)offs[t.e] + first;  // output row of TMEM lane 0
+        const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * BN;
+        if (kSwiGLU) {
+          constexpr int kChunks = (BN / 2) / 32 / kParts;
 #pragma unroll 1
-        for (int c = 0; c < (BN / 2) / 32; ++c) {
-          uint32_t g[32], u[32];
-          tmem_ld_32cols(t_row + c * 32, g);
-          tmem_ld_32cols(t_row + BN / 2 + c * 32, u);
-          tmem_ld_wait2(g, u);
-          const int32_t col0 = t.n * (BN / 2) + c * 32;
-          uint32_t packed[16];
+          for (int c = half * kChunks; c < (half + 1) * kChunks; ++c) {
+            uint32_t g[32], u[32];
+            tmem_ld_32cols(t_row + c * 32, g);
+            tmem_ld_32cols(t_row + BN / 2 + c * 32, u);
+            tmem_ld_wait2(g, u);
+            const int32_t col0 = t.n * (BN / 2) + c * 32;
+            uint32_t packed[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
-            const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
-            // silu(g) = g / (1 + e^-g); the fast division (no IEEE slow path) is exact to a
-            // few ulp, far below the bf16 rounding of the result
-            const float a0 = __fdividef(g0, 1.0f + __expf(-g0)) * u0;
-            const float a1 = __fdividef(g1, 1.0f + __expf(-g1)) * u1;
-            packed[i] = pack_bf16x2(a0, a1);
+            for (int i = 0; i < 16; ++i) {
+              const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+              const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+              // silu(g) = g / (1 + e^-g); the fast division (no IEEE slow path) is exact to a
+              // few ulp, far below the bf16 rounding of the result
+              const float a0 = __fdividef(g0, 1.0f + __expf(-g0)) * u0;
+              const float a1 = __fdividef(g1, 1.0f + __expf(-g1)) * u1;
+              packed[i] = pack_bf16x2(a0, a1);
+            }
+            store_block(packed, wbuf, lane, q, row_ok, rows_valid, row_base, col0, p, out,
+                        out_rows);
           }
-          store_block(packed, wbuf, lane, q, row_ok, rows_valid, row_base, col0, p, out, out_rows);
-        }
-      } else {
+        } else {
+          constexpr int kChunks = BN / 32 / kParts;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t acc[32];
-          tmem_ld_32cols(t_row + c * 32, acc);
-          tmem_ld_wait(acc);
-          const int32_t col0 = t.n * BN + c * 32;
-          uint32_t packed[16];
+          for (int c = half * kChunks; c < (half + 1) * kChunks; ++c) {
+            uint32_t acc[32];
+            tmem_ld_32cols(t_row + c * 32, acc);
+            tmem_ld_wait(acc);
+            const int32_t col0 = t.n * BN + c * 32;
+            uint32_t packed[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            packed[i] = pack_bf16x2(__uint_as_float(acc[2 * i]), __uint_as_float(acc[2 * i + 1]));
-          store_block(packed, wbuf, lane, q, row_ok, rows_valid, row_base, col0, p, out, out_rows);
+            for (int i = 0; i < 16; ++i)
+              packed[i] =
+                  pack_bf16x2(__uint_as_float(acc[2 * i]), __uint_as_float(acc[2 * i + 1]));
+            store_block(packed, wbuf, lane, q, row_ok, rows_valid, row_base, col0, p, out,
+                        out_rows);
+          }
         }
+        tc_fence_before();
+        if (kPair) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
+        else mbar_arrive(&ctl->tempty[buf]);
+        ++use[h];
       }
-      tc_fence_before();
-      if (kPair) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
-      else mbar_arrive(&ctl->tempty[buf]);
     }
   }
 
@@ -576,12 +735,12 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   }
 }
 
-template <bool kSwiGLU, bool kGather>
-__global__ void __launch_bounds__(gemm_threads<kGather>(), 1)
+template <bool kSwiGLU, bool kGather, bool kTwoM>
+__global__ void __launch_bounds__(gemm_threads<kGather, kTwoM>(), 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
                         const KParams p) {
-  gemm_body<kSwiGLU, false, kGather>(&tmA, &tmB, p);
+  gemm_body<kSwiGLU, false, kGather, kTwoM>(&tmA, &tmB, p);
 }
 
 // Launched with a cluster of 2 CTAs (cudaLaunchAttributeClusterDimension).
@@ -590,7 +749,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmB,
                              const KParams p) {
-  gemm_body<kSwiGLU, true, false>(&tmA, &tmB, p);
+  gemm_body<kSwiGLU, true, false, false>(&tmA, &tmB, p);
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -650,9 +809,18 @@ bool make_tma_3d_f32(CUtensorMap* m, void* base, int32_t E, int32_t M, int32_t N
 
 bool gemm_supports_gather() { return MOE_GEMM_2SM == 0; }
 
+// Which single-CTA variant a GEMM kind runs: two 128-row sub-tiles per 256-row tile
+// (MOE_GEMM_TWO_M bit 0: gate/up, bit 1: down) or one 128-row tile.
+bool gemm_two_m(bool swiglu) {
+  if (MOE_GEMM_2SM != 0) return false;
+  return ((MOE_GEMM_TWO_M >> (swiglu ? 0 : 1)) & 1) != 0;
+}
+
 int64_t gemm_total_tiles(const int32_t* counts_host, int32_t E, int32_t out_cols, bool swiglu) {
   const int32_t bn = swiglu ? BN / 2 : BN;
-  const int32_t tm = Geo<MOE_GEMM_2SM != 0>::kTileM;
+  const int32_t tm = MOE_GEMM_2SM != 0 ? Geo<true>::kTileM
+                     : gemm_two_m(swiglu)  ? Geo<false, true>::kTileM
+                                           : Geo<false>::kTileM;
   const int64_t n_tiles = (out_cols + bn - 1) / bn;
   int64_t m_tiles = 0;
   for (int32_t e = 0; e < E; ++e) m_tiles += (counts_host[e] + tm - 1) / tm;
@@ -662,6 +830,7 @@ int64_t gemm_total_tiles(const int32_t* counts_host, int32_t E, int32_t out_cols
 cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cudaStream_t s,
                                 int* err_detail) {
   constexpr bool kPair = MOE_GEMM_2SM != 0;
+  const bool two_m = gemm_two_m(swiglu);
   *err_detail = 0;
   if (a.total_tiles <= 0) return cudaSuccess;
   if (a.total_tiles > 0x7fffffff || a.E > kMaxE) {
@@ -701,7 +870,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
   p.gsrc_rows = a.gather_src_rows;
   p.out_rows = a.rows;
   p.K = a.K;
-  constexpr size_t smem = smem_bytes<kPair>();
+  const size_t smem = two_m ? smem_bytes<false, true>() : smem_bytes<kPair>();
   cudaError_t e;
   if (kPair) {
     auto k = swiglu ? grouped_gemm_pair_kernel<true> : grouped_gemm_pair_kernel<false>;
@@ -735,12 +904,18 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
     e = cudaLaunchKernelEx(&cfg, k, mA, mB, p);
     if (e != cudaSuccess) return e;
   } else {
-    auto k = gather ? grouped_gemm_kernel<true, true>
-                    : (swiglu ? grouped_gemm_kernel<true, false> : grouped_gemm_kernel<false, false>);
+    auto k = two_m ? (gather ? grouped_gemm_kernel<true, true, true>
+                             : (swiglu ? grouped_gemm_kernel<true, false, true>
+                                       : grouped_gemm_kernel<false, false, true>))
+                   : (gather ? grouped_gemm_kernel<true, true, false>
+                             : (swiglu ? grouped_gemm_kernel<true, false, false>
+                                       : grouped_gemm_kernel<false, false, false>));
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int streams = (int)(a.total_tiles < num_sms ? a.total_tiles : num_sms);
-    k<<<streams, gather ? gemm_threads<true>() : gemm_threads<false>(), smem, s>>>(mA, mB, p);
+    const int threads = two_m ? (gather ? gemm_threads<true, true>() : gemm_threads<false, true>())
+                              : (gather ? gemm_threads<true>() : gemm_threads<false>());
+    k<<<streams, threads, smem, s>>>(mA, mB, p);
   }
   return cudaGetLastError();
 }
