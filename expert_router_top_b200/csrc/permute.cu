@@ -116,7 +116,85 @@ __global__ void __launch_bounds__(kRowThreads) unpermute_kernel(const uint4* __r
   }
 }
 
+// The same combine with k fixed at compile time: a warp issues the loads of all k rows'
+// 16-byte vectors before the first FMA, so k x 512 bytes per warp are in flight instead of
+// one row's, and loops over tokens (grid-stride) so that the grid can be sized to the GPU.
+// The arithmetic is the kernel's above: acc = 0, then acc = fma(w_j, y_j, acc) for
+// j = 0 .. k-1, so both give the same bits.
+template <int KT>
+__global__ void __launch_bounds__(kRowThreads) unpermute_k_kernel(const uint4* __restrict__ Y,
+                                                                  const int32_t* __restrict__ dst,
+                                                                  const float* __restrict__ w,
+                                                                  int64_t Tc, int32_t H8,
+                                                                  uint4* __restrict__ out,
+                                                                  int64_t rows_cap) {
+  const int lane = threadIdx.x & 31;
+  const int64_t n_warps = (int64_t)gridDim.x * kTokPerCta;
+  for (int64_t t = (int64_t)blockIdx.x * kTokPerCta + (threadIdx.x >> 5); t < Tc; t += n_warps) {
+    const int32_t d_lane = lane < KT ? dst[t * KT + lane] : 0;
+    const float w_lane = lane < KT ? w[t * KT + lane] : 0.f;
+    const uint4* row[KT];
+    float wj[KT];
+    bool ok[KT];
+#pragma unroll
+    for (int j = 0; j < KT; ++j) {
+      const int32_t d = __shfl_sync(0xffffffffu, d_lane, j);
+      wj[j] = __shfl_sync(0xffffffffu, w_lane, j);
+      ok[j] = check_row(d, rows_cap, &g_range_flags);
+      row[j] = Y + (int64_t)(ok[j] ? d : 0) * H8;
+    }
+    for (int32_t v = lane; v < H8; v += 32) {
+      uint4 y[KT];
+#pragma unroll
+      for (int j = 0; j < KT; ++j) y[j] = ldg_stream(row[j] + v);
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+      for (int j = 0; j < KT; ++j) {
+        if (!ok[j]) continue;
+        const uint32_t q[4] = {y[j].x, y[j].y, y[j].z, y[j].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[2 * i] = fmaf(wj[j], bf16lo(q[i]), acc[2 * i]);
+          acc[2 * i + 1] = fmaf(wj[j], bf16hi(q[i]), acc[2 * i + 1]);
+        }
+      }
+      uint4 o;
+      o.x = pack_bf16x2(acc[0], acc[1]);
+      o.y = pack_bf16x2(acc[2], acc[3]);
+      o.z = pack_bf16x2(acc[4], acc[5]);
+      o.w = pack_bf16x2(acc[6], acc[7]);
+      out[t * H8 + v] = o;
+    }
+  }
+}
+
 inline unsigned grid_for(int64_t Tc) { return (unsigned)((Tc + kTokPerCta - 1) / kTokPerCta); }
+
+#ifndef MOE_UNPERM_CTAS_PER_SM
+#define MOE_UNPERM_CTAS_PER_SM 4  // grid of the compile-time-k combine: CTAs per SM
+#endif
+
+int num_sms_cached() {
+  static int n[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int& v = n[dev & 63];
+  if (v <= 0 && cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    v = 148;
+  return v;
+}
+
+template <int KT>
+cudaError_t launch_unpermute_k(const void* Y, const int32_t* dst, const float* w, int64_t Tc,
+                               int32_t H, void* out, int64_t rows_cap, cudaStream_t s) {
+  const int64_t cap = (int64_t)num_sms_cached() * MOE_UNPERM_CTAS_PER_SM;
+  const int64_t need = grid_for(Tc);
+  unpermute_k_kernel<KT><<<(unsigned)(need < cap ? need : cap), kRowThreads, 0, s>>>(
+      static_cast<const uint4*>(Y), dst, w, Tc, H / 8, static_cast<uint4*>(out), rows_cap);
+  return cudaGetLastError();
+}
 
 }  // namespace
 
@@ -131,6 +209,16 @@ cudaError_t launch_permute(const void* hidden, const int32_t* dst, int64_t Tc, i
 cudaError_t launch_unpermute(const void* Y, const int32_t* dst, const float* w, int64_t Tc,
                              int32_t H, int32_t k, void* out, int64_t rows_cap, cudaStream_t s) {
   if (Tc <= 0) return cudaSuccess;
+#if MOE_UNPERM_CTAS_PER_SM > 0
+  switch (k) {
+    case 1: return launch_unpermute_k<1>(Y, dst, w, Tc, H, out, rows_cap, s);
+    case 2: return launch_unpermute_k<2>(Y, dst, w, Tc, H, out, rows_cap, s);
+    case 4: return launch_unpermute_k<4>(Y, dst, w, Tc, H, out, rows_cap, s);
+    case 6: return launch_unpermute_k<6>(Y, dst, w, Tc, H, out, rows_cap, s);
+    case 8: return launch_unpermute_k<8>(Y, dst, w, Tc, H, out, rows_cap, s);
+    default: break;
+  }
+#endif
   unpermute_kernel<2><<<grid_for(Tc), kRowThreads, 0, s>>>(
       static_cast<const uint4*>(Y), dst, w, Tc, H / 8, k, static_cast<uint4*>(out), rows_cap);
   return cudaGetLastError();
