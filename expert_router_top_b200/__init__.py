@@ -127,6 +127,18 @@ def load():
     L.moe_profile_read.restype = st
     L.moe_profile_timeline.argtypes = [ctypes.POINTER(LaunchRecord), i32, ctypes.POINTER(i32)]
     L.moe_profile_timeline.restype = st
+    L.moe_ep_plan.argtypes = [p, i32, i32, i32, p, p]
+    L.moe_ep_plan.restype = st
+    L.moe_ep_dispatch.argtypes = [p, p, p, p, p, i64, i32, i32, i32, i32, i64, p]
+    L.moe_ep_dispatch.restype = st
+    L.moe_ep_combine.argtypes = [p, p, p, p, p, i64, i32, i32, i32, i32, i64, p, p]
+    L.moe_ep_combine.restype = st
+    L.moe_ipc_handle.argtypes = [p, p, ctypes.POINTER(i64)]
+    L.moe_ipc_handle.restype = st
+    L.moe_ipc_open.argtypes = [p, i64, ctypes.POINTER(p)]
+    L.moe_ipc_open.restype = st
+    L.moe_ipc_close.argtypes = [p, i64]
+    L.moe_ipc_close.restype = st
     _lib = L
     return L
 
@@ -490,3 +502,64 @@ def profile_timeline(capacity: int = 65536) -> list:
     return [dict(kind=KERNEL_KINDS[r.kind], stream=STREAM_NAMES[r.stream], call=int(r.call),
                  rows=int(r.rows), start_ms=float(r.start_ms), end_ms=float(r.end_ms))
             for r in recs[:min(n.value, capacity)]]
+
+
+# ---- expert parallelism over several GPUs (see expert_router_top_b200.ep) -------------------
+
+def ep_plan(counts_all, rank: int):
+    """counts_all [W][E] int (one chunk's expert counts of every rank) -> (send_delta [E],
+    recv_offsets [E/W + 1]) as int32 numpy arrays (moe_ep_plan, host arithmetic)."""
+    c = np.ascontiguousarray(counts_all, dtype=np.int32)
+    W, E = c.shape
+    delta = np.zeros(E, np.int32)
+    offs = np.zeros(E // max(W, 1) + 1, np.int32)
+    _check(load().moe_ep_plan(_ptr(c), W, rank, E, _ptr(delta), _ptr(offs)), "moe_ep_plan")
+    return delta, offs
+
+
+def _ptr_table(ptrs, device):
+    """Device array of W raw device pointers (int64) for the EP kernels."""
+    return torch.tensor([int(x) for x in ptrs], dtype=torch.int64, device=device)
+
+
+def ep_dispatch(hidden, top_k_index, dst_rows, send_delta, recv_table, E: int, W: int,
+                rows_cap: int, stream=None):
+    """recv[rank(e)][dst + delta[e]] = hidden[t] for every copy of the chunk (moe_ep_dispatch).
+    recv_table: int64 device tensor of W receive-buffer pointers."""
+    _need(hidden, torch.bfloat16, "hidden")
+    Tc, H = hidden.shape
+    k = top_k_index.shape[1]
+    _check(load().moe_ep_dispatch(_ptr(hidden), _ptr(top_k_index), _ptr(dst_rows),
+                                  _ptr(send_delta), _ptr(recv_table), Tc, H, k, E, W, rows_cap,
+                                  _stream(stream)), "moe_ep_dispatch")
+
+
+def ep_combine(expert_table, top_k_index, dst_rows, send_delta, top_k_weights, H: int, E: int,
+               W: int, rows_cap: int, out=None, stream=None):
+    """out[t] = sum_j w[t,j] Y[rank(e)][dst + delta[e]], fp32 in ascending j (moe_ep_combine)."""
+    Tc, k = top_k_index.shape
+    if out is None:
+        out = torch.empty((Tc, H), dtype=torch.bfloat16, device=top_k_index.device)
+    _check(load().moe_ep_combine(_ptr(expert_table), _ptr(top_k_index), _ptr(dst_rows),
+                                 _ptr(send_delta), _ptr(top_k_weights), Tc, H, k, E, W, rows_cap,
+                                 _ptr(out), _stream(stream)), "moe_ep_combine")
+    return out
+
+
+def ipc_handle(t: torch.Tensor):
+    """(handle bytes, offset) of a device tensor's allocation, for ipc_open in another process."""
+    h = ctypes.create_string_buffer(64)
+    off = ctypes.c_int64(0)
+    _check(load().moe_ipc_handle(_ptr(t), h, ctypes.byref(off)), "moe_ipc_handle")
+    return h.raw, off.value
+
+
+def ipc_open(handle: bytes, offset: int) -> int:
+    """Device address of another process's buffer (moe_ipc_open)."""
+    out = ctypes.c_void_p(0)
+    _check(load().moe_ipc_open(handle, offset, ctypes.byref(out)), "moe_ipc_open")
+    return out.value
+
+
+def ipc_close(ptr: int, offset: int):
+    _check(load().moe_ipc_close(ctypes.c_void_p(ptr), offset), "moe_ipc_close")

@@ -12,7 +12,8 @@ LIB = os.path.join(PKG, "libmoe.so")
 LIB_CHECKS = os.path.join(PKG, "libmoe_checks.so")  # every row index range-checked
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
-SOURCES = ["metadata.cu", "permute.cu", "gemm.cu", "moe.cu", "noalloc.cu", "backward.cu", "selftest.cu"]
+SOURCES = ["metadata.cu", "permute.cu", "gemm.cu", "moe.cu", "noalloc.cu", "backward.cu", "selftest.cu",
+           "ep.cu"]
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",

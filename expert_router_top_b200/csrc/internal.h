@@ -48,6 +48,7 @@ cudaError_t launch_unpermute(const void* Y, const int32_t* dst, const float* w, 
 uint32_t checks_take_permute();
 uint32_t checks_take_gemm();
 uint32_t checks_take_backward();
+uint32_t checks_take_ep();
 
 // ---- grouped GEMM (gemm.cu) -------------------------------------------------------------
 

@@ -1272,7 +1272,8 @@ int32_t moe_checks_enabled(void) { return MOE_CHECKS ? 1 : 0; }
 moe_status_t moe_checks_read(uint32_t* flags) {
   if (!flags) return MOE_ERR_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
-  *flags = checks_take_permute() | checks_take_gemm() | checks_take_backward();
+  *flags = checks_take_permute() | checks_take_gemm() | checks_take_backward() |
+           checks_take_ep();
   return MOE_OK;
 }
 

@@ -381,6 +381,86 @@ MOE_API moe_status_t moe_checks_read(uint32_t* flags);
  * wait completed, MOE_ERR_ARG / MOE_ERR_ALIGN / MOE_ERR_CUDA otherwise. */
 MOE_API moe_status_t moe_selftest_wait_timeout(uint32_t* status, uint32_t limit_us, void* stream);
 
+/* ---- Expert parallelism over several GPUs ----------------------------------------------
+ * [ChunkMoE] "一张专业时序图" (per chunk: All-to-All dispatch, expert computation, All-to-All
+ * combine) and "操作指南" (expert_parallel_size): the E experts are split over W ranks, one
+ * GPU each; rank d owns experts [d*E/W, (d+1)*E/W).  Each rank routes its own tokens.  On
+ * NVLink/NVSwitch the exchange is fused into the row kernels: moe_ep_dispatch stores every
+ * token copy straight into its row of the owning rank's receive buffer (peer stores) and
+ * moe_ep_combine reads the expert outputs back from the owning ranks (peer loads) while it
+ * forms the weighted sum.  Plain 16-byte loads and stores; no TMA, no multicast.
+ *
+ * One chunk on every rank, in order:
+ *   1. moe_metadata(top_k_index, ..., ep_groups = W, num_chunks, ...) -> expert_counts of
+ *      each chunk and dst_rows (the chunk-local, expert-major row of each copy);
+ *   2. all-gather the chunk's expert_counts [E] over the ranks -> counts_all [W][E] (the
+ *      caller's collective, e.g. torch.distributed);
+ *   3. moe_ep_plan -> send_delta [E] (copy it to the device) and recv_offsets [E/W + 1];
+ *   4. moe_ep_dispatch into the ranks' receive buffers; then every rank must see all
+ *      ranks' dispatches complete (a barrier: a collective on the stream, or the host);
+ *   5. moe_grouped_gateup / moe_grouped_down on the receive rows with the local weights
+ *      (E/W experts, offsets = recv_offsets), Y written into the receive buffer; barrier;
+ *   6. moe_ep_combine -> out rows of the chunk; a barrier before the receive buffer is
+ *      reused.
+ * Receive layout on rank d: local expert by local expert; inside an expert the source
+ * ranks ascending, each source's rows in its own stable (t, j) order.  The results equal
+ * moe_forward on all ranks' tokens with all experts, bit for bit (each row meets the same
+ * GEMM and the same ascending-j sum).
+ * Peer buffers: moe_ipc_handle / moe_ipc_open map another process's device buffer on this
+ * GPU (CUDA IPC); the device tables recv_rows / expert_rows hold W such pointers (this
+ * rank's own buffer at index rank). */
+#define MOE_EP_MAX_RANKS 64
+#define MOE_IPC_HANDLE_BYTES 64
+
+/* Host arithmetic.  counts_all [W][E]: expert counts of one chunk on every rank (row s =
+ * rank s's expert_counts for the chunk).  Writes, for this rank:
+ *   send_delta [E]: the row offset to add to dst_rows of a copy of expert e to get its
+ *     row in the receive buffer of rank e / (E/W);
+ *   recv_offsets [E/W + 1]: where each local expert's rows start in this rank's receive
+ *     buffer, and (last entry) the rows it receives.
+ * Errors: MOE_ERR_ARG for NULL pointers, W <= 0, E % W != 0, rank outside [0, W) or a
+ * negative count; MOE_ERR_UNSUPPORTED beyond MOE_MAX_EXPERTS / MOE_EP_MAX_RANKS or for
+ * offsets beyond int32. */
+MOE_API moe_status_t moe_ep_plan(const int32_t* counts_all, int32_t W, int32_t rank, int32_t E,
+                                 int32_t* send_delta, int32_t* recv_offsets);
+
+/* recv_rows[e / (E/W)][dst_rows[t*k+j] + send_delta[e]] = hidden[t] for every copy (t, j)
+ * of one chunk, e = top_k_index[t*k+j].
+ *   hidden [Tc][H] bf16 dev (the chunk's rows, 16-byte aligned); top_k_index, dst_rows
+ *   [Tc*k] int32 dev (the chunk's slice, dst_rows chunk-local from moe_metadata with
+ *   ep_groups = W); send_delta [E] int32 dev (moe_ep_plan); recv_rows: dev array of W
+ *   device pointers, each to a receive buffer of rows_cap rows x H bf16 (peer-mapped).
+ * Enqueued on `stream`; returns without waiting.  Entries of top_k_index outside [0, E)
+ * are skipped (moe_metadata reports them first).  Errors: MOE_ERR_ARG / MOE_ERR_ALIGN /
+ * MOE_ERR_UNSUPPORTED from the host checks, MOE_ERR_CUDA if the launch fails. */
+MOE_API moe_status_t moe_ep_dispatch(const void* hidden, const int32_t* top_k_index,
+                                     const int32_t* dst_rows, const int32_t* send_delta,
+                                     void* const* recv_rows, int64_t Tc, int32_t H, int32_t k,
+                                     int32_t E, int32_t W, int64_t rows_cap, void* stream);
+
+/* out[t] = bf16( sum_{j<k} top_k_weights[t*k+j] * expert_rows[r][dst + delta] ), fp32
+ * accumulation in ascending j (the arithmetic of moe_unpermute), r = e / (E/W), reading
+ * each expert output row from the rank that computed it.  expert_rows: dev array of W
+ * device pointers to the ranks' expert-output rows (rows_cap x H bf16, peer-mapped);
+ * out [Tc][H] bf16 dev, 16-byte aligned, fully overwritten.  Otherwise as
+ * moe_ep_dispatch. */
+MOE_API moe_status_t moe_ep_combine(void* const* expert_rows, const int32_t* top_k_index,
+                                    const int32_t* dst_rows, const int32_t* send_delta,
+                                    const float* top_k_weights, int64_t Tc, int32_t H, int32_t k,
+                                    int32_t E, int32_t W, int64_t rows_cap, void* out,
+                                    void* stream);
+
+/* CUDA IPC of a caller-owned device buffer (any pointer into a cudaMalloc allocation,
+ * e.g. a torch tensor): writes the MOE_IPC_HANDLE_BYTES handle of its allocation and the
+ * pointer's offset inside it.  moe_ipc_open, in another process on the same node, maps it
+ * and returns the pointer (allocation base + offset); moe_ipc_close unmaps it.  Errors:
+ * MOE_ERR_ARG for NULL or a negative offset, MOE_ERR_CUDA if the CUDA call fails (a
+ * process cannot open its own handle). */
+MOE_API moe_status_t moe_ipc_handle(const void* dev_ptr, void* handle /* host [64] */,
+                                    int64_t* offset);
+MOE_API moe_status_t moe_ipc_open(const void* handle, int64_t offset, void** dev_ptr);
+MOE_API moe_status_t moe_ipc_close(void* dev_ptr, int64_t offset);
+
 /* ---- Kernel timing -----------------------------------------------------------------
  * When enabled, every kernel launch of the calls above is bracketed by two CUDA events
  * recorded on the stream the kernel is launched on.  moe_profile_read synchronizes the
