@@ -257,6 +257,14 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   constexpr int STAGES = G::kStages;
   constexpr int kEpiWarps = G::kEpiWarps;
   constexpr int kFirstGatherWarp = 2 + kEpiWarps;
+  // Gathering threads keep kGatherDepth + 1 stages of copies in flight and arrive on a
+  // stage's full barrier only once they have issued the copies of the kGatherDepth stages
+  // after it, so those stages must be free (released by the MMA warp) by then.
+  constexpr int kGatherDepth = STAGES - 2 > 0 ? STAGES - 2 : 1;
+  // kTwoM: stages whose second-sub-tile MMAs the MMA warp may hold back (each held stage
+  // stays unreleased); with gathered A the gathering threads' run-ahead must stay free.
+  constexpr int kMaxHeld = STAGES - 1 - (kGather ? kGatherDepth : 0);
+  static_assert(!kTwoM || kMaxHeld >= 0, "ring too shallow for the gathered two-sub-tile kernel");
   static_assert(!(kGather && kPair), "gathered A rows are implemented for single CTAs");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -384,7 +392,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
     // 128-byte row segments.  A thread keeps kDepth + 1 stages of copies in flight; when
     // its oldest stage has landed it makes the writes visible to the async proxy and
     // arrives on that stage's full barrier.
-    constexpr int kDepth = STAGES - 2 > 0 ? STAGES - 2 : 1;
+    constexpr int kDepth = kGatherDepth;
     constexpr int kSub = G::kSubM;
     const int gw = warp - kFirstGatherWarp, j = lane & 7, sub = lane >> 3;
     int stage = 0;
@@ -547,7 +555,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
           if (m1) {
             if (!acc1) {
               acc1 = mbar_test_wait(&ctl->tempty[1], (use[1] & 1u) ^ 1u);
-              if (!acc1 && (npend == STAGES - 1 || kb == p.num_kb - 1)) {
+              if (!acc1 && (npend >= kMaxHeld || kb == p.num_kb - 1)) {
                 if (!mbar_wait(&ctl->tempty[1], (use[1] & 1u) ^ 1u, abort, p.status)) {
                   ok = false;
                   break;

@@ -75,13 +75,38 @@ def test_clock_summary_keeps_only_the_timed_window():
     assert s.summary(5.0, 6.0) is None
 
 
-def test_tensor_peak_scales_the_burst_figure_by_the_sampled_clock():
-    peaks = {"bf16_tflops": 1679.8, "bf16_tflops_sustained": 1394.0, "hbm_gbs": 6549.4}
+def test_tensor_peak_follows_the_sampled_clock():
+    """The roof at clock f: the sustained figure scaled from its own clock, capped by the
+    burst figure; without a sample, the burst figure."""
+    peaks = {"bf16_tflops": 1679.8, "bf16_tflops_sustained": 1394.0, "hbm_gbs": 6549.4,
+             "sustained_mhz": 1335.0, "burst_mhz": None}
     assert bench.tensor_peak(peaks, None) == (1679.8, 1.0)
     p, sc = bench.tensor_peak(peaks, {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0})
-    assert (p, sc) == (1679.8, 1.0)
+    assert (p, sc) == (1679.8, 1.0)                       # capped by the burst figure
+    p, sc = bench.tensor_peak(peaks, {"sm_mhz": 1335.0, "sm_max_mhz": 1965.0})
+    assert p == pytest.approx(1394.0)                     # the sustained point itself
+    p, sc = bench.tensor_peak(peaks, {"sm_mhz": 1417.0, "sm_max_mhz": 1965.0})
+    assert p == pytest.approx(1394.0 * 1417 / 1335) and sc == pytest.approx(p / 1679.8)
+    # no recorded sustained clock: the burst figure scaled by clock / max clock
+    peaks["sustained_mhz"] = None
     p, sc = bench.tensor_peak(peaks, {"sm_mhz": 1310.0, "sm_max_mhz": 1965.0})
     assert sc == pytest.approx(2 / 3) and p == pytest.approx(1679.8 * 2 / 3)
+
+
+def test_measured_peaks_clock_keys(tmp_path, monkeypatch):
+    """Clock entries of MEASURED_PEAKS.json are found by name (nested or flat)."""
+    import json
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({
+        "hbm_gbs": 6549.4, "bf16_tflops": 1679.8, "bf16_tflops_sustained": 1394.0,
+        "clocks": {"bf16_sustained_sm_mhz_median": 1335, "bf16_burst_sm_mhz": 1860,
+                   "sm_max_mhz": 1965}}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    peaks, src = bench.load_peaks()
+    assert src == "measured" and peaks["sustained_mhz"] == 1335.0
+    assert peaks["burst_mhz"] == 1860.0
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path / "none"))
+    peaks, src = bench.load_peaks()
+    assert src == "fallback" and peaks["sustained_mhz"] == bench.FALLBACK_SUSTAINED_MHZ
 
 
 def test_gemm_roofline_reproduces_from_its_per_launch_figures():
@@ -90,14 +115,16 @@ def test_gemm_roofline_reproduces_from_its_per_launch_figures():
     cfg = LayerConfig("u", T=16384, H=2048, E=128, k=8, I=768, routing="normal")
     counts = np.full((2, 128), 512, np.int32)
     units = bench.algorithmic_units(cfg, counts, 4, "fused", True)
-    peaks = {"bf16_tflops": 1679.8, "bf16_tflops_sustained": 1394.0, "hbm_gbs": 6549.4}
+    peaks = {"bf16_tflops": 1679.8, "bf16_tflops_sustained": 1394.0, "hbm_gbs": 6549.4,
+             "sustained_mhz": 1335.0, "burst_mhz": None}
     m = {"units": units, "steps": 4, "dispatch": "fused",
          "prof": {"gateup": {"launches": 8, "ms": 8 * 0.4}},
-         "clk": {"sm_mhz": 1800.0, "sm_max_mhz": 1965.0}}
+         "clk": {"sm_mhz": 1450.0, "sm_max_mhz": 1965.0}}
     r = bench.gemm_roofline(m, peaks, "measured")
     pl = r["per_launch"]
     assert r["bound"] == "tensor"
     assert pl["flops"] == pytest.approx(4.0 * 65536 * 2048 * 768)
-    want = pl["flops"] / (pl["ms"] / 1e3) / 1e12 / (1679.8 * 1800 / 1965)
-    assert r["frac"] == pytest.approx(want)
-    assert r["tensor_frac_of_burst"] == pytest.approx(want * 1800 / 1965)
+    tf = pl["flops"] / (pl["ms"] / 1e3) / 1e12
+    assert r["frac"] == pytest.approx(tf / (1394.0 * 1450 / 1335))
+    assert r["tensor_frac_of_burst"] == pytest.approx(tf / 1679.8)
+    assert r["tensor_frac_of_burst_x_clock_ratio"] == pytest.approx(tf / (1679.8 * 1450 / 1965))
