@@ -186,6 +186,14 @@ __device__ __forceinline__ void cp_async_16(uint32_t smem_dst, const void* src, 
                : "memory");
 }
 
+// The same copy with an L2 cache-eviction policy for the source line (createpolicy).
+__device__ __forceinline__ void cp_async_16_hint(uint32_t smem_dst, const void* src,
+                                                 uint32_t src_bytes, uint64_t policy) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(smem_dst),
+               "l"(src), "r"(src_bytes), "l"(policy)
+               : "memory");
+}
+
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }

@@ -57,6 +57,15 @@
 #ifndef MOE_GEMM_BAND
 #define MOE_GEMM_BAND 16  // M tiles per raster band: an expert's A rows stay in L2 across N tiles
 #endif
+#ifndef MOE_GEMM_HALF_TAILS
+#define MOE_GEMM_HALF_TAILS 1  // a 128-row tile with at most 64 valid rows runs M=64 MMAs
+#endif
+#ifndef MOE_GEMM_GATHER_B_POLICY
+#define MOE_GEMM_GATHER_B_POLICY 2  // gathered-A kernel: L2 policy of the weight loads
+#endif
+#ifndef MOE_GEMM_GATHER_A_POLICY
+#define MOE_GEMM_GATHER_A_POLICY 0  // gathered-A kernel: 0 no hint, else L2 policy of the rows
+#endif
 #ifndef MOE_GEMM_TWO_M
 #define MOE_GEMM_TWO_M 0  // 256-row tiles of two 128-row sub-tiles: bit 0 gate/up, bit 1 down
 #endif
@@ -99,6 +108,10 @@ struct Geo {
   static constexpr uint32_t kStageBytes = kAStageBytes + kBBytes;           // per CTA
   static constexpr uint32_t kTxBytes = kPair ? 2 * kStageBytes : kStageBytes;  // per stage
   static constexpr uint32_t kIdesc = umma_idesc_bf16_f32(kPair ? 2 * kRowsPerCta : kRowsPerCta, BN);
+  // single CTA, one sub-tile: a tile holding at most 64 rows of its expert runs M=64 MMAs
+  // (the accumulator's row r then sits in TMEM lane 32 (r / 16) + r % 16)
+  static constexpr bool kHalfTails = !kPair && !kTwoM && MOE_GEMM_HALF_TAILS != 0;
+  static constexpr uint32_t kIdescHalf = umma_idesc_bf16_f32(kRowsPerCta / 2, BN);
   // epilogue warps: kTwoM may use two per TMEM lane quarter (each takes half the columns)
   static constexpr int kEpiWarps = kTwoM ? MOE_GEMM_EPI_WARPS_2M : 4;
 };
@@ -199,10 +212,14 @@ __device__ __forceinline__ Tile decode_tile(int32_t L, const int32_t* tile_start
 // Stores the 32 x 32 bf16 block of one epilogue warp: lane i holds row (32 q + i) of the
 // tile as 16 packed bf16 pairs.  Rows at or past rows_valid (past the expert's end) and
 // columns at or past out_cols are never written.
+// kRpw: rows per warp, 32 (M=128 accumulator: lane i of quarter q is tile row 32 q + i) or
+// 16 (M=64 accumulator: lanes 0..15 of quarter q hold tile rows 16 q + i, lanes 16..31
+// nothing).
 __device__ __forceinline__ void store_block(const uint32_t (&packed)[16], uint8_t* wbuf, int lane,
                                             int q, bool row_ok, int32_t rows_valid,
                                             int64_t row_base, int32_t col0, const KParams& p,
-                                            __nv_bfloat16* out, int64_t out_rows) {
+                                            __nv_bfloat16* out, int64_t out_rows,
+                                            int rpw = 32) {
 #if MOE_GEMM_EPI_STAGE
   uint4* mine = reinterpret_cast<uint4*>(wbuf + lane * kEpiRowBytes);
 #pragma unroll
@@ -215,8 +232,9 @@ __device__ __forceinline__ void store_block(const uint32_t (&packed)[16], uint8_
 #pragma unroll
   for (int pass = 0; pass < 4; ++pass) {
     const int rr = pass * 8 + (lane >> 2);
+    if (pass * 8 >= rpw) break;
     const uint4 v = *reinterpret_cast<const uint4*>(wbuf + rr * kEpiRowBytes + seg * 16);
-    const int32_t tr = q * 32 + rr;  // row inside the CTA's 128 rows
+    const int32_t tr = q * rpw + rr;  // row inside the CTA's 128 rows
     if (tr < rows_valid && col < p.out_cols &&
         check_row(row_base + tr, out_rows, &g_range_flags))
       *reinterpret_cast<uint4*>(out + (row_base + tr) * p.out_cols + col) = v;
@@ -226,8 +244,8 @@ __device__ __forceinline__ void store_block(const uint32_t (&packed)[16], uint8_
 #else
   (void)wbuf;
   (void)rows_valid;
-  if (row_ok && check_row(row_base + q * 32 + lane, out_rows, &g_range_flags)) {
-    uint4* dst = reinterpret_cast<uint4*>(out + (row_base + q * 32 + lane) * p.out_cols + col0);
+  if (row_ok && check_row(row_base + q * rpw + lane, out_rows, &g_range_flags)) {
+    uint4* dst = reinterpret_cast<uint4*>(out + (row_base + q * rpw + lane) * p.out_cols + col0);
 #pragma unroll
     for (int v = 0; v < 4; ++v)
       if (col0 + v * 8 < p.out_cols)
@@ -346,13 +364,19 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   auto has_m1 = [&](const Tile& t) {
     return kTwoM && off[t.e + 1] - off[t.e] > t.m * G::kTileM + kRowsPerCta;
   };
+  // kHalfTails: whether tile t holds at most 64 rows of its expert (M=64 MMAs)
+  auto is_half = [&](const Tile& t) {
+    return G::kHalfTails && off[t.e + 1] - off[t.e] - t.m * G::kTileM <= kRowsPerCta / 2;
+  };
 
   if (warp == 0 && kGather) {
     // ---------------- weight producer, gathered A (lane 0) ----------------
     // The A rows of a stage come from the gathering warps (below); this lane arms the stage
     // with the weight bytes and loads the weight box(es) with TMA.
     if (lane == 0) {
-      const uint64_t pol_w = l2_policy_evict_last();
+      const uint64_t pol_w = MOE_GEMM_GATHER_B_POLICY == 1   ? l2_policy_evict_first()
+                             : MOE_GEMM_GATHER_B_POLICY == 2 ? l2_policy_evict_last()
+                                                             : l2_policy_evict_normal();
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;
@@ -395,6 +419,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
     constexpr int kDepth = kGatherDepth;
     constexpr int kSub = G::kSubM;
     const int gw = warp - kFirstGatherWarp, j = lane & 7, sub = lane >> 3;
+    const uint64_t pol_a = MOE_GEMM_GATHER_A_POLICY == 1 ? l2_policy_evict_first()
+                           : MOE_GEMM_GATHER_A_POLICY == 2 ? l2_policy_evict_last()
+                                                           : l2_policy_evict_normal();
     int stage = 0;
     uint32_t phase = 0;
     int32_t issued = 0, arrived = 0;
@@ -405,6 +432,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       const int32_t row0 = off[t.e] + t.m * G::kTileM;
       const int32_t last = off[t.e + 1] - 1;  // rows past the expert re-read its last row
       const int n_sub = has_m1(t) ? 2 : 1;
+      // half tiles: only rows 0..63 are read by the M=64 MMAs (gathering warps 0 and 1)
+      const bool skip = is_half(t) && gw >= 2;
       const uint8_t* src[kSub * 8];
 #pragma unroll
       for (int h = 0; h < kSub; ++h)
@@ -424,12 +453,15 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
         const uint32_t nbytes = (kb * BK + j * 8 < p.K) ? 16u : 0u;  // zero past K
 #pragma unroll
         for (int h = 0; h < kSub; ++h) {
-          if (h < n_sub) {
+          if (h < n_sub && !skip) {
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
               const int32_t r = gw * 32 + 4 * i + sub;
-              cp_async_16(a + h * G::kABytes + r * (BK * 2) + ((j ^ (r & 7)) << 4),
-                          src[h * 8 + i] + kb * (BK * 2), nbytes);
+              const uint32_t dst_s = a + h * G::kABytes + r * (BK * 2) + ((j ^ (r & 7)) << 4);
+              if (MOE_GEMM_GATHER_A_POLICY == 0)
+                cp_async_16(dst_s, src[h * 8 + i] + kb * (BK * 2), nbytes);
+              else
+                cp_async_16_hint(dst_s, src[h * 8 + i] + kb * (BK * 2), nbytes, pol_a);
             }
           }
         }
@@ -614,6 +646,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * BN;
+        uint32_t idesc = G::kIdesc;
+        if (G::kHalfTails) {
+          const Tile t = decode_tile<G::kTileM>(L, tile_start, off, E, p.n_tiles);
+          if (is_half(t)) idesc = G::kIdescHalf;
+        }
         for (int32_t kb = 0; kb < p.num_kb; ++kb) {
           if (!mbar_wait(&ctl->full[stage], phase, abort, p.status)) {
             ok = false;
@@ -628,7 +665,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
             const uint64_t ad = kmajor_desc<kSwizzleBytes>(a_addr + kk * 32);
             const uint64_t bd = kmajor_desc<kSwizzleBytes>(b_addr + kk * 32);
             if (kPair) umma_bf16_pair(d_tmem, ad, bd, G::kIdesc, (kb | kk) != 0);
-            else umma_bf16(d_tmem, ad, bd, G::kIdesc, (kb | kk) != 0);
+            else umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
           }
           issued = true;
           if (kPair) umma_commit_pair(&ctl->empty[stage], 0x3);
@@ -681,7 +718,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
         const int64_t out_rows = p.out_rows;
         const int32_t first = t.m * G::kTileM + (int32_t)rank * kRowsPerCta + h * kRowsPerCta;
         const int32_t rows_valid = offs[t.e + 1] - offs[t.e] - first;
-        const bool row_ok = r < rows_valid;
+        const int rpw = is_half(t) ? 16 : 32;  // M=64 accumulator: 16 rows per lane quarter
+        const bool row_ok = rpw == 32 ? r < rows_valid : (lane < 16 && q * 16 + lane < rows_valid);
         const int64_t row_base = (int64_t)offs[t.e] + first;  // output row of TMEM lane 0
         const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * BN;
         if (kSwiGLU) {
@@ -705,7 +743,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
               packed[i] = pack_bf16x2(a0, a1);
             }
             store_block(packed, wbuf, lane, q, row_ok, rows_valid, row_base, col0, p, out,
-                        out_rows);
+                        out_rows, rpw);
           }
         } else {
           constexpr int kChunks = BN / 32 / kParts;
@@ -721,7 +759,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
               packed[i] =
                   pack_bf16x2(__uint_as_float(acc[2 * i]), __uint_as_float(acc[2 * i + 1]));
             store_block(packed, wbuf, lane, q, row_ok, rows_valid, row_base, col0, p, out,
-                        out_rows);
+                        out_rows, rpw);
           }
         }
         tc_fence_before();
