@@ -426,24 +426,36 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
     uint32_t phase = 0;
     int32_t issued = 0, arrived = 0;
     bool ok = true;
+    const int32_t* gat = p.gather;  // gathered A has one row segment
+    // token index of each row this thread copies in tile L (rows past the expert re-read
+    // its last row)
+    auto load_tokens = [&](int32_t L2, int32_t (&tok)[kSub * 8]) {
+      const Tile t2 = decode_tile<G::kTileM>(L2, tile_start, off, E, p.n_tiles);
+      const int32_t row0 = off[t2.e] + t2.m * G::kTileM;
+      const int32_t last = off[t2.e + 1] - 1;
+#pragma unroll
+      for (int h = 0; h < kSub; ++h)
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          tok[h * 8 + i] = gat[min(row0 + h * kRowsPerCta + gw * 32 + 4 * i + sub, last)];
+    };
+    // the next tile's indices are loaded when a tile starts, so that their latency is
+    // spent behind the tile's copies instead of at the next tile boundary
+    int32_t next_tok[kSub * 8];
+    if (stream_id < p.total_tiles) load_tokens(stream_id, next_tok);
     for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
       const Tile t = decode_tile<G::kTileM>(L, tile_start, off, E, p.n_tiles);
-      const int32_t* gat = p.gather;  // gathered A has one row segment
-      const int32_t row0 = off[t.e] + t.m * G::kTileM;
-      const int32_t last = off[t.e + 1] - 1;  // rows past the expert re-read its last row
       const int n_sub = has_m1(t) ? 2 : 1;
       // half tiles: only rows 0..63 are read by the M=64 MMAs (gathering warps 0 and 1)
       const bool skip = is_half(t) && gw >= 2;
       const uint8_t* src[kSub * 8];
 #pragma unroll
-      for (int h = 0; h < kSub; ++h)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int32_t r = h * kRowsPerCta + gw * 32 + 4 * i + sub;
-          int64_t tok = gat[min(row0 + r, last)];
-          if (!check_row(tok, p.gsrc_rows, &g_range_flags)) tok = 0;
-          src[h * 8 + i] = p.gsrc + tok * p.gsrc_stride + j * 16;
-        }
+      for (int x = 0; x < kSub * 8; ++x) {
+        int64_t tok = next_tok[x];
+        if (!check_row(tok, p.gsrc_rows, &g_range_flags)) tok = 0;
+        src[x] = p.gsrc + tok * p.gsrc_stride + j * 16;
+      }
+      if (L + n_streams < p.total_tiles) load_tokens(L + n_streams, next_tok);
       for (int32_t kb = 0; kb < p.num_kb; ++kb) {
         if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort, p.status)) {
           ok = false;

@@ -42,8 +42,12 @@ cudaError_t launch_metadata(const MetaArgs& a, cudaStream_t s);
 // against it.
 cudaError_t launch_permute(const void* hidden, const int32_t* dst, int64_t Tc, int32_t H,
                            int32_t k, void* X, int64_t rows_cap, cudaStream_t s);
+// ctas_per_sm: CTAs of the compile-time-k combine per SM (0: the build's default).  A combine
+// that runs beside a grouped GEMM takes fewer, so that every CTA of it is resident next to
+// the GEMM's one CTA per SM and all its tokens progress together.
 cudaError_t launch_unpermute(const void* Y, const int32_t* dst, const float* w, int64_t Tc,
-                             int32_t H, int32_t k, void* out, int64_t rows_cap, cudaStream_t s);
+                             int32_t H, int32_t k, void* out, int64_t rows_cap, cudaStream_t s,
+                             int ctas_per_sm = 0);
 // Range-violation flags of the checks build, one word per translation unit: read and clear.
 uint32_t checks_take_permute();
 uint32_t checks_take_gemm();

@@ -34,6 +34,10 @@ namespace {
 
 using namespace moe;
 
+#ifndef MOE_UNPERM_BESIDE_GEMM_CTAS_PER_SM
+#define MOE_UNPERM_BESIDE_GEMM_CTAS_PER_SM 1  // combine CTAs per SM while a GEMM holds the SMs
+#endif
+
 constexpr size_t kAlign = 256;
 constexpr int kStatusWords = 4;  // packed block: status words, then counts, then splits
 constexpr int kMaxDevices = 64;
@@ -743,10 +747,15 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
       if (cudaEventRecord(ctx->ev_gemm[0], sg) != cudaSuccess ||
           cudaStreamWaitEvent(sm, ctx->ev_gemm[0], 0) != cudaSuccess)
         return MOE_ERR_CUDA;
+      // a pair's combines run beside the next pair's gate/up GEMM (fewer CTAs, all resident
+      // next to it) unless this is the last pair
+      const bool beside_gemm = 2 * (m + 1) < n_live;
       for (int c = c0; c <= c1; ++c) {
         ProfScope ps(MOE_KERNEL_UNPERMUTE, sm, len(c) * k, 0, 1);
         if (launch_unpermute(y_pair, dst + bounds[c] * k, top_k_weights + bounds[c] * k, len(c),
-                             H, k, outp + bounds[c] * H, pair_cap, sm) != cudaSuccess)
+                             H, k, outp + bounds[c] * H, pair_cap, sm,
+                             beside_gemm ? MOE_UNPERM_BESIDE_GEMM_CTAS_PER_SM : 0) !=
+            cudaSuccess)
           return MOE_ERR_CUDA;
       }
       if (cudaEventRecord(ctx->ev_unperm[0], sm) != cudaSuccess) return MOE_ERR_CUDA;

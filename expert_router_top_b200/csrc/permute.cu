@@ -188,8 +188,10 @@ int num_sms_cached() {
 
 template <int KT>
 cudaError_t launch_unpermute_k(const void* Y, const int32_t* dst, const float* w, int64_t Tc,
-                               int32_t H, void* out, int64_t rows_cap, cudaStream_t s) {
-  const int64_t cap = (int64_t)num_sms_cached() * MOE_UNPERM_CTAS_PER_SM;
+                               int32_t H, void* out, int64_t rows_cap, cudaStream_t s,
+                               int ctas_per_sm) {
+  const int64_t cap =
+      (int64_t)num_sms_cached() * (ctas_per_sm > 0 ? ctas_per_sm : MOE_UNPERM_CTAS_PER_SM);
   const int64_t need = grid_for(Tc);
   unpermute_k_kernel<KT><<<(unsigned)(need < cap ? need : cap), kRowThreads, 0, s>>>(
       static_cast<const uint4*>(Y), dst, w, Tc, H / 8, static_cast<uint4*>(out), rows_cap);
@@ -207,15 +209,16 @@ cudaError_t launch_permute(const void* hidden, const int32_t* dst, int64_t Tc, i
 }
 
 cudaError_t launch_unpermute(const void* Y, const int32_t* dst, const float* w, int64_t Tc,
-                             int32_t H, int32_t k, void* out, int64_t rows_cap, cudaStream_t s) {
+                             int32_t H, int32_t k, void* out, int64_t rows_cap, cudaStream_t s,
+                             int ctas_per_sm) {
   if (Tc <= 0) return cudaSuccess;
 #if MOE_UNPERM_CTAS_PER_SM > 0
   switch (k) {
-    case 1: return launch_unpermute_k<1>(Y, dst, w, Tc, H, out, rows_cap, s);
-    case 2: return launch_unpermute_k<2>(Y, dst, w, Tc, H, out, rows_cap, s);
-    case 4: return launch_unpermute_k<4>(Y, dst, w, Tc, H, out, rows_cap, s);
-    case 6: return launch_unpermute_k<6>(Y, dst, w, Tc, H, out, rows_cap, s);
-    case 8: return launch_unpermute_k<8>(Y, dst, w, Tc, H, out, rows_cap, s);
+    case 1: return launch_unpermute_k<1>(Y, dst, w, Tc, H, out, rows_cap, s, ctas_per_sm);
+    case 2: return launch_unpermute_k<2>(Y, dst, w, Tc, H, out, rows_cap, s, ctas_per_sm);
+    case 4: return launch_unpermute_k<4>(Y, dst, w, Tc, H, out, rows_cap, s, ctas_per_sm);
+    case 6: return launch_unpermute_k<6>(Y, dst, w, Tc, H, out, rows_cap, s, ctas_per_sm);
+    case 8: return launch_unpermute_k<8>(Y, dst, w, Tc, H, out, rows_cap, s, ctas_per_sm);
     default: break;
   }
 #endif
