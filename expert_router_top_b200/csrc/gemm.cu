@@ -57,6 +57,9 @@
 #ifndef MOE_GEMM_BAND
 #define MOE_GEMM_BAND 16  // M tiles per raster band: an expert's A rows stay in L2 across N tiles
 #endif
+#ifndef MOE_GEMM_GATHER_MODE
+#define MOE_GEMM_GATHER_MODE 0  // gathered A: 0 every warp a slice of every slot, 1 a slot per warp
+#endif
 #ifndef MOE_GEMM_HALF_TAILS
 #define MOE_GEMM_HALF_TAILS 1  // a 128-row tile with at most 64 valid rows runs M=64 MMAs
 #endif
@@ -282,6 +285,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   // kTwoM: stages whose second-sub-tile MMAs the MMA warp may hold back (each held stage
   // stays unreleased); with gathered A the gathering threads' run-ahead must stay free.
   constexpr int kMaxHeld = STAGES - 1 - (kGather ? kGatherDepth : 0);
+  // Gathered A, one ring slot per gathering warp (the single-sub-tile ring of 4 slots)
+  constexpr bool kWarpStages =
+      kGather && !kTwoM && MOE_GEMM_GATHER_MODE == 1 && STAGES == kGatherThreads / 32;
   static_assert(!kTwoM || kMaxHeld >= 0, "ring too shallow for the gathered two-sub-tile kernel");
   static_assert(!(kGather && kPair), "gathered A rows are implemented for single CTAs");
   extern __shared__ uint8_t smem_raw[];
@@ -305,8 +311,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   for (int32_t i = threadIdx.x; i <= E; i += blockDim.x) off[i] = p.offsets[i];
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      // gathered A: the weight producer's arrival plus one per A-gathering thread
-      mbar_init(&ctl->full[s], kGather ? 1 + kGatherThreads : 1);
+      // gathered A: the weight producer's arrival plus one per A-gathering thread (or one
+      // per slot-owning gathering warp)
+      mbar_init(&ctl->full[s], kGather ? 1 + (kWarpStages ? 1 : kGatherThreads) : 1);
       mbar_init(&ctl->empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -407,6 +414,71 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
         for (int s = 0; s < STAGES; ++s)
           if (armed & (1u << s)) mbar_drain(&ctl->full[s], (armed_parity >> s) & 1u, 100000000ull);
     }
+  } else if (kGather && kWarpStages && warp >= kFirstGatherWarp) {
+    // ---------------- A producers, gathered rows, one ring slot per warp ----------------
+    // Gathering warp w fills ring slot w (the ring has as many slots as there are gathering
+    // warps): for each K block that lands in slot w it copies all of the tile's A rows --
+    // lane (8 s + j) copies 16-byte chunk j of rows 4 i + s, i < 32 -- into the
+    // 128-byte-swizzled K-major layout, waits for its own copies, makes them visible to the
+    // async proxy, and one lane arrives on the slot's full barrier.  A slot is thus reported
+    // full as soon as its copies have landed, and each slot's copies are in flight for up to
+    // a whole lap of the ring.  Lane l holds the token indices of rows l, l+32, l+64, l+96.
+    const int gw = warp - kFirstGatherWarp, j = lane & 7, sub = lane >> 3;
+    const uint64_t pol_a = MOE_GEMM_GATHER_A_POLICY == 1 ? l2_policy_evict_first()
+                           : MOE_GEMM_GATHER_A_POLICY == 2 ? l2_policy_evict_last()
+                                                           : l2_policy_evict_normal();
+    const int32_t* gat = p.gather;
+    auto load_tokens = [&](int32_t L2, int32_t (&tok)[4]) {
+      const Tile t2 = decode_tile<G::kTileM>(L2, tile_start, off, E, p.n_tiles);
+      const int32_t row0 = off[t2.e] + t2.m * G::kTileM;
+      const int32_t last = off[t2.e + 1] - 1;  // rows past the expert re-read its last row
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tok[q] = gat[min(row0 + q * 32 + lane, last)];
+    };
+    int32_t next_tok[4];
+    if (stream_id < p.total_tiles) load_tokens(stream_id, next_tok);
+    uint32_t phase = 0;  // phase of this warp's slot
+    int32_t sigma = 0;   // K blocks of this CTA so far (ring position)
+    bool ok = true;
+    for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
+      const Tile t = decode_tile<G::kTileM>(L, tile_start, off, E, p.n_tiles);
+      const bool half = is_half(t);  // M=64 MMAs read rows 0..63 only
+      int32_t tok[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        tok[q] = next_tok[q];
+        if (!check_row(tok[q], p.gsrc_rows, &g_range_flags)) tok[q] = 0;
+      }
+      if (L + n_streams < p.total_tiles) load_tokens(L + n_streams, next_tok);
+      for (int32_t kb = 0; kb < p.num_kb; ++kb, ++sigma) {
+        if ((sigma & (STAGES - 1)) != gw) continue;
+        if (!mbar_wait(&ctl->empty[gw], phase ^ 1u, abort, p.status)) {
+          ok = false;
+          break;
+        }
+        const uint32_t a = smem_u32(sA + gw * G::kAStageBytes);
+        const uint32_t nbytes = (kb * BK + j * 8 < p.K) ? 16u : 0u;  // zero past K
+        const uint8_t* base = p.gsrc + j * 16 + kb * (BK * 2);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if (half && i >= 16) break;
+          const int32_t r = 4 * i + sub;
+          const int64_t tk = __shfl_sync(0xffffffffu, tok[i / 8], 4 * (i % 8) + sub);
+          const uint32_t dst_s = a + r * (BK * 2) + ((j ^ (r & 7)) << 4);
+          if (MOE_GEMM_GATHER_A_POLICY == 0)
+            cp_async_16(dst_s, base + tk * p.gsrc_stride, nbytes);
+          else
+            cp_async_16_hint(dst_s, base + tk * p.gsrc_stride, nbytes, pol_a);
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->full[gw]);
+        phase ^= 1u;
+      }
+    }
+    (void)ok;
   } else if (kGather && warp >= kFirstGatherWarp) {
     // ---------------- A producers, gathered rows (4 warps, LSU) ----------------
     // The tile's A rows are the token rows src_tok[row] of `hidden`.  Per K block, lane
@@ -793,8 +865,12 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   }
 }
 
+// At most 128 registers per thread: with 10 warps on the 4 SM sub-partitions (3, 3, 2, 2)
+// a sub-partition holding 3 of them keeps 4096 of its 16384 registers free, room for two
+// warps of a 64-register combine CTA of 8 warps -- the combine that runs beside this kernel
+// must be able to reside next to it.
 template <bool kSwiGLU, bool kGather, bool kTwoM>
-__global__ void __launch_bounds__(gemm_threads<kGather, kTwoM>(), 1)
+__global__ void __maxnreg__(128)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
                         const KParams p) {
