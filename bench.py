@@ -618,7 +618,7 @@ def run_ours(args, cfg):
 
     # ---- the headline: K timed steps at the requested chunk count and dispatch
     head = run.measure(chunks, args.dispatch, args.steps, args.warmup, args.per_chunk_gemms,
-                       spin_s=0.5)
+                       spin_s=args.spinup_s)
     ms_max = max_over_ranks(head["ms"], pg, dev)
     ms_per_step = ms_max / args.steps
     value = job_tokens_per_s(world, cfg.T, args.steps, ms_max)
@@ -664,6 +664,10 @@ def run_ours(args, cfg):
                            "timelines": timelines}, f, indent=1)
     if clocks:
         clocks.stop()
+        if args.clock_trace:
+            with open(args.clock_trace, "w") as f:
+                json.dump([(round(t - clocks.samples[0][0], 4), mhz, sorted(r))
+                           for t, mhz, _, r in clocks.samples], f)
 
     ms_n1 = per_n.get("1", {}).get("ms_per_step")
     line = {
@@ -693,7 +697,7 @@ def run_ours(args, cfg):
         "ms_per_step_num_chunks_1": ms_n1,
         "send_splits": head["meta"]["send"].tolist() if cfg.G > 1 else None,
         "gpu_launches": int(head["prof"]["kernels"]),
-        "spinup_steps": head["spinup_steps"],
+        "spinup_steps": head["spinup_steps"], "spinup_s": args.spinup_s,
         "e2e": e2e,
         "clocks": head["clk"],
         "peaks": dict(peaks, source=peak_src),
@@ -778,7 +782,7 @@ def run_backward(args, cfg):
     if clocks:
         clocks.start()
     t_load = time.perf_counter()
-    spinup = spin_up(step)
+    spinup = spin_up(step, args.spinup_s)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -854,7 +858,7 @@ def run_backward(args, cfg):
         "kernels": kinds,
         "backward_workspace_bytes": ws_per_n,
         "gpu_launches": int(prof["kernels"]),
-        "spinup_steps": spinup,
+        "spinup_steps": spinup, "spinup_s": args.spinup_s,
         "e2e": None,
         "clocks": clk,
     }
@@ -924,6 +928,11 @@ def main():
                          "train (forward then backward per step)")
     ap.add_argument("--per-chunk-gemms", action="store_true",
                     help="fused dispatch: one GEMM sweep per chunk instead of per pair")
+    ap.add_argument("--spinup-s", type=float, default=2.0,
+                    help="untimed steps before the first timed region, in seconds: long enough "
+                         "for the power-capped SM clock to settle after an idle GPU starts")
+    ap.add_argument("--clock-trace", default="",
+                    help="write every SM clock sample of the run (host time, MHz, reasons) here")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the workload's token count (small cases for profiling)")
     ap.add_argument("--per-n", type=int, nargs="*", default=[1, 2, 4],
