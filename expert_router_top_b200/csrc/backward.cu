@@ -558,15 +558,28 @@ __global__ void __launch_bounds__(kRowThreads)
     const int32_t d = dstp[t * k + j];
     if (!check_row(d, rows_cap, &g_range_flags)) continue;
     float dot = 0.f;
-    for (int32_t v = lane; v < H8; v += 32) {
-      const uint4 g = dout[t * H8 + v];
-      const uint4 y = Y[(int64_t)d * H8 + v];
-      const uint32_t ga[4] = {g.x, g.y, g.z, g.w};
-      const uint32_t ya[4] = {y.x, y.y, y.z, y.w};
+    // 8 columns of 16 bytes per lane at a time: all 16 loads are issued before the FMAs,
+    // which then run in the same order as one column at a time (v ascending)
+    for (int32_t v0 = lane; v0 < H8; v0 += 32 * 8) {
+      uint4 g[8], y[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        dot = fmaf(bf16lo(ga[i]), bf16lo(ya[i]), dot);
-        dot = fmaf(bf16hi(ga[i]), bf16hi(ya[i]), dot);
+      for (int u = 0; u < 8; ++u) {
+        const int32_t v = v0 + 32 * u;
+        if (v < H8) {
+          g[u] = __ldg(dout + t * H8 + v);
+          y[u] = __ldg(Y + (int64_t)d * H8 + v);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (v0 + 32 * u >= H8) break;
+        const uint32_t ga[4] = {g[u].x, g[u].y, g[u].z, g[u].w};
+        const uint32_t ya[4] = {y[u].x, y[u].y, y[u].z, y[u].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          dot = fmaf(bf16lo(ga[i]), bf16lo(ya[i]), dot);
+          dot = fmaf(bf16hi(ga[i]), bf16hi(ya[i]), dot);
+        }
       }
     }
 #pragma unroll
