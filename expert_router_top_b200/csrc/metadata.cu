@@ -113,10 +113,17 @@ __global__ void __launch_bounds__(kMetaThreads) meta_count_kernel(MetaArgs a) {
   if (e >= a.E) return;
   int32_t* h = a.hist + (int64_t)c * a.tiles_per_chunk * a.E + e;
   int32_t run = 0;
-  for (int32_t lt = 0; lt < a.tiles_per_chunk; ++lt) {
-    const int32_t v = h[(int64_t)lt * a.E];
-    h[(int64_t)lt * a.E] = run;
-    run += v;
+  // 8 tiles at a time: the 8 loads are issued together instead of one round trip per tile
+  for (int32_t lt0 = 0; lt0 < a.tiles_per_chunk; lt0 += 8) {
+    int32_t v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      v[u] = lt0 + u < a.tiles_per_chunk ? h[(int64_t)(lt0 + u) * a.E] : 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (lt0 + u < a.tiles_per_chunk) h[(int64_t)(lt0 + u) * a.E] = run;
+      run += v[u];
+    }
   }
   a.counts[(int64_t)c * a.E + e] = run;
 }
@@ -181,12 +188,24 @@ __global__ void __launch_bounds__(kMetaThreads) meta_finalize_kernel(MetaArgs a)
   int32_t* dst = a.dst + ts.tok0 * a.k;
   int32_t* src = a.src_tok ? a.src_tok + ts.chunk_tok0 * a.k : nullptr;
   const int32_t tok_in_chunk0 = (int32_t)(ts.tok0 - ts.chunk_tok0);
-  for (int32_t s = threadIdx.x; s < ts.slots; s += kMetaThreads) {
-    const int32_t e = idx[s];
-    if (e < 0 || e >= a.E) continue;
-    const int32_t r = off[e] + base[e] + dst[s];
-    dst[s] = r;
-    if (src) src[r] = (int32_t)((a.src_relative ? 0 : ts.chunk_tok0) + tok_in_chunk0 + s / a.k);
+  // 8 slots per thread at a time: their index and rank loads are issued together
+  for (int32_t s0 = threadIdx.x; s0 < ts.slots; s0 += 8 * kMetaThreads) {
+    int32_t e[8], rk[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int32_t sl = s0 + u * kMetaThreads;
+      e[u] = sl < ts.slots ? idx[sl] : -1;
+      rk[u] = sl < ts.slots ? dst[sl] : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int32_t sl = s0 + u * kMetaThreads;
+      if (e[u] < 0 || e[u] >= a.E) continue;
+      const int32_t r = off[e[u]] + base[e[u]] + rk[u];
+      dst[sl] = r;
+      if (src)
+        src[r] = (int32_t)((a.src_relative ? 0 : ts.chunk_tok0) + tok_in_chunk0 + sl / a.k);
+    }
   }
 }
 
