@@ -255,7 +255,9 @@ def test_forward_full_size_sampled(moe, name, n_tok):
 @pytest.mark.parametrize("E,k,T,H,I", [(1024, 8, 1536, 128, 128),   # MOE_MAX_EXPERTS
                                        (64, 32, 600, 256, 192),     # MOE_MAX_TOPK
                                        (1, 1, 300, 64, 64),         # one expert, top-1
-                                       (16, 4, 257, 136, 200)])     # H, I not multiples of 64
+                                       (16, 4, 257, 136, 200),      # H, I not multiples of 64
+                                       (16, 4, 300, 776, 200)])     # 3 down column tiles,
+                                                                    # the last one partial
 def test_forward_limits_and_odd_shapes(moe, E, k, T, H, I):
     """The kernels' table and tile limits: the most experts and the largest top-k the ABI
     takes, a single expert, and widths that are multiples of 8 but not of the 64-wide K
