@@ -31,7 +31,10 @@
 
 // Build-time tuning knobs (the defaults are the shipped configuration).
 #ifndef MOE_GEMM_2SM
-#define MOE_GEMM_2SM 0  // 1: CTA pairs (tcgen05 cta_group::2, 256-row tiles); 0: single CTAs
+// Which GEMMs run on CTA pairs (tcgen05 cta_group::2, 256-row tiles, M=128 across the pair
+// for a tile of at most 128 rows) instead of single CTAs: bit 0 gate/up with TMA-loaded
+// rows, bit 1 down, bit 2 gate/up with gathered rows (0: none, 7: all).
+#define MOE_GEMM_2SM 0
 #endif
 #ifndef MOE_GEMM_BK
 #define MOE_GEMM_BK 64  // K per stage: 64 (128-byte swizzle rows) or 32 (64-byte swizzle rows)
@@ -113,8 +116,14 @@ struct Geo {
   static constexpr uint32_t kIdesc = umma_idesc_bf16_f32(kPair ? 2 * kRowsPerCta : kRowsPerCta, BN);
   // single CTA, one sub-tile: a tile holding at most 64 rows of its expert runs M=64 MMAs
   // (the accumulator's row r then sits in TMEM lane 32 (r / 16) + r % 16)
-  static constexpr bool kHalfTails = !kPair && !kTwoM && MOE_GEMM_HALF_TAILS != 0;
-  static constexpr uint32_t kIdescHalf = umma_idesc_bf16_f32(kRowsPerCta / 2, BN);
+  // CTA pair: a tile holding at most 128 rows of its expert runs M=128 MMAs across the pair
+  // (64 rows per CTA; each CTA's accumulator then holds tile columns 0..127 in TMEM lanes
+  // 0..63 and columns 128..255 in lanes 64..127, 128 TMEM columns wide)
+  static constexpr bool kHalfTails = !kTwoM && MOE_GEMM_HALF_TAILS != 0;
+  static constexpr int kHalfRows = kPair ? kRowsPerCta : kRowsPerCta / 2;  // rows of a half tile
+  static constexpr uint32_t kIdescHalf = umma_idesc_bf16_f32(kPair ? kRowsPerCta : kRowsPerCta / 2, BN);
+  // bytes one stage of a pair's half tile brings to the leader's barrier (both CTAs)
+  static constexpr uint32_t kTxBytesHalf = 2 * (kABytes / 2 + kBBytes);
   // epilogue warps: kTwoM may use two per TMEM lane quarter (each takes half the columns)
   static constexpr int kEpiWarps = kTwoM ? MOE_GEMM_EPI_WARPS_2M : 4;
 };
@@ -260,7 +269,9 @@ __device__ __forceinline__ void store_block(const uint32_t (&packed)[16], uint8_
 // One persistent CTA (kPair = false) or CTA pair (kPair = true, cluster of 2) per tile
 // stream.  In a pair, the even CTA ("leader") owns the full-stage barriers and the MMA
 // issue; both CTAs load their own halves, run their own epilogue on their own TMEM rows,
-// and report back to the leader.
+// and report back to the leader.  A pair's tile of at most 128 rows of its expert runs
+// M=128 MMAs (64 rows per CTA, loaded as 64-row boxes); with gathered A rows each CTA's
+// gathering warps copy its own rows and arrive on the leader's barrier.
 //
 // kTwoM (single CTA): a tile is 256 rows of one expert by one N tile, staged as two 128-row
 // A sub-tiles that share every B stage, each with its own 128 x 256 TMEM accumulator (the
@@ -271,8 +282,10 @@ __device__ __forceinline__ void store_block(const uint32_t (&packed)[16], uint8_
 // accumulator to alternate with, the MMA warp starts a tile's first-sub-tile MMAs as soon
 // as the epilogue has read that accumulator, and holds back (up to kStages - 1 stages) the
 // second sub-tile's MMAs until the epilogue has read the other one.
+// tmA64 / tmB64: the same matrices with 64-row boxes (the CTA pair's half tiles).
 template <bool kSwiGLU, bool kPair, bool kGather, bool kTwoM>
 __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensorMap* tmB,
+                                          const CUtensorMap* tmA64, const CUtensorMap* tmB64,
                                           const KParams& p) {
   using G = Geo<kPair, kTwoM>;
   constexpr int STAGES = G::kStages;
@@ -289,7 +302,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   constexpr bool kWarpStages =
       kGather && !kTwoM && MOE_GEMM_GATHER_MODE == 1 && STAGES == kGatherThreads / 32;
   static_assert(!kTwoM || kMaxHeld >= 0, "ring too shallow for the gathered two-sub-tile kernel");
-  static_assert(!(kGather && kPair), "gathered A rows are implemented for single CTAs");
+  static_assert(!(kWarpStages && kPair), "one ring slot per gathering warp: single CTAs only");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -311,9 +324,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   for (int32_t i = threadIdx.x; i <= E; i += blockDim.x) off[i] = p.offsets[i];
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      // gathered A: the weight producer's arrival plus one per A-gathering thread (or one
-      // per slot-owning gathering warp)
-      mbar_init(&ctl->full[s], kGather ? 1 + (kWarpStages ? 1 : kGatherThreads) : 1);
+      // gathered A: the weight producer's arrival plus one per A-gathering warp (or one per
+      // slot-owning gathering warp); CTA pair: both CTAs' gathering warps arrive on the
+      // leader's barrier
+      mbar_init(&ctl->full[s],
+                kGather ? 1 + (kWarpStages ? 1 : (kPair ? 2 : 1) * (kGatherThreads / 32)) : 1);
       mbar_init(&ctl->empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -327,6 +342,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(tmA);
     tma_prefetch_desc(tmB);
+    if (kPair) {
+      tma_prefetch_desc(tmA64);
+      tma_prefetch_desc(tmB64);
+    }
   }
   if (warp == 1) {
     if (kPair) {
@@ -371,9 +390,31 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   auto has_m1 = [&](const Tile& t) {
     return kTwoM && off[t.e + 1] - off[t.e] > t.m * G::kTileM + kRowsPerCta;
   };
-  // kHalfTails: whether tile t holds at most 64 rows of its expert (M=64 MMAs)
+  // kHalfTails: whether tile t holds at most kHalfRows rows of its expert (single CTA: M=64
+  // MMAs; pair: M=128 MMAs, 64 rows per CTA)
   auto is_half = [&](const Tile& t) {
-    return G::kHalfTails && off[t.e + 1] - off[t.e] - t.m * G::kTileM <= kRowsPerCta / 2;
+    return G::kHalfTails && off[t.e + 1] - off[t.e] - t.m * G::kTileM <= G::kHalfRows;
+  };
+  // first tile row this CTA stages (pair: CTA 1 takes the second 128 rows, or of a half tile
+  // the second 64)
+  auto cta_row = [&](bool half) {
+    return kPair ? (int32_t)rank * (half ? kRowsPerCta / 2 : kRowsPerCta) : 0;
+  };
+  // B rows of tile t this CTA stages (pair: CTA 0 the gate rows of the 128-column tile and
+  // CTA 1 the up rows; of a gate/up half tile each CTA 64 gate rows and the same 64 up rows,
+  // so that the columns of one lane half pair gate with up)
+  auto stage_b = [&](const Tile& t, bool half, uint8_t* b_dst, uint32_t bar, int32_t kb,
+                     uint64_t pol) {
+    if (!kPair) return;
+    if (kSwiGLU && half) {
+      const int32_t g0 = t.e * p.b_rows + t.n * (BN / 2) + (int32_t)rank * (BN / 4);
+      tma_load_2d_pair(b_dst, tmB64, bar, kb * BK, g0, pol);
+      tma_load_2d_pair(b_dst + G::kBBytes / 2, tmB64, bar, kb * BK, g0 + p.up_off, pol);
+    } else {
+      const int32_t brow = kSwiGLU ? t.e * p.b_rows + t.n * (BN / 2) + (int32_t)rank * p.up_off
+                                   : t.e * p.b_rows + t.n * BN + (int32_t)rank * (BN / 2);
+      tma_load_2d_pair(b_dst, tmB, bar, kb * BK, brow, pol);
+    }
   };
 
   if (warp == 0 && kGather) {
@@ -391,17 +432,24 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
         const Tile t = decode_tile<G::kTileM>(L, tile_start, off, E, p.n_tiles);
         const int32_t brow = t.e * p.b_rows + t.n * (kSwiGLU ? BN / 2 : BN);
+        const bool half = is_half(t);
         for (int32_t kb = 0; kb < p.num_kb; ++kb) {
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort, p.status)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&ctl->full[stage], G::kBBytes);
           uint8_t* b_dst = sB + stage * G::kBBytes;
-          tma_load_2d(b_dst, tmB, &ctl->full[stage], kb * BK, brow, pol_w);
-          if (kSwiGLU)
-            tma_load_2d(b_dst + G::kBBytes / 2, tmB, &ctl->full[stage], kb * BK, brow + p.up_off,
-                        pol_w);
+          if (kPair) {
+            // both CTAs' weight halves count on the leader's barrier
+            if (leader) mbar_arrive_expect_tx(&ctl->full[stage], 2 * G::kBBytes);
+            stage_b(t, half, b_dst, mapa_shared(smem_u32(&ctl->full[stage]), 0), kb, pol_w);
+          } else {
+            mbar_arrive_expect_tx(&ctl->full[stage], G::kBBytes);
+            tma_load_2d(b_dst, tmB, &ctl->full[stage], kb * BK, brow, pol_w);
+            if (kSwiGLU)
+              tma_load_2d(b_dst + G::kBBytes / 2, tmB, &ctl->full[stage], kb * BK,
+                          brow + p.up_off, pol_w);
+          }
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -410,7 +458,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
           }
         }
       }
-      if (!ok)
+      if (!ok && leader)
         for (int s = 0; s < STAGES; ++s)
           if (armed & (1u << s)) mbar_drain(&ctl->full[s], (armed_parity >> s) & 1u, 100000000ull);
     }
@@ -452,7 +500,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       if (L + n_streams < p.total_tiles) load_tokens(L + n_streams, next_tok);
       for (int32_t kb = 0; kb < p.num_kb; ++kb, ++sigma) {
         if ((sigma & (STAGES - 1)) != gw) continue;
-        if (!mbar_wait(&ctl->empty[gw], phase ^ 1u, abort, p.status)) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&ctl->empty[gw], phase ^ 1u, abort, p.status))) {
           ok = false;
           break;
         }
@@ -486,8 +534,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
     // each 128-row sub-tile with cp.async, into the 128-byte-swizzled K-major layout the MMA
     // reads (chunk j of row r at position j ^ (r % 8)); a warp instruction covers 4 whole
     // 128-byte row segments.  A thread keeps kDepth + 1 stages of copies in flight; when
-    // its oldest stage has landed it makes the writes visible to the async proxy and
-    // arrives on that stage's full barrier.
+    // its oldest stage has landed it makes the writes visible to the async proxy, and once
+    // every lane of the warp has, one lane arrives on that stage's full barrier (one arrival
+    // per warp: for a CTA pair the arrivals cross to the other SM, and 128 per stage from
+    // each CTA would cost more than the copies).
     constexpr int kDepth = kGatherDepth;
     constexpr int kSub = G::kSubM;
     const int gw = warp - kFirstGatherWarp, j = lane & 7, sub = lane >> 3;
@@ -499,11 +549,13 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
     int32_t issued = 0, arrived = 0;
     bool ok = true;
     const int32_t* gat = p.gather;  // gathered A has one row segment
+    // (every wait's outcome is made warp-uniform, so that the lanes leave the loop together
+    // and the per-warp arrivals below never wait on a lane that has gone)
     // token index of each row this thread copies in tile L (rows past the expert re-read
     // its last row)
     auto load_tokens = [&](int32_t L2, int32_t (&tok)[kSub * 8]) {
       const Tile t2 = decode_tile<G::kTileM>(L2, tile_start, off, E, p.n_tiles);
-      const int32_t row0 = off[t2.e] + t2.m * G::kTileM;
+      const int32_t row0 = off[t2.e] + t2.m * G::kTileM + cta_row(is_half(t2));
       const int32_t last = off[t2.e + 1] - 1;
 #pragma unroll
       for (int h = 0; h < kSub; ++h)
@@ -515,6 +567,15 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
     // spent behind the tile's copies instead of at the next tile boundary
     int32_t next_tok[kSub * 8];
     if (stream_id < p.total_tiles) load_tokens(stream_id, next_tok);
+    // a stage's full barrier (the leader's, for a CTA pair: its MMAs read both CTAs' rows),
+    // once per warp after every lane's copies of the stage are visible to the async proxy
+    auto arrive_full = [&](int s) {
+      __syncwarp();
+      if (lane == 0) {
+        if (kPair) mbar_arrive_cluster(mapa_shared(smem_u32(&ctl->full[s]), 0));
+        else mbar_arrive(&ctl->full[s]);
+      }
+    };
     for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
       const Tile t = decode_tile<G::kTileM>(L, tile_start, off, E, p.n_tiles);
       const int n_sub = has_m1(t) ? 2 : 1;
@@ -529,7 +590,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       }
       if (L + n_streams < p.total_tiles) load_tokens(L + n_streams, next_tok);
       for (int32_t kb = 0; kb < p.num_kb; ++kb) {
-        if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, abort, p.status)) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&ctl->empty[stage], phase ^ 1u, abort, p.status))) {
           ok = false;
           break;
         }
@@ -554,7 +615,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
         if (issued - arrived > kDepth) {
           cp_async_wait<kDepth>();
           fence_async_smem();
-          mbar_arrive(&ctl->full[arrived % STAGES]);
+          arrive_full(arrived % STAGES);
           ++arrived;
         }
         if (++stage == STAGES) {
@@ -565,7 +626,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
     }
     cp_async_wait<0>();
     fence_async_smem();
-    for (; arrived < issued; ++arrived) mbar_arrive(&ctl->full[arrived % STAGES]);
+    for (; arrived < issued; ++arrived) arrive_full(arrived % STAGES);
     (void)ok;
   } else if (warp == 0) {
     // ---------------- TMA producer (both CTAs) ----------------
@@ -582,11 +643,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
         // A row and B row of tile L (of this CTA's tile stream)
         const Tile t = decode_tile<G::kTileM>(L, tile_start, off, E, p.n_tiles);
-        const int32_t row0 = off[t.e] + t.m * G::kTileM + (int32_t)rank * kRowsPerCta;
-        const int32_t brow =
-            kSwiGLU  // pair: the even CTA stages the gate rows, the odd one the up rows
-                ? t.e * p.b_rows + t.n * (BN / 2) + (kPair ? (int32_t)rank * p.up_off : 0)
-                : t.e * p.b_rows + t.n * BN + (kPair ? (int32_t)rank * (BN / 2) : 0);
+        const bool half = kPair && is_half(t);
+        const int32_t row0 = off[t.e] + t.m * G::kTileM + cta_row(half);
+        const int32_t brow = t.e * p.b_rows + t.n * (kSwiGLU ? BN / 2 : BN);  // single CTA
         const bool m1 = has_m1(t);
         const uint32_t tx = kTwoM ? (m1 ? G::kStageBytes : G::kABytes + G::kBBytes) : G::kTxBytes;
         const CUtensorMap* mapA = tmA;
@@ -598,10 +657,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
           uint8_t* a_dst = sA + stage * G::kAStageBytes;
           uint8_t* b_dst = sB + stage * G::kBBytes;
           if (kPair) {
-            if (leader) mbar_arrive_expect_tx(&ctl->full[stage], G::kTxBytes);
+            if (leader)
+              mbar_arrive_expect_tx(&ctl->full[stage], half ? G::kTxBytesHalf : G::kTxBytes);
             const uint32_t bar = mapa_shared(smem_u32(&ctl->full[stage]), 0);
-            tma_load_2d_pair(a_dst, mapA, bar, kb * BK, row0, pol_a);
-            tma_load_2d_pair(b_dst, tmB, bar, kb * BK, brow, pol_w);
+            tma_load_2d_pair(a_dst, half ? tmA64 : mapA, bar, kb * BK, row0, pol_a);
+            stage_b(t, half, b_dst, bar, kb, pol_w);
           } else {
             mbar_arrive_expect_tx(&ctl->full[stage], tx);
             tma_load_2d(a_dst, mapA, &ctl->full[stage], kb * BK, row0, pol_a);
@@ -736,7 +796,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
           if (is_half(t)) idesc = G::kIdescHalf;
         }
         for (int32_t kb = 0; kb < p.num_kb; ++kb) {
-          if (!mbar_wait(&ctl->full[stage], phase, abort, p.status)) {
+          // (pair with gathered rows: the other CTA's gathering threads released its rows)
+          if (!mbar_wait<kPair && kGather>(&ctl->full[stage], phase, abort, p.status)) {
             ok = false;
             break;
           }
@@ -748,7 +809,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
             // advance 16 bf16 = 32 bytes along K inside the swizzled row
             const uint64_t ad = kmajor_desc<kSwizzleBytes>(a_addr + kk * 32);
             const uint64_t bd = kmajor_desc<kSwizzleBytes>(b_addr + kk * 32);
-            if (kPair) umma_bf16_pair(d_tmem, ad, bd, G::kIdesc, (kb | kk) != 0);
+            if (kPair) umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0);
             else umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
           }
           issued = true;
@@ -800,13 +861,52 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
         const int32_t* offs = off;
         __nv_bfloat16* out = p.out;
         const int64_t out_rows = p.out_rows;
-        const int32_t first = t.m * G::kTileM + (int32_t)rank * kRowsPerCta + h * kRowsPerCta;
+        const bool hf = is_half(t);  // (`half` is the kTwoM column half of this warp)
+        const int32_t first = t.m * G::kTileM + cta_row(hf) + h * kRowsPerCta;
         const int32_t rows_valid = offs[t.e + 1] - offs[t.e] - first;
-        const int rpw = is_half(t) ? 16 : 32;  // M=64 accumulator: 16 rows per lane quarter
-        const bool row_ok = rpw == 32 ? r < rows_valid : (lane < 16 && q * 16 + lane < rows_valid);
         const int64_t row_base = (int64_t)offs[t.e] + first;  // output row of TMEM lane 0
         const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * BN;
-        if (kSwiGLU) {
+        if (kPair && hf) {
+          // M=128 across the pair: this CTA's 64 rows; lane quarter q holds rows
+          // 32 (q % 2) .. +31 and tile columns 128 (q / 2) .. +127 in TMEM columns 0..127
+          // (gate/up: gate columns 0..63 and the matching up columns 64..127)
+          const int rq = q & 1, ch = q >> 1;
+          const bool ok_row = rq * 32 + lane < rows_valid;
+          constexpr int kHalfChunks = kSwiGLU ? 2 : 4;
+#pragma unroll 1
+          for (int c = 0; c < kHalfChunks; ++c) {
+            uint32_t packed[16];
+            int32_t col0;
+            if (kSwiGLU) {
+              uint32_t g[32], u[32];
+              tmem_ld_32cols(t_row + c * 32, g);
+              tmem_ld_32cols(t_row + 64 + c * 32, u);
+              tmem_ld_wait2(g, u);
+              col0 = t.n * (BN / 2) + ch * 64 + c * 32;
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+                const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+                const float a0 = __fdividef(g0, 1.0f + __expf(-g0)) * u0;
+                const float a1 = __fdividef(g1, 1.0f + __expf(-g1)) * u1;
+                packed[i] = pack_bf16x2(a0, a1);
+              }
+            } else {
+              uint32_t acc[32];
+              tmem_ld_32cols(t_row + c * 32, acc);
+              tmem_ld_wait(acc);
+              col0 = t.n * BN + ch * 128 + c * 32;
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                packed[i] =
+                    pack_bf16x2(__uint_as_float(acc[2 * i]), __uint_as_float(acc[2 * i + 1]));
+            }
+            store_block(packed, wbuf, lane, rq, ok_row, rows_valid, row_base, col0, p,
+                        p.out, p.out_rows, 32);
+          }
+        } else if (kSwiGLU) {
+          const int rpw = hf ? 16 : 32;  // M=64 accumulator: 16 rows per lane quarter
+          const bool row_ok = rpw == 32 ? r < rows_valid : (lane < 16 && q * 16 + lane < rows_valid);
           constexpr int kChunks = (BN / 2) / 32 / kParts;
 #pragma unroll 1
           for (int c = half * kChunks; c < (half + 1) * kChunks; ++c) {
@@ -830,6 +930,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
                         out_rows, rpw);
           }
         } else {
+          const int rpw = hf ? 16 : 32;
+          const bool row_ok = rpw == 32 ? r < rows_valid : (lane < 16 && q * 16 + lane < rows_valid);
           constexpr int kChunks = BN / 32 / kParts;
 #pragma unroll 1
           for (int c = half * kChunks; c < (half + 1) * kChunks; ++c) {
@@ -874,16 +976,18 @@ __global__ void __maxnreg__(128)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
                         const KParams p) {
-  gemm_body<kSwiGLU, false, kGather, kTwoM>(&tmA, &tmB, p);
+  gemm_body<kSwiGLU, false, kGather, kTwoM>(&tmA, &tmB, &tmA, &tmB, p);
 }
 
-// Launched with a cluster of 2 CTAs (cudaLaunchAttributeClusterDimension).
-template <bool kSwiGLU>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+// Launched with a cluster of 2 CTAs (cudaLaunchAttributeClusterDimension).  The same
+// register cap as the single-CTA kernel, for the combine that runs beside it.
+template <bool kSwiGLU, bool kGather>
+__global__ void __maxnreg__(128)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmB,
-                             const KParams p) {
-  gemm_body<kSwiGLU, true, false, false>(&tmA, &tmB, p);
+                             const __grid_constant__ CUtensorMap tmA64,
+                             const __grid_constant__ CUtensorMap tmB64, const KParams p) {
+  gemm_body<kSwiGLU, true, kGather, false>(&tmA, &tmB, &tmA64, &tmB64, p);
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -941,20 +1045,27 @@ bool make_tma_3d_f32(CUtensorMap* m, void* base, int32_t E, int32_t M, int32_t N
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool gemm_supports_gather() { return MOE_GEMM_2SM == 0; }
+bool gemm_supports_gather() { return true; }
+
+// Whether a GEMM kind runs on CTA pairs (MOE_GEMM_2SM bits).
+bool gemm_pair(bool swiglu, bool gather) {
+  const int bit = !swiglu ? 1 : (gather ? 2 : 0);
+  return ((MOE_GEMM_2SM >> bit) & 1) != 0;
+}
 
 // Which single-CTA variant a GEMM kind runs: two 128-row sub-tiles per 256-row tile
 // (MOE_GEMM_TWO_M bit 0: gate/up, bit 1: down) or one 128-row tile.
-bool gemm_two_m(bool swiglu) {
-  if (MOE_GEMM_2SM != 0) return false;
+bool gemm_two_m(bool swiglu, bool gather) {
+  if (gemm_pair(swiglu, gather)) return false;
   return ((MOE_GEMM_TWO_M >> (swiglu ? 0 : 1)) & 1) != 0;
 }
 
-int64_t gemm_total_tiles(const int32_t* counts_host, int32_t E, int32_t out_cols, bool swiglu) {
+int64_t gemm_total_tiles(const int32_t* counts_host, int32_t E, int32_t out_cols, bool swiglu,
+                         bool gather) {
   const int32_t bn = swiglu ? BN / 2 : BN;
-  const int32_t tm = MOE_GEMM_2SM != 0 ? Geo<true>::kTileM
-                     : gemm_two_m(swiglu)  ? Geo<false, true>::kTileM
-                                           : Geo<false>::kTileM;
+  const int32_t tm = gemm_pair(swiglu, gather)    ? Geo<true>::kTileM
+                     : gemm_two_m(swiglu, gather) ? Geo<false, true>::kTileM
+                                                  : Geo<false>::kTileM;
   const int64_t n_tiles = (out_cols + bn - 1) / bn;
   int64_t m_tiles = 0;
   for (int32_t e = 0; e < E; ++e) m_tiles += (counts_host[e] + tm - 1) / tm;
@@ -963,8 +1074,9 @@ int64_t gemm_total_tiles(const int32_t* counts_host, int32_t E, int32_t out_cols
 
 cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cudaStream_t s,
                                 int* err_detail) {
-  constexpr bool kPair = MOE_GEMM_2SM != 0;
-  const bool two_m = gemm_two_m(swiglu);
+  const bool gather = a.gather != nullptr;
+  const bool kPair = gemm_pair(swiglu, gather);
+  const bool two_m = gemm_two_m(swiglu, gather);
   *err_detail = 0;
   if (a.total_tiles <= 0) return cudaSuccess;
   if (a.total_tiles > 0x7fffffff || a.E > kMaxE) {
@@ -973,8 +1085,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
   }
   CUtensorMap mA, mB;
   const int32_t bn = swiglu ? BN / 2 : BN;
-  const bool gather = a.gather != nullptr;
-  if (gather && (kPair || !swiglu)) {
+  if (gather && !swiglu) {
     *err_detail = 1;
     return cudaErrorInvalidValue;
   }
@@ -983,7 +1094,12 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
                                : make_map(&mA, a.A, a.rows, a.K, kRowsPerCta);
   const bool map_b_ok = make_map(&mB, a.B, (int64_t)a.E * a.b_rows, a.K,
                                  kPair ? BN / 2 : (swiglu ? BN / 2 : BN));
-  if (!map_a_ok || !map_b_ok) {
+  // the pair's half tiles: 64-row boxes of A (each CTA's rows) and of the weights
+  CUtensorMap mA64 = mA, mB64 = mB;
+  const bool map_h_ok =
+      !kPair || ((gather || make_map(&mA64, a.A, a.rows, a.K, kRowsPerCta / 2)) &&
+                 make_map(&mB64, a.B, (int64_t)a.E * a.b_rows, a.K, BN / 4));
+  if (!map_a_ok || !map_b_ok || !map_h_ok) {
     *err_detail = 2;
     return cudaErrorInvalidValue;
   }
@@ -1004,10 +1120,14 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
   p.gsrc_rows = a.gather_src_rows;
   p.out_rows = a.rows;
   p.K = a.K;
-  const size_t smem = two_m ? smem_bytes<false, true>() : smem_bytes<kPair>();
+  const size_t smem =
+      two_m ? smem_bytes<false, true>() : (kPair ? smem_bytes<true>() : smem_bytes<false>());
   cudaError_t e;
   if (kPair) {
-    auto k = swiglu ? grouped_gemm_pair_kernel<true> : grouped_gemm_pair_kernel<false>;
+    auto k = gather ? grouped_gemm_pair_kernel<true, true>
+                    : (swiglu ? grouped_gemm_pair_kernel<true, false>
+                              : grouped_gemm_pair_kernel<false, false>);
+    const int variant = gather ? 2 : (swiglu ? 1 : 0);
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchAttribute attr[1];
@@ -1016,16 +1136,16 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.blockDim = dim3(gather ? gemm_threads<true>() : gemm_threads<false>(), 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     // persistent: as many CTA pairs as can be resident at once
-    static int max_pairs[64] = {0};
+    static int max_pairs[3][64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
-    int& mp = max_pairs[dev & 63];
+    int& mp = max_pairs[variant][dev & 63];
     if (mp <= 0) {
       cfg.gridDim = dim3(num_sms, 1, 1);
       int n = 0;
@@ -1035,7 +1155,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
     }
     const int streams = (int)(a.total_tiles < mp ? a.total_tiles : mp);
     cfg.gridDim = dim3(2 * streams, 1, 1);
-    e = cudaLaunchKernelEx(&cfg, k, mA, mB, p);
+    e = cudaLaunchKernelEx(&cfg, k, mA, mB, mA64, mB64, p);
     if (e != cudaSuccess) return e;
   } else {
     auto k = two_m ? (gather ? grouped_gemm_kernel<true, true, true>

@@ -88,11 +88,12 @@ bool make_tma_2d_bf16(CUtensorMap* m, const void* base, int64_t rows, int32_t co
 // True when the build's grouped GEMM supports a gathered A operand.
 bool gemm_supports_gather();
 
-// Number of 128-row x N-column output tiles for the given host counts.
 // 3-D fp32 tensor map over [E][M][N] (row-major per expert) with a 32 x 32 box and the
 // 128-byte swizzle: the target of the weight-gradient stores and add-reductions.
 bool make_tma_3d_f32(CUtensorMap* m, void* base, int32_t E, int32_t M, int32_t N);
-int64_t gemm_total_tiles(const int32_t* counts_host, int32_t E, int32_t out_cols, bool swiglu);
+// Output tiles of a GEMM launch (tile height per the kernel variant that runs it).
+int64_t gemm_total_tiles(const int32_t* counts_host, int32_t E, int32_t out_cols, bool swiglu,
+                         bool gather);
 
 cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cudaStream_t s,
                                 int* err_detail);

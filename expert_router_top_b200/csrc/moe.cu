@@ -462,7 +462,7 @@ moe_status_t gemm_call(const void* A, int64_t rows, const void* B, void* out,
   g.K = K;
   g.out_cols = out_cols;
   g.b_rows = b_rows;
-  g.total_tiles = gemm_total_tiles(counts_host, E, out_cols, swiglu);
+  g.total_tiles = gemm_total_tiles(counts_host, E, out_cols, swiglu, gather != nullptr);
   g.status = status;
   if (g.total_tiles == 0) return MOE_OK;
   int detail = 0;
