@@ -29,7 +29,9 @@ __device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
 
 __device__ uint32_t g_range_flags;  // checks build: a row index outside its buffer was seen
 
-// X[dst[t*k+j]] = hidden[t] for every j < k.
+// X[dst[t*k+j]] = hidden[t] for every j < k.  The warp loads the next U x 512 bytes of the
+// token row before it stores the k copies of the current ones, so the row's (usually cold)
+// reads stay in flight while the stores issue.
 template <int U>
 __global__ void __launch_bounds__(kRowThreads) permute_kernel(const uint4* __restrict__ hidden,
                                                               const int32_t* __restrict__ dst,
@@ -41,12 +43,18 @@ __global__ void __launch_bounds__(kRowThreads) permute_kernel(const uint4* __res
   if (t >= Tc) return;
   const int32_t d_lane = lane < k ? dst[t * k + lane] : 0;
   const uint4* src = hidden + t * H8;
+  uint4 cur[U], nxt[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int32_t v = u * 32 + lane;
+    cur[u] = v < H8 ? ldg_stream(src + v) : make_uint4(0, 0, 0, 0);
+  }
   for (int32_t v0 = 0; v0 < H8; v0 += 32 * U) {
-    uint4 val[U];
+    const int32_t v1 = v0 + 32 * U;
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int32_t v = v0 + u * 32 + lane;
-      if (v < H8) val[u] = ldg_stream(src + v);
+      const int32_t v = v1 + u * 32 + lane;
+      nxt[u] = v < H8 ? ldg_stream(src + v) : make_uint4(0, 0, 0, 0);
     }
     for (int j = 0; j < k; ++j) {
       const int32_t d = __shfl_sync(0xffffffffu, d_lane, j);
@@ -55,9 +63,11 @@ __global__ void __launch_bounds__(kRowThreads) permute_kernel(const uint4* __res
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int32_t v = v0 + u * 32 + lane;
-        if (v < H8) row[v] = val[u];
+        if (v < H8) row[v] = cur[u];
       }
     }
+#pragma unroll
+    for (int u = 0; u < U; ++u) cur[u] = nxt[u];
   }
 }
 
@@ -117,23 +127,26 @@ __global__ void __launch_bounds__(kRowThreads) unpermute_kernel(const uint4* __r
 }
 
 // The same combine with k fixed at compile time: a warp issues the loads of all k rows'
-// 16-byte vectors before the first FMA, so k x 512 bytes per warp are in flight instead of
-// one row's, and loops over tokens (grid-stride) so that the grid can be sized to the GPU.
-// The arithmetic is the kernel's above: acc = 0, then acc = fma(w_j, y_j, acc) for
-// j = 0 .. k-1, so both give the same bits.
+// 16-byte vectors -- for k < 8 of 8 / k vectors per lane -- before the first FMA, so about
+// 8 x 512 bytes per warp are in flight instead of one row's, and loops over tokens
+// (grid-stride) so that the grid can be sized to the GPU.  The arithmetic is the kernel's
+// above: acc = 0, then acc = fma(w_j, y_j, acc) for j = 0 .. k-1, so both give the same bits.
+// At most 64 registers per thread (four CTAs per SM): the combine that runs beside a grouped
+// GEMM must fit on the SM sub-partitions next to the GEMM's warps.
 template <int KT>
-__global__ void __launch_bounds__(kRowThreads) unpermute_k_kernel(const uint4* __restrict__ Y,
-                                                                  const int32_t* __restrict__ dst,
-                                                                  const float* __restrict__ w,
-                                                                  int64_t Tc, int32_t H8,
-                                                                  uint4* __restrict__ out,
-                                                                  int64_t rows_cap) {
+__global__ void __launch_bounds__(kRowThreads, 4) unpermute_k_kernel(const uint4* __restrict__ Y,
+                                                                     const int32_t* __restrict__ dst,
+                                                                     const float* __restrict__ w,
+                                                                     int64_t Tc, int32_t H8,
+                                                                     uint4* __restrict__ out,
+                                                                     int64_t rows_cap) {
+  constexpr int V = KT >= 8 ? 1 : 8 / KT;  // vectors per lane per pass
   const int lane = threadIdx.x & 31;
   const int64_t n_warps = (int64_t)gridDim.x * kTokPerCta;
   for (int64_t t = (int64_t)blockIdx.x * kTokPerCta + (threadIdx.x >> 5); t < Tc; t += n_warps) {
     const int32_t d_lane = lane < KT ? dst[t * KT + lane] : 0;
     const float w_lane = lane < KT ? w[t * KT + lane] : 0.f;
-    const uint4* row[KT];
+    int32_t row[KT];  // row index (a 32-bit register each; the address is formed per load)
     float wj[KT];
     bool ok[KT];
 #pragma unroll
@@ -141,31 +154,40 @@ __global__ void __launch_bounds__(kRowThreads) unpermute_k_kernel(const uint4* _
       const int32_t d = __shfl_sync(0xffffffffu, d_lane, j);
       wj[j] = __shfl_sync(0xffffffffu, w_lane, j);
       ok[j] = check_row(d, rows_cap, &g_range_flags);
-      row[j] = Y + (int64_t)(ok[j] ? d : 0) * H8;
+      row[j] = ok[j] ? d : 0;
     }
-    for (int32_t v = lane; v < H8; v += 32) {
-      uint4 y[KT];
+    for (int32_t v0 = lane; v0 < H8; v0 += 32 * V) {
+      uint4 y[V][KT];
 #pragma unroll
-      for (int j = 0; j < KT; ++j) y[j] = ldg_stream(row[j] + v);
-      float acc[8];
+      for (int u = 0; u < V; ++u)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-#pragma unroll
-      for (int j = 0; j < KT; ++j) {
-        if (!ok[j]) continue;
-        const uint32_t q[4] = {y[j].x, y[j].y, y[j].z, y[j].w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          acc[2 * i] = fmaf(wj[j], bf16lo(q[i]), acc[2 * i]);
-          acc[2 * i + 1] = fmaf(wj[j], bf16hi(q[i]), acc[2 * i + 1]);
+        for (int j = 0; j < KT; ++j) {
+          const int32_t v = v0 + 32 * u;
+          y[u][j] = v < H8 ? ldg_stream(Y + (int64_t)row[j] * H8 + v) : make_uint4(0, 0, 0, 0);
         }
+#pragma unroll
+      for (int u = 0; u < V; ++u) {
+        const int32_t v = v0 + 32 * u;
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+        for (int j = 0; j < KT; ++j) {
+          if (!ok[j]) continue;
+          const uint32_t q[4] = {y[u][j].x, y[u][j].y, y[u][j].z, y[u][j].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            acc[2 * i] = fmaf(wj[j], bf16lo(q[i]), acc[2 * i]);
+            acc[2 * i + 1] = fmaf(wj[j], bf16hi(q[i]), acc[2 * i + 1]);
+          }
+        }
+        uint4 o;
+        o.x = pack_bf16x2(acc[0], acc[1]);
+        o.y = pack_bf16x2(acc[2], acc[3]);
+        o.z = pack_bf16x2(acc[4], acc[5]);
+        o.w = pack_bf16x2(acc[6], acc[7]);
+        if (v < H8) out[t * H8 + v] = o;
       }
-      uint4 o;
-      o.x = pack_bf16x2(acc[0], acc[1]);
-      o.y = pack_bf16x2(acc[2], acc[3]);
-      o.z = pack_bf16x2(acc[4], acc[5]);
-      o.w = pack_bf16x2(acc[6], acc[7]);
-      out[t * H8 + v] = o;
     }
   }
 }
