@@ -70,28 +70,9 @@ __device__ __forceinline__ void fence_mbar_init() {
 #define MOE_WAIT_HINT_NS 200000
 #endif
 
-// kCluster: acquire at cluster scope (arrivals released by threads of the other CTA of a
-// pair, whose shared-memory writes the waiting thread's MMAs then read).
-template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
-  if (kCluster && MOE_WAIT_HINT_NS > 0) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "n"(MOE_WAIT_HINT_NS)
-        : "memory");
-  } else if (kCluster) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-  } else if (MOE_WAIT_HINT_NS > 0) {
+  if (MOE_WAIT_HINT_NS > 0) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
@@ -137,13 +118,12 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 // Bounded wait for the phase with the given parity.  Returns false when it gave up: on
 // its own timeout after limit_ns (then it sets *abort and ORs MOE_DEV_TIMEOUT into *status)
 // or because another role of the CTA already raised *abort.
-template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint32_t* status, uint64_t limit_ns = kWaitLimitNs) {
-  if (mbar_try_wait<kCluster>(bar, parity)) return true;
+  if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t n = 1;; ++n) {
-    if (mbar_try_wait<kCluster>(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     // (with a long suspend hint every return is after a sleep: check every time)
     if (MOE_WAIT_HINT_NS >= 10000 || (n & 31u) == 0) {
       if (*abort) return false;
@@ -406,8 +386,13 @@ __device__ __forceinline__ void cluster_sync() {
 }
 
 // Arrive on an mbarrier that may live in another CTA of the cluster.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+// Arrive on an mbarrier of either CTA of the pair (a shared::cluster address), release at
+// CTA scope: the form cluster pipelines use for the other CTA's barriers.  (A release at
+// cluster scope waits for every memory operation the thread still has in flight -- the
+// copies of later stages, the stores of the epilogue -- which cost a gathering warp ~2000
+// cycles per stage.)
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
 }
 

@@ -75,6 +75,9 @@
 #ifndef MOE_GEMM_TWO_M
 #define MOE_GEMM_TWO_M 0  // 256-row tiles of two 128-row sub-tiles: bit 0 gate/up, bit 1 down
 #endif
+#ifndef MOE_GEMM_GATHER_DEPTH_2SM
+#define MOE_GEMM_GATHER_DEPTH_2SM 2  // CTA pair, gathered A: stages of copies run ahead
+#endif
 #ifndef MOE_GEMM_B_POLICY
 #define MOE_GEMM_B_POLICY 2  // L2 policy of weight loads: 0 normal, 1 evict_first, 2 evict_last
 #endif
@@ -293,8 +296,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   constexpr int kFirstGatherWarp = 2 + kEpiWarps;
   // Gathering threads keep kGatherDepth + 1 stages of copies in flight and arrive on a
   // stage's full barrier only once they have issued the copies of the kGatherDepth stages
-  // after it, so those stages must be free (released by the MMA warp) by then.
-  constexpr int kGatherDepth = STAGES - 2 > 0 ? STAGES - 2 : 1;
+  // after it, so those stages must be free (released by the MMA warp) by then: the MMAs of
+  // stage s wait for those of stage s + kGatherDepth - STAGES.
+  constexpr int kGatherDepth =
+      kPair ? MOE_GEMM_GATHER_DEPTH_2SM : (STAGES - 2 > 0 ? STAGES - 2 : 1);
   // kTwoM: stages whose second-sub-tile MMAs the MMA warp may hold back (each held stage
   // stays unreleased); with gathered A the gathering threads' run-ahead must stay free.
   constexpr int kMaxHeld = STAGES - 1 - (kGather ? kGatherDepth : 0);
@@ -569,10 +574,13 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
     if (stream_id < p.total_tiles) load_tokens(stream_id, next_tok);
     // a stage's full barrier (the leader's, for a CTA pair: its MMAs read both CTAs' rows),
     // once per warp after every lane's copies of the stage are visible to the async proxy
+    // (CTA pair: released at CTA scope like the other arrivals of a pair on the leader's
+    // barriers -- at cluster scope the release waits for every copy the thread still has in
+    // flight, ~2000 cycles per stage)
     auto arrive_full = [&](int s) {
       __syncwarp();
       if (lane == 0) {
-        if (kPair) mbar_arrive_cluster(mapa_shared(smem_u32(&ctl->full[s]), 0));
+        if (kPair) mbar_arrive_remote(mapa_shared(smem_u32(&ctl->full[s]), 0));
         else mbar_arrive(&ctl->full[s]);
       }
     };
@@ -797,7 +805,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
         }
         for (int32_t kb = 0; kb < p.num_kb; ++kb) {
           // (pair with gathered rows: the other CTA's gathering threads released its rows)
-          if (!mbar_wait<kPair && kGather>(&ctl->full[stage], phase, abort, p.status)) {
+          if (!mbar_wait(&ctl->full[stage], phase, abort, p.status)) {
             ok = false;
             break;
           }
@@ -949,7 +957,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
           }
         }
         tc_fence_before();
-        if (kPair) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
+        if (kPair) mbar_arrive_remote(buf ? tempty_leader1 : tempty_leader0);
         else mbar_arrive(&ctl->tempty[buf]);
         ++use[h];
       }
