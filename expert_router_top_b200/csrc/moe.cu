@@ -723,8 +723,9 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
     // Pairs (c0, c1) = (2m, 2m+1).  G: GU(m) D(m) GU(m+1) D(m+1) ..., where GU / D are the
     // gate/up and down GEMMs of the pair in one tile sweep over its rows, laid out per expert
     // across both chunks (each expert's weight tiles are fetched once for the pair, and a row
-    // tile may hold rows of both chunks); D(m+1) waits until U(c0), U(c1) have read the
-    // pair's Y rows.  M: U(c0) U(c1) after D(m), beside GU(m+1).  The pair's rows fill both
+    // tile may hold rows of both chunks); D(m+1) waits until U(m), the combine of both
+    // chunks in one launch, has read the pair's Y rows.  M: U(m) after D(m), beside GU(m+1).
+    // The pair's rows fill both
     // halves of the X|Y and Act double buffers; dst holds pair-local rows.
     const std::vector<int64_t> pb = dims_bounds(dm);
     void* y_pair = ws + L.xy[0];
@@ -749,13 +750,14 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
         return MOE_ERR_CUDA;
       // a pair's combines run beside the next pair's gate/up GEMM (fewer CTAs, all resident
       // next to it) unless this is the last pair
+      // (one launch for both chunks: their tokens are adjacent and dst holds pair-local rows)
       const bool beside_gemm = 2 * (m + 1) < n_live;
-      for (int c = c0; c <= c1; ++c) {
-        ProfScope ps(MOE_KERNEL_UNPERMUTE, sm, len(c) * k, 0, 1);
-        if (launch_unpermute(y_pair, dst + bounds[c] * k, top_k_weights + bounds[c] * k, len(c),
-                             H, k, outp + bounds[c] * H, pair_cap, sm,
-                             beside_gemm ? MOE_UNPERM_BESIDE_GEMM_CTAS_PER_SM : 0) !=
-            cudaSuccess)
+      {
+        const int64_t t0 = bounds[c0], tn = bounds[c1 + 1] - bounds[c0];
+        ProfScope ps(MOE_KERNEL_UNPERMUTE, sm, tn * k, 0, 1);
+        if (launch_unpermute(y_pair, dst + t0 * k, top_k_weights + t0 * k, tn, H, k,
+                             outp + t0 * H, pair_cap, sm,
+                             beside_gemm ? MOE_UNPERM_BESIDE_GEMM_CTAS_PER_SM : 0) != cudaSuccess)
           return MOE_ERR_CUDA;
       }
       if (cudaEventRecord(ctx->ev_unperm[0], sm) != cudaSuccess) return MOE_ERR_CUDA;
