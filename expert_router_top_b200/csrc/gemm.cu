@@ -141,7 +141,7 @@ struct KParams {
   int32_t out_cols;  // valid output columns
   int32_t b_rows;    // B rows per expert
   int32_t up_off;    // row offset of W_up inside one expert's W_gate_up (= I)
-  int32_t total_tiles;
+  int32_t total_tiles;  // -1: count them here from the offsets (skipped on a bad index)
   const int32_t* gather;  // gathered A: token row of each permuted row (nullptr: plain A)
   const uint8_t* gsrc;    // gathered A: the token rows (hidden), and their stride in bytes
   int64_t gsrc_stride;
@@ -390,6 +390,13 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
   volatile int* abort = &ctl->abort;
+  // Tiles of the launch: given by the host, or (total_tiles < 0: the host has not seen the
+  // counts) the prefix over the experts -- none when the metadata of this call flagged an
+  // expert index out of range, whose offsets are then not to be used.
+  const int32_t total = p.total_tiles >= 0 ? p.total_tiles
+                        : (*reinterpret_cast<volatile uint32_t*>(p.status) & MOE_DEV_BAD_INDEX)
+                            ? 0
+                            : tile_start[E];
 
   // kTwoM: whether tile t has a second 128-row sub-tile (its expert has rows past the first)
   auto has_m1 = [&](const Tile& t) {
@@ -434,7 +441,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;
       bool ok = true;
-      for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
+      for (int32_t L = stream_id; L < total && ok; L += n_streams) {
         const Tile t = decode_tile<G::kTileM>(L, tile_start, off, E, p.n_tiles);
         const int32_t brow = t.e * p.b_rows + t.n * (kSwiGLU ? BN / 2 : BN);
         const bool half = is_half(t);
@@ -489,11 +496,11 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       for (int q = 0; q < 4; ++q) tok[q] = gat[min(row0 + q * 32 + lane, last)];
     };
     int32_t next_tok[4];
-    if (stream_id < p.total_tiles) load_tokens(stream_id, next_tok);
+    if (stream_id < total) load_tokens(stream_id, next_tok);
     uint32_t phase = 0;  // phase of this warp's slot
     int32_t sigma = 0;   // K blocks of this CTA so far (ring position)
     bool ok = true;
-    for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
+    for (int32_t L = stream_id; L < total && ok; L += n_streams) {
       const Tile t = decode_tile<G::kTileM>(L, tile_start, off, E, p.n_tiles);
       const bool half = is_half(t);  // M=64 MMAs read rows 0..63 only
       int32_t tok[4];
@@ -502,7 +509,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
         tok[q] = next_tok[q];
         if (!check_row(tok[q], p.gsrc_rows, &g_range_flags)) tok[q] = 0;
       }
-      if (L + n_streams < p.total_tiles) load_tokens(L + n_streams, next_tok);
+      if (L + n_streams < total) load_tokens(L + n_streams, next_tok);
       for (int32_t kb = 0; kb < p.num_kb; ++kb, ++sigma) {
         if ((sigma & (STAGES - 1)) != gw) continue;
         if (!__all_sync(0xffffffffu, mbar_wait(&ctl->empty[gw], phase ^ 1u, abort, p.status))) {
@@ -571,7 +578,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
     // the next tile's indices are loaded when a tile starts, so that their latency is
     // spent behind the tile's copies instead of at the next tile boundary
     int32_t next_tok[kSub * 8];
-    if (stream_id < p.total_tiles) load_tokens(stream_id, next_tok);
+    if (stream_id < total) load_tokens(stream_id, next_tok);
     // a stage's full barrier (the leader's, for a CTA pair: its MMAs read both CTAs' rows),
     // once per warp after every lane's copies of the stage are visible to the async proxy
     // (CTA pair: released at CTA scope like the other arrivals of a pair on the leader's
@@ -584,7 +591,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
         else mbar_arrive(&ctl->full[s]);
       }
     };
-    for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
+    for (int32_t L = stream_id; L < total && ok; L += n_streams) {
       const Tile t = decode_tile<G::kTileM>(L, tile_start, off, E, p.n_tiles);
       const int n_sub = has_m1(t) ? 2 : 1;
       // half tiles: only rows 0..63 are read by the M=64 MMAs (gathering warps 0 and 1)
@@ -596,7 +603,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
         if (!check_row(tok, p.gsrc_rows, &g_range_flags)) tok = 0;
         src[x] = p.gsrc + tok * p.gsrc_stride + j * 16;
       }
-      if (L + n_streams < p.total_tiles) load_tokens(L + n_streams, next_tok);
+      if (L + n_streams < total) load_tokens(L + n_streams, next_tok);
       for (int32_t kb = 0; kb < p.num_kb; ++kb) {
         if (!__all_sync(0xffffffffu, mbar_wait(&ctl->empty[stage], phase ^ 1u, abort, p.status))) {
           ok = false;
@@ -648,7 +655,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;  // per-stage bits, for the abort drain
       bool ok = true;
-      for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
+      for (int32_t L = stream_id; L < total && ok; L += n_streams) {
         // A row and B row of tile L (of this CTA's tile stream)
         const Tile t = decode_tile<G::kTileM>(L, tile_start, off, E, p.n_tiles);
         const bool half = kPair && is_half(t);
@@ -715,7 +722,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
           umma_bf16(tmem_base + h * BN, ad, bd, G::kIdesc, (kb | kk) != 0);
         }
       };
-      for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams) {
+      for (int32_t L = stream_id; L < total && ok; L += n_streams) {
         const Tile t = decode_tile<G::kTileM>(L, tile_start, off, E, p.n_tiles);
         const bool m1 = has_m1(t);
         if (!mbar_wait(&ctl->tempty[0], (use[0] & 1u) ^ 1u, abort, p.status)) {
@@ -789,7 +796,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       uint32_t phase = 0;
       bool ok = true, issued = false;
       int32_t it = 0;
-      for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams, ++it) {
+      for (int32_t L = stream_id; L < total && ok; L += n_streams, ++it) {
         const int buf = it & 1;
         const uint32_t tphase = (it >> 1) & 1;
         if (!mbar_wait(&ctl->tempty[buf], tphase ^ 1u, abort, p.status)) {
@@ -854,7 +861,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
     uint32_t use[2] = {0, 0};
     int32_t it = 0;
     bool ok = true;
-    for (int32_t L = stream_id; L < p.total_tiles && ok; L += n_streams, ++it) {
+    for (int32_t L = stream_id; L < total && ok; L += n_streams, ++it) {
       const Tile t = decode_tile<G::kTileM>(L, tile_start, off, E, p.n_tiles);
       const int n_acc = has_m1(t) ? 2 : 1;
       for (int h = 0; h < n_acc; ++h) {
@@ -1086,8 +1093,9 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
   const bool kPair = gemm_pair(swiglu, gather);
   const bool two_m = gemm_two_m(swiglu, gather);
   *err_detail = 0;
-  if (a.total_tiles <= 0) return cudaSuccess;
-  if (a.total_tiles > 0x7fffffff || a.E > kMaxE) {
+  // total_tiles < 0: the kernel counts them (the grid is then one CTA, or pair, per SM)
+  if (a.total_tiles == 0 || a.rows <= 0) return cudaSuccess;
+  if (a.total_tiles > 0x7fffffff || a.E > kMaxE || (a.total_tiles < 0 && !a.status)) {
     *err_detail = 1;
     return cudaErrorInvalidValue;
   }
@@ -1161,7 +1169,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
         n = num_sms / 2;
       mp = n < num_sms / 2 ? n : num_sms / 2;
     }
-    const int streams = (int)(a.total_tiles < mp ? a.total_tiles : mp);
+    const int streams = (int)(a.total_tiles >= 0 && a.total_tiles < mp ? a.total_tiles : mp);
     cfg.gridDim = dim3(2 * streams, 1, 1);
     e = cudaLaunchKernelEx(&cfg, k, mA, mB, mA64, mB64, p);
     if (e != cudaSuccess) return e;
@@ -1174,7 +1182,8 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
                                        : grouped_gemm_kernel<false, false, false>));
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const int streams = (int)(a.total_tiles < num_sms ? a.total_tiles : num_sms);
+    const int streams =
+        (int)(a.total_tiles >= 0 && a.total_tiles < num_sms ? a.total_tiles : num_sms);
     const int threads = two_m ? (gather ? gemm_threads<true, true>() : gemm_threads<false, true>())
                               : (gather ? gemm_threads<true>() : gemm_threads<false>());
     k<<<streams, threads, smem, s>>>(mA, mB, p);

@@ -40,14 +40,17 @@ cudaError_t launch_metadata(const MetaArgs& a, cudaStream_t s);
 
 // rows_cap: rows of X (permute) or Y (unpermute); the checks build verifies every dst row
 // against it.
+// guard (optional): the call's status word; the kernel does nothing when it holds
+// MOE_DEV_BAD_INDEX (the metadata of the call found an expert index out of range).
 cudaError_t launch_permute(const void* hidden, const int32_t* dst, int64_t Tc, int32_t H,
-                           int32_t k, void* X, int64_t rows_cap, cudaStream_t s);
+                           int32_t k, void* X, int64_t rows_cap, cudaStream_t s,
+                           const uint32_t* guard = nullptr);
 // ctas_per_sm: CTAs of the compile-time-k combine per SM (0: the build's default).  A combine
 // that runs beside a grouped GEMM takes fewer, so that every CTA of it is resident next to
 // the GEMM's one CTA per SM and all its tokens progress together.
 cudaError_t launch_unpermute(const void* Y, const int32_t* dst, const float* w, int64_t Tc,
                              int32_t H, int32_t k, void* out, int64_t rows_cap, cudaStream_t s,
-                             int ctas_per_sm = 0);
+                             int ctas_per_sm = 0, const uint32_t* guard = nullptr);
 // Range-violation flags of the checks build, one word per translation unit: read and clear.
 uint32_t checks_take_permute();
 uint32_t checks_take_gemm();
@@ -71,7 +74,9 @@ struct GemmArgs {
   int32_t K;              // H for gate/up, I for down
   int32_t out_cols;       // I for gate/up, H for down
   int32_t b_rows;         // 2I for gate/up, H for down
-  int64_t total_tiles;    // sum over experts of ceil(rows_e / 128) * n_tiles
+  int64_t total_tiles;    // sum over experts of ceil(rows_e / tile rows) * n_tiles; -1: the
+                          // kernel counts them from the offsets, one CTA (or pair) per SM,
+                          // and does nothing when *status holds MOE_DEV_BAD_INDEX
   uint32_t* status;
   // Gathered A (gate/up only): A row r is row gather[r] of gather_src [gather_src_rows][K]
   // instead of row r of A.  nullptr = plain A.

@@ -221,7 +221,7 @@ struct DeviceCtx {
   int num_sms = 0;
   cudaStream_t side = nullptr;
   cudaEvent_t ev_start = nullptr, ev_join = nullptr, ev_perm[2] = {}, ev_gemm[2] = {},
-              ev_unperm[2] = {};
+              ev_unperm[2] = {}, ev_packed = nullptr;
   // host-buffer forward: copy-in / copy-out streams and their events
   cudaStream_t copy_in = nullptr, copy_out = nullptr;
   cudaEvent_t ev_in[2] = {}, ev_in_free[2] = {}, ev_out[2] = {}, ev_out_free[2] = {},
@@ -256,7 +256,8 @@ moe_status_t get_ctx(DeviceCtx** out) {
         cudaEventCreateWithFlags(&c.ev_gemm[0], fl) != cudaSuccess ||
         cudaEventCreateWithFlags(&c.ev_gemm[1], fl) != cudaSuccess ||
         cudaEventCreateWithFlags(&c.ev_unperm[0], fl) != cudaSuccess ||
-        cudaEventCreateWithFlags(&c.ev_unperm[1], fl) != cudaSuccess)
+        cudaEventCreateWithFlags(&c.ev_unperm[1], fl) != cudaSuccess ||
+        cudaEventCreateWithFlags(&c.ev_packed, cudaEventDisableTiming) != cudaSuccess)
       return MOE_ERR_CUDA;
     if (cudaStreamCreateWithFlags(&c.copy_in, cudaStreamNonBlocking) != cudaSuccess ||
         cudaStreamCreateWithFlags(&c.copy_out, cudaStreamNonBlocking) != cudaSuccess)
@@ -318,6 +319,9 @@ struct Prof {
   bool origin_set = false;
   int64_t calls = 0;
   std::vector<moe_launch_record_t> timeline;
+  // GEMM launches enqueued before the host had the call's counts: (pending index, counts
+  // row) whose active-expert count is filled in once the counts arrive
+  std::vector<std::pair<size_t, int>> fix_active;
 } g_prof;
 
 cudaEvent_t prof_event() {
@@ -345,6 +349,7 @@ int prof_stream_id(cudaStream_t s) {
 struct ProfCall {
   ProfCall() {
     if (g_prof.on) ++g_prof.calls;
+    g_prof.fix_active.clear();  // left by a call that returned early
   }
 };
 
@@ -352,6 +357,7 @@ struct ProfScope {
   bool on;
   ProfRec r;
   cudaStream_t s;
+  int fix_row = -1;  // >= 0: r.active comes later from this row of the call's counts
   ProfScope(int kind, cudaStream_t st, int64_t rows, int64_t active, int kernels)
       : on(g_prof.on), s(st) {
     if (!on) return;
@@ -373,9 +379,21 @@ struct ProfScope {
   ~ProfScope() {
     if (!on) return;
     cudaEventRecord(r.b, s);
+    if (fix_row >= 0) g_prof.fix_active.push_back({g_prof.pending.size(), fix_row});
     g_prof.pending.push_back(r);
   }
 };
+
+// The active-expert counts of the launches enqueued before the counts reached the host.
+void prof_fix_active(const int32_t* counts, int32_t E) {
+  for (const auto& f : g_prof.fix_active) {
+    if (f.first >= g_prof.pending.size()) continue;
+    int64_t a = 0;
+    for (int32_t e = 0; e < E; ++e) a += counts[(size_t)f.second * E + e] > 0;
+    g_prof.pending[f.first].active = a;
+  }
+  g_prof.fix_active.clear();
+}
 
 moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
@@ -421,6 +439,27 @@ moe_status_t run_metadata(const Dims& d, const int32_t* idx, uint8_t* ws, const 
   return MOE_OK;
 }
 
+// The single device-to-host copy of {status, counts, splits} for every chunk, enqueued on s
+// without waiting for it (fetch_packed_wait does).
+moe_status_t fetch_packed_async(DeviceCtx* c, const uint8_t* ws, const Layout& L,
+                                cudaStream_t s) {
+  moe_status_t st = ensure_host_stage(c, L.packed_bytes);
+  if (st != MOE_OK) return st;
+  if (cudaMemcpyAsync(c->host_stage, ws + L.packed, L.packed_bytes, cudaMemcpyDeviceToHost, s) !=
+          cudaSuccess ||
+      cudaEventRecord(c->ev_packed, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status_t fetch_packed_wait(DeviceCtx* c) {
+  if (cudaEventSynchronize(c->ev_packed) != cudaSuccess) return MOE_ERR_CUDA;
+  const uint32_t status = static_cast<uint32_t>(c->host_stage[0]);
+  if (status & MOE_DEV_BAD_INDEX) return MOE_ERR_INDEX;
+  if (status & MOE_DEV_TIMEOUT) return MOE_ERR_TIMEOUT;
+  return MOE_OK;
+}
+
 // The single device-to-host copy of {status, counts, splits} for every chunk.
 moe_status_t fetch_packed(DeviceCtx* c, const uint8_t* ws, const Layout& L, cudaStream_t s) {
   moe_status_t st = ensure_host_stage(c, L.packed_bytes);
@@ -447,9 +486,11 @@ moe_status_t gemm_call(const void* A, int64_t rows, const void* B, void* out,
                        int32_t K, int32_t out_cols, int32_t b_rows, bool swiglu,
                        uint32_t* status, int num_sms, cudaStream_t s,
                        const int32_t* gather = nullptr, const void* gather_src = nullptr,
-                       int64_t gather_src_rows = 0) {
+                       int64_t gather_src_rows = 0, int fix_row = -1) {
+  // counts_host == nullptr: the host has not seen the counts yet; the kernel counts its tiles
+  // from the device offsets (and the profile's active-expert count waits for row fix_row)
   GemmArgs g;
-  const int64_t active = active_experts(counts_host, E);
+  const int64_t active = counts_host ? active_experts(counts_host, E) : 0;
   g.gather = gather;
   g.gather_src = gather_src;
   g.gather_src_rows = gather_src_rows;
@@ -462,11 +503,13 @@ moe_status_t gemm_call(const void* A, int64_t rows, const void* B, void* out,
   g.K = K;
   g.out_cols = out_cols;
   g.b_rows = b_rows;
-  g.total_tiles = gemm_total_tiles(counts_host, E, out_cols, swiglu, gather != nullptr);
+  g.total_tiles =
+      counts_host ? gemm_total_tiles(counts_host, E, out_cols, swiglu, gather != nullptr) : -1;
   g.status = status;
-  if (g.total_tiles == 0) return MOE_OK;
+  if (g.total_tiles == 0 || rows == 0) return MOE_OK;
   int detail = 0;
   ProfScope ps(swiglu ? MOE_KERNEL_GATEUP : MOE_KERNEL_DOWN, s, rows, active, 1);
+  if (!counts_host) ps.fix_row = fix_row;
   cudaError_t e = launch_grouped_gemm(g, swiglu, num_sms, s, &detail);
   if (e != cudaSuccess) return detail == 1 ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
   return MOE_OK;
@@ -648,14 +691,14 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
   uint32_t* dev_status = reinterpret_cast<uint32_t*>(ws + L.packed);
 
   // 1) metadata for all chunks (with pair sweeps: for all pairs, so that each expert's rows
-  // are contiguous over both chunks of a pair), 2) the one device-to-host copy (the only
-  // host stall)
+  // are contiguous over both chunks of a pair), 2) the one device-to-host copy, which the
+  // host waits for only after it has enqueued the whole pipeline: nothing below needs the
+  // counts on the host (each GEMM counts its tiles from the device offsets), and every
+  // kernel does nothing when the metadata flagged an expert index out of range, in which
+  // case the call returns MOE_ERR_INDEX as before
   const Dims dm = pair_gemms ? pair_dims(d) : d;
   if ((st = run_metadata(dm, top_k_index, ws, L, dst, src, sm)) != MOE_OK) return st;
-  if ((st = fetch_packed(ctx, ws, L, sm)) != MOE_OK) return st;
-  // Copy what the pipeline needs out of the shared staging block.
-  std::vector<int32_t> counts(ctx->host_stage + kStatusWords,
-                              ctx->host_stage + kStatusWords + (size_t)dm.n * d.E);
+  if ((st = fetch_packed_async(ctx, ws, L, sm)) != MOE_OK) return st;
   std::vector<int64_t> bounds = dims_bounds(d);
   int n_live = 0;  // chunks with tokens; only trailing chunks can be empty
   while (n_live < d.n && bounds[n_live + 1] > bounds[n_live]) ++n_live;
@@ -669,7 +712,7 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
   auto permute = [&](int c) -> moe_status_t {
     ProfScope ps(MOE_KERNEL_PERMUTE, sm, len(c) * k, 0, 1);
     if (launch_permute(hid + bounds[c] * H, dst + bounds[c] * k, len(c), H, k, xy(c), L.rows_cap,
-                       sm) != cudaSuccess)
+                       sm, dev_status) != cudaSuccess)
       return MOE_ERR_CUDA;
     if (cudaEventRecord(ctx->ev_perm[c & 1], sm) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
@@ -682,16 +725,15 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
       if (cudaStreamWaitEvent(sg, ctx->ev_unperm[c & 1], 0) != cudaSuccess) return MOE_ERR_CUDA;
     }
     const int64_t rows = len(c) * k;
-    const int32_t* cnt = counts.data() + (size_t)c * E;
     const int32_t* offs = reinterpret_cast<const int32_t*>(ws + L.offsets) + (size_t)c * (E + 1);
     moe_status_t s2 =
-        fused ? gemm_call(nullptr, rows, W_gate_up, act(c), offs, cnt, E, H, I, 2 * I, true,
-                          dev_status, ctx->num_sms, sg, src + bounds[c] * k, hidden, T)
-              : gemm_call(xy(c), rows, W_gate_up, act(c), offs, cnt, E, H, I, 2 * I, true,
-                          dev_status, ctx->num_sms, sg);
+        fused ? gemm_call(nullptr, rows, W_gate_up, act(c), offs, nullptr, E, H, I, 2 * I, true,
+                          dev_status, ctx->num_sms, sg, src + bounds[c] * k, hidden, T, c)
+              : gemm_call(xy(c), rows, W_gate_up, act(c), offs, nullptr, E, H, I, 2 * I, true,
+                          dev_status, ctx->num_sms, sg, nullptr, nullptr, 0, c);
     if (s2 != MOE_OK) return s2;
-    s2 = gemm_call(act(c), rows, W_down, xy(c), offs, cnt, E, I, H, H, false, dev_status,
-                   ctx->num_sms, sg);
+    s2 = gemm_call(act(c), rows, W_down, xy(c), offs, nullptr, E, I, H, H, false, dev_status,
+                   ctx->num_sms, sg, nullptr, nullptr, 0, c);
     if (s2 != MOE_OK) return s2;
     if (cudaEventRecord(ctx->ev_gemm[c & 1], sg) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
@@ -700,7 +742,7 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
     if (cudaStreamWaitEvent(sm, ctx->ev_gemm[c & 1], 0) != cudaSuccess) return MOE_ERR_CUDA;
     ProfScope ps(MOE_KERNEL_UNPERMUTE, sm, len(c) * k, 0, 1);
     if (launch_unpermute(xy(c), dst + bounds[c] * k, top_k_weights + bounds[c] * k, len(c), H, k,
-                         outp + bounds[c] * H, L.rows_cap, sm) != cudaSuccess)
+                         outp + bounds[c] * H, L.rows_cap, sm, 0, dev_status) != cudaSuccess)
       return MOE_ERR_CUDA;
     if (fused && cudaEventRecord(ctx->ev_unperm[c & 1], sm) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
@@ -735,15 +777,15 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
       const int c0 = 2 * m, c1 = 2 * m + 1 < n_live ? 2 * m + 1 : 2 * m;
       NvtxRange pr("moe_forward pair: chunks %d-%d", c0, c1);
       const int64_t rows = (pb[m + 1] - pb[m]) * k;
-      const int32_t* cnt = counts.data() + (size_t)m * E;
       const int32_t* offs = reinterpret_cast<const int32_t*>(ws + L.offsets) + (size_t)m * (E + 1);
-      moe_status_t s2 = gemm_call(nullptr, rows, W_gate_up, act_pair, offs, cnt, E, H, I, 2 * I,
-                                  true, dev_status, ctx->num_sms, sg, src + pb[m] * k, hidden, T);
+      moe_status_t s2 = gemm_call(nullptr, rows, W_gate_up, act_pair, offs, nullptr, E, H, I,
+                                  2 * I, true, dev_status, ctx->num_sms, sg, src + pb[m] * k,
+                                  hidden, T, m);
       if (s2 != MOE_OK) return s2;
       if (m > 0 && cudaStreamWaitEvent(sg, ctx->ev_unperm[0], 0) != cudaSuccess)
         return MOE_ERR_CUDA;
-      s2 = gemm_call(act_pair, rows, W_down, y_pair, offs, cnt, E, I, H, H, false, dev_status,
-                     ctx->num_sms, sg);
+      s2 = gemm_call(act_pair, rows, W_down, y_pair, offs, nullptr, E, I, H, H, false, dev_status,
+                     ctx->num_sms, sg, nullptr, nullptr, 0, m);
       if (s2 != MOE_OK) return s2;
       if (cudaEventRecord(ctx->ev_gemm[0], sg) != cudaSuccess ||
           cudaStreamWaitEvent(sm, ctx->ev_gemm[0], 0) != cudaSuccess)
@@ -757,7 +799,8 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
         ProfScope ps(MOE_KERNEL_UNPERMUTE, sm, tn * k, 0, 1);
         if (launch_unpermute(y_pair, dst + t0 * k, top_k_weights + t0 * k, tn, H, k,
                              outp + t0 * H, pair_cap, sm,
-                             beside_gemm ? MOE_UNPERM_BESIDE_GEMM_CTAS_PER_SM : 0) != cudaSuccess)
+                             beside_gemm ? MOE_UNPERM_BESIDE_GEMM_CTAS_PER_SM : 0,
+                             dev_status) != cudaSuccess)
           return MOE_ERR_CUDA;
       }
       if (cudaEventRecord(ctx->ev_unperm[0], sm) != cudaSuccess) return MOE_ERR_CUDA;
@@ -774,7 +817,10 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
   if (cudaEventRecord(ctx->ev_join, sg) != cudaSuccess ||
       cudaStreamWaitEvent(sm, ctx->ev_join, 0) != cudaSuccess)
     return MOE_ERR_CUDA;
-  return MOE_OK;
+  // the metadata's host copy (enqueued right after it, long done by now on the device)
+  st = fetch_packed_wait(ctx);
+  if (g_prof.on) prof_fix_active(ctx->host_stage + kStatusWords, E);
+  return st;
 }
 
 size_t moe_workspace_bytes_host(const moe_shape_t* s) {

@@ -29,6 +29,11 @@ __device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
 
 __device__ uint32_t g_range_flags;  // checks build: a row index outside its buffer was seen
 
+// The call's metadata found an expert index out of range: its rows are not to be used.
+__device__ __forceinline__ bool guarded_out(const uint32_t* guard) {
+  return guard && (*reinterpret_cast<const volatile uint32_t*>(guard) & MOE_DEV_BAD_INDEX);
+}
+
 // X[dst[t*k+j]] = hidden[t] for every j < k.  The warp loads the next U x 512 bytes of the
 // token row before it stores the k copies of the current ones, so the row's (usually cold)
 // reads stay in flight while the stores issue.
@@ -37,10 +42,11 @@ __global__ void __launch_bounds__(kRowThreads) permute_kernel(const uint4* __res
                                                               const int32_t* __restrict__ dst,
                                                               int64_t Tc, int32_t H8, int32_t k,
                                                               uint4* __restrict__ X,
-                                                              int64_t rows_cap) {
+                                                              int64_t rows_cap,
+                                                              const uint32_t* guard) {
   const int64_t t = (int64_t)blockIdx.x * kTokPerCta + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (t >= Tc) return;
+  if (t >= Tc || guarded_out(guard)) return;
   const int32_t d_lane = lane < k ? dst[t * k + lane] : 0;
   const uint4* src = hidden + t * H8;
   uint4 cur[U], nxt[U];
@@ -78,10 +84,11 @@ __global__ void __launch_bounds__(kRowThreads) unpermute_kernel(const uint4* __r
                                                                 const float* __restrict__ w,
                                                                 int64_t Tc, int32_t H8, int32_t k,
                                                                 uint4* __restrict__ out,
-                                                                int64_t rows_cap) {
+                                                                int64_t rows_cap,
+                                                                const uint32_t* guard) {
   const int64_t t = (int64_t)blockIdx.x * kTokPerCta + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (t >= Tc) return;
+  if (t >= Tc || guarded_out(guard)) return;
   const int32_t d_lane = lane < k ? dst[t * k + lane] : 0;
   const float w_lane = lane < k ? w[t * k + lane] : 0.f;
   for (int32_t v0 = 0; v0 < H8; v0 += 32 * U) {
@@ -139,9 +146,11 @@ __global__ void __launch_bounds__(kRowThreads, 4) unpermute_k_kernel(const uint4
                                                                      const float* __restrict__ w,
                                                                      int64_t Tc, int32_t H8,
                                                                      uint4* __restrict__ out,
-                                                                     int64_t rows_cap) {
+                                                                     int64_t rows_cap,
+                                                                     const uint32_t* guard) {
   constexpr int V = KT >= 8 ? 1 : 8 / KT;  // vectors per lane per pass
   const int lane = threadIdx.x & 31;
+  if (guarded_out(guard)) return;
   const int64_t n_warps = (int64_t)gridDim.x * kTokPerCta;
   for (int64_t t = (int64_t)blockIdx.x * kTokPerCta + (threadIdx.x >> 5); t < Tc; t += n_warps) {
     const int32_t d_lane = lane < KT ? dst[t * KT + lane] : 0;
@@ -211,41 +220,45 @@ int num_sms_cached() {
 template <int KT>
 cudaError_t launch_unpermute_k(const void* Y, const int32_t* dst, const float* w, int64_t Tc,
                                int32_t H, void* out, int64_t rows_cap, cudaStream_t s,
-                               int ctas_per_sm) {
+                               int ctas_per_sm, const uint32_t* guard) {
   const int64_t cap =
       (int64_t)num_sms_cached() * (ctas_per_sm > 0 ? ctas_per_sm : MOE_UNPERM_CTAS_PER_SM);
   const int64_t need = grid_for(Tc);
   unpermute_k_kernel<KT><<<(unsigned)(need < cap ? need : cap), kRowThreads, 0, s>>>(
-      static_cast<const uint4*>(Y), dst, w, Tc, H / 8, static_cast<uint4*>(out), rows_cap);
+      static_cast<const uint4*>(Y), dst, w, Tc, H / 8, static_cast<uint4*>(out), rows_cap,
+      guard);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_permute(const void* hidden, const int32_t* dst, int64_t Tc, int32_t H,
-                           int32_t k, void* X, int64_t rows_cap, cudaStream_t s) {
+                           int32_t k, void* X, int64_t rows_cap, cudaStream_t s,
+                           const uint32_t* guard) {
   if (Tc <= 0) return cudaSuccess;
   permute_kernel<4><<<grid_for(Tc), kRowThreads, 0, s>>>(
-      static_cast<const uint4*>(hidden), dst, Tc, H / 8, k, static_cast<uint4*>(X), rows_cap);
+      static_cast<const uint4*>(hidden), dst, Tc, H / 8, k, static_cast<uint4*>(X), rows_cap,
+      guard);
   return cudaGetLastError();
 }
 
 cudaError_t launch_unpermute(const void* Y, const int32_t* dst, const float* w, int64_t Tc,
                              int32_t H, int32_t k, void* out, int64_t rows_cap, cudaStream_t s,
-                             int ctas_per_sm) {
+                             int ctas_per_sm, const uint32_t* guard) {
   if (Tc <= 0) return cudaSuccess;
 #if MOE_UNPERM_CTAS_PER_SM > 0
   switch (k) {
-    case 1: return launch_unpermute_k<1>(Y, dst, w, Tc, H, out, rows_cap, s, ctas_per_sm);
-    case 2: return launch_unpermute_k<2>(Y, dst, w, Tc, H, out, rows_cap, s, ctas_per_sm);
-    case 4: return launch_unpermute_k<4>(Y, dst, w, Tc, H, out, rows_cap, s, ctas_per_sm);
-    case 6: return launch_unpermute_k<6>(Y, dst, w, Tc, H, out, rows_cap, s, ctas_per_sm);
-    case 8: return launch_unpermute_k<8>(Y, dst, w, Tc, H, out, rows_cap, s, ctas_per_sm);
+    case 1: return launch_unpermute_k<1>(Y, dst, w, Tc, H, out, rows_cap, s, ctas_per_sm, guard);
+    case 2: return launch_unpermute_k<2>(Y, dst, w, Tc, H, out, rows_cap, s, ctas_per_sm, guard);
+    case 4: return launch_unpermute_k<4>(Y, dst, w, Tc, H, out, rows_cap, s, ctas_per_sm, guard);
+    case 6: return launch_unpermute_k<6>(Y, dst, w, Tc, H, out, rows_cap, s, ctas_per_sm, guard);
+    case 8: return launch_unpermute_k<8>(Y, dst, w, Tc, H, out, rows_cap, s, ctas_per_sm, guard);
     default: break;
   }
 #endif
   unpermute_kernel<2><<<grid_for(Tc), kRowThreads, 0, s>>>(
-      static_cast<const uint4*>(Y), dst, w, Tc, H / 8, k, static_cast<uint4*>(out), rows_cap);
+      static_cast<const uint4*>(Y), dst, w, Tc, H / 8, k, static_cast<uint4*>(out), rows_cap,
+      guard);
   return cudaGetLastError();
 }
 

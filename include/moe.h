@@ -203,7 +203,7 @@ MOE_API moe_status_t moe_metadata_shape(const moe_shape_t* shape, const int32_t*
  * "一张专业时序图", "一组关键公式"):
  *     out[t] = bf16( sum_{j<k} top_k_weights[t][j] * FFN_{top_k_index[t][j]}(hidden[t]) )
  * with the j-sum in fp32 in ascending j.  Steps: metadata for all chunks + one
- * device-to-host copy (the only host stall); then per chunk c: permute, gate/up grouped
+ * device-to-host copy; then per chunk c: permute, gate/up grouped
  * GEMM with SwiGLU, down grouped GEMM, weighted unpermute.  Chunks run as a two-stream
  * pair pipeline on two workspace buffers: the permute of chunk c+1 and the unpermute of
  * chunk c-1 overlap the expert GEMMs of chunk c.  The result is bit-identical for every
@@ -211,14 +211,18 @@ MOE_API moe_status_t moe_metadata_shape(const moe_shape_t* shape, const int32_t*
  *
  * In (dev):  hidden [T][H] bf16, top_k_index [T][k] int32, top_k_weights [T][k] fp32,
  *            W_gate_up [E][2I][H] bf16, W_down [E][H][I] bf16
- * Out (dev): out [T][H] bf16, fully overwritten (unspecified after an error)
+ * Out (dev): out [T][H] bf16, fully overwritten (unspecified after an error; after
+ *            MOE_ERR_INDEX not written at all)
  * workspace: dev, >= moe_workspace_bytes(shape), 256-byte aligned; it must not
  *            overlap any input or output.
  * hidden, out, W_gate_up, W_down must be 16-byte aligned; top_k_index and
  * top_k_weights 4-byte aligned.
- * Synchrony: the host blocks once, on the metadata copy.  Everything after it is
- * enqueued on `stream` (and on the library's second stream, which is joined back into
- * `stream` before the call returns); the caller synchronizes `stream` to read `out`.
+ * Synchrony: the whole pipeline is enqueued on `stream` (and on the library's second
+ * stream, which is joined back into `stream` before the call returns) without waiting for
+ * the metadata: the GEMMs count their tiles from the device offsets, and every kernel after
+ * the metadata does nothing when it found an expert index out of range.  The host then
+ * blocks once, on the metadata copy (done early on the device), to return that status;
+ * the caller synchronizes `stream` to read `out`.
  * T == 0 returns MOE_OK and launches nothing.
  * Errors: as moe_metadata.  A kernel that gives up a bounded wait records it in the
  * workspace; moe_check_device_status reports it. */

@@ -22,6 +22,26 @@ def test_forward_bad_index_returns_status(moe):
     assert bool(torch.isfinite(out.float()).all())
 
 
+@pytest.mark.parametrize("dispatch,pair_gemms", [("fused", True), ("fused", False),
+                                                 ("separate", False)])
+@pytest.mark.parametrize("N", [1, 3, 4])
+def test_forward_bad_index_leaves_output_untouched(moe, dispatch, pair_gemms, N):
+    """The pipeline is enqueued before the host sees the metadata: every kernel after it
+    must do nothing when an index is out of range (no row of `out` written), and the call
+    still returns the index status."""
+    cfg = CONFIGS["tiny"]
+    gpu = {k: v.cuda() for k, v in layer_inputs(cfg).items()}
+    bad = gpu["idx"].clone()
+    bad[cfg.T - 1, 0] = -1
+    out = torch.full((cfg.T, cfg.H), 7.0, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(moe.MoEError) as ei:
+        moe.forward(gpu["hidden"], bad, gpu["w"], gpu["wgu"], gpu["wd"], num_chunks=N, out=out,
+                    dispatch=dispatch, pair_gemms=pair_gemms)
+    assert ei.value.status == 2
+    torch.cuda.synchronize()
+    assert bool((out == 7.0).all())
+
+
 def test_forward_workspace_too_small(moe):
     cfg = CONFIGS["tiny"]
     gpu = {k: v.cuda() for k, v in layer_inputs(cfg).items()}
