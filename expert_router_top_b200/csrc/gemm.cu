@@ -1060,8 +1060,6 @@ bool make_tma_3d_f32(CUtensorMap* m, void* base, int32_t E, int32_t M, int32_t N
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool gemm_supports_gather() { return true; }
-
 // Whether a GEMM kind runs on CTA pairs (MOE_GEMM_2SM bits).
 bool gemm_pair(bool swiglu, bool gather) {
   const int bit = !swiglu ? 1 : (gather ? 2 : 0);

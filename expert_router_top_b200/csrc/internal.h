@@ -90,8 +90,6 @@ struct GemmArgs {
 bool make_tma_2d_bf16(CUtensorMap* m, const void* base, int64_t rows, int32_t cols,
                       int32_t box_rows);
 
-// True when the build's grouped GEMM supports a gathered A operand.
-bool gemm_supports_gather();
 
 // 3-D fp32 tensor map over [E][M][N] (row-major per expert) with a 32 x 32 box and the
 // 128-byte swizzle: the target of the weight-gradient stores and add-reductions.

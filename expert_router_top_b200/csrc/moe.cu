@@ -638,7 +638,7 @@ moe_status_t moe_metadata_shape(const moe_shape_t* shape, const int32_t* top_k_i
 int32_t moe_forward_dispatch(const moe_shape_t* shape, uint32_t flags) {
   const uint32_t both = MOE_FWD_FUSED_DISPATCH | MOE_FWD_SEPARATE_DISPATCH;
   if ((flags & ~(both | MOE_FWD_PER_CHUNK_GEMMS)) || (flags & both) == both || !shape) return -1;
-  if (!gemm_supports_gather() || (flags & MOE_FWD_SEPARATE_DISPATCH)) return 0;
+  if (flags & MOE_FWD_SEPARATE_DISPATCH) return 0;
   if (flags & MOE_FWD_FUSED_DISPATCH) return 1;
   if (check_shape(shape) != MOE_OK) return 0;
   const Dims d = make_dims(shape->T, shape->k, shape->E, shape->ep_groups, shape->num_chunks,
@@ -911,8 +911,7 @@ moe_status_t moe_forward_host_impl(const moe_shape_t* shape, const void* hidden_
   // Fused dispatch (gate/up GEMM gathering its rows from the chunk's staged input) where one
   // chunk's permuted copy would be a sizeable share of the GEMM traffic, as moe_forward
   // decides for one chunk; the gather map then indexes the chunk's own rows.
-  const bool fused =
-      gemm_supports_gather() && 4 * d.t_chunk * d.k >= (int64_t)d.E * shape->I;
+  const bool fused = 4 * d.t_chunk * d.k >= (int64_t)d.E * shape->I;
   if ((st = run_metadata(d, idx_dev, ws, L, dst, src, sm, fused)) != MOE_OK) return st;
   if ((st = fetch_packed(ctx, ws, L, sm)) != MOE_OK) return st;
   std::vector<int32_t> counts(ctx->host_stage + kStatusWords,
