@@ -213,6 +213,13 @@ __device__ __forceinline__ void cp_async_16_hint(uint32_t smem_dst, const void* 
                : "memory");
 }
 
+// Arrive on `bar` once every cp.async this thread issued before it has landed (the pending
+// count is not raised first: the barrier's expected count includes this arrival).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }

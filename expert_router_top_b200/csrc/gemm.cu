@@ -78,6 +78,14 @@
 #ifndef MOE_GEMM_GATHER_DEPTH_2SM
 #define MOE_GEMM_GATHER_DEPTH_2SM 2  // CTA pair, gathered A: stages of copies run ahead
 #endif
+#ifndef MOE_GEMM_GATHER_ARRIVE
+// Single-CTA gathered A: 1 -- each gathering thread's copies of a stage arrive on its full
+// barrier by themselves when they land (cp.async.mbarrier.arrive), so a stage is reported
+// full as soon as its rows are in and the MMAs may run the whole ring ahead; 0 -- the
+// threads wait for their oldest stage while they run ahead and arrive once per warp, which
+// ties the MMAs of stage s to those of stage s - 2.
+#define MOE_GEMM_GATHER_ARRIVE 1
+#endif
 #ifndef MOE_GEMM_B_POLICY
 #define MOE_GEMM_B_POLICY 2  // L2 policy of weight loads: 0 normal, 1 evict_first, 2 evict_last
 #endif
@@ -306,6 +314,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   // Gathered A, one ring slot per gathering warp (the single-sub-tile ring of 4 slots)
   constexpr bool kWarpStages =
       kGather && !kTwoM && MOE_GEMM_GATHER_MODE == 1 && STAGES == kGatherThreads / 32;
+  // Gathered A arriving through the copies themselves (single CTA; a pair's full barrier
+  // belongs to the other CTA)
+  constexpr bool kCopyArrive = kGather && !kPair && !kWarpStages && MOE_GEMM_GATHER_ARRIVE != 0;
   static_assert(!kTwoM || kMaxHeld >= 0, "ring too shallow for the gathered two-sub-tile kernel");
   static_assert(!(kWarpStages && kPair), "one ring slot per gathering warp: single CTAs only");
   extern __shared__ uint8_t smem_raw[];
@@ -333,7 +344,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       // slot-owning gathering warp); CTA pair: both CTAs' gathering warps arrive on the
       // leader's barrier
       mbar_init(&ctl->full[s],
-                kGather ? 1 + (kWarpStages ? 1 : (kPair ? 2 : 1) * (kGatherThreads / 32)) : 1);
+                kGather ? 1 + (kWarpStages ? 1
+                               : kCopyArrive ? kGatherThreads
+                                             : (kPair ? 2 : 1) * (kGatherThreads / 32))
+                        : 1);
       mbar_init(&ctl->empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -625,13 +639,17 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
             }
           }
         }
-        cp_async_commit();
-        ++issued;
-        if (issued - arrived > kDepth) {
-          cp_async_wait<kDepth>();
-          fence_async_smem();
-          arrive_full(arrived % STAGES);
-          ++arrived;
+        if (kCopyArrive) {
+          cp_async_arrive_noinc(&ctl->full[stage]);
+        } else {
+          cp_async_commit();
+          ++issued;
+          if (issued - arrived > kDepth) {
+            cp_async_wait<kDepth>();
+            fence_async_smem();
+            arrive_full(arrived % STAGES);
+            ++arrived;
+          }
         }
         if (++stage == STAGES) {
           stage = 0;
@@ -641,7 +659,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
     }
     cp_async_wait<0>();
     fence_async_smem();
-    for (; arrived < issued; ++arrived) arrive_full(arrived % STAGES);
+    if (!kCopyArrive)
+      for (; arrived < issued; ++arrived) arrive_full(arrived % STAGES);
     (void)ok;
   } else if (warp == 0) {
     // ---------------- TMA producer (both CTAs) ----------------
@@ -739,6 +758,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
             ok = false;
             break;
           }
+          if (kCopyArrive) fence_async_smem();
           tc_fence_after();
           mma_sub(0, stage, kb);
           issued = true;
@@ -816,6 +836,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
             ok = false;
             break;
           }
+          // copies that arrived by themselves wrote through the generic proxy: make them
+          // visible to the MMAs' (async-proxy) reads
+          if (kCopyArrive) fence_async_smem();
           tc_fence_after();
           const uint32_t a_addr = smem_u32(sA + stage * G::kAStageBytes);
           const uint32_t b_addr = smem_u32(sB + stage * G::kBBytes);
