@@ -675,10 +675,12 @@ def run_ours(args, cfg):
 
     per_n, isolated, timelines = {}, None, None
     if not args.headline_only:
-        # ---- the same workload at N = 1, 2, 4 (the library's own dispatch choice each)
+        # ---- the same workload at N = 1, 2, 4 (the library's own dispatch choice each),
+        # each after the same spin-up as the headline, so that every region runs at the
+        # power-capped clock of sustained work (after a short one the clock is still high)
         for n in args.per_n:
             m = head if (n == chunks and args.dispatch == "auto" and not args.per_chunk_gemms) \
-                else run.measure(n, "auto", args.steps, args.warmup)
+                else run.measure(n, "auto", args.steps, args.warmup, spin_s=args.spinup_s)
             per_n[str(n)] = per_n_entry(moe, cfg, m, peaks)
         # ---- permute and unpermute alone: cold-cache launches of the kernels, and the
         # same kernels inside an exposed step (separate dispatch, one chunk)
