@@ -86,6 +86,11 @@
 // ties the MMAs of stage s to those of stage s - 2.
 #define MOE_GEMM_GATHER_ARRIVE 1
 #endif
+#ifndef MOE_GEMM_DOWN_LSU
+// 1: the down GEMM's A rows (Act, contiguous) are copied by the gathering warps with cp.async
+// (through the SM's load path) instead of TMA, beside the weights' TMA loads
+#define MOE_GEMM_DOWN_LSU 0
+#endif
 #ifndef MOE_GEMM_B_POLICY
 #define MOE_GEMM_B_POLICY 2  // L2 policy of weight loads: 0 normal, 1 evict_first, 2 evict_last
 #endif
@@ -150,7 +155,9 @@ struct KParams {
   int32_t b_rows;    // B rows per expert
   int32_t up_off;    // row offset of W_up inside one expert's W_gate_up (= I)
   int32_t total_tiles;  // -1: count them here from the offsets (skipped on a bad index)
-  const int32_t* gather;  // gathered A: token row of each permuted row (nullptr: plain A)
+  const int32_t* gather;  // gathered A: token row of each permuted row (nullptr: plain A,
+                          // or in the gathered kernel row r itself: A copied by the gathering
+                          // warps instead of TMA)
   const uint8_t* gsrc;    // gathered A: the token rows (hidden), and their stride in bytes
   int64_t gsrc_stride;
   int32_t K;              // valid K columns (gathered A: the rest of the last block reads 0)
@@ -507,7 +514,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       const int32_t row0 = off[t2.e] + t2.m * G::kTileM;
       const int32_t last = off[t2.e + 1] - 1;  // rows past the expert re-read its last row
 #pragma unroll
-      for (int q = 0; q < 4; ++q) tok[q] = gat[min(row0 + q * 32 + lane, last)];
+      for (int q = 0; q < 4; ++q) {
+        const int32_t r = min(row0 + q * 32 + lane, last);
+        tok[q] = gat ? gat[r] : r;
+      }
     };
     int32_t next_tok[4];
     if (stream_id < total) load_tokens(stream_id, next_tok);
@@ -586,8 +596,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
 #pragma unroll
       for (int h = 0; h < kSub; ++h)
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          tok[h * 8 + i] = gat[min(row0 + h * kRowsPerCta + gw * 32 + 4 * i + sub, last)];
+        for (int i = 0; i < 8; ++i) {
+          const int32_t r = min(row0 + h * kRowsPerCta + gw * 32 + 4 * i + sub, last);
+          tok[h * 8 + i] = gat ? gat[r] : r;
+        }
     };
     // the next tile's indices are loaded when a tile starts, so that their latency is
     // spent behind the tile's copies instead of at the next tile boundary
@@ -1096,6 +1108,8 @@ bool gemm_two_m(bool swiglu, bool gather) {
   return ((MOE_GEMM_TWO_M >> (swiglu ? 0 : 1)) & 1) != 0;
 }
 
+bool gemm_down_lsu() { return MOE_GEMM_DOWN_LSU != 0; }
+
 int64_t gemm_total_tiles(const int32_t* counts_host, int32_t E, int32_t out_cols, bool swiglu,
                          bool gather) {
   const int32_t bn = swiglu ? BN / 2 : BN;
@@ -1110,7 +1124,9 @@ int64_t gemm_total_tiles(const int32_t* counts_host, int32_t E, int32_t out_cols
 
 cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cudaStream_t s,
                                 int* err_detail) {
-  const bool gather = a.gather != nullptr;
+  // gathered-kernel launch: rows through a map (a.gather), or A's own rows copied by the
+  // gathering warps (a.gather_src set, a.gather null: the down GEMM's Act rows)
+  const bool gather = a.gather != nullptr || a.gather_src != nullptr;
   const bool kPair = gemm_pair(swiglu, gather);
   const bool two_m = gemm_two_m(swiglu, gather);
   *err_detail = 0;
@@ -1122,7 +1138,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
   }
   CUtensorMap mA, mB;
   const int32_t bn = swiglu ? BN / 2 : BN;
-  if (gather && !swiglu) {
+  if (gather && (a.gather_src_rows < a.rows && a.gather == nullptr)) {
     *err_detail = 1;
     return cudaErrorInvalidValue;
   }
@@ -1161,10 +1177,11 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
       two_m ? smem_bytes<false, true>() : (kPair ? smem_bytes<true>() : smem_bytes<false>());
   cudaError_t e;
   if (kPair) {
-    auto k = gather ? grouped_gemm_pair_kernel<true, true>
+    auto k = gather ? (swiglu ? grouped_gemm_pair_kernel<true, true>
+                              : grouped_gemm_pair_kernel<false, true>)
                     : (swiglu ? grouped_gemm_pair_kernel<true, false>
                               : grouped_gemm_pair_kernel<false, false>);
-    const int variant = gather ? 2 : (swiglu ? 1 : 0);
+    const int variant = (gather ? 2 : 0) + (swiglu ? 1 : 0);
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchAttribute attr[1];
@@ -1179,7 +1196,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     // persistent: as many CTA pairs as can be resident at once
-    static int max_pairs[3][64] = {};
+    static int max_pairs[4][64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     int& mp = max_pairs[variant][dev & 63];
@@ -1195,10 +1212,12 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, bool swiglu, int num_sms, cud
     e = cudaLaunchKernelEx(&cfg, k, mA, mB, mA64, mB64, p);
     if (e != cudaSuccess) return e;
   } else {
-    auto k = two_m ? (gather ? grouped_gemm_kernel<true, true, true>
+    auto k = two_m ? (gather ? (swiglu ? grouped_gemm_kernel<true, true, true>
+                                       : grouped_gemm_kernel<false, true, true>)
                              : (swiglu ? grouped_gemm_kernel<true, false, true>
                                        : grouped_gemm_kernel<false, false, true>))
-                   : (gather ? grouped_gemm_kernel<true, true, false>
+                   : (gather ? (swiglu ? grouped_gemm_kernel<true, true, false>
+                                       : grouped_gemm_kernel<false, true, false>)
                              : (swiglu ? grouped_gemm_kernel<true, false, false>
                                        : grouped_gemm_kernel<false, false, false>));
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

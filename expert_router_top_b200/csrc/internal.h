@@ -94,6 +94,8 @@ bool make_tma_2d_bf16(CUtensorMap* m, const void* base, int64_t rows, int32_t co
 // 3-D fp32 tensor map over [E][M][N] (row-major per expert) with a 32 x 32 box and the
 // 128-byte swizzle: the target of the weight-gradient stores and add-reductions.
 bool make_tma_3d_f32(CUtensorMap* m, void* base, int32_t E, int32_t M, int32_t N);
+// Whether the down GEMM copies its A rows with the gathering warps (build option).
+bool gemm_down_lsu();
 // Output tiles of a GEMM launch (tile height per the kernel variant that runs it).
 int64_t gemm_total_tiles(const int32_t* counts_host, int32_t E, int32_t out_cols, bool swiglu,
                          bool gather);

@@ -491,6 +491,10 @@ moe_status_t gemm_call(const void* A, int64_t rows, const void* B, void* out,
   // from the device offsets (and the profile's active-expert count waits for row fix_row)
   GemmArgs g;
   const int64_t active = counts_host ? active_experts(counts_host, E) : 0;
+  if (!swiglu && !gather_src && gemm_down_lsu()) {
+    gather_src = A;  // the A rows themselves, copied by the gathering warps
+    gather_src_rows = rows;
+  }
   g.gather = gather;
   g.gather_src = gather_src;
   g.gather_src_rows = gather_src_rows;
@@ -504,7 +508,8 @@ moe_status_t gemm_call(const void* A, int64_t rows, const void* B, void* out,
   g.out_cols = out_cols;
   g.b_rows = b_rows;
   g.total_tiles =
-      counts_host ? gemm_total_tiles(counts_host, E, out_cols, swiglu, gather != nullptr) : -1;
+      counts_host ? gemm_total_tiles(counts_host, E, out_cols, swiglu, gather_src != nullptr)
+                  : -1;
   g.status = status;
   if (g.total_tiles == 0 || rows == 0) return MOE_OK;
   int detail = 0;
