@@ -521,6 +521,23 @@ __global__ void pad_rows_kernel(const int32_t* idx, const int32_t* dst, const in
   dstp[s] = check_row(d, rows_cap, &g_range_flags) ? d : 0;
 }
 
+// Zero the pad rows of a padded row buffer: rows offp[e] + (off[e+1] - off[e]) .. offp[e+1]
+// of each expert e (fewer than kPadRows per expert), the only rows the permutes leave
+// unwritten that the GEMMs read.  One CTA per expert.
+__global__ void __launch_bounds__(256)
+    zero_pad_rows_kernel(const int32_t* __restrict__ off, const int32_t* __restrict__ offp,
+                         int32_t E, int32_t H8, uint4* __restrict__ buf, int64_t rows_cap) {
+  for (int32_t e = blockIdx.x; e < E; e += gridDim.x) {
+    const int64_t r0 = (int64_t)offp[e] + (off[e + 1] - off[e]);
+    const int64_t r1 = offp[e + 1];
+    const int64_t n = (r1 - r0) * H8;
+    for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
+      const int64_t r = r0 + i / H8;
+      if (check_row(r, rows_cap, &g_range_flags)) buf[r * H8 + i % H8] = make_uint4(0, 0, 0, 0);
+    }
+  }
+}
+
 // dY[dstp(t,j)] = bf16(w[t][j] * dout[t]) for every j < k: a weighted permute of dout that
 // needs nothing from the recomputed forward.  One warp per token.
 __global__ void __launch_bounds__(kRowThreads)
@@ -688,6 +705,13 @@ cudaError_t launch_pad_offsets(const int32_t* counts, int32_t E, int32_t n_chunk
                                int32_t* first, cudaStream_t s) {
   pad_offsets_kernel<<<n_chunks, 32, 0, s>>>(counts, E, offp);
   first_chunk_kernel<<<(E + 127) / 128, 128, 0, s>>>(counts, E, n_chunks, first);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_zero_pad_rows(const int32_t* off, const int32_t* offp, int32_t E, int32_t H,
+                                 void* buf, int64_t rows_cap, cudaStream_t s) {
+  zero_pad_rows_kernel<<<(unsigned)(E < 1024 ? E : 1024), 256, 0, s>>>(
+      off, offp, E, H / 8, static_cast<uint4*>(buf), rows_cap);
   return cudaGetLastError();
 }
 

@@ -137,6 +137,9 @@ int bwd_pad_rows();
 cudaError_t launch_bwd_gemm(const BwdGemmArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_pad_offsets(const int32_t* counts, int32_t E, int32_t n_chunks, int32_t* offp,
                                int32_t* first, cudaStream_t s);
+// Zero the pad rows (offp[e] + count_e .. offp[e+1]) of a padded bf16 [rows][H] buffer.
+cudaError_t launch_zero_pad_rows(const int32_t* off, const int32_t* offp, int32_t E, int32_t H,
+                                 void* buf, int64_t rows_cap, cudaStream_t s);
 cudaError_t launch_pad_rows(const int32_t* idx, const int32_t* dst, const int32_t* off,
                             const int32_t* offp, int64_t n, int32_t* dstp, int64_t rows_cap,
                             cudaStream_t s);

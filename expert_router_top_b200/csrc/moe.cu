@@ -1187,8 +1187,8 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
   // once W(m-2) is done with that buffer
   auto P = [&](int m) -> moe_status_t {
     if (m >= 2 && !ok(cudaStreamWaitEvent(s, ctx->ev_bw[m % 2], 0))) return MOE_ERR_CUDA;
-    ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(m) * k, 0, 2);
-    if (!ok(cudaMemsetAsync(x_of(m), 0, 2 * (size_t)R[m] * H, s)) ||
+    ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(m) * k, 0, 3);
+    if (!ok(launch_zero_pad_rows(off_m(m), offp_m(m), E, H, x_of(m), B.rows_cap, s)) ||
         !ok(launch_pad_rows(top_k_index + bounds[m] * k, dst + bounds[m] * k, off_m(m),
                             offp_m(m), len(m) * k, dstp_m(m), B.rows_cap, s)) ||
         !ok(launch_permute(hid + bounds[m] * H, dstp_m(m), len(m), H, k, x_of(m), B.rows_cap,
@@ -1235,8 +1235,8 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
   // nothing from the recompute, only the previous pair's weight gradients to be done with
   // the dY rows
   auto DYS = [&](int m) -> moe_status_t {
-    ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(m) * k, 0, 1);
-    if (!ok(cudaMemsetAsync(dy, 0, 2 * (size_t)R[m] * H, s)) ||
+    ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(m) * k, 0, 2);
+    if (!ok(launch_zero_pad_rows(off_m(m), offp_m(m), E, H, dy, B.rows_cap, s)) ||
         !ok(launch_dy_scatter(dout + bounds[m] * H, dstp_m(m), top_k_weights + bounds[m] * k,
                               len(m), H, k, dy, B.rows_cap, s)) ||
         !ok(cudaEventRecord(ctx->ev_bdy[0], s)))
