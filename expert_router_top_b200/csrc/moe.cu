@@ -646,12 +646,11 @@ int32_t moe_forward_dispatch(const moe_shape_t* shape, uint32_t flags) {
   if (flags & MOE_FWD_SEPARATE_DISPATCH) return 0;
   if (flags & MOE_FWD_FUSED_DISPATCH) return 1;
   if (check_shape(shape) != MOE_OK) return 0;
-  const Dims d = make_dims(shape->T, shape->k, shape->E, shape->ep_groups, shape->num_chunks,
-                           shape->chunk_size);
-  // two or more chunks: the pair sweeps halve the weight stream, which outweighs the cost
-  // of the row gathers; one chunk: gather only when the permuted copy is a sizeable share
-  if (d.n >= 2) return 1;
-  return 4 * d.t_chunk * d.k >= (int64_t)d.E * shape->I ? 1 : 0;
+  // the gathered rows (their copies arriving on the ring by themselves) cost the gate/up
+  // GEMM less than the permute kernel and its permuted copy cost the step, at every measured
+  // shape and chunk count; with two or more chunks the pair sweeps also halve the weight
+  // stream
+  return 1;
 }
 
 moe_status_t moe_forward(const moe_shape_t* shape, const void* hidden, const int32_t* top_k_index,

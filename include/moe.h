@@ -247,10 +247,8 @@ MOE_API moe_status_t moe_forward(const moe_shape_t* shape, const void* hidden, c
  * metadata then runs per pair, so each expert's rows are contiguous over both chunks and a
  * row tile may span them; the workspace is unchanged (the pair's two chunk buffers are
  * resident anyway and hold its rows as one buffer).  flags = 0 (what
- * moe_forward does) chooses fused whenever there are two or more chunks (the pair sweeps
- * halve the weight stream), and with one chunk when it holds at least I/4 rows per expert
- * on average (4 * T * k >= E * I: the permuted copy it saves is then a sizeable share of
- * the GEMMs' memory traffic, which the expert weights dominate otherwise).
+ * moe_forward does) chooses fused: it saves the permute kernel and the permuted copy, and
+ * with two or more chunks the pair sweeps halve the weight stream.
  * Every choice gives bit-identical outputs; arguments, workspace and errors are as
  * moe_forward (unknown flag bits, or both flags: MOE_ERR_ARG). */
 MOE_API moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,

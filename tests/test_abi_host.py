@@ -256,26 +256,22 @@ def test_profile_api_without_launches():
 
 def test_forward_dispatch_choice():
     """moe_forward_dispatch (host logic): flags force a dispatch; flags = 0 gathers in the
-    gate/up GEMM whenever there are two or more chunks (pair sweeps), and with one chunk
-    when it holds at least I/4 rows per expert (4 T k >= E I)."""
+    gate/up GEMM (fused) at every shape and chunk count."""
     import expert_router_top_b200 as moe
     q, m, d = CONFIGS["qwen3"], CONFIGS["mixtral"], CONFIGS["deepseek"]
     for N in (1, 2, 4, 8):
         assert moe.forward_dispatch(q.T, q.H, q.I, q.E, q.k, num_chunks=N) == "fused"
-    assert moe.forward_dispatch(m.T, m.H, m.I, m.E, m.k, num_chunks=1) == "separate"
-    assert moe.forward_dispatch(m.T, m.H, m.I, m.E, m.k, num_chunks=2) == "fused"
-    assert moe.forward_dispatch(d.T, d.H, d.I, d.E, d.k, ep_groups=d.G) == "separate"
-    assert moe.forward_dispatch(d.T, d.H, d.I, d.E, d.k, ep_groups=d.G, num_chunks=4) == "fused"
-    # the one-chunk boundary: 4 * 96 * 2 = 768 = 8 * 96
-    assert moe.forward_dispatch(96, 64, 96, 8, 2) == "fused"
-    assert moe.forward_dispatch(95, 64, 96, 8, 2) == "separate"
+        assert moe.forward_dispatch(m.T, m.H, m.I, m.E, m.k, num_chunks=N) == "fused"
+        assert moe.forward_dispatch(d.T, d.H, d.I, d.E, d.k, ep_groups=d.G, num_chunks=N) == "fused"
+    assert moe.forward_dispatch(95, 64, 96, 8, 2) == "fused"
     assert moe.forward_dispatch(q.T, q.H, q.I, q.E, q.k, "separate", num_chunks=4) == "separate"
+    assert moe.forward_dispatch(m.T, m.H, m.I, m.E, m.k, "separate") == "separate"
     assert moe.forward_dispatch(m.T, m.H, m.I, m.E, m.k, "fused") == "fused"
     L = moe.load()
     s = moe.shape(16, 64, 64, 4, 2, 1, 1, 0)
     assert L.moe_forward_dispatch(ctypes.byref(s), 3) == -1
     assert L.moe_forward_dispatch(ctypes.byref(s), 8) == -1
-    assert L.moe_forward_dispatch(ctypes.byref(s), 4) == 0  # a valid flag; auto: separate here
+    assert L.moe_forward_dispatch(ctypes.byref(s), 4) == 1  # a valid flag; auto: fused
 
 
 def test_selftest_argument_checks_run_on_host():
