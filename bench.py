@@ -780,9 +780,8 @@ def backward_units(cfg, counts):
     seen_before = np.cumsum(active, axis=0) - active  # earlier pairs with rows
     dw_bytes = 12.0 * H * I * (active.sum() + (active & (seen_before > 0)).sum())
     return {
-        "flops": {"bwd_gateup": 4 * rows * H * I, "down": 2 * rows * H * I,
-                  "bwd_dswiglu": 2 * rows * H * I, "bwd_dx": 4 * rows * H * I,
-                  "bwd_wgrad": 6 * rows * H * I},
+        "flops": {"bwd_gateup": 4 * rows * H * I, "bwd_dswiglu": 2 * rows * H * I,
+                  "bwd_dx": 4 * rows * H * I, "bwd_wgrad": 6 * rows * H * I},
         "wgrad_bytes": float((rows_c * (2 * H + 3 * I) * 2).sum()) + dw_bytes,
     }
 

@@ -6,10 +6,13 @@
 // paragraph on the timing diagram) and the expert computation may be recomputed to keep the
 // activation peak low (chunk_moe_recompute, sections 一组关键公式 and 操作指南).  For one
 // copy (t, j) routed to expert e, with x = hidden[t]:
-//   g = W_gate x, u = W_up x, h = silu(g) u, y = W_down h        (recomputed)
-//   d_w[t][j] = <dout[t], y>;  dY = w[t][j] dout[t];  dh = W_down^T dY
+//   g = W_gate x, u = W_up x, h = silu(g) u                      (recomputed)
+//   a = W_down^T dout[t];  d_w[t][j] = <dout[t], W_down h> = <a, h>;  dh = w[t][j] a
 //   du = dh silu(g);  dg = dh u silu'(g);  dX = W_gate^T dg + W_up^T du
-//   d_hidden[t] = sum_j dX;  dW_down[e] += dY h^T;  dW_gate|up[e] += dg|du x^T
+//   d_hidden[t] = sum_j dX;  dW_down[e] += dout[t] (w[t][j] h)^T;  dW_gate|up[e] += dg|du x^T
+// The output y = W_down h of the copy is never formed: its only use in the backward pass,
+// d_w, is the same inner product taken on the I side, where the SwiGLU-backward epilogue
+// already holds both a and h.
 //
 // Backward buffers hold each expert's rows of one unit padded to a multiple of 64 (zero
 // rows), so that the weight-gradient GEMMs reduce over an expert's rows in whole 64-row K
@@ -19,8 +22,9 @@
 // The GEMMs run on one tcgen05 kernel (one CTA per SM, TMA producer warp, one MMA thread,
 // four epilogue warps, 4-stage ring, double-buffered TMEM, as the forward kernel) in four
 // modes:
-//   kRawGU    [g u] = X W_gate_up^T           A rows K-major, B K-major   epilogue: g, u, h
-//   kDSwiGLU  dh = dY W_down                  B MN-major                  epilogue: dg, du
+//   kRawGU    [g u] = X W_gate_up^T           A rows K-major, B K-major   epilogue: g, u, w h
+//   kDSwiGLU  a = dY W_down (dY = dout rows)  B MN-major                  epilogue: dg, du,
+//                                                                         partial <a, h>
 //   kDPlain   dX = [dg du] W_gate_up          B MN-major                  epilogue: bf16 store
 //   kWGrad    dW[e] += S_A[e]^T S_B[e]        A and B MN-major, K = rows  epilogue: TMA fp32
 //             (K = the expert's padded rows of one pair of chunks)      store / add-reduce
@@ -70,8 +74,12 @@ struct BParams {
   int32_t total_tiles;
   __nv_bfloat16* out0;      // kRawGU: GU [rows][2I]; kDSwiGLU: [dg du] [rows][2I]
                             // (may be aux: each block is read before it is stored); kDPlain: [rows][N]
-  __nv_bfloat16* out1;      // kRawGU: Act [rows][I]
+  __nv_bfloat16* out1;      // kRawGU: Act = w h [rows][I]
   const __nv_bfloat16* aux; // kDSwiGLU: GU [rows][2I]
+  const float* wrow;        // kRawGU, kDSwiGLU: routing weight of each row [rows] (0 on pads)
+  float* dwp;               // kDSwiGLU: [rows][dw_slots] partial <a, h> of each (tile column,
+                            // epilogue warp column half), or nullptr
+  int32_t dw_slots;         // kDSwiGLU: 2 * n_tiles
   float* acc;               // kWGrad: [E][M][N] fp32 (written through tmC)
   const int32_t* first;     // kWGrad: [E] first unit (pair of chunks) with rows of each expert
   int32_t chunk;            // kWGrad: the unit of this launch (store where first == chunk)
@@ -353,6 +361,11 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
         }
       };
       if (kMode == kDSwiGLU) load_aux(part * kC, gq, uq);
+      // routing weight of this thread's row (0 for rows past the expert's)
+      float wr = 0.f;
+      if ((kMode == kRawGU || kMode == kDSwiGLU) && r < rows_here &&
+          check_row(row_g, p.rows, &g_range_flags))
+        wr = __ldg(p.wrow + row_g);
       if (!mbar_wait(&ctl->tfull[buf], (it >> 1) & 1, abort, p.status)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * BN;
@@ -413,13 +426,14 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
               const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
               pg[i] = pack_bf16x2(g0, g1);
               pu[i] = pack_bf16x2(u0, u1);
-              ph[i] = pack_bf16x2(silu_f(g0) * u0, silu_f(g1) * u1);
+              ph[i] = pack_bf16x2(wr * (silu_f(g0) * u0), wr * (silu_f(g1) * u1));
             }
             store_block_staged(pg, wbuf, lane, o0, row0w, 2 * p.I, col0, p.I, nrows, cap);
             store_block_staged(pu, wbuf, lane, o0 + p.I, row0w, 2 * p.I, col0, p.I, nrows, cap);
             store_block_staged(ph, wbuf, lane, o1, row0w, p.I, col0, p.I, nrows, cap);
           }
         } else {
+          float dwa = 0.f;  // kDSwiGLU: <a, h> over this warp's columns, in column order
 #pragma unroll 1
           for (int c = part * kC; c < (part + 1) * kC; ++c) {
             uint32_t v[32];
@@ -443,8 +457,10 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
                   for (int h = 0; h < 2; ++h) {
                     const float gv = h ? bf16hi(ga[i]) : bf16lo(ga[i]);
                     const float uv = h ? bf16hi(ua[i]) : bf16lo(ua[i]);
-                    const float dh = __uint_as_float(v[v4 * 8 + 2 * i + h]);
+                    const float a = __uint_as_float(v[v4 * 8 + 2 * i + h]);
                     const float sig = __fdividef(1.0f, 1.0f + __expf(-gv));
+                    dwa = fmaf(gv * sig * uv, a, dwa);
+                    const float dh = wr * a;
                     duv[h] = dh * gv * sig;
                     dgv[h] = dh * uv * (sig + gv * sig * (1.0f - sig));
                   }
@@ -468,6 +484,10 @@ __global__ void __launch_bounds__(Cfg<kMode>::kThreads, 1)
               store_block_staged(pk, wbuf, lane, o0, row0w, p.N, col0, p.N, nrows, cap);
             }
           }
+          // every slot of a row of the expert is written, 0 where its columns are past I
+          if (kMode == kDSwiGLU && p.dwp && r < rows_here &&
+              check_row(row_g, cap, &g_range_flags))
+            p.dwp[row_g * p.dw_slots + t.n * kParts + part] = dwa;
         }
       }
       tc_fence_before();
@@ -511,25 +531,33 @@ __global__ void first_chunk_kernel(const int32_t* counts, int32_t E, int32_t n_c
   first[e] = c;
 }
 
-// Padded row of each copy of one chunk: dstp = dst - off[e] + offp[e].
+// Padded row of each copy of one chunk, dstp = dst - off[e] + offp[e], and the copy's
+// routing weight at that row: wrow[dstp] = w.
 __global__ void pad_rows_kernel(const int32_t* idx, const int32_t* dst, const int32_t* off,
-                                const int32_t* offp, int64_t n, int32_t* dstp, int64_t rows_cap) {
+                                const int32_t* offp, const float* w, int64_t n, int32_t* dstp,
+                                float* wrow, int64_t rows_cap) {
   const int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (s >= n) return;
   const int32_t e = idx[s];
   const int32_t d = dst[s] - off[e] + offp[e];
-  dstp[s] = check_row(d, rows_cap, &g_range_flags) ? d : 0;
+  const bool in = check_row(d, rows_cap, &g_range_flags);
+  dstp[s] = in ? d : 0;
+  if (in) wrow[d] = w[s];
 }
 
 // Zero the pad rows of a padded row buffer: rows offp[e] + (off[e+1] - off[e]) .. offp[e+1]
 // of each expert e (fewer than kPadRows per expert), the only rows the permutes leave
-// unwritten that the GEMMs read.  One CTA per expert.
+// unwritten that the GEMMs read; and, where wrow is given, the routing weight of those rows.
+// One CTA per expert.
 __global__ void __launch_bounds__(256)
     zero_pad_rows_kernel(const int32_t* __restrict__ off, const int32_t* __restrict__ offp,
-                         int32_t E, int32_t H8, uint4* __restrict__ buf, int64_t rows_cap) {
+                         int32_t E, int32_t H8, uint4* __restrict__ buf, float* __restrict__ wrow,
+                         int64_t rows_cap) {
   for (int32_t e = blockIdx.x; e < E; e += gridDim.x) {
     const int64_t r0 = (int64_t)offp[e] + (off[e + 1] - off[e]);
     const int64_t r1 = offp[e + 1];
+    if (wrow && r0 + threadIdx.x < r1 && check_row(r0 + threadIdx.x, rows_cap, &g_range_flags))
+      wrow[r0 + threadIdx.x] = 0.f;  // fewer than kPadRows <= blockDim.x pad rows
     const int64_t n = (r1 - r0) * H8;
     for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
       const int64_t r = r0 + i / H8;
@@ -538,71 +566,17 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// dY[dstp(t,j)] = bf16(w[t][j] * dout[t]) for every j < k: a weighted permute of dout that
-// needs nothing from the recomputed forward.  One warp per token.
-__global__ void __launch_bounds__(kRowThreads)
-    dy_scatter_kernel(const uint4* __restrict__ dout, const int32_t* __restrict__ dstp,
-                      const float* __restrict__ w, int64_t Tc, int32_t H8, int32_t k,
-                      uint4* __restrict__ dY, int64_t rows_cap) {
-  const int64_t t = (int64_t)blockIdx.x * kTokPerCta + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (t >= Tc) return;
-  for (int j = 0; j < k; ++j) {
-    const int32_t d = dstp[t * k + j];
-    if (!check_row(d, rows_cap, &g_range_flags)) continue;  // d is the same in every lane
-    const float wj = w[t * k + j];
-    for (int32_t v = lane; v < H8; v += 32) {
-      const uint4 g = dout[t * H8 + v];
-      const uint32_t ga[4] = {g.x, g.y, g.z, g.w};
-      uint32_t o[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) o[i] = pack_bf16x2(wj * bf16lo(ga[i]), wj * bf16hi(ga[i]));
-      dY[(int64_t)d * H8 + v] = make_uint4(o[0], o[1], o[2], o[3]);
-    }
-  }
-}
-
-// d_w[t][j] = <dout[t], Y[dstp(t,j)]> in fp32 (lane-strided partial sums, then a warp tree
-// reduction in a fixed order): one warp per token.
-__global__ void __launch_bounds__(kRowThreads)
-    dw_dot_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ Y,
-                  const int32_t* __restrict__ dstp, int64_t Tc, int32_t H8, int32_t k,
-                  float* __restrict__ dw, int64_t rows_cap) {
-  const int64_t t = (int64_t)blockIdx.x * kTokPerCta + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (t >= Tc) return;
-  for (int j = 0; j < k; ++j) {
-    const int32_t d = dstp[t * k + j];
-    if (!check_row(d, rows_cap, &g_range_flags)) continue;
-    float dot = 0.f;
-    // 8 columns of 16 bytes per lane at a time: all 16 loads are issued before the FMAs,
-    // which then run in the same order as one column at a time (v ascending)
-    for (int32_t v0 = lane; v0 < H8; v0 += 32 * 8) {
-      uint4 g[8], y[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int32_t v = v0 + 32 * u;
-        if (v < H8) {
-          g[u] = __ldg(dout + t * H8 + v);
-          y[u] = __ldg(Y + (int64_t)d * H8 + v);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (v0 + 32 * u >= H8) break;
-        const uint32_t ga[4] = {g[u].x, g[u].y, g[u].z, g[u].w};
-        const uint32_t ya[4] = {y[u].x, y[u].y, y[u].z, y[u].w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          dot = fmaf(bf16lo(ga[i]), bf16lo(ya[i]), dot);
-          dot = fmaf(bf16hi(ga[i]), bf16hi(ya[i]), dot);
-        }
-      }
-    }
-#pragma unroll
-    for (int sh = 16; sh > 0; sh >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, sh);
-    if (lane == 0) dw[t * k + j] = dot;
-  }
+// d_w[t][j] = the sum, in slot order, of the dSwiGLU epilogue's partial inner products of
+// the copy's row.  One thread per copy.
+__global__ void dw_sum_kernel(const float* __restrict__ dwp, const int32_t* __restrict__ dstp,
+                              int64_t n, int32_t slots, float* __restrict__ dw, int64_t rows_cap) {
+  const int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (s >= n) return;
+  const int32_t d = dstp[s];
+  if (!check_row(d, rows_cap, &g_range_flags)) return;
+  float acc = 0.f;
+  for (int32_t i = 0; i < slots; ++i) acc += dwp[(int64_t)d * slots + i];
+  dw[s] = acc;
 }
 
 // d_hidden[t] = bf16( sum_{j<k} dX[dstp(t,j)] ), fp32 in ascending j.
@@ -648,6 +622,11 @@ inline unsigned row_grid(int64_t Tc) { return (unsigned)((Tc + kTokPerCta - 1) /
 
 int bwd_pad_rows() { return kPadRows; }
 
+int32_t bwd_dw_slots(int32_t I) {
+  static_assert(Cfg<kDSwiGLU>::kEpi / 4 == 2, "two epilogue warps per lane quarter");
+  return 2 * ((I + BN - 1) / BN);
+}
+
 cudaError_t launch_bwd_gemm(const BwdGemmArgs& a, int num_sms, cudaStream_t s) {
   if (a.E > kMaxE) return cudaErrorInvalidValue;
   // host tile count from the padded per-expert rows
@@ -688,6 +667,10 @@ cudaError_t launch_bwd_gemm(const BwdGemmArgs& a, int num_sms, cudaStream_t s) {
   p.out0 = static_cast<__nv_bfloat16*>(a.out0);
   p.out1 = static_cast<__nv_bfloat16*>(a.out1);
   p.aux = static_cast<const __nv_bfloat16*>(a.aux);
+  p.wrow = a.wrow;
+  p.dwp = a.dwp;
+  p.dw_slots = a.mode == kDSwiGLU ? 2 * n_tiles : 0;
+  if ((a.mode == kRawGU || a.mode == kDSwiGLU) && !a.wrow) return cudaErrorInvalidValue;
   p.acc = a.acc;
   p.first = a.first;
   p.chunk = a.chunk;
@@ -709,36 +692,26 @@ cudaError_t launch_pad_offsets(const int32_t* counts, int32_t E, int32_t n_chunk
 }
 
 cudaError_t launch_zero_pad_rows(const int32_t* off, const int32_t* offp, int32_t E, int32_t H,
-                                 void* buf, int64_t rows_cap, cudaStream_t s) {
+                                 void* buf, float* wrow, int64_t rows_cap, cudaStream_t s) {
+  static_assert(kPadRows <= 256, "one thread per pad row");
   zero_pad_rows_kernel<<<(unsigned)(E < 1024 ? E : 1024), 256, 0, s>>>(
-      off, offp, E, H / 8, static_cast<uint4*>(buf), rows_cap);
+      off, offp, E, H / 8, static_cast<uint4*>(buf), wrow, rows_cap);
   return cudaGetLastError();
 }
 
 cudaError_t launch_pad_rows(const int32_t* idx, const int32_t* dst, const int32_t* off,
-                            const int32_t* offp, int64_t n, int32_t* dstp, int64_t rows_cap,
-                            cudaStream_t s) {
+                            const int32_t* offp, const float* w, int64_t n, int32_t* dstp,
+                            float* wrow, int64_t rows_cap, cudaStream_t s) {
   if (n <= 0) return cudaSuccess;
-  pad_rows_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(idx, dst, off, offp, n, dstp,
-                                                               rows_cap);
+  pad_rows_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(idx, dst, off, offp, w, n, dstp,
+                                                               wrow, rows_cap);
   return cudaGetLastError();
 }
 
-cudaError_t launch_dy_scatter(const void* dout, const int32_t* dstp, const float* w, int64_t Tc,
-                              int32_t H, int32_t k, void* dY, int64_t rows_cap, cudaStream_t s) {
-  if (Tc <= 0) return cudaSuccess;
-  dy_scatter_kernel<<<row_grid(Tc), kRowThreads, 0, s>>>(static_cast<const uint4*>(dout), dstp, w,
-                                                         Tc, H / 8, k, static_cast<uint4*>(dY),
-                                                         rows_cap);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_dw_dot(const void* dout, const void* Y, const int32_t* dstp, int64_t Tc,
-                          int32_t H, int32_t k, float* dw, int64_t rows_cap, cudaStream_t s) {
-  if (Tc <= 0) return cudaSuccess;
-  dw_dot_kernel<<<row_grid(Tc), kRowThreads, 0, s>>>(static_cast<const uint4*>(dout),
-                                                     static_cast<const uint4*>(Y), dstp, Tc,
-                                                     H / 8, k, dw, rows_cap);
+cudaError_t launch_dw_sum(const float* dwp, const int32_t* dstp, int64_t n, int32_t slots,
+                          float* dw, int64_t rows_cap, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  dw_sum_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(dwp, dstp, n, slots, dw, rows_cap);
   return cudaGetLastError();
 }
 

@@ -126,6 +126,8 @@ struct BwdGemmArgs {
   void* out0;
   void* out1;
   const void* aux;
+  const float* wrow;           // kBwdRawGU, kBwdDSwiGLU: dev [A_rows] routing weight per row
+  float* dwp;                  // kBwdDSwiGLU: dev [A_rows][bwd_dw_slots(I)] partial d_w, or null
   float* acc;                  // kBwdWGrad: [E][M][N] fp32 gradient
   const int32_t* first;        // kBwdWGrad: dev [E] first unit (pair of chunks) with rows of
                                // each expert
@@ -134,21 +136,22 @@ struct BwdGemmArgs {
 };
 
 int bwd_pad_rows();
+// Partial inner products per row that the SwiGLU-backward GEMM writes for d_w.
+int32_t bwd_dw_slots(int32_t I);
 cudaError_t launch_bwd_gemm(const BwdGemmArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_pad_offsets(const int32_t* counts, int32_t E, int32_t n_chunks, int32_t* offp,
                                int32_t* first, cudaStream_t s);
-// Zero the pad rows (offp[e] + count_e .. offp[e+1]) of a padded bf16 [rows][H] buffer.
+// Zero the pad rows (offp[e] + count_e .. offp[e+1]) of a padded bf16 [rows][H] buffer and,
+// where wrow is not null, the same entries of the per-row routing weights.
 cudaError_t launch_zero_pad_rows(const int32_t* off, const int32_t* offp, int32_t E, int32_t H,
-                                 void* buf, int64_t rows_cap, cudaStream_t s);
+                                 void* buf, float* wrow, int64_t rows_cap, cudaStream_t s);
+// dstp = padded row of each of n copies; wrow[dstp] = w of the copy.
 cudaError_t launch_pad_rows(const int32_t* idx, const int32_t* dst, const int32_t* off,
-                            const int32_t* offp, int64_t n, int32_t* dstp, int64_t rows_cap,
-                            cudaStream_t s);
-// dY[dstp(t,j)] = bf16(w[t][j] dout[t]) (needs nothing from the forward), and
-// d_w[t][j] = <dout[t], Y[dstp(t,j)]> (needs the recomputed Y).
-cudaError_t launch_dy_scatter(const void* dout, const int32_t* dstp, const float* w, int64_t Tc,
-                              int32_t H, int32_t k, void* dY, int64_t rows_cap, cudaStream_t s);
-cudaError_t launch_dw_dot(const void* dout, const void* Y, const int32_t* dstp, int64_t Tc,
-                          int32_t H, int32_t k, float* dw, int64_t rows_cap, cudaStream_t s);
+                            const int32_t* offp, const float* w, int64_t n, int32_t* dstp,
+                            float* wrow, int64_t rows_cap, cudaStream_t s);
+// d_w of each of n copies = the sum of its row's slots partials (fixed order).
+cudaError_t launch_dw_sum(const float* dwp, const int32_t* dstp, int64_t n, int32_t slots,
+                          float* dw, int64_t rows_cap, cudaStream_t s);
 cudaError_t launch_sum_rows(const void* dX, const int32_t* dstp, int64_t Tc, int32_t H, int32_t k,
                             void* out, int64_t rows_cap, cudaStream_t s);
 

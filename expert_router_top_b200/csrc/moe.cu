@@ -1030,15 +1030,18 @@ struct BwdLayout {
   Layout meta;  // metadata regions (status/counts/splits, offsets, histograms, dst, src)
   size_t offp, first, dstp, total;
   int nx;  // X buffers: one per pair in flight (up to 2)
-  size_t xp[2], gu, act, ydx, dy;  // gu later holds [dg du] in place; ydx holds Y, then dX
+  size_t xp[2], wrow[2];  // X rows and their routing weights, per pair in flight
+  size_t gu, act, dx, dy;  // gu later holds [dg du] in place
+  size_t dwp;              // partial d_w of each row
+  int32_t dw_slots;
   int64_t rows_cap;
 };
 
 // The backward runs per pair of chunks: the metadata is taken per pair, so each expert's
 // rows are contiguous over both chunks and padded once per pair to a multiple of 64; every
-// pair's rows fit in rows_cap rows.  The pipeline keeps pair m's permuted rows in X buffer
-// m % 2 (the next pair is permuted while pair m computes; X is read until the pair's
-// weight-gradient GEMM) and its other rows in one buffer set.  The SwiGLU backward
+// pair's rows fit in rows_cap rows.  The pipeline keeps pair m's permuted rows and their
+// routing weights in buffer set m % 2 (the next pair is permuted while pair m computes; X is
+// read until the pair's weight-gradient GEMM) and its other rows in one buffer set.  The SwiGLU backward
 // overwrites the saved [g u] rows with [dg du] (each epilogue thread has read a block before
 // any lane stores it), so one buffer holds both.
 BwdLayout make_bwd_layout(const Dims& d, int32_t H, int32_t I) {
@@ -1059,15 +1062,20 @@ BwdLayout make_bwd_layout(const Dims& d, int32_t H, int32_t I) {
   for (int b = 0; b < B.nx; ++b) {
     B.xp[b] = o;
     o += al(2 * R * H);
+    B.wrow[b] = o;
+    o += al(sizeof(float) * R);
   }
   B.gu = o;
   o += al(2 * R * 2 * I);
   B.act = o;
   o += al(2 * R * I);
-  B.ydx = o;
+  B.dx = o;
   o += al(2 * R * H);
   B.dy = o;
   o += al(2 * R * H);
+  B.dw_slots = bwd_dw_slots(I);
+  B.dwp = o;
+  o += al(sizeof(float) * R * B.dw_slots);
   B.total = o;
   return B;
 }
@@ -1169,10 +1177,12 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
       R[m] += v;
     }
   auto x_of = [&](int m) { return ws + B.xp[m % B.nx]; };
+  auto wrow_of = [&](int m) { return reinterpret_cast<float*>(ws + B.wrow[m % B.nx]); };
   uint8_t* const gu = ws + B.gu;    // [g u], later [dg du]
-  uint8_t* const act = ws + B.act;  // h
-  uint8_t* const ydx = ws + B.ydx;  // Y, later dX
-  uint8_t* const dy = ws + B.dy;    // dY
+  uint8_t* const act = ws + B.act;  // w h
+  uint8_t* const dxr = ws + B.dx;   // dX
+  uint8_t* const dy = ws + B.dy;    // dY: the dout row of each copy
+  float* const dwp = reinterpret_cast<float*>(ws + B.dwp);
   auto off_m = [&](int m) {
     return reinterpret_cast<const int32_t*>(ws + B.meta.offsets) + (size_t)m * (E + 1);
   };
@@ -1182,14 +1192,16 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
   auto len = [&](int m) { return bounds[m + 1] - bounds[m]; };
   auto ok = [](cudaError_t e) { return e == cudaSuccess; };
 
-  // P(m), stream M: padded permute of the pair's rows into X buffer m % 2 (zero pad rows),
-  // once W(m-2) is done with that buffer
+  // P(m), stream M: padded permute of the pair's rows into X buffer m % 2 and their routing
+  // weights into the weight buffer m % 2 (zero pad rows), once W(m-2) is done with them
   auto P = [&](int m) -> moe_status_t {
     if (m >= 2 && !ok(cudaStreamWaitEvent(s, ctx->ev_bw[m % 2], 0))) return MOE_ERR_CUDA;
     ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(m) * k, 0, 3);
-    if (!ok(launch_zero_pad_rows(off_m(m), offp_m(m), E, H, x_of(m), B.rows_cap, s)) ||
+    if (!ok(launch_zero_pad_rows(off_m(m), offp_m(m), E, H, x_of(m), wrow_of(m), B.rows_cap,
+                                 s)) ||
         !ok(launch_pad_rows(top_k_index + bounds[m] * k, dst + bounds[m] * k, off_m(m),
-                            offp_m(m), len(m) * k, dstp_m(m), B.rows_cap, s)) ||
+                            offp_m(m), top_k_weights + bounds[m] * k, len(m) * k, dstp_m(m),
+                            wrow_of(m), B.rows_cap, s)) ||
         !ok(launch_permute(hid + bounds[m] * H, dstp_m(m), len(m), H, k, x_of(m), B.rows_cap,
                            s)) ||
         !ok(cudaEventRecord(ctx->ev_bp[m % 2], s)))
@@ -1215,63 +1227,62 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
     ProfScope ps(kind, sg, R[m], active_experts(rows_pad_m(m), E), 1);
     return launch_bwd_gemm(a, ctx->num_sms, sg);
   };
-  // F(m), stream G: recompute [g u], h and Y = h W_down^T on the padded rows, once P(m) is
-  // done and S(m-1) has read the previous pair's dX rows
+  // F(m), stream G: recompute [g u] and w h on the padded rows, once P(m) is done
   auto F = [&](int m) -> moe_status_t {
     if (!ok(cudaStreamWaitEvent(sg, ctx->ev_bp[m % 2], 0))) return MOE_ERR_CUDA;
-    if (m >= 1 && !ok(cudaStreamWaitEvent(sg, ctx->ev_bsum[0], 0))) return MOE_ERR_CUDA;
     BwdGemmArgs g = rowwise(m, kBwdRawGU);
     g.A = x_of(m), g.A_rows = R[m], g.A_cols = H;
     g.B = W_gate_up, g.B_rows = (int64_t)E * 2 * I, g.B_cols = H;
-    g.N = 2 * I, g.K = H, g.b_rows = 2 * I, g.out0 = gu, g.out1 = act;
-    if (!ok(launch_unit(MOE_KERNEL_BWD_GATEUP, g, m))) return MOE_ERR_CUDA;
-    moe_status_t s2 = gemm_call(act, R[m], W_down, ydx, offp_m(m), rows_pad_m(m), E, I, H, H,
-                                false, dev_status, ctx->num_sms, sg);
-    if (s2 != MOE_OK) return s2;
-    return ok(cudaEventRecord(ctx->ev_bf[0], sg)) ? MOE_OK : MOE_ERR_CUDA;
+    g.N = 2 * I, g.K = H, g.b_rows = 2 * I, g.out0 = gu, g.out1 = act, g.wrow = wrow_of(m);
+    return ok(launch_unit(MOE_KERNEL_BWD_GATEUP, g, m)) ? MOE_OK : MOE_ERR_CUDA;
   };
-  // DYS(m), stream M: dY = w dout into the pair's padded rows (zero pad rows); it needs
-  // nothing from the recompute, only the previous pair's weight gradients to be done with
-  // the dY rows
+  // DYS(m), stream M: the dout row of each copy into the pair's padded dY rows (zero pad
+  // rows); it needs nothing from the recompute, only the previous pair's weight gradients to
+  // be done with the dY rows
   auto DYS = [&](int m) -> moe_status_t {
     ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(m) * k, 0, 2);
-    if (!ok(launch_zero_pad_rows(off_m(m), offp_m(m), E, H, dy, B.rows_cap, s)) ||
-        !ok(launch_dy_scatter(dout + bounds[m] * H, dstp_m(m), top_k_weights + bounds[m] * k,
-                              len(m), H, k, dy, B.rows_cap, s)) ||
+    if (!ok(launch_zero_pad_rows(off_m(m), offp_m(m), E, H, dy, nullptr, B.rows_cap, s)) ||
+        !ok(launch_permute(dout + bounds[m] * H, dstp_m(m), len(m), H, k, dy, B.rows_cap, s)) ||
         !ok(cudaEventRecord(ctx->ev_bdy[0], s)))
       return MOE_ERR_CUDA;
     return MOE_OK;
   };
-  // DW(m), stream M: d_weights = <dout, Y> with the recomputed Y rows
+  // DW(m), stream M: d_weights = the sum of each copy's partials, once the SwiGLU-backward
+  // GEMM of the pair has written them
   auto DW = [&](int m) -> moe_status_t {
-    if (!ok(cudaStreamWaitEvent(s, ctx->ev_bf[0], 0))) return MOE_ERR_CUDA;
+    if (!ok(cudaStreamWaitEvent(s, ctx->ev_bdy[1], 0))) return MOE_ERR_CUDA;
     ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(m) * k, 0, 1);
-    if (!ok(launch_dw_dot(dout + bounds[m] * H, ydx, dstp_m(m), len(m), H, k,
-                          d_weights + bounds[m] * k, B.rows_cap, s)) ||
-        !ok(cudaEventRecord(ctx->ev_bdy[1], s)))
+    if (!ok(launch_dw_sum(dwp, dstp_m(m), len(m) * k, B.dw_slots, d_weights + bounds[m] * k,
+                          B.rows_cap, s)) ||
+        !ok(cudaEventRecord(ctx->ev_bf[0], s)))
       return MOE_ERR_CUDA;
     return MOE_OK;
   };
-  // Bd(m), stream G: dh with the SwiGLU backward, then dX
+  // Bd(m), stream G: the SwiGLU backward (dg, du and the partials of d_w), once the pair's dY
+  // rows are in and DW(m-1) has read the previous partials; then dX, once S(m-1) has read
+  // the previous pair's dX rows
   auto Bd = [&](int m) -> moe_status_t {
     if (!ok(cudaStreamWaitEvent(sg, ctx->ev_bdy[0], 0))) return MOE_ERR_CUDA;  // dY rows
+    if (m >= 1 && !ok(cudaStreamWaitEvent(sg, ctx->ev_bf[0], 0))) return MOE_ERR_CUDA;
     BwdGemmArgs g = rowwise(m, kBwdDSwiGLU);
     g.A = dy, g.A_rows = R[m], g.A_cols = H;
     g.B = W_down, g.B_rows = (int64_t)E * H, g.B_cols = I;
     g.N = I, g.K = H, g.b_rows = H, g.out0 = gu, g.aux = gu;  // in place
-    if (!ok(launch_unit(MOE_KERNEL_BWD_DSWIGLU, g, m))) return MOE_ERR_CUDA;
-    // dX overwrites the Y rows: d_weights must have read them
-    if (!ok(cudaStreamWaitEvent(sg, ctx->ev_bdy[1], 0))) return MOE_ERR_CUDA;
+    g.wrow = wrow_of(m), g.dwp = dwp;
+    if (!ok(launch_unit(MOE_KERNEL_BWD_DSWIGLU, g, m)) ||
+        !ok(cudaEventRecord(ctx->ev_bdy[1], sg)))
+      return MOE_ERR_CUDA;
+    if (m >= 1 && !ok(cudaStreamWaitEvent(sg, ctx->ev_bsum[0], 0))) return MOE_ERR_CUDA;
     g = rowwise(m, kBwdDPlain);
     g.A = gu, g.A_rows = R[m], g.A_cols = 2 * I;
     g.B = W_gate_up, g.B_rows = (int64_t)E * 2 * I, g.B_cols = H;
-    g.N = H, g.K = 2 * I, g.b_rows = 2 * I, g.out0 = ydx;
+    g.N = H, g.K = 2 * I, g.b_rows = 2 * I, g.out0 = dxr;
     if (!ok(launch_unit(MOE_KERNEL_BWD_DX, g, m)) || !ok(cudaEventRecord(ctx->ev_bdx[0], sg)))
       return MOE_ERR_CUDA;
     return MOE_OK;
   };
   // W(m), stream G: both weight gradients, K over the pair's padded rows:
-  //   dW_down[e] (+)= dY^T h ;  dW_gate_up[e] (+)= [dg du]^T X
+  //   dW_down[e] (+)= dY^T (w h) ;  dW_gate_up[e] (+)= [dg du]^T X
   // An expert's first pair with rows stores; later pairs add.
   auto W = [&](int m) -> moe_status_t {
     BwdGemmArgs g = rowwise(m, kBwdWGrad);
@@ -1291,7 +1302,7 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
   auto S = [&](int m) -> moe_status_t {
     if (!ok(cudaStreamWaitEvent(s, ctx->ev_bdx[0], 0))) return MOE_ERR_CUDA;
     ProfScope ps(MOE_KERNEL_BWD_ROWS, s, len(m) * k, 0, 1);
-    if (!ok(launch_sum_rows(ydx, dstp_m(m), len(m), H, k, dx_out + bounds[m] * H, B.rows_cap,
+    if (!ok(launch_sum_rows(dxr, dstp_m(m), len(m), H, k, dx_out + bounds[m] * H, B.rows_cap,
                             s)) ||
         !ok(cudaEventRecord(ctx->ev_bsum[0], s)))
       return MOE_ERR_CUDA;
@@ -1300,21 +1311,21 @@ moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
 
   // The mirrored pair pipeline, one unit per pair of chunks:
   //   G: F(0) DSwiGLU(0) DX(0) W(0) F(1) DSwiGLU(1) ...
-  //   M: P(0) DYS(0) | DW(0) P(1) S(0) DYS(1) | DW(1) P(2) S(1) ...
-  // dY needs nothing from the recompute, so it is scattered while F runs; d_weights reads
-  // the recomputed Y beside the SwiGLU-backward GEMM, before dX overwrites those rows; the
-  // next pair is permuted beside the dX and weight-gradient GEMMs, and its dY is scattered
-  // once W(m) is done with the dY rows.  Host enqueue order keeps each event wait on the
-  // record it is meant for.
+  //   M: P(0) DYS(0) | P(1) DW(0) S(0) DYS(1) | P(2) DW(1) S(1) ...
+  // dY needs nothing from the recompute, so it is scattered while F runs; the next pair is
+  // permuted beside the SwiGLU-backward GEMM, d_weights is summed beside the dX GEMM, and
+  // the next pair's dY is scattered once W(m) is done with the dY rows.  Host enqueue order
+  // keeps each event wait on the record it is meant for.
   if (!ok(cudaEventRecord(ctx->ev_start, s)) || !ok(cudaStreamWaitEvent(sg, ctx->ev_start, 0)))
     return MOE_ERR_CUDA;
   if (n_live > 0) {
     if ((st = P(0)) != MOE_OK || (st = F(0)) != MOE_OK || (st = DYS(0)) != MOE_OK) return st;
     for (int m = 0; m < n_live; ++m) {
       NvtxRange pr("moe_backward pair %d", m, 0);
-      if ((st = DW(m)) != MOE_OK) return st;
       if (m + 1 < n_live && (st = P(m + 1)) != MOE_OK) return st;
-      if ((st = Bd(m)) != MOE_OK || (st = S(m)) != MOE_OK || (st = W(m)) != MOE_OK) return st;
+      if ((st = Bd(m)) != MOE_OK || (st = DW(m)) != MOE_OK || (st = S(m)) != MOE_OK ||
+          (st = W(m)) != MOE_OK)
+        return st;
       if (m + 1 < n_live) {
         if ((st = F(m + 1)) != MOE_OK) return st;
         if (!ok(cudaStreamWaitEvent(s, ctx->ev_bf[1], 0))) return MOE_ERR_CUDA;  // W(m) done

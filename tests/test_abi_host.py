@@ -115,13 +115,16 @@ def test_workspace_follows_pair_double_buffer(name):
 def _bwd_row_buffer_bytes(cfg, N):
     """Backward rows by construction: the units are the pairs of chunks, ceil(N/2) of them,
     each of at most 2*ceil(T/N) tokens, whose rows padded per expert to 64 fit in
-    tokens*k + 63*E rows; the permuted rows X (H wide) in min(units, 2) unit buffers, and
-    one unit set of [g u] (2I), h (I), Y/dX (H) and dY (H), all bf16."""
+    tokens*k + 63*E rows; the permuted rows X (H wide, bf16) and their routing weights (fp32)
+    in min(units, 2) unit buffers, and one unit set of [g u] (2I), w h (I), dX (H) and dY (H),
+    all bf16, with two fp32 partials of d_w per 256 columns of I."""
     n = max(N, 1)
     tu = min(2 * -(-cfg.T // n), cfg.T)
     units = -(-n // 2)
     rows = tu * cfg.k + 63 * cfg.E
-    return (min(units, 2) * cfg.H + 3 * cfg.I + 2 * cfg.H) * rows * 2, units, tu
+    per_row = (min(units, 2) * (2 * cfg.H + 4) + 2 * (3 * cfg.I + 2 * cfg.H)
+               + 4 * 2 * -(-cfg.I // 256))
+    return per_row * rows, units, tu
 
 
 @pytest.mark.parametrize("name", ["mixtral", "qwen3", "deepseek", "tiny", "edge", "edge_varlen"])
