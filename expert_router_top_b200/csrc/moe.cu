@@ -695,14 +695,18 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
   uint32_t* dev_status = reinterpret_cast<uint32_t*>(ws + L.packed);
 
   // 1) metadata for all chunks (with pair sweeps: for all pairs, so that each expert's rows
-  // are contiguous over both chunks of a pair), 2) the one device-to-host copy, which the
-  // host waits for only after it has enqueued the whole pipeline: nothing below needs the
-  // counts on the host (each GEMM counts its tiles from the device offsets), and every
-  // kernel does nothing when the metadata flagged an expert index out of range, in which
-  // case the call returns MOE_ERR_INDEX as before
+  // are contiguous over both chunks of a pair), 2) the one device-to-host copy, on the side
+  // stream so that the next launch on this stream need not wait for it, and which the host
+  // waits for only after it has enqueued the whole pipeline: nothing below needs the counts
+  // on the host (each GEMM counts its tiles from the device offsets), and every kernel does
+  // nothing when the metadata flagged an expert index out of range, in which case the call
+  // returns MOE_ERR_INDEX as before
   const Dims dm = pair_gemms ? pair_dims(d) : d;
   if ((st = run_metadata(dm, top_k_index, ws, L, dst, src, sm)) != MOE_OK) return st;
-  if ((st = fetch_packed_async(ctx, ws, L, sm)) != MOE_OK) return st;
+  if (cudaEventRecord(ctx->ev_start, sm) != cudaSuccess ||
+      cudaStreamWaitEvent(sg, ctx->ev_start, 0) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if ((st = fetch_packed_async(ctx, ws, L, sg)) != MOE_OK) return st;
   std::vector<int64_t> bounds = dims_bounds(d);
   int n_live = 0;  // chunks with tokens; only trailing chunks can be empty
   while (n_live < d.n && bounds[n_live + 1] > bounds[n_live]) ++n_live;
@@ -753,9 +757,6 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
   };
 
   // 3) the pair pipeline
-  if (cudaEventRecord(ctx->ev_start, sm) != cudaSuccess ||
-      cudaStreamWaitEvent(sg, ctx->ev_start, 0) != cudaSuccess)
-    return MOE_ERR_CUDA;
   if (n_live > 0 && !fused) {
     // M: P(0) P(1) U(0) P(2) U(1) ...; G: E(0) E(1) E(2) ...
     if ((st = permute(0)) != MOE_OK || (st = experts(0)) != MOE_OK) return st;
@@ -766,13 +767,15 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
       if ((st = unpermute(c)) != MOE_OK) return st;
     }
   } else if (n_live > 0 && pair_gemms) {
-    // Pairs (c0, c1) = (2m, 2m+1).  G: GU(m) D(m) GU(m+1) D(m+1) ..., where GU / D are the
-    // gate/up and down GEMMs of the pair in one tile sweep over its rows, laid out per expert
-    // across both chunks (each expert's weight tiles are fetched once for the pair, and a row
-    // tile may hold rows of both chunks); D(m+1) waits until U(m), the combine of both
-    // chunks in one launch, has read the pair's Y rows.  M: U(m) after D(m), beside GU(m+1).
-    // The pair's rows fill both
-    // halves of the X|Y and Act double buffers; dst holds pair-local rows.
+    // Pairs (c0, c1) = (2m, 2m+1).  M: GU(m) D(m) GU(m+1) D(m+1) ... U(last), where GU / D
+    // are the gate/up and down GEMMs of the pair in one tile sweep over its rows, laid out
+    // per expert across both chunks (each expert's weight tiles are fetched once for the
+    // pair, and a row tile may hold rows of both chunks), and U the combine of both chunks
+    // of a pair in one launch; G: U(m) after D(m), beside GU(m+1), for every pair but the
+    // last.  D(m+1) waits until U(m) has read the pair's Y rows.  The GEMMs and the last
+    // combine follow the metadata on the caller's stream, so that no launch on the critical
+    // path waits for another stream.  The pair's rows fill both halves of the X|Y and Act
+    // double buffers; dst holds pair-local rows.
     const std::vector<int64_t> pb = dims_bounds(dm);
     void* y_pair = ws + L.xy[0];
     void* act_pair = ws + L.act[0];
@@ -783,31 +786,33 @@ moe_status_t moe_forward_ex(const moe_shape_t* shape, const void* hidden,
       const int64_t rows = (pb[m + 1] - pb[m]) * k;
       const int32_t* offs = reinterpret_cast<const int32_t*>(ws + L.offsets) + (size_t)m * (E + 1);
       moe_status_t s2 = gemm_call(nullptr, rows, W_gate_up, act_pair, offs, nullptr, E, H, I,
-                                  2 * I, true, dev_status, ctx->num_sms, sg, src + pb[m] * k,
+                                  2 * I, true, dev_status, ctx->num_sms, sm, src + pb[m] * k,
                                   hidden, T, m);
       if (s2 != MOE_OK) return s2;
-      if (m > 0 && cudaStreamWaitEvent(sg, ctx->ev_unperm[0], 0) != cudaSuccess)
+      if (m > 0 && cudaStreamWaitEvent(sm, ctx->ev_unperm[0], 0) != cudaSuccess)
         return MOE_ERR_CUDA;
       s2 = gemm_call(act_pair, rows, W_down, y_pair, offs, nullptr, E, I, H, H, false, dev_status,
-                     ctx->num_sms, sg, nullptr, nullptr, 0, m);
+                     ctx->num_sms, sm, nullptr, nullptr, 0, m);
       if (s2 != MOE_OK) return s2;
-      if (cudaEventRecord(ctx->ev_gemm[0], sg) != cudaSuccess ||
-          cudaStreamWaitEvent(sm, ctx->ev_gemm[0], 0) != cudaSuccess)
-        return MOE_ERR_CUDA;
-      // a pair's combines run beside the next pair's gate/up GEMM (fewer CTAs, all resident
-      // next to it) unless this is the last pair
+      // a pair's combine runs on the side stream beside the next pair's gate/up GEMM (fewer
+      // CTAs, all resident next to it) unless this is the last pair
       // (one launch for both chunks: their tokens are adjacent and dst holds pair-local rows)
       const bool beside_gemm = 2 * (m + 1) < n_live;
+      cudaStream_t su = beside_gemm ? sg : sm;
+      if (beside_gemm && (cudaEventRecord(ctx->ev_gemm[0], sm) != cudaSuccess ||
+                          cudaStreamWaitEvent(sg, ctx->ev_gemm[0], 0) != cudaSuccess))
+        return MOE_ERR_CUDA;
       {
         const int64_t t0 = bounds[c0], tn = bounds[c1 + 1] - bounds[c0];
-        ProfScope ps(MOE_KERNEL_UNPERMUTE, sm, tn * k, 0, 1);
+        ProfScope ps(MOE_KERNEL_UNPERMUTE, su, tn * k, 0, 1);
         if (launch_unpermute(y_pair, dst + t0 * k, top_k_weights + t0 * k, tn, H, k,
-                             outp + t0 * H, pair_cap, sm,
+                             outp + t0 * H, pair_cap, su,
                              beside_gemm ? MOE_UNPERM_BESIDE_GEMM_CTAS_PER_SM : 0,
                              dev_status) != cudaSuccess)
           return MOE_ERR_CUDA;
       }
-      if (cudaEventRecord(ctx->ev_unperm[0], sm) != cudaSuccess) return MOE_ERR_CUDA;
+      if (beside_gemm && cudaEventRecord(ctx->ev_unperm[0], sg) != cudaSuccess)
+        return MOE_ERR_CUDA;
     }
   } else if (n_live > 0) {
     // G: E(0) E(1) E(2) ... (E(c+2) after U(c) freed buffer c % 2); M: U(0) U(1) ...
