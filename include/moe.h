@@ -299,8 +299,9 @@ MOE_API size_t moe_backward_workspace_bytes(const moe_shape_t* shape);
  *   dW_gate_up [E][2I][H] fp32    gradient of W_gate_up (gate rows, then up rows)
  *   dW_down [E][H][I] fp32        gradient of W_down
  * All four outputs are overwritten.  Inputs as moe_forward plus d_out [T][H] bf16.  The
- * intermediate g, u, h, Y, dY, dg, du and dX rows are bf16 (fp32 accumulation in every GEMM
- * and reduction).  Chunks run as the mirrored pair pipeline on the caller's stream and the
+ * intermediate g, u, w h, dY (the d_out row of each copy), dg, du and dX rows are bf16 (fp32
+ * accumulation in every GEMM and reduction); d_weights is taken on the I side as
+ * <W_down^T d_out[t], h(t,j)> in fp32, so the copies' outputs y are never formed.  Chunks run as the mirrored pair pipeline on the caller's stream and the
  * library's second stream, one unit per pair of chunks (2m, 2m+1): the routing metadata is
  * taken per pair, so each expert's rows are contiguous over both chunks (padded to a
  * multiple of 64 inside the workspace), every GEMM is one tile sweep over the pair's rows,
@@ -308,8 +309,9 @@ MOE_API size_t moe_backward_workspace_bytes(const moe_shape_t* shape);
  * rows stores, later pairs add through TMA reductions).  d_hidden and d_weights are
  * bit-identical for every chunking; dW_* are equal up to the fp32 summation order.
  * workspace: dev, >= moe_backward_workspace_bytes(shape): the metadata plus two pair
- * buffers of permuted rows (the next pair is permuted while one computes) and one pair set
- * of the other row buffers (dg | du overwrite the recomputed g | u rows in place).  The
+ * buffers of permuted rows and their routing weights (the next pair is permuted while one
+ * computes) and one pair set of the other row buffers (dg | du overwrite the recomputed
+ * g | u rows in place) and of the fp32 partials of d_weights.  The
  * host blocks once, on the metadata copy.
  * Errors: as moe_forward; MOE_ERR_ARG also for H % 64 or I % 32 != 0. */
 MOE_API moe_status_t moe_backward(const moe_shape_t* shape, const void* hidden,
@@ -473,12 +475,13 @@ typedef enum {
   MOE_KERNEL_GATEUP = 2,
   MOE_KERNEL_DOWN = 3,
   MOE_KERNEL_UNPERMUTE = 4,
-  /* moe_backward (its recomputed down GEMM counts as MOE_KERNEL_DOWN) */
-  MOE_KERNEL_BWD_GATEUP = 5,   /* recomputed [g u] = X W_gate_up^T with h = silu(g) u      */
-  MOE_KERNEL_BWD_DSWIGLU = 6,  /* dh = dY W_down with the SwiGLU backward -> [dg du]        */
+  /* moe_backward */
+  MOE_KERNEL_BWD_GATEUP = 5,   /* recomputed [g u] = X W_gate_up^T with w h = w silu(g) u   */
+  MOE_KERNEL_BWD_DSWIGLU = 6,  /* a = dY W_down (dY = d_out rows): SwiGLU backward -> [dg du]
+                                  with dh = w a, and the partials of d_w = <a, h>           */
   MOE_KERNEL_BWD_DX = 7,       /* dX = [dg du] W_gate_up                                    */
-  MOE_KERNEL_BWD_WGRAD = 8,    /* dW_down += dY^T h and dW_gate_up += [dg du]^T X           */
-  MOE_KERNEL_BWD_ROWS = 9,     /* row kernels: padded permute, dY and d_weights, d_hidden   */
+  MOE_KERNEL_BWD_WGRAD = 8,    /* dW_down += dY^T (w h) and dW_gate_up += [dg du]^T X       */
+  MOE_KERNEL_BWD_ROWS = 9,     /* row kernels: padded permute, dY, d_weights sums, d_hidden */
   MOE_KERNEL_KINDS = 10
 } moe_kernel_kind_t;
 
