@@ -26,7 +26,8 @@ struct MetaArgs {
   int32_t* counts;          // [n_chunks][E]
   int32_t* offsets;         // [n_chunks][E+1]
   int32_t* splits;          // [n_chunks][G]
-  uint32_t* status;         // device status word
+  uint32_t* status;         // device status words: cleared by the kernel, then [0] flags
+  int32_t status_words = 1; // words at status to clear
 };
 
 inline int32_t meta_tile_tokens(int32_t k) {

@@ -8,7 +8,9 @@
 // the flat copy index t*k+j ascending, which makes the permutation deterministic and
 // independent of the number of chunks.
 //
-// Three small kernels, no atomics on the data path (only on the error flag):
+// One cooperative kernel in three phases separated by grid-wide barriers (its CTAs loop over
+// the tiles, so that every CTA of the grid is resident), no atomics on the data path (only
+// on the error flag):
 //   rank:     per tile of copies, a stable in-tile rank of every copy within its expert
 //             (warp match + per-warp histograms) and the tile's expert histogram;
 //   count:    per (chunk, expert), an exclusive scan of the tile histograms over the
@@ -16,6 +18,10 @@
 //   finalize: per tile, the chunk's expert offsets (scan of counts), the final row
 //             dst = offset[e] + tile base[e] + in-tile rank, the inverse map src_tok, and
 //             (first tile of each chunk) the offsets and group splits.
+// The status words are cleared by the kernel itself, before the first barrier; a bad index
+// seen in the rank phase is recorded after the last one.
+#include <cooperative_groups.h>
+
 #include "device.cuh"
 #include "internal.h"
 
@@ -49,13 +55,13 @@ __device__ __forceinline__ int32_t warp_segment(int32_t slots) {
   return ((slots + kWarps * 32 - 1) / (kWarps * 32)) * 32;
 }
 
-__global__ void __launch_bounds__(kMetaThreads) meta_rank_kernel(MetaArgs a) {
-  extern __shared__ int32_t sm[];
+// Returns whether the tile holds an expert index outside [0, E).
+__device__ bool meta_rank_tile(const MetaArgs& a, int32_t tile, int32_t* sm) {
   int32_t* whist = sm;                       // [kWarps][E]
-  int32_t* lrank = sm + kWarps * a.E;        // [kMetaSlotsPerTile]
-  const int32_t tile = blockIdx.x;
+  int32_t* lrank = sm + kWarps * a.E;        // [kMetaSlotsPerTile]: e << 16 | rank, or -1
   const TileSpan ts = tile_span(a, tile);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  bool bad = false;
   for (int i = threadIdx.x; i < kWarps * a.E; i += kMetaThreads) whist[i] = 0;
   __syncthreads();
 
@@ -64,21 +70,30 @@ __global__ void __launch_bounds__(kMetaThreads) meta_rank_kernel(MetaArgs a) {
   int32_t* my_hist = whist + warp * a.E;
   const int32_t s_begin = warp * seg;
   const int32_t s_end = min(ts.slots, s_begin + seg);
-  for (int32_t base = s_begin; base < s_end; base += 32) {
-    const int32_t s = base + lane;
-    int32_t e = -1;
-    if (s < s_end) {
-      e = idx[s];
-      if (e < 0 || e >= a.E) {
-        atomicOr(a.status, MOE_DEV_BAD_INDEX);
-        e = -1;
-      }
+  // the warp's expert indices, all loads issued before the first use (seg <= 32 * kIt)
+  constexpr int kIt = kMetaSlotsPerTile / kMetaThreads;
+  static_assert(kMetaSlotsPerTile % kMetaThreads == 0, "whole segments");
+  int32_t ev[kIt];
+#pragma unroll
+  for (int u = 0; u < kIt; ++u) {
+    const int32_t s = s_begin + u * 32 + lane;
+    ev[u] = s < s_end ? idx[s] : -1;
+  }
+#pragma unroll
+  for (int u = 0; u < kIt; ++u) {
+    const int32_t s = s_begin + u * 32 + lane;
+    if (s_begin + u * 32 >= s_end) break;  // warp-uniform
+    int32_t e = ev[u];
+    if (s < s_end && (e < 0 || e >= a.E)) {
+      bad = true;
+      lrank[s] = -1;
+      e = -1;
     }
     const uint32_t peers = __match_any_sync(0xffffffffu, e);
     int32_t prior = 0;
     if (e >= 0) {
       prior = my_hist[e];
-      lrank[s] = prior + __popc(peers & lanemask_lt());
+      lrank[s] = e << 16 | (prior + __popc(peers & lanemask_lt()));
     }
     __syncwarp();
     if (e >= 0 && (__ffs(peers) - 1) == lane) my_hist[e] = prior + __popc(peers);
@@ -101,31 +116,32 @@ __global__ void __launch_bounds__(kMetaThreads) meta_rank_kernel(MetaArgs a) {
 
   int32_t* dst = a.dst + ts.tok0 * a.k;
   for (int32_t s = threadIdx.x; s < ts.slots; s += kMetaThreads) {
-    const int32_t e = idx[s];
-    if (e < 0 || e >= a.E) continue;
-    dst[s] = whist[(s / seg) * a.E + e] + lrank[s];  // rank inside the tile
+    const int32_t v = lrank[s];
+    if (v < 0) continue;
+    dst[s] = whist[(s / seg) * a.E + (v >> 16)] + (v & 0xffff);  // rank inside the tile
   }
+  __syncthreads();  // the shared arrays are reused by the next tile
+  return bad;
 }
 
-__global__ void __launch_bounds__(kMetaThreads) meta_count_kernel(MetaArgs a) {
-  const int32_t c = blockIdx.x;
-  const int32_t e = blockIdx.y * kMetaThreads + threadIdx.x;
-  if (e >= a.E) return;
+// Column (c, e) of the tile histograms, one warp: exclusive scan over the chunk's tiles, in
+// place, 32 tiles per round (a lane per tile, warp scan), and the chunk's count of expert e.
+__device__ void meta_count_column(const MetaArgs& a, int32_t c, int32_t e, int lane) {
   int32_t* h = a.hist + (int64_t)c * a.tiles_per_chunk * a.E + e;
   int32_t run = 0;
-  // 8 tiles at a time: the 8 loads are issued together instead of one round trip per tile
-  for (int32_t lt0 = 0; lt0 < a.tiles_per_chunk; lt0 += 8) {
-    int32_t v[8];
+  for (int32_t lt0 = 0; lt0 < a.tiles_per_chunk; lt0 += 32) {
+    const int32_t lt = lt0 + lane;
+    const int32_t v = lt < a.tiles_per_chunk ? h[(int64_t)lt * a.E] : 0;
+    int32_t incl = v;
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
-      v[u] = lt0 + u < a.tiles_per_chunk ? h[(int64_t)(lt0 + u) * a.E] : 0;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (lt0 + u < a.tiles_per_chunk) h[(int64_t)(lt0 + u) * a.E] = run;
-      run += v[u];
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
     }
+    if (lt < a.tiles_per_chunk) h[(int64_t)lt * a.E] = run + incl - v;
+    run += __shfl_sync(0xffffffffu, incl, 31);
   }
-  a.counts[(int64_t)c * a.E + e] = run;
+  if (lane == 0) a.counts[(int64_t)c * a.E + e] = run;
 }
 
 // Block-wide exclusive scan of counts[0..E) into off[0..E] (off[E] = total).
@@ -165,11 +181,9 @@ __device__ void block_exclusive_scan(const int32_t* counts, int32_t E, int32_t* 
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kMetaThreads) meta_finalize_kernel(MetaArgs a) {
-  extern __shared__ int32_t sm[];
+__device__ void meta_finalize_tile(const MetaArgs& a, int32_t tile, int32_t* sm) {
   int32_t* off = sm;                  // [E+1]
   int32_t* warp_tot = sm + a.E + 1;   // [kWarps]
-  const int32_t tile = blockIdx.x;
   const int32_t c = tile / a.tiles_per_chunk;
   const int32_t lt = tile - c * a.tiles_per_chunk;
   const TileSpan ts = tile_span(a, tile);
@@ -207,6 +221,27 @@ __global__ void __launch_bounds__(kMetaThreads) meta_finalize_kernel(MetaArgs a)
         src[r] = (int32_t)((a.src_relative ? 0 : ts.chunk_tok0) + tok_in_chunk0 + sl / a.k);
     }
   }
+  __syncthreads();  // off is reused by the next tile
+}
+
+__global__ void __launch_bounds__(kMetaThreads) meta_kernel(MetaArgs a) {
+  extern __shared__ int32_t sm[];
+  cooperative_groups::grid_group grid = cooperative_groups::this_grid();
+  const int32_t n_tiles = a.n_chunks * a.tiles_per_chunk;
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < a.status_words; i += kMetaThreads) a.status[i] = 0;
+  bool bad = false;
+  for (int32_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x)
+    bad |= meta_rank_tile(a, tile, sm);
+  grid.sync();
+  const int32_t cols = a.n_chunks * a.E;
+  const int warp = threadIdx.x >> 5;
+  for (int32_t i = blockIdx.x * kWarps + warp; i < cols; i += gridDim.x * kWarps)
+    meta_count_column(a, i / a.E, i % a.E, threadIdx.x & 31);
+  grid.sync();
+  for (int32_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x)
+    meta_finalize_tile(a, tile, sm);
+  if (bad) atomicOr(a.status, MOE_DEV_BAD_INDEX);  // after the clear: two barriers later
 }
 
 }  // namespace
@@ -215,12 +250,36 @@ cudaError_t launch_metadata(const MetaArgs& a, cudaStream_t s) {
   const int32_t n_tiles = a.n_chunks * a.tiles_per_chunk;
   const size_t rank_smem = sizeof(int32_t) * ((size_t)kWarps * a.E + kMetaSlotsPerTile);
   const size_t fin_smem = sizeof(int32_t) * ((size_t)a.E + 1 + kWarps);
-  // rank_smem <= (8 * 1024 + 2048) * 4 B = 40 KB: within the default 48 KB limit
-  meta_rank_kernel<<<n_tiles, kMetaThreads, rank_smem, s>>>(a);
-  meta_count_kernel<<<dim3(a.n_chunks, (a.E + kMetaThreads - 1) / kMetaThreads), kMetaThreads, 0,
-                      s>>>(a);
-  meta_finalize_kernel<<<n_tiles, kMetaThreads, fin_smem, s>>>(a);
-  return cudaGetLastError();
+  // <= (8 * 1024 + 2048) * 4 B = 40 KB: within the default 48 KB limit
+  const size_t smem = rank_smem > fin_smem ? rank_smem : fin_smem;
+  // every CTA of a cooperative grid must be resident: at most the device's capacity at the
+  // largest shared-memory size (E = 1024, the most experts), looked up once per device; the
+  // CTAs loop over the tiles
+  constexpr int kMaxDevices = 64;
+  static int cap_of[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (cap_of[dev] <= 0) {
+    constexpr size_t kMaxSmem = sizeof(int32_t) * ((size_t)kWarps * 1024 + kMetaSlotsPerTile);
+    static_assert(kMaxSmem <= 48 * 1024, "within the default dynamic shared-memory limit");
+    int sms = 0, per_sm = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, meta_kernel, kMetaThreads,
+                                                        kMaxSmem);
+    if (e != cudaSuccess) return e;
+    cap_of[dev] = sms * per_sm;
+  }
+  const int64_t cap = cap_of[dev];
+  if (cap <= 0 || smem > sizeof(int32_t) * ((size_t)kWarps * 1024 + kMetaSlotsPerTile))
+    return cudaErrorInvalidConfiguration;
+  const int grid = (int)(n_tiles < cap ? (n_tiles > 0 ? n_tiles : 1) : cap);
+  MetaArgs args = a;
+  void* params[] = {&args};
+  return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(meta_kernel), dim3(grid),
+                                     dim3(kMetaThreads), params, smem, s);
 }
 
 }  // namespace moe

@@ -430,10 +430,9 @@ moe_status_t run_metadata(const Dims& d, const int32_t* idx, uint8_t* ws, const 
   a.counts = packed + kStatusWords;
   a.splits = a.counts + (size_t)d.n * d.E;
   a.offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
-  if (cudaMemsetAsync(packed, 0, sizeof(int32_t) * kStatusWords, s) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  a.status_words = kStatusWords;  // cleared by the kernel
   {
-    ProfScope ps(MOE_KERNEL_METADATA, s, d.T, 0, 3);
+    ProfScope ps(MOE_KERNEL_METADATA, s, d.T, 0, 1);
     if (launch_metadata(a, s) != cudaSuccess) return MOE_ERR_CUDA;
   }
   return MOE_OK;

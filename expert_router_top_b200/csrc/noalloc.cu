@@ -129,9 +129,9 @@ moe_status_t moe_metadata_noalloc(const int32_t* top_k_index, int64_t T, int32_t
   a.counts = packed + kStatusWords;
   a.splits = a.counts + (size_t)p.n * E;
   a.offsets = reinterpret_cast<int32_t*>(ws + p.offsets);
-  // the status word must start at zero; the previous call may have left a flag in it
-  if (cudaMemsetAsync(packed, 0, sizeof(int32_t) * kStatusWords, s) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  // the status words must start at zero (the previous call may have left a flag in them):
+  // the metadata kernel clears them
+  a.status_words = kStatusWords;
   if (moe::launch_metadata(a, s) != cudaSuccess) return MOE_ERR_CUDA;
   // the single device-to-host copy, into the fixed host array
   if (cudaMemcpyAsync(g_host_pack, packed, p.packed_bytes, cudaMemcpyDeviceToHost, s) !=
