@@ -84,6 +84,24 @@ def test_metadata_many_tiles_per_chunk(moe):
         _compare(moe, idx, E, 4, N)
 
 
+def test_metadata_more_tiles_than_resident_ctas(moe):
+    """More tiles than one cooperative grid holds at once (at most 5 CTAs of the largest
+    shared-memory size per SM, 148 SMs): the metadata kernel's CTAs each loop over several
+    tiles in every phase, and a bad index in a late tile still reaches the status word."""
+    rng = np.random.default_rng(11)
+    T, k, E = 60000, 32, 1024  # 64 tokens per tile of 2048 copies: ~940 tiles
+    idx = rng.integers(0, E, size=(T, k)).astype(np.int32)
+    idx[rng.random((T, k)) < 0.2] = 17
+    for N in (1, 5):
+        _compare(moe, idx, E, 8, N)
+    bad = idx.copy()
+    bad[T - 1, 3] = E
+    with pytest.raises(moe.MoEError) as ei:
+        moe.metadata(torch.from_numpy(bad).cuda(), E, 8, 5)
+    assert ei.value.status == 2
+    _compare(moe, idx, E, 8, 5)
+
+
 def test_metadata_bad_index(moe):
     idx = np.zeros((100, 2), np.int32)
     idx[37, 1] = 8
